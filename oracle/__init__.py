@@ -1,0 +1,240 @@
+"""CPU oracle for the gated delta rule (fp64).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline / reference arm are the only callers.  Nothing here is
+imported by the CUDA path, and nothing here imports it.
+
+Three independent restatements of what the operator computes:
+
+* :func:`recurrent` -- the plain token-by-token recurrence in C (fp64,
+  OpenMP over (batch, head)), ``gdn_oracle.c``.  This is the oracle proper.
+  Sources: the delta rule as online gradient descent ("OSDN: Improving Delta
+  Rule with Provable Online Preconditioning in Linear Attention", sec. 1), and
+  the scalar / per-dimension gated forms ("Moonshot AI's New Attention
+  Architecture: Key Innovations Explained", sec. 2 Core Operator).
+* :func:`brute_force` -- NumPy, the state written out as explicit products of
+  d_k x d_k transition matrices, in the pages' S = M^T orientation; tiny T only.
+* :func:`chunk_form` -- NumPy fp64 restatement of the chunkwise state
+  recurrence and output ("Moonshot AI's New Attention Architecture", sec. 3
+  Hardware-Friendly Algorithm) with the UT/WY factors T = (I + A)^-1,
+  W = T diag(beta) K_bar, U = T diag(beta) V obtained by forward substitution
+  ("OSDN ...", sec. 2.1: the chunk Gram matrix and the WY pipeline).
+
+Readings taken where the pages are garbled or silent (each is pinned by a test
+in tests/test_oracle.py):
+  * orientation: S_t k_t = v_t after an exact write, so in M = S^T form
+    M_t = (I - b k k^T) Diag(a) M_{t-1} + b k v^T and o_t = M_t^T q_t;
+  * per-dimension decay acts before the erase (Diag(a_t) next to S_{t-1});
+  * the output uses the post-update state, so the intra-chunk mask is
+    inclusive of the diagonal;
+  * the query in the chunk output is scaled by the decay from the chunk start
+    to its own position (Gamma_r), the key of the state update by the decay
+    from its position to the chunk end (Gamma_C / Gamma_i);
+  * g = log a is the gate input, cumulated in the log domain;
+  * no 1/sqrt(d) scale on q; q and k are used as given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+GATE_NONE, GATE_SCALAR, GATE_PER_DIM = 0, 1, 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_SO = os.path.join(_BUILD, "libgdn_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile gdn_oracle.c (gcc, -O2, OpenMP, no fast-math) into _build/."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off",
+                               "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.gdn_oracle_recurrent.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, dp, dp, dp,
+                                             ctypes.c_long, ctypes.c_long, ctypes.c_long,
+                                             ctypes.c_long, ctypes.c_long, ctypes.c_int]
+        lib.gdn_oracle_recurrent.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+def recurrent(q, k, v, beta, g, gate_kind, S0=None, threads: int | None = None):
+    """Token-by-token recurrence in fp64.
+
+    q, k: [B, T, H, Dk]; v: [B, T, H, Dv]; beta: [B, T, H];
+    g = log a: [B, T, H] (scalar gate) or [B, T, H, Dk] (per-dimension) or None;
+    S0: [B, H, Dk, Dv] (M = S^T) or None.  Returns (o [B,T,H,Dv], S [B,H,Dk,Dv]).
+    """
+    q, k, v, beta, g, S0 = map(_f64, (q, k, v, beta, g, S0))
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if gate_kind == GATE_NONE:
+        g = None
+    o = np.empty((B, T, H, Dv), np.float64)
+    S = np.empty((B, H, Dk, Dv), np.float64)
+    rc = _load().gdn_oracle_recurrent(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g),
+                                      int(gate_kind), _ptr(S0), _ptr(o), _ptr(S),
+                                      B, T, H, Dk, Dv, int(threads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"gdn_oracle_recurrent failed with code {rc}")
+    return o, S
+
+
+def _decay_vector(g, gate_kind, b, t, h, Dk):
+    if gate_kind == GATE_NONE:
+        return np.ones(Dk)
+    if gate_kind == GATE_SCALAR:
+        return np.full(Dk, np.exp(g[b, t, h]))
+    return np.exp(g[b, t, h])
+
+
+def brute_force(q, k, v, beta, g, gate_kind, S0=None):
+    """Explicit-product expansion of the recurrence, in the S (d_v x d_k) form.
+
+    With E_t = Diag(a_t) (I - beta_t k_t k_t^T) (a d_k x d_k matrix; scalar gate:
+    Diag(a_t) = a_t I), the recurrence S_t = S_{t-1} E_t + beta_t v_t k_t^T gives
+        S_t = S_0 E_1 ... E_t + sum_{i<=t} beta_i v_i k_i^T E_{i+1} ... E_t,
+    evaluated here literally for every t; o_t = S_t q_t.  Meant for T <= 8.
+    Returns (o [B,T,H,Dv], M_final = S_T^T [B,H,Dk,Dv]).
+    """
+    q, k, v, beta, g, S0 = map(_f64, (q, k, v, beta, g, S0))
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    o = np.zeros((B, T, H, Dv))
+    M_final = np.zeros((B, H, Dk, Dv))
+    I = np.eye(Dk)
+    for b in range(B):
+        for h in range(H):
+            E = []
+            for t in range(T):
+                kt = k[b, t, h][:, None]
+                a = _decay_vector(g, gate_kind, b, t, h, Dk)
+                E.append(np.diag(a) @ (I - beta[b, t, h] * (kt @ kt.T)))
+            for t in range(T):
+                prod = I.copy()
+                for s in range(t + 1):
+                    prod = prod @ E[s]
+                S_t = (np.zeros((Dv, Dk)) if S0 is None else S0[b, h].T) @ prod
+                for i in range(t + 1):
+                    tail = I.copy()
+                    for s in range(i + 1, t + 1):
+                        tail = tail @ E[s]
+                    S_t = S_t + beta[b, i, h] * (v[b, i, h][:, None] @ k[b, i, h][None, :]) @ tail
+                o[b, t, h] = S_t @ q[b, t, h]
+                if t == T - 1:
+                    M_final[b, h] = S_t.T
+            if T == 0:
+                M_final[b, h] = 0 if S0 is None else S0[b, h]
+    return o, M_final
+
+
+def forward_substitution_inverse(A):
+    """T = (I + A)^{-1} for strictly lower-triangular A, row by row:
+    row r of (I + A) T = I gives T_r = e_r - sum_{i<r} A_ri T_i."""
+    n = A.shape[0]
+    Tm = np.zeros_like(A)
+    for r in range(n):
+        row = np.zeros(n)
+        row[r] = 1.0
+        for i in range(r):
+            row -= A[r, i] * Tm[i]
+        Tm[r] = row
+    return Tm
+
+
+def chunk_form(q, k, v, beta, g, gate_kind, S0=None, C: int = 64):
+    """Chunkwise evaluation (fp64) of the same operator, chunk length C.
+
+    Per chunk, with h the entering M (= S^T, d_k x d_v), G_r = sum_{i<=r} log a_i
+    (within the chunk, per key dimension), Gamma_r = exp(G_r):
+      A   = StrictTril(diag(beta) (K_bar K_breve^T)), where
+            (K_bar K_breve^T)_ri = sum_d k_rd k_id exp(G_rd - G_id)
+      T   = (I + A)^{-1}                      (forward substitution)
+      W   = T diag(beta) K_bar,  U = T diag(beta) V,   K_bar = Gamma * K
+      D   = U - W h                            (the chunk's pseudo-values)
+      O   = Q_bar h + Tril_incl(Q_bar K_breve^T) D,   Q_bar = Gamma * Q
+      h'  = Diag(gamma_C) h + K_tilde^T D,  K_tilde_i = k_i * Gamma_C / Gamma_i
+    The last chunk may be shorter than C.  Returns (o, M_final).
+    """
+    q, k, v, beta, g, S0 = map(_f64, (q, k, v, beta, g, S0))
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    o = np.zeros((B, T, H, Dv))
+    M_final = np.zeros((B, H, Dk, Dv))
+    for b in range(B):
+        for h_ in range(H):
+            h = np.zeros((Dk, Dv)) if S0 is None else S0[b, h_].copy()
+            for c0 in range(0, T, C):
+                c1 = min(T, c0 + C)
+                n = c1 - c0
+                Q = q[b, c0:c1, h_]
+                K = k[b, c0:c1, h_]
+                V = v[b, c0:c1, h_]
+                bt = beta[b, c0:c1, h_]
+                if gate_kind == GATE_NONE:
+                    logs = np.zeros((n, Dk))
+                elif gate_kind == GATE_SCALAR:
+                    logs = np.repeat(g[b, c0:c1, h_][:, None], Dk, axis=1)
+                else:
+                    logs = g[b, c0:c1, h_]
+                G = np.cumsum(logs, axis=0)               # [n, Dk], log domain
+                Gam = np.exp(G)
+                gamma_C = Gam[n - 1]
+                # pairwise decay exp(G_r - G_i), only where i <= r (no overflow)
+                diff = G[:, None, :] - G[None, :, :]       # [r, i, d]
+                lower = np.tril(np.ones((n, n), bool))
+                diff = np.where(lower[:, :, None], diff, -np.inf)
+                dec = np.exp(diff)
+                KK = np.einsum("rd,id,rid->ri", K, K, dec)
+                QK = np.einsum("rd,id,rid->ri", Q, K, dec)
+                A = np.tril(bt[:, None] * KK, -1)
+                Tm = forward_substitution_inverse(A)
+                K_bar = Gam * K
+                W = Tm @ (bt[:, None] * K_bar)
+                U = Tm @ (bt[:, None] * V)
+                D = U - W @ h
+                Q_bar = Gam * Q
+                o[b, c0:c1, h_] = Q_bar @ h + np.tril(QK) @ D
+                K_tilde = K * np.exp(G[n - 1][None, :] - G)
+                h = gamma_C[:, None] * h + K_tilde.T @ D
+            M_final[b, h_] = h
+    return o, M_final
+
+
+def rel_err(x, ref) -> float:
+    """max|x - ref| / max|ref| over the whole tensor (0 when both are zero)."""
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.max(np.abs(ref)) if ref.size else 0.0
+    num = np.max(np.abs(x - ref)) if ref.size else 0.0
+    if den == 0.0:
+        return float(num)
+    return float(num / den)
