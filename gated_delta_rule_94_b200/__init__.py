@@ -1,0 +1,10 @@
+"""Gated delta-rule linear attention on NVIDIA B200 (sm_100a).
+
+The operator runs in libgdn.so (C ABI in include/gdn.h); this package holds
+its thin ctypes binding (:mod:`._lib`), the in-tree build script
+(:mod:`.build`) and the seeded synthetic-input generator (:mod:`.inputs`).
+"""
+from ._lib import (GDN_BF16, GDN_F32, GDN_GATE_NONE, GDN_GATE_PER_DIM, GDN_GATE_SCALAR,  # noqa: F401
+                   GdnError, chunk_fwd, decode_step, gdn_abi_version, gdn_chunk_fwd,
+                   gdn_chunk_fwd_workspace_bytes, gdn_decode_step, gdn_read_device_status,
+                   gdn_status_string)

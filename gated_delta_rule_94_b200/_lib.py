@@ -1,0 +1,182 @@
+"""ctypes binding of libgdn.so (include/gdn.h).
+
+Argument marshalling only: every step of the operator runs in the library's
+CUDA kernels.  The functions named like the C entry points take torch tensors
+(device memory allocated by the caller), pass their data pointers and the
+current CUDA stream through the C ABI and turn a non-OK status into
+:class:`GdnError`.  If libgdn.so has not been built, every call raises --
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, \
+    GDN_ERR_TIMEOUT = range(6)
+GDN_BF16, GDN_F32 = 0, 1
+GDN_GATE_NONE, GDN_GATE_SCALAR, GDN_GATE_PER_DIM = 0, 1, 2
+
+EXPORTED = ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_decode_step",
+            "gdn_read_device_status", "gdn_status_string", "gdn_abi_version")
+
+_lib = None
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load() -> ctypes.CDLL:
+    """Load libgdn.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libgdn.so is not built ({LIB_PATH}); run "
+                           "`python -m gated_delta_rule_94_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.gdn_chunk_fwd.restype = i
+    lib.gdn_chunk_fwd_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    lib.gdn_chunk_fwd_workspace_bytes.restype = sz
+    lib.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, vp]
+    lib.gdn_decode_step.restype = i
+    lib.gdn_read_device_status.argtypes = [vp]
+    lib.gdn_read_device_status.restype = i
+    lib.gdn_status_string.argtypes = [i]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_abi_version.argtypes = []
+    lib.gdn_abi_version.restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().gdn_status_string(int(status)).decode()
+
+
+def gdn_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def gdn_abi_version() -> int:
+    return load().gdn_abi_version()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return GDN_BF16
+    if dt == torch.float32:
+        return GDN_F32
+    raise TypeError(f"unsupported dtype {dt}; use bfloat16 or float32")
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check_contig(**tensors):
+    for name, t in tensors.items():
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16,
+                                  gate_kind=GDN_GATE_SCALAR) -> int:
+    n = load().gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, chunk, _dtype_code(dtype),
+                                             int(gate_kind))
+    if n == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd_workspace_bytes")
+    return n
+
+
+def gdn_chunk_fwd(q, k, v, beta, g, gate_kind, initial_state, o, final_state, *, chunk=64,
+                  workspace=None, stream=None) -> None:
+    """Enqueue the chunk forward on `stream` (default: torch's current stream).
+    Shapes: q, k [B,T,H,Dk]; v, o [B,T,H,Dv]; beta [B,T,H]; g [B,T,H] or
+    [B,T,H,Dk] or None; states [B,H,Dk,Dv] fp32 or None."""
+    _check_contig(q=q, k=k, v=v, beta=beta, g=g, initial_state=initial_state, o=o,
+                  final_state=final_state)
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dtype_code(q.dtype)
+    for name, t in (("k", k), ("v", v), ("beta", beta), ("g", g), ("o", o)):
+        if t is not None and t.dtype != q.dtype:
+            raise TypeError(f"{name} must have dtype {q.dtype}")
+    for name, t in (("initial_state", initial_state), ("final_state", final_state)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), int(gate_kind),
+                              _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, Dk, Dv,
+                              chunk, dt, _ptr(workspace), ws_bytes, _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd")
+
+
+def gdn_decode_step(q, k, v, beta, g, gate_kind, state, o, *, stream=None) -> None:
+    """Enqueue one decode step.  q, k [N,H,Dk]; v, o [N,H,Dv]; beta [N,H];
+    g [N,H] or [N,H,Dk] or None; state [N,H,Dk,Dv] fp32, updated in place."""
+    _check_contig(q=q, k=k, v=v, beta=beta, g=g, state=state, o=o)
+    N, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dtype_code(q.dtype)
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    st = load().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), int(gate_kind),
+                                _ptr(state), _ptr(o), N, H, Dk, Dv, dt, _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode_step")
+
+
+def gdn_read_device_status(stream=None) -> int:
+    return load().gdn_read_device_status(_stream(stream))
+
+
+# ----------------------------------------------------------------- convenience
+def chunk_fwd(q, k, v, beta, g=None, initial_state=None, *, output_final_state=True,
+              chunk=64, stream=None):
+    """Allocate o (and the final state) with torch and run gdn_chunk_fwd.
+    The gate kind follows g: None -> none, [B,T,H] -> scalar, [B,T,H,Dk] ->
+    per-dimension.  Returns (o, final_state or None)."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    gate = GDN_GATE_NONE if g is None else (GDN_GATE_SCALAR if g.dim() == 3 else GDN_GATE_PER_DIM)
+    o = torch.empty((B, T, H, Dv), dtype=q.dtype, device=q.device)
+    S = (torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+         if output_final_state else None)
+    ws_n = gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, chunk, q.dtype, gate)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
+    gdn_chunk_fwd(q, k, v, beta, g, gate, initial_state, o, S, chunk=chunk, workspace=ws,
+                  stream=stream)
+    return o, S
+
+
+def decode_step(q, k, v, beta, g, state, *, stream=None):
+    """One decode step; updates `state` in place and returns o."""
+    N, H, Dk = q.shape
+    gate = GDN_GATE_NONE if g is None else (GDN_GATE_SCALAR if g.dim() == 2 else GDN_GATE_PER_DIM)
+    o = torch.empty((N, H, v.shape[-1]), dtype=q.dtype, device=q.device)
+    gdn_decode_step(q, k, v, beta, g, gate, state, o, stream=stream)
+    return o

@@ -1,0 +1,56 @@
+// common.cuh -- small device helpers shared by the libgdn kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+enum Gate : int { kGateNone = 0, kGateScalar = 1, kGatePerDim = 2 };
+
+// Bits of the library's device status word (set by kernels that give up a
+// bounded wait; read and cleared by gdn_read_device_status).
+enum StatusBits : unsigned { kStatusTimeout = 1u };
+
+struct ChunkParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* beta;
+    const void* g;
+    const float* s0;   // may be null
+    void* o;
+    float* s_out;      // may be null
+    int B, T, H, Dk, Dv;
+    unsigned* status;  // device status word
+};
+
+struct DecodeParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* beta;
+    const void* g;
+    float* state;
+    void* o;
+    int N, H;
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+}  // namespace gdn
+
+// Launchers implemented in the kernel translation units.
+namespace gdn {
+cudaError_t launch_chunk_fwd_simt(const ChunkParams& p, int gate, bool bf16, cudaStream_t s);
+cudaError_t launch_decode_step(const DecodeParams& p, int Dk, int Dv, int gate, bool bf16,
+                               cudaStream_t s);
+}  // namespace gdn

@@ -1,0 +1,190 @@
+// gdn_api.cu -- host side of the libgdn C ABI (include/gdn.h): argument
+// validation, workspace sizing, kernel selection and launch on the caller's
+// stream.  Nothing here allocates device memory or synchronizes, except
+// gdn_read_device_status, which is documented to synchronize.
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "gdn.h"
+
+// The library's device status word: kernels OR in StatusBits when they give up
+// a bounded wait; gdn_read_device_status reads and clears it.
+__device__ unsigned gdn_device_status_word = 0u;
+
+namespace gdn {
+// Implemented in chunk_fwd_tc.cu (tensor-core path for bf16 inputs).
+bool chunk_fwd_tc_supported(int Dk, int Dv, int gate);
+cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, cudaStream_t s);
+}  // namespace gdn
+
+namespace {
+
+unsigned* status_word_ptr() {
+    // One device address per current device; cached per device ordinal.
+    static unsigned* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, gdn_device_status_word) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<unsigned*>(ptr);
+    }
+    return cache[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+bool supported_dim(int d) { return d == 64 || d == 128; }
+
+size_t elem_size(gdn_dtype dt) { return dt == GDN_BF16 ? 2 : 4; }
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+int gdn_abi_version(void) { return 1; }
+
+size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk,
+                                     gdn_dtype dtype, gdn_gate gate_kind) {
+    if (B < 0 || T < 0 || H < 0) return (size_t)-1;
+    if (!supported_dim(Dk) || !supported_dim(Dv) || chunk != 64) return (size_t)-1;
+    if (dtype != GDN_BF16 && dtype != GDN_F32) return (size_t)-1;
+    if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return (size_t)-1;
+    return 0;
+}
+
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* beta,
+                         const void* g, gdn_gate gate_kind, const float* initial_state,
+                         void* o, float* final_state, int B, int T, int H, int Dk, int Dv,
+                         int chunk, gdn_dtype dtype, void* workspace, size_t workspace_bytes,
+                         gdn_stream_t stream) {
+    if (B < 0 || T < 0 || H < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return GDN_ERR_INVALID_ARG;
+    if (!supported_dim(Dk) || !supported_dim(Dv) || chunk != 64) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)B * T > INT32_MAX || (int64_t)B * H > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return GDN_OK;
+    const bool need_tokens = T > 0;
+    if (need_tokens && (!q || !k || !v || !beta || !o)) return GDN_ERR_INVALID_ARG;
+    if (need_tokens && (gate_kind == GDN_GATE_NONE) != (g == nullptr)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, beta, g, initial_state, o, final_state, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t es = elem_size(dtype);
+    const size_t ntok = (size_t)B * T * H;
+    const size_t state_bytes = (size_t)B * H * Dk * Dv * sizeof(float);
+    if (final_state) {
+        const size_t gbytes = gate_kind == GDN_GATE_PER_DIM ? ntok * Dk * es
+                              : gate_kind == GDN_GATE_SCALAR ? ntok * es : 0;
+        if (overlaps(final_state, state_bytes, q, ntok * Dk * es) ||
+            overlaps(final_state, state_bytes, k, ntok * Dk * es) ||
+            overlaps(final_state, state_bytes, v, ntok * Dv * es) ||
+            overlaps(final_state, state_bytes, beta, ntok * es) ||
+            overlaps(final_state, state_bytes, g, gbytes) ||
+            overlaps(final_state, state_bytes, o, ntok * Dv * es))
+            return GDN_ERR_INVALID_ARG;
+        if (initial_state && initial_state != final_state &&
+            overlaps(final_state, state_bytes, initial_state, state_bytes))
+            return GDN_ERR_INVALID_ARG;
+    }
+    if (need_tokens && initial_state && overlaps(o, ntok * Dv * es, initial_state, state_bytes))
+        return GDN_ERR_INVALID_ARG;
+    const size_t ws_need = gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, chunk, dtype, gate_kind);
+    if (ws_need > 0 && (workspace_bytes < ws_need || !workspace)) return GDN_ERR_WORKSPACE;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        // No tokens: the final state is the initial state (or zero).
+        if (!final_state) return GDN_OK;
+        cudaError_t e = initial_state
+                            ? (initial_state == final_state
+                                   ? cudaSuccess
+                                   : cudaMemcpyAsync(final_state, initial_state, state_bytes,
+                                                     cudaMemcpyDeviceToDevice, s))
+                            : cudaMemsetAsync(final_state, 0, state_bytes, s);
+        return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    }
+
+    gdn::ChunkParams p;
+    p.q = q; p.k = k; p.v = v; p.beta = beta; p.g = g;
+    p.s0 = initial_state; p.o = o; p.s_out = final_state;
+    p.B = B; p.T = T; p.H = H; p.Dk = Dk; p.Dv = Dv;
+    p.status = status_word_ptr();
+    if (!p.status) return GDN_ERR_CUDA;
+    cudaError_t e;
+    if (dtype == GDN_BF16 && gdn::chunk_fwd_tc_supported(Dk, Dv, gate_kind))
+        e = gdn::launch_chunk_fwd_tc(p, gate_kind, s);
+    else
+        e = gdn::launch_chunk_fwd_simt(p, gate_kind, dtype == GDN_BF16, s);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const void* beta,
+                           const void* g, gdn_gate gate_kind, float* state, void* o, int N,
+                           int H, int Dk, int Dv, gdn_dtype dtype, gdn_stream_t stream) {
+    if (N < 0 || H < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return GDN_ERR_INVALID_ARG;
+    if (!supported_dim(Dk) || !supported_dim(Dv)) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)N * H > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+    if (N == 0 || H == 0) return GDN_OK;
+    if (!q || !k || !v || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
+    if ((gate_kind == GDN_GATE_NONE) != (g == nullptr)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, beta, g, state, o};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t es = elem_size(dtype);
+    const size_t nh = (size_t)N * H;
+    const size_t state_bytes = nh * Dk * Dv * sizeof(float);
+    const size_t gbytes = gate_kind == GDN_GATE_PER_DIM ? nh * Dk * es
+                          : gate_kind == GDN_GATE_SCALAR ? nh * es : 0;
+    if (overlaps(state, state_bytes, o, nh * Dv * es) ||
+        overlaps(state, state_bytes, q, nh * Dk * es) ||
+        overlaps(state, state_bytes, k, nh * Dk * es) ||
+        overlaps(state, state_bytes, v, nh * Dv * es) ||
+        overlaps(state, state_bytes, beta, nh * es) ||
+        overlaps(state, state_bytes, g, gbytes))
+        return GDN_ERR_INVALID_ARG;
+
+    gdn::DecodeParams p;
+    p.q = q; p.k = k; p.v = v; p.beta = beta; p.g = g;
+    p.state = state; p.o = o; p.N = N; p.H = H;
+    cudaError_t e = gdn::launch_decode_step(p, Dk, Dv, gate_kind, dtype == GDN_BF16,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_read_device_status(gdn_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+    unsigned word = 0;
+    if (cudaMemcpyFromSymbol(&word, gdn_device_status_word, sizeof(word)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (word) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(gdn_device_status_word, &zero, sizeof(zero)) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    return (word & gdn::kStatusTimeout) ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the gated delta-rule linear-attention operator
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operator (state stored as M = S^T, one d_k x d_v matrix per sequence and
+ * head):
+ *     M_t = (I - beta_t k_t k_t^T) Diag(a_t) M_{t-1} + beta_t k_t v_t^T
+ *     o_t = M_t^T q_t
+ * with a_t = exp(g_t), either one scalar per token and head (Gated DeltaNet)
+ * or one value per key dimension (the per-dimension gate).  Sources: the delta
+ * rule as an online gradient step ("OSDN: Improving Delta Rule with Provable
+ * Online Preconditioning in Linear Attention", sec. 1) and its scalar- and
+ * per-dimension-gated forms ("Moonshot AI's New Attention Architecture: Key
+ * Innovations Explained", sec. 2 Core Operator).  With S = M^T this is
+ * S_t = S_{t-1} Diag(a_t)(I - beta_t k_t k_t^T) + beta_t v_t k_t^T, the form in
+ * which an exact write (beta = 1, |k| = 1) gives S_t k_t = v_t.
+ *
+ * Conventions shared by every entry point:
+ *   - Ownership: the caller owns every buffer (inputs, outputs, workspace).
+ *     The library never allocates or frees memory.
+ *   - Execution: every call only enqueues work on `stream` and returns; it
+ *     never synchronizes (gdn_read_device_status excepted).  Outputs are valid
+ *     once the stream has reached the enqueued work.
+ *   - Errors: argument errors are detected on the host before anything is
+ *     enqueued and return a status; nothing is launched and no output is
+ *     touched.  A failed launch returns GDN_ERR_CUDA.  Nothing throws.
+ *   - Pointers are device pointers (or managed memory) and must be 16-byte
+ *     aligned; tensors are dense and row-major in the layouts given below.
+ *   - q and k are used as given: no L2 normalisation and no 1/sqrt(d) scale.
+ *   - beta and g have the same element type as q, k, v; states are fp32.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-identical to cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st* gdn_stream_t;
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, negative size, bad overlap */
+    GDN_ERR_UNSUPPORTED = 2,  /* valid request outside the built shapes / dtypes */
+    GDN_ERR_WORKSPACE = 3,    /* workspace smaller than gdn_chunk_fwd_workspace_bytes */
+    GDN_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+    GDN_ERR_TIMEOUT = 5       /* a kernel gave up a bounded wait (reported by
+                                 gdn_read_device_status) */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
+
+typedef enum {
+    GDN_GATE_NONE = 0,     /* a_t = 1 (DeltaNet)                     */
+    GDN_GATE_SCALAR = 1,   /* g: [.., H]      one log-decay per head */
+    GDN_GATE_PER_DIM = 2   /* g: [.., H, Dk]  one log-decay per key dimension */
+} gdn_gate;
+
+/*
+ * gdn_chunk_fwd -- chunkwise forward over a whole sequence batch.
+ *
+ * Computes o_t for every token and (optionally) the final state, splitting
+ * each sequence into chunks of `chunk` tokens: parallel within a chunk, the
+ * state carried serially between chunks ("Moonshot AI's New Attention
+ * Architecture: Key Innovations Explained", sec. 3 Hardware-Friendly
+ * Algorithm, the state recurrence and the output with its causal Tril).  Per
+ * chunk the intra-chunk lower-triangular system A (the chunk Gram matrix of
+ * the keys, gated and scaled by beta) is inverted by forward substitution,
+ * T = (I + A)^-1, giving the WY factors W = T diag(beta) K_bar and
+ * U = T diag(beta) V ("OSDN ...", sec. 2.1: the WY pipeline).  Gates are
+ * cumulated in the log domain within each chunk (Moonshot page, sec. 5).
+ *
+ *   q, k          [B, T, H, Dk]  element type `dtype`
+ *   v             [B, T, H, Dv]  element type `dtype`
+ *   beta          [B, T, H]      element type `dtype`, the write strength
+ *   g             log a_t <= 0: [B, T, H] (GDN_GATE_SCALAR) or [B, T, H, Dk]
+ *                 (GDN_GATE_PER_DIM), element type `dtype`; must be NULL iff
+ *                 gate_kind == GDN_GATE_NONE
+ *   initial_state [B, H, Dk, Dv] fp32 (M = S^T), or NULL for a zero state
+ *   o             [B, T, H, Dv]  element type `dtype` (output)
+ *   final_state   [B, H, Dk, Dv] fp32 (output) or NULL; may be the same
+ *                 pointer as initial_state (updated in place), any other
+ *                 overlap with an input is GDN_ERR_INVALID_ARG
+ *   B, T, H       batch, tokens per sequence, heads; T = 0 is allowed (no
+ *                 output tokens; final_state = initial_state or 0); B = 0 or
+ *                 H = 0 is a no-op
+ *   Dk, Dv        64 or 128 each
+ *   chunk         64
+ *   dtype         GDN_BF16 (tensor-core path, fp32 accumulation and fp32
+ *                 state) or GDN_F32 (fp32 CUDA-core path)
+ *   workspace     device scratch of at least gdn_chunk_fwd_workspace_bytes
+ *                 bytes (may be NULL when that is 0)
+ * Returns GDN_OK once the work is enqueued.
+ */
+GDN_API gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v,
+                         const void* beta, const void* g, gdn_gate gate_kind,
+                         const float* initial_state, void* o, float* final_state,
+                         int B, int T, int H, int Dk, int Dv, int chunk,
+                         gdn_dtype dtype, void* workspace, size_t workspace_bytes,
+                         gdn_stream_t stream);
+
+/* Bytes of device workspace gdn_chunk_fwd needs for these arguments (0 when
+ * none).  Returns (size_t)-1 for an unsupported or invalid shape. */
+GDN_API size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk,
+                                     gdn_dtype dtype, gdn_gate gate_kind);
+
+/*
+ * gdn_decode_step -- one recurrent step for N independent sequences: the
+ * linear layers' constant-size-state decoding ("Moonshot AI's New Attention
+ * Architecture", sec. 1) applied to the gated delta rule above.  Per (n, h):
+ *     M' = Diag(a) M;  x = M'^T k;  r = beta (v - x);
+ *     M  <- M' + k r^T (in place);  o = M^T q = M'^T q + r (k . q).
+ * One pass over the state: each element is read once and written once.
+ *
+ *   q, k   [N, H, Dk]  element type `dtype`
+ *   v      [N, H, Dv]  element type `dtype`
+ *   beta   [N, H]      element type `dtype`
+ *   g      [N, H] (scalar) or [N, H, Dk] (per-dimension), or NULL iff
+ *          gate_kind == GDN_GATE_NONE
+ *   state  [N, H, Dk, Dv] fp32, read and updated in place
+ *   o      [N, H, Dv]  element type `dtype` (output; must not overlap state)
+ *   N, H   >= 0 (0 is a no-op);  Dk, Dv in {64, 128}
+ */
+GDN_API gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
+                           const void* beta, const void* g, gdn_gate gate_kind,
+                           float* state, void* o, int N, int H, int Dk, int Dv,
+                           gdn_dtype dtype, gdn_stream_t stream);
+
+/* Synchronizes `stream`, then reads and clears the library's device status
+ * word.  Returns GDN_ERR_TIMEOUT if any kernel since the last call gave up a
+ * bounded wait, GDN_ERR_CUDA if the stream reports an error, else GDN_OK. */
+GDN_API gdn_status gdn_read_device_status(gdn_stream_t stream);
+
+/* A static, human-readable name for a status code. */
+GDN_API const char* gdn_status_string(gdn_status s);
+
+/* Library ABI version, currently 1. */
+GDN_API int gdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

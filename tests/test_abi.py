@@ -1,0 +1,131 @@
+"""Host-only tests of the C ABI: the library builds, loads and exports every
+symbol include/gdn.h declares, and every argument error is reported by status
+code before anything is launched (no GPU needed; nothing here dereferences
+the fake device pointers, because validation rejects the call first)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import gated_delta_rule_94_b200 as gdn
+from gated_delta_rule_94_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+A = 0x10000          # a 16-byte-aligned fake device address (never dereferenced)
+MIS = 0x10008        # misaligned
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names.update(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = declared_symbols()
+    assert {"gdn_chunk_fwd", "gdn_decode_step"} <= names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(_lib.EXPORTED) == names
+
+
+def test_status_strings_and_version():
+    assert gdn.gdn_abi_version() == 1
+    assert gdn.gdn_status_string(0) == "GDN_OK"
+    assert gdn.gdn_status_string(3) == "GDN_ERR_WORKSPACE"
+    assert gdn.gdn_status_string(99) == "GDN_ERR_UNKNOWN"
+
+
+def test_workspace_bytes():
+    lib = _lib.load()
+    bad = ctypes.c_size_t(-1).value
+    assert lib.gdn_chunk_fwd_workspace_bytes(4, 2048, 16, 128, 128, 64, 0, 1) != bad
+    assert lib.gdn_chunk_fwd_workspace_bytes(4, 2048, 16, 96, 128, 64, 0, 1) == bad
+    assert lib.gdn_chunk_fwd_workspace_bytes(4, 2048, 16, 128, 128, 32, 0, 1) == bad
+    assert lib.gdn_chunk_fwd_workspace_bytes(-1, 2048, 16, 128, 128, 64, 0, 1) == bad
+
+
+def chunk_call(**over):
+    args = dict(q=A, k=A, v=A, beta=A, g=A, gate=1, s0=None, o=A * 2, s1=None, B=1, T=64, H=1,
+                Dk=64, Dv=64, chunk=64, dtype=0, ws=None, ws_bytes=0, stream=None)
+    args.update(over)
+    return _lib.load().gdn_chunk_fwd(args["q"], args["k"], args["v"], args["beta"], args["g"],
+                                     args["gate"], args["s0"], args["o"], args["s1"], args["B"],
+                                     args["T"], args["H"], args["Dk"], args["Dv"], args["chunk"],
+                                     args["dtype"], args["ws"], args["ws_bytes"], args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(o=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(beta=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(g=None), _lib.GDN_ERR_INVALID_ARG),                 # gate scalar needs g
+    (dict(gate=0), _lib.GDN_ERR_INVALID_ARG),                 # gate none forbids g
+    (dict(gate=3), _lib.GDN_ERR_INVALID_ARG),
+    (dict(dtype=7), _lib.GDN_ERR_INVALID_ARG),
+    (dict(B=-1), _lib.GDN_ERR_INVALID_ARG),
+    (dict(T=-5), _lib.GDN_ERR_INVALID_ARG),
+    (dict(Dk=96), _lib.GDN_ERR_UNSUPPORTED),
+    (dict(Dv=32), _lib.GDN_ERR_UNSUPPORTED),
+    (dict(chunk=128), _lib.GDN_ERR_UNSUPPORTED),
+    (dict(q=MIS), _lib.GDN_ERR_INVALID_ARG),
+    (dict(o=MIS), _lib.GDN_ERR_INVALID_ARG),
+    (dict(s1=A * 2), _lib.GDN_ERR_INVALID_ARG),               # final state overlaps o
+    (dict(s0=A * 4, s1=A * 4 + 4096), _lib.GDN_ERR_INVALID_ARG),  # partial state overlap
+    (dict(s0=A * 2), _lib.GDN_ERR_INVALID_ARG),               # o overlaps the initial state
+])
+def test_chunk_fwd_argument_errors(over, code):
+    assert chunk_call(**over) == code
+
+
+def test_chunk_fwd_noop_sizes():
+    assert chunk_call(B=0) == _lib.GDN_OK
+    assert chunk_call(H=0, q=None, o=None) == _lib.GDN_OK
+
+
+def decode_call(**over):
+    args = dict(q=A, k=A, v=A, beta=A, g=A, gate=1, state=A * 8, o=A * 2, N=2, H=2, Dk=64,
+                Dv=64, dtype=0, stream=None)
+    args.update(over)
+    return _lib.load().gdn_decode_step(args["q"], args["k"], args["v"], args["beta"], args["g"],
+                                       args["gate"], args["state"], args["o"], args["N"],
+                                       args["H"], args["Dk"], args["Dv"], args["dtype"],
+                                       args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(state=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(o=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(g=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(gate=2, g=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(N=-1), _lib.GDN_ERR_INVALID_ARG),
+    (dict(Dk=256), _lib.GDN_ERR_UNSUPPORTED),
+    (dict(state=A * 8 + 4), _lib.GDN_ERR_INVALID_ARG),
+    (dict(o=A * 8 + 256), _lib.GDN_ERR_INVALID_ARG),          # o inside the state
+])
+def test_decode_argument_errors(over, code):
+    assert decode_call(**over) == code
+
+
+def test_decode_noop_sizes():
+    assert decode_call(N=0, q=None) == _lib.GDN_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path only")
+def test_valid_call_without_a_device_reports_cuda_error():
+    assert chunk_call() == _lib.GDN_ERR_CUDA
+    assert decode_call() == _lib.GDN_ERR_CUDA
+
+
+def test_python_binding_rejects_bad_tensors():
+    q = torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        gdn.gdn_chunk_fwd(q, q, q, torch.zeros(1, 64, 1), None, 0, None, q, None)
+    with pytest.raises(ValueError):
+        gdn.gdn_chunk_fwd(q.transpose(1, 3), q, q, None, None, 0, None, q, None)
