@@ -23,7 +23,8 @@ GDN_BF16, GDN_F32 = 0, 1
 GDN_GATE_NONE, GDN_GATE_SCALAR, GDN_GATE_PER_DIM = 0, 1, 2
 
 EXPORTED = ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_decode_step",
-            "gdn_read_device_status", "gdn_status_string", "gdn_abi_version")
+            "gdn_read_device_status", "gdn_status_string", "gdn_abi_version",
+            "gdn_kernel_launch_count", "gdn_chunk_fwd_kernel_name")
 
 _lib = None
 
@@ -56,6 +57,10 @@ def load() -> ctypes.CDLL:
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_abi_version.argtypes = []
     lib.gdn_abi_version.restype = i
+    lib.gdn_kernel_launch_count.argtypes = []
+    lib.gdn_kernel_launch_count.restype = ctypes.c_ulonglong
+    lib.gdn_chunk_fwd_kernel_name.argtypes = [i, i, i, i]
+    lib.gdn_chunk_fwd_kernel_name.restype = ctypes.c_char_p
     _lib = lib
     return lib
 
@@ -70,6 +75,15 @@ def gdn_status_string(status: int) -> str:
 
 def gdn_abi_version() -> int:
     return load().gdn_abi_version()
+
+
+def gdn_kernel_launch_count() -> int:
+    return int(load().gdn_kernel_launch_count())
+
+
+def gdn_chunk_fwd_kernel_name(Dk, Dv, gate_kind, dtype=torch.bfloat16):
+    name = load().gdn_chunk_fwd_kernel_name(Dk, Dv, int(gate_kind), _dtype_code(dtype))
+    return None if name is None else name.decode()
 
 
 def _ptr(t):

@@ -5,6 +5,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "gdn.h"
 
@@ -41,6 +43,8 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return a0 < b0 + nb && b0 < a0 + na;
 }
 
+std::atomic<unsigned long long> g_launches{0};
+
 bool supported_dim(int d) { return d == 64 || d == 128; }
 
 size_t elem_size(gdn_dtype dt) { return dt == GDN_BF16 ? 2 : 4; }
@@ -62,6 +66,17 @@ const char* gdn_status_string(gdn_status s) {
 }
 
 int gdn_abi_version(void) { return 1; }
+
+unsigned long long gdn_kernel_launch_count(void) { return g_launches.load(); }
+
+const char* gdn_chunk_fwd_kernel_name(int Dk, int Dv, gdn_gate gate_kind, gdn_dtype dtype) {
+    if (!supported_dim(Dk) || !supported_dim(Dv)) return nullptr;
+    if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return nullptr;
+    if (dtype == GDN_BF16 && gdn::chunk_fwd_tc_supported(Dk, Dv, gate_kind))
+        return "chunk_fwd_tc_kernel";
+    if (dtype == GDN_BF16 || dtype == GDN_F32) return "chunk_fwd_simt_kernel";
+    return nullptr;
+}
 
 size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk,
                                      gdn_dtype dtype, gdn_gate gate_kind) {
@@ -135,7 +150,9 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
         e = gdn::launch_chunk_fwd_tc(p, gate_kind, s);
     else
         e = gdn::launch_chunk_fwd_simt(p, gate_kind, dtype == GDN_BF16, s);
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    g_launches.fetch_add(1);
+    return GDN_OK;
 }
 
 gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const void* beta,
@@ -170,7 +187,9 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const vo
     p.state = state; p.o = o; p.N = N; p.H = H;
     cudaError_t e = gdn::launch_decode_step(p, Dk, Dv, gate_kind, dtype == GDN_BF16,
                                             reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    g_launches.fetch_add(1);
+    return GDN_OK;
 }
 
 gdn_status gdn_read_device_status(gdn_stream_t stream) {

@@ -143,6 +143,15 @@ GDN_API gdn_status gdn_read_device_status(gdn_stream_t stream);
 /* A static, human-readable name for a status code. */
 GDN_API const char* gdn_status_string(gdn_status s);
 
+/* Number of kernels this library has launched in this process (all devices,
+ * all entry points), counted on the host at each successful launch. */
+GDN_API unsigned long long gdn_kernel_launch_count(void);
+
+/* Name of the kernel gdn_chunk_fwd launches for these arguments, or NULL if
+ * the combination is unsupported.  Static string; never freed. */
+GDN_API const char* gdn_chunk_fwd_kernel_name(int Dk, int Dv, gdn_gate gate_kind,
+                                              gdn_dtype dtype);
+
 /* Library ABI version, currently 1. */
 GDN_API int gdn_abi_version(void);
 
