@@ -70,16 +70,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: gives up after `limit` polls (each try_wait itself blocks for
-// a hardware-defined time slice), sets `*failed` and returns false.  Callers
-// then skip the work that depended on the barrier and finish normally.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait: gives up after `timeout_ns` of wall time (measured on the
+// global timer), sets `*failed` and returns false.  Callers then skip the work
+// that depended on the barrier and finish normally.  Once `*failed` is set,
+// later waits return false at once.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* failed,
-                                          uint32_t limit = 1u << 22) {
+                                          uint64_t timeout_ns = 2000000000ull) {
     if (*failed) return false;
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    *failed = 1;
-    return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > timeout_ns) {
+            *failed = 1;
+            return false;
+        }
+    }
+    return true;
 }
 
 // ------------------------------------------------------------------- TMA
@@ -171,6 +183,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t addr, const float (&v)[16]) {
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// After tcgen05.wait::ld: re-define the loaded registers in program order so
+// the compiler cannot move their uses above the wait (it sees no data
+// dependency between the wait and the registers otherwise).
+template <int N>
+__device__ __forceinline__ void reg_fence(float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
