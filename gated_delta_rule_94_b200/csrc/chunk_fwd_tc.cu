@@ -9,21 +9,27 @@
 // entering state M = S^T [d_k][d_v], G the in-chunk log-decay cumsum:
 //   S  = [K; Q] K^T                 (one 128-row MMA: K K^T and Q K^T)
 //   A  = StrictTril(beta_r e^(G_r-G_i) (K K^T)_ri),  P = Tril(e^(G_r-G_i) (Q K^T)_ri)
-//   T  = (I + A)^-1                 (forward substitution, fp32 CUDA cores)
-//   W^T = K^T (T diag(beta e^G))^T  (MN-major K tile, M = d_k = 128)
+//   T  = (I + A)^-1                 (blocked forward substitution, fp32)
+//   [0; W] = [0; T diag(beta e^G)] K
 //   X  = [T diag(beta); 0] V        = [U; 0]
 //   X += [-W; Q_bar] h              -> rows 0..63: D = U - W h, rows 64..127: Q_bar h
 //   X += [0; P] D                   -> rows 64..127: O = Q_bar h + P D
 //   h  = e^(G_C) h + K^T (diag(e^(G_C - G_i)) D)
-// Every product is a tcgen05.mma with M = 128, operands in 128 B-swizzled
-// shared memory: the K/Q/V tiles exactly as TMA loads them (K-major for the
-// token rows, MN-major when tokens are the reduction dimension), the other
+// Every product is a tcgen05.mma with M = 128; operands live in 128 B-swizzled
+// shared memory: the K/Q/V tiles exactly as TMA loads them (K-major when the
+// tokens are rows, MN-major when they are the reduction dimension), the other
 // operands written by the threads in the same canonical layouts.
 //
-// One CTA of 4 warps owns one (batch, head) and walks its chunks in order;
-// thread t owns TMEM lane t.  TMA prefetches the next chunk's K/Q while the
-// current one is processed.  Every mbarrier wait is bounded; a wait that gives
-// up sets the library status word and the CTA leaves the loop.
+// One CTA owns one (batch, head) and walks its chunks in order, as a pipeline
+// of three warp roles that hand work over through mbarriers:
+//   chain  (warps 0-3):  state -> bf16 operand, state decay, D and D~ from
+//                        TMEM, output epilogue of the previous chunk
+//   prep   (warps 4-11): for chunk n while the chain works on n-1: gates,
+//                        Q_bar, A and P from S, T, the W copy
+//   control (warp 12):   TMA for V and the first tiles, every tcgen05.mma
+// Thread t of a role group owns TMEM lane (warp % 4) * 32 + lane.  Every
+// mbarrier wait is bounded; a wait that gives up sets the library status word
+// and the kernel winds down without further waits.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
@@ -35,35 +41,43 @@ using namespace sm100;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int NT = 128;
-constexpr int LDF = 68;  // fp32 row stride of the A / T scratch (16 B-aligned rows)
+constexpr int NT = 416;          // 13 warps
+constexpr int NCH = 128;         // chain threads (warps 0-3)
+constexpr int NPR = 256;         // prep threads (warps 4-11)
+constexpr int LDF = 72;          // fp32 row stride of the A / T scratch (conflict-free mma fragments)
 
 // Shared memory layout (bytes from a 1 KB-aligned base).
-constexpr uint32_t KQ_STAGE = 32768;         // [K_b0 | Q_b0 | K_b1 | Q_b1], 8 KB each
-constexpr uint32_t OFF_KQ = 0;               // 2 stages
-constexpr uint32_t OFF_V = 65536;            // [V_b0 | V_b1], 8 KB each
-constexpr uint32_t OFF_TW = 81920;           // T diag(beta e^G), K-major [64 r][64 i]
-constexpr uint32_t OFF_TU = 90112;           // T diag(beta), followed by ...
-constexpr uint32_t OFF_Z = 98304;            // ... an 8 KB zero block, followed by ...
-constexpr uint32_t OFF_P = 106496;           // ... P, K-major [64 r][64 i]
-constexpr uint32_t OFF_WQ = 114688;          // MN-major [d][64 r]: -W^T block, Q_bar^T block
-constexpr uint32_t OFF_HB = 147456;          // h (bf16) MN-major [d][64 v] x 2 blocks; after
-constexpr uint32_t OFF_DL = 147456;          //   the c-MMA: D  [i][64 v] x 2 blocks
-constexpr uint32_t OFF_DT = 163840;          //   and D~ = diag(e^(G_C-G_i)) D
-constexpr uint32_t OFF_AF = 180224;          // A fp32 [64][LDF]
+constexpr uint32_t KQ_STAGE = 32768;   // [K_b0 | Q_b0 | K_b1 | Q_b1], 8 KB each, K-major
+constexpr uint32_t OFF_KQ = 0;         // 2 stages
+constexpr uint32_t OFF_V = 65536;      // [V_b0 | V_b1]
+constexpr uint32_t OFF_TU = 81920;     // T diag(beta)          } [T_u; Z] and
+constexpr uint32_t OFF_Z = 90112;      // zero block            } [Z; T_w] are
+constexpr uint32_t OFF_TW = 98304;     // T diag(beta e^G)      } 128-row stacks
+constexpr uint32_t OFF_Z2 = 106496;    // zero block            } [Z2; P]
+constexpr uint32_t OFF_P = 114688;     // P, K-major [64 r][64 i]
+constexpr uint32_t OFF_WQ = 122880;    // [-W_b0 | Qbar_b0 | -W_b1 | Qbar_b1], K-major
+constexpr uint32_t OFF_HB = 155648;    // h (bf16) MN-major [d][64 v] x 2; after the
+constexpr uint32_t OFF_DL = 155648;    //   c-MMA: D [i][64 v] x 2
+constexpr uint32_t OFF_DT = 172032;    //   and D~ = diag(e^(G_C - G_i)) D
+constexpr uint32_t OFF_AF = 188416;    // A fp32 [64][LDF]
 constexpr uint32_t OFF_TF = OFF_AF + 64 * LDF * 4;
-constexpr uint32_t OFF_SMALL = OFF_TF + 64 * LDF * 4;   // G, e^G, e^(G_C-G), beta
-constexpr uint32_t OFF_BAR = OFF_SMALL + 4 * 64 * 4;
-constexpr uint32_t SMEM_USED = OFF_BAR + 64;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;     // alignment slack
-static_assert(OFF_TF + 64 * LDF * 4 == OFF_SMALL, "layout");
+constexpr uint32_t OFF_GATE = OFF_TF + 64 * LDF * 4;   // 2 x {G, e^G, e^(G_C-G), beta, u, w, flag}
+constexpr int GATE_FLOATS = 7 * 64;
+constexpr uint32_t OFF_BAR = OFF_GATE + 2 * GATE_FLOATS * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 32 * 8 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // TMEM columns (512 allocated).
 constexpr uint32_t TM_H = 0;      // state, lanes d, 128 columns v (fp32)
-constexpr uint32_t TM_X = 128;    // [U->D ; Q_bar h->O], lanes r / 64 + r, 128 columns v
-constexpr uint32_t TM_S = 256;    // [K K^T ; Q K^T], 64 columns
-constexpr uint32_t TM_W = 320;    // W^T, lanes d, 64 columns r
+constexpr uint32_t TM_X0 = 128;   // X for even chunks, lanes r / 64 + r, 128 columns v
+constexpr uint32_t TM_X1 = 256;   // X for odd chunks
+constexpr uint32_t TM_SW = 384;   // S (64 columns), then [0; W] (128 columns)
+
+// mbarrier indices
+enum Bar {
+    B_KQ0, B_KQ1, B_VFULL, B_SDONE, B_WUDONE, B_CDONE, B_DDONE,
+    B_GREADY0, B_GREADY1, B_TREADY, B_WQREADY, B_HBREADY, B_DREADY, B_FINAL, B_COUNT
+};
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
@@ -80,52 +94,118 @@ __device__ __forceinline__ void st_row_chunk(uint8_t* tile, int row, int j, cons
     *reinterpret_cast<uint4*>(tile + sw128_offset(row, 8 * j)) = w;
 }
 
-// T = (I + A)^-1 for strictly lower-triangular A (64 x 64, fp32), blocked in
-// 16 x 16 tiles: the four diagonal tiles by column-parallel substitution, then
-// the off-diagonal tiles by distance, T_ij = -T_ii sum_{j<=k<i} A_ik T_kj.
-// The strictly upper tiles of Tm serve as scratch for the inner sums.
-__device__ __forceinline__ void forward_substitution(const float* A, float* Tm, int tid) {
-    if (tid < 64) {
-        const int o = 16 * (tid >> 4), c = tid & 15;
-        float x[16];
+__device__ __forceinline__ void named_bar(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void ld_cols(uint32_t addr, float (&v)[N]) {
+    static_assert(N % 16 == 0, "");
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = 0.f;
+    for (int j = 0; j < N / 16; ++j)
+        tmem_ld16(addr + 16 * j, *reinterpret_cast<float(*)[16]>(v + 16 * j));
+    tmem_wait_ld();
+    reg_fence(v);
+}
+
+template <int N>
+__device__ __forceinline__ void st_cols(uint32_t addr, float (&v)[N]) {
 #pragma unroll
-            for (int i = 0; i < r; ++i) acc = fmaf(A[(o + r) * LDF + o + i], x[i], acc);
-            x[r] = (r == c) ? 1.f : (r < c ? 0.f : -acc);
+    for (int j = 0; j < N / 16; ++j)
+        tmem_st16(addr + 16 * j, *reinterpret_cast<float(*)[16]>(v + 16 * j));
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// d (16 x 8, fp32) += a (16 x 8) * b (8 x 8), warp-level tensor-core MMA on tf32
+// operands.  Fragments (g = lane / 4, t = lane % 4): a0 (g, t), a1 (g + 8, t),
+// a2 (g, t + 4), a3 (g + 8, t + 4); b0 (k = t, n = g), b1 (k = t + 4, n = g);
+// d0 (g, 2t), d1 (g, 2t + 1), d2 (g + 8, 2t), d3 (g + 8, 2t + 1).
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const float* M, int r0, int k0,
+                                                const float* N, int kn0, int n0, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t a0 = to_tf32(M[(r0 + g) * LDF + k0 + t]);
+    const uint32_t a1 = to_tf32(M[(r0 + g + 8) * LDF + k0 + t]);
+    const uint32_t a2 = to_tf32(M[(r0 + g) * LDF + k0 + t + 4]);
+    const uint32_t a3 = to_tf32(M[(r0 + g + 8) * LDF + k0 + t + 4]);
+    const uint32_t b0 = to_tf32(N[(kn0 + t) * LDF + n0 + g]);
+    const uint32_t b1 = to_tf32(N[(kn0 + t + 4) * LDF + n0 + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void store_16x8(float* X, int r0, int n0, const float (&d)[4], float s,
+                                           int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2*>(X + (r0 + g) * LDF + n0 + 2 * t) = make_float2(s * d[0], s * d[1]);
+    *reinterpret_cast<float2*>(X + (r0 + g + 8) * LDF + n0 + 2 * t) = make_float2(s * d[2], s * d[3]);
+}
+
+// T = (I + A)^-1 for strictly lower-triangular A (64 x 64, fp32), 256 threads
+// (8 warps).  (1) the four diagonal 16 x 16 inverses by right-looking
+// substitution on CUDA cores, one column per thread; (2) 16 -> 32:
+// T_10 = -T_11 (A_10 T_00) for the two diagonal 32 x 32 blocks; (3) 32 -> 64:
+// the same with 32 x 32 blocks.  The block products run as warp MMAs on tf32
+// operands with fp32 accumulation (T is rounded to bf16 right after, so the
+// tf32 operand rounding stays well below that); the inner product X goes
+// through the strictly upper part of Tm, which T never uses.
+__device__ __forceinline__ void forward_substitution(const float* A, float* Tm, int pt) {
+    const int lane = pt & 31, w = pt >> 5;
+    if (pt < 64) {
+        const int o = 16 * (pt >> 4), c = pt & 15;
+        float p[16], x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) p[r] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            x[i] = (i == c) ? 1.f : (i < c ? 0.f : -p[i]);
+#pragma unroll
+            for (int r = i + 1; r < 16; ++r) p[r] = fmaf(A[(o + r) * LDF + o + i], x[i], p[r]);
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) Tm[(o + r) * LDF + o + c] = x[r];
     }
-    __syncthreads();
-#pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-        const int nb = 4 - d;
-        for (int e = tid; e < nb * 256; e += NT) {
-            const int j = e >> 8, i = j + d, r = (e >> 4) & 15, c = e & 15;
-            const float* arow = A + (16 * i + r) * LDF;
-            float acc = 0.f;
-#pragma unroll 1
-            for (int k = j; k < i; ++k) {
+    named_bar(2, NPR);
+    if (w < 4) {   // 16 -> 32: pair pr, n-tile nt of the 16 x 16 block (2pr+1, 2pr)
+        const int pr = w >> 1, nt = w & 1;
+        const int ri = 16 * (2 * pr + 1), cj = 16 * (2 * pr);
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    acc = fmaf(arow[16 * k + q], Tm[(16 * k + q) * LDF + 16 * j + c], acc);
-            }
-            Tm[(16 * j + r) * LDF + 16 * i + c] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nb * 256; e += NT) {
-            const int j = e >> 8, i = j + d, r = (e >> 4) & 15, c = e & 15;
-            float acc = 0.f;
+        for (int ks = 0; ks < 2; ++ks) mma_tf32_16x8x8(d, A, ri, cj + 8 * ks, Tm, cj + 8 * ks, cj + 8 * nt, lane);
+        store_16x8(Tm, cj, ri + 8 * nt, d, 1.f, lane);       // X in the upper block (cj, ri)
+        __syncwarp();
+        float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-                if (q <= r)
-                    acc = fmaf(Tm[(16 * i + r) * LDF + 16 * i + q], Tm[(16 * j + q) * LDF + 16 * i + c], acc);
-            Tm[(16 * i + r) * LDF + 16 * j + c] = -acc;
-        }
-        __syncthreads();
+        for (int ks = 0; ks < 2; ++ks) mma_tf32_16x8x8(e, Tm, ri, ri + 8 * ks, Tm, cj + 8 * ks, ri + 8 * nt, lane);
+        store_16x8(Tm, ri, cj + 8 * nt, e, -1.f, lane);
     }
+    named_bar(2, NPR);
+    const int rt = w >> 2, nt = w & 3;    // 32 -> 64: row tile rt (16 rows), n-tile nt (8 cols)
+    {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            if (8 * ks + 7 >= 8 * nt)      // rows of T32_00 above its diagonal are zero
+                mma_tf32_16x8x8(d, A, 32 + 16 * rt, 8 * ks, Tm, 8 * ks, 8 * nt, lane);
+        store_16x8(Tm, 16 * rt, 32 + 8 * nt, d, 1.f, lane);  // X in the upper-right quadrant
+    }
+    named_bar(2, NPR);
+    {
+        float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            if (8 * ks <= 16 * rt + 15)    // columns of T32_11 right of its diagonal are zero
+                mma_tf32_16x8x8(e, Tm + 32, 32 + 16 * rt, 8 * ks, Tm + 32, 8 * ks, 8 * nt, lane);
+        store_16x8(Tm, 32 + 16 * rt, 8 * nt, e, -1.f, lane);
+    }
+    named_bar(2, NPR);
 }
 
 struct TcMaps {
@@ -139,34 +219,20 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
-    float* sG = reinterpret_cast<float*>(sm + OFF_SMALL);
-    float* sGam = sG + 64;
-    float* sFt = sG + 128;
-    float* sBeta = sG + 192;
     float* Af = reinterpret_cast<float*>(sm + OFF_AF);
     float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
-    uint64_t* bar_kq = reinterpret_cast<uint64_t*>(sm + OFF_BAR);   // [2]
-    uint64_t* bar_v = bar_kq + 2;
-    uint64_t* bar_mma = bar_kq + 3;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     __shared__ uint32_t s_tmem;
-    __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, T = p.T;
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int NC = (T + C - 1) / C;
-    const __nv_bfloat16* gq = static_cast<const __nv_bfloat16*>(p.g);
-    const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(p.beta);
     int failed = 0;
-    uint32_t mma_phase = 0;
 
     if (tid == 0) {
-        mbar_init(&bar_kq[0], 1);
-        mbar_init(&bar_kq[1], 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
-        s_abort = 0;
         prefetch_tmap(&maps.q);
         prefetch_tmap(&maps.k);
         prefetch_tmap(&maps.v);
@@ -175,324 +241,336 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
         tmem_alloc(&s_tmem, 512);
         tmem_relinquish();
     }
-    for (int i = tid; i < 512; i += NT) reinterpret_cast<uint4*>(sm + OFF_Z)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < 1024; i += NT) {   // the two zero blocks
+        const uint32_t off = (i < 512) ? OFF_Z + 16 * i : OFF_Z2 + 16 * (i - 512);
+        *reinterpret_cast<uint4*>(sm + off) = make_uint4(0, 0, 0, 0);
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tH = tmem + TM_H, tX = tmem + TM_X, tS = tmem + TM_S, tW = tmem + TM_W;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
 
-    auto load_kq = [&](int n, int s) {
-        mbar_arrive_expect_tx(&bar_kq[s], 4 * 8192);
+    auto gate_buf = [&](int n) { return reinterpret_cast<float*>(sm + OFF_GATE) + (n & 1) * GATE_FLOATS; };
+    auto wait = [&](int bar, uint32_t parity) {
+        if (!mbar_wait(&bars[bar], parity, &failed)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+    };
+    auto load_kq = [&](int n) {
+        const int s = n & 1;
+        mbar_arrive_expect_tx(&bars[B_KQ0 + s], 4 * 8192);
         uint8_t* st = sm + OFF_KQ + s * KQ_STAGE;
         for (int blk = 0; blk < 2; ++blk) {
-            tma_load_3d(st + blk * 16384, &maps.k, &bar_kq[s], h * D + 64 * blk, n * C, b);
-            tma_load_3d(st + blk * 16384 + 8192, &maps.q, &bar_kq[s], h * D + 64 * blk, n * C, b);
+            tma_load_3d(st + blk * 16384, &maps.k, &bars[B_KQ0 + s], h * D + 64 * blk, n * C, b);
+            tma_load_3d(st + blk * 16384 + 8192, &maps.q, &bars[B_KQ0 + s], h * D + 64 * blk, n * C, b);
         }
     };
     auto load_v = [&](int n) {
-        mbar_arrive_expect_tx(bar_v, 2 * 8192);
+        mbar_arrive_expect_tx(&bars[B_VFULL], 2 * 8192);
         for (int blk = 0; blk < 2; ++blk)
-            tma_load_3d(sm + OFF_V + blk * 8192, &maps.v, bar_v, h * D + 64 * blk, n * C, b);
-    };
-    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-        if (!mbar_wait(bar, parity, &failed)) {
-            atomicOr(p.status, kStatusTimeout);
-            s_abort = 1;
-        }
-        __syncwarp();
+            tma_load_3d(sm + OFF_V + blk * 8192, &maps.v, &bars[B_VFULL], h * D + 64 * blk, n * C, b);
     };
 
-    // initial state -> TMEM, row d = tid
-    {
-        const float* s0 = p.s0 ? p.s0 + ((size_t)bh * D + tid) * D : nullptr;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 16) {
-            float v[16];
+    if (warp == 12) {
+        // =========================== control: TMA + every tcgen05.mma
+        const bool leader = lane == 0;   // issues only while no wait has failed
+        auto issue_S = [&](int n) {
+            const uint32_t st = sb + OFF_KQ + (n & 1) * KQ_STAGE;
+            const uint32_t id = idesc_bf16_f32(128, 64, false, false);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = s0 ? s0[c0 + j] : 0.f;
-            tmem_st16(tH + lane_off + c0, v);
-        }
-        tmem_wait_st();
-    }
-    if (tid == 0 && NC > 0) {
-        load_kq(0, 0);
-        load_v(0);
-    }
-    float g_next = 0.f, b_next = 0.f;
-    if (tid < 64 && tid < T) {
-        const size_t tok = ((size_t)b * T + tid) * H + h;
-        b_next = __bfloat162float(gb[tok]);
-        if constexpr (GATE == kGateScalar) g_next = __bfloat162float(gq[tok]);
-    }
-
-#pragma unroll 1
-    for (int n = 0; n < NC; ++n) {
-        const int s = n & 1;
-        const int t0 = n * C;
-        const int nval = min(C, T - t0);
-        uint8_t* stage = sm + OFF_KQ + s * KQ_STAGE;
-        const uint32_t stage_a = sb + OFF_KQ + s * KQ_STAGE;
-
-        // ---- gates of this chunk
-        if (tid < 64) {
-            sG[tid] = g_next;
-            sBeta[tid] = b_next;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            if constexpr (GATE == kGateScalar) {
-                const float a0 = sG[2 * lane], a1 = sG[2 * lane + 1];
-                float incl = a0 + a1;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += y;
-                }
-                float excl = __shfl_up_sync(0xffffffffu, incl, 1);
-                if (lane == 0) excl = 0.f;
-                const float G0 = excl + a0, G1 = incl;
-                const float Gl = __shfl_sync(0xffffffffu, incl, 31);
-                sG[2 * lane] = G0;
-                sG[2 * lane + 1] = G1;
-                sGam[2 * lane] = expf(G0);
-                sGam[2 * lane + 1] = expf(G1);
-                sFt[2 * lane] = expf(Gl - G0);
-                sFt[2 * lane + 1] = expf(Gl - G1);
-            } else {
-                sG[2 * lane] = sG[2 * lane + 1] = 0.f;
-                sGam[2 * lane] = sGam[2 * lane + 1] = 1.f;
-                sFt[2 * lane] = sFt[2 * lane + 1] = 1.f;
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t a = st + (k >> 2) * 16384 + (k & 3) * 32;
+                mma_bf16(tmem + TM_SW, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, k > 0);
             }
-        }
-        // ---- S = [K; Q] K^T
-        if (tid == 0) {
-            if (mbar_wait(&bar_kq[s], (n >> 1) & 1, &failed)) {
-                const uint32_t id = idesc_bf16_f32(128, 64, false, false);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t a = stage_a + (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_bf16(tS, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, k > 0);
-                }
-            }
-            mma_commit(bar_mma);
-            if (n + 1 < NC) {
-                fence_async_smem();
-                load_kq(n + 1, s ^ 1);
-            }
-        }
-        if (tid < 64 && n + 1 < NC) {
-            g_next = 0.f;
-            b_next = 0.f;
-            if (t0 + C + tid < T) {
-                const size_t tok = ((size_t)b * T + t0 + C + tid) * H + h;
-                b_next = __bfloat162float(gb[tok]);
-                if constexpr (GATE == kGateScalar) g_next = __bfloat162float(gq[tok]);
-            }
-        }
-        wait_all(&bar_kq[s], (n >> 1) & 1);
-        __syncthreads();
-        if (s_abort) break;
-
-        // ---- Q_bar^T (MN-major [d][64 r]) = e^(G_r) Q[r][d], thread d
-        {
-            const int d = tid, dc = d & 63;
-            const uint8_t* qt = stage + (d >> 6) * 16384 + 8192;
-            uint8_t* dst = sm + OFF_WQ + 16384;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint32_t w[4];
-#pragma unroll
-                for (int q2 = 0; q2 < 4; ++q2) {
-                    const int r0 = 8 * j + 2 * q2;
-                    const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qt + sw128_offset(r0, dc)));
-                    const float x1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qt + sw128_offset(r0 + 1, dc)));
-                    w[q2] = pack_bf16(x0 * sGam[r0], x1 * sGam[r0 + 1]);
-                }
-                *reinterpret_cast<uint4*>(dst + sw128_offset(d, 8 * j)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-        }
-        // ---- A (fp32) and P (bf16) from S
-        wait_all(bar_mma, mma_phase & 1);
-        ++mma_phase;
-        tc_fence_after();
-        {
-            float sv[64];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tmem_ld16(tS + lane_off + 16 * j, *reinterpret_cast<float(*)[16]>(sv + 16 * j));
-            tmem_wait_ld();
-            reg_fence(sv);
-            if (tid < 64) {
-                const int r = tid;
-                const float Gr = sG[r], br = sBeta[r];
-                float* arow = Af + r * LDF;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) arow[i] = (i < r) ? br * expf(Gr - sG[i]) * sv[i] : 0.f;
-            } else {
-                const int r = tid - 64;
-                const float Gr = sG[r];
-#pragma unroll
-                for (int i = 0; i < 64; ++i) sv[i] = (i <= r) ? expf(Gr - sG[i]) * sv[i] : 0.f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) st_row_chunk(sm + OFF_P, r, j, sv + 8 * j, 1.f);
-            }
-        }
-        fence_async_smem();
-        __syncthreads();
-        if (s_abort) break;
-
-        // ---- T = (I + A)^-1, then T diag(beta e^G) and T diag(beta) as bf16
-        forward_substitution(Af, Tf, tid);
-        {
-            const int r = tid >> 1, half = tid & 1;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int j = 4 * half + jj;
-                float tw[8], tu[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = 8 * j + e;
-                    const float tv = (i <= r) ? Tf[r * LDF + i] : 0.f;
-                    tu[e] = tv * sBeta[i];
-                    tw[e] = tu[e] * sGam[i];
-                }
-                st_row_chunk(sm + OFF_TW, r, j, tw, 1.f);
-                st_row_chunk(sm + OFF_TU, r, j, tu, 1.f);
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (s_abort) break;
-
-        // ---- W^T = K^T (T diag(beta e^G))^T ; X = [T diag(beta); 0] V
-        if (tid == 0) {
-            if (mbar_wait(bar_v, n & 1, &failed)) {
-                const uint32_t idw = idesc_bf16_f32(128, 64, true, false);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16(tW, sdesc_sw128(stage_a + k * 2048, 16384, 1024),
-                             sdesc_sw128(sb + OFF_TW + k * 32, 16, 1024), idw, k > 0);
-                const uint32_t idu = idesc_bf16_f32(128, 128, false, true);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16(tX, sdesc_sw128(sb + OFF_TU + k * 32, 16, 1024),
-                             sdesc_sw128(sb + OFF_V + k * 2048, 8192, 1024), idu, k > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        wait_all(bar_mma, mma_phase & 1);
-        ++mma_phase;
-        tc_fence_after();
-        if (tid == 0 && n + 1 < NC) {
+            mma_commit(&bars[B_SDONE]);
+        };
+        if (leader) {
             fence_async_smem();
-            load_v(n + 1);
+            load_kq(0);
+            if (NC > 1) load_kq(1);
+            load_v(0);
         }
-        // -W^T -> MN-major block 0 of WQ, row d = tid
-        {
-            float wv[64];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tmem_ld16(tW + lane_off + 16 * j, *reinterpret_cast<float(*)[16]>(wv + 16 * j));
-            tmem_wait_ld();
-            reg_fence(wv);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) st_row_chunk(sm + OFF_WQ, tid, j, wv + 8 * j, -1.f);
-        }
-        // state -> bf16 h (MN-major [d][64 v] x 2), then state *= e^(G_C) in TMEM
-        {
-            const float gam = sGam[63];
+        wait(B_KQ0, 0);
+        tc_fence_after();
+        if (leader && !failed) issue_S(0);
 #pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float hv[64];
+        for (int n = 0; n < NC; ++n) {
+            const int s = n & 1;
+            const uint32_t st = sb + OFF_KQ + s * KQ_STAGE;
+            const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
+            wait(B_TREADY, n & 1);
+            wait(B_VFULL, n & 1);
+            tc_fence_after();
+            if (leader && !failed) {
+                const uint32_t idw = idesc_bf16_f32(128, 128, false, true);
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    tmem_ld16(tH + lane_off + 64 * half + 16 * j, *reinterpret_cast<float(*)[16]>(hv + 16 * j));
-                tmem_wait_ld();
-                reg_fence(hv);
+                for (int k = 0; k < 4; ++k)   // [0; W] = [Z; T_w] K
+                    mma_bf16(tmem + TM_SW, sdesc_sw128(sb + OFF_Z + k * 32, 16, 1024),
+                             sdesc_sw128(st + k * 2048, 16384, 1024), idw, k > 0);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) st_row_chunk(sm + OFF_HB + half * 16384, tid, j, hv + 8 * j, 1.f);
-                if constexpr (GATE != kGateNone) {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) hv[e] *= gam;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tmem_st16(tH + lane_off + 64 * half + 16 * j, *reinterpret_cast<float(*)[16]>(hv + 16 * j));
+                for (int k = 0; k < 4; ++k)   // X = [T_u; Z] V
+                    mma_bf16(tX, sdesc_sw128(sb + OFF_TU + k * 32, 16, 1024),
+                             sdesc_sw128(sb + OFF_V + k * 2048, 8192, 1024), idw, k > 0);
+                mma_commit(&bars[B_WUDONE]);
+            }
+            wait(B_WQREADY, n & 1);
+            wait(B_HBREADY, n & 1);
+            tc_fence_after();
+            if (leader && !failed) {
+                if (n + 1 < NC) {
+                    fence_async_smem();
+                    load_v(n + 1);
                 }
+                const uint32_t idc = idesc_bf16_f32(128, 128, false, true);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // X += [-W; Q_bar] h
+                    mma_bf16(tX, sdesc_sw128(sb + OFF_WQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                             sdesc_sw128(sb + OFF_HB + k * 2048, 16384, 1024), idc, true);
+                mma_commit(&bars[B_CDONE]);
+            }
+            if (n + 1 < NC) {
+                wait(B_KQ0 + (s ^ 1), ((n + 1) >> 1) & 1);
+                tc_fence_after();
+                if (leader && !failed) issue_S(n + 1);
+            }
+            wait(B_DREADY, n & 1);
+            tc_fence_after();
+            if (leader && !failed) {
+                const uint32_t id2 = idesc_bf16_f32(128, 128, true, true);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)   // state += K^T D~
+                    mma_bf16(tmem + TM_H, sdesc_sw128(st + k * 2048, 16384, 1024),
+                             sdesc_sw128(sb + OFF_DT + k * 2048, 8192, 1024), id2, true);
+                const uint32_t id1 = idesc_bf16_f32(128, 128, false, true);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)   // X += [Z2; P] D
+                    mma_bf16(tX, sdesc_sw128(sb + OFF_Z2 + k * 32, 16, 1024),
+                             sdesc_sw128(sb + OFF_DL + k * 2048, 8192, 1024), id1, true);
+                mma_commit(&bars[B_DDONE]);
+            }
+        }
+        // nothing issued by this warp may still run when TMEM is released
+        if (leader) mma_commit(&bars[B_FINAL]);
+        int final_failed = 0;
+        if (!mbar_wait(&bars[B_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+    } else if (warp >= 4) {
+        // =========================== prep: gates, Q_bar, A / P, T, W copy
+        const int pt = tid - NCH;                 // 0..255
+        const int q4 = warp & 3, ch = (warp - 4) >> 2;
+        const int L = q4 * 32 + lane;             // TMEM lane of this thread
+        const __nv_bfloat16* gq = static_cast<const __nv_bfloat16*>(p.g);
+        const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(p.beta);
+        float g_next = 0.f, b_next = 0.f;
+        if (pt < 64 && pt < T) {
+            const size_t tok = ((size_t)b * T + pt) * H + h;
+            b_next = __bfloat162float(gb[tok]);
+            if constexpr (GATE == kGateScalar) g_next = __bfloat162float(gq[tok]);
+        }
+#pragma unroll 1
+        for (int n = 0; n < NC; ++n) {
+            const int s = n & 1;
+            float* gbuf = gate_buf(n);   // G, e^G, e^(G_C - G), beta
+            uint8_t* stage = sm + OFF_KQ + s * KQ_STAGE;
+            // ---- gates
+            if (pt < 64) {
+                gbuf[pt] = g_next;
+                gbuf[192 + pt] = b_next;
+            }
+            named_bar(2, NPR);
+            if (pt < 32) {
+                if constexpr (GATE == kGateScalar) {
+                    const float a0 = gbuf[2 * lane], a1 = gbuf[2 * lane + 1];
+                    float incl = a0 + a1;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, incl, off);
+                        if (lane >= off) incl += y;
+                    }
+                    float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+                    if (lane == 0) excl = 0.f;
+                    const float G0 = excl + a0, G1 = incl;
+                    const float Gl = __shfl_sync(0xffffffffu, incl, 31);
+                    const float Gm = __shfl_sync(0xffffffffu, incl, 15);   // G_31
+                    const float G00 = __shfl_sync(0xffffffffu, G0, 0);
+                    gbuf[2 * lane] = G0;
+                    gbuf[2 * lane + 1] = G1;
+                    gbuf[64 + 2 * lane] = expf(G0);
+                    gbuf[64 + 2 * lane + 1] = expf(G1);
+                    gbuf[128 + 2 * lane] = expf(Gl - G0);
+                    gbuf[128 + 2 * lane + 1] = expf(Gl - G1);
+                    // e^(G_r - G_i) = u_r w_i about the middle of the chunk; both
+                    // factors stay finite while the in-chunk decay is below e^160
+                    gbuf[256 + 2 * lane] = expf(G0 - Gm);
+                    gbuf[256 + 2 * lane + 1] = expf(G1 - Gm);
+                    gbuf[320 + 2 * lane] = expf(Gm - G0);
+                    gbuf[320 + 2 * lane + 1] = expf(Gm - G1);
+                    if (lane == 0) gbuf[384] = (G00 - Gl < 160.f) ? 1.f : 0.f;
+                } else {
+                    gbuf[2 * lane] = gbuf[2 * lane + 1] = 0.f;
+                    gbuf[64 + 2 * lane] = gbuf[64 + 2 * lane + 1] = 1.f;
+                    gbuf[128 + 2 * lane] = gbuf[128 + 2 * lane + 1] = 1.f;
+                    gbuf[256 + 2 * lane] = gbuf[256 + 2 * lane + 1] = 1.f;
+                    gbuf[320 + 2 * lane] = gbuf[320 + 2 * lane + 1] = 1.f;
+                    if (lane == 0) gbuf[384] = 1.f;
+                }
+            }
+            if (pt < 64 && n + 1 < NC) {
+                g_next = 0.f;
+                b_next = 0.f;
+                if ((n + 1) * C + pt < T) {
+                    const size_t tok = ((size_t)b * T + (n + 1) * C + pt) * H + h;
+                    b_next = __bfloat162float(gb[tok]);
+                    if constexpr (GATE == kGateScalar) g_next = __bfloat162float(gq[tok]);
+                }
+            }
+            named_bar(2, NPR);
+            if (pt == 0) mbar_arrive(&bars[B_GREADY0 + s]);
+            const float* sG = gbuf;
+            const float* sGam = gbuf + 64;
+            const float* sBeta = gbuf + 192;
+
+            // ---- S is in TMEM (this also means the c-MMA of chunk n-1 is done)
+            wait(B_SDONE, n & 1);
+            tc_fence_after();
+            // Q_bar = diag(e^G) Q into the Q rows of WQ (same swizzled layout)
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int idx = pt + NPR * it;            // 16-byte chunk 0..1023
+                const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+                const uint32_t off = blk * 16384 + 8192 + r * 128 + j * 16;
+                uint4 raw = *reinterpret_cast<const uint4*>(stage + off);
+                const float gmul = sGam[r];
+                __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+                uint4 outv;
+                uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(e2[e]);
+                    o32[e] = pack_bf16(f.x * gmul, f.y * gmul);
+                }
+                *reinterpret_cast<uint4*>(sm + OFF_WQ + off) = outv;
+            }
+            // A (fp32, rows 0..63) and P (bf16, rows 64..127, kept in registers)
+            uint32_t pP[16];
+            {
+                float sv[32];
+                ld_cols<32>(tmem + TM_SW + lane_off + 32 * ch, sv);
+                const float* sU = gbuf + 256;
+                const float* sW = gbuf + 320;
+                const bool fact = gbuf[384] != 0.f;
+                if (L < 64) {
+                    const int r = L;
+                    if (fact) {
+                        const float cr = sBeta[r] * sU[r];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int i = 32 * ch + e;
+                            sv[e] = (i < r) ? cr * sW[i] * sv[e] : 0.f;
+                        }
+                    } else {
+                        const float Gr = sG[r], br = sBeta[r];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int i = 32 * ch + e;
+                            sv[e] = (i < r) ? br * __expf(Gr - sG[i]) * sv[e] : 0.f;
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(Af + r * LDF + 32 * ch + e) =
+                            make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                } else {
+                    const int r = L - 64;
+                    if (fact) {
+                        const float cr = sU[r];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int i = 32 * ch + e;
+                            sv[e] = (i <= r) ? cr * sW[i] * sv[e] : 0.f;
+                        }
+                    } else {
+                        const float Gr = sG[r];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int i = 32 * ch + e;
+                            sv[e] = (i <= r) ? __expf(Gr - sG[i]) * sv[e] : 0.f;
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) pP[e >> 1] = pack_bf16(sv[e], sv[e + 1]);
+                }
+            }
+            named_bar(2, NPR);
+            forward_substitution(Af, Tf, pt);
+            // T diag(beta) and T diag(beta e^G) as bf16, K-major [r][i]
+            {
+                const int r = pt >> 2, j0 = 2 * (pt & 3);
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int j = j0 + jj;
+                    float tu[8], tw[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = 8 * j + e;
+                        const float tv = (i <= r) ? Tf[r * LDF + i] : 0.f;
+                        tu[e] = tv * sBeta[i];
+                        tw[e] = tu[e] * sGam[i];
+                    }
+                    st_row_chunk(sm + OFF_TU, r, j, tu, 1.f);
+                    st_row_chunk(sm + OFF_TW, r, j, tw, 1.f);
+                }
+            }
+            // P once the d-MMAs of chunk n-1 are done with the buffer
+            if (n > 0) wait(B_DDONE, (n - 1) & 1);
+            if (L >= 64) {
+                const int r = L - 64;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                    *reinterpret_cast<uint4*>(sm + OFF_P + sw128_offset(r, 8 * (4 * ch + jj))) =
+                        make_uint4(pP[4 * jj], pP[4 * jj + 1], pP[4 * jj + 2], pP[4 * jj + 3]);
+            }
+            fence_async_smem();
+            named_bar(2, NPR);
+            if (pt == 0) mbar_arrive(&bars[B_TREADY]);
+            // ---- -W (TMEM lanes 64..127) -> the W rows of WQ
+            wait(B_WUDONE, n & 1);
+            tc_fence_after();
+            if (L >= 64) {
+                const int r = L - 64;
+                float wv[64];
+                ld_cols<64>(tmem + TM_SW + lane_off + 64 * ch, wv);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) st_row_chunk(sm + OFF_WQ + ch * 16384, r, j, wv + 8 * j, -1.f);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_bar(2, NPR);
+            if (pt == 0) mbar_arrive(&bars[B_WQREADY]);
+        }
+    } else {
+        // =========================== chain: state, D, output
+        {
+            const float* s0 = p.s0 ? p.s0 + ((size_t)bh * D + tid) * D : nullptr;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = s0 ? s0[c0 + j] : 0.f;
+                tmem_st16(tmem + TM_H + lane_off + c0, v);
             }
             tmem_wait_st();
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (s_abort) break;
-
-        // ---- X += [-W; Q_bar] h
-        if (tid == 0) {
-            const uint32_t id = idesc_bf16_f32(128, 128, true, true);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_bf16(tX, sdesc_sw128(sb + OFF_WQ + k * 2048, 16384, 1024),
-                         sdesc_sw128(sb + OFF_HB + k * 2048, 16384, 1024), id, true);
-            mma_commit(bar_mma);
-        }
-        wait_all(bar_mma, mma_phase & 1);
-        ++mma_phase;
-        tc_fence_after();
-        if (tid < 64) {   // D rows (lanes 0..63) -> D and D~ as MN-major [i][64 v] x 2
-            const float ft = sFt[tid];
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float dv[64];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    tmem_ld16(tX + lane_off + 64 * half + 16 * j, *reinterpret_cast<float(*)[16]>(dv + 16 * j));
-                tmem_wait_ld();
-                reg_fence(dv);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    st_row_chunk(sm + OFF_DL + half * 8192, tid, j, dv + 8 * j, 1.f);
-                    st_row_chunk(sm + OFF_DT + half * 8192, tid, j, dv + 8 * j, ft);
-                }
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (s_abort) break;
-
-        // ---- state += K^T D~ ; X += [0; P] D
-        if (tid == 0) {
-            const uint32_t id2 = idesc_bf16_f32(128, 128, true, true);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                mma_bf16(tH, sdesc_sw128(stage_a + k * 2048, 16384, 1024),
-                         sdesc_sw128(sb + OFF_DT + k * 2048, 8192, 1024), id2, true);
-            const uint32_t id1 = idesc_bf16_f32(128, 128, false, true);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                mma_bf16(tX, sdesc_sw128(sb + OFF_Z + k * 32, 16, 1024),
-                         sdesc_sw128(sb + OFF_DL + k * 2048, 8192, 1024), id1, true);
-            mma_commit(bar_mma);
-        }
-        wait_all(bar_mma, mma_phase & 1);
-        ++mma_phase;
-        tc_fence_after();
-        if (tid >= 64) {   // O rows (lanes 64..127)
-            const int r = tid - 64;
+        auto out_epilogue = [&](int m) {   // chunk m's O, warps 2-3 (TMEM lanes 64..127)
+            const int r = tid - 64, t0 = m * C;
+            const int nval = min(C, T - t0);
+            const uint32_t tX = tmem + ((m & 1) ? TM_X1 : TM_X0);
             __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + (((size_t)b * T + t0 + r) * H + h) * D;
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 float ov[64];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    tmem_ld16(tX + lane_off + 64 * half + 16 * j, *reinterpret_cast<float(*)[16]>(ov + 16 * j));
-                tmem_wait_ld();
-                reg_fence(ov);
+                ld_cols<64>(tX + lane_off + 64 * half, ov);
                 if (r < nval) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -505,31 +583,92 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
                     }
                 }
             }
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (s_abort) break;
-    }
-
-    if (!s_abort && p.s_out) {
-        float* dst = p.s_out + ((size_t)bh * D + tid) * D;
+        };
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            float hv[64];
+        for (int n = 0; n < NC; ++n) {
+            const int s = n & 1;
+            if (n > 0) {
+                wait(B_DDONE, (n - 1) & 1);
+                tc_fence_after();
+                if (tid == 0 && n + 1 < NC) {
+                    fence_async_smem();
+                    load_kq(n + 1);
+                }
+            }
+            // state -> bf16 operand h (MN-major [d][64 v] x 2), row d = tid
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float hv[64];
+                ld_cols<64>(tmem + TM_H + lane_off + 64 * half, hv);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                tmem_ld16(tH + lane_off + 64 * half + 16 * j, *reinterpret_cast<float(*)[16]>(hv + 16 * j));
-            tmem_wait_ld();
-            reg_fence(hv);
+                for (int j = 0; j < 8; ++j) st_row_chunk(sm + OFF_HB + half * 16384, tid, j, hv + 8 * j, 1.f);
+            }
+            fence_async_smem();
+            named_bar(1, NCH);
+            if (tid == 0) mbar_arrive(&bars[B_HBREADY]);
+            // state *= e^(G_C) (before the state update of this chunk)
+            wait(B_GREADY0 + s, (n >> 1) & 1);
+            const float* gbuf = gate_buf(n);
+            if constexpr (GATE != kGateNone) {
+                const float gam = gbuf[64 + 63];
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float hv[64];
+                    ld_cols<64>(tmem + TM_H + lane_off + 64 * half, hv);
 #pragma unroll
-            for (int e = 0; e < 64; e += 4)
-                *reinterpret_cast<float4*>(dst + 64 * half + e) = make_float4(hv[e], hv[e + 1], hv[e + 2], hv[e + 3]);
+                    for (int e = 0; e < 64; ++e) hv[e] *= gam;
+                    st_cols<64>(tmem + TM_H + lane_off + 64 * half, hv);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            named_bar(1, NCH);
+            if (warp >= 2) {
+                if (n > 0) out_epilogue(n - 1);
+            } else {
+                wait(B_CDONE, n & 1);
+                tc_fence_after();
+                const float ft = gbuf[128 + tid];
+                const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float dv[64];
+                    ld_cols<64>(tX + lane_off + 64 * half, dv);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        st_row_chunk(sm + OFF_DL + half * 8192, tid, j, dv + 8 * j, 1.f);
+                        st_row_chunk(sm + OFF_DT + half * 8192, tid, j, dv + 8 * j, ft);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_bar(1, NCH);
+            if (tid == 0) mbar_arrive(&bars[B_DREADY]);
+        }
+        if (NC > 0) {
+            wait(B_DDONE, (NC - 1) & 1);
+            tc_fence_after();
+            if (warp >= 2) out_epilogue(NC - 1);
+            if (!failed && p.s_out) {
+                float* dst = p.s_out + ((size_t)bh * D + tid) * D;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float hv[64];
+                    ld_cols<64>(tmem + TM_H + lane_off + 64 * half, hv);
+#pragma unroll
+                    for (int e = 0; e < 64; e += 4)
+                        *reinterpret_cast<float4*>(dst + 64 * half + e) = make_float4(hv[e], hv[e + 1], hv[e + 2], hv[e + 3]);
+                }
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
 }
 
 bool make_maps(const ChunkParams& p, TcMaps* m) {
