@@ -314,25 +314,27 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
                              sdesc_sw128(sb + OFF_V + k * 2048, 8192, 1024), idw, k > 0);
                 mma_commit(&bars[B_WUDONE]);
             }
+            // the W copy is out of TMEM: the next chunk's S may go first (the
+            // prep of chunk n + 1 is the longer path), then c for this chunk
             wait(B_WQREADY, n & 1);
+            if (leader && !failed && n + 1 < NC) {
+                fence_async_smem();
+                load_v(n + 1);
+            }
+            if (n + 1 < NC) {
+                wait(B_KQ0 + (s ^ 1), ((n + 1) >> 1) & 1);
+                tc_fence_after();
+                if (leader && !failed) issue_S(n + 1);
+            }
             wait(B_HBREADY, n & 1);
             tc_fence_after();
             if (leader && !failed) {
-                if (n + 1 < NC) {
-                    fence_async_smem();
-                    load_v(n + 1);
-                }
                 const uint32_t idc = idesc_bf16_f32(128, 128, false, true);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)   // X += [-W; Q_bar] h
                     mma_bf16(tX, sdesc_sw128(sb + OFF_WQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
                              sdesc_sw128(sb + OFF_HB + k * 2048, 16384, 1024), idc, true);
                 mma_commit(&bars[B_CDONE]);
-            }
-            if (n + 1 < NC) {
-                wait(B_KQ0 + (s ^ 1), ((n + 1) >> 1) & 1);
-                tc_fence_after();
-                if (leader && !failed) issue_S(n + 1);
             }
             wait(B_DREADY, n & 1);
             tc_fence_after();
@@ -434,24 +436,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
             // ---- S is in TMEM (this also means the c-MMA of chunk n-1 is done)
             wait(B_SDONE, n & 1);
             tc_fence_after();
-            // Q_bar = diag(e^G) Q into the Q rows of WQ (same swizzled layout)
-#pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int idx = pt + NPR * it;            // 16-byte chunk 0..1023
-                const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
-                const uint32_t off = blk * 16384 + 8192 + r * 128 + j * 16;
-                uint4 raw = *reinterpret_cast<const uint4*>(stage + off);
-                const float gmul = sGam[r];
-                __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
-                uint4 outv;
-                uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(e2[e]);
-                    o32[e] = pack_bf16(f.x * gmul, f.y * gmul);
-                }
-                *reinterpret_cast<uint4*>(sm + OFF_WQ + off) = outv;
-            }
             // A (fp32, rows 0..63) and P (bf16, rows 64..127, kept in registers)
             uint32_t pP[16];
             {
@@ -510,12 +494,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
 #pragma unroll
                 for (int jj = 0; jj < 2; ++jj) {
                     const int j = j0 + jj;
+                    const float4 t0 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j);
+                    const float4 t1 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j + 4);
+                    const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
                     float tu[8], tw[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int i = 8 * j + e;
-                        const float tv = (i <= r) ? Tf[r * LDF + i] : 0.f;
-                        tu[e] = tv * sBeta[i];
+                        tu[e] = (i <= r) ? tv[e] * sBeta[i] : 0.f;
                         tw[e] = tu[e] * sGam[i];
                     }
                     st_row_chunk(sm + OFF_TU, r, j, tu, 1.f);
@@ -534,6 +520,26 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
             fence_async_smem();
             named_bar(2, NPR);
             if (pt == 0) mbar_arrive(&bars[B_TREADY]);
+            // Q_bar = diag(e^G) Q into the Q rows of WQ (same swizzled layout), while
+            // the W / U products run, once the c-MMA of chunk n-1 is done with WQ
+            if (n > 0) wait(B_CDONE, (n - 1) & 1);
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int idx = pt + NPR * it;            // 16-byte chunk 0..1023
+                const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+                const uint32_t off = blk * 16384 + 8192 + r * 128 + j * 16;
+                uint4 raw = *reinterpret_cast<const uint4*>(stage + off);
+                const float gmul = sGam[r];
+                __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+                uint4 outv;
+                uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(e2[e]);
+                    o32[e] = pack_bf16(f.x * gmul, f.y * gmul);
+                }
+                *reinterpret_cast<uint4*>(sm + OFF_WQ + off) = outv;
+            }
             // ---- -W (TMEM lanes 64..127) -> the W rows of WQ
             wait(B_WUDONE, n & 1);
             tc_fence_after();
