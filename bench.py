@@ -161,9 +161,11 @@ def dist_init():
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Maximum of a per-rank scalar (the slowest rank's time) over all ranks."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
