@@ -250,10 +250,12 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     kname = gdn.gdn_chunk_fwd_kernel_name(Dk, Dv, d["gate_kind"], d["q"].dtype)
+    nws = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, 64, d["q"].dtype, d["gate_kind"])
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev) if nws else None
 
     def step():
         gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["gate_kind"], d["S0"], o, S,
-                          stream=stream)
+                          workspace=ws, stream=stream)
 
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     sampler.start()

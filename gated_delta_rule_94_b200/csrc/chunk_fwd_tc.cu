@@ -9,7 +9,7 @@
 // entering state M = S^T [d_k][d_v], G the in-chunk log-decay cumsum:
 //   S  = [K; Q] K^T                 (one 128-row MMA: K K^T and Q K^T)
 //   A  = StrictTril(beta_r e^(G_r-G_i) (K K^T)_ri),  P = Tril(e^(G_r-G_i) (Q K^T)_ri)
-//   T  = (I + A)^-1                 (blocked forward substitution, fp32)
+//   T  = (I + A)^-1                 (blocked forward substitution)
 //   [0; W] = [0; T diag(beta e^G)] K
 //   X  = [T diag(beta); 0] V        = [U; 0]
 //   X += [-W; Q_bar] h              -> rows 0..63: D = U - W h, rows 64..127: Q_bar h
@@ -18,18 +18,22 @@
 // Every product is a tcgen05.mma with M = 128; operands live in 128 B-swizzled
 // shared memory: the K/Q/V tiles exactly as TMA loads them (K-major when the
 // tokens are rows, MN-major when they are the reduction dimension), the other
-// operands written by the threads in the same canonical layouts.
+// operands written in the same canonical layouts.
 //
-// One CTA owns one (batch, head) and walks its chunks in order, as a pipeline
-// of three warp roles that hand work over through mbarriers:
-//   chain  (warps 0-3):  state -> bf16 operand, state decay, D and D~ from
-//                        TMEM, output epilogue of the previous chunk
-//   prep   (warps 4-11): for chunk n while the chain works on n-1: gates,
-//                        Q_bar, A and P from S, T, the W copy
-//   control (warp 12):   TMA for V and the first tiles, every tcgen05.mma
-// Thread t of a role group owns TMEM lane (warp % 4) * 32 + lane.  Every
-// mbarrier wait is bounded; a wait that gives up sets the library status word
-// and the kernel winds down without further waits.
+// Two kernels per wave of chunks:
+//   chunk_prep_tc_kernel  one CTA per chunk, fully parallel: gates, S, A, P,
+//                         T, and the bf16 operands T diag(beta),
+//                         T diag(beta e^G), P plus the gate factors, written
+//                         to the workspace as the exact shared-memory image
+//                         the chain kernel uses (the wave is sized so the
+//                         workspace stays in L2);
+//   chunk_fwd_tc_kernel   one CTA per (batch, head), the serial state chain:
+//                         bulk-copies the prep images, W / U products, the
+//                         c- and d-products, state and output, with warp roles
+//                         chain (0-3), stager (4-7) and control (8) handing
+//                         over through mbarriers.
+// Every mbarrier wait is bounded; a wait that gives up sets the library status
+// word and the kernel winds down without further waits.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
@@ -41,43 +45,17 @@ using namespace sm100;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int NT = 416;          // 13 warps
-constexpr int NCH = 128;         // chain threads (warps 0-3)
-constexpr int NPR = 256;         // prep threads (warps 4-11)
+constexpr int NPR = 256;         // prep kernel threads (8 warps)
 constexpr int LDF = 72;          // fp32 row stride of the A / T scratch (conflict-free mma fragments)
+constexpr int GATE_FLOATS = 7 * 64;   // G, e^G, e^(G_C-G), beta, u, w, flag
 
-// Shared memory layout (bytes from a 1 KB-aligned base).
-constexpr uint32_t KQ_STAGE = 32768;   // [K_b0 | Q_b0 | K_b1 | Q_b1], 8 KB each, K-major
-constexpr uint32_t OFF_KQ = 0;         // 2 stages
-constexpr uint32_t OFF_V = 65536;      // [V_b0 | V_b1]
-constexpr uint32_t OFF_TU = 81920;     // T diag(beta)          } [T_u; Z] and
-constexpr uint32_t OFF_Z = 90112;      // zero block            } [Z; T_w] are
-constexpr uint32_t OFF_TW = 98304;     // T diag(beta e^G)      } 128-row stacks
-constexpr uint32_t OFF_Z2 = 106496;    // zero block            } [Z2; P]
-constexpr uint32_t OFF_P = 114688;     // P, K-major [64 r][64 i]
-constexpr uint32_t OFF_WQ = 122880;    // [-W_b0 | Qbar_b0 | -W_b1 | Qbar_b1], K-major
-constexpr uint32_t OFF_HB = 155648;    // h (bf16) MN-major [d][64 v] x 2; after the
-constexpr uint32_t OFF_DL = 155648;    //   c-MMA: D [i][64 v] x 2
-constexpr uint32_t OFF_DT = 172032;    //   and D~ = diag(e^(G_C - G_i)) D
-constexpr uint32_t OFF_AF = 188416;    // A fp32 [64][LDF]
-constexpr uint32_t OFF_TF = OFF_AF + 64 * LDF * 4;
-constexpr uint32_t OFF_GATE = OFF_TF + 64 * LDF * 4;   // 2 x {G, e^G, e^(G_C-G), beta, u, w, flag}
-constexpr int GATE_FLOATS = 7 * 64;
-constexpr uint32_t OFF_BAR = OFF_GATE + 2 * GATE_FLOATS * 4;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 32 * 8 + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-
-// TMEM columns (512 allocated).
-constexpr uint32_t TM_H = 0;      // state, lanes d, 128 columns v (fp32)
-constexpr uint32_t TM_X0 = 128;   // X for even chunks, lanes r / 64 + r, 128 columns v
-constexpr uint32_t TM_X1 = 256;   // X for odd chunks
-constexpr uint32_t TM_SW = 384;   // S (64 columns), then [0; W] (128 columns)
-
-// mbarrier indices
-enum Bar {
-    B_KQ0, B_KQ1, B_VFULL, B_SDONE, B_WUDONE, B_CDONE, B_DDONE,
-    B_GREADY0, B_GREADY1, B_TREADY, B_WQREADY, B_HBREADY, B_DREADY, B_FINAL, B_COUNT
-};
+// Workspace image of one chunk (bytes).
+constexpr uint32_t WS_TU = 0;          // T diag(beta), K-major [64 r][64 i], swizzled
+constexpr uint32_t WS_TW = 8192;       // T diag(beta e^G)
+constexpr uint32_t WS_P = 16384;       // P
+constexpr uint32_t WS_FAC = 24576;     // e^G [64], e^(G_C - G) [64] (fp32)
+constexpr uint32_t WS_CHUNK = WS_FAC + 2 * 64 * 4;
+constexpr size_t WAVE_BYTES = size_t(32) << 20;   // workspace per wave (kept L2-resident)
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
@@ -208,26 +186,271 @@ __device__ __forceinline__ void forward_substitution(const float* A, float* Tm, 
     named_bar(2, NPR);
 }
 
+
+// In-chunk gates for one scalar-gated chunk, by one warp: inclusive scan of g
+// (two tokens per lane), e^G, e^(G_C - G), and the factors u_r = e^(G_r - G_31),
+// w_i = e^(G_31 - G_i) with e^(G_r - G_i) = u_r w_i, usable while the in-chunk
+// decay stays below e^160 (flag).  gbuf[0..63] holds g on entry.
+template <int GATE>
+__device__ __forceinline__ void chunk_gates(float* gbuf, int lane) {
+    if constexpr (GATE == kGateScalar) {
+        const float a0 = gbuf[2 * lane], a1 = gbuf[2 * lane + 1];
+        float incl = a0 + a1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+        if (lane == 0) excl = 0.f;
+        const float G0 = excl + a0, G1 = incl;
+        const float Gl = __shfl_sync(0xffffffffu, incl, 31);
+        const float Gm = __shfl_sync(0xffffffffu, incl, 15);   // G_31
+        const float G00 = __shfl_sync(0xffffffffu, G0, 0);
+        gbuf[2 * lane] = G0;
+        gbuf[2 * lane + 1] = G1;
+        gbuf[64 + 2 * lane] = expf(G0);
+        gbuf[64 + 2 * lane + 1] = expf(G1);
+        gbuf[128 + 2 * lane] = expf(Gl - G0);
+        gbuf[128 + 2 * lane + 1] = expf(Gl - G1);
+        gbuf[256 + 2 * lane] = expf(G0 - Gm);
+        gbuf[256 + 2 * lane + 1] = expf(G1 - Gm);
+        gbuf[320 + 2 * lane] = expf(Gm - G0);
+        gbuf[320 + 2 * lane + 1] = expf(Gm - G1);
+        if (lane == 0) gbuf[384] = (G00 - Gl < 160.f) ? 1.f : 0.f;
+    } else {
+        gbuf[2 * lane] = gbuf[2 * lane + 1] = 0.f;
+        gbuf[64 + 2 * lane] = gbuf[64 + 2 * lane + 1] = 1.f;
+        gbuf[128 + 2 * lane] = gbuf[128 + 2 * lane + 1] = 1.f;
+        gbuf[256 + 2 * lane] = gbuf[256 + 2 * lane + 1] = 1.f;
+        gbuf[320 + 2 * lane] = gbuf[320 + 2 * lane + 1] = 1.f;
+        if (lane == 0) gbuf[384] = 1.f;
+    }
+}
+
+struct PrepMaps {
+    CUtensorMap q, k;
+};
+
+// Prep shared memory (bytes from a 1 KB-aligned base).
+constexpr uint32_t P_OFF_KQ = 0;                          // [K_b0 | Q_b0 | K_b1 | Q_b1]
+constexpr uint32_t P_OFF_AF = 32768;                      // A fp32 [64][LDF]
+constexpr uint32_t P_OFF_TF = P_OFF_AF + 64 * LDF * 4;    // T fp32 [64][LDF]
+constexpr uint32_t P_OFF_GATE = P_OFF_TF + 64 * LDF * 4;
+constexpr uint32_t P_OFF_BAR = P_OFF_GATE + GATE_FLOATS * 4;
+constexpr uint32_t P_SMEM = P_OFF_BAR + 16 + 1024;
+
+// One CTA per chunk of the wave: everything that does not depend on the state.
+template <int GATE>
+__global__ void __launch_bounds__(NPR)
+chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    float* Af = reinterpret_cast<float*>(sm + P_OFF_AF);
+    float* Tf = reinterpret_cast<float*>(sm + P_OFF_TF);
+    float* gbuf = reinterpret_cast<float*>(sm + P_OFF_GATE);
+    uint64_t* bar_kq = reinterpret_cast<uint64_t*>(sm + P_OFF_BAR);
+    uint64_t* bar_s = bar_kq + 1;
+    __shared__ uint32_t s_tmem;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.H, T = p.T;
+    const int bh = blockIdx.x / p.nchunks, nl = blockIdx.x % p.nchunks;
+    const int b = bh / H, h = bh % H;
+    const int n = p.chunk0 + nl;
+    uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * WS_CHUNK;
+    int failed = 0;
+
+    if (tid == 0) {
+        mbar_init(bar_kq, 1);
+        mbar_init(bar_s, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar_kq, 4 * 8192);
+        for (int blk = 0; blk < 2; ++blk) {
+            tma_load_3d(sm + P_OFF_KQ + blk * 16384, &maps.k, bar_kq, h * D + 64 * blk, n * C, b);
+            tma_load_3d(sm + P_OFF_KQ + blk * 16384 + 8192, &maps.q, bar_kq, h * D + 64 * blk, n * C, b);
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 64);
+        tmem_relinquish();
+    }
+    if (tid < 64) {
+        const int t = n * C + tid;
+        float gv = 0.f, bv = 0.f;
+        if (t < T) {
+            const size_t tok = ((size_t)b * T + t) * H + h;
+            bv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.beta)[tok]);
+            if constexpr (GATE == kGateScalar) gv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.g)[tok]);
+        }
+        gbuf[tid] = gv;
+        gbuf[192 + tid] = bv;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    if (warp == 0) chunk_gates<GATE>(gbuf, lane);
+    if (tid == 32) {   // S = [K; Q] K^T
+        if (mbar_wait(bar_kq, 0, &failed)) {
+            const uint32_t st = smem_u32(sm + P_OFF_KQ);
+            const uint32_t id = idesc_bf16_f32(128, 64, false, false);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t a = st + (k >> 2) * 16384 + (k & 3) * 32;
+                mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, k > 0);
+            }
+            mma_commit(bar_s);
+        } else {
+            atomicOr(p.status, kStatusTimeout);
+        }
+    }
+    __syncthreads();
+    const float* sG = gbuf;
+    const float* sGam = gbuf + 64;
+    const float* sFt = gbuf + 128;
+    const float* sBeta = gbuf + 192;
+    const float* sU = gbuf + 256;
+    const float* sW = gbuf + 320;
+    const bool fact = gbuf[384] != 0.f;
+    if (!mbar_wait(bar_s, 0, &failed)) atomicOr(p.status, kStatusTimeout);
+    __syncwarp();
+    tc_fence_after();
+    // A (fp32 scratch, rows 0..63) and P (bf16 image, rows 64..127)
+    {
+        const int q4 = warp & 3, ch = warp >> 2;
+        const int L = q4 * 32 + lane;
+        float sv[32];
+        ld_cols<32>(tmem + ((uint32_t)(q4 * 32) << 16) + 32 * ch, sv);
+        if (L < 64) {
+            const int r = L;
+            if (fact) {
+                const float cr = sBeta[r] * sU[r];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = 32 * ch + e;
+                    sv[e] = (i < r) ? cr * sW[i] * sv[e] : 0.f;
+                }
+            } else {
+                const float Gr = sG[r], br = sBeta[r];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = 32 * ch + e;
+                    sv[e] = (i < r) ? br * __expf(Gr - sG[i]) * sv[e] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(Af + r * LDF + 32 * ch + e) =
+                    make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+        } else {
+            const int r = L - 64;
+            if (fact) {
+                const float cr = sU[r];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = 32 * ch + e;
+                    sv[e] = (i <= r) ? cr * sW[i] * sv[e] : 0.f;
+                }
+            } else {
+                const float Gr = sG[r];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = 32 * ch + e;
+                    sv[e] = (i <= r) ? __expf(Gr - sG[i]) * sv[e] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) st_row_chunk(img + WS_P, r, 4 * ch + jj, sv + 8 * jj, 1.f);
+        }
+    }
+    __syncthreads();
+    forward_substitution(Af, Tf, tid);
+    // T diag(beta) and T diag(beta e^G) as bf16 images, K-major [r][i]
+    {
+        const int r = tid >> 2, j0 = 2 * (tid & 3);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int j = j0 + jj;
+            const float4 t0 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j);
+            const float4 t1 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j + 4);
+            const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            float tu[8], tw[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int i = 8 * j + e;
+                tu[e] = (i <= r) ? tv[e] * sBeta[i] : 0.f;
+                tw[e] = tu[e] * sGam[i];
+            }
+            st_row_chunk(img + WS_TU, r, j, tu, 1.f);
+            st_row_chunk(img + WS_TW, r, j, tw, 1.f);
+        }
+    }
+    if (tid < 64) {
+        float* fac = reinterpret_cast<float*>(img + WS_FAC);
+        fac[tid] = sGam[tid];
+        fac[64 + tid] = sFt[tid];
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
+}
+
+// Chain kernel shared memory (bytes from a 1 KB-aligned base).
+constexpr uint32_t KQ_STAGE = 32768;   // [K_b0 | Q_b0 | K_b1 | Q_b1], 8 KB each, K-major
+constexpr uint32_t OFF_KQ = 0;         // 2 stages
+constexpr uint32_t OFF_V = 65536;      // 2 buffers of [V_b0 | V_b1]
+constexpr uint32_t OFF_TU = 98304;     // T diag(beta)          } [T_u; Z] and
+constexpr uint32_t OFF_Z = 106496;     // zero block            } [Z; T_w] are
+constexpr uint32_t OFF_TW = 114688;    // T diag(beta e^G)      } 128-row stacks
+constexpr uint32_t OFF_Z2 = 122880;    // zero block            } [Z2; P]
+constexpr uint32_t OFF_P = 131072;     // P, K-major [64 r][64 i]
+constexpr uint32_t OFF_WQ = 139264;    // [-W_b0 | Qbar_b0 | -W_b1 | Qbar_b1], K-major
+constexpr uint32_t OFF_HB = 172032;    // h (bf16) MN-major [d][64 v] x 2; after the
+constexpr uint32_t OFF_DL = 172032;    //   c-MMA: D [i][64 v] x 2
+constexpr uint32_t OFF_DT = 188416;    //   and D~ = diag(e^(G_C - G_i)) D
+constexpr uint32_t OFF_FAC = 204800;   // 2 x {e^G [64], e^(G_C - G) [64]}
+constexpr uint32_t OFF_BAR = OFF_FAC + 2 * 128 * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 32 * 8 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+constexpr int NT = 288;          // 9 warps
+constexpr int NCH = 128;         // chain threads (warps 0-3)
+constexpr int NST = 128;         // stager threads (warps 4-7)
+
+// TMEM columns (512 allocated).
+constexpr uint32_t TM_H = 0;      // state, lanes d, 128 columns v (fp32)
+constexpr uint32_t TM_X0 = 128;   // X for even chunks, lanes r / 64 + r, 128 columns v
+constexpr uint32_t TM_X1 = 256;   // X for odd chunks
+constexpr uint32_t TM_W = 384;    // [0; W], lanes 64..127, 128 columns d
+
+enum Bar {
+    B_KQ0, B_KQ1, B_VFULL, B_TFULL, B_PFULL, B_FFULL0, B_FFULL1, B_WUDONE, B_CDONE, B_DDONE,
+    B_WQREADY, B_HBREADY, B_DREADY, B_XFREE, B_FINAL, B_COUNT
+};
+
 struct TcMaps {
     CUtensorMap q, k, v;
 };
 
-template <int GATE>
 __global__ void __launch_bounds__(NT, 1)
-chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
+chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, int gated) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
-    float* Af = reinterpret_cast<float*>(sm + OFF_AF);
-    float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     __shared__ uint32_t s_tmem;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, T = p.T;
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const int NC = (T + C - 1) / C;
+    const int NC = p.nchunks;              // local chunk nl = 0..NC-1 is chunk p.chunk0 + nl
+    const uint8_t* wsh = p.ws + (size_t)bh * p.cw * WS_CHUNK;
     int failed = 0;
 
     if (tid == 0) {
@@ -252,13 +475,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
     const uint32_t tmem = s_tmem;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
 
-    auto gate_buf = [&](int n) { return reinterpret_cast<float*>(sm + OFF_GATE) + (n & 1) * GATE_FLOATS; };
+    auto fac_buf = [&](int nl) { return reinterpret_cast<float*>(sm + OFF_FAC) + (nl & 1) * 128; };
     auto wait = [&](int bar, uint32_t parity) {
         if (!mbar_wait(&bars[bar], parity, &failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     };
-    auto load_kq = [&](int n) {
-        const int s = n & 1;
+    auto load_kq = [&](int nl) {
+        const int s = nl & 1, n = p.chunk0 + nl;
         mbar_arrive_expect_tx(&bars[B_KQ0 + s], 4 * 8192);
         uint8_t* st = sm + OFF_KQ + s * KQ_STAGE;
         for (int blk = 0; blk < 2; ++blk) {
@@ -266,67 +489,54 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
             tma_load_3d(st + blk * 16384 + 8192, &maps.q, &bars[B_KQ0 + s], h * D + 64 * blk, n * C, b);
         }
     };
-    auto load_v = [&](int n) {
+    auto load_v = [&](int nl) {
+        const int n = p.chunk0 + nl;
         mbar_arrive_expect_tx(&bars[B_VFULL], 2 * 8192);
         for (int blk = 0; blk < 2; ++blk)
-            tma_load_3d(sm + OFF_V + blk * 8192, &maps.v, &bars[B_VFULL], h * D + 64 * blk, n * C, b);
+            tma_load_3d(sm + OFF_V + (nl & 1) * 16384 + blk * 8192, &maps.v, &bars[B_VFULL],
+                        h * D + 64 * blk, n * C, b);
     };
 
-    if (warp == 12) {
-        // =========================== control: TMA + every tcgen05.mma
+    if (warp == 8) {
+        // =========================== control: TMA for the first tiles and V, every MMA
         const bool leader = lane == 0;   // issues only while no wait has failed
-        auto issue_S = [&](int n) {
-            const uint32_t st = sb + OFF_KQ + (n & 1) * KQ_STAGE;
-            const uint32_t id = idesc_bf16_f32(128, 64, false, false);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t a = st + (k >> 2) * 16384 + (k & 3) * 32;
-                mma_bf16(tmem + TM_SW, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, k > 0);
-            }
-            mma_commit(&bars[B_SDONE]);
-        };
         if (leader) {
             fence_async_smem();
             load_kq(0);
             if (NC > 1) load_kq(1);
-            load_v(0);
         }
-        wait(B_KQ0, 0);
-        tc_fence_after();
-        if (leader && !failed) issue_S(0);
-#pragma unroll 1
-        for (int n = 0; n < NC; ++n) {
-            const int s = n & 1;
+        // W and U of chunk nl: operands loaded, TMEM free (for nl >= 2 the output
+        // of chunk nl - 2 has been read out of X[nl & 1])
+        auto issue_wu = [&](int nl) {
+            const int s = nl & 1;
             const uint32_t st = sb + OFF_KQ + s * KQ_STAGE;
             const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
-            wait(B_TREADY, n & 1);
-            wait(B_VFULL, n & 1);
+            wait(B_TFULL, nl & 1);
+            wait(B_VFULL, nl & 1);
+            wait(B_KQ0 + s, (nl >> 1) & 1);
+            if (nl >= 2) wait(B_XFREE, (nl - 2) & 1);
             tc_fence_after();
             if (leader && !failed) {
                 const uint32_t idw = idesc_bf16_f32(128, 128, false, true);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)   // [0; W] = [Z; T_w] K
-                    mma_bf16(tmem + TM_SW, sdesc_sw128(sb + OFF_Z + k * 32, 16, 1024),
+                    mma_bf16(tmem + TM_W, sdesc_sw128(sb + OFF_Z + k * 32, 16, 1024),
                              sdesc_sw128(st + k * 2048, 16384, 1024), idw, k > 0);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)   // X = [T_u; Z] V
                     mma_bf16(tX, sdesc_sw128(sb + OFF_TU + k * 32, 16, 1024),
-                             sdesc_sw128(sb + OFF_V + k * 2048, 8192, 1024), idw, k > 0);
+                             sdesc_sw128(sb + OFF_V + s * 16384 + k * 2048, 8192, 1024), idw, k > 0);
                 mma_commit(&bars[B_WUDONE]);
             }
-            // the W copy is out of TMEM: the next chunk's S may go first (the
-            // prep of chunk n + 1 is the longer path), then c for this chunk
-            wait(B_WQREADY, n & 1);
-            if (leader && !failed && n + 1 < NC) {
-                fence_async_smem();
-                load_v(n + 1);
-            }
-            if (n + 1 < NC) {
-                wait(B_KQ0 + (s ^ 1), ((n + 1) >> 1) & 1);
-                tc_fence_after();
-                if (leader && !failed) issue_S(n + 1);
-            }
-            wait(B_HBREADY, n & 1);
+        };
+        if (NC > 0) issue_wu(0);
+#pragma unroll 1
+        for (int nl = 0; nl < NC; ++nl) {
+            const int s = nl & 1;
+            const uint32_t st = sb + OFF_KQ + s * KQ_STAGE;
+            const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
+            wait(B_WQREADY, nl & 1);
+            wait(B_HBREADY, nl & 1);
             tc_fence_after();
             if (leader && !failed) {
                 const uint32_t idc = idesc_bf16_f32(128, 128, false, true);
@@ -336,7 +546,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
                              sdesc_sw128(sb + OFF_HB + k * 2048, 16384, 1024), idc, true);
                 mma_commit(&bars[B_CDONE]);
             }
-            wait(B_DREADY, n & 1);
+            // the next chunk's W / U run while the chain turns D of this one
+            if (nl + 1 < NC) issue_wu(nl + 1);
+            wait(B_DREADY, nl & 1);
+            wait(B_PFULL, nl & 1);
             tc_fence_after();
             if (leader && !failed) {
                 const uint32_t id2 = idesc_bf16_f32(128, 128, true, true);
@@ -358,202 +571,70 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
         if (!mbar_wait(&bars[B_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     } else if (warp >= 4) {
-        // =========================== prep: gates, Q_bar, A / P, T, W copy
-        const int pt = tid - NCH;                 // 0..255
-        const int q4 = warp & 3, ch = (warp - 4) >> 2;
-        const int L = q4 * 32 + lane;             // TMEM lane of this thread
-        const __nv_bfloat16* gq = static_cast<const __nv_bfloat16*>(p.g);
-        const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(p.beta);
-        float g_next = 0.f, b_next = 0.f;
-        if (pt < 64 && pt < T) {
-            const size_t tok = ((size_t)b * T + pt) * H + h;
-            b_next = __bfloat162float(gb[tok]);
-            if constexpr (GATE == kGateScalar) g_next = __bfloat162float(gq[tok]);
-        }
+        // =========================== stager: prep images in, -W and Q_bar operands
+        const int st_id = tid - NCH;                // 0..127
+        const int L = (warp & 3) * 32 + lane;       // TMEM lane of this thread
 #pragma unroll 1
-        for (int n = 0; n < NC; ++n) {
-            const int s = n & 1;
-            float* gbuf = gate_buf(n);   // G, e^G, e^(G_C - G), beta
-            uint8_t* stage = sm + OFF_KQ + s * KQ_STAGE;
-            // ---- gates
-            if (pt < 64) {
-                gbuf[pt] = g_next;
-                gbuf[192 + pt] = b_next;
+        for (int nl = 0; nl < NC; ++nl) {
+            const int s = nl & 1;
+            const uint8_t* img = wsh + (size_t)nl * WS_CHUNK;
+            if (st_id == 0) {   // W/U of chunk nl-1 are done with T_u / T_w, and the chain is
+                                // done with the factors of chunk nl-2 (both waited below)
+                mbar_arrive_expect_tx(&bars[B_TFULL], 2 * 8192);
+                bulk_load(sm + OFF_TU, img + WS_TU, 8192, &bars[B_TFULL]);
+                bulk_load(sm + OFF_TW, img + WS_TW, 8192, &bars[B_TFULL]);
+                mbar_arrive_expect_tx(&bars[B_FFULL0 + s], 512);
+                bulk_load(fac_buf(nl), img + WS_FAC, 512, &bars[B_FFULL0 + s]);
+                fence_async_smem();
+                load_v(nl);   // V buffer nl & 1: U of chunk nl-2 is long done
             }
-            named_bar(2, NPR);
-            if (pt < 32) {
-                if constexpr (GATE == kGateScalar) {
-                    const float a0 = gbuf[2 * lane], a1 = gbuf[2 * lane + 1];
-                    float incl = a0 + a1;
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const float y = __shfl_up_sync(0xffffffffu, incl, off);
-                        if (lane >= off) incl += y;
-                    }
-                    float excl = __shfl_up_sync(0xffffffffu, incl, 1);
-                    if (lane == 0) excl = 0.f;
-                    const float G0 = excl + a0, G1 = incl;
-                    const float Gl = __shfl_sync(0xffffffffu, incl, 31);
-                    const float Gm = __shfl_sync(0xffffffffu, incl, 15);   // G_31
-                    const float G00 = __shfl_sync(0xffffffffu, G0, 0);
-                    gbuf[2 * lane] = G0;
-                    gbuf[2 * lane + 1] = G1;
-                    gbuf[64 + 2 * lane] = expf(G0);
-                    gbuf[64 + 2 * lane + 1] = expf(G1);
-                    gbuf[128 + 2 * lane] = expf(Gl - G0);
-                    gbuf[128 + 2 * lane + 1] = expf(Gl - G1);
-                    // e^(G_r - G_i) = u_r w_i about the middle of the chunk; both
-                    // factors stay finite while the in-chunk decay is below e^160
-                    gbuf[256 + 2 * lane] = expf(G0 - Gm);
-                    gbuf[256 + 2 * lane + 1] = expf(G1 - Gm);
-                    gbuf[320 + 2 * lane] = expf(Gm - G0);
-                    gbuf[320 + 2 * lane + 1] = expf(Gm - G1);
-                    if (lane == 0) gbuf[384] = (G00 - Gl < 160.f) ? 1.f : 0.f;
-                } else {
-                    gbuf[2 * lane] = gbuf[2 * lane + 1] = 0.f;
-                    gbuf[64 + 2 * lane] = gbuf[64 + 2 * lane + 1] = 1.f;
-                    gbuf[128 + 2 * lane] = gbuf[128 + 2 * lane + 1] = 1.f;
-                    gbuf[256 + 2 * lane] = gbuf[256 + 2 * lane + 1] = 1.f;
-                    gbuf[320 + 2 * lane] = gbuf[320 + 2 * lane + 1] = 1.f;
-                    if (lane == 0) gbuf[384] = 1.f;
-                }
-            }
-            if (pt < 64 && n + 1 < NC) {
-                g_next = 0.f;
-                b_next = 0.f;
-                if ((n + 1) * C + pt < T) {
-                    const size_t tok = ((size_t)b * T + (n + 1) * C + pt) * H + h;
-                    b_next = __bfloat162float(gb[tok]);
-                    if constexpr (GATE == kGateScalar) g_next = __bfloat162float(gq[tok]);
-                }
-            }
-            named_bar(2, NPR);
-            if (pt == 0) mbar_arrive(&bars[B_GREADY0 + s]);
-            const float* sG = gbuf;
-            const float* sGam = gbuf + 64;
-            const float* sBeta = gbuf + 192;
-
-            // ---- S is in TMEM (this also means the c-MMA of chunk n-1 is done)
-            wait(B_SDONE, n & 1);
-            tc_fence_after();
-            // A (fp32, rows 0..63) and P (bf16, rows 64..127, kept in registers)
-            uint32_t pP[16];
+            // Q_bar = diag(e^G) Q into the Q rows of WQ (same swizzled layout), once the
+            // c-product of chunk nl-1 is done with WQ
+            if (nl > 0) wait(B_CDONE, (nl - 1) & 1);
+            wait(B_FFULL0 + s, (nl >> 1) & 1);
+            wait(B_KQ0 + s, (nl >> 1) & 1);
             {
-                float sv[32];
-                ld_cols<32>(tmem + TM_SW + lane_off + 32 * ch, sv);
-                const float* sU = gbuf + 256;
-                const float* sW = gbuf + 320;
-                const bool fact = gbuf[384] != 0.f;
-                if (L < 64) {
-                    const int r = L;
-                    if (fact) {
-                        const float cr = sBeta[r] * sU[r];
+                const float* sGam = fac_buf(nl);
+                const uint8_t* stage = sm + OFF_KQ + s * KQ_STAGE;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int i = 32 * ch + e;
-                            sv[e] = (i < r) ? cr * sW[i] * sv[e] : 0.f;
-                        }
-                    } else {
-                        const float Gr = sG[r], br = sBeta[r];
+                for (int it = 0; it < 8; ++it) {
+                    const int idx = st_id + NST * it;          // 16-byte chunk 0..1023
+                    const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+                    const uint32_t off = blk * 16384 + 8192 + r * 128 + j * 16;
+                    uint4 raw = *reinterpret_cast<const uint4*>(stage + off);
+                    const float gmul = sGam[r];
+                    __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+                    uint4 outv;
+                    uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int i = 32 * ch + e;
-                            sv[e] = (i < r) ? br * __expf(Gr - sG[i]) * sv[e] : 0.f;
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(e2[e]);
+                        o32[e] = pack_bf16(f.x * gmul, f.y * gmul);
                     }
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4*>(Af + r * LDF + 32 * ch + e) =
-                            make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
-                } else {
-                    const int r = L - 64;
-                    if (fact) {
-                        const float cr = sU[r];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int i = 32 * ch + e;
-                            sv[e] = (i <= r) ? cr * sW[i] * sv[e] : 0.f;
-                        }
-                    } else {
-                        const float Gr = sG[r];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int i = 32 * ch + e;
-                            sv[e] = (i <= r) ? __expf(Gr - sG[i]) * sv[e] : 0.f;
-                        }
-                    }
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) pP[e >> 1] = pack_bf16(sv[e], sv[e + 1]);
+                    *reinterpret_cast<uint4*>(sm + OFF_WQ + off) = outv;
                 }
             }
-            named_bar(2, NPR);
-            forward_substitution(Af, Tf, pt);
-            // T diag(beta) and T diag(beta e^G) as bf16, K-major [r][i]
-            {
-                const int r = pt >> 2, j0 = 2 * (pt & 3);
-#pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {
-                    const int j = j0 + jj;
-                    const float4 t0 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j);
-                    const float4 t1 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j + 4);
-                    const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                    float tu[8], tw[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int i = 8 * j + e;
-                        tu[e] = (i <= r) ? tv[e] * sBeta[i] : 0.f;
-                        tw[e] = tu[e] * sGam[i];
-                    }
-                    st_row_chunk(sm + OFF_TU, r, j, tu, 1.f);
-                    st_row_chunk(sm + OFF_TW, r, j, tw, 1.f);
-                }
-            }
-            // P once the d-MMAs of chunk n-1 are done with the buffer
-            if (n > 0) wait(B_DDONE, (n - 1) & 1);
-            if (L >= 64) {
-                const int r = L - 64;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-                    *reinterpret_cast<uint4*>(sm + OFF_P + sw128_offset(r, 8 * (4 * ch + jj))) =
-                        make_uint4(pP[4 * jj], pP[4 * jj + 1], pP[4 * jj + 2], pP[4 * jj + 3]);
-            }
-            fence_async_smem();
-            named_bar(2, NPR);
-            if (pt == 0) mbar_arrive(&bars[B_TREADY]);
-            // Q_bar = diag(e^G) Q into the Q rows of WQ (same swizzled layout), while
-            // the W / U products run, once the c-MMA of chunk n-1 is done with WQ
-            if (n > 0) wait(B_CDONE, (n - 1) & 1);
-#pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int idx = pt + NPR * it;            // 16-byte chunk 0..1023
-                const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
-                const uint32_t off = blk * 16384 + 8192 + r * 128 + j * 16;
-                uint4 raw = *reinterpret_cast<const uint4*>(stage + off);
-                const float gmul = sGam[r];
-                __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
-                uint4 outv;
-                uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(e2[e]);
-                    o32[e] = pack_bf16(f.x * gmul, f.y * gmul);
-                }
-                *reinterpret_cast<uint4*>(sm + OFF_WQ + off) = outv;
-            }
-            // ---- -W (TMEM lanes 64..127) -> the W rows of WQ
-            wait(B_WUDONE, n & 1);
+            // -W (TMEM lanes 64..127, warps 6-7) -> the W rows of WQ
+            wait(B_WUDONE, nl & 1);
             tc_fence_after();
             if (L >= 64) {
                 const int r = L - 64;
-                float wv[64];
-                ld_cols<64>(tmem + TM_SW + lane_off + 64 * ch, wv);
+                float wv[128];
+                ld_cols<128>(tmem + TM_W + lane_off, wv);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) st_row_chunk(sm + OFF_WQ + ch * 16384, r, j, wv + 8 * j, -1.f);
+                for (int j = 0; j < 16; ++j)
+                    st_row_chunk(sm + OFF_WQ + (j >> 3) * 16384, r, j & 7, wv + 8 * j, -1.f);
             }
             fence_async_smem();
             tc_fence_before();
-            named_bar(2, NPR);
-            if (pt == 0) mbar_arrive(&bars[B_WQREADY]);
+            named_bar(3, NST);
+            if (st_id == 0) mbar_arrive(&bars[B_WQREADY]);
+            // P of chunk nl once the d-products of chunk nl-1 are done with the buffer
+            if (nl > 0) wait(B_DDONE, (nl - 1) & 1);
+            if (st_id == 0) {
+                mbar_arrive_expect_tx(&bars[B_PFULL], 8192);
+                bulk_load(sm + OFF_P, img + WS_P, 8192, &bars[B_PFULL]);
+            }
         }
     } else {
         // =========================== chain: state, D, output
@@ -568,83 +649,79 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p) {
             }
             tmem_wait_st();
         }
-        auto out_epilogue = [&](int m) {   // chunk m's O, warps 2-3 (TMEM lanes 64..127)
-            const int r = tid - 64, t0 = m * C;
+        auto out_epilogue = [&](int ml) {   // chunk ml's O, warps 2-3 (TMEM lanes 64..127)
+            const int r = tid - 64, t0 = (p.chunk0 + ml) * C;
             const int nval = min(C, T - t0);
-            const uint32_t tX = tmem + ((m & 1) ? TM_X1 : TM_X0);
+            const uint32_t tX = tmem + ((ml & 1) ? TM_X1 : TM_X0);
             __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + (((size_t)b * T + t0 + r) * H + h) * D;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float ov[64];
-                ld_cols<64>(tX + lane_off + 64 * half, ov);
-                if (r < nval) {
+            float ov[128];
+            ld_cols<128>(tX + lane_off, ov);
+            if (r < nval) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint4 w;
-                        w.x = pack_bf16(ov[8 * j + 0], ov[8 * j + 1]);
-                        w.y = pack_bf16(ov[8 * j + 2], ov[8 * j + 3]);
-                        w.z = pack_bf16(ov[8 * j + 4], ov[8 * j + 5]);
-                        w.w = pack_bf16(ov[8 * j + 6], ov[8 * j + 7]);
-                        *reinterpret_cast<uint4*>(orow + 64 * half + 8 * j) = w;
-                    }
+                for (int j = 0; j < 16; ++j) {
+                    uint4 w;
+                    w.x = pack_bf16(ov[8 * j + 0], ov[8 * j + 1]);
+                    w.y = pack_bf16(ov[8 * j + 2], ov[8 * j + 3]);
+                    w.z = pack_bf16(ov[8 * j + 4], ov[8 * j + 5]);
+                    w.w = pack_bf16(ov[8 * j + 6], ov[8 * j + 7]);
+                    *reinterpret_cast<uint4*>(orow + 8 * j) = w;
                 }
             }
         };
 #pragma unroll 1
-        for (int n = 0; n < NC; ++n) {
-            const int s = n & 1;
-            if (n > 0) {
-                wait(B_DDONE, (n - 1) & 1);
+        for (int nl = 0; nl < NC; ++nl) {
+            const int s = nl & 1;
+            if (nl > 0) {
+                wait(B_DDONE, (nl - 1) & 1);
                 tc_fence_after();
-                if (tid == 0 && n + 1 < NC) {
+                if (tid == 0 && nl + 1 < NC) {
                     fence_async_smem();
-                    load_kq(n + 1);
+                    load_kq(nl + 1);
                 }
             }
             // state -> bf16 operand h (MN-major [d][64 v] x 2), row d = tid
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float hv[64];
-                ld_cols<64>(tmem + TM_H + lane_off + 64 * half, hv);
+            {
+                float hv[128];
+                ld_cols<128>(tmem + TM_H + lane_off, hv);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) st_row_chunk(sm + OFF_HB + half * 16384, tid, j, hv + 8 * j, 1.f);
+                for (int j = 0; j < 16; ++j)
+                    st_row_chunk(sm + OFF_HB + (j >> 3) * 16384, tid, j & 7, hv + 8 * j, 1.f);
             }
             fence_async_smem();
             named_bar(1, NCH);
             if (tid == 0) mbar_arrive(&bars[B_HBREADY]);
             // state *= e^(G_C) (before the state update of this chunk)
-            wait(B_GREADY0 + s, (n >> 1) & 1);
-            const float* gbuf = gate_buf(n);
-            if constexpr (GATE != kGateNone) {
-                const float gam = gbuf[64 + 63];
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float hv[64];
-                    ld_cols<64>(tmem + TM_H + lane_off + 64 * half, hv);
+            wait(B_FFULL0 + s, (nl >> 1) & 1);
+            const float* fac = fac_buf(nl);
+            if (gated) {
+                const float gam = fac[63];
+                float hv[128];
+                ld_cols<128>(tmem + TM_H + lane_off, hv);
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) hv[e] *= gam;
-                    st_cols<64>(tmem + TM_H + lane_off + 64 * half, hv);
-                }
+                for (int e = 0; e < 128; ++e) hv[e] *= gam;
+                st_cols<128>(tmem + TM_H + lane_off, hv);
                 tmem_wait_st();
             }
             tc_fence_before();
             named_bar(1, NCH);
             if (warp >= 2) {
-                if (n > 0) out_epilogue(n - 1);
+                if (nl > 0) {
+                    out_epilogue(nl - 1);
+                    tc_fence_before();
+                    named_bar(4, 64);
+                    if (tid == 64) mbar_arrive(&bars[B_XFREE]);   // X[(nl - 1) & 1] is free
+                }
             } else {
-                wait(B_CDONE, n & 1);
+                wait(B_CDONE, nl & 1);
                 tc_fence_after();
-                const float ft = gbuf[128 + tid];
+                const float ft = fac[64 + tid];
                 const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float dv[64];
-                    ld_cols<64>(tX + lane_off + 64 * half, dv);
+                float dv[128];
+                ld_cols<128>(tX + lane_off, dv);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        st_row_chunk(sm + OFF_DL + half * 8192, tid, j, dv + 8 * j, 1.f);
-                        st_row_chunk(sm + OFF_DT + half * 8192, tid, j, dv + 8 * j, ft);
-                    }
+                for (int j = 0; j < 16; ++j) {
+                    st_row_chunk(sm + OFF_DL + (j >> 3) * 8192, tid, j & 7, dv + 8 * j, 1.f);
+                    st_row_chunk(sm + OFF_DT + (j >> 3) * 8192, tid, j & 7, dv + 8 * j, ft);
                 }
             }
             fence_async_smem();
@@ -686,15 +763,13 @@ bool make_maps(const ChunkParams& p, TcMaps* m) {
            make_tmap_bf16(&m->v, p.v, 3, dims, strides, box);
 }
 
-template <int GATE>
-cudaError_t launch_gate(const ChunkParams& p, cudaStream_t s) {
-    TcMaps maps;
-    if (!make_maps(p, &maps)) return cudaErrorInvalidValue;
-    auto kern = chunk_fwd_tc_kernel<GATE>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    kern<<<(unsigned)((size_t)p.B * p.H), NT, SMEM_BYTES, s>>>(maps, p);
-    return cudaGetLastError();
+// Chunk slots per (batch, head) of one wave: as many as keep the wave's
+// workspace near WAVE_BYTES (L2-resident), at least 4.
+int wave_chunks(int nbh, int NC) {
+    long long cw = (long long)(WAVE_BYTES / ((size_t)nbh * WS_CHUNK));
+    if (cw < 4) cw = 4;
+    if (cw > NC) cw = NC;
+    return (int)(cw < 1 ? 1 : cw);
 }
 
 }  // namespace
@@ -703,9 +778,47 @@ bool chunk_fwd_tc_supported(int Dk, int Dv, int gate) {
     return Dk == D && Dv == D && (gate == kGateNone || gate == kGateScalar);
 }
 
-cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, cudaStream_t s) {
-    if (gate == kGateScalar) return launch_gate<kGateScalar>(p, s);
-    return launch_gate<kGateNone>(p, s);
+size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H) {
+    const int NC = (T + C - 1) / C;
+    if (NC == 0 || B == 0 || H == 0) return 0;
+    const int nbh = B * H;
+    const int cw = wave_chunks(nbh, NC);
+    const int nw = (NC + cw - 1) / cw;
+    size_t bytes = (size_t)nbh * cw * WS_CHUNK;
+    if (nw > 1) bytes += (size_t)nbh * D * D * sizeof(float);   // state between waves
+    return bytes;
+}
+
+cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s, int* launches) {
+    *launches = 0;
+    TcMaps maps;
+    if (!make_maps(p0, &maps)) return cudaErrorInvalidValue;
+    PrepMaps pmaps;
+    pmaps.q = maps.q;
+    pmaps.k = maps.k;
+    auto prep = gate == kGateScalar ? chunk_prep_tc_kernel<kGateScalar> : chunk_prep_tc_kernel<kGateNone>;
+    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const int NC = (p0.T + C - 1) / C;
+    const int nbh = p0.B * p0.H;
+    const int cw = wave_chunks(nbh, NC);
+    const int nw = (NC + cw - 1) / cw;
+    float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + (size_t)nbh * cw * WS_CHUNK) : nullptr;
+    for (int w = 0; w < nw; ++w) {
+        ChunkParams p = p0;
+        p.cw = cw;
+        p.chunk0 = w * cw;
+        p.nchunks = (w + 1 < nw) ? cw : NC - w * cw;
+        p.s0 = (w == 0) ? p0.s0 : carry;
+        p.s_out = (w + 1 == nw) ? p0.s_out : carry;
+        prep<<<(unsigned)(nbh * p.nchunks), NPR, P_SMEM, s>>>(pmaps, p);
+        ++*launches;
+        chunk_fwd_tc_kernel<<<(unsigned)nbh, NT, SMEM_BYTES, s>>>(maps, p, gate == kGateScalar ? 1 : 0);
+        ++*launches;
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace gdn

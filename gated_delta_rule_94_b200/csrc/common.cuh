@@ -24,6 +24,11 @@ struct ChunkParams {
     float* s_out;      // may be null
     int B, T, H, Dk, Dv;
     unsigned* status;  // device status word
+    // tensor-core path: workspace and the wave of chunks one launch pair covers
+    uint8_t* ws;       // per-chunk prep images, [B*H][cw] x WS_CHUNK bytes
+    int cw;            // chunk slots per (batch, head) in the workspace
+    int chunk0;        // first chunk of this wave
+    int nchunks;       // chunks in this wave
 };
 
 struct DecodeParams {
@@ -51,6 +56,10 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Launchers implemented in the kernel translation units.
 namespace gdn {
 cudaError_t launch_chunk_fwd_simt(const ChunkParams& p, int gate, bool bf16, cudaStream_t s);
+bool chunk_fwd_tc_supported(int Dk, int Dv, int gate);
+size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H);
+// Enqueues the tensor-core forward; *launches receives the number of kernels.
+cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, cudaStream_t s, int* launches);
 cudaError_t launch_decode_step(const DecodeParams& p, int Dk, int Dv, int gate, bool bf16,
                                cudaStream_t s);
 }  // namespace gdn

@@ -14,12 +14,6 @@
 // a bounded wait; gdn_read_device_status reads and clears it.
 __device__ unsigned gdn_device_status_word = 0u;
 
-namespace gdn {
-// Implemented in chunk_fwd_tc.cu (tensor-core path for bf16 inputs).
-bool chunk_fwd_tc_supported(int Dk, int Dv, int gate);
-cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, cudaStream_t s);
-}  // namespace gdn
-
 namespace {
 
 unsigned* status_word_ptr() {
@@ -84,6 +78,8 @@ size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int ch
     if (!supported_dim(Dk) || !supported_dim(Dv) || chunk != 64) return (size_t)-1;
     if (dtype != GDN_BF16 && dtype != GDN_F32) return (size_t)-1;
     if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return (size_t)-1;
+    if (dtype == GDN_BF16 && gdn::chunk_fwd_tc_supported(Dk, Dv, gate_kind))
+        return gdn::chunk_fwd_tc_workspace_bytes(B, T, H);
     return 0;
 }
 
@@ -144,14 +140,19 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
     p.s0 = initial_state; p.o = o; p.s_out = final_state;
     p.B = B; p.T = T; p.H = H; p.Dk = Dk; p.Dv = Dv;
     p.status = status_word_ptr();
+    p.ws = static_cast<uint8_t*>(workspace);
+    p.cw = 0;
+    p.chunk0 = 0;
+    p.nchunks = 0;
     if (!p.status) return GDN_ERR_CUDA;
     cudaError_t e;
+    int launches = 1;
     if (dtype == GDN_BF16 && gdn::chunk_fwd_tc_supported(Dk, Dv, gate_kind))
-        e = gdn::launch_chunk_fwd_tc(p, gate_kind, s);
+        e = gdn::launch_chunk_fwd_tc(p, gate_kind, s, &launches);
     else
         e = gdn::launch_chunk_fwd_simt(p, gate_kind, dtype == GDN_BF16, s);
+    g_launches.fetch_add((unsigned long long)launches);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
-    g_launches.fetch_add(1);
     return GDN_OK;
 }
 

@@ -26,7 +26,10 @@ def gpu_chunk(x: dict, *, final=True, alias=False):
         S1 = S0
     else:
         S1 = torch.full((B, H, Dk, Dv), float("nan"), device="cuda") if final else None
-    gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], x["gate_kind"], S0, o, S1)
+    nws = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, 64, d["q"].dtype, x["gate_kind"])
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device="cuda") if nws else None
+    gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], x["gate_kind"], S0, o, S1,
+                      workspace=ws)
     torch.cuda.synchronize()
     return o, S1
 
