@@ -24,7 +24,8 @@ GDN_GATE_NONE, GDN_GATE_SCALAR, GDN_GATE_PER_DIM = 0, 1, 2
 
 EXPORTED = ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_decode_step",
             "gdn_read_device_status", "gdn_status_string", "gdn_abi_version",
-            "gdn_kernel_launch_count", "gdn_chunk_fwd_kernel_name")
+            "gdn_kernel_launch_count", "gdn_chunk_fwd_kernel_name", "gdn_chunk_fwd_noalloc",
+            "gdn_chunk_fwd_noalloc_scratch_bytes")
 
 _lib = None
 
@@ -61,6 +62,10 @@ def load() -> ctypes.CDLL:
     lib.gdn_kernel_launch_count.restype = ctypes.c_ulonglong
     lib.gdn_chunk_fwd_kernel_name.argtypes = [i, i, i, i]
     lib.gdn_chunk_fwd_kernel_name.restype = ctypes.c_char_p
+    lib.gdn_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    lib.gdn_chunk_fwd_noalloc.restype = i
+    lib.gdn_chunk_fwd_noalloc_scratch_bytes.argtypes = []
+    lib.gdn_chunk_fwd_noalloc_scratch_bytes.restype = sz
     _lib = lib
     return lib
 

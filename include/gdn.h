@@ -143,6 +143,39 @@ GDN_API gdn_status gdn_read_device_status(gdn_stream_t stream);
 /* A static, human-readable name for a status code. */
 GDN_API const char* gdn_status_string(gdn_status s);
 
+/*
+ * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate
+ * device memory (no counterpart on the source pages: it is a deployment aid).
+ *
+ * Same arguments and results as gdn_chunk_fwd, minus the workspace: the
+ * library supplies it from a fixed scratch array of
+ * gdn_chunk_fwd_noalloc_scratch_bytes() bytes (48 MiB) that every GPU loading
+ * the library reserves until the process exits.  For callers that cannot call
+ * cudaMalloc -- inside a host framework that owns all device memory, or on a
+ * path where allocation is forbidden.
+ *   - No allocation: the call never calls cudaMalloc, cudaFree or any
+ *     allocating library routine.
+ *   - Limit: shapes whose gdn_chunk_fwd_workspace_bytes exceeds the scratch
+ *     return GDN_ERR_WORKSPACE (nothing is enqueued); argument errors are
+ *     reported exactly as by gdn_chunk_fwd.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture on the device.
+ *   - Sharing: all calls on a device share the array and it keeps the last
+ *     call's contents (the forward needs no cleared scratch).  Calls whose
+ *     work overlaps on the GPU -- different streams, or unordered host
+ *     threads -- race on it; order them on one stream.
+ */
+GDN_API gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                         const void* beta, const void* g, gdn_gate gate_kind,
+                                         const float* initial_state, void* o,
+                                         float* final_state, int B, int T, int H, int Dk,
+                                         int Dv, int chunk, gdn_dtype dtype,
+                                         gdn_stream_t stream);
+
+/* Size in bytes of the scratch array gdn_chunk_fwd_noalloc uses. */
+GDN_API size_t gdn_chunk_fwd_noalloc_scratch_bytes(void);
+
 /* Number of kernels this library has launched in this process (all devices,
  * all entry points), counted on the host at each successful launch. */
 GDN_API unsigned long long gdn_kernel_launch_count(void);
