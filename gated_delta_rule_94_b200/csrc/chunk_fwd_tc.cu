@@ -411,9 +411,9 @@ constexpr uint32_t OFF_Z2 = 122880;    // zero block            } [Z2; P]
 constexpr uint32_t OFF_P = 131072;     // P, K-major [64 r][64 i]
 constexpr uint32_t OFF_WQ = 139264;    // [-W_b0 | Qbar_b0 | -W_b1 | Qbar_b1], K-major
 constexpr uint32_t OFF_HB = 172032;    // h (bf16) MN-major [d][64 v] x 2; after the
-constexpr uint32_t OFF_DL = 172032;    //   c-MMA: D [i][64 v] x 2
-constexpr uint32_t OFF_DT = 188416;    //   and D~ = diag(e^(G_C - G_i)) D
-constexpr uint32_t OFF_FAC = 204800;   // 2 x {e^G [64], e^(G_C - G) [64]}
+constexpr uint32_t OFF_DL = 172032;    //   c-MMA: D [i][64 v] x 2 (first 16 KB)
+constexpr uint32_t OFF_KT = 204800;    // K~ = diag(e^(G_C - G_i)) K, [K~_b0 | K~_b1]
+constexpr uint32_t OFF_FAC = 221184;   // 2 x {e^G [64], e^(G_C - G) [64]}
 constexpr uint32_t OFF_BAR = OFF_FAC + 2 * 128 * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 32 * 8 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -554,9 +554,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
             if (leader && !failed) {
                 const uint32_t id2 = idesc_bf16_f32(128, 128, true, true);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)   // state += K^T D~
-                    mma_bf16(tmem + TM_H, sdesc_sw128(st + k * 2048, 16384, 1024),
-                             sdesc_sw128(sb + OFF_DT + k * 2048, 8192, 1024), id2, true);
+                for (int k = 0; k < 4; ++k)   // state += K~^T D
+                    mma_bf16(tmem + TM_H, sdesc_sw128(sb + OFF_KT + k * 2048, 8192, 1024),
+                             sdesc_sw128(sb + OFF_DL + k * 2048, 8192, 1024), id2, true);
                 const uint32_t id1 = idesc_bf16_f32(128, 128, false, true);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)   // X += [Z2; P] D
@@ -588,21 +588,21 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
                 fence_async_smem();
                 load_v(nl);   // V buffer nl & 1: U of chunk nl-2 is long done
             }
-            // Q_bar = diag(e^G) Q into the Q rows of WQ (same swizzled layout), once the
-            // c-product of chunk nl-1 is done with WQ
+            // Q_bar = diag(e^G) Q into the Q rows of WQ (same swizzled layout) once the
+            // c-product of chunk nl-1 is done with WQ, and K~ = diag(e^(G_C - G)) K
+            // once the state update of chunk nl-1 is done with K~
             if (nl > 0) wait(B_CDONE, (nl - 1) & 1);
             wait(B_FFULL0 + s, (nl >> 1) & 1);
             wait(B_KQ0 + s, (nl >> 1) & 1);
-            {
-                const float* sGam = fac_buf(nl);
-                const uint8_t* stage = sm + OFF_KQ + s * KQ_STAGE;
+            const float* fac = fac_buf(nl);
+            const uint8_t* stage = sm + OFF_KQ + s * KQ_STAGE;
+            auto scale_rows = [&](uint32_t src_off, uint8_t* dst, const float* rowf) {
 #pragma unroll
                 for (int it = 0; it < 8; ++it) {
                     const int idx = st_id + NST * it;          // 16-byte chunk 0..1023
                     const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
-                    const uint32_t off = blk * 16384 + 8192 + r * 128 + j * 16;
-                    uint4 raw = *reinterpret_cast<const uint4*>(stage + off);
-                    const float gmul = sGam[r];
+                    uint4 raw = *reinterpret_cast<const uint4*>(stage + blk * 16384 + src_off + r * 128 + j * 16);
+                    const float gmul = rowf[r];
                     __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
                     uint4 outv;
                     uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
@@ -611,9 +611,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
                         const float2 f = __bfloat1622float2(e2[e]);
                         o32[e] = pack_bf16(f.x * gmul, f.y * gmul);
                     }
-                    *reinterpret_cast<uint4*>(sm + OFF_WQ + off) = outv;
+                    *reinterpret_cast<uint4*>(dst + blk * (dst == sm + OFF_KT ? 8192 : 16384) + r * 128 + j * 16) = outv;
                 }
-            }
+            };
+            scale_rows(8192, sm + OFF_WQ + 8192, fac);   // Q rows -> Q_bar rows of WQ
             // -W (TMEM lanes 64..127, warps 6-7) -> the W rows of WQ
             wait(B_WUDONE, nl & 1);
             tc_fence_after();
@@ -629,8 +630,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
             tc_fence_before();
             named_bar(3, NST);
             if (st_id == 0) mbar_arrive(&bars[B_WQREADY]);
-            // P of chunk nl once the d-products of chunk nl-1 are done with the buffer
+            // P and K~ of chunk nl once the d-products of chunk nl-1 are done with them
             if (nl > 0) wait(B_DDONE, (nl - 1) & 1);
+            scale_rows(0, sm + OFF_KT, fac + 64);          // K rows -> K~
+            fence_async_smem();
+            named_bar(3, NST);
             if (st_id == 0) {
                 mbar_arrive_expect_tx(&bars[B_PFULL], 8192);
                 bulk_load(sm + OFF_P, img + WS_P, 8192, &bars[B_PFULL]);
@@ -714,15 +718,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
             } else {
                 wait(B_CDONE, nl & 1);
                 tc_fence_after();
-                const float ft = fac[64 + tid];
                 const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
                 float dv[128];
                 ld_cols<128>(tX + lane_off, dv);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
+                for (int j = 0; j < 16; ++j)
                     st_row_chunk(sm + OFF_DL + (j >> 3) * 8192, tid, j & 7, dv + 8 * j, 1.f);
-                    st_row_chunk(sm + OFF_DT + (j >> 3) * 8192, tid, j & 7, dv + 8 * j, ft);
-                }
             }
             fence_async_smem();
             tc_fence_before();
