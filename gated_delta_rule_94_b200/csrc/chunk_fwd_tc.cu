@@ -259,7 +259,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p)
     const int bh = blockIdx.x / p.nchunks, nl = blockIdx.x % p.nchunks;
     const int b = bh / H, h = bh % H;
     const int n = p.chunk0 + nl;
-    uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * WS_CHUNK;
+    uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * p.ws_chunk;
     int failed = 0;
 
     if (tid == 0) {
@@ -400,6 +400,274 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p)
     }
 }
 
+// ------------------------------------------------------------------ per-dim
+// Workspace image of one per-dimension-gated chunk: the scalar layout
+// (T diag(beta) in both T slots, P, factors = e^(G_C) per key dimension),
+// followed by the chain's three per-element-scaled operand tiles.
+constexpr uint32_t WS_QB = WS_CHUNK;             // Q (.) e^G            [Q_b0 | Q_b1]
+constexpr uint32_t WS_KG = WS_QB + 16384;        // K (.) e^G            [K_b0 | K_b1]
+constexpr uint32_t WS_KT = WS_KG + 16384;        // K (.) e^(G_C - G)    [K_b0 | K_b1]
+constexpr uint32_t WS_CHUNK_PD = WS_KT + 16384;
+
+struct PrepPdMaps {
+    CUtensorMap q, k, g;
+};
+
+// Per-dim prep shared memory (bytes from a 1 KB-aligned base).
+constexpr int LDG = 132;                                  // fp32 row stride of G [64][128]
+constexpr uint32_t D_OFF_KQ = 0;                          // [K_b0 | Q_b0 | K_b1 | Q_b1] -> scaled in place
+constexpr uint32_t D_OFF_G16 = 32768;                     // g tile bf16 [g_b0 | g_b1]
+constexpr uint32_t D_OFF_KB = 49152;                      // K_breve [K_b0 | K_b1], K-major rows i
+constexpr uint32_t D_OFF_AF = 65536;                      // A fp32 [64][LDF]; G fp32 before it
+constexpr uint32_t D_OFF_TF = D_OFF_AF + 64 * LDF * 4;    // T fp32 [64][LDF]
+constexpr uint32_t D_OFF_SMALL = D_OFF_TF + 64 * LDF * 4; // beta[64], m[128], c[128], flag
+constexpr uint32_t D_OFF_BAR = D_OFF_SMALL + (64 + 4 * 128 + 4) * 4;
+constexpr uint32_t D_SMEM = D_OFF_BAR + 16 + 1024;
+static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A/T scratch");
+
+// One CTA per chunk of the wave (per-dimension gate).  With G the in-chunk
+// cumsum of g per key dimension, m = G_31 and c = G_63 per dimension:
+//   S = [K e^(G-m); Q e^(G-m)] (K e^(m-G))^T  -> A = StrictTril(beta S_kk),
+//   P = Tril(S_qk); both factors stay finite while every dimension decays by
+//   less than e^160 inside the chunk, else A and P are formed exactly on CUDA
+//   cores.  The chain's operands Q e^G, K e^G and K e^(G_C - G) go to the
+//   workspace as shared-memory images; T diag(beta) fills both T slots (the
+//   decay sits on K e^G for W).
+__global__ void __launch_bounds__(NPR)
+chunk_prep_pd_kernel(const __grid_constant__ PrepPdMaps maps, const ChunkParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    float* Af = reinterpret_cast<float*>(sm + D_OFF_AF);
+    float* Tf = reinterpret_cast<float*>(sm + D_OFF_TF);
+    float* Gs = reinterpret_cast<float*>(sm + D_OFF_AF);   // G, dead before A is written
+    float* sBeta = reinterpret_cast<float*>(sm + D_OFF_SMALL);
+    float* sM = sBeta + 64;
+    float* sC = sM + 128;
+    float* sEm = sC + 128;
+    float* sEcm = sEm + 128;
+    int* sFlag = reinterpret_cast<int*>(sEcm + 128);
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + D_OFF_BAR);
+    uint64_t* bar_s = bar_ld + 1;
+    __shared__ uint32_t s_tmem;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.H, T = p.T;
+    const int bh = blockIdx.x / p.nchunks, nl = blockIdx.x % p.nchunks;
+    const int b = bh / H, h = bh % H;
+    const int n = p.chunk0 + nl;
+    uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * p.ws_chunk;
+    int failed = 0;
+
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_s, 1);
+        fence_mbar_init();
+        *sFlag = 0;
+        mbar_arrive_expect_tx(bar_ld, 6 * 8192);
+        for (int blk = 0; blk < 2; ++blk) {
+            tma_load_3d(sm + D_OFF_KQ + blk * 16384, &maps.k, bar_ld, h * D + 64 * blk, n * C, b);
+            tma_load_3d(sm + D_OFF_KQ + blk * 16384 + 8192, &maps.q, bar_ld, h * D + 64 * blk, n * C, b);
+            tma_load_3d(sm + D_OFF_G16 + blk * 8192, &maps.g, bar_ld, h * D + 64 * blk, n * C, b);
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 64);
+        tmem_relinquish();
+    }
+    if (tid < 64) {
+        const int t = n * C + tid;
+        sBeta[tid] = (t < T) ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.beta)[((size_t)b * T + t) * H + h]) : 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    if (!mbar_wait(bar_ld, 0, &failed)) atomicOr(p.status, kStatusTimeout);
+    __syncwarp();
+    // ---- G = in-chunk cumsum of g per dimension: thread (d, half), 32 rows each
+    {
+        const int d = tid & 127, hh = tid >> 7;
+        const uint8_t* gt = sm + D_OFF_G16 + (d >> 6) * 8192;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int r = 32 * hh; r < 32 * hh + 32; ++r) {
+            acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(gt + sw128_offset(r, d & 63)));
+            Gs[r * LDG + d] = acc;
+        }
+    }
+    __syncthreads();
+    {
+        const int d = tid & 127, hh = tid >> 7;
+        if (hh == 1) {
+            const float carry = Gs[31 * LDG + d];
+#pragma unroll 8
+            for (int r = 32; r < 64; ++r) Gs[r * LDG + d] += carry;
+        }
+    }
+    __syncthreads();
+    if (tid < 128) {
+        const float m = Gs[31 * LDG + tid], c = Gs[63 * LDG + tid];
+        sM[tid] = m;
+        sC[tid] = c;
+        sEm[tid] = expf(m);
+        sEcm[tid] = expf(c - m);
+        if (Gs[tid] - c >= 160.f) atomicOr(sFlag, 1);
+    }
+    __syncthreads();
+    const bool exact = *sFlag != 0;
+    // ---- one pass over the tiles: Gram operands in place / K_breve, chain images
+#pragma unroll 1
+    for (int it = 0; it < 4; ++it) {
+        const int idx = tid + NPR * it;                 // 16-byte chunk 0..1023
+        const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+        const int d0 = blk * 64 + 8 * (j ^ (r & 7));    // logical columns of this chunk
+        const uint32_t rowoff = (uint32_t)(r * 128 + j * 16);
+        uint4 kraw = *reinterpret_cast<const uint4*>(sm + D_OFF_KQ + blk * 16384 + rowoff);
+        uint4 qraw = *reinterpret_cast<const uint4*>(sm + D_OFF_KQ + blk * 16384 + 8192 + rowoff);
+        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
+        const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
+        uint32_t kb[4], qb[4], kr[4], qg[4], kg[4], kt[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 kf = __bfloat1622float2(k2[e]);
+            const float2 qf = __bfloat1622float2(q2[e]);
+            float ef[2], er[2], eg[2], et[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int d = d0 + 2 * e + u;
+                const float G = Gs[r * LDG + d], m = sM[d];
+                if (!exact) {
+                    ef[u] = expf(G - m);
+                    er[u] = expf(m - G);
+                    eg[u] = sEm[d] * ef[u];     // e^G <= 1
+                    et[u] = sEcm[d] * er[u];    // e^(G_C - G) <= 1
+                } else {
+                    ef[u] = er[u] = 0.f;
+                    eg[u] = expf(G);
+                    et[u] = expf(sC[d] - G);
+                }
+            }
+            kb[e] = pack_bf16(kf.x * ef[0], kf.y * ef[1]);
+            qb[e] = pack_bf16(qf.x * ef[0], qf.y * ef[1]);
+            kr[e] = pack_bf16(kf.x * er[0], kf.y * er[1]);
+            qg[e] = pack_bf16(qf.x * eg[0], qf.y * eg[1]);
+            kg[e] = pack_bf16(kf.x * eg[0], kf.y * eg[1]);
+            kt[e] = pack_bf16(kf.x * et[0], kf.y * et[1]);
+        }
+        const uint32_t ioff = blk * 8192 + rowoff;
+        *reinterpret_cast<uint4*>(img + WS_QB + ioff) = make_uint4(qg[0], qg[1], qg[2], qg[3]);
+        *reinterpret_cast<uint4*>(img + WS_KG + ioff) = make_uint4(kg[0], kg[1], kg[2], kg[3]);
+        *reinterpret_cast<uint4*>(img + WS_KT + ioff) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
+        if (!exact) {
+            *reinterpret_cast<uint4*>(sm + D_OFF_KQ + blk * 16384 + rowoff) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
+            *reinterpret_cast<uint4*>(sm + D_OFF_KQ + blk * 16384 + 8192 + rowoff) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
+            *reinterpret_cast<uint4*>(sm + D_OFF_KB + ioff) = make_uint4(kr[0], kr[1], kr[2], kr[3]);
+        }
+    }
+    if (tid < 128) reinterpret_cast<float*>(img + WS_FAC)[tid] = expf(sC[tid]);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (!exact) {
+        if (tid == 32) {   // S = [K e^(G-m); Q e^(G-m)] (K e^(m-G))^T
+            const uint32_t st = smem_u32(sm + D_OFF_KQ), kbr = smem_u32(sm + D_OFF_KB);
+            const uint32_t id = idesc_bf16_f32(128, 64, false, false);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t a = st + (k >> 2) * 16384 + (k & 3) * 32;
+                const uint32_t bb = kbr + (k >> 2) * 8192 + (k & 3) * 32;
+                mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id, k > 0);
+            }
+            mma_commit(bar_s);
+        }
+        if (!mbar_wait(bar_s, 0, &failed)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+        tc_fence_after();
+        __syncthreads();   // G (aliased with A) is dead from here on
+        const int q4 = warp & 3, ch = warp >> 2;
+        const int L = q4 * 32 + lane;
+        float sv[32];
+        ld_cols<32>(tmem + ((uint32_t)(q4 * 32) << 16) + 32 * ch, sv);
+        if (L < 64) {
+            const int r = L;
+            const float br = sBeta[r];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sv[e] = (32 * ch + e < r) ? br * sv[e] : 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(Af + r * LDF + 32 * ch + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+        } else {
+            const int r = L - 64;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sv[e] = (32 * ch + e <= r) ? sv[e] : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) st_row_chunk(img + WS_P, r, 4 * ch + jj, sv + 8 * jj, 1.f);
+        }
+    } else {
+        // exact A and P: sum_d k_rd k_id e^(G_rd - G_id) with every exponent <= 0;
+        // A goes to registers first since it shares space with G
+        const int q4 = warp & 3, ch = warp >> 2;
+        const int L = q4 * 32 + lane;
+        const int r = L & 63;
+        const bool isq = L >= 64;
+        const uint8_t* rowt = sm + D_OFF_KQ + (isq ? 8192 : 0);
+        float sv[32];
+#pragma unroll 1
+        for (int e = 0; e < 32; ++e) {
+            const int i = 32 * ch + e;
+            float acc = 0.f;
+            if (isq ? (i <= r) : (i < r)) {
+#pragma unroll 4
+                for (int d = 0; d < D; ++d) {
+                    const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                        rowt + (d >> 6) * 16384 + sw128_offset(r, d & 63)));
+                    const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                        sm + D_OFF_KQ + (d >> 6) * 16384 + sw128_offset(i, d & 63)));
+                    acc = fmaf(x * kk, expf(Gs[r * LDG + d] - Gs[i * LDG + d]), acc);
+                }
+            }
+            sv[e] = isq ? acc : sBeta[r] * acc;
+        }
+        __syncthreads();   // G (aliased with A) is dead from here on
+        if (!isq) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(Af + r * LDF + 32 * ch + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) st_row_chunk(img + WS_P, r, 4 * ch + jj, sv + 8 * jj, 1.f);
+        }
+    }
+    __syncthreads();
+    forward_substitution(Af, Tf, tid);
+    {
+        const int r = tid >> 2, j0 = 2 * (tid & 3);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int j = j0 + jj;
+            const float4 t0 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j);
+            const float4 t1 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j + 4);
+            const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            float tu[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int i = 8 * j + e;
+                tu[e] = (i <= r) ? tv[e] * sBeta[i] : 0.f;
+            }
+            st_row_chunk(img + WS_TU, r, j, tu, 1.f);
+            st_row_chunk(img + WS_TW, r, j, tu, 1.f);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
+}
+
 // Chain kernel shared memory (bytes from a 1 KB-aligned base).
 constexpr uint32_t KQ_STAGE = 32768;   // [K_b0 | Q_b0 | K_b1 | Q_b1], 8 KB each, K-major
 constexpr uint32_t OFF_KQ = 0;         // 2 stages
@@ -430,7 +698,7 @@ constexpr uint32_t TM_W = 384;    // [0; W], lanes 64..127, 128 columns d
 
 enum Bar {
     B_KQ0, B_KQ1, B_VFULL, B_TFULL, B_PFULL, B_FFULL0, B_FFULL1, B_WUDONE, B_CDONE, B_DDONE,
-    B_WQREADY, B_HBREADY, B_DREADY, B_XFREE, B_FINAL, B_COUNT
+    B_WQREADY, B_HBREADY, B_DREADY, B_XFREE, B_QFULL, B_FINAL, B_COUNT
 };
 
 struct TcMaps {
@@ -438,7 +706,7 @@ struct TcMaps {
 };
 
 __global__ void __launch_bounds__(NT, 1)
-chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, int gated) {
+chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, int gated, int perdim) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -450,7 +718,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
     const int H = p.H, T = p.T;
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int NC = p.nchunks;              // local chunk nl = 0..NC-1 is chunk p.chunk0 + nl
-    const uint8_t* wsh = p.ws + (size_t)bh * p.cw * WS_CHUNK;
+    const uint8_t* wsh = p.ws + (size_t)bh * p.cw * p.ws_chunk;
     int failed = 0;
 
     if (tid == 0) {
@@ -500,7 +768,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
     if (warp == 8) {
         // =========================== control: TMA for the first tiles and V, every MMA
         const bool leader = lane == 0;   // issues only while no wait has failed
-        if (leader) {
+        if (leader && !perdim) {
             fence_async_smem();
             load_kq(0);
             if (NC > 1) load_kq(1);
@@ -513,7 +781,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
             const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
             wait(B_TFULL, nl & 1);
             wait(B_VFULL, nl & 1);
-            wait(B_KQ0 + s, (nl >> 1) & 1);
+            if (!perdim) wait(B_KQ0 + s, (nl >> 1) & 1);
             if (nl >= 2) wait(B_XFREE, (nl - 2) & 1);
             tc_fence_after();
             if (leader && !failed) {
@@ -533,7 +801,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            const uint32_t st = sb + OFF_KQ + s * KQ_STAGE;
             const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
             wait(B_WQREADY, nl & 1);
             wait(B_HBREADY, nl & 1);
@@ -577,12 +844,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            const uint8_t* img = wsh + (size_t)nl * WS_CHUNK;
+            const uint8_t* img = wsh + (size_t)nl * p.ws_chunk;
             if (st_id == 0) {   // W/U of chunk nl-1 are done with T_u / T_w, and the chain is
                                 // done with the factors of chunk nl-2 (both waited below)
-                mbar_arrive_expect_tx(&bars[B_TFULL], 2 * 8192);
+                mbar_arrive_expect_tx(&bars[B_TFULL], perdim ? 4 * 8192 : 2 * 8192);
                 bulk_load(sm + OFF_TU, img + WS_TU, 8192, &bars[B_TFULL]);
                 bulk_load(sm + OFF_TW, img + WS_TW, 8192, &bars[B_TFULL]);
+                if (perdim) {   // K e^G into the K slots of stage nl & 1 (W of chunk nl-2 is done)
+                    uint8_t* stg = sm + OFF_KQ + s * KQ_STAGE;
+                    bulk_load(stg, img + WS_KG, 8192, &bars[B_TFULL]);
+                    bulk_load(stg + 16384, img + WS_KG + 8192, 8192, &bars[B_TFULL]);
+                }
                 mbar_arrive_expect_tx(&bars[B_FFULL0 + s], 512);
                 bulk_load(fac_buf(nl), img + WS_FAC, 512, &bars[B_FFULL0 + s]);
                 fence_async_smem();
@@ -593,7 +865,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
             // once the state update of chunk nl-1 is done with K~
             if (nl > 0) wait(B_CDONE, (nl - 1) & 1);
             wait(B_FFULL0 + s, (nl >> 1) & 1);
-            wait(B_KQ0 + s, (nl >> 1) & 1);
+            if (!perdim) wait(B_KQ0 + s, (nl >> 1) & 1);
             const float* fac = fac_buf(nl);
             const uint8_t* stage = sm + OFF_KQ + s * KQ_STAGE;
             auto scale_rows = [&](uint32_t src_off, uint8_t* dst, const float* rowf) {
@@ -614,7 +886,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
                     *reinterpret_cast<uint4*>(dst + blk * (dst == sm + OFF_KT ? 8192 : 16384) + r * 128 + j * 16) = outv;
                 }
             };
-            scale_rows(8192, sm + OFF_WQ + 8192, fac);   // Q rows -> Q_bar rows of WQ
+            if (!perdim) {
+                scale_rows(8192, sm + OFF_WQ + 8192, fac);   // Q rows -> Q_bar rows of WQ
+            } else if (st_id == 0) {                         // Q e^G image -> Q_bar rows of WQ
+                mbar_arrive_expect_tx(&bars[B_QFULL], 2 * 8192);
+                bulk_load(sm + OFF_WQ + 8192, img + WS_QB, 8192, &bars[B_QFULL]);
+                bulk_load(sm + OFF_WQ + 8192 + 16384, img + WS_QB + 8192, 8192, &bars[B_QFULL]);
+            }
             // -W (TMEM lanes 64..127, warps 6-7) -> the W rows of WQ
             wait(B_WUDONE, nl & 1);
             tc_fence_after();
@@ -626,18 +904,22 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
                 for (int j = 0; j < 16; ++j)
                     st_row_chunk(sm + OFF_WQ + (j >> 3) * 16384, r, j & 7, wv + 8 * j, -1.f);
             }
+            if (perdim) wait(B_QFULL, nl & 1);
             fence_async_smem();
             tc_fence_before();
             named_bar(3, NST);
             if (st_id == 0) mbar_arrive(&bars[B_WQREADY]);
             // P and K~ of chunk nl once the d-products of chunk nl-1 are done with them
             if (nl > 0) wait(B_DDONE, (nl - 1) & 1);
-            scale_rows(0, sm + OFF_KT, fac + 64);          // K rows -> K~
-            fence_async_smem();
-            named_bar(3, NST);
+            if (!perdim) {
+                scale_rows(0, sm + OFF_KT, fac + 64);      // K rows -> K~
+                fence_async_smem();
+                named_bar(3, NST);
+            }
             if (st_id == 0) {
-                mbar_arrive_expect_tx(&bars[B_PFULL], 8192);
+                mbar_arrive_expect_tx(&bars[B_PFULL], perdim ? 3 * 8192 : 8192);
                 bulk_load(sm + OFF_P, img + WS_P, 8192, &bars[B_PFULL]);
+                if (perdim) bulk_load(sm + OFF_KT, img + WS_KT, 16384, &bars[B_PFULL]);
             }
         }
     } else {
@@ -678,7 +960,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
             if (nl > 0) {
                 wait(B_DDONE, (nl - 1) & 1);
                 tc_fence_after();
-                if (tid == 0 && nl + 1 < NC) {
+                if (tid == 0 && nl + 1 < NC && !perdim) {
                     fence_async_smem();
                     load_kq(nl + 1);
                 }
@@ -698,7 +980,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
             wait(B_FFULL0 + s, (nl >> 1) & 1);
             const float* fac = fac_buf(nl);
             if (gated) {
-                const float gam = fac[63];
+                const float gam = perdim ? fac[tid] : fac[63];
                 float hv[128];
                 ld_cols<128>(tmem + TM_H + lane_off, hv);
 #pragma unroll
@@ -766,8 +1048,8 @@ bool make_maps(const ChunkParams& p, TcMaps* m) {
 
 // Chunk slots per (batch, head) of one wave: as many as keep the wave's
 // workspace near WAVE_BYTES (L2-resident), at least 4.
-int wave_chunks(int nbh, int NC) {
-    long long cw = (long long)(WAVE_BYTES / ((size_t)nbh * WS_CHUNK));
+int wave_chunks(int nbh, int NC, uint32_t image_bytes) {
+    long long cw = (long long)(WAVE_BYTES / ((size_t)nbh * image_bytes));
     if (cw < 4) cw = 4;
     if (cw > NC) cw = NC;
     return (int)(cw < 1 ? 1 : cw);
@@ -776,16 +1058,20 @@ int wave_chunks(int nbh, int NC) {
 }  // namespace
 
 bool chunk_fwd_tc_supported(int Dk, int Dv, int gate) {
-    return Dk == D && Dv == D && (gate == kGateNone || gate == kGateScalar);
+    return Dk == D && Dv == D && (gate == kGateNone || gate == kGateScalar || gate == kGatePerDim);
 }
 
-size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H) {
+namespace {
+uint32_t image_bytes(int gate) { return gate == kGatePerDim ? WS_CHUNK_PD : WS_CHUNK; }
+}  // namespace
+
+size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H, int gate) {
     const int NC = (T + C - 1) / C;
     if (NC == 0 || B == 0 || H == 0) return 0;
     const int nbh = B * H;
-    const int cw = wave_chunks(nbh, NC);
+    const int cw = wave_chunks(nbh, NC, image_bytes(gate));
     const int nw = (NC + cw - 1) / cw;
-    size_t bytes = (size_t)nbh * cw * WS_CHUNK;
+    size_t bytes = (size_t)nbh * cw * image_bytes(gate);
     if (nw > 1) bytes += (size_t)nbh * D * D * sizeof(float);   // state between waves
     return bytes;
 }
@@ -794,29 +1080,47 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s,
     *launches = 0;
     TcMaps maps;
     if (!make_maps(p0, &maps)) return cudaErrorInvalidValue;
+    const bool perdim = gate == kGatePerDim;
     PrepMaps pmaps;
     pmaps.q = maps.q;
     pmaps.k = maps.k;
+    PrepPdMaps dmaps;
+    dmaps.q = maps.q;
+    dmaps.k = maps.k;
+    if (perdim) {
+        const uint64_t dims[3] = {(uint64_t)p0.H * D, (uint64_t)p0.T, (uint64_t)p0.B};
+        const uint64_t strides[2] = {(uint64_t)p0.H * D * 2, (uint64_t)p0.T * p0.H * D * 2};
+        const uint32_t box[3] = {64, 64, 1};
+        if (!make_tmap_bf16(&dmaps.g, p0.g, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
     auto prep = gate == kGateScalar ? chunk_prep_tc_kernel<kGateScalar> : chunk_prep_tc_kernel<kGateNone>;
     cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk_prep_pd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)D_SMEM);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int NC = (p0.T + C - 1) / C;
     const int nbh = p0.B * p0.H;
-    const int cw = wave_chunks(nbh, NC);
+    const uint32_t img = image_bytes(gate);
+    const int cw = wave_chunks(nbh, NC, img);
     const int nw = (NC + cw - 1) / cw;
-    float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + (size_t)nbh * cw * WS_CHUNK) : nullptr;
+    float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + (size_t)nbh * cw * img) : nullptr;
     for (int w = 0; w < nw; ++w) {
         ChunkParams p = p0;
         p.cw = cw;
+        p.ws_chunk = (int)img;
         p.chunk0 = w * cw;
         p.nchunks = (w + 1 < nw) ? cw : NC - w * cw;
         p.s0 = (w == 0) ? p0.s0 : carry;
         p.s_out = (w + 1 == nw) ? p0.s_out : carry;
-        prep<<<(unsigned)(nbh * p.nchunks), NPR, P_SMEM, s>>>(pmaps, p);
+        if (perdim)
+            chunk_prep_pd_kernel<<<(unsigned)(nbh * p.nchunks), NPR, D_SMEM, s>>>(dmaps, p);
+        else
+            prep<<<(unsigned)(nbh * p.nchunks), NPR, P_SMEM, s>>>(pmaps, p);
         ++*launches;
-        chunk_fwd_tc_kernel<<<(unsigned)nbh, NT, SMEM_BYTES, s>>>(maps, p, gate == kGateScalar ? 1 : 0);
+        chunk_fwd_tc_kernel<<<(unsigned)nbh, NT, SMEM_BYTES, s>>>(maps, p, gate != kGateNone ? 1 : 0,
+                                                                  perdim ? 1 : 0);
         ++*launches;
     }
     return cudaGetLastError();

@@ -29,6 +29,7 @@ struct ChunkParams {
     int cw;            // chunk slots per (batch, head) in the workspace
     int chunk0;        // first chunk of this wave
     int nchunks;       // chunks in this wave
+    int ws_chunk;      // bytes of one chunk's workspace image
 };
 
 struct DecodeParams {
@@ -57,7 +58,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 namespace gdn {
 cudaError_t launch_chunk_fwd_simt(const ChunkParams& p, int gate, bool bf16, cudaStream_t s);
 bool chunk_fwd_tc_supported(int Dk, int Dv, int gate);
-size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H);
+size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H, int gate);
 // Enqueues the tensor-core forward; *launches receives the number of kernels.
 cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, cudaStream_t s, int* launches);
 cudaError_t launch_decode_step(const DecodeParams& p, int Dk, int Dv, int gate, bool bf16,

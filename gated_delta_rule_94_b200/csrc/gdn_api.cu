@@ -79,7 +79,7 @@ size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int ch
     if (dtype != GDN_BF16 && dtype != GDN_F32) return (size_t)-1;
     if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return (size_t)-1;
     if (dtype == GDN_BF16 && gdn::chunk_fwd_tc_supported(Dk, Dv, gate_kind))
-        return gdn::chunk_fwd_tc_workspace_bytes(B, T, H);
+        return gdn::chunk_fwd_tc_workspace_bytes(B, T, H, gate_kind);
     return 0;
 }
 
@@ -144,6 +144,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
     p.cw = 0;
     p.chunk0 = 0;
     p.nchunks = 0;
+    p.ws_chunk = 0;
     if (!p.status) return GDN_ERR_CUDA;
     cudaError_t e;
     int launches = 1;

@@ -174,3 +174,17 @@ def test_device_status_clear():
     x = gi.make_inputs(1, 64, 1, 64, 64, dtype=torch.bfloat16, seed=0)
     gpu_chunk(x)
     assert gdn.gdn_read_device_status() == 0
+
+
+@pytest.mark.parametrize("gate", ["per_dim", "scalar"])
+def test_extreme_decay_exact_fallback(gate):
+    """Log-decay of ~3.5 per token: the in-chunk decay range (~220) exceeds what
+    the factorized exponentials can hold, so the per-dimension prep takes its
+    exact CUDA-core path for A and P (and the scalar gate its per-element
+    exponentials); the result must still match the oracle."""
+    x = gi.make_inputs(2, 160, 2, 128, 128, dtype=torch.bfloat16, gate=gate, gate_scale=5.0,
+                       s0_std=1.0, seed=21)
+    o, S = gpu_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check("o", o, o_ref, TOL[torch.bfloat16])
+    check("S", S, S_ref, TOL[torch.bfloat16])
