@@ -189,8 +189,9 @@ __device__ __forceinline__ void forward_substitution(const float* A, float* Tm, 
 
 // In-chunk gates for one scalar-gated chunk, by one warp: inclusive scan of g
 // (two tokens per lane), e^G, e^(G_C - G), and the factors u_r = e^(G_r - G_31),
-// w_i = e^(G_31 - G_i) with e^(G_r - G_i) = u_r w_i, usable while the in-chunk
-// decay stays below e^160 (flag).  gbuf[0..63] holds g on entry.
+// w_i = e^(G_31 - G_i) with e^(G_r - G_i) = u_r w_i, usable while each half of
+// the chunk decays by less than e^80, so that every factor and its reciprocal
+// stay normal fp32 numbers (flag).  gbuf[0..63] holds g on entry.
 template <int GATE>
 __device__ __forceinline__ void chunk_gates(float* gbuf, int lane) {
     if constexpr (GATE == kGateScalar) {
@@ -217,7 +218,7 @@ __device__ __forceinline__ void chunk_gates(float* gbuf, int lane) {
         gbuf[256 + 2 * lane + 1] = expf(G1 - Gm);
         gbuf[320 + 2 * lane] = expf(Gm - G0);
         gbuf[320 + 2 * lane + 1] = expf(Gm - G1);
-        if (lane == 0) gbuf[384] = (G00 - Gl < 160.f) ? 1.f : 0.f;
+        if (lane == 0) gbuf[384] = (G00 - Gm < 80.f && Gm - Gl < 80.f) ? 1.f : 0.f;
     } else {
         gbuf[2 * lane] = gbuf[2 * lane + 1] = 0.f;
         gbuf[64 + 2 * lane] = gbuf[64 + 2 * lane + 1] = 1.f;
@@ -428,9 +429,9 @@ static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A/T scratch");
 // One CTA per chunk of the wave (per-dimension gate).  With G the in-chunk
 // cumsum of g per key dimension, m = G_31 and c = G_63 per dimension:
 //   S = [K e^(G-m); Q e^(G-m)] (K e^(m-G))^T  -> A = StrictTril(beta S_kk),
-//   P = Tril(S_qk); both factors stay finite while every dimension decays by
-//   less than e^160 inside the chunk, else A and P are formed exactly on CUDA
-//   cores.  The chain's operands Q e^G, K e^G and K e^(G_C - G) go to the
+//   P = Tril(S_qk); both factors and their reciprocals stay normal fp32 while
+//   every dimension decays by less than e^80 in each half of the chunk, else
+//   A and P are formed exactly on CUDA cores.  The chain's operands Q e^G, K e^G and K e^(G_C - G) go to the
 //   workspace as shared-memory images; T diag(beta) fills both T slots (the
 //   decay sits on K e^G for W).
 __global__ void __launch_bounds__(NPR)
@@ -512,7 +513,7 @@ chunk_prep_pd_kernel(const __grid_constant__ PrepPdMaps maps, const ChunkParams 
         sC[tid] = c;
         sEm[tid] = expf(m);
         sEcm[tid] = expf(c - m);
-        if (Gs[tid] - c >= 160.f) atomicOr(sFlag, 1);
+        if (Gs[tid] - m >= 80.f || m - c >= 80.f) atomicOr(sFlag, 1);
     }
     __syncthreads();
     const bool exact = *sFlag != 0;

@@ -188,3 +188,22 @@ def test_extreme_decay_exact_fallback(gate):
     o_ref, S_ref = oracle_chunk(x)
     check("o", o, o_ref, TOL[torch.bfloat16])
     check("S", S, S_ref, TOL[torch.bfloat16])
+
+
+@pytest.mark.parametrize("gate", ["per_dim", "scalar"])
+def test_one_sided_decay_in_chunk(gate):
+    """Every chunk decays by ~100 in its first half and not at all in its
+    second: the whole-chunk range is moderate, but a half-chunk factor would
+    leave the fp32 range, so the prep must take its exact path (a full chunk
+    and the ragged tail both meet this)."""
+    x = gi.make_inputs(1, 160, 2, 128, 128, dtype=torch.bfloat16, gate=gate, s0_std=1.0,
+                       seed=23)
+    g = x["g"]
+    pos = torch.arange(160) % 64
+    step = torch.where(pos < 32, torch.tensor(-3.2), torch.tensor(0.0))
+    shape = [1, 160] + [1] * (g.dim() - 2)
+    x["g"] = torch.broadcast_to(step.view(shape), g.shape).contiguous().to(g.dtype)
+    o, S = gpu_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check("o", o, o_ref, TOL[torch.bfloat16])
+    check("S", S, S_ref, TOL[torch.bfloat16])
