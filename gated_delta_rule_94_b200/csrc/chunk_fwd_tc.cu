@@ -4,34 +4,34 @@
 // The chunkwise algorithm of "Moonshot AI's New Attention Architecture: Key
 // Innovations Explained" (sec. 3, state recurrence and causal output) with the
 // UT/WY transform of "OSDN: Improving Delta Rule with Provable Online
-// Preconditioning in Linear Attention" (sec. 2.1, chunk Gram matrix + WY),
-// for a scalar (or no) forget gate.  Per chunk of C = 64 tokens, h the
-// entering state M = S^T [d_k][d_v], G the in-chunk log-decay cumsum:
-//   S  = [K; Q] K^T                 (one 128-row MMA: K K^T and Q K^T)
-//   A  = StrictTril(beta_r e^(G_r-G_i) (K K^T)_ri),  P = Tril(e^(G_r-G_i) (Q K^T)_ri)
-//   T  = (I + A)^-1                 (blocked forward substitution)
-//   [0; W] = [0; T diag(beta e^G)] K
-//   X  = [T diag(beta); 0] V        = [U; 0]
-//   X += [-W; Q_bar] h              -> rows 0..63: D = U - W h, rows 64..127: Q_bar h
-//   X += [0; P] D                   -> rows 64..127: O = Q_bar h + P D
-//   h  = e^(G_C) h + K^T (diag(e^(G_C - G_i)) D)
-// Every product is a tcgen05.mma with M = 128; operands live in 128 B-swizzled
-// shared memory: the K/Q/V tiles exactly as TMA loads them (K-major when the
-// tokens are rows, MN-major when they are the reduction dimension), the other
-// operands written in the same canonical layouts.
+// Preconditioning in Linear Attention" (sec. 2.1, chunk Gram matrix + WY).
+// Per chunk of C = 64 tokens, h the entering state M = S^T [d_k][d_v], G the
+// in-chunk log-decay cumsum (per token, or per token and key dimension):
+//   A  = StrictTril(diag(beta) (K e^G)(K e^-G)^T),  P = Tril((Q e^G)(K e^-G)^T)
+//   T  = (I + A)^-1                               (blocked forward substitution)
+//   W  = T diag(beta) (K e^G),  U = T diag(beta) V,  K~ = K e^(G_C - G)
+//   D  = U - W h,  O = (Q e^G) h + P D,  h' = Diag(e^(G_C)) h + K~^T D.
+// Substituting D, each chunk is an affine map of the entering state:
+//   h' = (Diag(gamma) + Phi) h + Psi,     Phi = -K~^T W,  Psi = K~^T U
+//   O  = Qp h + P U,                      Qp = Q e^G - P W
+// with gamma = e^(G_C).  Phi, Psi, Qp, P U and gamma depend on the chunk's
+// inputs only, so they are formed for every chunk at once, and only the
+// product with h remains on the serial path.
 //
 // Two kernels per wave of chunks:
-//   chunk_prep_tc_kernel  one CTA per chunk, fully parallel: gates, S, A, P,
-//                         T, and the bf16 operands T diag(beta),
-//                         T diag(beta e^G), P plus the gate factors, written
-//                         to the workspace as the exact shared-memory image
-//                         the chain kernel uses (the wave is sized so the
-//                         workspace stays in L2);
-//   chunk_fwd_tc_kernel   one CTA per (batch, head), the serial state chain:
-//                         bulk-copies the prep images, W / U products, the
-//                         c- and d-products, state and output, with warp roles
-//                         chain (0-3), stager (4-7) and control (8) handing
-//                         over through mbarriers.
+//   chunk_prep_kernel   one CTA per (batch, head, chunk), fully parallel: the
+//                       gates, S = [K;Q]K^T, A and P, T, the WY factors as
+//                       W^T = K^T T^T and U^T = V^T T^T, then
+//                       [Phi | Psi] = -/+ K~^T [W | U] and [P W | P U]; writes
+//                       the chunk's step image (Phi, Psi, Qp, P U in bf16,
+//                       gamma in fp32) to the workspace, laid out exactly as
+//                       the chain kernel's shared-memory operands (the wave is
+//                       sized so the workspace stays in L2);
+//   chunk_chain_kernel  one CTA per (batch, head), the serial state chain:
+//                       per chunk one 8-step MMA h += Phi h_bf16 onto the
+//                       decayed fp32 state in TMEM, the state pass
+//                       (h + Psi -> bf16 operand, decay) and, off the serial
+//                       path, O^T = h^T Qp^T + (P U)^T.
 // Every mbarrier wait is bounded; a wait that gives up sets the library status
 // word and the kernel winds down without further waits.
 #include "common.cuh"
@@ -47,21 +47,23 @@ constexpr int C = 64;
 constexpr int D = 128;
 constexpr int NPR = 256;         // prep kernel threads (8 warps)
 constexpr int LDF = 72;          // fp32 row stride of the A / T scratch (conflict-free mma fragments)
-constexpr int GATE_FLOATS = 7 * 64;   // G, e^G, e^(G_C-G), beta, u, w, flag
 
-// Workspace image of one chunk (bytes).
-constexpr uint32_t WS_TU = 0;          // T diag(beta), K-major [64 r][64 i], swizzled
-constexpr uint32_t WS_TW = 8192;       // T diag(beta e^G)
-constexpr uint32_t WS_P = 16384;       // P
-constexpr uint32_t WS_FAC = 24576;     // e^G [64], e^(G_C - G) [64] (fp32)
-constexpr uint32_t WS_CHUNK = WS_FAC + 2 * 64 * 4;
-constexpr size_t WAVE_BYTES = size_t(32) << 20;   // workspace per wave (kept L2-resident)
+// Step image of one chunk (bytes).  Tiles of bf16 rows of 64 elements with the
+// 128-byte swizzle; a [rows][128] matrix is two such column blocks.
+constexpr uint32_t IMG_PHI = 0;        // Phi  [128 d][128 d'],  blocks of 16 KB (K-major A)
+constexpr uint32_t IMG_PSI = 32768;    // Psi  [128 d][128 v],   blocks of 16 KB
+constexpr uint32_t IMG_QP = 65536;     // Qp   [64 r][128 d],    blocks of 8 KB (K-major B)
+constexpr uint32_t IMG_PU = 81920;     // P U  [64 r][128 v],    blocks of 8 KB
+constexpr uint32_t IMG_GAM = 98304;    // gamma fp32 [128]
+constexpr uint32_t IMG_BYTES = 98816;
+constexpr size_t WAVE_BYTES = size_t(40) << 20;   // workspace per wave (kept L2-resident)
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&t);
 }
 
+// Chunk j (8 elements) of row `row` of a [rows][64] swizzled bf16 tile.
 __device__ __forceinline__ void st_row_chunk(uint8_t* tile, int row, int j, const float* v,
                                              float scale) {
     uint4 w;
@@ -70,6 +72,18 @@ __device__ __forceinline__ void st_row_chunk(uint8_t* tile, int row, int j, cons
     w.z = pack_bf16(v[4] * scale, v[5] * scale);
     w.w = pack_bf16(v[6] * scale, v[7] * scale);
     *reinterpret_cast<uint4*>(tile + sw128_offset(row, 8 * j)) = w;
+}
+
+// Row `row` (128 elements) of a [rows][128] matrix stored as two swizzled
+// column blocks `bstride` bytes apart.
+__device__ __forceinline__ void st_row128(uint8_t* tile, uint32_t bstride, int row, const float* v,
+                                          float scale) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) st_row_chunk(tile + (j >> 3) * bstride, row, j & 7, v + 8 * j, scale);
+}
+
+__device__ __forceinline__ float ld_bf16(const uint8_t* tile, int row, int col) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + sw128_offset(row, col)));
 }
 
 __device__ __forceinline__ void named_bar(int id, int count) {
@@ -186,7 +200,6 @@ __device__ __forceinline__ void forward_substitution(const float* A, float* Tm, 
     named_bar(2, NPR);
 }
 
-
 // In-chunk gates for one scalar-gated chunk, by one warp: inclusive scan of g
 // (two tokens per lane), e^G, e^(G_C - G), and the factors u_r = e^(G_r - G_31),
 // w_i = e^(G_31 - G_i) with e^(G_r - G_i) = u_r w_i, usable while each half of
@@ -230,51 +243,96 @@ __device__ __forceinline__ void chunk_gates(float* gbuf, int lane) {
 }
 
 struct PrepMaps {
-    CUtensorMap q, k;
+    CUtensorMap q, k, v, g;   // g only for the per-dimension gate
 };
 
 // Prep shared memory (bytes from a 1 KB-aligned base).
-constexpr uint32_t P_OFF_KQ = 0;                          // [K_b0 | Q_b0 | K_b1 | Q_b1]
-constexpr uint32_t P_OFF_AF = 32768;                      // A fp32 [64][LDF]
-constexpr uint32_t P_OFF_TF = P_OFF_AF + 64 * LDF * 4;    // T fp32 [64][LDF]
-constexpr uint32_t P_OFF_GATE = P_OFF_TF + 64 * LDF * 4;
-constexpr uint32_t P_OFF_BAR = P_OFF_GATE + GATE_FLOATS * 4;
-constexpr uint32_t P_SMEM = P_OFF_BAR + 16 + 1024;
+constexpr uint32_t P_KQ = 0;                 // [K_b0 | Q_b0 | K_b1 | Q_b1] (TMA)
+constexpr uint32_t P_V = 32768;              // [V_b0 | V_b1] (TMA)
+constexpr uint32_t P_AF = 49152;             // A fp32 [64][LDF]; later [W^T; U^T] bf16 [256][64]
+constexpr uint32_t P_TF = P_AF + 64 * LDF * 4;   // T fp32 [64][LDF]
+constexpr uint32_t P_WUT = P_AF;
+constexpr uint32_t P_TW = 86016;             // T diag(beta e^G) bf16 [64 r][64 i]
+constexpr uint32_t P_TU = 94208;             // T diag(beta)
+constexpr uint32_t P_KT = 102400;            // K~ = K e^(G_C - G)  [b0 | b1]
+constexpr uint32_t P_P = 118784;             // P bf16 [64 r][64 i]
+constexpr uint32_t P_GATE = 126976;          // G, e^G, e^(G_C-G), beta, u, w, flag (7 x 64 floats)
+constexpr uint32_t P_BAR = P_GATE + 7 * 64 * 4;
+constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;
+// per-dimension gate extras
+constexpr uint32_t X_G16 = 129024;           // g tile bf16 [g_b0 | g_b1] (TMA)
+constexpr uint32_t X_KB = X_G16 + 16384;     // K e^(m - G)      [b0 | b1]
+constexpr uint32_t X_KG = X_KB + 16384;      // K e^G            [b0 | b1]
+constexpr uint32_t X_QB = X_KG + 16384;      // Q e^G            [b0 | b1]
+constexpr uint32_t X_SMALL = X_QB + 16384;   // m, c, e^m, e^(c-m) [128 each], flag
+constexpr uint32_t P_SMEM_PD = X_SMALL + 4 * 128 * 4 + 16 + 1024;
+constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (aliases A / T)
+static_assert(P_TF + 64 * LDF * 4 <= P_TW, "A / T scratch");
+static_assert(P_WUT + 32768 <= P_TW, "[W^T; U^T] tile");
+static_assert(P_BAR + 64 <= X_G16, "prep layout");
+static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
+static_assert(P_SMEM_PD <= 232448, "prep shared memory");
 
-// One CTA per chunk of the wave: everything that does not depend on the state.
+// TMEM columns of the prep kernel (512 allocated).
+constexpr uint32_t TM_S = 0;       // [K;Q] K^T, 64 columns
+constexpr uint32_t TM_WT = 64;     // W^T, lanes d, 64 columns r
+constexpr uint32_t TM_UT = 128;    // U^T, lanes v, 64 columns r
+constexpr uint32_t TM_FP = 256;    // [K~^T W | K~^T U], 256 columns
+constexpr uint32_t TM_PP = 0;      // [P W | P U] (M = 64: rows in lanes 0-15 of each quarter)
+
+// One CTA per (batch, head, chunk) of the wave: every state-independent part
+// of the chunk, written to the workspace as the chunk's step image.
 template <int GATE>
-__global__ void __launch_bounds__(NPR)
-chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
+__global__ void __launch_bounds__(NPR, 1)
+chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-    float* Af = reinterpret_cast<float*>(sm + P_OFF_AF);
-    float* Tf = reinterpret_cast<float*>(sm + P_OFF_TF);
-    float* gbuf = reinterpret_cast<float*>(sm + P_OFF_GATE);
-    uint64_t* bar_kq = reinterpret_cast<uint64_t*>(sm + P_OFF_BAR);
-    uint64_t* bar_s = bar_kq + 1;
+    float* Af = reinterpret_cast<float*>(sm + P_AF);
+    float* Tf = reinterpret_cast<float*>(sm + P_TF);
+    float* gbuf = reinterpret_cast<float*>(sm + P_GATE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P_BAR);   // ld, s, wu, f
     __shared__ uint32_t s_tmem;
+    constexpr bool PD = GATE == kGatePerDim;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, T = p.T;
     const int bh = blockIdx.x / p.nchunks, nl = blockIdx.x % p.nchunks;
     const int b = bh / H, h = bh % H;
     const int n = p.chunk0 + nl;
-    uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * p.ws_chunk;
+    uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * IMG_BYTES;
+    const uint32_t sb = smem_u32(sm);
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int failed = 0;
+    auto wait = [&](int i, uint32_t parity) {
+        if (!mbar_wait(&bars[i], parity, &failed)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+    };
+
+    float* sBeta = gbuf + 192;
+    // per-dimension gate scratch
+    float* Gs = reinterpret_cast<float*>(sm + P_AF);   // G [64][LDG], dead before A is written
+    float* sM = reinterpret_cast<float*>(sm + X_SMALL);
+    float* sC = sM + 128;
+    float* sEm = sC + 128;
+    float* sEcm = sEm + 128;
+    int* sFlag = reinterpret_cast<int*>(sEcm + 128);
 
     if (tid == 0) {
-        mbar_init(bar_kq, 1);
-        mbar_init(bar_s, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar_kq, 4 * 8192);
+        if constexpr (PD) *sFlag = 0;
+        mbar_arrive_expect_tx(&bars[0], (PD ? 8 : 6) * 8192);
         for (int blk = 0; blk < 2; ++blk) {
-            tma_load_3d(sm + P_OFF_KQ + blk * 16384, &maps.k, bar_kq, h * D + 64 * blk, n * C, b);
-            tma_load_3d(sm + P_OFF_KQ + blk * 16384 + 8192, &maps.q, bar_kq, h * D + 64 * blk, n * C, b);
+            tma_load_3d(sm + P_KQ + blk * 16384, &maps.k, &bars[0], h * D + 64 * blk, n * C, b);
+            tma_load_3d(sm + P_KQ + blk * 16384 + 8192, &maps.q, &bars[0], h * D + 64 * blk, n * C, b);
+            tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[0], h * D + 64 * blk, n * C, b);
+            if constexpr (PD)
+                tma_load_3d(sm + X_G16 + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b);
         }
     }
     if (warp == 0) {
-        tmem_alloc(&s_tmem, 64);
+        tmem_alloc(&s_tmem, 512);
         tmem_relinquish();
     }
     if (tid < 64) {
@@ -286,90 +344,214 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p)
             if constexpr (GATE == kGateScalar) gv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.g)[tok]);
         }
         gbuf[tid] = gv;
-        gbuf[192 + tid] = bv;
+        sBeta[tid] = bv;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    if (warp == 0) chunk_gates<GATE>(gbuf, lane);
-    if (tid == 32) {   // S = [K; Q] K^T
-        if (mbar_wait(bar_kq, 0, &failed)) {
-            const uint32_t st = smem_u32(sm + P_OFF_KQ);
+
+    bool exact = false;
+    if constexpr (!PD) {
+        if (warp == 0) chunk_gates<GATE>(gbuf, lane);
+        if (tid == 32) {   // S = [K; Q] K^T
+            if (mbar_wait(&bars[0], 0, &failed)) {
+                const uint32_t id = idesc_bf16_f32(128, 64, false, false);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t a = sb + P_KQ + (k >> 2) * 16384 + (k & 3) * 32;
+                    mma_bf16(tmem + TM_S, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, k > 0);
+                }
+                mma_commit(&bars[1]);
+            } else {
+                atomicOr(p.status, kStatusTimeout);
+            }
+        }
+        __syncthreads();
+    } else {
+        wait(0, 0);
+        // G = in-chunk cumsum of g per dimension: thread (d, half), 32 rows each
+        {
+            const int d = tid & 127, hh = tid >> 7;
+            const uint8_t* gt = sm + X_G16 + (d >> 6) * 8192;
+            float acc = 0.f;
+#pragma unroll 8
+            for (int r = 32 * hh; r < 32 * hh + 32; ++r) {
+                acc += ld_bf16(gt, r, d & 63);
+                Gs[r * LDG + d] = acc;
+            }
+        }
+        __syncthreads();
+        {
+            const int d = tid & 127, hh = tid >> 7;
+            if (hh == 1) {
+                const float carry = Gs[31 * LDG + d];
+#pragma unroll 8
+                for (int r = 32; r < 64; ++r) Gs[r * LDG + d] += carry;
+            }
+        }
+        __syncthreads();
+        if (tid < 128) {
+            const float m = Gs[31 * LDG + tid], c = Gs[63 * LDG + tid];
+            sM[tid] = m;
+            sC[tid] = c;
+            sEm[tid] = expf(m);
+            sEcm[tid] = expf(c - m);
+            if (Gs[tid] - m >= 80.f || m - c >= 80.f) atomicOr(sFlag, 1);
+        }
+        __syncthreads();
+        exact = *sFlag != 0;
+        // one pass over the tiles: the Gram operands (in place / K_breve) and
+        // the per-element decayed copies K e^G, K e^(G_C - G), Q e^G
+#pragma unroll 1
+        for (int it = 0; it < 4; ++it) {
+            const int idx = tid + NPR * it;                 // 16-byte chunk 0..1023
+            const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+            const int d0 = blk * 64 + 8 * (j ^ (r & 7));    // logical columns of this chunk
+            const uint32_t rowoff = (uint32_t)(r * 128 + j * 16);
+            uint4 kraw = *reinterpret_cast<const uint4*>(sm + P_KQ + blk * 16384 + rowoff);
+            uint4 qraw = *reinterpret_cast<const uint4*>(sm + P_KQ + blk * 16384 + 8192 + rowoff);
+            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
+            const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
+            uint32_t kb[4], qb[4], kr[4], qg[4], kg[4], kt[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 kf = __bfloat1622float2(k2[e]);
+                const float2 qf = __bfloat1622float2(q2[e]);
+                float ef[2], er[2], eg[2], et[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int d = d0 + 2 * e + u;
+                    const float G = Gs[r * LDG + d], m = sM[d];
+                    if (!exact) {
+                        ef[u] = expf(G - m);
+                        er[u] = expf(m - G);
+                        eg[u] = sEm[d] * ef[u];     // e^G <= 1
+                        et[u] = sEcm[d] * er[u];    // e^(G_C - G) <= 1
+                    } else {
+                        ef[u] = er[u] = 0.f;
+                        eg[u] = expf(G);
+                        et[u] = expf(sC[d] - G);
+                    }
+                }
+                kb[e] = pack_bf16(kf.x * ef[0], kf.y * ef[1]);
+                qb[e] = pack_bf16(qf.x * ef[0], qf.y * ef[1]);
+                kr[e] = pack_bf16(kf.x * er[0], kf.y * er[1]);
+                qg[e] = pack_bf16(qf.x * eg[0], qf.y * eg[1]);
+                kg[e] = pack_bf16(kf.x * eg[0], kf.y * eg[1]);
+                kt[e] = pack_bf16(kf.x * et[0], kf.y * et[1]);
+            }
+            const uint32_t ioff = blk * 8192 + rowoff;
+            *reinterpret_cast<uint4*>(sm + X_QB + ioff) = make_uint4(qg[0], qg[1], qg[2], qg[3]);
+            *reinterpret_cast<uint4*>(sm + X_KG + ioff) = make_uint4(kg[0], kg[1], kg[2], kg[3]);
+            *reinterpret_cast<uint4*>(sm + P_KT + ioff) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
+            if (!exact) {
+                *reinterpret_cast<uint4*>(sm + P_KQ + blk * 16384 + rowoff) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
+                *reinterpret_cast<uint4*>(sm + P_KQ + blk * 16384 + 8192 + rowoff) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
+                *reinterpret_cast<uint4*>(sm + X_KB + ioff) = make_uint4(kr[0], kr[1], kr[2], kr[3]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (!exact && tid == 32) {   // S = [K e^(G-m); Q e^(G-m)] (K e^(m-G))^T
             const uint32_t id = idesc_bf16_f32(128, 64, false, false);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const uint32_t a = st + (k >> 2) * 16384 + (k & 3) * 32;
-                mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, k > 0);
+                const uint32_t a = sb + P_KQ + (k >> 2) * 16384 + (k & 3) * 32;
+                const uint32_t bb = sb + X_KB + (k >> 2) * 8192 + (k & 3) * 32;
+                mma_bf16(tmem + TM_S, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id, k > 0);
             }
-            mma_commit(bar_s);
-        } else {
-            atomicOr(p.status, kStatusTimeout);
+            mma_commit(&bars[1]);
         }
     }
-    __syncthreads();
-    const float* sG = gbuf;
-    const float* sGam = gbuf + 64;
-    const float* sFt = gbuf + 128;
-    const float* sBeta = gbuf + 192;
-    const float* sU = gbuf + 256;
-    const float* sW = gbuf + 320;
-    const bool fact = gbuf[384] != 0.f;
-    if (!mbar_wait(bar_s, 0, &failed)) atomicOr(p.status, kStatusTimeout);
-    __syncwarp();
-    tc_fence_after();
-    // A (fp32 scratch, rows 0..63) and P (bf16 image, rows 64..127)
+
+    // ---- A (fp32 scratch) and P (bf16, K-major [r][i]) from S
     {
         const int q4 = warp & 3, ch = warp >> 2;
         const int L = q4 * 32 + lane;
         float sv[32];
-        ld_cols<32>(tmem + ((uint32_t)(q4 * 32) << 16) + 32 * ch, sv);
-        if (L < 64) {
-            const int r = L;
-            if (fact) {
-                const float cr = sBeta[r] * sU[r];
+        if (!exact) {
+            wait(1, 0);
+            tc_fence_after();
+            if constexpr (PD) __syncthreads();   // G (aliased with A) is dead from here on
+            ld_cols<32>(tmem + TM_S + lane_off + 32 * ch, sv);
+            const float* sG = gbuf;
+            const float* sU = gbuf + 256;
+            const float* sW = gbuf + 320;
+            const bool fact = PD || gbuf[384] != 0.f;
+            if (L < 64) {
+                const int r = L;
+                if (fact) {
+                    const float cr = PD ? sBeta[r] : sBeta[r] * sU[r];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = 32 * ch + e;
-                    sv[e] = (i < r) ? cr * sW[i] * sv[e] : 0.f;
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = 32 * ch + e;
+                        sv[e] = (i < r) ? (PD ? cr : cr * sW[i]) * sv[e] : 0.f;
+                    }
+                } else {
+                    const float Gr = sG[r], br = sBeta[r];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = 32 * ch + e;
+                        sv[e] = (i < r) ? br * __expf(Gr - sG[i]) * sv[e] : 0.f;
+                    }
                 }
             } else {
-                const float Gr = sG[r], br = sBeta[r];
+                const int r = L - 64;
+                if (fact) {
+                    const float cr = PD ? 1.f : sU[r];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = 32 * ch + e;
-                    sv[e] = (i < r) ? br * __expf(Gr - sG[i]) * sv[e] : 0.f;
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = 32 * ch + e;
+                        sv[e] = (i <= r) ? (PD ? cr : cr * sW[i]) * sv[e] : 0.f;
+                    }
+                } else {
+                    const float Gr = sG[r];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = 32 * ch + e;
+                        sv[e] = (i <= r) ? __expf(Gr - sG[i]) * sv[e] : 0.f;
+                    }
                 }
             }
+        } else if constexpr (PD) {
+            // exact A and P: sum_d k_rd k_id e^(G_rd - G_id) with every exponent <= 0
+            const int r = L & 63;
+            const bool isq = L >= 64;
+            const uint8_t* rowt = sm + P_KQ + (isq ? 8192 : 0);
+#pragma unroll 1
+            for (int e = 0; e < 32; ++e) {
+                const int i = 32 * ch + e;
+                float acc = 0.f;
+                if (isq ? (i <= r) : (i < r)) {
+#pragma unroll 4
+                    for (int d = 0; d < D; ++d) {
+                        const float x = ld_bf16(rowt + (d >> 6) * 16384, r, d & 63);
+                        const float kk = ld_bf16(sm + P_KQ + (d >> 6) * 16384, i, d & 63);
+                        acc = fmaf(x * kk, expf(Gs[r * LDG + d] - Gs[i * LDG + d]), acc);
+                    }
+                }
+                sv[e] = isq ? acc : sBeta[r] * acc;
+            }
+            __syncthreads();   // G (aliased with A) is dead from here on
+        }
+        if (L < 64) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
-                *reinterpret_cast<float4*>(Af + r * LDF + 32 * ch + e) =
+                *reinterpret_cast<float4*>(Af + L * LDF + 32 * ch + e) =
                     make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
         } else {
-            const int r = L - 64;
-            if (fact) {
-                const float cr = sU[r];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = 32 * ch + e;
-                    sv[e] = (i <= r) ? cr * sW[i] * sv[e] : 0.f;
-                }
-            } else {
-                const float Gr = sG[r];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = 32 * ch + e;
-                    sv[e] = (i <= r) ? __expf(Gr - sG[i]) * sv[e] : 0.f;
-                }
-            }
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) st_row_chunk(img + WS_P, r, 4 * ch + jj, sv + 8 * jj, 1.f);
+            for (int jj = 0; jj < 4; ++jj) st_row_chunk(sm + P_P, L - 64, 4 * ch + jj, sv + 8 * jj, 1.f);
         }
     }
     __syncthreads();
     forward_substitution(Af, Tf, tid);
-    // T diag(beta) and T diag(beta e^G) as bf16 images, K-major [r][i]
+    // T diag(beta) and T diag(beta e^G) as bf16 K-major [r][i]
     {
+        const float* sGam = gbuf + 64;
         const int r = tid >> 2, j0 = 2 * (tid & 3);
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
@@ -382,653 +564,108 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p)
             for (int e = 0; e < 8; ++e) {
                 const int i = 8 * j + e;
                 tu[e] = (i <= r) ? tv[e] * sBeta[i] : 0.f;
-                tw[e] = tu[e] * sGam[i];
+                tw[e] = PD ? tu[e] : tu[e] * sGam[i];
             }
-            st_row_chunk(img + WS_TU, r, j, tu, 1.f);
-            st_row_chunk(img + WS_TW, r, j, tw, 1.f);
+            st_row_chunk(sm + P_TU, r, j, tu, 1.f);
+            st_row_chunk(sm + P_TW, r, j, tw, 1.f);
         }
     }
-    if (tid < 64) {
-        float* fac = reinterpret_cast<float*>(img + WS_FAC);
-        fac[tid] = sGam[tid];
-        fac[64 + tid] = sFt[tid];
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 64);
-    }
-}
-
-// ------------------------------------------------------------------ per-dim
-// Workspace image of one per-dimension-gated chunk: the scalar layout
-// (T diag(beta) in both T slots, P, factors = e^(G_C) per key dimension),
-// followed by the chain's three per-element-scaled operand tiles.
-constexpr uint32_t WS_QB = WS_CHUNK;             // Q (.) e^G            [Q_b0 | Q_b1]
-constexpr uint32_t WS_KG = WS_QB + 16384;        // K (.) e^G            [K_b0 | K_b1]
-constexpr uint32_t WS_KT = WS_KG + 16384;        // K (.) e^(G_C - G)    [K_b0 | K_b1]
-constexpr uint32_t WS_CHUNK_PD = WS_KT + 16384;
-
-struct PrepPdMaps {
-    CUtensorMap q, k, g;
-};
-
-// Per-dim prep shared memory (bytes from a 1 KB-aligned base).
-constexpr int LDG = 132;                                  // fp32 row stride of G [64][128]
-constexpr uint32_t D_OFF_KQ = 0;                          // [K_b0 | Q_b0 | K_b1 | Q_b1] -> scaled in place
-constexpr uint32_t D_OFF_G16 = 32768;                     // g tile bf16 [g_b0 | g_b1]
-constexpr uint32_t D_OFF_KB = 49152;                      // K_breve [K_b0 | K_b1], K-major rows i
-constexpr uint32_t D_OFF_AF = 65536;                      // A fp32 [64][LDF]; G fp32 before it
-constexpr uint32_t D_OFF_TF = D_OFF_AF + 64 * LDF * 4;    // T fp32 [64][LDF]
-constexpr uint32_t D_OFF_SMALL = D_OFF_TF + 64 * LDF * 4; // beta[64], m[128], c[128], flag
-constexpr uint32_t D_OFF_BAR = D_OFF_SMALL + (64 + 4 * 128 + 4) * 4;
-constexpr uint32_t D_SMEM = D_OFF_BAR + 16 + 1024;
-static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A/T scratch");
-
-// One CTA per chunk of the wave (per-dimension gate).  With G the in-chunk
-// cumsum of g per key dimension, m = G_31 and c = G_63 per dimension:
-//   S = [K e^(G-m); Q e^(G-m)] (K e^(m-G))^T  -> A = StrictTril(beta S_kk),
-//   P = Tril(S_qk); both factors and their reciprocals stay normal fp32 while
-//   every dimension decays by less than e^80 in each half of the chunk, else
-//   A and P are formed exactly on CUDA cores.  The chain's operands Q e^G, K e^G and K e^(G_C - G) go to the
-//   workspace as shared-memory images; T diag(beta) fills both T slots (the
-//   decay sits on K e^G for W).
-__global__ void __launch_bounds__(NPR)
-chunk_prep_pd_kernel(const __grid_constant__ PrepPdMaps maps, const ChunkParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-    float* Af = reinterpret_cast<float*>(sm + D_OFF_AF);
-    float* Tf = reinterpret_cast<float*>(sm + D_OFF_TF);
-    float* Gs = reinterpret_cast<float*>(sm + D_OFF_AF);   // G, dead before A is written
-    float* sBeta = reinterpret_cast<float*>(sm + D_OFF_SMALL);
-    float* sM = sBeta + 64;
-    float* sC = sM + 128;
-    float* sEm = sC + 128;
-    float* sEcm = sEm + 128;
-    int* sFlag = reinterpret_cast<int*>(sEcm + 128);
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + D_OFF_BAR);
-    uint64_t* bar_s = bar_ld + 1;
-    __shared__ uint32_t s_tmem;
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = p.H, T = p.T;
-    const int bh = blockIdx.x / p.nchunks, nl = blockIdx.x % p.nchunks;
-    const int b = bh / H, h = bh % H;
-    const int n = p.chunk0 + nl;
-    uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * p.ws_chunk;
-    int failed = 0;
-
-    if (tid == 0) {
-        mbar_init(bar_ld, 1);
-        mbar_init(bar_s, 1);
-        fence_mbar_init();
-        *sFlag = 0;
-        mbar_arrive_expect_tx(bar_ld, 6 * 8192);
-        for (int blk = 0; blk < 2; ++blk) {
-            tma_load_3d(sm + D_OFF_KQ + blk * 16384, &maps.k, bar_ld, h * D + 64 * blk, n * C, b);
-            tma_load_3d(sm + D_OFF_KQ + blk * 16384 + 8192, &maps.q, bar_ld, h * D + 64 * blk, n * C, b);
-            tma_load_3d(sm + D_OFF_G16 + blk * 8192, &maps.g, bar_ld, h * D + 64 * blk, n * C, b);
-        }
-    }
-    if (warp == 0) {
-        tmem_alloc(&s_tmem, 64);
-        tmem_relinquish();
-    }
-    if (tid < 64) {
-        const int t = n * C + tid;
-        sBeta[tid] = (t < T) ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.beta)[((size_t)b * T + t) * H + h]) : 0.f;
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    if (!mbar_wait(bar_ld, 0, &failed)) atomicOr(p.status, kStatusTimeout);
-    __syncwarp();
-    // ---- G = in-chunk cumsum of g per dimension: thread (d, half), 32 rows each
-    {
-        const int d = tid & 127, hh = tid >> 7;
-        const uint8_t* gt = sm + D_OFF_G16 + (d >> 6) * 8192;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int r = 32 * hh; r < 32 * hh + 32; ++r) {
-            acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(gt + sw128_offset(r, d & 63)));
-            Gs[r * LDG + d] = acc;
-        }
-    }
-    __syncthreads();
-    {
-        const int d = tid & 127, hh = tid >> 7;
-        if (hh == 1) {
-            const float carry = Gs[31 * LDG + d];
-#pragma unroll 8
-            for (int r = 32; r < 64; ++r) Gs[r * LDG + d] += carry;
-        }
-    }
-    __syncthreads();
-    if (tid < 128) {
-        const float m = Gs[31 * LDG + tid], c = Gs[63 * LDG + tid];
-        sM[tid] = m;
-        sC[tid] = c;
-        sEm[tid] = expf(m);
-        sEcm[tid] = expf(c - m);
-        if (Gs[tid] - m >= 80.f || m - c >= 80.f) atomicOr(sFlag, 1);
-    }
-    __syncthreads();
-    const bool exact = *sFlag != 0;
-    // ---- one pass over the tiles: Gram operands in place / K_breve, chain images
-#pragma unroll 1
-    for (int it = 0; it < 4; ++it) {
-        const int idx = tid + NPR * it;                 // 16-byte chunk 0..1023
-        const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
-        const int d0 = blk * 64 + 8 * (j ^ (r & 7));    // logical columns of this chunk
-        const uint32_t rowoff = (uint32_t)(r * 128 + j * 16);
-        uint4 kraw = *reinterpret_cast<const uint4*>(sm + D_OFF_KQ + blk * 16384 + rowoff);
-        uint4 qraw = *reinterpret_cast<const uint4*>(sm + D_OFF_KQ + blk * 16384 + 8192 + rowoff);
-        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
-        const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
-        uint32_t kb[4], qb[4], kr[4], qg[4], kg[4], kt[4];
+    if constexpr (!PD) {   // K~ = diag(e^(G_C - G_i)) K
+        const float* sFt = gbuf + 128;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 kf = __bfloat1622float2(k2[e]);
-            const float2 qf = __bfloat1622float2(q2[e]);
-            float ef[2], er[2], eg[2], et[2];
+        for (int it = 0; it < 4; ++it) {
+            const int idx = tid + NPR * it;                 // 16-byte chunk 0..1023
+            const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+            uint4 raw = *reinterpret_cast<const uint4*>(sm + P_KQ + blk * 16384 + r * 128 + j * 16);
+            const float f = sFt[r];
+            __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+            uint4 outv;
+            uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int d = d0 + 2 * e + u;
-                const float G = Gs[r * LDG + d], m = sM[d];
-                if (!exact) {
-                    ef[u] = expf(G - m);
-                    er[u] = expf(m - G);
-                    eg[u] = sEm[d] * ef[u];     // e^G <= 1
-                    et[u] = sEcm[d] * er[u];    // e^(G_C - G) <= 1
-                } else {
-                    ef[u] = er[u] = 0.f;
-                    eg[u] = expf(G);
-                    et[u] = expf(sC[d] - G);
-                }
+            for (int e = 0; e < 4; ++e) {
+                const float2 fv = __bfloat1622float2(e2[e]);
+                o32[e] = pack_bf16(fv.x * f, fv.y * f);
             }
-            kb[e] = pack_bf16(kf.x * ef[0], kf.y * ef[1]);
-            qb[e] = pack_bf16(qf.x * ef[0], qf.y * ef[1]);
-            kr[e] = pack_bf16(kf.x * er[0], kf.y * er[1]);
-            qg[e] = pack_bf16(qf.x * eg[0], qf.y * eg[1]);
-            kg[e] = pack_bf16(kf.x * eg[0], kf.y * eg[1]);
-            kt[e] = pack_bf16(kf.x * et[0], kf.y * et[1]);
+            *reinterpret_cast<uint4*>(sm + P_KT + blk * 8192 + r * 128 + j * 16) = outv;
         }
-        const uint32_t ioff = blk * 8192 + rowoff;
-        *reinterpret_cast<uint4*>(img + WS_QB + ioff) = make_uint4(qg[0], qg[1], qg[2], qg[3]);
-        *reinterpret_cast<uint4*>(img + WS_KG + ioff) = make_uint4(kg[0], kg[1], kg[2], kg[3]);
-        *reinterpret_cast<uint4*>(img + WS_KT + ioff) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
-        if (!exact) {
-            *reinterpret_cast<uint4*>(sm + D_OFF_KQ + blk * 16384 + rowoff) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
-            *reinterpret_cast<uint4*>(sm + D_OFF_KQ + blk * 16384 + 8192 + rowoff) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
-            *reinterpret_cast<uint4*>(sm + D_OFF_KB + ioff) = make_uint4(kr[0], kr[1], kr[2], kr[3]);
-        }
-    }
-    if (tid < 128) reinterpret_cast<float*>(img + WS_FAC)[tid] = expf(sC[tid]);
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (!exact) {
-        if (tid == 32) {   // S = [K e^(G-m); Q e^(G-m)] (K e^(m-G))^T
-            const uint32_t st = smem_u32(sm + D_OFF_KQ), kbr = smem_u32(sm + D_OFF_KB);
-            const uint32_t id = idesc_bf16_f32(128, 64, false, false);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t a = st + (k >> 2) * 16384 + (k & 3) * 32;
-                const uint32_t bb = kbr + (k >> 2) * 8192 + (k & 3) * 32;
-                mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id, k > 0);
-            }
-            mma_commit(bar_s);
-        }
-        if (!mbar_wait(bar_s, 0, &failed)) atomicOr(p.status, kStatusTimeout);
-        __syncwarp();
-        tc_fence_after();
-        __syncthreads();   // G (aliased with A) is dead from here on
-        const int q4 = warp & 3, ch = warp >> 2;
-        const int L = q4 * 32 + lane;
-        float sv[32];
-        ld_cols<32>(tmem + ((uint32_t)(q4 * 32) << 16) + 32 * ch, sv);
-        if (L < 64) {
-            const int r = L;
-            const float br = sBeta[r];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sv[e] = (32 * ch + e < r) ? br * sv[e] : 0.f;
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-                *reinterpret_cast<float4*>(Af + r * LDF + 32 * ch + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
-        } else {
-            const int r = L - 64;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sv[e] = (32 * ch + e <= r) ? sv[e] : 0.f;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) st_row_chunk(img + WS_P, r, 4 * ch + jj, sv + 8 * jj, 1.f);
-        }
-    } else {
-        // exact A and P: sum_d k_rd k_id e^(G_rd - G_id) with every exponent <= 0;
-        // A goes to registers first since it shares space with G
-        const int q4 = warp & 3, ch = warp >> 2;
-        const int L = q4 * 32 + lane;
-        const int r = L & 63;
-        const bool isq = L >= 64;
-        const uint8_t* rowt = sm + D_OFF_KQ + (isq ? 8192 : 0);
-        float sv[32];
-#pragma unroll 1
-        for (int e = 0; e < 32; ++e) {
-            const int i = 32 * ch + e;
-            float acc = 0.f;
-            if (isq ? (i <= r) : (i < r)) {
-#pragma unroll 4
-                for (int d = 0; d < D; ++d) {
-                    const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                        rowt + (d >> 6) * 16384 + sw128_offset(r, d & 63)));
-                    const float kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                        sm + D_OFF_KQ + (d >> 6) * 16384 + sw128_offset(i, d & 63)));
-                    acc = fmaf(x * kk, expf(Gs[r * LDG + d] - Gs[i * LDG + d]), acc);
-                }
-            }
-            sv[e] = isq ? acc : sBeta[r] * acc;
-        }
-        __syncthreads();   // G (aliased with A) is dead from here on
-        if (!isq) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-                *reinterpret_cast<float4*>(Af + r * LDF + 32 * ch + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) st_row_chunk(img + WS_P, r, 4 * ch + jj, sv + 8 * jj, 1.f);
-        }
-    }
-    __syncthreads();
-    forward_substitution(Af, Tf, tid);
-    {
-        const int r = tid >> 2, j0 = 2 * (tid & 3);
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-            const int j = j0 + jj;
-            const float4 t0 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j);
-            const float4 t1 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j + 4);
-            const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-            float tu[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int i = 8 * j + e;
-                tu[e] = (i <= r) ? tv[e] * sBeta[i] : 0.f;
-            }
-            st_row_chunk(img + WS_TU, r, j, tu, 1.f);
-            st_row_chunk(img + WS_TW, r, j, tu, 1.f);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 64);
-    }
-}
-
-// Chain kernel shared memory (bytes from a 1 KB-aligned base).
-constexpr uint32_t KQ_STAGE = 32768;   // [K_b0 | Q_b0 | K_b1 | Q_b1], 8 KB each, K-major
-constexpr uint32_t OFF_KQ = 0;         // 2 stages
-constexpr uint32_t OFF_V = 65536;      // 2 buffers of [V_b0 | V_b1]
-constexpr uint32_t OFF_TU = 98304;     // T diag(beta)          } [T_u; Z] and
-constexpr uint32_t OFF_Z = 106496;     // zero block            } [Z; T_w] are
-constexpr uint32_t OFF_TW = 114688;    // T diag(beta e^G)      } 128-row stacks
-constexpr uint32_t OFF_Z2 = 122880;    // zero block            } [Z2; P]
-constexpr uint32_t OFF_P = 131072;     // P, K-major [64 r][64 i]
-constexpr uint32_t OFF_WQ = 139264;    // [-W_b0 | Qbar_b0 | -W_b1 | Qbar_b1], K-major
-constexpr uint32_t OFF_HB = 172032;    // h (bf16) MN-major [d][64 v] x 2; after the
-constexpr uint32_t OFF_DL = 172032;    //   c-MMA: D [i][64 v] x 2 (first 16 KB)
-constexpr uint32_t OFF_KT = 204800;    // K~ = diag(e^(G_C - G_i)) K, [K~_b0 | K~_b1]
-constexpr uint32_t OFF_FAC = 221184;   // 2 x {e^G [64], e^(G_C - G) [64]}
-constexpr uint32_t OFF_BAR = OFF_FAC + 2 * 128 * 4;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 32 * 8 + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-
-constexpr int NT = 288;          // 9 warps
-constexpr int NCH = 128;         // chain threads (warps 0-3)
-constexpr int NST = 128;         // stager threads (warps 4-7)
-
-// TMEM columns (512 allocated).
-constexpr uint32_t TM_H = 0;      // state, lanes d, 128 columns v (fp32)
-constexpr uint32_t TM_X0 = 128;   // X for even chunks, lanes r / 64 + r, 128 columns v
-constexpr uint32_t TM_X1 = 256;   // X for odd chunks
-constexpr uint32_t TM_W = 384;    // [0; W], lanes 64..127, 128 columns d
-
-enum Bar {
-    B_KQ0, B_KQ1, B_VFULL, B_TFULL, B_PFULL, B_FFULL0, B_FFULL1, B_WUDONE, B_CDONE, B_DDONE,
-    B_WQREADY, B_HBREADY, B_DREADY, B_XFREE, B_QFULL, B_FINAL, B_COUNT
-};
-
-struct TcMaps {
-    CUtensorMap q, k, v;
-};
-
-__global__ void __launch_bounds__(NT, 1)
-chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, int gated, int perdim) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-    const uint32_t sb = smem_u32(sm);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-    __shared__ uint32_t s_tmem;
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = p.H, T = p.T;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const int NC = p.nchunks;              // local chunk nl = 0..NC-1 is chunk p.chunk0 + nl
-    const uint8_t* wsh = p.ws + (size_t)bh * p.cw * p.ws_chunk;
-    int failed = 0;
-
-    if (tid == 0) {
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], 1);
-        fence_mbar_init();
-        prefetch_tmap(&maps.q);
-        prefetch_tmap(&maps.k);
-        prefetch_tmap(&maps.v);
-    }
-    if (warp == 0) {
-        tmem_alloc(&s_tmem, 512);
-        tmem_relinquish();
-    }
-    for (int i = tid; i < 1024; i += NT) {   // the two zero blocks
-        const uint32_t off = (i < 512) ? OFF_Z + 16 * i : OFF_Z2 + 16 * (i - 512);
-        *reinterpret_cast<uint4*>(sm + off) = make_uint4(0, 0, 0, 0);
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-
-    auto fac_buf = [&](int nl) { return reinterpret_cast<float*>(sm + OFF_FAC) + (nl & 1) * 128; };
-    auto wait = [&](int bar, uint32_t parity) {
-        if (!mbar_wait(&bars[bar], parity, &failed)) atomicOr(p.status, kStatusTimeout);
-        __syncwarp();
-    };
-    auto load_kq = [&](int nl) {
-        const int s = nl & 1, n = p.chunk0 + nl;
-        mbar_arrive_expect_tx(&bars[B_KQ0 + s], 4 * 8192);
-        uint8_t* st = sm + OFF_KQ + s * KQ_STAGE;
-        for (int blk = 0; blk < 2; ++blk) {
-            tma_load_3d(st + blk * 16384, &maps.k, &bars[B_KQ0 + s], h * D + 64 * blk, n * C, b);
-            tma_load_3d(st + blk * 16384 + 8192, &maps.q, &bars[B_KQ0 + s], h * D + 64 * blk, n * C, b);
-        }
-    };
-    auto load_v = [&](int nl) {
-        const int n = p.chunk0 + nl;
-        mbar_arrive_expect_tx(&bars[B_VFULL], 2 * 8192);
-        for (int blk = 0; blk < 2; ++blk)
-            tma_load_3d(sm + OFF_V + (nl & 1) * 16384 + blk * 8192, &maps.v, &bars[B_VFULL],
-                        h * D + 64 * blk, n * C, b);
-    };
-
-    if (warp == 8) {
-        // =========================== control: TMA for the first tiles and V, every MMA
-        const bool leader = lane == 0;   // issues only while no wait has failed
-        if (leader && !perdim) {
-            fence_async_smem();
-            load_kq(0);
-            if (NC > 1) load_kq(1);
-        }
-        // W and U of chunk nl: operands loaded, TMEM free (for nl >= 2 the output
-        // of chunk nl - 2 has been read out of X[nl & 1])
-        auto issue_wu = [&](int nl) {
-            const int s = nl & 1;
-            const uint32_t st = sb + OFF_KQ + s * KQ_STAGE;
-            const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
-            wait(B_TFULL, nl & 1);
-            wait(B_VFULL, nl & 1);
-            if (!perdim) wait(B_KQ0 + s, (nl >> 1) & 1);
-            if (nl >= 2) wait(B_XFREE, (nl - 2) & 1);
-            tc_fence_after();
-            if (leader && !failed) {
-                const uint32_t idw = idesc_bf16_f32(128, 128, false, true);
+    if (tid == 32 && !failed) {
+        // W^T = (K e^G)^T T_w^T (scalar gate: the decay sits in T_w), U^T = V^T T_u^T
+        const uint32_t id = idesc_bf16_f32(128, 64, true, false);
+        const uint32_t ka = PD ? sb + X_KG : sb + P_KQ;
+        const uint32_t klbo = PD ? 8192 : 16384;
 #pragma unroll
-                for (int k = 0; k < 4; ++k)   // [0; W] = [Z; T_w] K
-                    mma_bf16(tmem + TM_W, sdesc_sw128(sb + OFF_Z + k * 32, 16, 1024),
-                             sdesc_sw128(st + k * 2048, 16384, 1024), idw, k > 0);
+        for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem + TM_WT, sdesc_sw128(ka + k * 2048, klbo, 1024),
+                     sdesc_sw128(sb + P_TW + k * 32, 16, 1024), id, k > 0);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)   // X = [T_u; Z] V
-                    mma_bf16(tX, sdesc_sw128(sb + OFF_TU + k * 32, 16, 1024),
-                             sdesc_sw128(sb + OFF_V + s * 16384 + k * 2048, 8192, 1024), idw, k > 0);
-                mma_commit(&bars[B_WUDONE]);
-            }
-        };
-        if (NC > 0) issue_wu(0);
-#pragma unroll 1
-        for (int nl = 0; nl < NC; ++nl) {
-            const int s = nl & 1;
-            const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
-            wait(B_WQREADY, nl & 1);
-            wait(B_HBREADY, nl & 1);
-            tc_fence_after();
-            if (leader && !failed) {
-                const uint32_t idc = idesc_bf16_f32(128, 128, false, true);
+        for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem + TM_UT, sdesc_sw128(sb + P_V + k * 2048, 8192, 1024),
+                     sdesc_sw128(sb + P_TU + k * 32, 16, 1024), id, k > 0);
+        mma_commit(&bars[2]);
+    }
+    wait(2, 0);
+    tc_fence_after();
+    {   // [W^T; U^T] as one K-major bf16 tile of 256 rows (tokens contiguous)
+        const int row = (warp & 3) * 32 + lane;
+        float v[64];
+        ld_cols<64>(tmem + (warp < 4 ? TM_WT : TM_UT) + lane_off, v);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // X += [-W; Q_bar] h
-                    mma_bf16(tX, sdesc_sw128(sb + OFF_WQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                             sdesc_sw128(sb + OFF_HB + k * 2048, 16384, 1024), idc, true);
-                mma_commit(&bars[B_CDONE]);
-            }
-            // the next chunk's W / U run while the chain turns D of this one
-            if (nl + 1 < NC) issue_wu(nl + 1);
-            wait(B_DREADY, nl & 1);
-            wait(B_PFULL, nl & 1);
-            tc_fence_after();
-            if (leader && !failed) {
-                const uint32_t id2 = idesc_bf16_f32(128, 128, true, true);
+        for (int j = 0; j < 8; ++j) st_row_chunk(sm + P_WUT, (warp < 4 ? 0 : 128) + row, j, v + 8 * j, 1.f);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 32 && !failed) {
+        const uint32_t id1 = idesc_bf16_f32(128, 256, true, false);   // K~^T [W | U]
 #pragma unroll
-                for (int k = 0; k < 4; ++k)   // state += K~^T D
-                    mma_bf16(tmem + TM_H, sdesc_sw128(sb + OFF_KT + k * 2048, 8192, 1024),
-                             sdesc_sw128(sb + OFF_DL + k * 2048, 8192, 1024), id2, true);
-                const uint32_t id1 = idesc_bf16_f32(128, 128, false, true);
+        for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem + TM_FP, sdesc_sw128(sb + P_KT + k * 2048, 8192, 1024),
+                     sdesc_sw128(sb + P_WUT + k * 32, 16, 1024), id1, k > 0);
+        const uint32_t id2 = idesc_bf16_f32(64, 256, false, false);   // P [W | U]
 #pragma unroll
-                for (int k = 0; k < 4; ++k)   // X += [Z2; P] D
-                    mma_bf16(tX, sdesc_sw128(sb + OFF_Z2 + k * 32, 16, 1024),
-                             sdesc_sw128(sb + OFF_DL + k * 2048, 8192, 1024), id1, true);
-                mma_commit(&bars[B_DDONE]);
-            }
-        }
-        // nothing issued by this warp may still run when TMEM is released
-        if (leader) mma_commit(&bars[B_FINAL]);
-        int final_failed = 0;
-        if (!mbar_wait(&bars[B_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
-        __syncwarp();
-    } else if (warp >= 4) {
-        // =========================== stager: prep images in, -W and Q_bar operands
-        const int st_id = tid - NCH;                // 0..127
-        const int L = (warp & 3) * 32 + lane;       // TMEM lane of this thread
-#pragma unroll 1
-        for (int nl = 0; nl < NC; ++nl) {
-            const int s = nl & 1;
-            const uint8_t* img = wsh + (size_t)nl * p.ws_chunk;
-            if (st_id == 0) {   // W/U of chunk nl-1 are done with T_u / T_w, and the chain is
-                                // done with the factors of chunk nl-2 (both waited below)
-                mbar_arrive_expect_tx(&bars[B_TFULL], perdim ? 4 * 8192 : 2 * 8192);
-                bulk_load(sm + OFF_TU, img + WS_TU, 8192, &bars[B_TFULL]);
-                bulk_load(sm + OFF_TW, img + WS_TW, 8192, &bars[B_TFULL]);
-                if (perdim) {   // K e^G into the K slots of stage nl & 1 (W of chunk nl-2 is done)
-                    uint8_t* stg = sm + OFF_KQ + s * KQ_STAGE;
-                    bulk_load(stg, img + WS_KG, 8192, &bars[B_TFULL]);
-                    bulk_load(stg + 16384, img + WS_KG + 8192, 8192, &bars[B_TFULL]);
+        for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem + TM_PP, sdesc_sw128(sb + P_P + k * 32, 16, 1024),
+                     sdesc_sw128(sb + P_WUT + k * 32, 16, 1024), id2, k > 0);
+        mma_commit(&bars[3]);
+    }
+    wait(3, 0);
+    tc_fence_after();
+    {   // Phi = -K~^T W (warps 0-3) and Psi = K~^T U (warps 4-7), row d = lane
+        const int d = (warp & 3) * 32 + lane;
+        float v[128];
+        ld_cols<128>(tmem + TM_FP + lane_off + (warp < 4 ? 0 : 128), v);
+        if (!failed) st_row128(img + (warp < 4 ? IMG_PHI : IMG_PSI), 16384, d, v, warp < 4 ? -1.f : 1.f);
+    }
+    {   // Qp = Q e^G - P W (warps 0-3) and P U (warps 4-7); row r = 16 (warp & 3) + lane
+        float v[128];
+        ld_cols<128>(tmem + TM_PP + lane_off + (warp < 4 ? 0 : 128), v);
+        const int r = 16 * (warp & 3) + lane;
+        if (lane < 16 && !failed) {
+            if (warp < 4) {
+                const float eg = gbuf[64 + r];
+#pragma unroll
+                for (int dd = 0; dd < D; ++dd) {
+                    const float qb = PD ? ld_bf16(sm + X_QB + (dd >> 6) * 8192, r, dd & 63)
+                                        : eg * ld_bf16(sm + P_KQ + (dd >> 6) * 16384 + 8192, r, dd & 63);
+                    v[dd] = qb - v[dd];
                 }
-                mbar_arrive_expect_tx(&bars[B_FFULL0 + s], 512);
-                bulk_load(fac_buf(nl), img + WS_FAC, 512, &bars[B_FFULL0 + s]);
-                fence_async_smem();
-                load_v(nl);   // V buffer nl & 1: U of chunk nl-2 is long done
-            }
-            // Q_bar = diag(e^G) Q into the Q rows of WQ (same swizzled layout) once the
-            // c-product of chunk nl-1 is done with WQ, and K~ = diag(e^(G_C - G)) K
-            // once the state update of chunk nl-1 is done with K~
-            if (nl > 0) wait(B_CDONE, (nl - 1) & 1);
-            wait(B_FFULL0 + s, (nl >> 1) & 1);
-            if (!perdim) wait(B_KQ0 + s, (nl >> 1) & 1);
-            const float* fac = fac_buf(nl);
-            const uint8_t* stage = sm + OFF_KQ + s * KQ_STAGE;
-            auto scale_rows = [&](uint32_t src_off, uint8_t* dst, const float* rowf) {
-#pragma unroll
-                for (int it = 0; it < 8; ++it) {
-                    const int idx = st_id + NST * it;          // 16-byte chunk 0..1023
-                    const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
-                    uint4 raw = *reinterpret_cast<const uint4*>(stage + blk * 16384 + src_off + r * 128 + j * 16);
-                    const float gmul = rowf[r];
-                    __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
-                    uint4 outv;
-                    uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(e2[e]);
-                        o32[e] = pack_bf16(f.x * gmul, f.y * gmul);
-                    }
-                    *reinterpret_cast<uint4*>(dst + blk * (dst == sm + OFF_KT ? 8192 : 16384) + r * 128 + j * 16) = outv;
-                }
-            };
-            if (!perdim) {
-                scale_rows(8192, sm + OFF_WQ + 8192, fac);   // Q rows -> Q_bar rows of WQ
-            } else if (st_id == 0) {                         // Q e^G image -> Q_bar rows of WQ
-                mbar_arrive_expect_tx(&bars[B_QFULL], 2 * 8192);
-                bulk_load(sm + OFF_WQ + 8192, img + WS_QB, 8192, &bars[B_QFULL]);
-                bulk_load(sm + OFF_WQ + 8192 + 16384, img + WS_QB + 8192, 8192, &bars[B_QFULL]);
-            }
-            // -W (TMEM lanes 64..127, warps 6-7) -> the W rows of WQ
-            wait(B_WUDONE, nl & 1);
-            tc_fence_after();
-            if (L >= 64) {
-                const int r = L - 64;
-                float wv[128];
-                ld_cols<128>(tmem + TM_W + lane_off, wv);
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    st_row_chunk(sm + OFF_WQ + (j >> 3) * 16384, r, j & 7, wv + 8 * j, -1.f);
-            }
-            if (perdim) wait(B_QFULL, nl & 1);
-            fence_async_smem();
-            tc_fence_before();
-            named_bar(3, NST);
-            if (st_id == 0) mbar_arrive(&bars[B_WQREADY]);
-            // P and K~ of chunk nl once the d-products of chunk nl-1 are done with them
-            if (nl > 0) wait(B_DDONE, (nl - 1) & 1);
-            if (!perdim) {
-                scale_rows(0, sm + OFF_KT, fac + 64);      // K rows -> K~
-                fence_async_smem();
-                named_bar(3, NST);
-            }
-            if (st_id == 0) {
-                mbar_arrive_expect_tx(&bars[B_PFULL], perdim ? 3 * 8192 : 8192);
-                bulk_load(sm + OFF_P, img + WS_P, 8192, &bars[B_PFULL]);
-                if (perdim) bulk_load(sm + OFF_KT, img + WS_KT, 16384, &bars[B_PFULL]);
-            }
-        }
-    } else {
-        // =========================== chain: state, D, output
-        {
-            const float* s0 = p.s0 ? p.s0 + ((size_t)bh * D + tid) * D : nullptr;
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                float v[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] = s0 ? s0[c0 + j] : 0.f;
-                tmem_st16(tmem + TM_H + lane_off + c0, v);
-            }
-            tmem_wait_st();
-        }
-        auto out_epilogue = [&](int ml) {   // chunk ml's O, warps 2-3 (TMEM lanes 64..127)
-            const int r = tid - 64, t0 = (p.chunk0 + ml) * C;
-            const int nval = min(C, T - t0);
-            const uint32_t tX = tmem + ((ml & 1) ? TM_X1 : TM_X0);
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + (((size_t)b * T + t0 + r) * H + h) * D;
-            float ov[128];
-            ld_cols<128>(tX + lane_off, ov);
-            if (r < nval) {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    uint4 w;
-                    w.x = pack_bf16(ov[8 * j + 0], ov[8 * j + 1]);
-                    w.y = pack_bf16(ov[8 * j + 2], ov[8 * j + 3]);
-                    w.z = pack_bf16(ov[8 * j + 4], ov[8 * j + 5]);
-                    w.w = pack_bf16(ov[8 * j + 6], ov[8 * j + 7]);
-                    *reinterpret_cast<uint4*>(orow + 8 * j) = w;
-                }
-            }
-        };
-#pragma unroll 1
-        for (int nl = 0; nl < NC; ++nl) {
-            const int s = nl & 1;
-            if (nl > 0) {
-                wait(B_DDONE, (nl - 1) & 1);
-                tc_fence_after();
-                if (tid == 0 && nl + 1 < NC && !perdim) {
-                    fence_async_smem();
-                    load_kq(nl + 1);
-                }
-            }
-            // state -> bf16 operand h (MN-major [d][64 v] x 2), row d = tid
-            {
-                float hv[128];
-                ld_cols<128>(tmem + TM_H + lane_off, hv);
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    st_row_chunk(sm + OFF_HB + (j >> 3) * 16384, tid, j & 7, hv + 8 * j, 1.f);
-            }
-            fence_async_smem();
-            named_bar(1, NCH);
-            if (tid == 0) mbar_arrive(&bars[B_HBREADY]);
-            // state *= e^(G_C) (before the state update of this chunk)
-            wait(B_FFULL0 + s, (nl >> 1) & 1);
-            const float* fac = fac_buf(nl);
-            if (gated) {
-                const float gam = perdim ? fac[tid] : fac[63];
-                float hv[128];
-                ld_cols<128>(tmem + TM_H + lane_off, hv);
-#pragma unroll
-                for (int e = 0; e < 128; ++e) hv[e] *= gam;
-                st_cols<128>(tmem + TM_H + lane_off, hv);
-                tmem_wait_st();
-            }
-            tc_fence_before();
-            named_bar(1, NCH);
-            if (warp >= 2) {
-                if (nl > 0) {
-                    out_epilogue(nl - 1);
-                    tc_fence_before();
-                    named_bar(4, 64);
-                    if (tid == 64) mbar_arrive(&bars[B_XFREE]);   // X[(nl - 1) & 1] is free
-                }
+                st_row128(img + IMG_QP, 8192, r, v, 1.f);
             } else {
-                wait(B_CDONE, nl & 1);
-                tc_fence_after();
-                const uint32_t tX = tmem + (s ? TM_X1 : TM_X0);
-                float dv[128];
-                ld_cols<128>(tX + lane_off, dv);
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    st_row_chunk(sm + OFF_DL + (j >> 3) * 8192, tid, j & 7, dv + 8 * j, 1.f);
-            }
-            fence_async_smem();
-            tc_fence_before();
-            named_bar(1, NCH);
-            if (tid == 0) mbar_arrive(&bars[B_DREADY]);
-        }
-        if (NC > 0) {
-            wait(B_DDONE, (NC - 1) & 1);
-            tc_fence_after();
-            if (warp >= 2) out_epilogue(NC - 1);
-            if (!failed && p.s_out) {
-                float* dst = p.s_out + ((size_t)bh * D + tid) * D;
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float hv[64];
-                    ld_cols<64>(tmem + TM_H + lane_off + 64 * half, hv);
-#pragma unroll
-                    for (int e = 0; e < 64; e += 4)
-                        *reinterpret_cast<float4*>(dst + 64 * half + e) = make_float4(hv[e], hv[e + 1], hv[e + 2], hv[e + 3]);
-                }
+                st_row128(img + IMG_PU, 8192, r, v, 1.f);
             }
         }
+    }
+    if (tid < 128 && !failed) {
+        float gam;
+        if constexpr (PD) gam = expf(sC[tid]);
+        else gam = gbuf[64 + 63];
+        reinterpret_cast<float*>(img + IMG_GAM)[tid] = gam;
     }
     tc_fence_before();
     __syncthreads();
@@ -1038,22 +675,265 @@ chunk_fwd_tc_kernel(const __grid_constant__ TcMaps maps, const ChunkParams p, in
     }
 }
 
-bool make_maps(const ChunkParams& p, TcMaps* m) {
+// ------------------------------------------------------------------ chain
+// Chain kernel shared memory (bytes from a 1 KB-aligned base).
+constexpr uint32_t CH_PHI = 0;          // 2 slots of Phi   (32 KB each)
+constexpr uint32_t CH_PSI = 65536;      // 2 slots of Psi   (32 KB each)
+constexpr uint32_t CH_QP = 131072;      // Qp   (16 KB)
+constexpr uint32_t CH_PU = 147456;      // P U  (16 KB)
+constexpr uint32_t CH_HB = 163840;      // 2 slots of h (bf16) MN-major [d][64 v] x 2 blocks
+constexpr uint32_t CH_GAM = 229376;     // 2 slots of gamma (512 B each)
+constexpr uint32_t CH_BAR = 230400;
+constexpr uint32_t CH_SMEM = CH_BAR + 32 * 8 + 1024;
+static_assert(CH_SMEM <= 232448, "chain shared memory");
+
+constexpr int CH_THREADS = 448;   // 14 warps: loader, MMA, 4 output, 8 state
+constexpr int NHP = 256;          // state-pass threads (warps 6-13)
+
+// TMEM columns of the chain kernel (256 allocated).
+constexpr uint32_t TM_H = 0;      // state, lanes d, 128 columns v (fp32)
+constexpr uint32_t TM_O = 128;    // O^T, lanes v, 2 slots of 64 columns r
+
+enum ChainBar {
+    CB_PHI0, CB_PHI1, CB_PSI0, CB_PSI1, CB_QP, CB_PU, CB_HREADY, CB_SDONE, CB_SFREE0, CB_SFREE1,
+    CB_PSIFREE0, CB_PSIFREE1, CB_ODONE, CB_OFREE0, CB_OFREE1, CB_FINAL, CB_COUNT
+};
+
+// One CTA per (batch, head): walks the wave's chunks in order.  Chunk n's
+// image slot is n & 1; every barrier that a role waits on completes at most
+// once ahead of that wait, so the parity waits never fall two phases behind.
+__global__ void __launch_bounds__(CH_THREADS, 1)
+chunk_chain_kernel(const ChunkParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CH_BAR);
+    __shared__ uint32_t s_tmem;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.H, T = p.T;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int NC = p.nchunks;
+    const uint8_t* wsh = p.ws + (size_t)bh * p.cw * IMG_BYTES;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int failed = 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < CB_COUNT; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    auto wait = [&](int bar, uint32_t parity) {
+        if (!mbar_wait(&bars[bar], parity, &failed)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+    };
+    auto img = [&](int nl) { return wsh + (size_t)nl * IMG_BYTES; };
+
+    if (warp == 0) {
+        // =========================== loader: Phi + gamma and Psi of every chunk
+        if (lane == 0) {
+#pragma unroll 1
+            for (int nl = 0; nl < NC; ++nl) {
+                const int s = nl & 1;
+                if (nl >= 2) {
+                    if (!mbar_wait(&bars[CB_SFREE0 + s], ((nl - 2) >> 1) & 1, &failed)) break;
+                }
+                mbar_arrive_expect_tx(&bars[CB_PHI0 + s], 32768 + 512);
+                bulk_load(sm + CH_PHI + s * 32768, img(nl) + IMG_PHI, 32768, &bars[CB_PHI0 + s]);
+                bulk_load(sm + CH_GAM + s * 512, img(nl) + IMG_GAM, 512, &bars[CB_PHI0 + s]);
+                if (nl >= 2) {
+                    if (!mbar_wait(&bars[CB_PSIFREE0 + s], ((nl - 2) >> 1) & 1, &failed)) break;
+                }
+                mbar_arrive_expect_tx(&bars[CB_PSI0 + s], 32768);
+                bulk_load(sm + CH_PSI + s * 32768, img(nl) + IMG_PSI, 32768, &bars[CB_PSI0 + s]);
+            }
+            if (failed) atomicOr(p.status, kStatusTimeout);
+        }
+    } else if (warp == 1) {
+        // =========================== MMA issuer
+        const bool leader = lane == 0;
+        const uint32_t ids = idesc_bf16_f32(128, 128, false, true);   // h += Phi h_bf16
+        const uint32_t ido = idesc_bf16_f32(128, 64, true, false);    // O^T = h^T Qp^T
+#pragma unroll 1
+        for (int nl = 0; nl < NC; ++nl) {
+            const int s = nl & 1;
+            const uint32_t hb = sb + CH_HB + s * 32768;
+            wait(CB_HREADY, nl & 1);
+            wait(CB_PHI0 + s, (nl >> 1) & 1);
+            tc_fence_after();
+            if (leader && !failed) {
+                const uint32_t phi = sb + CH_PHI + s * 32768;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16(tmem + TM_H, sdesc_sw128(phi + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                             sdesc_sw128(hb + k * 2048, 16384, 1024), ids, true);
+                mma_commit(&bars[CB_SDONE]);
+                mma_commit(&bars[CB_SFREE0 + s]);
+            }
+            wait(CB_QP, nl & 1);
+            if (nl >= 2) wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
+            tc_fence_after();
+            if (leader && !failed) {
+                const uint32_t qp = sb + CH_QP;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16(tmem + TM_O + 64 * s, sdesc_sw128(hb + k * 2048, 16384, 1024),
+                             sdesc_sw128(qp + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ido, k > 0);
+                mma_commit(&bars[CB_ODONE]);
+            }
+        }
+        // nothing issued by this warp may still run when TMEM is released
+        if (leader) mma_commit(&bars[CB_FINAL]);
+        int final_failed = 0;
+        if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+    } else if (warp < 6) {
+        // =========================== output: O = (O^T)^T + P U, bf16 to o
+        const int v = (warp & 3) * 32 + lane;
+        const bool leader = warp == 2 && lane == 0;
+        if (leader && NC > 0) {
+            mbar_arrive_expect_tx(&bars[CB_QP], 16384);
+            bulk_load(sm + CH_QP, img(0) + IMG_QP, 16384, &bars[CB_QP]);
+            mbar_arrive_expect_tx(&bars[CB_PU], 16384);
+            bulk_load(sm + CH_PU, img(0) + IMG_PU, 16384, &bars[CB_PU]);
+        }
+#pragma unroll 1
+        for (int nl = 0; nl < NC; ++nl) {
+            const int s = nl & 1;
+            wait(CB_ODONE, nl & 1);
+            if (leader && !failed && nl + 1 < NC) {   // Qp slot is free once O of chunk nl is done
+                mbar_arrive_expect_tx(&bars[CB_QP], 16384);
+                bulk_load(sm + CH_QP, img(nl + 1) + IMG_QP, 16384, &bars[CB_QP]);
+            }
+            wait(CB_PU, nl & 1);
+            tc_fence_after();
+            float ov[64];
+            ld_cols<64>(tmem + TM_O + 64 * s + lane_off, ov);
+            const int t0 = (p.chunk0 + nl) * C;
+            const int nval = min(C, T - t0);
+            __nv_bfloat16* ocol = static_cast<__nv_bfloat16*>(p.o) + (((size_t)b * T + t0) * H + h) * D + v;
+            const uint8_t* pu = sm + CH_PU + (v >> 6) * 8192;
+            if (!failed) {
+#pragma unroll
+                for (int r = 0; r < C; ++r)
+                    if (r < nval) ocol[(size_t)r * H * D] = __float2bfloat16_rn(ov[r] + ld_bf16(pu, r, v & 63));
+            }
+            tc_fence_before();
+            named_bar(2, 128);
+            if (leader) {
+                mbar_arrive(&bars[CB_OFREE0 + s]);
+                if (!failed && nl + 1 < NC) {
+                    mbar_arrive_expect_tx(&bars[CB_PU], 16384);
+                    bulk_load(sm + CH_PU, img(nl + 1) + IMG_PU, 16384, &bars[CB_PU]);
+                }
+            }
+        }
+    } else {
+        // =========================== state pass: h + Psi -> bf16 operand, decay
+        const int d = (warp & 3) * 32 + lane;
+        const int c = (warp - 6) >> 2;              // column half
+        const bool leader = warp == 6 && lane == 0;
+        const uint32_t haddr = tmem + TM_H + lane_off + 64 * c;
+        auto add_psi = [&](int nl, float (&hv)[64]) {
+            const uint8_t* row = sm + CH_PSI + (nl & 1) * 32768 + c * 16384 + d * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint4 raw = *reinterpret_cast<const uint4*>(row + ((j ^ (d & 7)) * 16));
+                const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(e2[e]);
+                    hv[8 * j + 2 * e] += f.x;
+                    hv[8 * j + 2 * e + 1] += f.y;
+                }
+            }
+        };
+#pragma unroll 1
+        for (int nl = 0; nl < NC; ++nl) {
+            const int s = nl & 1;
+            float hv[64];
+            if (nl == 0) {
+                const float* s0 = p.s0 ? p.s0 + ((size_t)bh * D + d) * D + 64 * c : nullptr;
+#pragma unroll
+                for (int e = 0; e < 64; e += 4) {
+                    const float4 x = s0 ? *reinterpret_cast<const float4*>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    hv[e] = x.x; hv[e + 1] = x.y; hv[e + 2] = x.z; hv[e + 3] = x.w;
+                }
+            } else {
+                wait(CB_SDONE, (nl - 1) & 1);
+                wait(CB_PSI0 + ((nl - 1) & 1), ((nl - 1) >> 1) & 1);
+                tc_fence_after();
+                ld_cols<64>(haddr, hv);
+                add_psi(nl - 1, hv);
+            }
+            wait(CB_PHI0 + s, (nl >> 1) & 1);
+            const float gam = reinterpret_cast<const float*>(sm + CH_GAM + s * 512)[d];
+            uint8_t* hb = sm + CH_HB + s * 32768 + c * 16384;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) st_row_chunk(hb, d, j, hv + 8 * j, 1.f);
+#pragma unroll
+            for (int e = 0; e < 64; ++e) hv[e] *= gam;
+            st_cols<64>(haddr, hv);
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            named_bar(1, NHP);
+            if (leader) {
+                mbar_arrive(&bars[CB_HREADY]);
+                if (nl >= 1) mbar_arrive(&bars[CB_PSIFREE0 + ((nl - 1) & 1)]);
+            }
+        }
+        if (NC > 0) {   // final state = h + Psi of the last chunk
+            wait(CB_SDONE, (NC - 1) & 1);
+            wait(CB_PSI0 + ((NC - 1) & 1), ((NC - 1) >> 1) & 1);
+            tc_fence_after();
+            float hv[64];
+            ld_cols<64>(haddr, hv);
+            add_psi(NC - 1, hv);
+            if (!failed && p.s_out) {
+                float* dst = p.s_out + ((size_t)bh * D + d) * D + 64 * c;
+#pragma unroll
+                for (int e = 0; e < 64; e += 4)
+                    *reinterpret_cast<float4*>(dst + e) = make_float4(hv[e], hv[e + 1], hv[e + 2], hv[e + 3]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+bool make_maps(const ChunkParams& p, bool perdim, PrepMaps* m) {
     const uint64_t dims[3] = {(uint64_t)p.H * D, (uint64_t)p.T, (uint64_t)p.B};
     const uint64_t strides[2] = {(uint64_t)p.H * D * 2, (uint64_t)p.T * p.H * D * 2};
     const uint32_t box[3] = {64, 64, 1};
-    return make_tmap_bf16(&m->q, p.q, 3, dims, strides, box) &&
-           make_tmap_bf16(&m->k, p.k, 3, dims, strides, box) &&
-           make_tmap_bf16(&m->v, p.v, 3, dims, strides, box);
+    bool ok = make_tmap_bf16(&m->q, p.q, 3, dims, strides, box) &&
+              make_tmap_bf16(&m->k, p.k, 3, dims, strides, box) &&
+              make_tmap_bf16(&m->v, p.v, 3, dims, strides, box);
+    m->g = m->q;
+    if (ok && perdim) ok = make_tmap_bf16(&m->g, p.g, 3, dims, strides, box);
+    return ok;
 }
 
 // Chunk slots per (batch, head) of one wave: as many as keep the wave's
-// workspace near WAVE_BYTES (L2-resident), at least 4.
-int wave_chunks(int nbh, int NC, uint32_t image_bytes) {
-    long long cw = (long long)(WAVE_BYTES / ((size_t)nbh * image_bytes));
-    if (cw < 4) cw = 4;
+// workspace near WAVE_BYTES (L2-resident), at least one.
+int wave_chunks(int nbh, int NC) {
+    long long cw = (long long)(WAVE_BYTES / ((size_t)nbh * IMG_BYTES));
+    if (cw < 1) cw = 1;
     if (cw > NC) cw = NC;
-    return (int)(cw < 1 ? 1 : cw);
+    return (int)cw;
 }
 
 }  // namespace
@@ -1062,66 +942,47 @@ bool chunk_fwd_tc_supported(int Dk, int Dv, int gate) {
     return Dk == D && Dv == D && (gate == kGateNone || gate == kGateScalar || gate == kGatePerDim);
 }
 
-namespace {
-uint32_t image_bytes(int gate) { return gate == kGatePerDim ? WS_CHUNK_PD : WS_CHUNK; }
-}  // namespace
-
 size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H, int gate) {
+    (void)gate;
     const int NC = (T + C - 1) / C;
     if (NC == 0 || B == 0 || H == 0) return 0;
     const int nbh = B * H;
-    const int cw = wave_chunks(nbh, NC, image_bytes(gate));
+    const int cw = wave_chunks(nbh, NC);
     const int nw = (NC + cw - 1) / cw;
-    size_t bytes = (size_t)nbh * cw * image_bytes(gate);
+    size_t bytes = (size_t)nbh * cw * IMG_BYTES;
     if (nw > 1) bytes += (size_t)nbh * D * D * sizeof(float);   // state between waves
     return bytes;
 }
 
 cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s, int* launches) {
     *launches = 0;
-    TcMaps maps;
-    if (!make_maps(p0, &maps)) return cudaErrorInvalidValue;
     const bool perdim = gate == kGatePerDim;
-    PrepMaps pmaps;
-    pmaps.q = maps.q;
-    pmaps.k = maps.k;
-    PrepPdMaps dmaps;
-    dmaps.q = maps.q;
-    dmaps.k = maps.k;
-    if (perdim) {
-        const uint64_t dims[3] = {(uint64_t)p0.H * D, (uint64_t)p0.T, (uint64_t)p0.B};
-        const uint64_t strides[2] = {(uint64_t)p0.H * D * 2, (uint64_t)p0.T * p0.H * D * 2};
-        const uint32_t box[3] = {64, 64, 1};
-        if (!make_tmap_bf16(&dmaps.g, p0.g, 3, dims, strides, box)) return cudaErrorInvalidValue;
-    }
-    auto prep = gate == kGateScalar ? chunk_prep_tc_kernel<kGateScalar> : chunk_prep_tc_kernel<kGateNone>;
-    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
+    PrepMaps maps;
+    if (!make_maps(p0, perdim, &maps)) return cudaErrorInvalidValue;
+    auto prep = gate == kGateScalar ? chunk_prep_kernel<kGateScalar>
+                : gate == kGatePerDim ? chunk_prep_kernel<kGatePerDim>
+                                      : chunk_prep_kernel<kGateNone>;
+    const uint32_t prep_smem = perdim ? P_SMEM_PD : P_SMEM;
+    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_prep_pd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)D_SMEM);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    e = cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CH_SMEM);
     if (e != cudaSuccess) return e;
     const int NC = (p0.T + C - 1) / C;
     const int nbh = p0.B * p0.H;
-    const uint32_t img = image_bytes(gate);
-    const int cw = wave_chunks(nbh, NC, img);
+    const int cw = wave_chunks(nbh, NC);
     const int nw = (NC + cw - 1) / cw;
-    float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + (size_t)nbh * cw * img) : nullptr;
+    float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + (size_t)nbh * cw * IMG_BYTES) : nullptr;
     for (int w = 0; w < nw; ++w) {
         ChunkParams p = p0;
         p.cw = cw;
-        p.ws_chunk = (int)img;
+        p.ws_chunk = (int)IMG_BYTES;
         p.chunk0 = w * cw;
         p.nchunks = (w + 1 < nw) ? cw : NC - w * cw;
         p.s0 = (w == 0) ? p0.s0 : carry;
         p.s_out = (w + 1 == nw) ? p0.s_out : carry;
-        if (perdim)
-            chunk_prep_pd_kernel<<<(unsigned)(nbh * p.nchunks), NPR, D_SMEM, s>>>(dmaps, p);
-        else
-            prep<<<(unsigned)(nbh * p.nchunks), NPR, P_SMEM, s>>>(pmaps, p);
+        prep<<<(unsigned)(nbh * p.nchunks), NPR, prep_smem, s>>>(maps, p);
         ++*launches;
-        chunk_fwd_tc_kernel<<<(unsigned)nbh, NT, SMEM_BYTES, s>>>(maps, p, gate != kGateNone ? 1 : 0,
-                                                                  perdim ? 1 : 0);
+        chunk_chain_kernel<<<(unsigned)nbh, CH_THREADS, CH_SMEM, s>>>(p);
         ++*launches;
     }
     return cudaGetLastError();
