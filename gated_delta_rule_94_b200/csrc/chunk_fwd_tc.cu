@@ -12,26 +12,30 @@
 //   W  = T diag(beta) (K e^G),  U = T diag(beta) V,  K~ = K e^(G_C - G)
 //   D  = U - W h,  O = (Q e^G) h + P D,  h' = Diag(e^(G_C)) h + K~^T D.
 // Substituting D, each chunk is an affine map of the entering state:
-//   h' = (Diag(gamma) + Phi) h + Psi,     Phi = -K~^T W,  Psi = K~^T U
-//   O  = Qp h + P U,                      Qp = Q e^G - P W
-// with gamma = e^(G_C).  Phi, Psi, Qp, P U and gamma depend on the chunk's
-// inputs only, so they are formed for every chunk at once, and only the
-// product with h remains on the serial path.
+//   h' = Diag(gamma) h + Phi h + K~^T U,    Phi = -K~^T W,  gamma = e^(G_C)
+//   O  = Qp h + P U,                        Qp  = Q e^G - P W
+// Phi, K~, U, Qp, P U and gamma depend on the chunk's inputs only, so they are
+// formed for every chunk at once, and only the products with h remain on the
+// serial path.  The decay stays an fp32 multiply of the fp32 state (a bf16
+// gamma - 1 folded into Phi would leave 2^-9 |h| per chunk behind, large
+// against a strongly decayed h').
 //
 // Two kernels per wave of chunks:
 //   chunk_prep_kernel   one CTA per (batch, head, chunk), fully parallel: the
 //                       gates, S = [K;Q]K^T, A and P, T, the WY factors as
-//                       W^T = K^T T^T and U^T = V^T T^T, then
-//                       [Phi | Psi] = -/+ K~^T [W | U] and [P W | P U]; writes
-//                       the chunk's step image (Phi, Psi, Qp, P U in bf16,
-//                       gamma in fp32) to the workspace, laid out exactly as
-//                       the chain kernel's shared-memory operands (the wave is
-//                       sized so the workspace stays in L2);
+//                       W^T = K^T T^T and U^T = V^T T^T, then K~^T W and
+//                       [P W | P U]; writes the chunk's step image (Phi, K~,
+//                       U^T, Qp, P U in bf16, gamma in fp32) to the workspace
+//                       by bulk copies,
+//                       laid out exactly as the chain kernel's shared-memory
+//                       operands (the wave is sized so the workspace stays in
+//                       L2);
 //   chunk_chain_kernel  one CTA per (batch, head), the serial state chain:
-//                       per chunk one 8-step MMA h += Phi h_bf16 onto the
-//                       decayed fp32 state in TMEM, the state pass
-//                       (h + Psi -> bf16 operand, decay) and, off the serial
-//                       path, O^T = h^T Qp^T + (P U)^T.
+//                       X = K~^T U (one chunk ahead) + Phi h_bf16 (8 MMA
+//                       steps) in TMEM, then the state pass h' = gamma h + X
+//                       in fp32 and its bf16 copy as the next operand; off the
+//                       serial path O^T = h^T Qp^T, added to P U in shared
+//                       memory and written by a TMA tensor store.
 // Every mbarrier wait is bounded; a wait that gives up sets the library status
 // word and the kernel winds down without further waits.
 #include "common.cuh"
@@ -51,7 +55,8 @@ constexpr int LDF = 72;          // fp32 row stride of the A / T scratch (confli
 // Step image of one chunk (bytes).  Tiles of bf16 rows of 64 elements with the
 // 128-byte swizzle; a [rows][128] matrix is two such column blocks.
 constexpr uint32_t IMG_PHI = 0;        // Phi  [128 d][128 d'],  blocks of 16 KB (K-major A)
-constexpr uint32_t IMG_PSI = 32768;    // Psi  [128 d][128 v],   blocks of 16 KB
+constexpr uint32_t IMG_KT = 32768;     // K~   [64 i][128 d],    blocks of 8 KB (MN-major A)
+constexpr uint32_t IMG_UT = 49152;     // U^T  [128 v][64 i]     (K-major B)
 constexpr uint32_t IMG_QP = 65536;     // Qp   [64 r][128 d],    blocks of 8 KB (K-major B)
 constexpr uint32_t IMG_PU = 81920;     // P U  [64 r][128 v],    blocks of 8 KB
 constexpr uint32_t IMG_GAM = 98304;    // gamma fp32 [128]
@@ -256,11 +261,15 @@ constexpr uint32_t P_TW = 86016;             // T diag(beta e^G) bf16 [64 r][64 
 constexpr uint32_t P_TU = 94208;             // T diag(beta)
 constexpr uint32_t P_KT = 102400;            // K~ = K e^(G_C - G)  [b0 | b1]
 constexpr uint32_t P_P = 118784;             // P bf16 [64 r][64 i]
-constexpr uint32_t P_GATE = 126976;          // G, e^G, e^(G_C-G), beta, u, w, flag (7 x 64 floats)
+constexpr uint32_t P_GATE = 131072;          // G, e^G, e^(G_C-G), beta, u, w, flag (7 x 64 floats)
 constexpr uint32_t P_BAR = P_GATE + 7 * 64 * 4;
 constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;
+// staging of the step image for its bulk stores (buffers dead by then)
+constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
+constexpr uint32_t S_PU = 65536;             // over the U^T rows (after their own store has read them)
+constexpr uint32_t S_QP = 86016;             // over T_w / T_u
 // per-dimension gate extras
-constexpr uint32_t X_G16 = 129024;           // g tile bf16 [g_b0 | g_b1] (TMA)
+constexpr uint32_t X_G16 = 133120;           // g tile bf16 [g_b0 | g_b1] (TMA)
 constexpr uint32_t X_KB = X_G16 + 16384;     // K e^(m - G)      [b0 | b1]
 constexpr uint32_t X_KG = X_KB + 16384;      // K e^G            [b0 | b1]
 constexpr uint32_t X_QB = X_KG + 16384;      // Q e^G            [b0 | b1]
@@ -270,6 +279,7 @@ constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (
 static_assert(P_TF + 64 * LDF * 4 <= P_TW, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_TW, "[W^T; U^T] tile");
 static_assert(P_BAR + 64 <= X_G16, "prep layout");
+static_assert(S_PHI + 32768 <= S_PU && S_PU + 16384 <= P_TW && S_QP + 16384 <= P_KT, "staging");
 static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
 static_assert(P_SMEM_PD <= 232448, "prep shared memory");
 
@@ -277,7 +287,7 @@ static_assert(P_SMEM_PD <= 232448, "prep shared memory");
 constexpr uint32_t TM_S = 0;       // [K;Q] K^T, 64 columns
 constexpr uint32_t TM_WT = 64;     // W^T, lanes d, 64 columns r
 constexpr uint32_t TM_UT = 128;    // U^T, lanes v, 64 columns r
-constexpr uint32_t TM_FP = 256;    // [K~^T W | K~^T U], 256 columns
+constexpr uint32_t TM_FP = 256;    // K~^T W, 128 columns
 constexpr uint32_t TM_PP = 0;      // [P W | P U] (M = 64: rows in lanes 0-15 of each quarter)
 
 // One CTA per (batch, head, chunk) of the wave: every state-independent part
@@ -593,6 +603,10 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (tid == 0 && !failed) {   // K~ is final: its image goes out now
+        bulk_store(img + IMG_KT, sm + P_KT, 16384);
+        bulk_commit();
+    }
     if (tid == 32 && !failed) {
         // W^T = (K e^G)^T T_w^T (scalar gate: the decay sits in T_w), U^T = V^T T_u^T
         const uint32_t id = idesc_bf16_f32(128, 64, true, false);
@@ -621,8 +635,12 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (tid == 0 && !failed) {   // U^T is final
+        bulk_store(img + IMG_UT, sm + P_WUT + 16384, 16384);
+        bulk_commit();
+    }
     if (tid == 32 && !failed) {
-        const uint32_t id1 = idesc_bf16_f32(128, 256, true, false);   // K~^T [W | U]
+        const uint32_t id1 = idesc_bf16_f32(128, 128, true, false);   // K~^T W
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_FP, sdesc_sw128(sb + P_KT + k * 2048, 8192, 1024),
@@ -635,37 +653,48 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         mma_commit(&bars[3]);
     }
     wait(3, 0);
+    if (tid == 0) bulk_wait_read();   // the U^T rows become the P U staging
     tc_fence_after();
-    {   // Phi = -K~^T W (warps 0-3) and Psi = K~^T U (warps 4-7), row d = lane
-        const int d = (warp & 3) * 32 + lane;
+    __syncthreads();
+    if (warp < 4) {   // Phi = -K~^T W, row d; gamma_d
+        const int d = warp * 32 + lane;
         float v[128];
-        ld_cols<128>(tmem + TM_FP + lane_off + (warp < 4 ? 0 : 128), v);
-        if (!failed) st_row128(img + (warp < 4 ? IMG_PHI : IMG_PSI), 16384, d, v, warp < 4 ? -1.f : 1.f);
+        ld_cols<128>(tmem + TM_FP + lane_off, v);
+        st_row128(sm + S_PHI, 16384, d, v, -1.f);
+        float gam;
+        if constexpr (PD) gam = expf(sC[d]);
+        else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
+        if (!failed) reinterpret_cast<float*>(img + IMG_GAM)[d] = gam;
+    } else {          // P U, row r = 16 (warp & 3) + lane
+        float v[128];
+        ld_cols<128>(tmem + TM_PP + lane_off + 128, v);
+        if (lane < 16) st_row128(sm + S_PU, 8192, 16 * (warp & 3) + lane, v, 1.f);
     }
-    {   // Qp = Q e^G - P W (warps 0-3) and P U (warps 4-7); row r = 16 (warp & 3) + lane
+    if (warp < 4) {   // Qp = Q e^G - P W, row r = 16 warp + lane
         float v[128];
-        ld_cols<128>(tmem + TM_PP + lane_off + (warp < 4 ? 0 : 128), v);
-        const int r = 16 * (warp & 3) + lane;
-        if (lane < 16 && !failed) {
-            if (warp < 4) {
-                const float eg = gbuf[64 + r];
+        ld_cols<128>(tmem + TM_PP + lane_off, v);
+        const int r = 16 * warp + lane;
+        if (lane < 16) {
+            const float eg = gbuf[64 + r];
 #pragma unroll
-                for (int dd = 0; dd < D; ++dd) {
-                    const float qb = PD ? ld_bf16(sm + X_QB + (dd >> 6) * 8192, r, dd & 63)
-                                        : eg * ld_bf16(sm + P_KQ + (dd >> 6) * 16384 + 8192, r, dd & 63);
-                    v[dd] = qb - v[dd];
-                }
-                st_row128(img + IMG_QP, 8192, r, v, 1.f);
-            } else {
-                st_row128(img + IMG_PU, 8192, r, v, 1.f);
+            for (int dd = 0; dd < D; ++dd) {
+                const float qb = PD ? ld_bf16(sm + X_QB + (dd >> 6) * 8192, r, dd & 63)
+                                    : eg * ld_bf16(sm + P_KQ + (dd >> 6) * 16384 + 8192, r, dd & 63);
+                v[dd] = qb - v[dd];
             }
+            st_row128(sm + S_QP, 8192, r, v, 1.f);
         }
     }
-    if (tid < 128 && !failed) {
-        float gam;
-        if constexpr (PD) gam = expf(sC[tid]);
-        else gam = gbuf[64 + 63];
-        reinterpret_cast<float*>(img + IMG_GAM)[tid] = gam;
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        if (!failed) {
+            bulk_store(img + IMG_PHI, sm + S_PHI, 32768);
+            bulk_store(img + IMG_QP, sm + S_QP, 16384);
+            bulk_store(img + IMG_PU, sm + S_PU, 16384);
+            bulk_commit();
+        }
+        bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -678,32 +707,39 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 // ------------------------------------------------------------------ chain
 // Chain kernel shared memory (bytes from a 1 KB-aligned base).
 constexpr uint32_t CH_PHI = 0;          // 2 slots of Phi   (32 KB each)
-constexpr uint32_t CH_PSI = 65536;      // 2 slots of Psi   (32 KB each)
-constexpr uint32_t CH_QP = 131072;      // Qp   (16 KB)
-constexpr uint32_t CH_PU = 147456;      // P U  (16 KB)
+constexpr uint32_t CH_KT = 65536;       // K~   (16 KB, one slot)
+constexpr uint32_t CH_UT = 81920;       // U^T  (16 KB, one slot)
+constexpr uint32_t CH_QP = 98304;       // 2 slots of Qp (16 KB each)
+constexpr uint32_t CH_PU = 131072;      // 2 slots of P U, then O in place for its TMA store
 constexpr uint32_t CH_HB = 163840;      // 2 slots of h (bf16) MN-major [d][64 v] x 2 blocks
 constexpr uint32_t CH_GAM = 229376;     // 2 slots of gamma (512 B each)
 constexpr uint32_t CH_BAR = 230400;
-constexpr uint32_t CH_SMEM = CH_BAR + 32 * 8 + 1024;
+constexpr uint32_t CH_SMEM = CH_BAR + 256 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
 
 constexpr int CH_THREADS = 448;   // 14 warps: loader, MMA, 4 output, 8 state
-constexpr int NHP = 256;          // state-pass threads (warps 6-13)
 
-// TMEM columns of the chain kernel (256 allocated).
-constexpr uint32_t TM_H = 0;      // state, lanes d, 128 columns v (fp32)
+// TMEM columns of the chain kernel (512 allocated).
+constexpr uint32_t TM_H = 0;      // state h, lanes d, 128 columns v (fp32, the state pass's own)
 constexpr uint32_t TM_O = 128;    // O^T, lanes v, 2 slots of 64 columns r
+constexpr uint32_t TM_X = 256;    // X = K~^T U + Phi h, lanes d, 2 slots of 128 columns v
 
 enum ChainBar {
-    CB_PHI0, CB_PHI1, CB_PSI0, CB_PSI1, CB_QP, CB_PU, CB_HREADY, CB_SDONE, CB_SFREE0, CB_SFREE1,
-    CB_PSIFREE0, CB_PSIFREE1, CB_ODONE, CB_OFREE0, CB_OFREE1, CB_FINAL, CB_COUNT
+    CB_IMG0, CB_IMG1, CB_KU, CB_QP0, CB_QP1, CB_PU0, CB_PU1,
+    CB_HREADY, CB_XFREE0, CB_XFREE1, CB_SDONE, CB_SFREE0, CB_SFREE1, CB_KUFREE,
+    CB_ODONE0, CB_ODONE1, CB_OFREE0, CB_OFREE1, CB_FINAL, CB_COUNT
 };
+static_assert(CB_COUNT * 8 <= 256, "barrier space");
 
-// One CTA per (batch, head): walks the wave's chunks in order.  Chunk n's
-// image slot is n & 1; every barrier that a role waits on completes at most
-// once ahead of that wait, so the parity waits never fall two phases behind.
-__global__ void __launch_bounds__(CH_THREADS, 1)
-chunk_chain_kernel(const ChunkParams p) {
+// One CTA per (batch, head): walks the wave's chunks in order.  Per chunk n
+// (slot s = n & 1), h_n the entering state:
+//   X_n = K~_n^T U_n (issued one chunk ahead) + Phi_n bf16(h_n)   in TMEM
+//   h_{n+1} = gamma_n h_n + X_n                                  (state pass, fp32)
+//   O_n^T = bf16(h_n)^T Qp_n^T,  O_n = O_n^T^T + (P U)_n          (output warps)
+// Every barrier that a role waits on is per slot or completes at most once
+// ahead of that wait, so no parity wait can fall two phases behind.
+__global__ void __maxnreg__(128)
+chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -712,7 +748,7 @@ chunk_chain_kernel(const ChunkParams p) {
     __shared__ uint32_t s_tmem;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = p.H, T = p.T;
+    const int H = p.H;
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int NC = p.nchunks;
     const uint8_t* wsh = p.ws + (size_t)bh * p.cw * IMG_BYTES;
@@ -720,11 +756,13 @@ chunk_chain_kernel(const ChunkParams p) {
     int failed = 0;
 
     if (tid == 0) {
-        for (int i = 0; i < CB_COUNT; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < CB_COUNT; ++i)
+            mbar_init(&bars[i], (i == CB_HREADY || i == CB_XFREE0 || i == CB_XFREE1) ? 8 : 1);
         fence_mbar_init();
+        prefetch_tmap(&omap);
     }
     if (warp == 1) {
-        tmem_alloc(&s_tmem, 256);
+        tmem_alloc(&s_tmem, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -739,56 +777,74 @@ chunk_chain_kernel(const ChunkParams p) {
     auto img = [&](int nl) { return wsh + (size_t)nl * IMG_BYTES; };
 
     if (warp == 0) {
-        // =========================== loader: Phi + gamma and Psi of every chunk
+        // =========================== loader: Phi + gamma (2 slots) and K~, U^T
         if (lane == 0) {
 #pragma unroll 1
             for (int nl = 0; nl < NC; ++nl) {
                 const int s = nl & 1;
-                if (nl >= 2) {
-                    if (!mbar_wait(&bars[CB_SFREE0 + s], ((nl - 2) >> 1) & 1, &failed)) break;
-                }
-                mbar_arrive_expect_tx(&bars[CB_PHI0 + s], 32768 + 512);
-                bulk_load(sm + CH_PHI + s * 32768, img(nl) + IMG_PHI, 32768, &bars[CB_PHI0 + s]);
-                bulk_load(sm + CH_GAM + s * 512, img(nl) + IMG_GAM, 512, &bars[CB_PHI0 + s]);
-                if (nl >= 2) {
-                    if (!mbar_wait(&bars[CB_PSIFREE0 + s], ((nl - 2) >> 1) & 1, &failed)) break;
-                }
-                mbar_arrive_expect_tx(&bars[CB_PSI0 + s], 32768);
-                bulk_load(sm + CH_PSI + s * 32768, img(nl) + IMG_PSI, 32768, &bars[CB_PSI0 + s]);
+                if (nl >= 2 && !mbar_wait(&bars[CB_SFREE0 + s], ((nl - 2) >> 1) & 1, &failed)) break;
+                mbar_arrive_expect_tx(&bars[CB_IMG0 + s], 32768 + 512);
+                bulk_load(sm + CH_PHI + s * 32768, img(nl) + IMG_PHI, 32768, &bars[CB_IMG0 + s]);
+                bulk_load(sm + CH_GAM + s * 512, img(nl) + IMG_GAM, 512, &bars[CB_IMG0 + s]);
+                if (nl >= 1 && !mbar_wait(&bars[CB_KUFREE], (nl - 1) & 1, &failed)) break;
+                mbar_arrive_expect_tx(&bars[CB_KU], 32768);
+                bulk_load(sm + CH_KT, img(nl) + IMG_KT, 16384, &bars[CB_KU]);
+                bulk_load(sm + CH_UT, img(nl) + IMG_UT, 16384, &bars[CB_KU]);
             }
             if (failed) atomicOr(p.status, kStatusTimeout);
         }
     } else if (warp == 1) {
-        // =========================== MMA issuer
+        // =========================== MMA issuer (descriptors built once; a k-step
+        // adds its byte offset / 16 to the start-address field)
         const bool leader = lane == 0;
-        const uint32_t ids = idesc_bf16_f32(128, 128, false, true);   // h += Phi h_bf16
-        const uint32_t ido = idesc_bf16_f32(128, 64, true, false);    // O^T = h^T Qp^T
+        const uint32_t id_ku = idesc_bf16_f32(128, 128, true, false);   // K~^T U
+        const uint32_t id_ph = idesc_bf16_f32(128, 128, false, true);   // Phi h_bf16
+        const uint32_t id_o = idesc_bf16_f32(128, 64, true, false);     // h^T Qp^T
+        const uint64_t d_phi = sdesc_sw128(sb + CH_PHI, 16, 1024);
+        const uint64_t d_kt = sdesc_sw128(sb + CH_KT, 8192, 1024);
+        const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
+        const uint64_t d_hb = sdesc_sw128(sb + CH_HB, 16384, 1024);
+        const uint64_t d_qp = sdesc_sw128(sb + CH_QP, 16, 1024);
+        // K~^T U of chunk nl into X slot nl & 1 once K~, U^T are in and the state
+        // pass has read X of chunk nl - 2 there
+        auto issue_ku = [&](int nl) {
+            const int s = nl & 1;
+            wait(CB_KU, nl & 1);
+            if (nl >= 2) wait(CB_XFREE0 + s, ((nl - 2) >> 1) & 1);
+            tc_fence_after();
+            if (leader && !failed) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tmem + TM_X + 128 * s, d_kt + ((k * 2048) >> 4), d_ut + ((k * 32) >> 4),
+                             id_ku, k > 0);
+                mma_commit(&bars[CB_KUFREE]);
+            }
+        };
+        if (NC > 0) issue_ku(0);
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            const uint32_t hb = sb + CH_HB + s * 32768;
             wait(CB_HREADY, nl & 1);
-            wait(CB_PHI0 + s, (nl >> 1) & 1);
+            wait(CB_IMG0 + s, (nl >> 1) & 1);
             tc_fence_after();
             if (leader && !failed) {
-                const uint32_t phi = sb + CH_PHI + s * 32768;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_bf16(tmem + TM_H, sdesc_sw128(phi + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                             sdesc_sw128(hb + k * 2048, 16384, 1024), ids, true);
+                    mma_bf16(tmem + TM_X + 128 * s, d_phi + ((s * 32768 + (k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                             d_hb + ((s * 32768 + k * 2048) >> 4), id_ph, true);
                 mma_commit(&bars[CB_SDONE]);
                 mma_commit(&bars[CB_SFREE0 + s]);
             }
-            wait(CB_QP, nl & 1);
+            if (nl + 1 < NC) issue_ku(nl + 1);
+            wait(CB_QP0 + s, (nl >> 1) & 1);
             if (nl >= 2) wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
             tc_fence_after();
             if (leader && !failed) {
-                const uint32_t qp = sb + CH_QP;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_bf16(tmem + TM_O + 64 * s, sdesc_sw128(hb + k * 2048, 16384, 1024),
-                             sdesc_sw128(qp + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ido, k > 0);
-                mma_commit(&bars[CB_ODONE]);
+                    mma_bf16(tmem + TM_O + 64 * s, d_hb + ((s * 32768 + k * 2048) >> 4),
+                             d_qp + ((s * 16384 + (k >> 2) * 8192 + (k & 3) * 32) >> 4), id_o, k > 0);
+                mma_commit(&bars[CB_ODONE0 + s]);
             }
         }
         // nothing issued by this warp may still run when TMEM is released
@@ -797,70 +853,78 @@ chunk_chain_kernel(const ChunkParams p) {
         if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     } else if (warp < 6) {
-        // =========================== output: O = (O^T)^T + P U, bf16 to o
+        // =========================== output: O = (O^T)^T + P U in place, TMA store
         const int v = (warp & 3) * 32 + lane;
         const bool leader = warp == 2 && lane == 0;
-        if (leader && NC > 0) {
-            mbar_arrive_expect_tx(&bars[CB_QP], 16384);
-            bulk_load(sm + CH_QP, img(0) + IMG_QP, 16384, &bars[CB_QP]);
-            mbar_arrive_expect_tx(&bars[CB_PU], 16384);
-            bulk_load(sm + CH_PU, img(0) + IMG_PU, 16384, &bars[CB_PU]);
+        auto load_qp = [&](int nl) {
+            mbar_arrive_expect_tx(&bars[CB_QP0 + (nl & 1)], 16384);
+            bulk_load(sm + CH_QP + (nl & 1) * 16384, img(nl) + IMG_QP, 16384, &bars[CB_QP0 + (nl & 1)]);
+        };
+        auto load_pu = [&](int nl) {
+            mbar_arrive_expect_tx(&bars[CB_PU0 + (nl & 1)], 16384);
+            bulk_load(sm + CH_PU + (nl & 1) * 16384, img(nl) + IMG_PU, 16384, &bars[CB_PU0 + (nl & 1)]);
+        };
+        if (leader) {
+            for (int nl = 0; nl < 2 && nl < NC; ++nl) {
+                load_qp(nl);
+                load_pu(nl);
+            }
         }
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            wait(CB_ODONE, nl & 1);
-            if (leader && !failed && nl + 1 < NC) {   // Qp slot is free once O of chunk nl is done
-                mbar_arrive_expect_tx(&bars[CB_QP], 16384);
-                bulk_load(sm + CH_QP, img(nl + 1) + IMG_QP, 16384, &bars[CB_QP]);
-            }
-            wait(CB_PU, nl & 1);
+            wait(CB_ODONE0 + s, (nl >> 1) & 1);
+            if (leader && !failed && nl + 2 < NC) load_qp(nl + 2);   // O of chunk nl is done with Qp
+            wait(CB_PU0 + s, (nl >> 1) & 1);
             tc_fence_after();
-            float ov[64];
-            ld_cols<64>(tmem + TM_O + 64 * s + lane_off, ov);
-            const int t0 = (p.chunk0 + nl) * C;
-            const int nval = min(C, T - t0);
-            __nv_bfloat16* ocol = static_cast<__nv_bfloat16*>(p.o) + (((size_t)b * T + t0) * H + h) * D + v;
-            const uint8_t* pu = sm + CH_PU + (v >> 6) * 8192;
-            if (!failed) {
+            uint8_t* pu = sm + CH_PU + s * 16384 + (v >> 6) * 8192;
 #pragma unroll
-                for (int r = 0; r < C; ++r)
-                    if (r < nval) ocol[(size_t)r * H * D] = __float2bfloat16_rn(ov[r] + ld_bf16(pu, r, v & 63));
+            for (int half = 0; half < 2; ++half) {
+                float ov[32], pv[32];
+                ld_cols<32>(tmem + TM_O + 64 * s + 32 * half + lane_off, ov);
+#pragma unroll
+                for (int r = 0; r < 32; ++r)
+                    pv[r] = ld_bf16(pu, 32 * half + r, v & 63);
+#pragma unroll
+                for (int r = 0; r < 32; ++r)
+                    *reinterpret_cast<__nv_bfloat16*>(pu + sw128_offset(32 * half + r, v & 63)) =
+                        __float2bfloat16_rn(ov[r] + pv[r]);
             }
+            fence_async_smem();
             tc_fence_before();
             named_bar(2, 128);
             if (leader) {
                 mbar_arrive(&bars[CB_OFREE0 + s]);
-                if (!failed && nl + 1 < NC) {
-                    mbar_arrive_expect_tx(&bars[CB_PU], 16384);
-                    bulk_load(sm + CH_PU, img(nl + 1) + IMG_PU, 16384, &bars[CB_PU]);
+                if (!failed) {
+                    const int t0 = (p.chunk0 + nl) * C;
+                    tma_store_3d(&omap, sm + CH_PU + s * 16384, h * D, t0, b);
+                    tma_store_3d(&omap, sm + CH_PU + s * 16384 + 8192, h * D + 64, t0, b);
+                    bulk_commit();
+                    if (nl + 2 < NC) {
+                        bulk_wait_read();
+                        load_pu(nl + 2);
+                    }
                 }
             }
         }
+        if (leader) bulk_wait_all();
     } else {
-        // =========================== state pass: h + Psi -> bf16 operand, decay
+        // =========================== state pass: h' = gamma h + X -> bf16 operand
         const int d = (warp & 3) * 32 + lane;
         const int c = (warp - 6) >> 2;              // column half
-        const bool leader = warp == 6 && lane == 0;
         const uint32_t haddr = tmem + TM_H + lane_off + 64 * c;
-        auto add_psi = [&](int nl, float (&hv)[64]) {
-            const uint8_t* row = sm + CH_PSI + (nl & 1) * 32768 + c * 16384 + d * 128;
+        float gam = 1.f;                            // gamma of the chunk before
+        float hv[64];
+        auto advance = [&](int nl) {                // hv = gamma_{nl-1} h_{nl-1} + X_{nl-1}
+            float xv[64];
+            ld_cols<64>(haddr, hv);
+            ld_cols<64>(tmem + TM_X + 128 * ((nl - 1) & 1) + lane_off + 64 * c, xv);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint4 raw = *reinterpret_cast<const uint4*>(row + ((j ^ (d & 7)) * 16));
-                const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(e2[e]);
-                    hv[8 * j + 2 * e] += f.x;
-                    hv[8 * j + 2 * e + 1] += f.y;
-                }
-            }
+            for (int e = 0; e < 64; ++e) hv[e] = fmaf(gam, hv[e], xv[e]);
         };
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            float hv[64];
             if (nl == 0) {
                 const float* s0 = p.s0 ? p.s0 + ((size_t)bh * D + d) * D + 64 * c : nullptr;
 #pragma unroll
@@ -870,35 +934,29 @@ chunk_chain_kernel(const ChunkParams p) {
                 }
             } else {
                 wait(CB_SDONE, (nl - 1) & 1);
-                wait(CB_PSI0 + ((nl - 1) & 1), ((nl - 1) >> 1) & 1);
                 tc_fence_after();
-                ld_cols<64>(haddr, hv);
-                add_psi(nl - 1, hv);
+                advance(nl);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[CB_XFREE0 + ((nl - 1) & 1)]);
             }
-            wait(CB_PHI0 + s, (nl >> 1) & 1);
-            const float gam = reinterpret_cast<const float*>(sm + CH_GAM + s * 512)[d];
             uint8_t* hb = sm + CH_HB + s * 32768 + c * 16384;
 #pragma unroll
             for (int j = 0; j < 8; ++j) st_row_chunk(hb, d, j, hv + 8 * j, 1.f);
-#pragma unroll
-            for (int e = 0; e < 64; ++e) hv[e] *= gam;
-            st_cols<64>(haddr, hv);
-            tmem_wait_st();
+            // gamma of this chunk before HREADY: its slot is refilled only after
+            // the MMA that HREADY releases
+            wait(CB_IMG0 + s, (nl >> 1) & 1);
+            gam = reinterpret_cast<const float*>(sm + CH_GAM + s * 512)[d];
             fence_async_smem();
-            tc_fence_before();
-            named_bar(1, NHP);
-            if (leader) {
-                mbar_arrive(&bars[CB_HREADY]);
-                if (nl >= 1) mbar_arrive(&bars[CB_PSIFREE0 + ((nl - 1) & 1)]);
-            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[CB_HREADY]);
+            st_cols<64>(haddr, hv);                 // the fp32 state, read back next chunk
+            tmem_wait_st();
         }
-        if (NC > 0) {   // final state = h + Psi of the last chunk
+        if (NC > 0) {   // final state
             wait(CB_SDONE, (NC - 1) & 1);
-            wait(CB_PSI0 + ((NC - 1) & 1), ((NC - 1) >> 1) & 1);
             tc_fence_after();
-            float hv[64];
-            ld_cols<64>(haddr, hv);
-            add_psi(NC - 1, hv);
+            advance(NC);
             if (!failed && p.s_out) {
                 float* dst = p.s_out + ((size_t)bh * D + d) * D + 64 * c;
 #pragma unroll
@@ -911,7 +969,7 @@ chunk_chain_kernel(const ChunkParams p) {
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -959,6 +1017,13 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s,
     const bool perdim = gate == kGatePerDim;
     PrepMaps maps;
     if (!make_maps(p0, perdim, &maps)) return cudaErrorInvalidValue;
+    CUtensorMap omap;
+    {
+        const uint64_t dims[3] = {(uint64_t)p0.H * D, (uint64_t)p0.T, (uint64_t)p0.B};
+        const uint64_t strides[2] = {(uint64_t)p0.H * D * 2, (uint64_t)p0.T * p0.H * D * 2};
+        const uint32_t box[3] = {64, 64, 1};
+        if (!make_tmap_bf16(&omap, p0.o, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
     auto prep = gate == kGateScalar ? chunk_prep_kernel<kGateScalar>
                 : gate == kGatePerDim ? chunk_prep_kernel<kGatePerDim>
                                       : chunk_prep_kernel<kGateNone>;
@@ -982,7 +1047,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s,
         p.s_out = (w + 1 == nw) ? p0.s_out : carry;
         prep<<<(unsigned)(nbh * p.nchunks), NPR, prep_smem, s>>>(maps, p);
         ++*launches;
-        chunk_chain_kernel<<<(unsigned)nbh, CH_THREADS, CH_SMEM, s>>>(p);
+        chunk_chain_kernel<<<(unsigned)nbh, CH_THREADS, CH_SMEM, s>>>(omap, p);
         ++*launches;
     }
     return cudaGetLastError();
