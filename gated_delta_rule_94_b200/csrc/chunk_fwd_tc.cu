@@ -23,10 +23,10 @@
 // Two kernels per wave of chunks:
 //   chunk_prep_kernel   one CTA per (batch, head, chunk), fully parallel: the
 //                       gates, S = [K;Q]K^T, A and P, T, the WY factors as
-//                       W^T = K^T T^T and U^T = V^T T^T, then K~^T W and
-//                       [P W | P U]; writes the chunk's step image (Phi, K~,
-//                       U^T, Qp, P U in bf16, gamma in fp32) to the workspace
-//                       by bulk copies,
+//                       W^T = K^T T^T and U^T = V^T T^T, then K~^T W, W^T P^T
+//                       and U^T P^T; writes the chunk's step image (Phi, K~,
+//                       U^T, Qp^T, (P U)^T in bf16, gamma in fp32) to the
+//                       workspace by bulk copies,
 //                       laid out exactly as the chain kernel's shared-memory
 //                       operands (the wave is sized so the workspace stays in
 //                       L2);
@@ -57,8 +57,8 @@ constexpr int LDF = 72;          // fp32 row stride of the A / T scratch (confli
 constexpr uint32_t IMG_PHI = 0;        // Phi  [128 d][128 d'],  blocks of 16 KB (K-major A)
 constexpr uint32_t IMG_KT = 32768;     // K~   [64 i][128 d],    blocks of 8 KB (MN-major A)
 constexpr uint32_t IMG_UT = 49152;     // U^T  [128 v][64 i]     (K-major B)
-constexpr uint32_t IMG_QP = 65536;     // Qp   [64 r][128 d],    blocks of 8 KB (K-major B)
-constexpr uint32_t IMG_PU = 81920;     // P U  [64 r][128 v],    blocks of 8 KB
+constexpr uint32_t IMG_QP = 65536;     // Qp^T [128 d][64 r]     (MN-major B)
+constexpr uint32_t IMG_PU = 81920;     // (P U)^T [128 v][64 r]
 constexpr uint32_t IMG_GAM = 98304;    // gamma fp32 [128]
 constexpr uint32_t IMG_BYTES = 98816;
 constexpr size_t WAVE_BYTES = size_t(40) << 20;   // workspace per wave (kept L2-resident)
@@ -251,49 +251,52 @@ struct PrepMaps {
     CUtensorMap q, k, v, g;   // g only for the per-dimension gate
 };
 
-// Prep shared memory (bytes from a 1 KB-aligned base).
-constexpr uint32_t P_KQ = 0;                 // [K_b0 | Q_b0 | K_b1 | Q_b1] (TMA)
+// Prep shared memory (bytes from a 1 KB-aligned base); 110 KB for the scalar
+// gate, so two CTAs share an SM.
+constexpr uint32_t P_KQ = 0;                 // [K_b0 | Q_b0 | K_b1 | Q_b1] (TMA); K~ over K (scalar gate)
 constexpr uint32_t P_V = 32768;              // [V_b0 | V_b1] (TMA)
 constexpr uint32_t P_AF = 49152;             // A fp32 [64][LDF]; later [W^T; U^T] bf16 [256][64]
 constexpr uint32_t P_TF = P_AF + 64 * LDF * 4;   // T fp32 [64][LDF]
 constexpr uint32_t P_WUT = P_AF;
 constexpr uint32_t P_TW = 86016;             // T diag(beta e^G) bf16 [64 r][64 i]
 constexpr uint32_t P_TU = 94208;             // T diag(beta)
-constexpr uint32_t P_KT = 102400;            // K~ = K e^(G_C - G)  [b0 | b1]
-constexpr uint32_t P_P = 118784;             // P bf16 [64 r][64 i]
-constexpr uint32_t P_GATE = 131072;          // G, e^G, e^(G_C-G), beta, u, w, flag (7 x 64 floats)
+constexpr uint32_t P_P = 102400;             // P bf16 [64 r][64 i]
+constexpr uint32_t P_GATE = 110592;          // G, e^G, e^(G_C-G), beta, u, w, flag (7 x 64 floats)
 constexpr uint32_t P_BAR = P_GATE + 7 * 64 * 4;
 constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;
 // staging of the step image for its bulk stores (buffers dead by then)
 constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
-constexpr uint32_t S_PU = 65536;             // over the U^T rows (after their own store has read them)
-constexpr uint32_t S_QP = 86016;             // over T_w / T_u
+constexpr uint32_t S_QPT = 65536;            // over the U^T rows (after their own store has read them)
+constexpr uint32_t S_PUT = 86016;            // over T_w / T_u
 // per-dimension gate extras
-constexpr uint32_t X_G16 = 133120;           // g tile bf16 [g_b0 | g_b1] (TMA)
+constexpr uint32_t X_G16 = 113664;           // g tile bf16 [g_b0 | g_b1] (TMA)
 constexpr uint32_t X_KB = X_G16 + 16384;     // K e^(m - G)      [b0 | b1]
 constexpr uint32_t X_KG = X_KB + 16384;      // K e^G            [b0 | b1]
 constexpr uint32_t X_QB = X_KG + 16384;      // Q e^G            [b0 | b1]
-constexpr uint32_t X_SMALL = X_QB + 16384;   // m, c, e^m, e^(c-m) [128 each], flag
+constexpr uint32_t X_KT = X_QB + 16384;      // K e^(G_C - G)    [b0 | b1]
+constexpr uint32_t X_SMALL = X_KT + 16384;   // m, c, e^m, e^(c-m) [128 each], flag
 constexpr uint32_t P_SMEM_PD = X_SMALL + 4 * 128 * 4 + 16 + 1024;
 constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (aliases A / T)
 static_assert(P_TF + 64 * LDF * 4 <= P_TW, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_TW, "[W^T; U^T] tile");
 static_assert(P_BAR + 64 <= X_G16, "prep layout");
-static_assert(S_PHI + 32768 <= S_PU && S_PU + 16384 <= P_TW && S_QP + 16384 <= P_KT, "staging");
+static_assert(S_PHI + 32768 <= S_QPT && S_QPT + 16384 <= S_PUT && S_PUT + 16384 <= P_P, "staging");
 static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
+static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
 static_assert(P_SMEM_PD <= 232448, "prep shared memory");
 
-// TMEM columns of the prep kernel (512 allocated).
+// TMEM columns of the prep kernel (256 allocated: two CTAs per SM).
 constexpr uint32_t TM_S = 0;       // [K;Q] K^T, 64 columns
 constexpr uint32_t TM_WT = 64;     // W^T, lanes d, 64 columns r
 constexpr uint32_t TM_UT = 128;    // U^T, lanes v, 64 columns r
-constexpr uint32_t TM_FP = 256;    // K~^T W, 128 columns
-constexpr uint32_t TM_PP = 0;      // [P W | P U] (M = 64: rows in lanes 0-15 of each quarter)
+constexpr uint32_t TM_FP = 0;      // K~^T W, lanes d, 128 columns d'   (after S, W^T, U^T are read)
+constexpr uint32_t TM_PWT = 128;   // W^T P^T, lanes d, 64 columns r
+constexpr uint32_t TM_PUT = 192;   // U^T P^T, lanes v, 64 columns r
 
 // One CTA per (batch, head, chunk) of the wave: every state-independent part
 // of the chunk, written to the workspace as the chunk's step image.
 template <int GATE>
-__global__ void __launch_bounds__(NPR, 1)
+__global__ void __launch_bounds__(NPR, GATE == kGatePerDim ? 1 : 2)
 chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -342,7 +345,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         }
     }
     if (warp == 0) {
-        tmem_alloc(&s_tmem, 512);
+        tmem_alloc(&s_tmem, 256);
         tmem_relinquish();
     }
     if (tid < 64) {
@@ -454,7 +457,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             const uint32_t ioff = blk * 8192 + rowoff;
             *reinterpret_cast<uint4*>(sm + X_QB + ioff) = make_uint4(qg[0], qg[1], qg[2], qg[3]);
             *reinterpret_cast<uint4*>(sm + X_KG + ioff) = make_uint4(kg[0], kg[1], kg[2], kg[3]);
-            *reinterpret_cast<uint4*>(sm + P_KT + ioff) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
+            *reinterpret_cast<uint4*>(sm + X_KT + ioff) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
             if (!exact) {
                 *reinterpret_cast<uint4*>(sm + P_KQ + blk * 16384 + rowoff) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
                 *reinterpret_cast<uint4*>(sm + P_KQ + blk * 16384 + 8192 + rowoff) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
@@ -465,6 +468,10 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid == 0 && !failed) {   // K~ is final: its image goes out now
+            bulk_store(img + IMG_KT, sm + X_KT, 16384);
+            bulk_commit();
+        }
         if (!exact && tid == 32) {   // S = [K e^(G-m); Q e^(G-m)] (K e^(m-G))^T
             const uint32_t id = idesc_bf16_f32(128, 64, false, false);
 #pragma unroll
@@ -580,33 +587,10 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             st_row_chunk(sm + P_TW, r, j, tw, 1.f);
         }
     }
-    if constexpr (!PD) {   // K~ = diag(e^(G_C - G_i)) K
-        const float* sFt = gbuf + 128;
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int idx = tid + NPR * it;                 // 16-byte chunk 0..1023
-            const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
-            uint4 raw = *reinterpret_cast<const uint4*>(sm + P_KQ + blk * 16384 + r * 128 + j * 16);
-            const float f = sFt[r];
-            __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
-            uint4 outv;
-            uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 fv = __bfloat1622float2(e2[e]);
-                o32[e] = pack_bf16(fv.x * f, fv.y * f);
-            }
-            *reinterpret_cast<uint4*>(sm + P_KT + blk * 8192 + r * 128 + j * 16) = outv;
-        }
-    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0 && !failed) {   // K~ is final: its image goes out now
-        bulk_store(img + IMG_KT, sm + P_KT, 16384);
-        bulk_commit();
-    }
     if (tid == 32 && !failed) {
         // W^T = (K e^G)^T T_w^T (scalar gate: the decay sits in T_w), U^T = V^T T_u^T
         const uint32_t id = idesc_bf16_f32(128, 64, true, false);
@@ -631,76 +615,106 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) st_row_chunk(sm + P_WUT, (warp < 4 ? 0 : 128) + row, j, v + 8 * j, 1.f);
     }
+    if constexpr (!PD) {   // K~ = diag(e^(G_C - G_i)) K over K (the W product is done with K)
+        const float* sFt = gbuf + 128;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int idx = tid + NPR * it;                 // 16-byte chunk 0..1023
+            const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+            uint4* p16 = reinterpret_cast<uint4*>(sm + P_KQ + blk * 16384 + r * 128 + j * 16);
+            uint4 raw = *p16;
+            const float f = sFt[r];
+            __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+            uint4 outv;
+            uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 fv = __bfloat1622float2(e2[e]);
+                o32[e] = pack_bf16(fv.x * f, fv.y * f);
+            }
+            *p16 = outv;
+        }
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0 && !failed) {   // U^T is final
+    if (tid == 0 && !failed) {   // U^T (and the scalar gate's K~) are final
         bulk_store(img + IMG_UT, sm + P_WUT + 16384, 16384);
+        if constexpr (!PD) {
+            bulk_store(img + IMG_KT, sm + P_KQ, 8192);
+            bulk_store(img + IMG_KT + 8192, sm + P_KQ + 16384, 8192);
+        }
         bulk_commit();
     }
     if (tid == 32 && !failed) {
+        const uint32_t kt = PD ? sb + X_KT : sb + P_KQ;
+        const uint32_t ktlbo = PD ? 8192 : 16384;
         const uint32_t id1 = idesc_bf16_f32(128, 128, true, false);   // K~^T W
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem + TM_FP, sdesc_sw128(sb + P_KT + k * 2048, 8192, 1024),
+            mma_bf16(tmem + TM_FP, sdesc_sw128(kt + k * 2048, ktlbo, 1024),
                      sdesc_sw128(sb + P_WUT + k * 32, 16, 1024), id1, k > 0);
-        const uint32_t id2 = idesc_bf16_f32(64, 256, false, false);   // P [W | U]
+        const uint32_t id2 = idesc_bf16_f32(128, 64, false, false);   // W^T P^T, U^T P^T
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem + TM_PP, sdesc_sw128(sb + P_P + k * 32, 16, 1024),
-                     sdesc_sw128(sb + P_WUT + k * 32, 16, 1024), id2, k > 0);
+            mma_bf16(tmem + TM_PWT, sdesc_sw128(sb + P_WUT + k * 32, 16, 1024),
+                     sdesc_sw128(sb + P_P + k * 32, 16, 1024), id2, k > 0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem + TM_PUT, sdesc_sw128(sb + P_WUT + 16384 + k * 32, 16, 1024),
+                     sdesc_sw128(sb + P_P + k * 32, 16, 1024), id2, k > 0);
         mma_commit(&bars[3]);
     }
     wait(3, 0);
-    if (tid == 0) bulk_wait_read();   // the U^T rows become the P U staging
+    if (tid == 0) bulk_wait_read();   // the U^T rows become the Qp^T staging
     tc_fence_after();
     __syncthreads();
+    const int row = (warp & 3) * 32 + lane;
     if (warp < 4) {   // Phi = -K~^T W, row d; gamma_d
-        const int d = warp * 32 + lane;
-        float v[128];
-        ld_cols<128>(tmem + TM_FP + lane_off, v);
-        st_row128(sm + S_PHI, 16384, d, v, -1.f);
-        float gam;
-        if constexpr (PD) gam = expf(sC[d]);
-        else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
-        if (!failed) reinterpret_cast<float*>(img + IMG_GAM)[d] = gam;
-    } else {          // P U, row r = 16 (warp & 3) + lane
-        float v[128];
-        ld_cols<128>(tmem + TM_PP + lane_off + 128, v);
-        if (lane < 16) st_row128(sm + S_PU, 8192, 16 * (warp & 3) + lane, v, 1.f);
-    }
-    if (warp < 4) {   // Qp = Q e^G - P W, row r = 16 warp + lane
-        float v[128];
-        ld_cols<128>(tmem + TM_PP + lane_off, v);
-        const int r = 16 * warp + lane;
-        if (lane < 16) {
-            const float eg = gbuf[64 + r];
 #pragma unroll
-            for (int dd = 0; dd < D; ++dd) {
-                const float qb = PD ? ld_bf16(sm + X_QB + (dd >> 6) * 8192, r, dd & 63)
-                                    : eg * ld_bf16(sm + P_KQ + (dd >> 6) * 16384 + 8192, r, dd & 63);
-                v[dd] = qb - v[dd];
-            }
-            st_row128(sm + S_QP, 8192, r, v, 1.f);
+        for (int hh = 0; hh < 2; ++hh) {
+            float v[64];
+            ld_cols<64>(tmem + TM_FP + lane_off + 64 * hh, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_PHI + hh * 16384, row, j, v + 8 * j, -1.f);
         }
+        float gam;
+        if constexpr (PD) gam = expf(sC[row]);
+        else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
+        if (!failed) reinterpret_cast<float*>(img + IMG_GAM)[row] = gam;
+    } else {          // Qp^T = (Q e^G)^T - W^T P^T and (P U)^T = U^T P^T, row d / v
+        float v[64];
+        ld_cols<64>(tmem + TM_PWT + lane_off, v);
+        const int d = row;
+#pragma unroll
+        for (int r = 0; r < C; ++r) {
+            const float qb = PD ? ld_bf16(sm + X_QB + (d >> 6) * 8192, r, d & 63)
+                                : gbuf[64 + r] * ld_bf16(sm + P_KQ + (d >> 6) * 16384 + 8192, r, d & 63);
+            v[r] = qb - v[r];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_QPT, d, j, v + 8 * j, 1.f);
+        ld_cols<64>(tmem + TM_PUT + lane_off, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_PUT, row, j, v + 8 * j, 1.f);
     }
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
         if (!failed) {
             bulk_store(img + IMG_PHI, sm + S_PHI, 32768);
-            bulk_store(img + IMG_QP, sm + S_QP, 16384);
-            bulk_store(img + IMG_PU, sm + S_PU, 16384);
+            bulk_store(img + IMG_QP, sm + S_QPT, 16384);
+            bulk_store(img + IMG_PU, sm + S_PUT, 16384);
             bulk_commit();
         }
-        bulk_wait_all();
+        bulk_wait_read();
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, 256);
     }
 }
 
@@ -709,15 +723,17 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 constexpr uint32_t CH_PHI = 0;          // 2 slots of Phi   (32 KB each)
 constexpr uint32_t CH_KT = 65536;       // K~   (16 KB, one slot)
 constexpr uint32_t CH_UT = 81920;       // U^T  (16 KB, one slot)
-constexpr uint32_t CH_QP = 98304;       // 2 slots of Qp (16 KB each)
-constexpr uint32_t CH_PU = 131072;      // 2 slots of P U, then O in place for its TMA store
+constexpr uint32_t CH_QP = 98304;       // 2 slots of Qp^T (16 KB each); then the O tile for its TMA store
+constexpr uint32_t CH_PU = 131072;      // 2 slots of (P U)^T (16 KB each)
 constexpr uint32_t CH_HB = 163840;      // 2 slots of h (bf16) MN-major [d][64 v] x 2 blocks
 constexpr uint32_t CH_GAM = 229376;     // 2 slots of gamma (512 B each)
 constexpr uint32_t CH_BAR = 230400;
 constexpr uint32_t CH_SMEM = CH_BAR + 256 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
 
-constexpr int CH_THREADS = 448;   // 14 warps: loader, MMA, 4 output, 8 state
+constexpr int CH_THREADS = 480;   // 15 warps: loader, 2 MMA issuers, 4 output, 8 state
+constexpr int W_OUT = 3;          // first output warp
+constexpr int W_ST = 7;           // first state-pass warp
 
 // TMEM columns of the chain kernel (512 allocated).
 constexpr uint32_t TM_H = 0;      // state h, lanes d, 128 columns v (fp32, the state pass's own)
@@ -725,9 +741,9 @@ constexpr uint32_t TM_O = 128;    // O^T, lanes v, 2 slots of 64 columns r
 constexpr uint32_t TM_X = 256;    // X = K~^T U + Phi h, lanes d, 2 slots of 128 columns v
 
 enum ChainBar {
-    CB_IMG0, CB_IMG1, CB_KU, CB_QP0, CB_QP1, CB_PU0, CB_PU1,
-    CB_HREADY, CB_XFREE0, CB_XFREE1, CB_SDONE, CB_SFREE0, CB_SFREE1, CB_KUFREE,
-    CB_ODONE0, CB_ODONE1, CB_OFREE0, CB_OFREE1, CB_FINAL, CB_COUNT
+    CB_IMG0, CB_IMG1, CB_KU, CB_QP0, CB_QP1, CB_PU0, CB_PU1, CB_HREADY0, CB_HREADY1,
+    CB_XFREE0, CB_XFREE1, CB_SDONE, CB_SFREE0, CB_SFREE1, CB_KUFREE, CB_ODONE0, CB_ODONE1,
+    CB_OFREE0, CB_OFREE1, CB_HBFREE0, CB_HBFREE1, CB_FINAL, CB_OFINAL, CB_COUNT
 };
 static_assert(CB_COUNT * 8 <= 256, "barrier space");
 
@@ -736,8 +752,10 @@ static_assert(CB_COUNT * 8 <= 256, "barrier space");
 //   X_n = K~_n^T U_n (issued one chunk ahead) + Phi_n bf16(h_n)   in TMEM
 //   h_{n+1} = gamma_n h_n + X_n                                  (state pass, fp32)
 //   O_n^T = bf16(h_n)^T Qp_n^T,  O_n = O_n^T^T + (P U)_n          (output warps)
-// Every barrier that a role waits on is per slot or completes at most once
-// ahead of that wait, so no parity wait can fall two phases behind.
+// The state products and the output product come from two issuing threads, so
+// the output never holds up the serial chain.  Every barrier that a role waits
+// on is per slot or completes at most once ahead of that wait, so no parity
+// wait can fall two phases behind.
 __global__ void __maxnreg__(128)
 chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -757,7 +775,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
 
     if (tid == 0) {
         for (int i = 0; i < CB_COUNT; ++i)
-            mbar_init(&bars[i], (i == CB_HREADY || i == CB_XFREE0 || i == CB_XFREE1) ? 8 : 1);
+            mbar_init(&bars[i], (i == CB_HREADY0 || i == CB_HREADY1 || i == CB_XFREE0 || i == CB_XFREE1) ? 8 : 1);
         fence_mbar_init();
         prefetch_tmap(&omap);
     }
@@ -775,6 +793,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
         __syncwarp();
     };
     auto img = [&](int nl) { return wsh + (size_t)nl * IMG_BYTES; };
+    const uint64_t d_hb = sdesc_sw128(sb + CH_HB, 16384, 1024);
 
     if (warp == 0) {
         // =========================== loader: Phi + gamma (2 slots) and K~, U^T
@@ -794,17 +813,14 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
             if (failed) atomicOr(p.status, kStatusTimeout);
         }
     } else if (warp == 1) {
-        // =========================== MMA issuer (descriptors built once; a k-step
-        // adds its byte offset / 16 to the start-address field)
+        // =========================== state-product issuer (descriptors built once;
+        // a k-step adds its byte offset / 16 to the start-address field)
         const bool leader = lane == 0;
         const uint32_t id_ku = idesc_bf16_f32(128, 128, true, false);   // K~^T U
         const uint32_t id_ph = idesc_bf16_f32(128, 128, false, true);   // Phi h_bf16
-        const uint32_t id_o = idesc_bf16_f32(128, 64, true, false);     // h^T Qp^T
         const uint64_t d_phi = sdesc_sw128(sb + CH_PHI, 16, 1024);
         const uint64_t d_kt = sdesc_sw128(sb + CH_KT, 8192, 1024);
         const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
-        const uint64_t d_hb = sdesc_sw128(sb + CH_HB, 16384, 1024);
-        const uint64_t d_qp = sdesc_sw128(sb + CH_QP, 16, 1024);
         // K~^T U of chunk nl into X slot nl & 1 once K~, U^T are in and the state
         // pass has read X of chunk nl - 2 there
         auto issue_ku = [&](int nl) {
@@ -824,7 +840,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            wait(CB_HREADY, nl & 1);
+            wait(CB_HREADY0 + s, (nl >> 1) & 1);
             wait(CB_IMG0 + s, (nl >> 1) & 1);
             tc_fence_after();
             if (leader && !failed) {
@@ -836,6 +852,20 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
                 mma_commit(&bars[CB_SFREE0 + s]);
             }
             if (nl + 1 < NC) issue_ku(nl + 1);
+        }
+        if (leader) mma_commit(&bars[CB_FINAL]);
+        int final_failed = 0;
+        if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+    } else if (warp == 2) {
+        // =========================== output-product issuer: O^T = h^T Qp^T
+        const bool leader = lane == 0;
+        const uint32_t id_o = idesc_bf16_f32(128, 64, true, true);
+        const uint64_t d_qp = sdesc_sw128(sb + CH_QP, 8192, 1024);
+#pragma unroll 1
+        for (int nl = 0; nl < NC; ++nl) {
+            const int s = nl & 1;
+            wait(CB_HREADY0 + s, (nl >> 1) & 1);
             wait(CB_QP0 + s, (nl >> 1) & 1);
             if (nl >= 2) wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
             tc_fence_after();
@@ -843,52 +873,57 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     mma_bf16(tmem + TM_O + 64 * s, d_hb + ((s * 32768 + k * 2048) >> 4),
-                             d_qp + ((s * 16384 + (k >> 2) * 8192 + (k & 3) * 32) >> 4), id_o, k > 0);
+                             d_qp + ((s * 16384 + k * 2048) >> 4), id_o, k > 0);
                 mma_commit(&bars[CB_ODONE0 + s]);
+                mma_commit(&bars[CB_HBFREE0 + s]);
             }
         }
-        // nothing issued by this warp may still run when TMEM is released
-        if (leader) mma_commit(&bars[CB_FINAL]);
+        if (leader) mma_commit(&bars[CB_OFINAL]);
         int final_failed = 0;
-        if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
+        if (!mbar_wait(&bars[CB_OFINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
-    } else if (warp < 6) {
-        // =========================== output: O = (O^T)^T + P U in place, TMA store
+    } else if (warp < W_ST) {
+        // =========================== output: O + P U into the Qp slot, TMA store
         const int v = (warp & 3) * 32 + lane;
-        const bool leader = warp == 2 && lane == 0;
-        auto load_qp = [&](int nl) {
-            mbar_arrive_expect_tx(&bars[CB_QP0 + (nl & 1)], 16384);
-            bulk_load(sm + CH_QP + (nl & 1) * 16384, img(nl) + IMG_QP, 16384, &bars[CB_QP0 + (nl & 1)]);
-        };
-        auto load_pu = [&](int nl) {
-            mbar_arrive_expect_tx(&bars[CB_PU0 + (nl & 1)], 16384);
-            bulk_load(sm + CH_PU + (nl & 1) * 16384, img(nl) + IMG_PU, 16384, &bars[CB_PU0 + (nl & 1)]);
+        const bool leader = warp == W_OUT && lane == 0;
+        auto load_qp_pu = [&](int nl) {
+            const int s = nl & 1;
+            mbar_arrive_expect_tx(&bars[CB_QP0 + s], 16384);
+            bulk_load(sm + CH_QP + s * 16384, img(nl) + IMG_QP, 16384, &bars[CB_QP0 + s]);
+            mbar_arrive_expect_tx(&bars[CB_PU0 + s], 16384);
+            bulk_load(sm + CH_PU + s * 16384, img(nl) + IMG_PU, 16384, &bars[CB_PU0 + s]);
         };
         if (leader) {
-            for (int nl = 0; nl < 2 && nl < NC; ++nl) {
-                load_qp(nl);
-                load_pu(nl);
-            }
+            for (int nl = 0; nl < 2 && nl < NC; ++nl) load_qp_pu(nl);
         }
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            wait(CB_ODONE0 + s, (nl >> 1) & 1);
-            if (leader && !failed && nl + 2 < NC) load_qp(nl + 2);   // O of chunk nl is done with Qp
+            wait(CB_ODONE0 + s, (nl >> 1) & 1);   // O is in TMEM; Qp slot s is free
             wait(CB_PU0 + s, (nl >> 1) & 1);
             tc_fence_after();
-            uint8_t* pu = sm + CH_PU + s * 16384 + (v >> 6) * 8192;
+            const uint8_t* pu = sm + CH_PU + s * 16384 + v * 128;   // (P U)^T row v
+            uint8_t* ot = sm + CH_QP + s * 16384 + (v >> 6) * 8192;  // O tile [r][64 v] x 2
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                float ov[32], pv[32];
+                float ov[32];
                 ld_cols<32>(tmem + TM_O + 64 * s + 32 * half + lane_off, ov);
 #pragma unroll
-                for (int r = 0; r < 32; ++r)
-                    pv[r] = ld_bf16(pu, 32 * half + r, v & 63);
+                for (int j = 0; j < 4; ++j) {
+                    const int jj = 4 * half + j;
+                    uint4 raw = *reinterpret_cast<const uint4*>(pu + ((jj ^ (v & 7)) * 16));
+                    const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(e2[e]);
+                        ov[8 * j + 2 * e] += f.x;
+                        ov[8 * j + 2 * e + 1] += f.y;
+                    }
+                }
 #pragma unroll
                 for (int r = 0; r < 32; ++r)
-                    *reinterpret_cast<__nv_bfloat16*>(pu + sw128_offset(32 * half + r, v & 63)) =
-                        __float2bfloat16_rn(ov[r] + pv[r]);
+                    *reinterpret_cast<__nv_bfloat16*>(ot + sw128_offset(32 * half + r, v & 63)) =
+                        __float2bfloat16_rn(ov[r]);
             }
             fence_async_smem();
             tc_fence_before();
@@ -897,12 +932,12 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
                 mbar_arrive(&bars[CB_OFREE0 + s]);
                 if (!failed) {
                     const int t0 = (p.chunk0 + nl) * C;
-                    tma_store_3d(&omap, sm + CH_PU + s * 16384, h * D, t0, b);
-                    tma_store_3d(&omap, sm + CH_PU + s * 16384 + 8192, h * D + 64, t0, b);
+                    tma_store_3d(&omap, sm + CH_QP + s * 16384, h * D, t0, b);
+                    tma_store_3d(&omap, sm + CH_QP + s * 16384 + 8192, h * D + 64, t0, b);
                     bulk_commit();
                     if (nl + 2 < NC) {
                         bulk_wait_read();
-                        load_pu(nl + 2);
+                        load_qp_pu(nl + 2);
                     }
                 }
             }
@@ -911,7 +946,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
     } else {
         // =========================== state pass: h' = gamma h + X -> bf16 operand
         const int d = (warp & 3) * 32 + lane;
-        const int c = (warp - 6) >> 2;              // column half
+        const int c = (warp - W_ST) >> 2;           // column half
         const uint32_t haddr = tmem + TM_H + lane_off + 64 * c;
         float gam = 1.f;                            // gamma of the chunk before
         float hv[64];
@@ -940,6 +975,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[CB_XFREE0 + ((nl - 1) & 1)]);
             }
+            if (nl >= 2) wait(CB_HBFREE0 + s, ((nl - 2) >> 1) & 1);   // O of chunk nl - 2 is done with it
             uint8_t* hb = sm + CH_HB + s * 32768 + c * 16384;
 #pragma unroll
             for (int j = 0; j < 8; ++j) st_row_chunk(hb, d, j, hv + 8 * j, 1.f);
@@ -949,7 +985,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
             gam = reinterpret_cast<const float*>(sm + CH_GAM + s * 512)[d];
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CB_HREADY]);
+            if (lane == 0) mbar_arrive(&bars[CB_HREADY0 + s]);
             st_cols<64>(haddr, hv);                 // the fp32 state, read back next chunk
             tmem_wait_st();
         }
