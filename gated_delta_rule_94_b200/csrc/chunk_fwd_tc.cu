@@ -61,7 +61,7 @@ constexpr uint32_t IMG_QP = 65536;     // Qp^T [128 d][64 r]     (MN-major B)
 constexpr uint32_t IMG_PU = 81920;     // (P U)^T [128 v][64 r]
 constexpr uint32_t IMG_GAM = 98304;    // gamma fp32 [128]
 constexpr uint32_t IMG_BYTES = 98816;
-constexpr size_t WAVE_BYTES = size_t(40) << 20;   // workspace per wave (kept L2-resident)
+constexpr size_t WAVE_BYTES = size_t(32) << 20;   // workspace per wave buffer (kept L2-resident)
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
@@ -90,6 +90,13 @@ __device__ __forceinline__ void st_row128(uint8_t* tile, uint32_t bstride, int r
 __device__ __forceinline__ float ld_bf16(const uint8_t* tile, int row, int col) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + sw128_offset(row, col)));
 }
+
+// Programmatic dependent launch: let the next kernel in the stream start now /
+// wait until the previous one has completed and its writes are visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -308,6 +315,15 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     __shared__ uint32_t s_tmem;
     constexpr bool PD = GATE == kGatePerDim;
 
+    // The grid's last block only waits for the kernel before it (the previous
+    // wave's chain): this grid then completes after that chain, so the chain of
+    // this wave -- and the prep of the next wave, which reuses the previous
+    // wave's image buffer -- start only once it is done.  The other blocks write
+    // this wave's buffer, which nothing in flight reads.
+    if (blockIdx.x == gridDim.x - 1) {
+        pdl_wait();
+        return;
+    }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, T = p.T;
     const int bh = blockIdx.x / p.nchunks, nl = blockIdx.x % p.nchunks;
@@ -743,7 +759,8 @@ constexpr uint32_t TM_X = 256;    // X = K~^T U + Phi h, lanes d, 2 slots of 128
 enum ChainBar {
     CB_IMG0, CB_IMG1, CB_KU, CB_QP0, CB_QP1, CB_PU0, CB_PU1, CB_HREADY0, CB_HREADY1,
     CB_XFREE0, CB_XFREE1, CB_SDONE, CB_SFREE0, CB_SFREE1, CB_KUFREE, CB_ODONE0, CB_ODONE1,
-    CB_OFREE0, CB_OFREE1, CB_HBFREE0, CB_HBFREE1, CB_FINAL, CB_OFINAL, CB_COUNT
+    CB_OFREE0, CB_OFREE1, CB_HBFREE0, CB_HBFREE1, CB_FINAL, CB_OFINAL, CB_S0, CB_SDONEO0,
+    CB_SDONEO1, CB_COUNT
 };
 static_assert(CB_COUNT * 8 <= 256, "barrier space");
 
@@ -783,6 +800,10 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
         tmem_alloc(&s_tmem, 512);
         tmem_relinquish();
     }
+    // the next wave's prep may start on the SMs this grid leaves idle; the
+    // images and the carried state of this wave are read only after the wait
+    pdl_launch_dependents();
+    pdl_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -798,6 +819,10 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
     if (warp == 0) {
         // =========================== loader: Phi + gamma (2 slots) and K~, U^T
         if (lane == 0) {
+            if (p.s0 && NC > 0) {   // the entering state, one 64 KB block, staged over the h slots
+                mbar_arrive_expect_tx(&bars[CB_S0], 65536);
+                bulk_load(sm + CH_HB, p.s0 + (size_t)bh * D * D, 65536, &bars[CB_S0]);
+            }
 #pragma unroll 1
             for (int nl = 0; nl < NC; ++nl) {
                 const int s = nl & 1;
@@ -850,6 +875,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
                              d_hb + ((s * 32768 + k * 2048) >> 4), id_ph, true);
                 mma_commit(&bars[CB_SDONE]);
                 mma_commit(&bars[CB_SFREE0 + s]);
+                mma_commit(&bars[CB_SDONEO0 + s]);
             }
             if (nl + 1 < NC) issue_ku(nl + 1);
         }
@@ -858,14 +884,16 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
         if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     } else if (warp == 2) {
-        // =========================== output-product issuer: O^T = h^T Qp^T
+        // =========================== output-product issuer: O^T = h^T Qp^T, issued
+        // once the state product of the chunk is done, so that it fills the
+        // tensor pipe while the state pass works instead of delaying the chain
         const bool leader = lane == 0;
         const uint32_t id_o = idesc_bf16_f32(128, 64, true, true);
         const uint64_t d_qp = sdesc_sw128(sb + CH_QP, 8192, 1024);
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            wait(CB_HREADY0 + s, (nl >> 1) & 1);
+            wait(CB_SDONEO0 + s, (nl >> 1) & 1);
             wait(CB_QP0 + s, (nl >> 1) & 1);
             if (nl >= 2) wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
             tc_fence_after();
@@ -961,11 +989,18 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
             if (nl == 0) {
-                const float* s0 = p.s0 ? p.s0 + ((size_t)bh * D + d) * D + 64 * c : nullptr;
+                if (p.s0) {   // row d of the staged state
+                    wait(CB_S0, 0);
+                    const float* row = reinterpret_cast<const float*>(sm + CH_HB) + d * D + 64 * c;
 #pragma unroll
-                for (int e = 0; e < 64; e += 4) {
-                    const float4 x = s0 ? *reinterpret_cast<const float4*>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    hv[e] = x.x; hv[e + 1] = x.y; hv[e + 2] = x.z; hv[e + 3] = x.w;
+                    for (int j = 0; j < 16; ++j) {
+                        const float4 x = *reinterpret_cast<const float4*>(row + 4 * j);
+                        hv[4 * j] = x.x; hv[4 * j + 1] = x.y; hv[4 * j + 2] = x.z; hv[4 * j + 3] = x.w;
+                    }
+                    named_bar(1, 256);   // everyone has read the staging before h slot 0 is written
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) hv[e] = 0.f;
                 }
             } else {
                 wait(CB_SDONE, (nl - 1) & 1);
@@ -989,15 +1024,26 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
             st_cols<64>(haddr, hv);                 // the fp32 state, read back next chunk
             tmem_wait_st();
         }
-        if (NC > 0) {   // final state
+        if (NC > 0) {   // final state, staged over the Phi slots (free once the last
+                        // state product is done) and written by one bulk copy
             wait(CB_SDONE, (NC - 1) & 1);
             tc_fence_after();
             advance(NC);
-            if (!failed && p.s_out) {
-                float* dst = p.s_out + ((size_t)bh * D + d) * D + 64 * c;
+            if (p.s_out) {
+                float* row = reinterpret_cast<float*>(sm + CH_PHI) + d * D + 64 * c;
 #pragma unroll
-                for (int e = 0; e < 64; e += 4)
-                    *reinterpret_cast<float4*>(dst + e) = make_float4(hv[e], hv[e + 1], hv[e + 2], hv[e + 3]);
+                for (int j = 0; j < 16; ++j)
+                    *reinterpret_cast<float4*>(row + 4 * j) =
+                        make_float4(hv[4 * j], hv[4 * j + 1], hv[4 * j + 2], hv[4 * j + 3]);
+                fence_async_smem();
+                named_bar(1, 256);
+                if (warp == W_ST && lane == 0) {
+                    if (!failed) {
+                        bulk_store(p.s_out + (size_t)bh * D * D, sm + CH_PHI, 65536);
+                        bulk_commit();
+                    }
+                    bulk_wait_all();
+                }
             }
         }
     }
@@ -1043,8 +1089,8 @@ size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H, int gate) {
     const int nbh = B * H;
     const int cw = wave_chunks(nbh, NC);
     const int nw = (NC + cw - 1) / cw;
-    size_t bytes = (size_t)nbh * cw * IMG_BYTES;
-    if (nw > 1) bytes += (size_t)nbh * D * D * sizeof(float);   // state between waves
+    size_t bytes = (size_t)nbh * cw * IMG_BYTES * (nw > 1 ? 2 : 1);   // two alternating buffers
+    if (nw > 1) bytes += (size_t)nbh * D * D * sizeof(float);           // state between waves
     return bytes;
 }
 
@@ -1072,18 +1118,39 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s,
     const int nbh = p0.B * p0.H;
     const int cw = wave_chunks(nbh, NC);
     const int nw = (NC + cw - 1) / cw;
-    float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + (size_t)nbh * cw * IMG_BYTES) : nullptr;
+    const size_t buf_bytes = (size_t)nbh * cw * IMG_BYTES;
+    float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + 2 * buf_bytes) : nullptr;
+    // Every launch but the first may start before its predecessor ends
+    // (programmatic dependent launch); the kernels order themselves with
+    // griddepcontrol (see chunk_prep_kernel and chunk_chain_kernel).
+    cudaLaunchAttribute pdl;
+    pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl.val.programmaticStreamSerializationAllowed = 1;
     for (int w = 0; w < nw; ++w) {
         ChunkParams p = p0;
+        p.ws = p0.ws + (size_t)(w & 1) * buf_bytes;
         p.cw = cw;
         p.ws_chunk = (int)IMG_BYTES;
         p.chunk0 = w * cw;
         p.nchunks = (w + 1 < nw) ? cw : NC - w * cw;
         p.s0 = (w == 0) ? p0.s0 : carry;
         p.s_out = (w + 1 == nw) ? p0.s_out : carry;
-        prep<<<(unsigned)(nbh * p.nchunks), NPR, prep_smem, s>>>(maps, p);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(nbh * p.nchunks + 1));
+        cfg.blockDim = dim3(NPR);
+        cfg.dynamicSmemBytes = prep_smem;
+        cfg.stream = s;
+        cfg.attrs = &pdl;
+        cfg.numAttrs = w > 0 ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, prep, maps, p);
+        if (e != cudaSuccess) return e;
         ++*launches;
-        chunk_chain_kernel<<<(unsigned)nbh, CH_THREADS, CH_SMEM, s>>>(omap, p);
+        cfg.gridDim = dim3((unsigned)nbh);
+        cfg.blockDim = dim3(CH_THREADS);
+        cfg.dynamicSmemBytes = CH_SMEM;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, chunk_chain_kernel, omap, p);
+        if (e != cudaSuccess) return e;
         ++*launches;
     }
     return cudaGetLastError();
