@@ -22,7 +22,7 @@
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(96) << 20;   // 96 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(128) << 20;   // 128 MiB
 
 static __device__ __align__(256) unsigned char gdn_noalloc_scratch[kNoAllocScratchBytes];
 

@@ -61,7 +61,8 @@ constexpr uint32_t IMG_QP = 65536;     // Qp^T [128 d][64 r]     (MN-major B)
 constexpr uint32_t IMG_PU = 81920;     // (P U)^T [128 v][64 r]
 constexpr uint32_t IMG_GAM = 98304;    // gamma fp32 [128]
 constexpr uint32_t IMG_BYTES = 98816;
-constexpr size_t WAVE_BYTES = size_t(32) << 20;   // workspace per wave buffer (kept L2-resident)
+constexpr size_t WAVE_BYTES = size_t(56) << 20;   // cap of one wave's image buffer
+constexpr int PREP_SLOTS = 2 * 148;                // prep CTAs resident at once on a B200
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
@@ -1067,13 +1068,20 @@ bool make_maps(const ChunkParams& p, bool perdim, PrepMaps* m) {
     return ok;
 }
 
-// Chunk slots per (batch, head) of one wave: as many as keep the wave's
-// workspace near WAVE_BYTES (L2-resident), at least one.
+// Chunks per (batch, head) of one wave: the wave's image buffer stays within
+// WAVE_BYTES, and among such lengths the longest whose prep CTAs fill their
+// last round of resident CTAs to at least 90 % (a nearly empty last round costs
+// a whole CTA lifetime); at least one.
 int wave_chunks(int nbh, int NC) {
-    long long cw = (long long)(WAVE_BYTES / ((size_t)nbh * IMG_BYTES));
-    if (cw < 1) cw = 1;
-    if (cw > NC) cw = NC;
-    return (int)cw;
+    long long cmax = (long long)(WAVE_BYTES / ((size_t)nbh * IMG_BYTES));
+    if (cmax < 1) cmax = 1;
+    if (cmax > NC) cmax = NC;
+    for (long long c = cmax; c >= 1; --c) {
+        const long long items = c * nbh;
+        const long long rounds = (items + PREP_SLOTS - 1) / PREP_SLOTS;
+        if (c == NC || 10 * items >= 9 * rounds * PREP_SLOTS) return (int)c;
+    }
+    return (int)cmax;
 }
 
 }  // namespace

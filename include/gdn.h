@@ -149,7 +149,7 @@ GDN_API const char* gdn_status_string(gdn_status s);
  *
  * Same arguments and results as gdn_chunk_fwd, minus the workspace: the
  * library supplies it from a fixed scratch array of
- * gdn_chunk_fwd_noalloc_scratch_bytes() bytes (96 MiB) that every GPU loading
+ * gdn_chunk_fwd_noalloc_scratch_bytes() bytes (128 MiB) that every GPU loading
  * the library reserves until the process exits.  For callers that cannot call
  * cudaMalloc -- inside a host framework that owns all device memory, or on a
  * path where allocation is forbidden.
