@@ -67,7 +67,7 @@ const char* gdn_chunk_fwd_kernel_name(int Dk, int Dv, gdn_gate gate_kind, gdn_dt
     if (!supported_dim(Dk) || !supported_dim(Dv)) return nullptr;
     if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return nullptr;
     if (dtype == GDN_BF16 && gdn::chunk_fwd_tc_supported(Dk, Dv, gate_kind))
-        return "chunk_fwd_tc_kernel";
+        return "chunk_prep_kernel,chunk_chain_kernel";
     if (dtype == GDN_BF16 || dtype == GDN_F32) return "chunk_fwd_simt_kernel";
     return nullptr;
 }

@@ -180,8 +180,9 @@ GDN_API size_t gdn_chunk_fwd_noalloc_scratch_bytes(void);
  * all entry points), counted on the host at each successful launch. */
 GDN_API unsigned long long gdn_kernel_launch_count(void);
 
-/* Name of the kernel gdn_chunk_fwd launches for these arguments, or NULL if
- * the combination is unsupported.  Static string; never freed. */
+/* Names of the kernels gdn_chunk_fwd launches for these arguments (comma
+ * separated when it launches more than one), or NULL if the combination is
+ * unsupported.  Static string; never freed. */
 GDN_API const char* gdn_chunk_fwd_kernel_name(int Dk, int Dv, gdn_gate gate_kind,
                                               gdn_dtype dtype);
 
