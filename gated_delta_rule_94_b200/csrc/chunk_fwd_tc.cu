@@ -99,6 +99,16 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Drop `bytes` (a multiple of 128) of L2 lines at p without writing them back:
+// for data that is dead once read (a step image after its chain has loaded it),
+// so the L2 does not spend DRAM bandwidth evicting it.  One warp, lanes split
+// the lines.
+__device__ __forceinline__ void l2_discard(const void* p, uint32_t bytes, int lane) {
+    const char* c = static_cast<const char*>(p);
+    for (uint32_t off = 128u * lane; off < bytes; off += 128u * 32u)
+        asm volatile("discard.global.L2 [%0], 128;" ::"l"(c + off) : "memory");
+}
+
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
@@ -312,7 +322,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     float* Af = reinterpret_cast<float*>(sm + P_AF);
     float* Tf = reinterpret_cast<float*>(sm + P_TF);
     float* gbuf = reinterpret_cast<float*>(sm + P_GATE);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P_BAR);   // ld, s, wu, f
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P_BAR);   // kq, s, wu, f, v
     __shared__ uint32_t s_tmem;
     constexpr bool PD = GATE == kGatePerDim;
 
@@ -349,17 +359,20 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     int* sFlag = reinterpret_cast<int*>(sEcm + 128);
 
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         if constexpr (PD) *sFlag = 0;
-        mbar_arrive_expect_tx(&bars[0], (PD ? 8 : 6) * 8192);
+        // K, Q (and g) first: the Gram product needs only them; V lands behind
+        mbar_arrive_expect_tx(&bars[0], (PD ? 6 : 4) * 8192);
+        mbar_arrive_expect_tx(&bars[4], 2 * 8192);
         for (int blk = 0; blk < 2; ++blk) {
             tma_load_3d(sm + P_KQ + blk * 16384, &maps.k, &bars[0], h * D + 64 * blk, n * C, b);
             tma_load_3d(sm + P_KQ + blk * 16384 + 8192, &maps.q, &bars[0], h * D + 64 * blk, n * C, b);
-            tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[0], h * D + 64 * blk, n * C, b);
             if constexpr (PD)
                 tma_load_3d(sm + X_G16 + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b);
         }
+        for (int blk = 0; blk < 2; ++blk)
+            tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b);
     }
     if (warp == 0) {
         tmem_alloc(&s_tmem, 256);
@@ -617,6 +630,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_WT, sdesc_sw128(ka + k * 2048, klbo, 1024),
                      sdesc_sw128(sb + P_TW + k * 32, 16, 1024), id, k > 0);
+        if (!mbar_wait(&bars[4], 0, &failed)) atomicOr(p.status, kStatusTimeout);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_UT, sdesc_sw128(sb + P_V + k * 2048, 8192, 1024),
@@ -688,7 +702,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     tc_fence_after();
     __syncthreads();
     const int row = (warp & 3) * 32 + lane;
-    if (warp < 4) {   // Phi = -K~^T W, row d; gamma_d
+    if (warp < 4) {   // Phi = -K~^T W, row d (stored as soon as it is staged), then (P U)^T
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             float v[64];
@@ -696,11 +710,17 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_PHI + hh * 16384, row, j, v + 8 * j, -1.f);
         }
-        float gam;
-        if constexpr (PD) gam = expf(sC[row]);
-        else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
-        if (!failed) reinterpret_cast<float*>(img + IMG_GAM)[row] = gam;
-    } else {          // Qp^T = (Q e^G)^T - W^T P^T and (P U)^T = U^T P^T, row d / v
+        fence_async_smem();
+        named_bar(1, 128);
+        if (tid == 0 && !failed) {
+            bulk_store(img + IMG_PHI, sm + S_PHI, 32768);
+            bulk_commit();
+        }
+        float v[64];
+        ld_cols<64>(tmem + TM_PUT + lane_off, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_PUT, row, j, v + 8 * j, 1.f);
+    } else {          // Qp^T = (Q e^G)^T - W^T P^T, row d; gamma_d
         float v[64];
         ld_cols<64>(tmem + TM_PWT + lane_off, v);
         const int d = row;
@@ -712,15 +732,15 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_QPT, d, j, v + 8 * j, 1.f);
-        ld_cols<64>(tmem + TM_PUT + lane_off, v);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_PUT, row, j, v + 8 * j, 1.f);
+        float gam;
+        if constexpr (PD) gam = expf(sC[d]);
+        else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
+        if (!failed) reinterpret_cast<float*>(img + IMG_GAM)[d] = gam;
     }
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
         if (!failed) {
-            bulk_store(img + IMG_PHI, sm + S_PHI, 32768);
             bulk_store(img + IMG_QP, sm + S_QPT, 16384);
             bulk_store(img + IMG_PU, sm + S_PUT, 16384);
             bulk_commit();
@@ -748,9 +768,12 @@ constexpr uint32_t CH_BAR = 230400;
 constexpr uint32_t CH_SMEM = CH_BAR + 256 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
 
-constexpr int CH_THREADS = 480;   // 15 warps: loader, 2 MMA issuers, 4 output, 8 state
+constexpr int CH_THREADS = 736;   // 23 warps: loader, 2 MMA issuers, 4 output, 16 state
 constexpr int W_OUT = 3;          // first output warp
 constexpr int W_ST = 7;           // first state-pass warp
+constexpr int N_ST = 16;          // state-pass warps: lane quarter x column quarter
+// Registers: warps spread over the SM's four sub-partitions of 16 K registers
+// each, so 23 warps (six on some sub-partitions) allow at most 85 a thread.
 
 // TMEM columns of the chain kernel (512 allocated).
 constexpr uint32_t TM_H = 0;      // state h, lanes d, 128 columns v (fp32, the state pass's own)
@@ -774,7 +797,7 @@ static_assert(CB_COUNT * 8 <= 256, "barrier space");
 // the output never holds up the serial chain.  Every barrier that a role waits
 // on is per slot or completes at most once ahead of that wait, so no parity
 // wait can fall two phases behind.
-__global__ void __maxnreg__(128)
+__global__ void __maxnreg__(80)
 chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -793,7 +816,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
 
     if (tid == 0) {
         for (int i = 0; i < CB_COUNT; ++i)
-            mbar_init(&bars[i], (i == CB_HREADY0 || i == CB_HREADY1 || i == CB_XFREE0 || i == CB_XFREE1) ? 8 : 1);
+            mbar_init(&bars[i], (i == CB_HREADY0 || i == CB_HREADY1 || i == CB_XFREE0 || i == CB_XFREE1) ? N_ST : 1);
         fence_mbar_init();
         prefetch_tmap(&omap);
     }
@@ -818,25 +841,36 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
     const uint64_t d_hb = sdesc_sw128(sb + CH_HB, 16384, 1024);
 
     if (warp == 0) {
-        // =========================== loader: Phi + gamma (2 slots) and K~, U^T
-        if (lane == 0) {
-            if (p.s0 && NC > 0) {   // the entering state, one 64 KB block, staged over the h slots
-                mbar_arrive_expect_tx(&bars[CB_S0], 65536);
-                bulk_load(sm + CH_HB, p.s0 + (size_t)bh * D * D, 65536, &bars[CB_S0]);
-            }
+        // =========================== loader: Phi + gamma (2 slots) and K~, U^T;
+        // the images it has seen consumed are dropped from L2
+        if (lane == 0 && p.s0 && NC > 0) {   // the entering state, one 64 KB block, staged over the h slots
+            mbar_arrive_expect_tx(&bars[CB_S0], 65536);
+            bulk_load(sm + CH_HB, p.s0 + (size_t)bh * D * D, 65536, &bars[CB_S0]);
+        }
 #pragma unroll 1
-            for (int nl = 0; nl < NC; ++nl) {
-                const int s = nl & 1;
-                if (nl >= 2 && !mbar_wait(&bars[CB_SFREE0 + s], ((nl - 2) >> 1) & 1, &failed)) break;
+        for (int nl = 0; nl < NC; ++nl) {
+            const int s = nl & 1;
+            if (nl >= 2) {
+                wait(CB_SFREE0 + s, ((nl - 2) >> 1) & 1);
+                if (failed) break;
+                l2_discard(img(nl - 2) + IMG_PHI, 32768, lane);
+                l2_discard(img(nl - 2) + IMG_GAM, 512, lane);
+            }
+            if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[CB_IMG0 + s], 32768 + 512);
                 bulk_load(sm + CH_PHI + s * 32768, img(nl) + IMG_PHI, 32768, &bars[CB_IMG0 + s]);
                 bulk_load(sm + CH_GAM + s * 512, img(nl) + IMG_GAM, 512, &bars[CB_IMG0 + s]);
-                if (nl >= 1 && !mbar_wait(&bars[CB_KUFREE], (nl - 1) & 1, &failed)) break;
+            }
+            if (nl >= 1) {
+                wait(CB_KUFREE, (nl - 1) & 1);
+                if (failed) break;
+                l2_discard(img(nl - 1) + IMG_KT, 32768, lane);   // K~ and U^T
+            }
+            if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[CB_KU], 32768);
                 bulk_load(sm + CH_KT, img(nl) + IMG_KT, 16384, &bars[CB_KU]);
                 bulk_load(sm + CH_UT, img(nl) + IMG_UT, 16384, &bars[CB_KU]);
             }
-            if (failed) atomicOr(p.status, kStatusTimeout);
         }
     } else if (warp == 1) {
         // =========================== state-product issuer (descriptors built once;
@@ -957,6 +991,10 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
             fence_async_smem();
             tc_fence_before();
             named_bar(2, 128);
+            if (warp == W_OUT) {   // both images were loaded and read: drop them from L2
+                l2_discard(img(nl) + IMG_QP, 16384, lane);
+                l2_discard(img(nl) + IMG_PU, 16384, lane);
+            }
             if (leader) {
                 mbar_arrive(&bars[CB_OFREE0 + s]);
                 if (!failed) {
@@ -975,16 +1013,16 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
     } else {
         // =========================== state pass: h' = gamma h + X -> bf16 operand
         const int d = (warp & 3) * 32 + lane;
-        const int c = (warp - W_ST) >> 2;           // column half
-        const uint32_t haddr = tmem + TM_H + lane_off + 64 * c;
+        const int c = (warp - W_ST) >> 2;           // column quarter
+        const uint32_t haddr = tmem + TM_H + lane_off + 32 * c;
         float gam = 1.f;                            // gamma of the chunk before
-        float hv[64];
+        float hv[32];
         auto advance = [&](int nl) {                // hv = gamma_{nl-1} h_{nl-1} + X_{nl-1}
-            float xv[64];
-            ld_cols<64>(haddr, hv);
-            ld_cols<64>(tmem + TM_X + 128 * ((nl - 1) & 1) + lane_off + 64 * c, xv);
+            float xv[32];
+            ld_cols<32>(haddr, hv);
+            ld_cols<32>(tmem + TM_X + 128 * ((nl - 1) & 1) + lane_off + 32 * c, xv);
 #pragma unroll
-            for (int e = 0; e < 64; ++e) hv[e] = fmaf(gam, hv[e], xv[e]);
+            for (int e = 0; e < 32; ++e) hv[e] = fmaf(gam, hv[e], xv[e]);
         };
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
@@ -992,16 +1030,16 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
             if (nl == 0) {
                 if (p.s0) {   // row d of the staged state
                     wait(CB_S0, 0);
-                    const float* row = reinterpret_cast<const float*>(sm + CH_HB) + d * D + 64 * c;
+                    const float* row = reinterpret_cast<const float*>(sm + CH_HB) + d * D + 32 * c;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
+                    for (int j = 0; j < 8; ++j) {
                         const float4 x = *reinterpret_cast<const float4*>(row + 4 * j);
                         hv[4 * j] = x.x; hv[4 * j + 1] = x.y; hv[4 * j + 2] = x.z; hv[4 * j + 3] = x.w;
                     }
-                    named_bar(1, 256);   // everyone has read the staging before h slot 0 is written
+                    named_bar(1, 32 * N_ST);   // everyone has read the staging before h slot 0 is written
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) hv[e] = 0.f;
+                    for (int e = 0; e < 32; ++e) hv[e] = 0.f;
                 }
             } else {
                 wait(CB_SDONE, (nl - 1) & 1);
@@ -1012,9 +1050,9 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
                 if (lane == 0) mbar_arrive(&bars[CB_XFREE0 + ((nl - 1) & 1)]);
             }
             if (nl >= 2) wait(CB_HBFREE0 + s, ((nl - 2) >> 1) & 1);   // O of chunk nl - 2 is done with it
-            uint8_t* hb = sm + CH_HB + s * 32768 + c * 16384;
+            uint8_t* hb = sm + CH_HB + s * 32768 + (c >> 1) * 16384;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) st_row_chunk(hb, d, j, hv + 8 * j, 1.f);
+            for (int j = 0; j < 4; ++j) st_row_chunk(hb, d, 4 * (c & 1) + j, hv + 8 * j, 1.f);
             // gamma of this chunk before HREADY: its slot is refilled only after
             // the MMA that HREADY releases
             wait(CB_IMG0 + s, (nl >> 1) & 1);
@@ -1022,7 +1060,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[CB_HREADY0 + s]);
-            st_cols<64>(haddr, hv);                 // the fp32 state, read back next chunk
+            st_cols<32>(haddr, hv);                 // the fp32 state, read back next chunk
             tmem_wait_st();
         }
         if (NC > 0) {   // final state, staged over the Phi slots (free once the last
@@ -1031,13 +1069,13 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
             tc_fence_after();
             advance(NC);
             if (p.s_out) {
-                float* row = reinterpret_cast<float*>(sm + CH_PHI) + d * D + 64 * c;
+                float* row = reinterpret_cast<float*>(sm + CH_PHI) + d * D + 32 * c;
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
+                for (int j = 0; j < 8; ++j)
                     *reinterpret_cast<float4*>(row + 4 * j) =
                         make_float4(hv[4 * j], hv[4 * j + 1], hv[4 * j + 2], hv[4 * j + 3]);
                 fence_async_smem();
-                named_bar(1, 256);
+                named_bar(1, 32 * N_ST);
                 if (warp == W_ST && lane == 0) {
                     if (!failed) {
                         bulk_store(p.s_out + (size_t)bh * D * D, sm + CH_PHI, 65536);
