@@ -269,9 +269,10 @@ struct PrepMaps {
     CUtensorMap q, k, v, g;   // g only for the per-dimension gate
 };
 
-// Prep shared memory (bytes from a 1 KB-aligned base); 110 KB for the scalar
+// Prep shared memory (bytes from a 1 KB-aligned base); 111 KB for either
 // gate, so two CTAs share an SM.
-constexpr uint32_t P_KQ = 0;                 // [K_b0 | Q_b0 | K_b1 | Q_b1] (TMA); K~ over K (scalar gate)
+constexpr uint32_t P_KQ = 0;                 // [K_b0 | Q_b0 | K_b1 | Q_b1] (TMA); scalar gate: K~ over K
+                                             // per-dimension gate: K e^(G-c), Q e^(G-c) over K, Q
 constexpr uint32_t P_V = 32768;              // [V_b0 | V_b1] (TMA)
 constexpr uint32_t P_AF = 49152;             // A fp32 [64][LDF]; later [W^T; U^T] bf16 [256][64]
 constexpr uint32_t P_TF = P_AF + 64 * LDF * 4;   // T fp32 [64][LDF]
@@ -279,29 +280,25 @@ constexpr uint32_t P_WUT = P_AF;
 constexpr uint32_t P_TW = 86016;             // T diag(beta e^G) bf16 [64 r][64 i]
 constexpr uint32_t P_TU = 94208;             // T diag(beta)
 constexpr uint32_t P_P = 102400;             // P bf16 [64 r][64 i]
-constexpr uint32_t P_GATE = 110592;          // G, e^G, e^(G_C-G), beta, u, w, flag (7 x 64 floats)
-constexpr uint32_t P_BAR = P_GATE + 7 * 64 * 4;
+constexpr uint32_t P_GATE = 110592;          // scalar: G, e^G, e^(G_C-G), beta, u, w, flag;
+                                             // per-dimension: beta, gamma_d, e^(ref_d)  (512 floats)
+constexpr uint32_t P_BAR = P_GATE + 8 * 64 * 4;
 constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;
+// per-dimension gate: K~ where the scalar gate keeps T_w / T_u (the g tile
+// lands there first), T diag(beta) over the dead A scratch
+constexpr uint32_t PD_KT = P_TW;             // g bf16 (TMA), then K~ = K e^(G_C - G) [b0 | b1]
+constexpr uint32_t PD_T = P_AF;              // T diag(beta) bf16 [64 r][64 i]
 // staging of the step image for its bulk stores (buffers dead by then)
 constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
 constexpr uint32_t S_QPT = 65536;            // over the U^T rows (after their own store has read them)
-constexpr uint32_t S_PUT = 86016;            // over T_w / T_u
-// per-dimension gate extras
-constexpr uint32_t X_G16 = 113664;           // g tile bf16 [g_b0 | g_b1] (TMA)
-constexpr uint32_t X_KB = X_G16 + 16384;     // K e^(m - G)      [b0 | b1]
-constexpr uint32_t X_KG = X_KB + 16384;      // K e^G            [b0 | b1]
-constexpr uint32_t X_QB = X_KG + 16384;      // Q e^G            [b0 | b1]
-constexpr uint32_t X_KT = X_QB + 16384;      // K e^(G_C - G)    [b0 | b1]
-constexpr uint32_t X_SMALL = X_KT + 16384;   // m, c, e^m, e^(c-m) [128 each], flag
-constexpr uint32_t P_SMEM_PD = X_SMALL + 4 * 128 * 4 + 16 + 1024;
-constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (aliases A / T)
+constexpr uint32_t S_PUT = 86016;            // over T_w / T_u (per-dimension gate: over K~)
+constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (exact fallback; aliases A / T)
 static_assert(P_TF + 64 * LDF * 4 <= P_TW, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_TW, "[W^T; U^T] tile");
-static_assert(P_BAR + 64 <= X_G16, "prep layout");
+static_assert(PD_KT + 16384 <= P_P && PD_T + 8192 <= P_TF, "per-dimension tiles");
 static_assert(S_PHI + 32768 <= S_QPT && S_QPT + 16384 <= S_PUT && S_PUT + 16384 <= P_P, "staging");
 static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
 static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
-static_assert(P_SMEM_PD <= 232448, "prep shared memory");
 
 // TMEM columns of the prep kernel (256 allocated: two CTAs per SM).
 constexpr uint32_t TM_S = 0;       // [K;Q] K^T, 64 columns
@@ -314,7 +311,7 @@ constexpr uint32_t TM_PUT = 192;   // U^T P^T, lanes v, 64 columns r
 // One CTA per (batch, head, chunk) of the wave: every state-independent part
 // of the chunk, written to the workspace as the chunk's step image.
 template <int GATE>
-__global__ void __launch_bounds__(NPR, GATE == kGatePerDim ? 1 : 2)
+__global__ void __launch_bounds__(NPR, 2)
 chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -350,18 +347,14 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     };
 
     float* sBeta = gbuf + 192;
-    // per-dimension gate scratch
-    float* Gs = reinterpret_cast<float*>(sm + P_AF);   // G [64][LDG], dead before A is written
-    float* sM = reinterpret_cast<float*>(sm + X_SMALL);
-    float* sC = sM + 128;
-    float* sEm = sC + 128;
-    float* sEcm = sEm + 128;
-    int* sFlag = reinterpret_cast<int*>(sEcm + 128);
+    // per-dimension gate
+    float* Gs = reinterpret_cast<float*>(sm + P_AF);   // exact fallback: G [64][LDG], dead before A is written
+    float* sGamD = gbuf + 256;                         // gamma_d = e^(c_d)
+    float* sRef = gbuf + 384;                          // e^(c_d); 1 in the exact fallback
 
     if (tid == 0) {
         for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
-        if constexpr (PD) *sFlag = 0;
         // K, Q (and g) first: the Gram product needs only them; V lands behind
         mbar_arrive_expect_tx(&bars[0], (PD ? 6 : 4) * 8192);
         mbar_arrive_expect_tx(&bars[4], 2 * 8192);
@@ -369,7 +362,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             tma_load_3d(sm + P_KQ + blk * 16384, &maps.k, &bars[0], h * D + 64 * blk, n * C, b);
             tma_load_3d(sm + P_KQ + blk * 16384 + 8192, &maps.q, &bars[0], h * D + 64 * blk, n * C, b);
             if constexpr (PD)
-                tma_load_3d(sm + X_G16 + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b);
+                tma_load_3d(sm + PD_KT + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b);
         }
         for (int blk = 0; blk < 2; ++blk)
             tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b);
@@ -413,101 +406,114 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         __syncthreads();
     } else {
         wait(0, 0);
-        // G = in-chunk cumsum of g per dimension: thread (d, half), 32 rows each
-        {
-            const int d = tid & 127, hh = tid >> 7;
-            const uint8_t* gt = sm + X_G16 + (d >> 6) * 8192;
-            float acc = 0.f;
-#pragma unroll 8
-            for (int r = 32 * hh; r < 32 * hh + 32; ++r) {
-                acc += ld_bf16(gt, r, d & 63);
-                Gs[r * LDG + d] = acc;
-            }
-        }
-        __syncthreads();
-        {
-            const int d = tid & 127, hh = tid >> 7;
-            if (hh == 1) {
-                const float carry = Gs[31 * LDG + d];
-#pragma unroll 8
-                for (int r = 32; r < 64; ++r) Gs[r * LDG + d] += carry;
-            }
-        }
-        __syncthreads();
-        if (tid < 128) {
-            const float m = Gs[31 * LDG + tid], c = Gs[63 * LDG + tid];
-            sM[tid] = m;
-            sC[tid] = c;
-            sEm[tid] = expf(m);
-            sEcm[tid] = expf(c - m);
-            if (Gs[tid] - m >= 80.f || m - c >= 80.f) atomicOr(sFlag, 1);
-        }
-        __syncthreads();
-        exact = *sFlag != 0;
-        // one pass over the tiles: the Gram operands (in place / K_breve) and
-        // the per-element decayed copies K e^G, K e^(G_C - G), Q e^G
-#pragma unroll 1
-        for (int it = 0; it < 4; ++it) {
-            const int idx = tid + NPR * it;                 // 16-byte chunk 0..1023
-            const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
-            const int d0 = blk * 64 + 8 * (j ^ (r & 7));    // logical columns of this chunk
-            const uint32_t rowoff = (uint32_t)(r * 128 + j * 16);
-            uint4 kraw = *reinterpret_cast<const uint4*>(sm + P_KQ + blk * 16384 + rowoff);
-            uint4 qraw = *reinterpret_cast<const uint4*>(sm + P_KQ + blk * 16384 + 8192 + rowoff);
-            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
-            const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
-            uint32_t kb[4], qb[4], kr[4], qg[4], kg[4], kt[4];
+        // G = in-chunk cumsum of g per key dimension by a segmented scan in
+        // registers: lane pair (segment of 4 rows) x column group of 8
+        // dimensions, then across the 16 segments; c = G_C per dimension.  The
+        // reference c keeps every factor e^(G - c) below e^80 while the chunk
+        // decays by less than that in every dimension; otherwise (exact) A and P
+        // are formed on CUDA cores.
+        const int cg = 2 * warp + (lane & 1), seg = lane >> 1;
+        const int gblk = cg >> 3, gj = cg & 7, r0 = 4 * seg;
+        float Gp[4][8], cv[8];
+        bool wide = false;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = r0 + i;
+            const uint4 raw = *reinterpret_cast<const uint4*>(sm + PD_KT + gblk * 8192 + r * 128 + ((gj ^ (r & 7)) * 16));
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 kf = __bfloat1622float2(k2[e]);
-                const float2 qf = __bfloat1622float2(q2[e]);
-                float ef[2], er[2], eg[2], et[2];
+                const float2 f = __bfloat1622float2(g2[e]);
+                Gp[i][2 * e] = i ? Gp[i - 1][2 * e] + f.x : f.x;
+                Gp[i][2 * e + 1] = i ? Gp[i - 1][2 * e + 1] + f.y : f.y;
+            }
+        }
+        {
+            float tot[8];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int d = d0 + 2 * e + u;
-                    const float G = Gs[r * LDG + d], m = sM[d];
-                    if (!exact) {
-                        ef[u] = expf(G - m);
-                        er[u] = expf(m - G);
-                        eg[u] = sEm[d] * ef[u];     // e^G <= 1
-                        et[u] = sEcm[d] * er[u];    // e^(G_C - G) <= 1
-                    } else {
-                        ef[u] = er[u] = 0.f;
-                        eg[u] = expf(G);
-                        et[u] = expf(sC[d] - G);
-                    }
+            for (int e = 0; e < 8; ++e) tot[e] = Gp[3][e];
+#pragma unroll
+            for (int off = 2; off < 32; off <<= 1) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float y = __shfl_up_sync(0xffffffffu, tot[e], off);
+                    if (lane >= off) tot[e] += y;
                 }
-                kb[e] = pack_bf16(kf.x * ef[0], kf.y * ef[1]);
-                qb[e] = pack_bf16(qf.x * ef[0], qf.y * ef[1]);
-                kr[e] = pack_bf16(kf.x * er[0], kf.y * er[1]);
-                qg[e] = pack_bf16(qf.x * eg[0], qf.y * eg[1]);
-                kg[e] = pack_bf16(kf.x * eg[0], kf.y * eg[1]);
-                kt[e] = pack_bf16(kf.x * et[0], kf.y * et[1]);
             }
-            const uint32_t ioff = blk * 8192 + rowoff;
-            *reinterpret_cast<uint4*>(sm + X_QB + ioff) = make_uint4(qg[0], qg[1], qg[2], qg[3]);
-            *reinterpret_cast<uint4*>(sm + X_KG + ioff) = make_uint4(kg[0], kg[1], kg[2], kg[3]);
-            *reinterpret_cast<uint4*>(sm + X_KT + ioff) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float ex = __shfl_up_sync(0xffffffffu, tot[e], 2);   // segments before this one
+                if (lane < 2) ex = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) Gp[i][e] += ex;
+                cv[e] = __shfl_sync(0xffffffffu, tot[e], 30 + (lane & 1));
+                const float g0 = __shfl_sync(0xffffffffu, Gp[0][e], lane & 1);
+                wide |= g0 - cv[e] >= 80.f;
+            }
+        }
+        exact = __syncthreads_or(wide) != 0;
+        if (seg == 15) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float gm = expf(cv[e]);
+                sGamD[8 * cg + e] = gm;
+                sRef[8 * cg + e] = exact ? 1.f : gm;
+            }
+        }
+        // K~ = K e^(c - G) over the g tile (each thread rewrites only what it
+        // has read); factored: K e^(G - c), Q e^(G - c) in place; exact: G kept
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = r0 + i;
+            const uint32_t ro = r * 128 + ((gj ^ (r & 7)) * 16);
+            uint8_t* kp = sm + P_KQ + gblk * 16384 + ro;
+            const uint4 kraw = *reinterpret_cast<const uint4*>(kp);
+            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
+            uint32_t kt[4];
             if (!exact) {
-                *reinterpret_cast<uint4*>(sm + P_KQ + blk * 16384 + rowoff) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
-                *reinterpret_cast<uint4*>(sm + P_KQ + blk * 16384 + 8192 + rowoff) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
-                *reinterpret_cast<uint4*>(sm + X_KB + ioff) = make_uint4(kr[0], kr[1], kr[2], kr[3]);
+                const uint4 qraw = *reinterpret_cast<const uint4*>(kp + 8192);
+                const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
+                uint32_t kc[4], qc[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kf = __bfloat1622float2(k2[e]);
+                    const float2 qf = __bfloat1622float2(q2[e]);
+                    const float x0 = Gp[i][2 * e] - cv[2 * e], x1 = Gp[i][2 * e + 1] - cv[2 * e + 1];
+                    const float f0 = __expf(x0), f1 = __expf(x1);
+                    const float b0 = __expf(-x0), b1 = __expf(-x1);
+                    kc[e] = pack_bf16(kf.x * f0, kf.y * f1);
+                    qc[e] = pack_bf16(qf.x * f0, qf.y * f1);
+                    kt[e] = pack_bf16(kf.x * b0, kf.y * b1);
+                }
+                *reinterpret_cast<uint4*>(kp) = make_uint4(kc[0], kc[1], kc[2], kc[3]);
+                *reinterpret_cast<uint4*>(kp + 8192) = make_uint4(qc[0], qc[1], qc[2], qc[3]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kf = __bfloat1622float2(k2[e]);
+                    kt[e] = pack_bf16(kf.x * __expf(cv[2 * e] - Gp[i][2 * e]),
+                                      kf.y * __expf(cv[2 * e + 1] - Gp[i][2 * e + 1]));
+                }
+                float* grow = Gs + r * LDG + 8 * cg;
+                *reinterpret_cast<float4*>(grow) = make_float4(Gp[i][0], Gp[i][1], Gp[i][2], Gp[i][3]);
+                *reinterpret_cast<float4*>(grow + 4) = make_float4(Gp[i][4], Gp[i][5], Gp[i][6], Gp[i][7]);
             }
+            *reinterpret_cast<uint4*>(sm + PD_KT + gblk * 8192 + ro) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         if (tid == 0 && !failed) {   // K~ is final: its image goes out now
-            bulk_store(img + IMG_KT, sm + X_KT, 16384);
+            bulk_store(img + IMG_KT, sm + PD_KT, 16384);
             bulk_commit();
         }
-        if (!exact && tid == 32) {   // S = [K e^(G-m); Q e^(G-m)] (K e^(m-G))^T
+        if (!exact && tid == 32) {   // S = [K e^(G-c); Q e^(G-c)] K~^T
             const uint32_t id = idesc_bf16_f32(128, 64, false, false);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const uint32_t a = sb + P_KQ + (k >> 2) * 16384 + (k & 3) * 32;
-                const uint32_t bb = sb + X_KB + (k >> 2) * 8192 + (k & 3) * 32;
+                const uint32_t bb = sb + PD_KT + (k >> 2) * 8192 + (k & 3) * 32;
                 mma_bf16(tmem + TM_S, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id, k > 0);
             }
             mma_commit(&bars[1]);
@@ -522,7 +528,6 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         if (!exact) {
             wait(1, 0);
             tc_fence_after();
-            if constexpr (PD) __syncthreads();   // G (aliased with A) is dead from here on
             ld_cols<32>(tmem + TM_S + lane_off + 32 * ch, sv);
             const float* sG = gbuf;
             const float* sU = gbuf + 256;
@@ -582,6 +587,32 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                 }
                 sv[e] = isq ? acc : sBeta[r] * acc;
             }
+            __syncthreads();   // raw K, Q and G read by every thread
+            {   // reference 0: K e^G, Q e^G in place (same elements as the scan's)
+                const int cg = 2 * warp + (lane & 1), r0 = 4 * (lane >> 1);
+                const int gblk = cg >> 3, gj = cg & 7;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = r0 + i;
+                    uint8_t* kp = sm + P_KQ + gblk * 16384 + r * 128 + ((gj ^ (r & 7)) * 16);
+                    const uint4 kraw = *reinterpret_cast<const uint4*>(kp);
+                    const uint4 qraw = *reinterpret_cast<const uint4*>(kp + 8192);
+                    const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
+                    const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
+                    const float* grow = Gs + r * LDG + 8 * cg;
+                    uint32_t kc[4], qc[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 kf = __bfloat1622float2(k2[e]);
+                        const float2 qf = __bfloat1622float2(q2[e]);
+                        const float f0 = __expf(grow[2 * e]), f1 = __expf(grow[2 * e + 1]);
+                        kc[e] = pack_bf16(kf.x * f0, kf.y * f1);
+                        qc[e] = pack_bf16(qf.x * f0, qf.y * f1);
+                    }
+                    *reinterpret_cast<uint4*>(kp) = make_uint4(kc[0], kc[1], kc[2], kc[3]);
+                    *reinterpret_cast<uint4*>(kp + 8192) = make_uint4(qc[0], qc[1], qc[2], qc[3]);
+                }
+            }
             __syncthreads();   // G (aliased with A) is dead from here on
         }
         if (L < 64) {
@@ -613,8 +644,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                 tu[e] = (i <= r) ? tv[e] * sBeta[i] : 0.f;
                 tw[e] = PD ? tu[e] : tu[e] * sGam[i];
             }
-            st_row_chunk(sm + P_TU, r, j, tu, 1.f);
-            st_row_chunk(sm + P_TW, r, j, tw, 1.f);
+            st_row_chunk(sm + (PD ? PD_T : P_TU), r, j, tu, 1.f);
+            if constexpr (!PD) st_row_chunk(sm + P_TW, r, j, tw, 1.f);
         }
     }
     fence_async_smem();
@@ -622,29 +653,31 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     __syncthreads();
     tc_fence_after();
     if (tid == 32 && !failed) {
-        // W^T = (K e^G)^T T_w^T (scalar gate: the decay sits in T_w), U^T = V^T T_u^T
+        // W^T = (K e^G)^T T_w^T, U^T = V^T T_u^T.  Scalar gate: the decay sits in
+        // T_w; per-dimension gate: (K e^(G-ref))^T T_u^T, rows d times e^(ref_d)
+        // in the epilogue
         const uint32_t id = idesc_bf16_f32(128, 64, true, false);
-        const uint32_t ka = PD ? sb + X_KG : sb + P_KQ;
-        const uint32_t klbo = PD ? 8192 : 16384;
+        const uint32_t tw = PD ? sb + PD_T : sb + P_TW;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem + TM_WT, sdesc_sw128(ka + k * 2048, klbo, 1024),
-                     sdesc_sw128(sb + P_TW + k * 32, 16, 1024), id, k > 0);
+            mma_bf16(tmem + TM_WT, sdesc_sw128(sb + P_KQ + k * 2048, 16384, 1024),
+                     sdesc_sw128(tw + k * 32, 16, 1024), id, k > 0);
         if (!mbar_wait(&bars[4], 0, &failed)) atomicOr(p.status, kStatusTimeout);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_UT, sdesc_sw128(sb + P_V + k * 2048, 8192, 1024),
-                     sdesc_sw128(sb + P_TU + k * 32, 16, 1024), id, k > 0);
+                     sdesc_sw128((PD ? sb + PD_T : sb + P_TU) + k * 32, 16, 1024), id, k > 0);
         mma_commit(&bars[2]);
     }
     wait(2, 0);
     tc_fence_after();
     {   // [W^T; U^T] as one K-major bf16 tile of 256 rows (tokens contiguous)
         const int row = (warp & 3) * 32 + lane;
+        const float sc = (PD && warp < 4) ? sRef[row] : 1.f;
         float v[64];
         ld_cols<64>(tmem + (warp < 4 ? TM_WT : TM_UT) + lane_off, v);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) st_row_chunk(sm + P_WUT, (warp < 4 ? 0 : 128) + row, j, v + 8 * j, 1.f);
+        for (int j = 0; j < 8; ++j) st_row_chunk(sm + P_WUT, (warp < 4 ? 0 : 128) + row, j, v + 8 * j, sc);
     }
     if constexpr (!PD) {   // K~ = diag(e^(G_C - G_i)) K over K (the W product is done with K)
         const float* sFt = gbuf + 128;
@@ -679,7 +712,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         bulk_commit();
     }
     if (tid == 32 && !failed) {
-        const uint32_t kt = PD ? sb + X_KT : sb + P_KQ;
+        const uint32_t kt = PD ? sb + PD_KT : sb + P_KQ;
         const uint32_t ktlbo = PD ? 8192 : 16384;
         const uint32_t id1 = idesc_bf16_f32(128, 128, true, false);   // K~^T W
 #pragma unroll
@@ -724,16 +757,16 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         float v[64];
         ld_cols<64>(tmem + TM_PWT + lane_off, v);
         const int d = row;
+        const float qs = PD ? sRef[d] : 1.f;
 #pragma unroll
         for (int r = 0; r < C; ++r) {
-            const float qb = PD ? ld_bf16(sm + X_QB + (d >> 6) * 8192, r, d & 63)
-                                : gbuf[64 + r] * ld_bf16(sm + P_KQ + (d >> 6) * 16384 + 8192, r, d & 63);
+            const float qb = (PD ? qs : gbuf[64 + r]) * ld_bf16(sm + P_KQ + (d >> 6) * 16384 + 8192, r, d & 63);
             v[r] = qb - v[r];
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_QPT, d, j, v + 8 * j, 1.f);
         float gam;
-        if constexpr (PD) gam = expf(sC[d]);
+        if constexpr (PD) gam = sGamD[d];
         else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
         if (!failed) reinterpret_cast<float*>(img + IMG_GAM)[d] = gam;
     }
@@ -1155,7 +1188,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s,
     auto prep = gate == kGateScalar ? chunk_prep_kernel<kGateScalar>
                 : gate == kGatePerDim ? chunk_prep_kernel<kGatePerDim>
                                       : chunk_prep_kernel<kGateNone>;
-    const uint32_t prep_smem = perdim ? P_SMEM_PD : P_SMEM;
+    const uint32_t prep_smem = P_SMEM;
     cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CH_SMEM);
