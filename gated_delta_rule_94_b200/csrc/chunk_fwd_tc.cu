@@ -38,6 +38,8 @@
 //                       memory and written by a TMA tensor store.
 // Every mbarrier wait is bounded; a wait that gives up sets the library status
 // word and the kernel winds down without further waits.
+#include <string.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
@@ -367,20 +369,20 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         for (int blk = 0; blk < 2; ++blk)
             tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b);
     }
-    if (warp == 0) {
+    if (warp == 1) {
         tmem_alloc(&s_tmem, 256);
         tmem_relinquish();
     }
-    if (tid < 64) {
-        const int t = n * C + tid;
+    if (warp == 2 || warp == 3) {   // beta and g, off the warps that set up barriers and TMEM
+        const int i = tid - 64, t = n * C + i;
         float gv = 0.f, bv = 0.f;
         if (t < T) {
             const size_t tok = ((size_t)b * T + t) * H + h;
             bv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.beta)[tok]);
             if constexpr (GATE == kGateScalar) gv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.g)[tok]);
         }
-        gbuf[tid] = gv;
-        sBeta[tid] = bv;
+        gbuf[i] = gv;
+        sBeta[i] = bv;
     }
     tc_fence_before();
     __syncthreads();
@@ -735,20 +737,22 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     tc_fence_after();
     __syncthreads();
     const int row = (warp & 3) * 32 + lane;
-    if (warp < 4) {   // Phi = -K~^T W, row d (stored as soon as it is staged), then (P U)^T
+    {   // Phi = -K~^T W, row d: warps 0-3 columns 0-63, warps 4-7 columns 64-127;
+        // each half stored as soon as it is staged
+        const int hh = warp >> 2;
+        float v[64];
+        ld_cols<64>(tmem + TM_FP + lane_off + 64 * hh, v);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float v[64];
-            ld_cols<64>(tmem + TM_FP + lane_off + 64 * hh, v);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_PHI + hh * 16384, row, j, v + 8 * j, -1.f);
-        }
+        for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_PHI + hh * 16384, row, j, v + 8 * j, -1.f);
         fence_async_smem();
-        named_bar(1, 128);
-        if (tid == 0 && !failed) {
-            bulk_store(img + IMG_PHI, sm + S_PHI, 32768);
+        if (hh == 0) named_bar(1, 128);
+        else named_bar(3, 128);
+        if ((tid & 127) == 0 && !failed) {
+            bulk_store(img + IMG_PHI + hh * 16384, sm + S_PHI + hh * 16384, 16384);
             bulk_commit();
         }
+    }
+    if (warp < 4) {   // (P U)^T, row v
         float v[64];
         ld_cols<64>(tmem + TM_PUT + lane_off, v);
 #pragma unroll
@@ -780,9 +784,10 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         }
         bulk_wait_read();
     }
+    if (tid == 128) bulk_wait_read();   // its half of Phi
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 256);
     }
@@ -821,6 +826,14 @@ enum ChainBar {
 };
 static_assert(CB_COUNT * 8 <= 256, "barrier space");
 
+// Tensor maps of the chain kernel: o (bf16, [B][T][H*D], 64 x 64 boxes) and the
+// entering / final state (fp32, [B*H][D][D], boxes of 128 rows x 32 columns =
+// 128 B, swizzled so that a lane per row reads its 16-byte chunks without bank
+// conflicts).
+struct ChainMaps {
+    CUtensorMap o, s_in, s_out;
+};
+
 // One CTA per (batch, head): walks the wave's chunks in order.  Per chunk n
 // (slot s = n & 1), h_n the entering state:
 //   X_n = K~_n^T U_n (issued one chunk ahead) + Phi_n bf16(h_n)   in TMEM
@@ -831,7 +844,7 @@ static_assert(CB_COUNT * 8 <= 256, "barrier space");
 // on is per slot or completes at most once ahead of that wait, so no parity
 // wait can fall two phases behind.
 __global__ void __maxnreg__(80)
-chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p) {
+chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -851,7 +864,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
         for (int i = 0; i < CB_COUNT; ++i)
             mbar_init(&bars[i], (i == CB_HREADY0 || i == CB_HREADY1 || i == CB_XFREE0 || i == CB_XFREE1) ? N_ST : 1);
         fence_mbar_init();
-        prefetch_tmap(&omap);
+        prefetch_tmap(&maps.o);
     }
     if (warp == 1) {
         tmem_alloc(&s_tmem, 512);
@@ -876,9 +889,10 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
     if (warp == 0) {
         // =========================== loader: Phi + gamma (2 slots) and K~, U^T;
         // the images it has seen consumed are dropped from L2
-        if (lane == 0 && p.s0 && NC > 0) {   // the entering state, one 64 KB block, staged over the h slots
+        if (lane == 0 && p.s0 && NC > 0) {   // the entering state, staged over the h slots
             mbar_arrive_expect_tx(&bars[CB_S0], 65536);
-            bulk_load(sm + CH_HB, p.s0 + (size_t)bh * D * D, 65536, &bars[CB_S0]);
+            for (int cb = 0; cb < 4; ++cb)
+                tma_load_3d(sm + CH_HB + cb * 16384, &maps.s_in, &bars[CB_S0], 32 * cb, 0, bh);
         }
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
@@ -1032,8 +1046,8 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
                 mbar_arrive(&bars[CB_OFREE0 + s]);
                 if (!failed) {
                     const int t0 = (p.chunk0 + nl) * C;
-                    tma_store_3d(&omap, sm + CH_QP + s * 16384, h * D, t0, b);
-                    tma_store_3d(&omap, sm + CH_QP + s * 16384 + 8192, h * D + 64, t0, b);
+                    tma_store_3d(&maps.o, sm + CH_QP + s * 16384, h * D, t0, b);
+                    tma_store_3d(&maps.o, sm + CH_QP + s * 16384 + 8192, h * D + 64, t0, b);
                     bulk_commit();
                     if (nl + 2 < NC) {
                         bulk_wait_read();
@@ -1061,12 +1075,12 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
             if (nl == 0) {
-                if (p.s0) {   // row d of the staged state
+                if (p.s0) {   // row d, columns 32c.. of the staged state (swizzled 16-byte chunks)
                     wait(CB_S0, 0);
-                    const float* row = reinterpret_cast<const float*>(sm + CH_HB) + d * D + 32 * c;
+                    const uint8_t* row = sm + CH_HB + c * 16384 + d * 128;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const float4 x = *reinterpret_cast<const float4*>(row + 4 * j);
+                        const float4 x = *reinterpret_cast<const float4*>(row + ((j ^ (d & 7)) * 16));
                         hv[4 * j] = x.x; hv[4 * j + 1] = x.y; hv[4 * j + 2] = x.z; hv[4 * j + 3] = x.w;
                     }
                     named_bar(1, 32 * N_ST);   // everyone has read the staging before h slot 0 is written
@@ -1097,24 +1111,25 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap omap, const ChunkParams p
             tmem_wait_st();
         }
         if (NC > 0) {   // final state, staged over the Phi slots (free once the last
-                        // state product is done) and written by one bulk copy
+                        // state product is done), written by four TMA stores
             wait(CB_SDONE, (NC - 1) & 1);
             tc_fence_after();
             advance(NC);
             if (p.s_out) {
-                float* row = reinterpret_cast<float*>(sm + CH_PHI) + d * D + 32 * c;
+                uint8_t* row = sm + CH_PHI + c * 16384 + d * 128;
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    *reinterpret_cast<float4*>(row + 4 * j) =
+                    *reinterpret_cast<float4*>(row + ((j ^ (d & 7)) * 16)) =
                         make_float4(hv[4 * j], hv[4 * j + 1], hv[4 * j + 2], hv[4 * j + 3]);
                 fence_async_smem();
                 named_bar(1, 32 * N_ST);
                 if (warp == W_ST && lane == 0) {
                     if (!failed) {
-                        bulk_store(p.s_out + (size_t)bh * D * D, sm + CH_PHI, 65536);
+                        for (int cb = 0; cb < 4; ++cb)
+                            tma_store_3d(&maps.s_out, sm + CH_PHI + cb * 16384, 32 * cb, 0, bh);
                         bulk_commit();
                     }
-                    bulk_wait_all();
+                    bulk_wait_read();
                 }
             }
         }
@@ -1178,13 +1193,22 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s,
     const bool perdim = gate == kGatePerDim;
     PrepMaps maps;
     if (!make_maps(p0, perdim, &maps)) return cudaErrorInvalidValue;
-    CUtensorMap omap;
+    ChainMaps cmap0;
+    memset(&cmap0, 0, sizeof(cmap0));
     {
         const uint64_t dims[3] = {(uint64_t)p0.H * D, (uint64_t)p0.T, (uint64_t)p0.B};
         const uint64_t strides[2] = {(uint64_t)p0.H * D * 2, (uint64_t)p0.T * p0.H * D * 2};
         const uint32_t box[3] = {64, 64, 1};
-        if (!make_tmap_bf16(&omap, p0.o, 3, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16(&cmap0.o, p0.o, 3, dims, strides, box)) return cudaErrorInvalidValue;
     }
+    // fp32 states [B*H][D rows][D columns], boxes of 128 rows x 32 columns
+    auto state_map = [&](CUtensorMap* m, const float* base) {
+        if (!base) return true;
+        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)D, (uint64_t)p0.B * p0.H};
+        const uint64_t strides[2] = {(uint64_t)D * 4, (uint64_t)D * D * 4};
+        const uint32_t box[3] = {32, 128, 1};
+        return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, 3, dims, strides, box);
+    };
     auto prep = gate == kGateScalar ? chunk_prep_kernel<kGateScalar>
                 : gate == kGatePerDim ? chunk_prep_kernel<kGatePerDim>
                                       : chunk_prep_kernel<kGateNone>;
@@ -1199,6 +1223,12 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s,
     const int nw = (NC + cw - 1) / cw;
     const size_t buf_bytes = (size_t)nbh * cw * IMG_BYTES;
     float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + 2 * buf_bytes) : nullptr;
+    CUtensorMap m_s0, m_sout, m_carry;
+    memset(&m_s0, 0, sizeof(m_s0));
+    memset(&m_sout, 0, sizeof(m_sout));
+    memset(&m_carry, 0, sizeof(m_carry));
+    if (!state_map(&m_s0, p0.s0) || !state_map(&m_sout, p0.s_out) || !state_map(&m_carry, carry))
+        return cudaErrorInvalidValue;
     // Every launch but the first may start before its predecessor ends
     // (programmatic dependent launch); the kernels order themselves with
     // griddepcontrol (see chunk_prep_kernel and chunk_chain_kernel).
@@ -1228,7 +1258,10 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s,
         cfg.blockDim = dim3(CH_THREADS);
         cfg.dynamicSmemBytes = CH_SMEM;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, chunk_chain_kernel, omap, p);
+        ChainMaps cm = cmap0;
+        cm.s_in = (w == 0) ? m_s0 : m_carry;
+        cm.s_out = (w + 1 == nw) ? m_sout : m_carry;
+        e = cudaLaunchKernelEx(&cfg, chunk_chain_kernel, cm, p);
         if (e != cudaSuccess) return e;
         ++*launches;
     }

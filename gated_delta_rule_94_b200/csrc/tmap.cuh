@@ -29,12 +29,13 @@ inline EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
-// bf16 tensor of `rank` dims (dims[0] innermost, contiguous), byte strides of
-// dims 1.. in strides[0..rank-2], box extents box[0..rank-1].  128 B swizzle,
-// out-of-bounds elements read as zero.  Returns false on failure.
-inline bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                           const uint64_t* strides, const uint32_t* box,
-                           CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+// Tensor of element type `dt` and `rank` dims (dims[0] innermost, contiguous),
+// byte strides of dims 1.. in strides[0..rank-2], box extents box[0..rank-1].
+// 128 B swizzle by default, out-of-bounds elements read as zero.  Returns false
+// on failure.
+inline bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, const void* base, int rank,
+                      const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                      CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return false;
     cuuint64_t d[5], s[4];
@@ -45,10 +46,16 @@ inline bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const u
         e[i] = 1;
     }
     for (int i = 0; i + 1 < rank; ++i) s[i] = strides[i];
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+    CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base),
                     d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+inline bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                           const uint64_t* strides, const uint32_t* box,
+                           CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+    return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides, box, swz);
 }
 
 }  // namespace gdn
