@@ -14,7 +14,7 @@
 // Substituting D, each chunk is an affine map of the entering state:
 //   h' = Diag(gamma) h + Phi h + K~^T U,    Phi = -K~^T W,  gamma = e^(G_C)
 //   O  = Qp h + P U,                        Qp  = Q e^G - P W
-// Phi, K~, U, Qp, P U and gamma depend on the chunk's inputs only, so they are
+// Phi, K~, U, Qp, P and gamma depend on the chunk's inputs only, so they are
 // formed for every chunk at once, and only the products with h remain on the
 // serial path.  The decay stays an fp32 multiply of the fp32 state (a bf16
 // gamma - 1 folded into Phi would leave 2^-9 |h| per chunk behind, large
@@ -23,19 +23,19 @@
 // Two kernels per wave of chunks:
 //   chunk_prep_kernel   one CTA per (batch, head, chunk), fully parallel: the
 //                       gates, S = [K;Q]K^T, A and P, T, the WY factors as
-//                       W^T = K^T T^T and U^T = V^T T^T, then K~^T W, W^T P^T
-//                       and U^T P^T; writes the chunk's step image (Phi, K~,
-//                       U^T, Qp^T, (P U)^T in bf16, gamma in fp32) to the
-//                       workspace by bulk copies,
-//                       laid out exactly as the chain kernel's shared-memory
-//                       operands (the wave is sized so the workspace stays in
-//                       L2);
+//                       W^T = K^T T^T and U^T = V^T T^T, then K~^T W and
+//                       W^T P^T; writes the chunk's step image (Phi, K~, U^T,
+//                       Qp^T, P in bf16, gamma in fp32) to the workspace by
+//                       bulk copies, laid out exactly as the chain kernel's
+//                       shared-memory operands (the wave is sized so the
+//                       workspace stays in L2);
 //   chunk_chain_kernel  one CTA per (batch, head), the serial state chain:
 //                       X = K~^T U (one chunk ahead) + Phi h_bf16 (8 MMA
 //                       steps) in TMEM, then the state pass h' = gamma h + X
-//                       in fp32 and its bf16 copy as the next operand; off the
-//                       serial path O^T = h^T Qp^T, added to P U in shared
-//                       memory and written by a TMA tensor store.
+//                       in fp32 registers and its bf16 copy as the next
+//                       operand; off the serial path O = Qp h_bf16 + P U as one
+//                       accumulation of 64 token rows, written by a TMA tensor
+//                       store.
 // Every mbarrier wait is bounded; a wait that gives up sets the library status
 // word and the kernel winds down without further waits.
 #include <string.h>
@@ -59,10 +59,10 @@ constexpr int LDF = 72;          // fp32 row stride of the A / T scratch (confli
 constexpr uint32_t IMG_PHI = 0;        // Phi  [128 d][128 d'],  blocks of 16 KB (K-major A)
 constexpr uint32_t IMG_KT = 32768;     // K~   [64 i][128 d],    blocks of 8 KB (MN-major A)
 constexpr uint32_t IMG_UT = 49152;     // U^T  [128 v][64 i]     (K-major B)
-constexpr uint32_t IMG_QP = 65536;     // Qp^T [128 d][64 r]     (MN-major B)
-constexpr uint32_t IMG_PU = 81920;     // (P U)^T [128 v][64 r]
-constexpr uint32_t IMG_GAM = 98304;    // gamma fp32 [128]
-constexpr uint32_t IMG_BYTES = 98816;
+constexpr uint32_t IMG_QP = 65536;     // Qp^T [128 d][64 r]     (MN-major A of the output product)
+constexpr uint32_t IMG_P = 81920;      // P    [64 r][64 i]      (K-major A)
+constexpr uint32_t IMG_GAM = 90112;    // gamma fp32 [128]
+constexpr uint32_t IMG_BYTES = 90624;
 constexpr size_t WAVE_BYTES = size_t(56) << 20;   // cap of one wave's image buffer
 constexpr int PREP_SLOTS = 2 * 148;                // prep CTAs resident at once on a B200
 
@@ -80,14 +80,6 @@ __device__ __forceinline__ void st_row_chunk(uint8_t* tile, int row, int j, cons
     w.z = pack_bf16(v[4] * scale, v[5] * scale);
     w.w = pack_bf16(v[6] * scale, v[7] * scale);
     *reinterpret_cast<uint4*>(tile + sw128_offset(row, 8 * j)) = w;
-}
-
-// Row `row` (128 elements) of a [rows][128] matrix stored as two swizzled
-// column blocks `bstride` bytes apart.
-__device__ __forceinline__ void st_row128(uint8_t* tile, uint32_t bstride, int row, const float* v,
-                                          float scale) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) st_row_chunk(tile + (j >> 3) * bstride, row, j & 7, v + 8 * j, scale);
 }
 
 __device__ __forceinline__ float ld_bf16(const uint8_t* tile, int row, int col) {
@@ -293,12 +285,11 @@ constexpr uint32_t PD_T = P_AF;              // T diag(beta) bf16 [64 r][64 i]
 // staging of the step image for its bulk stores (buffers dead by then)
 constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
 constexpr uint32_t S_QPT = 65536;            // over the U^T rows (after their own store has read them)
-constexpr uint32_t S_PUT = 86016;            // over T_w / T_u (per-dimension gate: over K~)
 constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (exact fallback; aliases A / T)
 static_assert(P_TF + 64 * LDF * 4 <= P_TW, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_TW, "[W^T; U^T] tile");
 static_assert(PD_KT + 16384 <= P_P && PD_T + 8192 <= P_TF, "per-dimension tiles");
-static_assert(S_PHI + 32768 <= S_QPT && S_QPT + 16384 <= S_PUT && S_PUT + 16384 <= P_P, "staging");
+static_assert(S_PHI + 32768 <= S_QPT && S_QPT + 16384 <= P_TW, "staging");
 static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
 static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
 
@@ -308,7 +299,6 @@ constexpr uint32_t TM_WT = 64;     // W^T, lanes d, 64 columns r
 constexpr uint32_t TM_UT = 128;    // U^T, lanes v, 64 columns r
 constexpr uint32_t TM_FP = 0;      // K~^T W, lanes d, 128 columns d'   (after S, W^T, U^T are read)
 constexpr uint32_t TM_PWT = 128;   // W^T P^T, lanes d, 64 columns r
-constexpr uint32_t TM_PUT = 192;   // U^T P^T, lanes v, 64 columns r
 
 // One CTA per (batch, head, chunk) of the wave: every state-independent part
 // of the chunk, written to the workspace as the chunk's step image.
@@ -705,8 +695,9 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0 && !failed) {   // U^T (and the scalar gate's K~) are final
+    if (tid == 0 && !failed) {   // U^T, P (and the scalar gate's K~) are final
         bulk_store(img + IMG_UT, sm + P_WUT + 16384, 16384);
+        bulk_store(img + IMG_P, sm + P_P, 8192);
         if constexpr (!PD) {
             bulk_store(img + IMG_KT, sm + P_KQ, 8192);
             bulk_store(img + IMG_KT + 8192, sm + P_KQ + 16384, 8192);
@@ -721,14 +712,10 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_FP, sdesc_sw128(kt + k * 2048, ktlbo, 1024),
                      sdesc_sw128(sb + P_WUT + k * 32, 16, 1024), id1, k > 0);
-        const uint32_t id2 = idesc_bf16_f32(128, 64, false, false);   // W^T P^T, U^T P^T
+        const uint32_t id2 = idesc_bf16_f32(128, 64, false, false);   // W^T P^T
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_PWT, sdesc_sw128(sb + P_WUT + k * 32, 16, 1024),
-                     sdesc_sw128(sb + P_P + k * 32, 16, 1024), id2, k > 0);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem + TM_PUT, sdesc_sw128(sb + P_WUT + 16384 + k * 32, 16, 1024),
                      sdesc_sw128(sb + P_P + k * 32, 16, 1024), id2, k > 0);
         mma_commit(&bars[3]);
     }
@@ -752,34 +739,32 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             bulk_commit();
         }
     }
-    if (warp < 4) {   // (P U)^T, row v
-        float v[64];
-        ld_cols<64>(tmem + TM_PUT + lane_off, v);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_PUT, row, j, v + 8 * j, 1.f);
-    } else {          // Qp^T = (Q e^G)^T - W^T P^T, row d; gamma_d
-        float v[64];
-        ld_cols<64>(tmem + TM_PWT + lane_off, v);
+    {   // Qp^T = (Q e^G)^T - W^T P^T, row d: warps 0-3 columns r 0-31, warps 4-7 r 32-63
+        const int hh = warp >> 2;
+        float v[32];
+        ld_cols<32>(tmem + TM_PWT + lane_off + 32 * hh, v);
         const int d = row;
         const float qs = PD ? sRef[d] : 1.f;
 #pragma unroll
-        for (int r = 0; r < C; ++r) {
+        for (int i = 0; i < 32; ++i) {
+            const int r = 32 * hh + i;
             const float qb = (PD ? qs : gbuf[64 + r]) * ld_bf16(sm + P_KQ + (d >> 6) * 16384 + 8192, r, d & 63);
-            v[r] = qb - v[r];
+            v[i] = qb - v[i];
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) st_row_chunk(sm + S_QPT, d, j, v + 8 * j, 1.f);
-        float gam;
-        if constexpr (PD) gam = sGamD[d];
-        else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
-        if (!failed) reinterpret_cast<float*>(img + IMG_GAM)[d] = gam;
+        for (int j = 0; j < 4; ++j) st_row_chunk(sm + S_QPT, d, 4 * hh + j, v + 8 * j, 1.f);
+        if (hh == 1 && !failed) {   // gamma_d
+            float gam;
+            if constexpr (PD) gam = sGamD[d];
+            else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
+            reinterpret_cast<float*>(img + IMG_GAM)[d] = gam;
+        }
     }
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
         if (!failed) {
             bulk_store(img + IMG_QP, sm + S_QPT, 16384);
-            bulk_store(img + IMG_PU, sm + S_PUT, 16384);
             bulk_commit();
         }
         bulk_wait_read();
@@ -797,9 +782,9 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 // Chain kernel shared memory (bytes from a 1 KB-aligned base).
 constexpr uint32_t CH_PHI = 0;          // 2 slots of Phi   (32 KB each)
 constexpr uint32_t CH_KT = 65536;       // K~   (16 KB, one slot)
-constexpr uint32_t CH_UT = 81920;       // U^T  (16 KB, one slot)
-constexpr uint32_t CH_QP = 98304;       // 2 slots of Qp^T (16 KB each); then the O tile for its TMA store
-constexpr uint32_t CH_PU = 131072;      // 2 slots of (P U)^T (16 KB each)
+constexpr uint32_t CH_UT = 81920;       // 2 slots of U^T (16 KB each)
+constexpr uint32_t CH_QP = 114688;      // 2 slots of Qp^T (16 KB each); then the O tile for its TMA store
+constexpr uint32_t CH_P = 147456;       // 2 slots of P (8 KB each)
 constexpr uint32_t CH_HB = 163840;      // 2 slots of h (bf16) MN-major [d][64 v] x 2 blocks
 constexpr uint32_t CH_GAM = 229376;     // 2 slots of gamma (512 B each)
 constexpr uint32_t CH_BAR = 230400;
@@ -814,12 +799,11 @@ constexpr int N_ST = 16;          // state-pass warps: lane quarter x column qua
 // each, so 23 warps (six on some sub-partitions) allow at most 85 a thread.
 
 // TMEM columns of the chain kernel (512 allocated).
-constexpr uint32_t TM_H = 0;      // state h, lanes d, 128 columns v (fp32, the state pass's own)
-constexpr uint32_t TM_O = 128;    // O^T, lanes v, 2 slots of 64 columns r
+constexpr uint32_t TM_O = 0;      // O (M = 64: row r in lane (r % 16) + 32 (r / 16)), 2 slots of 128 columns v
 constexpr uint32_t TM_X = 256;    // X = K~^T U + Phi h, lanes d, 2 slots of 128 columns v
 
 enum ChainBar {
-    CB_IMG0, CB_IMG1, CB_KU, CB_QP0, CB_QP1, CB_PU0, CB_PU1, CB_HREADY0, CB_HREADY1,
+    CB_IMG0, CB_IMG1, CB_KU, CB_QP0, CB_QP1, CB_P0, CB_P1, CB_HREADY0, CB_HREADY1,
     CB_XFREE0, CB_XFREE1, CB_SDONE, CB_SFREE0, CB_SFREE1, CB_KUFREE, CB_ODONE0, CB_ODONE1,
     CB_OFREE0, CB_OFREE1, CB_HBFREE0, CB_HBFREE1, CB_FINAL, CB_OFINAL, CB_S0, CB_SDONEO0,
     CB_SDONEO1, CB_COUNT
@@ -837,8 +821,8 @@ struct ChainMaps {
 // One CTA per (batch, head): walks the wave's chunks in order.  Per chunk n
 // (slot s = n & 1), h_n the entering state:
 //   X_n = K~_n^T U_n (issued one chunk ahead) + Phi_n bf16(h_n)   in TMEM
-//   h_{n+1} = gamma_n h_n + X_n                                  (state pass, fp32)
-//   O_n^T = bf16(h_n)^T Qp_n^T,  O_n = O_n^T^T + (P U)_n          (output warps)
+//   h_{n+1} = gamma_n h_n + X_n                       (state pass, fp32 in registers)
+//   O_n = Qp_n bf16(h_n) + P_n U_n                    (one M = 64 accumulation)
 // The state products and the output product come from two issuing threads, so
 // the output never holds up the serial chain.  Every barrier that a role waits
 // on is per slot or completes at most once ahead of that wait, so no parity
@@ -911,12 +895,17 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             if (nl >= 1) {
                 wait(CB_KUFREE, (nl - 1) & 1);
                 if (failed) break;
-                l2_discard(img(nl - 1) + IMG_KT, 32768, lane);   // K~ and U^T
+                l2_discard(img(nl - 1) + IMG_KT, 16384, lane);
+            }
+            if (nl >= 2) {   // the output product of chunk nl - 2 is done with U^T slot s
+                wait(CB_HBFREE0 + s, ((nl - 2) >> 1) & 1);
+                if (failed) break;
+                l2_discard(img(nl - 2) + IMG_UT, 16384, lane);
             }
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[CB_KU], 32768);
                 bulk_load(sm + CH_KT, img(nl) + IMG_KT, 16384, &bars[CB_KU]);
-                bulk_load(sm + CH_UT, img(nl) + IMG_UT, 16384, &bars[CB_KU]);
+                bulk_load(sm + CH_UT + s * 16384, img(nl) + IMG_UT, 16384, &bars[CB_KU]);
             }
         }
     } else if (warp == 1) {
@@ -938,8 +927,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             if (leader && !failed) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + TM_X + 128 * s, d_kt + ((k * 2048) >> 4), d_ut + ((k * 32) >> 4),
-                             id_ku, k > 0);
+                    mma_bf16(tmem + TM_X + 128 * s, d_kt + ((k * 2048) >> 4),
+                             d_ut + ((s * 16384 + k * 32) >> 4), id_ku, k > 0);
                 mma_commit(&bars[CB_KUFREE]);
             }
         };
@@ -966,24 +955,33 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     } else if (warp == 2) {
-        // =========================== output-product issuer: O^T = h^T Qp^T, issued
-        // once the state product of the chunk is done, so that it fills the
-        // tensor pipe while the state pass works instead of delaying the chain
+        // =========================== output-product issuer: O = Qp h + P U (M = 64
+        // rows r, N = 128 columns v), issued once the state product of the chunk
+        // is done, so that it fills the tensor pipe while the state pass works
+        // instead of delaying the chain
         const bool leader = lane == 0;
-        const uint32_t id_o = idesc_bf16_f32(128, 64, true, true);
+        const uint32_t id_qh = idesc_bf16_f32(64, 128, true, true);     // Qp (MN-major) h (MN-major)
+        const uint32_t id_pu = idesc_bf16_f32(64, 128, false, false);   // P (K-major) U (K-major)
         const uint64_t d_qp = sdesc_sw128(sb + CH_QP, 8192, 1024);
+        const uint64_t d_p = sdesc_sw128(sb + CH_P, 16, 1024);
+        const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
             wait(CB_SDONEO0 + s, (nl >> 1) & 1);
             wait(CB_QP0 + s, (nl >> 1) & 1);
+            wait(CB_P0 + s, (nl >> 1) & 1);
             if (nl >= 2) wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
             tc_fence_after();
             if (leader && !failed) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_bf16(tmem + TM_O + 64 * s, d_hb + ((s * 32768 + k * 2048) >> 4),
-                             d_qp + ((s * 16384 + k * 2048) >> 4), id_o, k > 0);
+                    mma_bf16(tmem + TM_O + 128 * s, d_qp + ((s * 16384 + k * 2048) >> 4),
+                             d_hb + ((s * 32768 + k * 2048) >> 4), id_qh, k > 0);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tmem + TM_O + 128 * s, d_p + ((s * 8192 + k * 32) >> 4),
+                             d_ut + ((s * 16384 + k * 32) >> 4), id_pu, true);
                 mma_commit(&bars[CB_ODONE0 + s]);
                 mma_commit(&bars[CB_HBFREE0 + s]);
             }
@@ -993,54 +991,42 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         if (!mbar_wait(&bars[CB_OFINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     } else if (warp < W_ST) {
-        // =========================== output: O + P U into the Qp slot, TMA store
-        const int v = (warp & 3) * 32 + lane;
+        // =========================== output: O (rows r = 16 (warp & 3) + lane, lanes
+        // 0-15) into the Qp slot, TMA store
+        const int r = 16 * (warp & 3) + lane;
         const bool leader = warp == W_OUT && lane == 0;
-        auto load_qp_pu = [&](int nl) {
+        auto load_qp_p = [&](int nl) {
             const int s = nl & 1;
             mbar_arrive_expect_tx(&bars[CB_QP0 + s], 16384);
             bulk_load(sm + CH_QP + s * 16384, img(nl) + IMG_QP, 16384, &bars[CB_QP0 + s]);
-            mbar_arrive_expect_tx(&bars[CB_PU0 + s], 16384);
-            bulk_load(sm + CH_PU + s * 16384, img(nl) + IMG_PU, 16384, &bars[CB_PU0 + s]);
+            mbar_arrive_expect_tx(&bars[CB_P0 + s], 8192);
+            bulk_load(sm + CH_P + s * 8192, img(nl) + IMG_P, 8192, &bars[CB_P0 + s]);
         };
         if (leader) {
-            for (int nl = 0; nl < 2 && nl < NC; ++nl) load_qp_pu(nl);
+            for (int nl = 0; nl < 2 && nl < NC; ++nl) load_qp_p(nl);
         }
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            wait(CB_ODONE0 + s, (nl >> 1) & 1);   // O is in TMEM; Qp slot s is free
-            wait(CB_PU0 + s, (nl >> 1) & 1);
+            wait(CB_ODONE0 + s, (nl >> 1) & 1);   // O is in TMEM; Qp and P slots s are free
             tc_fence_after();
-            const uint8_t* pu = sm + CH_PU + s * 16384 + v * 128;   // (P U)^T row v
-            uint8_t* ot = sm + CH_QP + s * 16384 + (v >> 6) * 8192;  // O tile [r][64 v] x 2
+            uint8_t* ot = sm + CH_QP + s * 16384;   // O tile [r][64 v] x 2
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            for (int q4 = 0; q4 < 4; ++q4) {
                 float ov[32];
-                ld_cols<32>(tmem + TM_O + 64 * s + 32 * half + lane_off, ov);
+                ld_cols<32>(tmem + TM_O + 128 * s + 32 * q4 + lane_off, ov);
+                if (lane < 16) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int jj = 4 * half + j;
-                    uint4 raw = *reinterpret_cast<const uint4*>(pu + ((jj ^ (v & 7)) * 16));
-                    const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(e2[e]);
-                        ov[8 * j + 2 * e] += f.x;
-                        ov[8 * j + 2 * e + 1] += f.y;
-                    }
+                    for (int j = 0; j < 4; ++j)
+                        st_row_chunk(ot + (q4 >> 1) * 8192, r, 4 * (q4 & 1) + j, ov + 8 * j, 1.f);
                 }
-#pragma unroll
-                for (int r = 0; r < 32; ++r)
-                    *reinterpret_cast<__nv_bfloat16*>(ot + sw128_offset(32 * half + r, v & 63)) =
-                        __float2bfloat16_rn(ov[r]);
             }
             fence_async_smem();
             tc_fence_before();
             named_bar(2, 128);
             if (warp == W_OUT) {   // both images were loaded and read: drop them from L2
                 l2_discard(img(nl) + IMG_QP, 16384, lane);
-                l2_discard(img(nl) + IMG_PU, 16384, lane);
+                l2_discard(img(nl) + IMG_P, 8192, lane);
             }
             if (leader) {
                 mbar_arrive(&bars[CB_OFREE0 + s]);
@@ -1051,7 +1037,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                     bulk_commit();
                     if (nl + 2 < NC) {
                         bulk_wait_read();
-                        load_qp_pu(nl + 2);
+                        load_qp_p(nl + 2);
                     }
                 }
             }
@@ -1061,12 +1047,10 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         // =========================== state pass: h' = gamma h + X -> bf16 operand
         const int d = (warp & 3) * 32 + lane;
         const int c = (warp - W_ST) >> 2;           // column quarter
-        const uint32_t haddr = tmem + TM_H + lane_off + 32 * c;
         float gam = 1.f;                            // gamma of the chunk before
-        float hv[32];
+        float hv[32];                               // the fp32 state, row d, columns 32c..
         auto advance = [&](int nl) {                // hv = gamma_{nl-1} h_{nl-1} + X_{nl-1}
             float xv[32];
-            ld_cols<32>(haddr, hv);
             ld_cols<32>(tmem + TM_X + 128 * ((nl - 1) & 1) + lane_off + 32 * c, xv);
 #pragma unroll
             for (int e = 0; e < 32; ++e) hv[e] = fmaf(gam, hv[e], xv[e]);
@@ -1107,8 +1091,6 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[CB_HREADY0 + s]);
-            st_cols<32>(haddr, hv);                 // the fp32 state, read back next chunk
-            tmem_wait_st();
         }
         if (NC > 0) {   // final state, staged over the Phi slots (free once the last
                         // state product is done), written by four TMA stores
