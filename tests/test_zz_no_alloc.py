@@ -52,15 +52,15 @@ def test_noalloc_matches_regular_entry_point_twice():
 
 
 def test_noalloc_rejects_shapes_beyond_the_scratch():
-    """512 heads x 4 chunks need more workspace than the scratch holds: the
+    """1024 heads x 4 chunks need more workspace than the scratch holds: the
     call returns GDN_ERR_WORKSPACE before touching the (fake, never
     dereferenced) device pointers."""
     lib = _lib.load()
     cap = lib.gdn_chunk_fwd_noalloc_scratch_bytes()
-    need = lib.gdn_chunk_fwd_workspace_bytes(1, 256, 512, 128, 128, 64, _lib.GDN_BF16, 1)
+    need = lib.gdn_chunk_fwd_workspace_bytes(1, 256, 1024, 128, 128, 64, _lib.GDN_BF16, 1)
     assert need > cap
     A = 1 << 40
     rc = lib.gdn_chunk_fwd_noalloc(A, A + (1 << 30), A + (2 << 30), A + (3 << 30), A + (4 << 30), 1,
-                                   None, A + (5 << 30), None, 1, 256, 512, 128, 128, 64,
+                                   None, A + (5 << 30), None, 1, 256, 1024, 128, 128, 64,
                                    _lib.GDN_BF16, None)
     assert rc == _lib.GDN_ERR_WORKSPACE
