@@ -22,7 +22,8 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUD
 GDN_BF16, GDN_F32 = 0, 1
 GDN_GATE_NONE, GDN_GATE_SCALAR, GDN_GATE_PER_DIM = 0, 1, 2
 
-EXPORTED = ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_decode_step",
+EXPORTED = ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd_workspace_min_bytes",
+            "gdn_decode_step",
             "gdn_read_device_status", "gdn_status_string", "gdn_abi_version",
             "gdn_kernel_launch_count", "gdn_chunk_fwd_kernel_name", "gdn_chunk_fwd_noalloc",
             "gdn_chunk_fwd_noalloc_scratch_bytes")
@@ -50,6 +51,8 @@ def load() -> ctypes.CDLL:
     lib.gdn_chunk_fwd.restype = i
     lib.gdn_chunk_fwd_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
     lib.gdn_chunk_fwd_workspace_bytes.restype = sz
+    lib.gdn_chunk_fwd_workspace_min_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    lib.gdn_chunk_fwd_workspace_min_bytes.restype = sz
     lib.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, vp]
     lib.gdn_decode_step.restype = i
     lib.gdn_read_device_status.argtypes = [vp]
@@ -127,6 +130,15 @@ def gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat1
                                              int(gate_kind))
     if n == ctypes.c_size_t(-1).value:
         raise GdnError(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd_workspace_bytes")
+    return n
+
+
+def gdn_chunk_fwd_workspace_min_bytes(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16,
+                                      gate_kind=GDN_GATE_SCALAR) -> int:
+    n = load().gdn_chunk_fwd_workspace_min_bytes(B, T, H, Dk, Dv, chunk, _dtype_code(dtype),
+                                                 int(gate_kind))
+    if n == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd_workspace_min_bytes")
     return n
 
 

@@ -53,7 +53,7 @@ gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, co
                                  const void* g, gdn_gate gate_kind, const float* initial_state,
                                  void* o, float* final_state, int B, int T, int H, int Dk, int Dv,
                                  int chunk, gdn_dtype dtype, gdn_stream_t stream) {
-    const size_t need = gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, chunk, dtype, gate_kind);
+    const size_t need = gdn_chunk_fwd_workspace_min_bytes(B, T, H, Dk, Dv, chunk, dtype, gate_kind);
     if (need == (size_t)-1 || need > kNoAllocScratchBytes) {
         // Let the regular entry point report the argument error, or
         // GDN_ERR_WORKSPACE when the shape needs more than the scratch holds;

@@ -40,6 +40,8 @@
 // word and the kernel winds down without further waits.
 #include <string.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
@@ -63,7 +65,7 @@ constexpr uint32_t IMG_QP = 65536;     // Qp^T [128 d][64 r]     (MN-major A of 
 constexpr uint32_t IMG_P = 81920;      // P    [64 r][64 i]      (K-major A)
 constexpr uint32_t IMG_GAM = 90112;    // gamma fp32 [128]
 constexpr uint32_t IMG_BYTES = 90624;
-constexpr size_t WAVE_BYTES = size_t(56) << 20;   // cap of one wave's image buffer
+constexpr size_t WAVE_BYTES = size_t(160) << 20;  // cap of one wave's image buffer
 constexpr int PREP_SLOTS = 2 * 148;                // prep CTAs resident at once on a B200
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -1136,20 +1138,37 @@ bool make_maps(const ChunkParams& p, bool perdim, PrepMaps* m) {
     return ok;
 }
 
-// Chunks per (batch, head) of one wave: the wave's image buffer stays within
-// WAVE_BYTES, and among such lengths the longest whose prep CTAs fill their
-// last round of resident CTAs to at least 90 % (a nearly empty last round costs
-// a whole CTA lifetime); at least one.
-int wave_chunks(int nbh, int NC) {
-    long long cmax = (long long)(WAVE_BYTES / ((size_t)nbh * IMG_BYTES));
+// Chunks per (batch, head) of one wave, for a workspace of `budget` bytes.
+// Short sequences (up to 4 chunks) run as one wave.  Otherwise two image
+// buffers alternate (plus the state carried between waves): the longest wave
+// whose buffer fits the budget and WAVE_BYTES, at most half the chunks (so that
+// a wave's chain overlaps the next wave's prep), and among such lengths the
+// longest whose prep CTAs fill their last round of resident CTAs to at least
+// 90 % (a nearly empty last round costs a whole CTA lifetime).  0 if even one
+// chunk per wave does not fit.
+int wave_chunks(int nbh, int NC, size_t budget) {
+    const size_t per = (size_t)nbh * IMG_BYTES;                  // one chunk of every head
+    const size_t carry = (size_t)nbh * D * D * sizeof(float);
+    const bool fits_one = (size_t)NC * per <= budget;
+    if (NC <= 4 && fits_one && (size_t)NC * per <= WAVE_BYTES) return NC;
+    if (budget < 2 * per + carry) return fits_one ? NC : 0;
+    long long cmax = std::min<long long>((long long)(WAVE_BYTES / per), (NC + 1) / 2);
+    cmax = std::min<long long>(cmax, (long long)((budget - carry) / (2 * per)));
     if (cmax < 1) cmax = 1;
-    if (cmax > NC) cmax = NC;
     for (long long c = cmax; c >= 1; --c) {
         const long long items = c * nbh;
         const long long rounds = (items + PREP_SLOTS - 1) / PREP_SLOTS;
-        if (c == NC || 10 * items >= 9 * rounds * PREP_SLOTS) return (int)c;
+        if (10 * items >= 9 * rounds * PREP_SLOTS) return (int)c;
     }
     return (int)cmax;
+}
+
+// Workspace of a forward whose waves are cw chunks long.
+size_t workspace_for(int nbh, int NC, int cw) {
+    const int nw = (NC + cw - 1) / cw;
+    size_t bytes = (size_t)nbh * cw * IMG_BYTES * (nw > 1 ? 2 : 1);   // two alternating buffers
+    if (nw > 1) bytes += (size_t)nbh * D * D * sizeof(float);           // state between waves
+    return bytes;
 }
 
 }  // namespace
@@ -1163,14 +1182,20 @@ size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H, int gate) {
     const int NC = (T + C - 1) / C;
     if (NC == 0 || B == 0 || H == 0) return 0;
     const int nbh = B * H;
-    const int cw = wave_chunks(nbh, NC);
-    const int nw = (NC + cw - 1) / cw;
-    size_t bytes = (size_t)nbh * cw * IMG_BYTES * (nw > 1 ? 2 : 1);   // two alternating buffers
-    if (nw > 1) bytes += (size_t)nbh * D * D * sizeof(float);           // state between waves
-    return bytes;
+    return workspace_for(nbh, NC, wave_chunks(nbh, NC, ~static_cast<size_t>(0)));
 }
 
-cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s, int* launches) {
+size_t chunk_fwd_tc_workspace_min_bytes(int B, int T, int H, int gate) {
+    (void)gate;
+    const int NC = (T + C - 1) / C;
+    if (NC == 0 || B == 0 || H == 0) return 0;
+    const size_t per = (size_t)B * H * IMG_BYTES;
+    const size_t two = 2 * per + (size_t)B * H * D * D * sizeof(float);
+    return std::min((size_t)NC * per, two);
+}
+
+cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes, cudaStream_t s,
+                                int* launches) {
     *launches = 0;
     const bool perdim = gate == kGatePerDim;
     PrepMaps maps;
@@ -1201,7 +1226,8 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, cudaStream_t s,
     if (e != cudaSuccess) return e;
     const int NC = (p0.T + C - 1) / C;
     const int nbh = p0.B * p0.H;
-    const int cw = wave_chunks(nbh, NC);
+    const int cw = wave_chunks(nbh, NC, ws_bytes);
+    if (cw < 1) return cudaErrorInvalidValue;
     const int nw = (NC + cw - 1) / cw;
     const size_t buf_bytes = (size_t)nbh * cw * IMG_BYTES;
     float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + 2 * buf_bytes) : nullptr;

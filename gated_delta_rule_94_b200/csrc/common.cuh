@@ -58,9 +58,14 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 namespace gdn {
 cudaError_t launch_chunk_fwd_simt(const ChunkParams& p, int gate, bool bf16, cudaStream_t s);
 bool chunk_fwd_tc_supported(int Dk, int Dv, int gate);
+// Workspace for the longest waves the forward uses / the least it runs with.
 size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H, int gate);
-// Enqueues the tensor-core forward; *launches receives the number of kernels.
-cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, cudaStream_t s, int* launches);
+size_t chunk_fwd_tc_workspace_min_bytes(int B, int T, int H, int gate);
+// Enqueues the tensor-core forward with a workspace of ws_bytes (at least the
+// minimum; waves as long as it allows); *launches receives the number of
+// kernels.
+cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, size_t ws_bytes, cudaStream_t s,
+                                int* launches);
 cudaError_t launch_decode_step(const DecodeParams& p, int Dk, int Dv, int gate, bool bf16,
                                cudaStream_t s);
 }  // namespace gdn

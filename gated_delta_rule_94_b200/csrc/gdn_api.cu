@@ -83,6 +83,17 @@ size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int ch
     return 0;
 }
 
+size_t gdn_chunk_fwd_workspace_min_bytes(int B, int T, int H, int Dk, int Dv, int chunk,
+                                         gdn_dtype dtype, gdn_gate gate_kind) {
+    if (B < 0 || T < 0 || H < 0) return (size_t)-1;
+    if (!supported_dim(Dk) || !supported_dim(Dv) || chunk != 64) return (size_t)-1;
+    if (dtype != GDN_BF16 && dtype != GDN_F32) return (size_t)-1;
+    if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return (size_t)-1;
+    if (dtype == GDN_BF16 && gdn::chunk_fwd_tc_supported(Dk, Dv, gate_kind))
+        return gdn::chunk_fwd_tc_workspace_min_bytes(B, T, H, gate_kind);
+    return 0;
+}
+
 gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* beta,
                          const void* g, gdn_gate gate_kind, const float* initial_state,
                          void* o, float* final_state, int B, int T, int H, int Dk, int Dv,
@@ -119,7 +130,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
     }
     if (need_tokens && initial_state && overlaps(o, ntok * Dv * es, initial_state, state_bytes))
         return GDN_ERR_INVALID_ARG;
-    const size_t ws_need = gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, chunk, dtype, gate_kind);
+    const size_t ws_need = gdn_chunk_fwd_workspace_min_bytes(B, T, H, Dk, Dv, chunk, dtype, gate_kind);
     if (ws_need > 0 && (workspace_bytes < ws_need || !workspace)) return GDN_ERR_WORKSPACE;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -149,7 +160,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
     cudaError_t e;
     int launches = 1;
     if (dtype == GDN_BF16 && gdn::chunk_fwd_tc_supported(Dk, Dv, gate_kind))
-        e = gdn::launch_chunk_fwd_tc(p, gate_kind, s, &launches);
+        e = gdn::launch_chunk_fwd_tc(p, gate_kind, workspace_bytes, s, &launches);
     else
         e = gdn::launch_chunk_fwd_simt(p, gate_kind, dtype == GDN_BF16, s);
     g_launches.fetch_add((unsigned long long)launches);

@@ -51,7 +51,7 @@ typedef enum {
     GDN_OK = 0,
     GDN_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, negative size, bad overlap */
     GDN_ERR_UNSUPPORTED = 2,  /* valid request outside the built shapes / dtypes */
-    GDN_ERR_WORKSPACE = 3,    /* workspace smaller than gdn_chunk_fwd_workspace_bytes */
+    GDN_ERR_WORKSPACE = 3,    /* workspace smaller than gdn_chunk_fwd_workspace_min_bytes */
     GDN_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
     GDN_ERR_TIMEOUT = 5       /* a kernel gave up a bounded wait (reported by
                                  gdn_read_device_status) */
@@ -97,8 +97,9 @@ typedef enum {
  *   chunk         64
  *   dtype         GDN_BF16 (tensor-core path, fp32 accumulation and fp32
  *                 state) or GDN_F32 (fp32 CUDA-core path)
- *   workspace     device scratch of at least gdn_chunk_fwd_workspace_bytes
- *                 bytes (may be NULL when that is 0)
+ *   workspace     device scratch of at least gdn_chunk_fwd_workspace_min_bytes
+ *                 bytes, gdn_chunk_fwd_workspace_bytes for full speed (may be
+ *                 NULL when the minimum is 0); workspace_bytes is its size
  * Returns GDN_OK once the work is enqueued.
  */
 GDN_API gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v,
@@ -108,10 +109,20 @@ GDN_API gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v,
                          gdn_dtype dtype, void* workspace, size_t workspace_bytes,
                          gdn_stream_t stream);
 
-/* Bytes of device workspace gdn_chunk_fwd needs for these arguments (0 when
- * none).  Returns (size_t)-1 for an unsupported or invalid shape. */
+/* Bytes of device workspace with which gdn_chunk_fwd runs fastest for these
+ * arguments (0 when it needs none).  Returns (size_t)-1 for an unsupported or
+ * invalid shape. */
 GDN_API size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk,
                                      gdn_dtype dtype, gdn_gate gate_kind);
+
+/* Least workspace gdn_chunk_fwd accepts for these arguments (0 when it needs
+ * none; never more than gdn_chunk_fwd_workspace_bytes).  Any size in between
+ * works: the forward runs the sequence in waves of chunks whose step images
+ * fit the workspace, so less workspace means shorter waves and less overlap,
+ * with results identical to the bit.  Returns (size_t)-1 for an unsupported
+ * or invalid shape. */
+GDN_API size_t gdn_chunk_fwd_workspace_min_bytes(int B, int T, int H, int Dk, int Dv, int chunk,
+                                                 gdn_dtype dtype, gdn_gate gate_kind);
 
 /*
  * gdn_decode_step -- one recurrent step for N independent sequences: the
@@ -155,9 +166,11 @@ GDN_API const char* gdn_status_string(gdn_status s);
  * path where allocation is forbidden.
  *   - No allocation: the call never calls cudaMalloc, cudaFree or any
  *     allocating library routine.
- *   - Limit: shapes whose gdn_chunk_fwd_workspace_bytes exceeds the scratch
- *     return GDN_ERR_WORKSPACE (nothing is enqueued); argument errors are
- *     reported exactly as by gdn_chunk_fwd.
+ *   - Limit: shapes whose gdn_chunk_fwd_workspace_min_bytes exceeds the
+ *     scratch return GDN_ERR_WORKSPACE (nothing is enqueued); argument errors
+ *     are reported exactly as by gdn_chunk_fwd.  Shapes whose
+ *     gdn_chunk_fwd_workspace_bytes exceeds the scratch run with the waves
+ *     the scratch allows.
  *   - Set-up: the first call on each device looks up the array's device
  *     address (cudaGetSymbolAddress) with that device current; make that
  *     first call before any stream capture on the device.

@@ -49,6 +49,23 @@ def test_workspace_bytes():
     assert lib.gdn_chunk_fwd_workspace_bytes(4, 2048, 16, 96, 128, 64, 0, 1) == bad
     assert lib.gdn_chunk_fwd_workspace_bytes(4, 2048, 16, 128, 128, 32, 0, 1) == bad
     assert lib.gdn_chunk_fwd_workspace_bytes(-1, 2048, 16, 128, 128, 64, 0, 1) == bad
+    assert lib.gdn_chunk_fwd_workspace_min_bytes(4, 2048, 16, 96, 128, 64, 0, 1) == bad
+    assert lib.gdn_chunk_fwd_workspace_min_bytes(-1, 2048, 16, 128, 128, 64, 0, 1) == bad
+
+
+@pytest.mark.parametrize("B,T,H", [(4, 2048, 16), (4, 4096, 16), (1, 65536, 32), (1, 64, 1),
+                                   (2, 200, 2), (1, 256, 1024), (3, 4097, 5)])
+def test_workspace_min_not_above_full_speed_size(B, T, H):
+    """The least workspace the forward accepts is at most the full-speed size;
+    both are 0 without tokens and grow with the number of heads."""
+    lib = _lib.load()
+    for gate in (0, 1, 2):
+        full = lib.gdn_chunk_fwd_workspace_bytes(B, T, H, 128, 128, 64, 0, gate)
+        least = lib.gdn_chunk_fwd_workspace_min_bytes(B, T, H, 128, 128, 64, 0, gate)
+        assert 0 < least <= full
+        assert lib.gdn_chunk_fwd_workspace_min_bytes(B, 0, H, 128, 128, 64, 0, gate) == 0
+        # the fp32 path needs none
+        assert lib.gdn_chunk_fwd_workspace_min_bytes(B, T, H, 128, 128, 64, 1, gate) == 0
 
 
 def chunk_call(**over):

@@ -207,3 +207,36 @@ def test_one_sided_decay_in_chunk(gate):
     o_ref, S_ref = oracle_chunk(x)
     check("o", o, o_ref, TOL[torch.bfloat16])
     check("S", S, S_ref, TOL[torch.bfloat16])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("gate", ["scalar", "per_dim"])
+def test_wave_length_follows_workspace_bit_exactly(gate):
+    """The same forward with the least workspace (one chunk per wave), a middle
+    size and the full-speed size: the waves differ, the results agree to the
+    bit (the state between waves is carried in fp32), and the oracle agrees."""
+    B, T, H, D = 2, 1000, 3, 128
+    x = gi.make_inputs(B, T, H, D, D, dtype=torch.bfloat16, gate=gate, s0_std=0.02, seed=21)
+    d = to_dev(x)
+    least = gdn.gdn_chunk_fwd_workspace_min_bytes(B, T, H, D, D, 64, torch.bfloat16, x["gate_kind"])
+    full = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, D, D, 64, torch.bfloat16, x["gate_kind"])
+    assert 0 < least < full
+    outs = []
+    for nbytes in (least, (least + full) // 2, full):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        o = torch.full((B, T, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        S = torch.full((B, H, D, D), float("nan"), device="cuda")
+        gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], x["gate_kind"], d["S0"], o,
+                          S, workspace=ws)
+        torch.cuda.synchronize()
+        outs.append((o.clone(), S.clone()))
+    for o, S in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(S, outs[0][1])
+    o_ref, S_ref = oracle_chunk(x)
+    check("o", outs[0][0], o_ref, TOL[torch.bfloat16])
+    check("S", outs[0][1], S_ref, TOL[torch.bfloat16])
+    too_small = torch.empty(least - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(gdn.GdnError):
+        gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], x["gate_kind"], d["S0"],
+                          outs[0][0], None, workspace=too_small)
+    assert gdn.gdn_read_device_status() == 0

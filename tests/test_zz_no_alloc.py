@@ -33,8 +33,10 @@ def test_noalloc_matches_regular_entry_point_twice():
                        seed=7)
     d = to_dev(x)
     B, T, H, D = 4, 2048, 16, 128
+    least = gdn.gdn_chunk_fwd_workspace_min_bytes(B, T, H, D, D, 64, torch.bfloat16,
+                                                  x["gate_kind"])
+    assert 0 < least <= _lib.load().gdn_chunk_fwd_noalloc_scratch_bytes()
     need = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, D, D, 64, torch.bfloat16, x["gate_kind"])
-    assert 0 < need <= _lib.load().gdn_chunk_fwd_noalloc_scratch_bytes()
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     o_ref = torch.empty(B, T, H, D, dtype=torch.bfloat16, device="cuda")
     S_ref = torch.empty(B, H, D, D, device="cuda")
@@ -57,7 +59,7 @@ def test_noalloc_rejects_shapes_beyond_the_scratch():
     dereferenced) device pointers."""
     lib = _lib.load()
     cap = lib.gdn_chunk_fwd_noalloc_scratch_bytes()
-    need = lib.gdn_chunk_fwd_workspace_bytes(1, 256, 1024, 128, 128, 64, _lib.GDN_BF16, 1)
+    need = lib.gdn_chunk_fwd_workspace_min_bytes(1, 256, 1024, 128, 128, 64, _lib.GDN_BF16, 1)
     assert need > cap
     A = 1 << 40
     rc = lib.gdn_chunk_fwd_noalloc(A, A + (1 << 30), A + (2 << 30), A + (3 << 30), A + (4 << 30), 1,
