@@ -100,6 +100,8 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // so the L2 does not spend DRAM bandwidth evicting it.  One warp, lanes split
 // the lines.
 __device__ __forceinline__ void l2_discard(const void* p, uint32_t bytes, int lane) {
+    if (reinterpret_cast<uintptr_t>(p) & 127u) return;   // whole lines only (a workspace need
+                                                          // only be 16-byte aligned)
     const char* c = static_cast<const char*>(p);
     for (uint32_t off = 128u * lane; off < bytes; off += 128u * 32u)
         asm volatile("discard.global.L2 [%0], 128;" ::"l"(c + off) : "memory");
@@ -805,10 +807,10 @@ constexpr uint32_t TM_O = 0;      // O (M = 64: row r in lane (r % 16) + 32 (r /
 constexpr uint32_t TM_X = 256;    // X = K~^T U + Phi h, lanes d, 2 slots of 128 columns v
 
 enum ChainBar {
-    CB_IMG0, CB_IMG1, CB_KU, CB_QP0, CB_QP1, CB_P0, CB_P1, CB_HREADY0, CB_HREADY1,
+    CB_IMG0, CB_IMG1, CB_KU0, CB_KU1, CB_UFREE0, CB_UFREE1, CB_QP0, CB_QP1, CB_P0, CB_P1, CB_HREADY0, CB_HREADY1,
     CB_XFREE0, CB_XFREE1, CB_SDONE, CB_SFREE0, CB_SFREE1, CB_KUFREE, CB_ODONE0, CB_ODONE1,
     CB_OFREE0, CB_OFREE1, CB_HBFREE0, CB_HBFREE1, CB_FINAL, CB_OFINAL, CB_S0, CB_SDONEO0,
-    CB_SDONEO1, CB_COUNT
+    CB_SDONEO1, CB_HREADYB0, CB_HREADYB1, CB_SDONEB, CB_COUNT
 };
 static_assert(CB_COUNT * 8 <= 256, "barrier space");
 
@@ -821,7 +823,9 @@ struct ChainMaps {
 };
 
 // One CTA per (batch, head): walks the wave's chunks in order.  Per chunk n
-// (slot s = n & 1), h_n the entering state:
+// (slot s = n & 1), h_n the entering state, in two column halves (v < 64 and
+// v >= 64) whose products and state passes interleave -- the state pass of one
+// half runs while the other half's product is on the tensor pipe:
 //   X_n = K~_n^T U_n (issued one chunk ahead) + Phi_n bf16(h_n)   in TMEM
 //   h_{n+1} = gamma_n h_n + X_n                       (state pass, fp32 in registers)
 //   O_n = Qp_n bf16(h_n) + P_n U_n                    (one M = 64 accumulation)
@@ -848,7 +852,9 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 
     if (tid == 0) {
         for (int i = 0; i < CB_COUNT; ++i)
-            mbar_init(&bars[i], (i == CB_HREADY0 || i == CB_HREADY1 || i == CB_XFREE0 || i == CB_XFREE1) ? N_ST : 1);
+            mbar_init(&bars[i], (i == CB_XFREE0 || i == CB_XFREE1) ? N_ST
+                                : (i == CB_HREADY0 || i == CB_HREADY1 || i == CB_HREADYB0 ||
+                                   i == CB_HREADYB1) ? N_ST / 2 : 1);
         fence_mbar_init();
         prefetch_tmap(&maps.o);
     }
@@ -880,34 +886,36 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             for (int cb = 0; cb < 4; ++cb)
                 tma_load_3d(sm + CH_HB + cb * 16384, &maps.s_in, &bars[CB_S0], 32 * cb, 0, bh);
         }
+        if (lane == 0) {   // the first images into L2 ahead of their loads
+            for (int nl = 0; nl < 2 && nl < NC; ++nl) bulk_prefetch_l2(img(nl), IMG_BYTES);
+        }
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            if (nl >= 2) {
-                wait(CB_SFREE0 + s, ((nl - 2) >> 1) & 1);
-                if (failed) break;
-                l2_discard(img(nl - 2) + IMG_PHI, 32768, lane);
-                l2_discard(img(nl - 2) + IMG_GAM, 512, lane);
+            // K~ and U^T first: the K~^T U product of chunk nl is issued right
+            // after the state product of chunk nl - 1
+            if (nl >= 1) wait(CB_KUFREE, (nl - 1) & 1);
+            if (nl >= 2) wait(CB_UFREE0 + s, ((nl - 2) >> 1) & 1);   // P U of nl - 2 done with U^T slot s
+            if (failed) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars[CB_KU0 + s], 32768);
+                bulk_load(sm + CH_KT, img(nl) + IMG_KT, 16384, &bars[CB_KU0 + s]);
+                bulk_load(sm + CH_UT + s * 16384, img(nl) + IMG_UT, 16384, &bars[CB_KU0 + s]);
             }
+            if (nl >= 2) wait(CB_SFREE0 + s, ((nl - 2) >> 1) & 1);
+            if (failed) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[CB_IMG0 + s], 32768 + 512);
                 bulk_load(sm + CH_PHI + s * 32768, img(nl) + IMG_PHI, 32768, &bars[CB_IMG0 + s]);
                 bulk_load(sm + CH_GAM + s * 512, img(nl) + IMG_GAM, 512, &bars[CB_IMG0 + s]);
+                if (nl + 2 < NC) bulk_prefetch_l2(img(nl + 2), IMG_BYTES);
             }
-            if (nl >= 1) {
-                wait(CB_KUFREE, (nl - 1) & 1);
-                if (failed) break;
-                l2_discard(img(nl - 1) + IMG_KT, 16384, lane);
-            }
-            if (nl >= 2) {   // the output product of chunk nl - 2 is done with U^T slot s
-                wait(CB_HBFREE0 + s, ((nl - 2) >> 1) & 1);
-                if (failed) break;
+            // the images already loaded into shared memory are dead in L2
+            if (nl >= 1) l2_discard(img(nl - 1) + IMG_KT, 16384, lane);
+            if (nl >= 2) {
                 l2_discard(img(nl - 2) + IMG_UT, 16384, lane);
-            }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&bars[CB_KU], 32768);
-                bulk_load(sm + CH_KT, img(nl) + IMG_KT, 16384, &bars[CB_KU]);
-                bulk_load(sm + CH_UT + s * 16384, img(nl) + IMG_UT, 16384, &bars[CB_KU]);
+                l2_discard(img(nl - 2) + IMG_PHI, 32768, lane);
+                l2_discard(img(nl - 2) + IMG_GAM, 512, lane);
             }
         }
     } else if (warp == 1) {
@@ -915,7 +923,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         // a k-step adds its byte offset / 16 to the start-address field)
         const bool leader = lane == 0;
         const uint32_t id_ku = idesc_bf16_f32(128, 128, true, false);   // K~^T U
-        const uint32_t id_ph = idesc_bf16_f32(128, 128, false, true);   // Phi h_bf16
+        const uint32_t id_ph = idesc_bf16_f32(128, 64, false, true);    // Phi h_bf16, one column half
         const uint64_t d_phi = sdesc_sw128(sb + CH_PHI, 16, 1024);
         const uint64_t d_kt = sdesc_sw128(sb + CH_KT, 8192, 1024);
         const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
@@ -923,7 +931,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         // pass has read X of chunk nl - 2 there
         auto issue_ku = [&](int nl) {
             const int s = nl & 1;
-            wait(CB_KU, nl & 1);
+            wait(CB_KU0 + s, (nl >> 1) & 1);
             if (nl >= 2) wait(CB_XFREE0 + s, ((nl - 2) >> 1) & 1);
             tc_fence_after();
             if (leader && !failed) {
@@ -938,15 +946,21 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            wait(CB_HREADY0 + s, (nl >> 1) & 1);
             wait(CB_IMG0 + s, (nl >> 1) & 1);
-            tc_fence_after();
-            if (leader && !failed) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16(tmem + TM_X + 128 * s, d_phi + ((s * 32768 + (k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                             d_hb + ((s * 32768 + k * 2048) >> 4), id_ph, true);
-                mma_commit(&bars[CB_SDONE]);
+            for (int hf = 0; hf < 2; ++hf) {   // column half hf of X += Phi h
+                wait((hf ? CB_HREADYB0 : CB_HREADY0) + s, (nl >> 1) & 1);
+                tc_fence_after();
+                if (leader && !failed) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_bf16(tmem + TM_X + 128 * s + 64 * hf,
+                                 d_phi + ((s * 32768 + (k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                                 d_hb + ((s * 32768 + hf * 16384 + k * 2048) >> 4), id_ph, true);
+                    mma_commit(&bars[hf ? CB_SDONEB : CB_SDONE]);
+                }
+            }
+            if (leader && !failed) {
                 mma_commit(&bars[CB_SFREE0 + s]);
                 mma_commit(&bars[CB_SDONEO0 + s]);
             }
@@ -957,10 +971,11 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     } else if (warp == 2) {
-        // =========================== output-product issuer: O = Qp h + P U (M = 64
-        // rows r, N = 128 columns v), issued once the state product of the chunk
-        // is done, so that it fills the tensor pipe while the state pass works
-        // instead of delaying the chain
+        // =========================== output-product issuer: O = P U + Qp h (M = 64
+        // rows r, N = 128 columns v).  P U needs no state: it is issued as soon
+        // as U^T and P are in, releasing the U^T slot early; Qp h once the state
+        // product of the chunk is done, so that it fills the tensor pipe while the
+        // state pass works instead of delaying the chain
         const bool leader = lane == 0;
         const uint32_t id_qh = idesc_bf16_f32(64, 128, true, true);     // Qp (MN-major) h (MN-major)
         const uint32_t id_pu = idesc_bf16_f32(64, 128, false, false);   // P (K-major) U (K-major)
@@ -970,20 +985,25 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            wait(CB_SDONEO0 + s, (nl >> 1) & 1);
-            wait(CB_QP0 + s, (nl >> 1) & 1);
+            wait(CB_KU0 + s, (nl >> 1) & 1);
             wait(CB_P0 + s, (nl >> 1) & 1);
             if (nl >= 2) wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
             tc_fence_after();
             if (leader && !failed) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16(tmem + TM_O + 128 * s, d_qp + ((s * 16384 + k * 2048) >> 4),
-                             d_hb + ((s * 32768 + k * 2048) >> 4), id_qh, k > 0);
-#pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_bf16(tmem + TM_O + 128 * s, d_p + ((s * 8192 + k * 32) >> 4),
-                             d_ut + ((s * 16384 + k * 32) >> 4), id_pu, true);
+                             d_ut + ((s * 16384 + k * 32) >> 4), id_pu, k > 0);
+                mma_commit(&bars[CB_UFREE0 + s]);
+            }
+            wait(CB_SDONEO0 + s, (nl >> 1) & 1);
+            wait(CB_QP0 + s, (nl >> 1) & 1);
+            tc_fence_after();
+            if (leader && !failed) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16(tmem + TM_O + 128 * s, d_qp + ((s * 16384 + k * 2048) >> 4),
+                             d_hb + ((s * 32768 + k * 2048) >> 4), id_qh, true);
                 mma_commit(&bars[CB_ODONE0 + s]);
                 mma_commit(&bars[CB_HBFREE0 + s]);
             }
@@ -1075,7 +1095,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                     for (int e = 0; e < 32; ++e) hv[e] = 0.f;
                 }
             } else {
-                wait(CB_SDONE, (nl - 1) & 1);
+                wait(c < 2 ? CB_SDONE : CB_SDONEB, (nl - 1) & 1);
                 tc_fence_after();
                 advance(nl);
                 tc_fence_before();
@@ -1092,14 +1112,15 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             gam = reinterpret_cast<const float*>(sm + CH_GAM + s * 512)[d];
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CB_HREADY0 + s]);
+            if (lane == 0) mbar_arrive(&bars[(c < 2 ? CB_HREADY0 : CB_HREADYB0) + s]);
         }
-        if (NC > 0) {   // final state, staged over the Phi slots (free once the last
-                        // state product is done), written by four TMA stores
-            wait(CB_SDONE, (NC - 1) & 1);
+        if (NC > 0) {   // final state, staged over the Phi slots (free once both halves
+                        // of the last state product are done), written by four TMA stores
+            wait(c < 2 ? CB_SDONE : CB_SDONEB, (NC - 1) & 1);
             tc_fence_after();
             advance(NC);
             if (p.s_out) {
+                if (c < 2) wait(CB_SDONEB, (NC - 1) & 1);   // the other half still reads Phi
                 uint8_t* row = sm + CH_PHI + c * 16384 + d * 128;
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
