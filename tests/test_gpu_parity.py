@@ -240,3 +240,51 @@ def test_wave_length_follows_workspace_bit_exactly(gate):
         gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], x["gate_kind"], d["S0"],
                           outs[0][0], None, workspace=too_small)
     assert gdn.gdn_read_device_status() == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("gate", ["scalar", "per_dim"])
+def test_more_heads_than_sms(gate):
+    """180 (batch, head) pairs: the chain grid has more CTAs than the GPU has
+    SMs, so chain CTAs wait for SMs across waves; every output and state still
+    matches the oracle."""
+    x = gi.make_inputs(3, 200, 60, 128, 128, dtype=torch.bfloat16, gate=gate, s0_std=0.02, seed=23)
+    o, S = gpu_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check("o", o, o_ref, TOL[torch.bfloat16])
+    check("S", S, S_ref, TOL[torch.bfloat16])
+    assert gdn.gdn_read_device_status() == 0
+
+
+@pytest.mark.gpu
+def test_one_chunk_waves_with_many_heads():
+    """3600 heads of one chunk: the images of one chunk of every head exceed a
+    wave buffer's cap, so the forward runs with one-chunk waves; a workspace of
+    the least size forces one-chunk waves on a longer sequence too."""
+    x = gi.make_inputs(2, 64, 1800, 128, 128, dtype=torch.bfloat16, gate="scalar", seed=24)
+    o, S = gpu_chunk(x)
+    heads = [0, 911, 1799]
+    f = gi.to_f64_numpy(x)
+    q, k, v, beta, g = (f[n][:, :, heads] for n in ("q", "k", "v", "beta", "g"))
+    o_ref, S_ref = oracle.recurrent(q, k, v, beta, g, x["gate_kind"], None)
+    check("o (sampled heads)", o[:, :, heads], o_ref, TOL[torch.bfloat16])
+    check("S (sampled heads)", S[:, heads], S_ref, TOL[torch.bfloat16])
+    # a longer sequence with the least workspace (one chunk per wave) against the full one
+    B, T, H, D = 2, 640, 100, 128
+    y = gi.make_inputs(B, T, H, D, D, dtype=torch.bfloat16, gate="scalar", s0_std=0.02, seed=25)
+    d = to_dev(y)
+    outs = []
+    for nbytes in (gdn.gdn_chunk_fwd_workspace_min_bytes(B, T, H, D, D, 64, torch.bfloat16, 1),
+                   gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, D, D, 64, torch.bfloat16, 1)):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        o2 = torch.full((B, T, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        S2 = torch.full((B, H, D, D), float("nan"), device="cuda")
+        gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], y["gate_kind"], d["S0"], o2,
+                          S2, workspace=ws)
+        torch.cuda.synchronize()
+        outs.append((o2, S2))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    o_ref2, S_ref2 = oracle_chunk(y, heads=[0, 57, 99])
+    check("o (least workspace, sampled heads)", outs[0][0][:, :, [0, 57, 99]], o_ref2, TOL[torch.bfloat16])
+    check("S (least workspace, sampled heads)", outs[0][1][:, [0, 57, 99]], S_ref2, TOL[torch.bfloat16])
+    assert gdn.gdn_read_device_status() == 0
