@@ -121,13 +121,6 @@ __device__ __forceinline__ void ld_cols(uint32_t addr, float (&v)[N]) {
     reg_fence(v);
 }
 
-template <int N>
-__device__ __forceinline__ void st_cols(uint32_t addr, float (&v)[N]) {
-#pragma unroll
-    for (int j = 0; j < N / 16; ++j)
-        tmem_st16(addr + 16 * j, *reinterpret_cast<float(*)[16]>(v + 16 * j));
-}
-
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));

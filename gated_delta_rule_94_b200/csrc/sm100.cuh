@@ -98,37 +98,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* f
     return true;
 }
 
-// Non-blocking test of a phase.
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred P;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, P;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait by polling (no suspension): for the few waits on a serial
-// critical path, where a suspended thread's wake-up would add latency.  Same
-// contract as mbar_wait.
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, int* failed,
-                                               uint64_t timeout_ns = 2000000000ull) {
-    if (*failed) return false;
-    if (mbar_test(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    uint32_t n = 0;
-    while (!mbar_test(bar, parity)) {
-        if ((++n & 255u) == 0u && globaltimer_ns() - t0 > timeout_ns) {
-            *failed = 1;
-            return false;
-        }
-    }
-    return true;
-}
-
 // ------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1) {
