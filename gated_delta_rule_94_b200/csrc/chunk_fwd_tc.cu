@@ -776,56 +776,90 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 }
 
 // ------------------------------------------------------------------ chain
+// The chain runs on the transposed state: h^T [v][d] (fp32 in the state-pass
+// registers, its bf16 copy in TMEM as the A operand of the products), so that
+// neither the state's bf16 copy nor the products' h operand touch shared
+// memory:
+//   X^T_n = U_n^T K~_n (issued ahead) + h_n^T Phi_n^T      (two halves of d')
+//   h_{n+1}^T = h_n^T Diag(gamma_n) + X^T_n                 (state pass)
+//   O^T_n = U_n^T P_n^T + h_n^T Qp_n^T                      (output product)
+// The step image is the one the prep writes: Phi is the K-major B operand of
+// h^T Phi^T, K~ the MN-major B of U^T K~, U^T the K-major A of both U^T
+// products, Qp^T the MN-major B and P the K-major B of the output product.
+
 // Chain kernel shared memory (bytes from a 1 KB-aligned base).
-constexpr uint32_t CH_PHI = 0;          // 2 slots of Phi   (32 KB each)
-constexpr uint32_t CH_KT = 65536;       // K~   (16 KB, one slot)
-constexpr uint32_t CH_UT = 81920;       // 2 slots of U^T (16 KB each)
-constexpr uint32_t CH_QP = 114688;      // 2 slots of Qp^T (16 KB each); then the O tile for its TMA store
-constexpr uint32_t CH_P = 147456;       // 2 slots of P (8 KB each)
-constexpr uint32_t CH_HB = 163840;      // 2 slots of h (bf16) MN-major [d][64 v] x 2 blocks
-constexpr uint32_t CH_GAM = 229376;     // 2 slots of gamma (512 B each)
-constexpr uint32_t CH_BAR = 230400;
-constexpr uint32_t CH_SMEM = CH_BAR + 256 + 1024;
+constexpr uint32_t CH_PHI = 0;          // 2 slots of Phi (32 KB each); the final state's staging
+constexpr uint32_t CH_KT = 65536;       // 2 slots of K~ (16 KB each)
+constexpr uint32_t CH_UT = 98304;       // 2 slots of U^T (16 KB each)
+constexpr uint32_t CH_QP = 131072;      // 2 slots of Qp^T (16 KB each) } the entering state's
+constexpr uint32_t CH_P = 163840;       // 2 slots of P (8 KB each)     } staging (64 KB)
+constexpr uint32_t CH_OT = 180224;      // 2 slots of the O tile [r][64 v] x 2 blocks for its TMA store
+constexpr uint32_t CH_GAM = 212992;     // 4 slots of gamma (512 B each)
+constexpr uint32_t CH_BAR = 215040;
+constexpr uint32_t CH_SMEM = CH_BAR + 512 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
+static_assert(CH_QP + 65536 <= CH_OT + 16384, "entering-state staging over Qp^T / P / O slot 0");
 
 constexpr int CH_THREADS = 736;   // 23 warps: loader, 2 MMA issuers, 4 output, 16 state
 constexpr int W_OUT = 3;          // first output warp
 constexpr int W_ST = 7;           // first state-pass warp
-constexpr int N_ST = 16;          // state-pass warps: lane quarter x column quarter
+constexpr int N_ST = 16;          // state-pass warps: lane quarter (v) x column quarter (d)
 // Registers: warps spread over the SM's four sub-partitions of 16 K registers
 // each, so 23 warps (six on some sub-partitions) allow at most 85 a thread.
 
 // TMEM columns of the chain kernel (512 allocated).
-constexpr uint32_t TM_O = 0;      // O (M = 64: row r in lane (r % 16) + 32 (r / 16)), 2 slots of 128 columns v
-constexpr uint32_t TM_X = 256;    // X = K~^T U + Phi h, lanes d, 2 slots of 128 columns v
+constexpr uint32_t TM_HT = 0;      // h^T bf16, lanes v, 2 slots of 64 columns (d pairs)
+constexpr uint32_t TM_OT = 128;    // O^T, lanes v, 2 slots of 64 columns r
+constexpr uint32_t TM_X = 256;     // X^T, lanes v, 2 slots of 128 columns d'
 
 enum ChainBar {
-    CB_IMG0, CB_IMG1, CB_KU0, CB_KU1, CB_UFREE0, CB_UFREE1, CB_QP0, CB_QP1, CB_P0, CB_P1, CB_HREADY0, CB_HREADY1,
-    CB_XFREE0, CB_XFREE1, CB_SDONE, CB_SFREE0, CB_SFREE1, CB_KUFREE, CB_ODONE0, CB_ODONE1,
-    CB_OFREE0, CB_OFREE1, CB_HBFREE0, CB_HBFREE1, CB_FINAL, CB_OFINAL, CB_S0, CB_SDONEO0,
-    CB_SDONEO1, CB_HREADYB0, CB_HREADYB1, CB_SDONEB, CB_COUNT
+    CB_IMG0, CB_IMG1, CB_GAM0, CB_GAM1, CB_GAM2, CB_GAM3, CB_KU0, CB_KU1, CB_KUFREE0, CB_KUFREE1,
+    CB_UFREE0, CB_UFREE1, CB_QP0, CB_QP1, CB_P0, CB_P1, CB_HREADYA0, CB_HREADYA1, CB_HREADYB0,
+    CB_HREADYB1, CB_XFREE0, CB_XFREE1, CB_SDONEA, CB_SDONEB, CB_SFREE0, CB_SFREE1, CB_SDONEO0,
+    CB_SDONEO1, CB_ODONE0, CB_ODONE1, CB_OFREE0, CB_OFREE1, CB_HBFREE0, CB_HBFREE1, CB_S0,
+    CB_S0FREE, CB_FINAL, CB_OFINAL, CB_COUNT
 };
-static_assert(CB_COUNT * 8 <= 256, "barrier space");
+static_assert(CB_COUNT * 8 <= 512, "barrier space");
 
 // Tensor maps of the chain kernel: o (bf16, [B][T][H*D], 64 x 64 boxes) and the
 // entering / final state (fp32, [B*H][D][D], boxes of 128 rows x 32 columns =
-// 128 B, swizzled so that a lane per row reads its 16-byte chunks without bank
-// conflicts).
+// 128 B, swizzled so that the lanes of a warp -- 32 consecutive columns v of
+// one row d -- read or write one row of a box without bank conflicts).
 struct ChainMaps {
     CUtensorMap o, s_in, s_out;
 };
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, A from tensor memory (row m in lane m, k
+// pairs packed two bf16 to a 32-bit column, 8 columns a k-step of 16).
+__device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_read_all_but_one() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// Element (d, v) of the entering / final state staged as four TMA boxes of
+// [128 d][32 v] fp32 (128-byte swizzle), box v / 32.
+__device__ __forceinline__ uint32_t st_off(int d, int v) {
+    return (uint32_t)(v >> 5) * 16384u + (uint32_t)d * 128u +
+           ((uint32_t)(((v & 31) >> 2) ^ (d & 7)) << 4) + ((uint32_t)(v & 3) << 2);
+}
+
 // One CTA per (batch, head): walks the wave's chunks in order.  Per chunk n
-// (slot s = n & 1), h_n the entering state, in two column halves (v < 64 and
-// v >= 64) whose products and state passes interleave -- the state pass of one
-// half runs while the other half's product is on the tensor pipe:
-//   X_n = K~_n^T U_n (issued one chunk ahead) + Phi_n bf16(h_n)   in TMEM
-//   h_{n+1} = gamma_n h_n + X_n                       (state pass, fp32 in registers)
-//   O_n = Qp_n bf16(h_n) + P_n U_n                    (one M = 64 accumulation)
-// The state products and the output product come from two issuing threads, so
-// the output never holds up the serial chain.  Every barrier that a role waits
-// on is per slot or completes at most once ahead of that wait, so no parity
-// wait can fall two phases behind.
+// (slot s = n & 1) the state product in two halves of d' (the state pass of
+// the first half runs while the second half's product is on the tensor pipe),
+// the U^T K~ product of the next chunk issued ahead, and the output product
+// from a second issuing thread, so the output never holds up the serial chain.
+// Every barrier that a role waits on is per slot (or per gamma slot) or
+// completes at most once ahead of that wait, so no parity wait can fall two
+// phases behind.
 __global__ void __maxnreg__(80)
 chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -845,9 +879,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 
     if (tid == 0) {
         for (int i = 0; i < CB_COUNT; ++i)
-            mbar_init(&bars[i], (i == CB_XFREE0 || i == CB_XFREE1) ? N_ST
-                                : (i == CB_HREADY0 || i == CB_HREADY1 || i == CB_HREADYB0 ||
-                                   i == CB_HREADYB1) ? N_ST / 2 : 1);
+            mbar_init(&bars[i], (i == CB_XFREE0 || i == CB_XFREE1 || i == CB_S0FREE) ? N_ST
+                                : (i >= CB_HREADYA0 && i <= CB_HREADYB1) ? N_ST / 2 : 1);
         fence_mbar_init();
         prefetch_tmap(&maps.o);
     }
@@ -869,59 +902,59 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         __syncwarp();
     };
     auto img = [&](int nl) { return wsh + (size_t)nl * IMG_BYTES; };
-    const uint64_t d_hb = sdesc_sw128(sb + CH_HB, 16384, 1024);
 
     if (warp == 0) {
-        // =========================== loader: Phi + gamma (2 slots) and K~, U^T;
-        // the images it has seen consumed are dropped from L2
-        if (lane == 0 && p.s0 && NC > 0) {   // the entering state, staged over the h slots
+        // =========================== loader: K~ and U^T (2 slots, two chunks
+        // ahead), Phi (2 slots), gamma (4 slots); each image prefetched into L2
+        // two chunks ahead, its lines dropped from L2 once loaded
+        if (lane == 0 && p.s0) {   // the entering state, staged over Qp^T / P / O slot 0
             mbar_arrive_expect_tx(&bars[CB_S0], 65536);
             for (int cb = 0; cb < 4; ++cb)
-                tma_load_3d(sm + CH_HB + cb * 16384, &maps.s_in, &bars[CB_S0], 32 * cb, 0, bh);
+                tma_load_3d(sm + CH_QP + cb * 16384, &maps.s_in, &bars[CB_S0], 32 * cb, 0, bh);
         }
-        if (lane == 0) {   // the first images into L2 ahead of their loads
+        if (lane == 0) {
             for (int nl = 0; nl < 2 && nl < NC; ++nl) bulk_prefetch_l2(img(nl), IMG_BYTES);
         }
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            // K~ and U^T first: the K~^T U product of chunk nl is issued right
-            // after the state product of chunk nl - 1
-            if (nl >= 1) wait(CB_KUFREE, (nl - 1) & 1);
-            if (nl >= 2) wait(CB_UFREE0 + s, ((nl - 2) >> 1) & 1);   // P U of nl - 2 done with U^T slot s
+            if (nl >= 2) {   // U^T K~ and P U of chunk nl - 2 are done with slot s
+                wait(CB_KUFREE0 + s, ((nl - 2) >> 1) & 1);
+                wait(CB_UFREE0 + s, ((nl - 2) >> 1) & 1);
+            }
             if (failed) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[CB_KU0 + s], 32768);
-                bulk_load(sm + CH_KT, img(nl) + IMG_KT, 16384, &bars[CB_KU0 + s]);
+                bulk_load(sm + CH_KT + s * 16384, img(nl) + IMG_KT, 16384, &bars[CB_KU0 + s]);
                 bulk_load(sm + CH_UT + s * 16384, img(nl) + IMG_UT, 16384, &bars[CB_KU0 + s]);
             }
             if (nl >= 2) wait(CB_SFREE0 + s, ((nl - 2) >> 1) & 1);
             if (failed) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&bars[CB_IMG0 + s], 32768 + 512);
+                mbar_arrive_expect_tx(&bars[CB_IMG0 + s], 32768);
                 bulk_load(sm + CH_PHI + s * 32768, img(nl) + IMG_PHI, 32768, &bars[CB_IMG0 + s]);
-                bulk_load(sm + CH_GAM + s * 512, img(nl) + IMG_GAM, 512, &bars[CB_IMG0 + s]);
+                mbar_arrive_expect_tx(&bars[CB_GAM0 + (nl & 3)], 512);
+                bulk_load(sm + CH_GAM + (nl & 3) * 512, img(nl) + IMG_GAM, 512, &bars[CB_GAM0 + (nl & 3)]);
                 if (nl + 2 < NC) bulk_prefetch_l2(img(nl + 2), IMG_BYTES);
             }
-            // the images already loaded into shared memory are dead in L2
-            if (nl >= 1) l2_discard(img(nl - 1) + IMG_KT, 16384, lane);
-            if (nl >= 2) {
-                l2_discard(img(nl - 2) + IMG_UT, 16384, lane);
+            if (nl >= 2) {   // loaded into shared memory: dead in L2 (gamma of chunk
+                             // nl - 3 is known to be in: the state pass has used it)
+                l2_discard(img(nl - 2) + IMG_KT, 32768, lane);   // K~ and U^T
                 l2_discard(img(nl - 2) + IMG_PHI, 32768, lane);
-                l2_discard(img(nl - 2) + IMG_GAM, 512, lane);
+                if (nl >= 3) l2_discard(img(nl - 3) + IMG_GAM, 512, lane);
             }
         }
     } else if (warp == 1) {
         // =========================== state-product issuer (descriptors built once;
         // a k-step adds its byte offset / 16 to the start-address field)
         const bool leader = lane == 0;
-        const uint32_t id_ku = idesc_bf16_f32(128, 128, true, false);   // K~^T U
-        const uint32_t id_ph = idesc_bf16_f32(128, 64, false, true);    // Phi h_bf16, one column half
+        const uint32_t id_ku = idesc_bf16_f32(128, 128, false, true);   // U^T (K-major) K~ (MN-major)
+        const uint32_t id_ph = idesc_bf16_f32(128, 64, false, false);   // h^T (TMEM) Phi^T half (K-major)
         const uint64_t d_phi = sdesc_sw128(sb + CH_PHI, 16, 1024);
         const uint64_t d_kt = sdesc_sw128(sb + CH_KT, 8192, 1024);
         const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
-        // K~^T U of chunk nl into X slot nl & 1 once K~, U^T are in and the state
-        // pass has read X of chunk nl - 2 there
+        // U^T K~ of chunk nl into X^T slot nl & 1 once K~, U^T are in and the
+        // state pass has read X^T of chunk nl - 2 there
         auto issue_ku = [&](int nl) {
             const int s = nl & 1;
             wait(CB_KU0 + s, (nl >> 1) & 1);
@@ -930,9 +963,9 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             if (leader && !failed) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + TM_X + 128 * s, d_kt + ((k * 2048) >> 4),
-                             d_ut + ((s * 16384 + k * 32) >> 4), id_ku, k > 0);
-                mma_commit(&bars[CB_KUFREE]);
+                    mma_bf16(tmem + TM_X + 128 * s, d_ut + ((s * 16384 + k * 32) >> 4),
+                             d_kt + ((s * 16384 + k * 2048) >> 4), id_ku, k > 0);
+                mma_commit(&bars[CB_KUFREE0 + s]);
             }
         };
         if (NC > 0) issue_ku(0);
@@ -940,20 +973,19 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
             wait(CB_IMG0 + s, (nl >> 1) & 1);
+            wait(CB_HREADYA0 + s, (nl >> 1) & 1);
+            wait(CB_HREADYB0 + s, (nl >> 1) & 1);
+            tc_fence_after();
+            if (leader && !failed) {
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {   // column half hf of X += Phi h
-                wait((hf ? CB_HREADYB0 : CB_HREADY0) + s, (nl >> 1) & 1);
-                tc_fence_after();
-                if (leader && !failed) {
+                for (int hf = 0; hf < 2; ++hf) {   // columns d' of half hf: Phi rows 64 hf..
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_bf16(tmem + TM_X + 128 * s + 64 * hf,
-                                 d_phi + ((s * 32768 + (k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                                 d_hb + ((s * 32768 + hf * 16384 + k * 2048) >> 4), id_ph, true);
-                    mma_commit(&bars[hf ? CB_SDONEB : CB_SDONE]);
+                        mma_bf16_ta(tmem + TM_X + 128 * s + 64 * hf, tmem + TM_HT + 64 * s + 8 * k,
+                                    d_phi + ((s * 32768 + (k >> 2) * 16384 + hf * 8192 + (k & 3) * 32) >> 4),
+                                    id_ph, true);
+                    mma_commit(&bars[hf ? CB_SDONEB : CB_SDONEA]);
                 }
-            }
-            if (leader && !failed) {
                 mma_commit(&bars[CB_SFREE0 + s]);
                 mma_commit(&bars[CB_SDONEO0 + s]);
             }
@@ -964,17 +996,17 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     } else if (warp == 2) {
-        // =========================== output-product issuer: O = P U + Qp h (M = 64
-        // rows r, N = 128 columns v).  P U needs no state: it is issued as soon
-        // as U^T and P are in, releasing the U^T slot early; Qp h once the state
-        // product of the chunk is done, so that it fills the tensor pipe while the
-        // state pass works instead of delaying the chain
+        // =========================== output-product issuer: O^T = U^T P^T + h^T Qp^T
+        // (lanes v, 64 columns r).  U^T P^T needs no state: it is issued as soon
+        // as U^T and P are in, releasing the U^T slot early; h^T Qp^T once the
+        // state product of the chunk is done, so that it fills the tensor pipe
+        // while the state pass works instead of delaying the chain
         const bool leader = lane == 0;
-        const uint32_t id_qh = idesc_bf16_f32(64, 128, true, true);     // Qp (MN-major) h (MN-major)
-        const uint32_t id_pu = idesc_bf16_f32(64, 128, false, false);   // P (K-major) U (K-major)
-        const uint64_t d_qp = sdesc_sw128(sb + CH_QP, 8192, 1024);
-        const uint64_t d_p = sdesc_sw128(sb + CH_P, 16, 1024);
+        const uint32_t id_pu = idesc_bf16_f32(128, 64, false, false);   // U^T (K-major) P (K-major)
+        const uint32_t id_qh = idesc_bf16_f32(128, 64, false, true);    // h^T (TMEM) Qp^T (MN-major)
         const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
+        const uint64_t d_p = sdesc_sw128(sb + CH_P, 16, 1024);
+        const uint64_t d_qp = sdesc_sw128(sb + CH_QP, 8192, 1024);
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
@@ -985,8 +1017,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             if (leader && !failed) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + TM_O + 128 * s, d_p + ((s * 8192 + k * 32) >> 4),
-                             d_ut + ((s * 16384 + k * 32) >> 4), id_pu, k > 0);
+                    mma_bf16(tmem + TM_OT + 64 * s, d_ut + ((s * 16384 + k * 32) >> 4),
+                             d_p + ((s * 8192 + k * 32) >> 4), id_pu, k > 0);
                 mma_commit(&bars[CB_UFREE0 + s]);
             }
             wait(CB_SDONEO0 + s, (nl >> 1) & 1);
@@ -995,8 +1027,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             if (leader && !failed) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_bf16(tmem + TM_O + 128 * s, d_qp + ((s * 16384 + k * 2048) >> 4),
-                             d_hb + ((s * 32768 + k * 2048) >> 4), id_qh, true);
+                    mma_bf16_ta(tmem + TM_OT + 64 * s, tmem + TM_HT + 64 * s + 8 * k,
+                                d_qp + ((s * 16384 + k * 2048) >> 4), id_qh, true);
                 mma_commit(&bars[CB_ODONE0 + s]);
                 mma_commit(&bars[CB_HBFREE0 + s]);
             }
@@ -1006,9 +1038,10 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         if (!mbar_wait(&bars[CB_OFINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     } else if (warp < W_ST) {
-        // =========================== output: O (rows r = 16 (warp & 3) + lane, lanes
-        // 0-15) into the Qp slot, TMA store
-        const int r = 16 * (warp & 3) + lane;
+        // =========================== output: O^T row v -> the O tile [r][v]
+        // (bf16, swizzled) in its slot -> TMA store; the Qp^T and P slots are
+        // refilled as soon as the output product is done with them
+        const int v = (warp & 3) * 32 + lane;
         const bool leader = warp == W_OUT && lane == 0;
         auto load_qp_p = [&](int nl) {
             const int s = nl & 1;
@@ -1018,23 +1051,28 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             bulk_load(sm + CH_P + s * 8192, img(nl) + IMG_P, 8192, &bars[CB_P0 + s]);
         };
         if (leader) {
+            if (p.s0) {   // the entering state's staging has been read
+                if (!mbar_wait(&bars[CB_S0FREE], 0, &failed)) atomicOr(p.status, kStatusTimeout);
+            }
             for (int nl = 0; nl < 2 && nl < NC; ++nl) load_qp_p(nl);
         }
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            wait(CB_ODONE0 + s, (nl >> 1) & 1);   // O is in TMEM; Qp and P slots s are free
+            if (leader && nl >= 2) bulk_wait_read_all_but_one();   // the store of chunk nl - 2 read slot s
+            named_bar(2, 128);
+            wait(CB_ODONE0 + s, (nl >> 1) & 1);
             tc_fence_after();
-            uint8_t* ot = sm + CH_QP + s * 16384;   // O tile [r][64 v] x 2
+            if (leader && !failed && nl + 2 < NC) load_qp_p(nl + 2);
+            uint8_t* ot = sm + CH_OT + s * 16384 + (v >> 6) * 8192;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int half = 0; half < 2; ++half) {
                 float ov[32];
-                ld_cols<32>(tmem + TM_O + 128 * s + 32 * q4 + lane_off, ov);
-                if (lane < 16) {
+                ld_cols<32>(tmem + TM_OT + 64 * s + 32 * half + lane_off, ov);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        st_row_chunk(ot + (q4 >> 1) * 8192, r, 4 * (q4 & 1) + j, ov + 8 * j, 1.f);
-                }
+                for (int r = 0; r < 32; ++r)
+                    *reinterpret_cast<__nv_bfloat16*>(ot + sw128_offset(32 * half + r, v & 63)) =
+                        __float2bfloat16_rn(ov[r]);
             }
             fence_async_smem();
             tc_fence_before();
@@ -1047,48 +1085,51 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 mbar_arrive(&bars[CB_OFREE0 + s]);
                 if (!failed) {
                     const int t0 = (p.chunk0 + nl) * C;
-                    tma_store_3d(&maps.o, sm + CH_QP + s * 16384, h * D, t0, b);
-                    tma_store_3d(&maps.o, sm + CH_QP + s * 16384 + 8192, h * D + 64, t0, b);
+                    tma_store_3d(&maps.o, sm + CH_OT + s * 16384, h * D, t0, b);
+                    tma_store_3d(&maps.o, sm + CH_OT + s * 16384 + 8192, h * D + 64, t0, b);
                     bulk_commit();
-                    if (nl + 2 < NC) {
-                        bulk_wait_read();
-                        load_qp_p(nl + 2);
-                    }
                 }
             }
         }
         if (leader) bulk_wait_all();
     } else {
-        // =========================== state pass: h' = gamma h + X -> bf16 operand
-        const int d = (warp & 3) * 32 + lane;
-        const int c = (warp - W_ST) >> 2;           // column quarter
-        float gam = 1.f;                            // gamma of the chunk before
-        float hv[32];                               // the fp32 state, row d, columns 32c..
-        auto advance = [&](int nl) {                // hv = gamma_{nl-1} h_{nl-1} + X_{nl-1}
+        // =========================== state pass: h'^T = h^T Diag(gamma) + X^T in
+        // fp32 registers (row v, columns d = 32c..), its bf16 copy into TMEM
+        const int v = (warp & 3) * 32 + lane;
+        const int c = (warp - W_ST) >> 2;           // column quarter of d
+        const int hf = c >> 1;                      // half of the state product it waits for
+        float hv[32];
+        auto advance = [&](int nl) {                // hv = h_{nl-1}^T Diag(gamma_{nl-1}) + X^T_{nl-1}
+            wait(CB_GAM0 + ((nl - 1) & 3), ((nl - 1) >> 2) & 1);
             float xv[32];
             ld_cols<32>(tmem + TM_X + 128 * ((nl - 1) & 1) + lane_off + 32 * c, xv);
+            const float* gp = reinterpret_cast<const float*>(sm + CH_GAM + ((nl - 1) & 3) * 512) + 32 * c;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) hv[e] = fmaf(gam, hv[e], xv[e]);
+            for (int j = 0; j < 8; ++j) {
+                const float4 g4 = *reinterpret_cast<const float4*>(gp + 4 * j);
+                hv[4 * j] = fmaf(g4.x, hv[4 * j], xv[4 * j]);
+                hv[4 * j + 1] = fmaf(g4.y, hv[4 * j + 1], xv[4 * j + 1]);
+                hv[4 * j + 2] = fmaf(g4.z, hv[4 * j + 2], xv[4 * j + 2]);
+                hv[4 * j + 3] = fmaf(g4.w, hv[4 * j + 3], xv[4 * j + 3]);
+            }
         };
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
             if (nl == 0) {
-                if (p.s0) {   // row d, columns 32c.. of the staged state (swizzled 16-byte chunks)
+                if (p.s0) {   // column v, rows d = 32c.. of the staged state
                     wait(CB_S0, 0);
-                    const uint8_t* row = sm + CH_HB + c * 16384 + d * 128;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float4 x = *reinterpret_cast<const float4*>(row + ((j ^ (d & 7)) * 16));
-                        hv[4 * j] = x.x; hv[4 * j + 1] = x.y; hv[4 * j + 2] = x.z; hv[4 * j + 3] = x.w;
-                    }
-                    named_bar(1, 32 * N_ST);   // everyone has read the staging before h slot 0 is written
+                    for (int e = 0; e < 32; ++e)
+                        hv[e] = *reinterpret_cast<const float*>(sm + CH_QP + st_off(32 * c + e, v));
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[CB_S0FREE]);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) hv[e] = 0.f;
                 }
             } else {
-                wait(c < 2 ? CB_SDONE : CB_SDONEB, (nl - 1) & 1);
+                wait(hf ? CB_SDONEB : CB_SDONEA, (nl - 1) & 1);
                 tc_fence_after();
                 advance(nl);
                 tc_fence_before();
@@ -1096,29 +1137,27 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 if (lane == 0) mbar_arrive(&bars[CB_XFREE0 + ((nl - 1) & 1)]);
             }
             if (nl >= 2) wait(CB_HBFREE0 + s, ((nl - 2) >> 1) & 1);   // O of chunk nl - 2 is done with it
-            uint8_t* hb = sm + CH_HB + s * 32768 + (c >> 1) * 16384;
+            {
+                float pk[16];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) st_row_chunk(hb, d, 4 * (c & 1) + j, hv + 8 * j, 1.f);
-            // gamma of this chunk before HREADY: its slot is refilled only after
-            // the MMA that HREADY releases
-            wait(CB_IMG0 + s, (nl >> 1) & 1);
-            gam = reinterpret_cast<const float*>(sm + CH_GAM + s * 512)[d];
-            fence_async_smem();
+                for (int e = 0; e < 16; ++e) pk[e] = __uint_as_float(pack_bf16(hv[2 * e], hv[2 * e + 1]));
+                tmem_st16(tmem + TM_HT + 64 * s + 16 * c + lane_off, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[(c < 2 ? CB_HREADY0 : CB_HREADYB0) + s]);
+            if (lane == 0) mbar_arrive(&bars[(hf ? CB_HREADYB0 : CB_HREADYA0) + s]);
         }
         if (NC > 0) {   // final state, staged over the Phi slots (free once both halves
                         // of the last state product are done), written by four TMA stores
-            wait(c < 2 ? CB_SDONE : CB_SDONEB, (NC - 1) & 1);
+            wait(hf ? CB_SDONEB : CB_SDONEA, (NC - 1) & 1);
             tc_fence_after();
             advance(NC);
             if (p.s_out) {
-                if (c < 2) wait(CB_SDONEB, (NC - 1) & 1);   // the other half still reads Phi
-                uint8_t* row = sm + CH_PHI + c * 16384 + d * 128;
+                if (hf == 0) wait(CB_SDONEB, (NC - 1) & 1);   // the other half still reads Phi
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    *reinterpret_cast<float4*>(row + ((j ^ (d & 7)) * 16)) =
-                        make_float4(hv[4 * j], hv[4 * j + 1], hv[4 * j + 2], hv[4 * j + 3]);
+                for (int e = 0; e < 32; ++e)
+                    *reinterpret_cast<float*>(sm + CH_PHI + st_off(32 * c + e, v)) = hv[e];
                 fence_async_smem();
                 named_bar(1, 32 * N_ST);
                 if (warp == W_ST && lane == 0) {
