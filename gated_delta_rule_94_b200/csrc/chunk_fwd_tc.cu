@@ -281,12 +281,13 @@ constexpr uint32_t PD_KT = P_TW;             // g bf16 (TMA), then K~ = K e^(G_C
 constexpr uint32_t PD_T = P_AF;              // T diag(beta) bf16 [64 r][64 i]
 // staging of the step image for its bulk stores (buffers dead by then)
 constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
-constexpr uint32_t S_QPT = 65536;            // over the U^T rows (after their own store has read them)
+constexpr uint32_t S_QPT = P_TW;             // over T_w / T_u (scalar gate) or K~ (per-dimension
+                                             // gate): dead once the K~^T W and W^T P^T products are done
 constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (exact fallback; aliases A / T)
 static_assert(P_TF + 64 * LDF * 4 <= P_TW, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_TW, "[W^T; U^T] tile");
 static_assert(PD_KT + 16384 <= P_P && PD_T + 8192 <= P_TF, "per-dimension tiles");
-static_assert(S_PHI + 32768 <= S_QPT && S_QPT + 16384 <= P_TW, "staging");
+static_assert(S_PHI + 32768 <= P_WUT + 16384 && S_QPT + 16384 <= P_P, "staging clear of the U^T rows and P");
 static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
 static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
 
@@ -717,7 +718,9 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         mma_commit(&bars[3]);
     }
     wait(3, 0);
-    if (tid == 0) bulk_wait_read();   // the U^T rows become the Qp^T staging
+    // the per-dimension gate's K~ tile becomes the Qp^T staging: its image store (the
+    // older of the two outstanding groups) must have read it
+    if (PD && tid == 0) bulk_wait_read_all_but_one();
     tc_fence_after();
     __syncthreads();
     const int row = (warp & 3) * 32 + lane;
@@ -841,9 +844,6 @@ __device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
-__device__ __forceinline__ void bulk_wait_read_all_but_one() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
 
 // Element (d, v) of the entering / final state staged as four TMA boxes of
 // [128 d][32 v] fp32 (128-byte swizzle), box v / 32.

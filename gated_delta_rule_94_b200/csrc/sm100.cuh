@@ -156,6 +156,12 @@ __device__ __forceinline__ void bulk_wait_read() {
 }
 
 // Wait until every committed bulk group of this thread has completed.
+// Wait until every bulk group of this thread but the most recent one has read
+// its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all_but_one() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned global address.
