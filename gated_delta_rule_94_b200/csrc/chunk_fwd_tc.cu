@@ -860,6 +860,9 @@ __device__ __forceinline__ uint32_t st_off(int d, int v) {
 // Every barrier that a role waits on is per slot (or per gamma slot) or
 // completes at most once ahead of that wait, so no parity wait can fall two
 // phases behind.
+// UNIFORM_GAMMA: every column of the state decays by the same gamma (scalar gate
+// or none), so the state pass reads one value per chunk, ahead of the product.
+template <bool UNIFORM_GAMMA>
 __global__ void __maxnreg__(80)
 chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -1099,14 +1102,21 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         const int c = (warp - W_ST) >> 2;           // column quarter of d
         const int hf = c >> 1;                      // half of the state product it waits for
         float hv[32];
-        auto advance = [&](int nl) {                // hv = h_{nl-1}^T Diag(gamma_{nl-1}) + X^T_{nl-1}
+        // hv = h_{nl-1}^T Diag(gamma_{nl-1}) + X^T_{nl-1}, once the state product of
+        // chunk nl - 1 is done (half hf); a uniform gamma is read before that wait
+        auto advance = [&](int nl) {
+            const float* gp = reinterpret_cast<const float*>(sm + CH_GAM + ((nl - 1) & 3) * 512) + 32 * c;
             wait(CB_GAM0 + ((nl - 1) & 3), ((nl - 1) >> 2) & 1);
+            float g1 = 1.f;
+            if constexpr (UNIFORM_GAMMA) g1 = *gp;
+            wait(hf ? CB_SDONEB : CB_SDONEA, (nl - 1) & 1);
+            tc_fence_after();
             float xv[32];
             ld_cols<32>(tmem + TM_X + 128 * ((nl - 1) & 1) + lane_off + 32 * c, xv);
-            const float* gp = reinterpret_cast<const float*>(sm + CH_GAM + ((nl - 1) & 3) * 512) + 32 * c;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float4 g4 = *reinterpret_cast<const float4*>(gp + 4 * j);
+                float4 g4 = make_float4(g1, g1, g1, g1);
+                if constexpr (!UNIFORM_GAMMA) g4 = *reinterpret_cast<const float4*>(gp + 4 * j);
                 hv[4 * j] = fmaf(g4.x, hv[4 * j], xv[4 * j]);
                 hv[4 * j + 1] = fmaf(g4.y, hv[4 * j + 1], xv[4 * j + 1]);
                 hv[4 * j + 2] = fmaf(g4.z, hv[4 * j + 2], xv[4 * j + 2]);
@@ -1129,8 +1139,6 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                     for (int e = 0; e < 32; ++e) hv[e] = 0.f;
                 }
             } else {
-                wait(hf ? CB_SDONEB : CB_SDONEA, (nl - 1) & 1);
-                tc_fence_after();
                 advance(nl);
                 tc_fence_before();
                 __syncwarp();
@@ -1150,8 +1158,6 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         }
         if (NC > 0) {   // final state, staged over the Phi slots (free once both halves
                         // of the last state product are done), written by four TMA stores
-            wait(hf ? CB_SDONEB : CB_SDONEA, (NC - 1) & 1);
-            tc_fence_after();
             advance(NC);
             if (p.s_out) {
                 if (hf == 0) wait(CB_SDONEB, (NC - 1) & 1);   // the other half still reads Phi
@@ -1275,7 +1281,8 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
     const uint32_t prep_smem = P_SMEM;
     cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CH_SMEM);
+    auto chain = gate == kGatePerDim ? chunk_chain_kernel<false> : chunk_chain_kernel<true>;
+    e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CH_SMEM);
     if (e != cudaSuccess) return e;
     const int NC = (p0.T + C - 1) / C;
     const int nbh = p0.B * p0.H;
@@ -1322,7 +1329,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
         ChainMaps cm = cmap0;
         cm.s_in = (w == 0) ? m_s0 : m_carry;
         cm.s_out = (w + 1 == nw) ? m_sout : m_carry;
-        e = cudaLaunchKernelEx(&cfg, chunk_chain_kernel, cm, p);
+        e = cudaLaunchKernelEx(&cfg, chain, cm, p);
         if (e != cudaSuccess) return e;
         ++*launches;
     }
