@@ -156,14 +156,17 @@ __device__ __forceinline__ void store_16x8(float* X, int r0, int n0, const float
 
 // T = (I + A)^-1 for strictly lower-triangular A (64 x 64, fp32), 256 threads
 // (8 warps).  (1) the four diagonal 16 x 16 inverses by right-looking
-// substitution on CUDA cores, one column per thread; (2) 16 -> 32:
+// substitution on CUDA cores, one column per thread (threads 64.. run `idle`
+// meanwhile); (2) 16 -> 32:
 // T_10 = -T_11 (A_10 T_00) for the two diagonal 32 x 32 blocks; (3) 32 -> 64:
 // the same with 32 x 32 blocks.  The block products run as warp MMAs on tf32
 // operands with fp32 accumulation (T is rounded to bf16 right after, so the
 // tf32 operand rounding stays well below that); the inner product X goes
 // through the strictly upper part of Tm, which T never uses.
-__device__ __forceinline__ void forward_substitution(const float* A, float* Tm, int pt) {
+template <typename Idle>
+__device__ __forceinline__ void forward_substitution(const float* A, float* Tm, int pt, Idle&& idle) {
     const int lane = pt & 31, w = pt >> 5;
+    if (pt >= 64) idle(pt - 64);   // other work while two warps take the diagonal blocks
     if (pt < 64) {
         const int o = 16 * (pt >> 4), c = pt & 15;
         float p[16], x[16];
@@ -262,31 +265,30 @@ struct PrepMaps {
 
 // Prep shared memory (bytes from a 1 KB-aligned base); 111 KB for either
 // gate, so two CTAs share an SM.
-constexpr uint32_t P_KQ = 0;                 // [K_b0 | Q_b0 | K_b1 | Q_b1] (TMA); scalar gate: K~ over K
+constexpr uint32_t P_KQ = 0;                 // [K_b0 | Q_b0 | K_b1 | Q_b1] (TMA);
                                              // per-dimension gate: K e^(G-c), Q e^(G-c) over K, Q
 constexpr uint32_t P_V = 32768;              // [V_b0 | V_b1] (TMA)
 constexpr uint32_t P_AF = 49152;             // A fp32 [64][LDF]; later [W^T; U^T] bf16 [256][64]
 constexpr uint32_t P_TF = P_AF + 64 * LDF * 4;   // T fp32 [64][LDF]
 constexpr uint32_t P_WUT = P_AF;
-constexpr uint32_t P_TW = 86016;             // T diag(beta e^G) bf16 [64 r][64 i]
-constexpr uint32_t P_TU = 94208;             // T diag(beta)
+constexpr uint32_t P_TU = P_AF;              // T diag(beta) bf16 [64 r][64 i] over the dead A scratch
+constexpr uint32_t P_TW = P_AF + 8192;       // T diag(beta e^G) (scalar gate)
+constexpr uint32_t P_KT = 86016;             // K~ = K e^(G_C - G) [b0 | b1] (per-dimension gate: the g
+                                             // tile lands there first)
 constexpr uint32_t P_P = 102400;             // P bf16 [64 r][64 i]
 constexpr uint32_t P_GATE = 110592;          // scalar: G, e^G, e^(G_C-G), beta, u, w, flag;
                                              // per-dimension: beta, gamma_d, e^(ref_d)  (512 floats)
 constexpr uint32_t P_BAR = P_GATE + 8 * 64 * 4;
 constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;
-// per-dimension gate: K~ where the scalar gate keeps T_w / T_u (the g tile
-// lands there first), T diag(beta) over the dead A scratch
-constexpr uint32_t PD_KT = P_TW;             // g bf16 (TMA), then K~ = K e^(G_C - G) [b0 | b1]
-constexpr uint32_t PD_T = P_AF;              // T diag(beta) bf16 [64 r][64 i]
+constexpr uint32_t PD_KT = P_KT;             // per-dimension gate: g bf16 (TMA), then K~
 // staging of the step image for its bulk stores (buffers dead by then)
 constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
-constexpr uint32_t S_QPT = P_TW;             // over T_w / T_u (scalar gate) or K~ (per-dimension
-                                             // gate): dead once the K~^T W and W^T P^T products are done
+constexpr uint32_t S_QPT = P_KT;             // over K~: dead once the K~^T W product is done and
+                                             // its image store has read it
 constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (exact fallback; aliases A / T)
-static_assert(P_TF + 64 * LDF * 4 <= P_TW, "A / T scratch");
-static_assert(P_WUT + 32768 <= P_TW, "[W^T; U^T] tile");
-static_assert(PD_KT + 16384 <= P_P && PD_T + 8192 <= P_TF, "per-dimension tiles");
+static_assert(P_TF + 64 * LDF * 4 <= P_KT, "A / T scratch");
+static_assert(P_WUT + 32768 <= P_KT, "[W^T; U^T] tile");
+static_assert(P_TW + 8192 <= P_TF && P_KT + 16384 <= P_P, "T_u / T_w over A, K~ tile");
 static_assert(S_PHI + 32768 <= P_WUT + 16384 && S_QPT + 16384 <= P_P, "staging clear of the U^T rows and P");
 static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
 static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
@@ -616,7 +618,31 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         }
     }
     __syncthreads();
-    forward_substitution(Af, Tf, tid);
+    forward_substitution(Af, Tf, tid, [&](int t) {
+        if constexpr (!PD) {   // K~ = diag(e^(G_C - G_i)) K into its own tile
+            const float* sFt = gbuf + 128;
+#pragma unroll 1
+            for (int idx = t; idx < 1024; idx += NPR - 64) {   // 16-byte chunks, row-swizzle kept
+                const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
+                uint4 raw = *reinterpret_cast<const uint4*>(sm + P_KQ + blk * 16384 + r * 128 + j * 16);
+                const float f = sFt[r];
+                __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
+                uint4 outv;
+                uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 fv = __bfloat1622float2(e2[e]);
+                    o32[e] = pack_bf16(fv.x * f, fv.y * f);
+                }
+                *reinterpret_cast<uint4*>(sm + P_KT + blk * 8192 + r * 128 + j * 16) = outv;
+            }
+            fence_async_smem();
+        }
+    });
+    if (!PD && tid == 0 && !failed) {   // K~ is final: its image goes out now
+        bulk_store(img + IMG_KT, sm + P_KT, 16384);
+        bulk_commit();
+    }
     // T diag(beta) and T diag(beta e^G) as bf16 K-major [r][i]
     {
         const float* sGam = gbuf + 64;
@@ -634,7 +660,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                 tu[e] = (i <= r) ? tv[e] * sBeta[i] : 0.f;
                 tw[e] = PD ? tu[e] : tu[e] * sGam[i];
             }
-            st_row_chunk(sm + (PD ? PD_T : P_TU), r, j, tu, 1.f);
+            st_row_chunk(sm + P_TU, r, j, tu, 1.f);
             if constexpr (!PD) st_row_chunk(sm + P_TW, r, j, tw, 1.f);
         }
     }
@@ -647,7 +673,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         // T_w; per-dimension gate: (K e^(G-ref))^T T_u^T, rows d times e^(ref_d)
         // in the epilogue
         const uint32_t id = idesc_bf16_f32(128, 64, true, false);
-        const uint32_t tw = PD ? sb + PD_T : sb + P_TW;
+        const uint32_t tw = PD ? sb + P_TU : sb + P_TW;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_WT, sdesc_sw128(sb + P_KQ + k * 2048, 16384, 1024),
@@ -656,7 +682,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_UT, sdesc_sw128(sb + P_V + k * 2048, 8192, 1024),
-                     sdesc_sw128((PD ? sb + PD_T : sb + P_TU) + k * 32, 16, 1024), id, k > 0);
+                     sdesc_sw128(sb + P_TU + k * 32, 16, 1024), id, k > 0);
         mma_commit(&bars[2]);
     }
     wait(2, 0);
@@ -669,42 +695,18 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) st_row_chunk(sm + P_WUT, (warp < 4 ? 0 : 128) + row, j, v + 8 * j, sc);
     }
-    if constexpr (!PD) {   // K~ = diag(e^(G_C - G_i)) K over K (the W product is done with K)
-        const float* sFt = gbuf + 128;
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int idx = tid + NPR * it;                 // 16-byte chunk 0..1023
-            const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
-            uint4* p16 = reinterpret_cast<uint4*>(sm + P_KQ + blk * 16384 + r * 128 + j * 16);
-            uint4 raw = *p16;
-            const float f = sFt[r];
-            __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
-            uint4 outv;
-            uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 fv = __bfloat1622float2(e2[e]);
-                o32[e] = pack_bf16(fv.x * f, fv.y * f);
-            }
-            *p16 = outv;
-        }
-    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0 && !failed) {   // U^T, P (and the scalar gate's K~) are final
+    if (tid == 0 && !failed) {   // U^T and P are final
         bulk_store(img + IMG_UT, sm + P_WUT + 16384, 16384);
         bulk_store(img + IMG_P, sm + P_P, 8192);
-        if constexpr (!PD) {
-            bulk_store(img + IMG_KT, sm + P_KQ, 8192);
-            bulk_store(img + IMG_KT + 8192, sm + P_KQ + 16384, 8192);
-        }
         bulk_commit();
     }
     if (tid == 32 && !failed) {
-        const uint32_t kt = PD ? sb + PD_KT : sb + P_KQ;
-        const uint32_t ktlbo = PD ? 8192 : 16384;
+        const uint32_t kt = sb + P_KT;
+        const uint32_t ktlbo = 8192;
         const uint32_t id1 = idesc_bf16_f32(128, 128, true, false);   // K~^T W
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -718,9 +720,9 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         mma_commit(&bars[3]);
     }
     wait(3, 0);
-    // the per-dimension gate's K~ tile becomes the Qp^T staging: its image store (the
-    // older of the two outstanding groups) must have read it
-    if (PD && tid == 0) bulk_wait_read_all_but_one();
+    // the K~ tile becomes the Qp^T staging: its image store (the older of the two
+    // outstanding groups) must have read it
+    if (tid == 0) bulk_wait_read_all_but_one();
     tc_fence_after();
     __syncthreads();
     const int row = (warp & 3) * 32 + lane;
