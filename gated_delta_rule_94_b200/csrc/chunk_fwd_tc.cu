@@ -27,15 +27,16 @@
 //                       W^T P^T; writes the chunk's step image (Phi, K~, U^T,
 //                       Qp^T, P in bf16, gamma in fp32) to the workspace by
 //                       bulk copies, laid out exactly as the chain kernel's
-//                       shared-memory operands (the wave is sized so the
-//                       workspace stays in L2);
-//   chunk_chain_kernel  one CTA per (batch, head), the serial state chain:
-//                       X = K~^T U (one chunk ahead) + Phi h_bf16 (8 MMA
-//                       steps) in TMEM, then the state pass h' = gamma h + X
-//                       in fp32 registers and its bf16 copy as the next
-//                       operand; off the serial path O = Qp h_bf16 + P U as one
-//                       accumulation of 64 token rows, written by a TMA tensor
-//                       store.
+//                       shared-memory operands;
+//   chunk_chain_kernel  one CTA per (batch, head), the serial state chain on
+//                       the transposed state h^T [v][d]: X^T = U^T K~ (one
+//                       chunk ahead) + h^T Phi^T in TMEM, with the bf16 copy
+//                       of h^T in TMEM as the MMA's A operand, then the state
+//                       pass h'^T = h^T Diag(gamma) + X^T in fp32 registers;
+//                       off the serial path O^T = U^T P^T + h^T Qp^T (value
+//                       rows in the TMEM lanes), written by TMA tensor stores.
+// A wave's prep overlaps the previous wave's chain (programmatic dependent
+// launch); two image buffers alternate between waves.
 // Every mbarrier wait is bounded; a wait that gives up sets the library status
 // word and the kernel winds down without further waits.
 #include <string.h>
@@ -58,11 +59,12 @@ constexpr int LDF = 72;          // fp32 row stride of the A / T scratch (confli
 
 // Step image of one chunk (bytes).  Tiles of bf16 rows of 64 elements with the
 // 128-byte swizzle; a [rows][128] matrix is two such column blocks.
-constexpr uint32_t IMG_PHI = 0;        // Phi  [128 d][128 d'],  blocks of 16 KB (K-major A)
-constexpr uint32_t IMG_KT = 32768;     // K~   [64 i][128 d],    blocks of 8 KB (MN-major A)
-constexpr uint32_t IMG_UT = 49152;     // U^T  [128 v][64 i]     (K-major B)
-constexpr uint32_t IMG_QP = 65536;     // Qp^T [128 d][64 r]     (MN-major A of the output product)
-constexpr uint32_t IMG_P = 81920;      // P    [64 r][64 i]      (K-major A)
+// (MMA roles in the chain's products h^T Phi^T, U^T K~, h^T Qp^T, U^T P^T)
+constexpr uint32_t IMG_PHI = 0;        // Phi  [128 d][128 d'],  blocks of 16 KB (K-major B)
+constexpr uint32_t IMG_KT = 32768;     // K~   [64 i][128 d],    blocks of 8 KB (MN-major B)
+constexpr uint32_t IMG_UT = 49152;     // U^T  [128 v][64 i]     (K-major A)
+constexpr uint32_t IMG_QP = 65536;     // Qp^T [128 d][64 r]     (MN-major B)
+constexpr uint32_t IMG_P = 81920;      // P    [64 r][64 i]      (K-major B)
 constexpr uint32_t IMG_GAM = 90112;    // gamma fp32 [128]
 constexpr uint32_t IMG_BYTES = 90624;
 constexpr size_t WAVE_BYTES = size_t(160) << 20;  // cap of one wave's image buffer
