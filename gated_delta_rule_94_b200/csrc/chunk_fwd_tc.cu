@@ -116,9 +116,15 @@ __device__ __forceinline__ void named_bar(int id, int count) {
 template <int N>
 __device__ __forceinline__ void ld_cols(uint32_t addr, float (&v)[N]) {
     static_assert(N % 16 == 0, "");
+    if constexpr (N % 32 == 0) {
 #pragma unroll
-    for (int j = 0; j < N / 16; ++j)
-        tmem_ld16(addr + 16 * j, *reinterpret_cast<float(*)[16]>(v + 16 * j));
+        for (int j = 0; j < N / 32; ++j)
+            tmem_ld32(addr + 32 * j, *reinterpret_cast<float(*)[32]>(v + 32 * j));
+    } else {
+#pragma unroll
+        for (int j = 0; j < N / 16; ++j)
+            tmem_ld16(addr + 16 * j, *reinterpret_cast<float(*)[16]>(v + 16 * j));
+    }
     tmem_wait_ld();
     reg_fence(v);
 }
