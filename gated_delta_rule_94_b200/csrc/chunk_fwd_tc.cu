@@ -116,7 +116,11 @@ __device__ __forceinline__ void named_bar(int id, int count) {
 template <int N>
 __device__ __forceinline__ void ld_cols(uint32_t addr, float (&v)[N]) {
     static_assert(N % 16 == 0, "");
-    if constexpr (N % 32 == 0) {
+    if constexpr (N % 64 == 0) {
+#pragma unroll
+        for (int j = 0; j < N / 64; ++j)
+            tmem_ld64(addr + 64 * j, *reinterpret_cast<float(*)[64]>(v + 64 * j));
+    } else if constexpr (N % 32 == 0) {
 #pragma unroll
         for (int j = 0; j < N / 32; ++j)
             tmem_ld32(addr + 32 * j, *reinterpret_cast<float(*)[32]>(v + 32 * j));
