@@ -106,6 +106,26 @@ def test_chunk_fwd_noop_sizes():
     assert chunk_call(H=0, q=None, o=None) == _lib.GDN_OK
 
 
+def test_chunk_fwd_workspace_errors():
+    """The tensor-core path (bf16, d = 128) needs its workspace: a buffer
+    smaller than gdn_chunk_fwd_workspace_min_bytes, or none at all, is refused
+    with GDN_ERR_WORKSPACE before anything is launched."""
+    lib = _lib.load()
+    least = lib.gdn_chunk_fwd_workspace_min_bytes(1, 256, 2, 128, 128, 64, 0, 1)
+    assert least > 0
+    base = dict(B=1, T=256, H=2, Dk=128, Dv=128, o=A * 64)
+    assert chunk_call(ws=A * 1024, ws_bytes=least - 16, **base) == _lib.GDN_ERR_WORKSPACE
+    assert chunk_call(ws=None, ws_bytes=least, **base) == _lib.GDN_ERR_WORKSPACE
+
+
+def test_chunk_fwd_index_range():
+    """Token and (batch, head) counts past 2^31 - 1 are refused as unsupported
+    (the kernels index tokens and heads with 32-bit integers)."""
+    assert chunk_call(B=65536, T=65536) == _lib.GDN_ERR_UNSUPPORTED
+    assert chunk_call(B=65536, H=65536) == _lib.GDN_ERR_UNSUPPORTED
+    assert decode_call(N=65536, H=65536) == _lib.GDN_ERR_UNSUPPORTED
+
+
 def decode_call(**over):
     args = dict(q=A, k=A, v=A, beta=A, g=A, gate=1, state=A * 8, o=A * 2, N=2, H=2, Dk=64,
                 Dv=64, dtype=0, stream=None)
