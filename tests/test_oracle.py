@@ -276,3 +276,62 @@ def test_planted_mistake_is_caught():
     g = np.log(np.array(case["a"], float)).reshape(1, 2, 1, 2)
     o = wrong_order(q, k, v, beta, g, np.zeros((1, 1, 2, 2)))
     assert np.max(np.abs(o[0, :, 0] - np.array(case["o"]))) > 1e-3
+
+
+# ------------------------------------------------------------------ rel_err
+# oracle.rel_err is the parity metric every GPU test and every oracle-vs-oracle
+# comparison above uses: max|x - ref| / max|ref| over the whole tensor (the
+# tolerance metric of the workloads: bf16 <= 1e-2, fp32 <= 1e-4).  The values
+# below are worked by hand; each case is chosen so that one plausible slip in
+# the metric changes its value.
+REL_ERR_CASES = [
+    # (x, ref, expected, what a wrong metric would give)
+    ([1.0, -3.0], [2.0, -1.0], 1.0),           # |diff| = (1, 2): max 2; max|ref| = 2
+    ([10.0, 0.0], [1.0, 0.0], 9.0),            # x larger than ref: den from x -> 0.9
+    ([1.0, 1.0, 1.0, 5.0], [1.0, 1.0, 1.0, 1.0], 4.0),   # mean |diff| -> 1.0
+    ([1.0, -5.0], [1.0, 1.0], 6.0),            # diff (0, -6): max without abs -> 0
+    ([-4.0, 3.0], [-4.0, 1.0], 0.5),           # max ref without abs -> 1 -> 2.0
+    ([[0.0, 2.0], [7.0, 1.0]], [[0.0, 2.0], [4.0, -8.0]], 9.0 / 8.0),  # 2-D, whole tensor
+    ([0.0, 0.0], [0.0, 0.0], 0.0),             # both zero
+]
+
+
+@pytest.mark.parametrize("x,ref,expected", REL_ERR_CASES)
+def test_rel_err_hand_worked(x, ref, expected):
+    assert oracle.rel_err(np.array(x), np.array(ref)) == pytest.approx(expected, rel=1e-15)
+
+
+def test_rel_err_zero_reference_reports_absolute_error():
+    """With an all-zero reference there is no scale: the metric is the largest
+    absolute deviation, so any nonzero output fails a tolerance of 1e-2."""
+    assert oracle.rel_err(np.array([0.0, -0.5]), np.zeros(2)) == 0.5
+
+
+def test_rel_err_planted_mistakes_fail_the_pins():
+    """Each plausible slip in the metric fails at least one hand-worked case."""
+    def denominator_from_x(x, ref):
+        return np.max(np.abs(x - ref)) / np.max(np.abs(x))
+
+    def mean_for_max(x, ref):
+        return np.mean(np.abs(x - ref)) / np.max(np.abs(ref))
+
+    def no_abs_numerator(x, ref):
+        return np.max(x - ref) / np.max(np.abs(ref))
+
+    def no_abs_denominator(x, ref):
+        return np.max(np.abs(x - ref)) / np.max(ref)
+
+    def per_row(x, ref):   # max over the last axis only, then the mean of rows
+        return float(np.mean(np.max(np.abs(x - ref), -1) / np.max(np.abs(ref), -1)))
+
+    for wrong in (denominator_from_x, mean_for_max, no_abs_numerator, no_abs_denominator,
+                  per_row):
+        failed = False
+        for x, ref, expected in REL_ERR_CASES:
+            if not np.any(ref):
+                continue
+            with np.errstate(all="ignore"):
+                got = wrong(np.array(x, float), np.array(ref, float))
+            if not np.isclose(got, expected, rtol=1e-12):
+                failed = True
+        assert failed, f"{wrong.__name__} passes every rel_err pin"
