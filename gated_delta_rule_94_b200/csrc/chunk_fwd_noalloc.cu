@@ -6,15 +6,24 @@
 // path, or a process that has handed its whole device memory to a caching
 // allocator it does not control.  gdn_chunk_fwd wants a caller-provided
 // workspace; this entry point supplies it from a fixed scratch array that the
-// library reserves in device memory when it is loaded, so the caller passes
-// only inputs and outputs.
+// library holds in device memory, so the caller passes only inputs and
+// outputs.
 //
 // The scratch is a file-scope __device__ array: every GPU that loads the
-// library holds its kNoAllocScratchBytes until the process exits.  It is shared
-// by every call on a device and keeps the last call's contents; the forward
-// writes every workspace byte it reads before reading it, so nothing needs
-// clearing between calls.  Calls whose work overlaps on the GPU (different
-// streams, or concurrent host threads without ordering) race on the array.
+// library holds its kNoAllocScratchBytes until the process exits.  The CUDA
+// runtime loads this file's module -- and so reserves the array -- the first
+// time the array is used on a device (lazy module loading, the default since
+// CUDA 12.2; with CUDA_MODULE_LOADING=EAGER it happens when the context is
+// created).  A call that has no work (B = 0 or H = 0) performs only that
+// set-up: a caller makes it once per device at start-up, before its own
+// framework takes the device memory and before any stream capture, so that no
+// later call reserves anything.
+//
+// The array is shared by every call on a device and keeps the last call's
+// contents; the forward writes every workspace byte it reads before reading
+// it, so nothing needs clearing between calls.  Calls whose work overlaps on
+// the GPU (different streams, or concurrent host threads without ordering)
+// race on the array.
 #include <mutex>
 
 #include "common.cuh"
@@ -29,15 +38,23 @@ static __device__ __align__(256) unsigned char gdn_noalloc_scratch[kNoAllocScrat
 // Device address of the scratch array on the current device, looked up once
 // per device with that device current.  Host code must not use the array's
 // name as a device pointer: on the host it names a stand-in, not device memory.
+// A failed lookup (for instance out of memory while the module loads) clears
+// the runtime's last-error state, so that no later, unrelated call reports it.
 void* scratch_address() {
     static std::mutex mu;
     static void* cache[64] = {nullptr};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
     std::lock_guard<std::mutex> lock(mu);
     if (!cache[dev]) {
         void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, gdn_noalloc_scratch) != cudaSuccess) return nullptr;
+        if (cudaGetSymbolAddress(&ptr, gdn_noalloc_scratch) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
         cache[dev] = ptr;
     }
     return cache[dev];
@@ -54,6 +71,11 @@ gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, co
                                  void* o, float* final_state, int B, int T, int H, int Dk, int Dv,
                                  int chunk, gdn_dtype dtype, gdn_stream_t stream) {
     const size_t need = gdn_chunk_fwd_workspace_min_bytes(B, T, H, Dk, Dv, chunk, dtype, gate_kind);
+    if ((B == 0 || H == 0) && need != (size_t)-1) {
+        // No work: only the set-up of the current device (module load and the
+        // array's address), so that later calls reserve nothing.
+        return scratch_address() ? GDN_OK : GDN_ERR_CUDA;
+    }
     if (need == (size_t)-1 || need > kNoAllocScratchBytes) {
         // Let the regular entry point report the argument error, or
         // GDN_ERR_WORKSPACE when the shape needs more than the scratch holds;

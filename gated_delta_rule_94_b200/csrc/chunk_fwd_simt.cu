@@ -252,8 +252,7 @@ cudaError_t launch_typed(const ChunkParams& p, cudaStream_t s) {
                                          (int)L::bytes);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((size_t)(p.Dv / BV) * p.H * p.B);
-    kern<<<grid, NT, L::bytes, s>>>(p);
-    return cudaGetLastError();
+    return launch_on(kern, dim3(grid), dim3(NT), L::bytes, s, p);
 }
 
 template <typename Tin>

@@ -43,6 +43,20 @@ struct DecodeParams {
     int N, H;
 };
 
+// Launches `kern` on `s` and returns that launch's own error (never one left
+// over from an earlier call, which cudaGetLastError after a <<<>>> launch
+// would report).
+template <typename... Params, typename... Args>
+inline cudaError_t launch_on(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

@@ -122,10 +122,10 @@ __global__ void __launch_bounds__(NT) decode_step_kernel(DecodeParams p) {
 template <typename Tin, int DK, int DV>
 cudaError_t launch_gate(const DecodeParams& p, int gate, cudaStream_t s) {
     const unsigned grid = (unsigned)((size_t)p.N * p.H);
-    if (gate == kGateNone) decode_step_kernel<Tin, DK, DV, kGateNone><<<grid, NT, 0, s>>>(p);
-    else if (gate == kGateScalar) decode_step_kernel<Tin, DK, DV, kGateScalar><<<grid, NT, 0, s>>>(p);
-    else decode_step_kernel<Tin, DK, DV, kGatePerDim><<<grid, NT, 0, s>>>(p);
-    return cudaGetLastError();
+    auto kern = gate == kGateNone     ? decode_step_kernel<Tin, DK, DV, kGateNone>
+                : gate == kGateScalar ? decode_step_kernel<Tin, DK, DV, kGateScalar>
+                                      : decode_step_kernel<Tin, DK, DV, kGatePerDim>;
+    return launch_on(kern, dim3(grid), dim3(NT), 0, s, p);
 }
 
 template <typename Tin>

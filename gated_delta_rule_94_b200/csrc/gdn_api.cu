@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 #include "gdn.h"
@@ -17,13 +18,24 @@ __device__ unsigned gdn_device_status_word = 0u;
 namespace {
 
 unsigned* status_word_ptr() {
-    // One device address per current device; cached per device ordinal.
+    // One device address per current device, looked up once per device
+    // ordinal under a lock (calls may come from several host threads).  A
+    // failed lookup clears the runtime's last-error state so that it is not
+    // reported later by an unrelated call.
+    static std::mutex mu;
     static unsigned* cache[64] = {nullptr};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
     if (!cache[dev]) {
         void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, gdn_device_status_word) != cudaSuccess) return nullptr;
+        if (cudaGetSymbolAddress(&ptr, gdn_device_status_word) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
         cache[dev] = static_cast<unsigned*>(ptr);
     }
     return cache[dev];

@@ -148,7 +148,9 @@ GDN_API gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
 
 /* Synchronizes `stream`, then reads and clears the library's device status
  * word.  Returns GDN_ERR_TIMEOUT if any kernel since the last call gave up a
- * bounded wait, GDN_ERR_CUDA if the stream reports an error, else GDN_OK. */
+ * bounded wait, GDN_ERR_CUDA if the stream reports an error, else GDN_OK.
+ * The status word's device address is looked up once per device ordinal and
+ * cached; the cache does not survive cudaDeviceReset. */
 GDN_API gdn_status gdn_read_device_status(gdn_stream_t stream);
 
 /* A static, human-readable name for a status code. */
@@ -171,9 +173,18 @@ GDN_API const char* gdn_status_string(gdn_status s);
  *     are reported exactly as by gdn_chunk_fwd.  Shapes whose
  *     gdn_chunk_fwd_workspace_bytes exceeds the scratch run with the waves
  *     the scratch allows.
- *   - Set-up: the first call on each device looks up the array's device
- *     address (cudaGetSymbolAddress) with that device current; make that
- *     first call before any stream capture on the device.
+ *   - Set-up: the array is reserved on a device when the library's module
+ *     holding it is loaded there -- under lazy module loading (the CUDA
+ *     default) on first use, not when the library is loaded.  A call with
+ *     B = 0 or H = 0 (and otherwise valid sizes) does nothing but that
+ *     set-up for the current device: it loads the module and looks up the
+ *     array's device address (cudaGetSymbolAddress) with that device current,
+ *     and returns GDN_OK, or GDN_ERR_CUDA if the device cannot hold the array.
+ *     Make this call once per device at start-up, before the caller's
+ *     framework reserves the device memory and before any stream capture;
+ *     without it the first call with work does the set-up.  The looked-up
+ *     address is cached per device ordinal and does not survive
+ *     cudaDeviceReset.
  *   - Sharing: all calls on a device share the array and it keeps the last
  *     call's contents (the forward needs no cleared scratch).  Calls whose
  *     work overlaps on the GPU -- different streams, or unordered host
