@@ -2,17 +2,23 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One JSON line on rank 0.  A step is one gdn_chunk_fwd over the GDN-style
-scalar-gated workload (B=4, H=16, T=2048, d_k=d_v=128, chunk 64, bf16 tokens,
-fp32 state), inputs resident in HBM; `value` is whole-job tokens/s (all ranks;
-weak scaling: every rank runs its own copy of the workload, no collective on
-the data path).  The same line carries the decode half of the metric: the
-recurrent decode step over 256 sequences x 32 heads (537 MB fp32 state updated
-in place), timed over 128 consecutive steps, as GB/s and fraction of HBM.
+One JSON line on rank 0.  A step is one gdn_chunk_fwd over a whole workload,
+inputs resident in HBM, L2 flushed before every step.  The headline is the
+largest single-GPU workload, the long-sequence scalar-gated forward (B=1,
+H=32, T=65536, d_k=d_v=128, chunk 64, bf16 tokens, fp32 state); `value` is
+its whole-job tokens/s.  The same line carries one record per other forward
+workload (GDN B4 H16 T2048; per-dimension gate B4 H16 T4096; fp32 B1 H2 T256
+d64) and the decode step (256 sequences x 32 heads, 537 MB fp32 state updated
+in place, 128 consecutive steps), each with its own roofline, end-to-end
+figure and CPU baseline.
+
+With N ranks (one per GPU) the heads of every workload are split across the
+ranks, no collective on the data path: total work is fixed (strong scaling).
 
 `--impl reference` times the fp64 CPU oracle (the plain token recurrence) on
-the host cores on the same workload and metric; it is the reference arm of
-this benchmark, a deliberately slow program, not a target.
+the host cores on a bounded sample of the headline workload, reported in the
+same unit; it is the reference arm of this benchmark, a deliberately slow
+program, not a target.
 """
 from __future__ import annotations
 
@@ -28,14 +34,17 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from gated_delta_rule_94_b200 import inputs as gi  # noqa: E402
 
 METRIC = "gated-delta fwd tokens/s & TFLOP/s (% bf16 peak); decode GB/s (% HBM)"
 C = 64
+HEADLINE = 3                      # long-sequence GDN forward, the largest single-GPU workload
+SUBRECORDS = (1, 2, 0)            # the other forward workloads
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 FMA peak of the CUDA-core path: 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def flops_per_token_head(Dk, Dv, chunk=C):
@@ -45,23 +54,26 @@ def flops_per_token_head(Dk, Dv, chunk=C):
     return 2 * chunk * (3 * Dk + 2 * Dv) + 6 * Dk * Dv
 
 
-def chunk_bytes(w: gi.Workload, final_state=True):
-    """Algorithmic HBM bytes of one chunk forward: every input and output
-    token tensor once, the states once each way (when present)."""
+def chunk_bytes(w: gi.Workload, H: int | None = None, final_state=True):
+    """Algorithmic HBM bytes of one chunk forward over H heads (default: all):
+    every input and output token tensor once, the states once each way (when
+    present)."""
+    H = w.H if H is None else H
     es = 2 if w.dtype == "bf16" else 4
-    ntok = w.B * w.T * w.H
+    ntok = w.B * w.T * H
     per_tok = es * (2 * w.Dk + 2 * w.Dv + 1)
     if w.gate == "scalar":
         per_tok += es
     elif w.gate == "per_dim":
         per_tok += es * w.Dk
-    state = w.B * w.H * w.Dk * w.Dv * 4
+    state = w.B * H * w.Dk * w.Dv * 4
     return ntok * per_tok + (state if w.s0_std is not None else 0) + (state if final_state else 0)
 
 
-def decode_bytes_per_step(w: gi.Workload):
+def decode_bytes_per_step(w: gi.Workload, H: int | None = None):
+    H = w.H if H is None else H
     es = 2
-    nh = w.B * w.H
+    nh = w.B * H
     per = 2 * w.Dk * w.Dv * 4 + es * (2 * w.Dk + 2 * w.Dv + 1)
     per += es if w.gate == "scalar" else (es * w.Dk if w.gate == "per_dim" else 0)
     return nh * per
@@ -77,23 +89,33 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback (earlier measurement on this pool)"
 
 
-def ncu_traffic(kernel_name):
-    """DRAM bytes per launch from the committed ncu capture, valid only while
-    the kernel's source is unchanged since the counters were taken."""
+def ncu_traffic(key):
+    """DRAM bytes per forward (or launch) from the committed ncu capture,
+    valid only while every source file it names is unchanged since."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel_name)
+            rec = json.load(f).get(key)
     except (OSError, ValueError):
         return None
     if not rec:
         return None
-    src = os.path.join(ROOT, "gated_delta_rule_94_b200", "csrc", rec["source"])
-    try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    except OSError:
-        return None
-    return rec["bytes_per_launch"] if sha == rec["source_sha256"] else None
+    for src, want in rec["sources"].items():
+        try:
+            sha = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+        except OSError:
+            return None
+        if sha != want:
+            return None
+    return rec["bytes_per_launch"]
+
+
+def shard_heads(H: int, world: int, rank: int) -> tuple[int, int]:
+    """Heads [h0, h1) of rank `rank` when H heads are split over `world` ranks:
+    contiguous, disjoint, covering all heads; sizes differ by at most one."""
+    base, extra = divmod(H, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
 
 
 class ClockSampler:
@@ -176,35 +198,71 @@ def barrier(world):
 
 
 # ----------------------------------------------------------------- CPU oracle
-def oracle_tokens_per_s(w: gi.Workload, min_seconds: float, x=None):
-    """The fp64 oracle on the host cores, over whole copies of the workload,
-    repeated until at least min_seconds of CPU time has run."""
+def oracle_sample(w: gi.Workload, seconds: float):
+    """The fp64 oracle on the host cores over a bounded sample of workload w:
+    min(H, cores) heads of the first B=1 sequence, the sequence cut to the
+    length that takes about `seconds`.  Returns (token-heads/s, cores, text)."""
     import oracle
     oracle.build()
-    if x is None:
-        x = gi.workload_inputs(w)
-    f = gi.to_f64_numpy(x)
     cores = len(os.sched_getaffinity(0))
-    reps, t0 = 0, time.perf_counter()
-    while True:
+    H = min(w.H, cores)
+    T = min(w.T, 512)
+    while True:   # grow the sample until one run takes a tenth of the budget
+        x = gi.workload_inputs(w, B=1, T=T, H=H)
+        f = gi.to_f64_numpy(x)
+        t0 = time.perf_counter()
         oracle.recurrent(f["q"], f["k"], f["v"], f["beta"], f["g"], f["gate_kind"], f["S0"],
                          threads=cores)
-        reps += 1
         el = time.perf_counter() - t0
-        if el >= min_seconds:
+        if el >= seconds / 10 or T >= w.T:
             break
-    return w.B * w.T * reps / el, cores, reps, el
+        T = min(w.T, T * 4)
+    reps, total = 1, el
+    while total < seconds:
+        t0 = time.perf_counter()
+        oracle.recurrent(f["q"], f["k"], f["v"], f["beta"], f["g"], f["gate_kind"], f["S0"],
+                         threads=cores)
+        total += time.perf_counter() - t0
+        reps += 1
+    rate = H * T * reps / total
+    return rate, cores, f"{H} heads x {T} tokens of one sequence, {reps} runs, {total:.1f} s"
+
+
+def oracle_decode_sample(w: gi.Workload, seconds: float):
+    """The oracle's decode: min(cores, N) sequences x H heads, one token step
+    from the workload's initial state, repeated for about `seconds`.
+    Returns (token-heads/s, cores, text)."""
+    import oracle
+    oracle.build()
+    cores = len(os.sched_getaffinity(0))
+    n = min(w.B, cores)
+    x = gi.workload_inputs(w, B=n, T=1)
+    f = gi.to_f64_numpy(x)
+    S0 = f["S0"]
+    reps, total = 0, 0.0
+    while total < seconds or reps == 0:
+        t0 = time.perf_counter()
+        oracle.recurrent(f["q"], f["k"], f["v"], f["beta"], f["g"], f["gate_kind"], S0,
+                         threads=cores)
+        total += time.perf_counter() - t0
+        reps += 1
+    rate = n * w.H * reps / total
+    return rate, cores, f"{n} sequences x {w.H} heads x 1 step, {reps} runs, {total:.1f} s"
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the oracle on a bounded sample of the headline
+    workload per step, rank 0 only."""
     if rank != 0:
         return
-    w = gi.WORKLOADS[1]
+    w = gi.WORKLOADS[HEADLINE]
     import oracle
     oracle.build()
-    x = gi.workload_inputs(w)
-    f = gi.to_f64_numpy(x)
     cores = len(os.sched_getaffinity(0))
+    H = min(w.H, cores)
+    T = 4096
+    x = gi.workload_inputs(w, B=1, T=T, H=H)
+    f = gi.to_f64_numpy(x)
 
     def step():
         oracle.recurrent(f["q"], f["k"], f["v"], f["beta"], f["g"], f["gate_kind"], f["S0"],
@@ -215,19 +273,21 @@ def run_reference(args, world, rank):
     for _ in range(args.steps):
         step()
     el = time.perf_counter() - t0
-    tok_s = w.B * w.T * args.steps / el
-    F = flops_per_token_head(w.Dk, w.Dv) * w.B * w.T * w.H
+    th_per_s = H * T * args.steps / el
+    tok_s = th_per_s / w.H          # tokens/s of the whole workload (all its heads)
+    F = flops_per_token_head(w.Dk, w.Dv)
     line = {
         "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": w.B * w.T / tok_s * 1e3, "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "Dk": w.Dk, "Dv": w.Dv,
                    "chunk": w.chunk, "gate": w.gate, "parallelism": "none (host threads)"},
-        "algorithmic_tflops": F * args.steps / el / 1e12,
+        "algorithmic_tflops": th_per_s * F / 1e12,
         "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"whole workload per step ({w.B * w.T * w.H} token-heads), "
-                                   f"{args.steps} steps"},
+                         "sample": f"{H} heads x {T} tokens of one sequence per step, "
+                                   f"{args.steps} steps; tokens/s of the whole workload = "
+                                   f"token-heads/s / {w.H} heads"},
         "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -235,171 +295,294 @@ def run_reference(args, world, rank):
 
 
 # ------------------------------------------------------------------ GPU arm
-def run_ours(args, world, rank, local):
-    import gated_delta_rule_94_b200 as gdn
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    peaks, peak_src = load_peaks()
-    w = gi.WORKLOADS[1]
-    x = gi.workload_inputs(w)
-    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-    B, T, H, Dk, Dv = w.B, w.T, w.H, w.Dk, w.Dv
-    o = torch.empty((B, T, H, Dv), dtype=d["q"].dtype, device=dev)
-    S = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    kname = gdn.gdn_chunk_fwd_kernel_name(Dk, Dv, d["gate_kind"], d["q"].dtype)
-    nws = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, 64, d["q"].dtype, d["gate_kind"])
-    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev) if nws else None
+class Ctx:
+    def __init__(self, args, world, rank, local):
+        import gated_delta_rule_94_b200 as gdn
+        self.gdn = gdn
+        self.args, self.world, self.rank = args, world, rank
+        torch.cuda.set_device(local)
+        self.dev = torch.device("cuda", local)
+        self.peaks, self.peak_src = load_peaks()
+        l2 = torch.cuda.get_device_properties(self.dev).L2_cache_size
+        self.l2 = l2
+        self.flush = torch.empty(2 * l2, dtype=torch.uint8, device=self.dev)
+        self.stream = torch.cuda.current_stream(self.dev)
+        self.sampler = ClockSampler(self.dev.index if self.dev.index is not None else 0)
 
-    def step():
-        gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["gate_kind"], d["S0"], o, S,
-                          workspace=ws, stream=stream)
 
-    sampler = ClockSampler(dev.index if dev.index is not None else 0)
-    sampler.start()
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    # ---- timed region: K chunk-forward steps, L2 flushed before each
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+def time_forward(ctx: Ctx, wid: int):
+    """Times K forwards of this rank's share of workload `wid` (L2 flushed
+    before each); returns the per-workload record (rank 0) and its launches."""
+    gdn, args, world, rank = ctx.gdn, ctx.args, ctx.world, ctx.rank
+    w = gi.WORKLOADS[wid]
+    h0, h1 = shard_heads(w.H, world, rank)
+    Hl = h1 - h0
+    B, T, Dk, Dv = w.B, w.T, w.Dk, w.Dv
+    launches, per_ms, e2e_ms = 0, [0.0], 0.0
+    kname = gdn.gdn_chunk_fwd_kernel_name(Dk, Dv, w.gate_kind, w.torch_dtype)
+    h2d = d2h = 0
+    if Hl > 0:
+        d = gi.workload_inputs(w, H=Hl, seed=w.seed + rank, device=ctx.dev)
+        o = torch.empty((B, T, Hl, Dv), dtype=w.torch_dtype, device=ctx.dev)
+        S = torch.empty((B, Hl, Dk, Dv), dtype=torch.float32, device=ctx.dev)
+        nws = gdn.gdn_chunk_fwd_workspace_bytes(B, T, Hl, Dk, Dv, 64, w.torch_dtype, w.gate_kind)
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=ctx.dev) if nws else None
+
+        def step():
+            gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], w.gate_kind, d["S0"], o,
+                              S, workspace=ws, stream=ctx.stream)
+        for _ in range(args.warmup):
+            ctx.flush.zero_()
+            step()
+        torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    n0 = gdn.gdn_kernel_launch_count()
     t_wall0 = time.perf_counter()
-    for i in range(args.steps):
-        flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize()
+    if Hl > 0:
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        n0 = gdn.gdn_kernel_launch_count()
+        for i in range(args.steps):
+            ctx.flush.zero_()
+            starts[i].record(ctx.stream)
+            step()
+            ends[i].record(ctx.stream)
+        torch.cuda.synchronize()
+        launches = gdn.gdn_kernel_launch_count() - n0
+        per_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     barrier(world)
-    t_wall1 = time.perf_counter()
-    launches = gdn.gdn_kernel_launch_count() - n0
-    sampler.mark(t_wall0, t_wall1)
-    per_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ctx.sampler.mark(t_wall0, time.perf_counter())
     ms = max_over_ranks(sum(per_ms) / len(per_ms), world)
-    tokens = B * T * world
-    value = tokens / (ms * 1e-3)
-    N_th = B * T * H
-    F = flops_per_token_head(Dk, Dv) * N_th
-    tflops = F / (ms * 1e-3) / 1e12
-    nbytes = chunk_bytes(w)
-    achieved_gbs = nbytes / (ms * 1e-3) / 1e9
+    ms_min = max_over_ranks(min(per_ms), world)
 
-    # ---- decode: 128 consecutive steps over the 256 x 32 state, in place
-    wd = gi.WORKLOADS[4]
-    xd = gi.workload_inputs(wd)
-    dd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in xd.items()}
-    state = dd["S0"].clone()
-    steps_d = wd.T
-    toks = [tuple(dd[n][:, t].contiguous() if dd[n] is not None else None
-                  for n in ("q", "k", "v", "beta", "g")) for t in range(steps_d)]
-    od = torch.empty((wd.B, wd.H, wd.Dv), dtype=dd["q"].dtype, device=dev)
+    # ---- end to end through the public API: pinned host -> device copies of
+    # this step's inputs, the forward, device -> host of o and the final state
+    if Hl > 0 and not args.no_e2e:
+        names = ("q", "k", "v", "beta", "g")
+        host = {n: d[n].cpu().pin_memory() for n in names if d[n] is not None}
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        S_h = torch.empty(S.shape, dtype=S.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = o.numel() * o.element_size() + S.numel() * S.element_size()
 
-    def decode_all():
-        for (q, k, v, b_, g) in toks:
-            gdn.gdn_decode_step(q, k, v, b_, g, dd["gate_kind"], state, od, stream=stream)
-    for _ in range(max(1, args.warmup // 3)):
-        decode_all()
-    torch.cuda.synchronize()
-    dec_ms = []
+        def e2e_step():
+            for n, t in host.items():
+                d[n].copy_(t, non_blocking=True)
+            step()
+            o_h.copy_(o, non_blocking=True)
+            S_h.copy_(S, non_blocking=True)
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
     barrier(world)
-    td0 = time.perf_counter()
-    for _ in range(args.steps):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        decode_all()
-        e1.record(stream)
-        e1.synchronize()
-        dec_ms.append(e0.elapsed_time(e1) / steps_d)
-    td1 = time.perf_counter()
-    sampler.mark(td0, td1)
-    dec_step_ms = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
-    dec_bytes = decode_bytes_per_step(wd)
-    dec_gbs = dec_bytes / (dec_step_ms * 1e-3) / 1e9
-
-    # ---- end to end through the public API: pinned host -> device, compute,
-    # device -> host of o and the final state, every step
-    host = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    S_h = torch.empty(S.shape, dtype=S.dtype).pin_memory()
-    names = ("q", "k", "v", "beta", "g")
-    h2d = sum(host[n].numel() * host[n].element_size() for n in names if host[n] is not None)
-    d2h = o.numel() * o.element_size() + S.numel() * S.element_size()
-
-    def e2e_step():
-        for n in names:
-            if host[n] is not None:
-                d[n].copy_(host[n], non_blocking=True)
-        step()
-        o_h.copy_(o, non_blocking=True)
-        S_h.copy_(S, non_blocking=True)
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    ee0 = torch.cuda.Event(enable_timing=True)
-    ee1 = torch.cuda.Event(enable_timing=True)
-    ee0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    ee1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(ee0.elapsed_time(ee1) / args.steps, world)
-    clocks = sampler.stop()
+    if Hl > 0 and not args.no_e2e:
+        ee0 = torch.cuda.Event(enable_timing=True)
+        ee1 = torch.cuda.Event(enable_timing=True)
+        ee0.record(ctx.stream)
+        for _ in range(args.steps):
+            e2e_step()
+        ee1.record(ctx.stream)
+        torch.cuda.synchronize()
+        e2e_ms = ee0.elapsed_time(ee1) / args.steps
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    h2d_all = max_over_ranks(float(h2d), world) * world
+    d2h_all = max_over_ranks(float(d2h), world) * world
+    if Hl > 0:
+        del d, o, S, ws
+    torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok_s, cores, reps, el = oracle_tokens_per_s(w, args.cpu_seconds, x=x)
-        cpu = {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"whole workload ({N_th} token-heads) x {reps} repetitions, "
-                         f"{el:.1f} s wall"}
+        rate, cores, sample = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": rate / w.H, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": sample + f"; tokens/s of the whole workload = token-heads/s / {w.H}"}
+    if rank != 0:
+        return None, launches
+    peaks = ctx.peaks
+    tokens = B * T                       # every head of every token, over all ranks
+    N_th = B * T * w.H
+    F = flops_per_token_head(Dk, Dv) * N_th
+    nbytes = chunk_bytes(w)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    tflops = F / (ms * 1e-3) / 1e12
+    bf16 = w.dtype == "bf16"
+    rec = {
+        "workload": w.name,
+        "config": {"workload": w.name, "B": B, "T": T, "H": w.H, "Dk": Dk, "Dv": Dv,
+                   "chunk": w.chunk, "gate": w.gate,
+                   "initial_state": "zero (NULL)" if w.s0_std is None else f"N(0, {w.s0_std})",
+                   "final_state": "written", "kernel": kname},
+        "dtype": "bf16" if bf16 else "f32",
+        "ms_per_step": ms, "ms_min": ms_min,
+        "tokens_per_s": tokens / (ms * 1e-3),
+        "tflops": tflops,
+        "pct_bf16_peak": tflops / peaks["bf16_tflops"] if bf16 else None,
+        "algorithmic_flops": F,
+        "hbm_gbs": gbs, "pct_hbm": gbs / peaks["hbm_gbs"],
+        # the forward's launches overlap one another (programmatic dependent
+        # launch), so the unit timed and compared with the roofline is the
+        # whole forward: its algorithmic bytes (or FLOPs) over the CUDA-event
+        # time of the call; traffic is the DRAM bytes of all its launches (ncu)
+        "roofline": ({"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                      "frac": gbs / peaks["hbm_gbs"], "traffic": ncu_traffic(f"chunk_fwd_w{wid}"),
+                      "algorithmic_bytes": nbytes,
+                      "kernel": f"{kname} (one forward: all its launches)",
+                      "peak_source": ctx.peak_src + ", hbm_gbs (copy bandwidth)"} if bf16 else
+                     {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS,
+                      "unit": "TFLOP/s", "frac": tflops / FP32_ALU_TFLOPS,
+                      "traffic": ncu_traffic(f"chunk_fwd_w{wid}"), "algorithmic_flops": F,
+                      "kernel": kname,
+                      "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz"}),
+        "e2e": {"value": tokens / (e2e_ms * 1e-3) if e2e_ms else None, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(h2d_all), "d2h_bytes_per_step": int(d2h_all),
+                "ms_per_step": e2e_ms or None},
+        "gpu_launches": launches,
+        "cpu_baseline": cpu,
+    }
+    return rec, launches
 
+
+def time_decode(ctx: Ctx):
+    """128 consecutive in-place decode steps over this rank's heads, timed as
+    one block per repetition."""
+    gdn, args, world, rank = ctx.gdn, ctx.args, ctx.world, ctx.rank
+    wd = gi.WORKLOADS[4]
+    h0, h1 = shard_heads(wd.H, world, rank)
+    Hl = h1 - h0
+    steps_d = wd.T
+    dec_ms, launches = [0.0], 0
+    if Hl > 0:
+        dd = gi.workload_inputs(wd, H=Hl, seed=wd.seed + rank, device=ctx.dev)
+        state = dd["S0"].clone()
+        toks = [tuple(dd[n][:, t].contiguous() if dd[n] is not None else None
+                      for n in ("q", "k", "v", "beta", "g")) for t in range(steps_d)]
+        od = torch.empty((wd.B, Hl, wd.Dv), dtype=dd["q"].dtype, device=ctx.dev)
+
+        def decode_all():
+            for (q, k, v, b_, g) in toks:
+                gdn.gdn_decode_step(q, k, v, b_, g, wd.gate_kind, state, od, stream=ctx.stream)
+        for _ in range(max(1, args.warmup // 3)):
+            decode_all()
+        torch.cuda.synchronize()
+    barrier(world)
+    td0 = time.perf_counter()
+    if Hl > 0:
+        dec_ms = []
+        n0 = gdn.gdn_kernel_launch_count()
+        for _ in range(args.steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(ctx.stream)
+            decode_all()
+            e1.record(ctx.stream)
+            e1.synchronize()
+            dec_ms.append(e0.elapsed_time(e1) / steps_d)
+        launches = gdn.gdn_kernel_launch_count() - n0
+    barrier(world)
+    ctx.sampler.mark(td0, time.perf_counter())
+    step_ms = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
+
+    # end to end: each step's tokens copied in from pinned host memory, o read
+    # back, the state resident on the device (as in serving)
+    e2e_ms, h2d, d2h = 0.0, 0, 0
+    if Hl > 0 and not args.no_e2e:
+        names = ("q", "k", "v", "beta", "g")
+        host = [[t.cpu().pin_memory() if t is not None else None for t in tk] for tk in toks]
+        od_h = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host[0] if t is not None)
+        d2h = od.numel() * od.element_size()
+
+        def e2e_all():
+            for tk, th in zip(toks, host):
+                for dst, src in zip(tk, th):
+                    if dst is not None:
+                        dst.copy_(src, non_blocking=True)
+                q, k, v, b_, g = tk
+                gdn.gdn_decode_step(q, k, v, b_, g, wd.gate_kind, state, od, stream=ctx.stream)
+                od_h.copy_(od, non_blocking=True)
+        e2e_all()
+        torch.cuda.synchronize()
+    barrier(world)
+    if Hl > 0 and not args.no_e2e:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(ctx.stream)
+        e2e_all()
+        e1.record(ctx.stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / steps_d
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    h2d_all = max_over_ranks(float(h2d), world) * world
+    d2h_all = max_over_ranks(float(d2h), world) * world
+    if Hl > 0:
+        del dd, state, toks, od
+    torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, sample = oracle_decode_sample(wd, args.cpu_seconds)
+        cpu = {"value": rate / wd.H, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": sample + f"; tokens/s = token-heads/s / {wd.H} heads"}
+    if rank != 0:
+        return None, launches
+    peaks = ctx.peaks
+    nbytes = decode_bytes_per_step(wd)
+    gbs = nbytes / (step_ms * 1e-3) / 1e9
+    rec = {
+        "workload": wd.name, "us_per_step": step_ms * 1e3,
+        "gbs": gbs, "pct_hbm": gbs / peaks["hbm_gbs"],
+        "tokens_per_s": wd.B / (step_ms * 1e-3),
+        "algorithmic_bytes_per_step": nbytes, "steps_timed": args.steps * steps_d,
+        "l2": "not flushed between the 128 consecutive steps of one repetition",
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "kernel": "decode_step_kernel",
+                     "traffic": ncu_traffic("decode_step_kernel")},
+        "e2e": {"value": wd.B / (e2e_ms * 1e-3) if e2e_ms else None, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(h2d_all), "d2h_bytes_per_step": int(d2h_all),
+                "us_per_step": e2e_ms * 1e3 if e2e_ms else None},
+        "gpu_launches": launches,
+        "cpu_baseline": cpu,
+    }
+    return rec, launches
+
+
+def run_ours(args, world, rank, local):
+    ctx = Ctx(args, world, rank, local)
+    ctx.sampler.start()
+    head, _ = time_forward(ctx, HEADLINE)
+    subs = {}
+    for wid in SUBRECORDS:
+        if str(wid) in args.workloads.split(","):
+            subs[str(wid)], _ = time_forward(ctx, wid)
+    dec = None
+    if not args.no_decode:
+        dec, _ = time_decode(ctx)
+    clocks = ctx.sampler.stop()
     if rank != 0:
         return
+    w = gi.WORKLOADS[HEADLINE]
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if kname.startswith("chunk_prep_kernel") else "f32",
-        "data": "synthetic",
-        "config": {"workload": w.name, "B": B, "T": T, "H": H, "Dk": Dk, "Dv": Dv,
-                   "chunk": w.chunk, "gate": w.gate, "initial_state": "zero (NULL)",
-                   "final_state": "written", "parallelism": f"dp{world} (whole workload per rank)",
-                   "l2": f"flushed before every step ({2 * l2 >> 20} MiB write)",
-                   "kernel": kname},
-        "tflops": tflops,
-        "pct_bf16_peak": tflops / peaks["bf16_tflops"],
-        "bf16_peak_tflops": peaks["bf16_tflops"],
-        # the forward's kernels overlap one another (programmatic dependent
-        # launch), so the unit timed and compared with the roofline is the
-        # whole forward: its algorithmic bytes over the CUDA-event time of the
-        # call; traffic is the DRAM bytes of all its launches (ncu)
-        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
-                     "traffic": ncu_traffic("chunk_fwd"), "algorithmic_bytes": nbytes,
-                     "kernel": kname + " (one forward: all its launches)",
-                     "peak_source": peak_src + ", hbm_gbs (copy bandwidth)"},
-        "decode": {"workload": wd.name, "us_per_step": dec_step_ms * 1e3,
-                   "gbs": dec_gbs, "pct_hbm": dec_gbs / peaks["hbm_gbs"],
-                   "tokens_per_s": wd.B * world / (dec_step_ms * 1e-3),
-                   "algorithmic_bytes_per_step": dec_bytes, "steps_timed": args.steps * steps_d,
-                   "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
-                                "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
-                                "kernel": "decode_step_kernel",
-                                "traffic": ncu_traffic("decode_step_kernel")}},
-        "e2e": {"value": B * T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": launches,
+        "metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": head["dtype"], "data": "synthetic",
+        "config": dict(head["config"],
+                       parallelism=(f"heads split over {world} ranks, no collective on the "
+                                    "data path" if world > 1 else "one GPU"),
+                       l2=f"flushed before every step ({2 * ctx.l2 >> 20} MiB write)",
+                       inputs="drawn on the device with the workload recipe (seed 0 + rank)"),
+        "tflops": head["tflops"], "pct_bf16_peak": head["pct_bf16_peak"],
+        "bf16_peak_tflops": ctx.peaks["bf16_tflops"],
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
         "clocks": clocks,
-        "cpu_baseline": cpu,
-        "gpu": torch.cuda.get_device_name(dev),
+        "cpu_baseline": head["cpu_baseline"],
+        "workloads": subs,
+        "decode": dec,
+        "gpu": torch.cuda.get_device_name(ctx.dev),
     }
+    _ = w
     print(json.dumps(line), flush=True)
 
 
@@ -409,9 +592,13 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
-                    help="minimum host time of the oracle CPU baseline")
+    ap.add_argument("--workloads", default="1,2,0",
+                    help="forward workloads reported beside the headline (comma separated)")
+    ap.add_argument("--cpu-seconds", type=float, default=3.0,
+                    help="host time of each oracle CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -68,25 +68,28 @@ WORKLOADS = {
 
 def make_inputs(B: int, T: int, H: int, Dk: int, Dv: int, *, dtype=torch.bfloat16,
                 gate: str = "scalar", gate_scale: float = 0.1,
-                s0_std: float | None = None, seed: int = 0) -> dict:
-    """Draw one seeded input set on the CPU.  Returns a dict of CPU tensors:
+                s0_std: float | None = None, seed: int = 0, device="cpu") -> dict:
+    """Draw one seeded input set.  Returns a dict of tensors on `device`:
     q, k, v, beta, g (None for gate "none"), S0 (None when s0_std is None),
-    plus ``gate_kind`` (int)."""
-    gen = torch.Generator(device="cpu").manual_seed(seed)
-    q = torch.randn(B, T, H, Dk, generator=gen)
-    k = torch.randn(B, T, H, Dk, generator=gen)
-    v = torch.randn(B, T, H, Dv, generator=gen)
-    beta_logit = torch.randn(B, T, H, generator=gen)
+    plus ``gate_kind`` (int).  The recipe is the same on every device; the
+    random stream is the device's own, so a CUDA draw gives other values than
+    the CPU draw of the same seed (the parity tests use the CPU draw)."""
+    gen = torch.Generator(device=device).manual_seed(seed)
+    kw = dict(generator=gen, device=device)
+    q = torch.randn(B, T, H, Dk, **kw)
+    k = torch.randn(B, T, H, Dk, **kw)
+    v = torch.randn(B, T, H, Dv, **kw)
+    beta_logit = torch.randn(B, T, H, **kw)
     g = None
     if gate == "scalar":
-        g = -F.softplus(torch.randn(B, T, H, generator=gen)) * gate_scale
+        g = -F.softplus(torch.randn(B, T, H, **kw)) * gate_scale
     elif gate == "per_dim":
-        g = -F.softplus(torch.randn(B, T, H, Dk, generator=gen)) * gate_scale
+        g = -F.softplus(torch.randn(B, T, H, Dk, **kw)) * gate_scale
     elif gate != "none":
         raise ValueError(f"unknown gate {gate!r}")
     S0 = None
     if s0_std is not None:
-        S0 = (torch.randn(B, H, Dk, Dv, generator=gen) * s0_std).contiguous()
+        S0 = (torch.randn(B, H, Dk, Dv, **kw) * s0_std).contiguous()
     q = q / q.norm(dim=-1, keepdim=True)
     k = k / k.norm(dim=-1, keepdim=True)
     beta = torch.sigmoid(beta_logit)
@@ -103,11 +106,13 @@ def make_inputs(B: int, T: int, H: int, Dk: int, Dv: int, *, dtype=torch.bfloat1
 
 
 def workload_inputs(w: Workload, *, T: int | None = None, B: int | None = None,
-                    H: int | None = None) -> dict:
-    """Inputs of a named workload; T/B/H may be overridden for a reduced case."""
-    return make_inputs(B or w.B, T or w.T, H or w.H, w.Dk, w.Dv, dtype=w.torch_dtype,
-                       gate=w.gate, gate_scale=w.gate_scale, s0_std=w.s0_std,
-                       seed=w.seed)
+                    H: int | None = None, seed: int | None = None, device="cpu") -> dict:
+    """Inputs of a named workload; T/B/H (and the seed) may be overridden for
+    a reduced case or one rank's share of the heads."""
+    return make_inputs(w.B if B is None else B, w.T if T is None else T,
+                       w.H if H is None else H, w.Dk, w.Dv, dtype=w.torch_dtype, gate=w.gate,
+                       gate_scale=w.gate_scale, s0_std=w.s0_std,
+                       seed=w.seed if seed is None else seed, device=device)
 
 
 def to_f64_numpy(inputs: dict) -> dict:
