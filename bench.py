@@ -546,7 +546,20 @@ def time_decode(ctx: Ctx):
     return rec, launches
 
 
+def run_only(args, world, rank, local):
+    """One forward workload alone (for profiling): its record, no CPU baseline."""
+    args.no_cpu_baseline = True
+    ctx = Ctx(args, world, rank, local)
+    ctx.sampler.start()
+    rec, _ = time_forward(ctx, args.only)
+    ctx.sampler.stop()
+    if rank == 0:
+        print(json.dumps(rec), flush=True)
+
+
 def run_ours(args, world, rank, local):
+    if args.only is not None:
+        return run_only(args, world, rank, local)
     ctx = Ctx(args, world, rank, local)
     ctx.sampler.start()
     head, _ = time_forward(ctx, HEADLINE)
@@ -599,6 +612,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", type=int, default=None, choices=(0, 1, 2, 3),
+                    help="time one forward workload alone and print its record (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -24,17 +24,18 @@
 //   chunk_prep_kernel   one CTA per (batch, head, chunk), fully parallel: the
 //                       gates, S = [K;Q]K^T, A and P, T, the WY factors as
 //                       W^T = K^T T^T and U^T = V^T T^T, then K~^T W and
-//                       W^T P^T; writes the chunk's step image (Phi, K~, U^T,
-//                       Qp^T, P in bf16, gamma in fp32) to the workspace by
-//                       bulk copies, laid out exactly as the chain kernel's
-//                       shared-memory operands;
+//                       W^T P^T; writes the chunk's step image ([Phi ; Qp],
+//                       [K~^T ; P], U^T in bf16, gamma in fp32) to the
+//                       workspace by bulk copies, laid out exactly as the chain
+//                       kernel's shared-memory operands;
 //   chunk_chain_kernel  one CTA per (batch, head), the serial state chain on
-//                       the transposed state h^T [v][d]: X^T = U^T K~ (one
-//                       chunk ahead) + h^T Phi^T in TMEM, with the bf16 copy
-//                       of h^T in TMEM as the MMA's A operand, then the state
-//                       pass h'^T = h^T Diag(gamma) + X^T in fp32 registers;
-//                       off the serial path O^T = U^T P^T + h^T Qp^T (value
-//                       rows in the TMEM lanes), written by TMA tensor stores.
+//                       the transposed state h^T [v][d]: per chunk two MMAs of
+//                       N = 192 into one TMEM accumulator, D = U^T [K~ | P^T]
+//                       (off the serial path) and D += h^T [Phi^T | Qp^T] with
+//                       the bf16 copy of h^T in TMEM as the A operand; columns
+//                       0..127 of D feed the state pass h'^T = h^T Diag(gamma)
+//                       + X^T in fp32 registers, columns 128..191 are O^T
+//                       (value rows in the TMEM lanes), written by TMA stores.
 // A wave's prep overlaps the previous wave's chain (programmatic dependent
 // launch); two image buffers alternate between waves.
 // Every mbarrier wait is bounded; a wait that gives up sets the library status
@@ -58,15 +59,19 @@ constexpr int NPR = 256;         // prep kernel threads (8 warps)
 constexpr int LDF = 72;          // fp32 row stride of the A / T scratch (conflict-free mma fragments)
 
 // Step image of one chunk (bytes).  Tiles of bf16 rows of 64 elements with the
-// 128-byte swizzle; a [rows][128] matrix is two such column blocks.
-// (MMA roles in the chain's products h^T Phi^T, U^T K~, h^T Qp^T, U^T P^T)
-constexpr uint32_t IMG_PHI = 0;        // Phi  [128 d][128 d'],  blocks of 16 KB (K-major B)
-constexpr uint32_t IMG_KT = 32768;     // K~   [64 i][128 d],    blocks of 8 KB (MN-major B)
-constexpr uint32_t IMG_UT = 49152;     // U^T  [128 v][64 i]     (K-major A)
-constexpr uint32_t IMG_QP = 65536;     // Qp^T [128 d][64 r]     (MN-major B)
-constexpr uint32_t IMG_P = 81920;      // P    [64 r][64 i]      (K-major B)
+// 128-byte swizzle.  The chain runs two products per chunk, each with one
+// K-major B operand of 192 rows (N = 192):
+//   D  = U^T [K~ | P^T]     B = [K~^T ; P]  rows d (128) then r (64), K = i
+//   D += h^T [Phi^T | Qp^T] B = [Phi ; Qp]  rows d' (128) then r (64), K = d
+// so that columns 0..127 of D are the state update X^T and 128..191 the
+// output O^T of the chunk.
+constexpr uint32_t IMG_PQ = 0;         // [Phi ; Qp]: two K-blocks (d 0..63, 64..127) of
+                                       //   [192][64] = 24 KB: Phi rows 0..127, Qp rows 128..191
+constexpr uint32_t IMG_KP = 49152;     // [K~^T ; P]: [192][64] (K~^T rows d, then P rows r)
+constexpr uint32_t IMG_UT = 73728;     // U^T  [128 v][64 i]     (K-major A)
 constexpr uint32_t IMG_GAM = 90112;    // gamma fp32 [128]
 constexpr uint32_t IMG_BYTES = 90624;
+constexpr uint32_t PQ_BLK = 24576;     // one K-block of [Phi ; Qp]
 constexpr size_t WAVE_BYTES = size_t(160) << 20;  // cap of one wave's image buffer
 constexpr int PREP_SLOTS = 2 * 148;                // prep CTAs resident at once on a B200
 
@@ -285,8 +290,8 @@ constexpr uint32_t P_TF = P_AF + 64 * LDF * 4;   // T fp32 [64][LDF]
 constexpr uint32_t P_WUT = P_AF;
 constexpr uint32_t P_TU = P_AF;              // T diag(beta) bf16 [64 r][64 i] over the dead A scratch
 constexpr uint32_t P_TW = P_AF + 8192;       // T diag(beta e^G) (scalar gate)
-constexpr uint32_t P_KT = 86016;             // K~ = K e^(G_C - G) [b0 | b1] (per-dimension gate: the g
-                                             // tile lands there first)
+constexpr uint32_t P_KT = 86016;             // K~^T [128 d][64 i] (K~ = K e^(G_C - G)); the
+                                             // per-dimension gate's g tile lands there first
 constexpr uint32_t P_P = 102400;             // P bf16 [64 r][64 i]
 constexpr uint32_t P_GATE = 110592;          // scalar: G, e^G, e^(G_C-G), beta, u, w, flag;
                                              // per-dimension: beta, gamma_d, e^(ref_d)  (512 floats)
@@ -295,8 +300,9 @@ constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;
 constexpr uint32_t PD_KT = P_KT;             // per-dimension gate: g bf16 (TMA), then K~
 // staging of the step image for its bulk stores (buffers dead by then)
 constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
-constexpr uint32_t S_QPT = P_KT;             // over K~: dead once the K~^T W product is done and
-                                             // its image store has read it
+constexpr uint32_t S_QPT = P_KT;             // Qp [64 r][128 d] as two [64][64] blocks, over K~^T:
+                                             // dead once the K~^T W product is done and its
+                                             // image store has read it
 constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (exact fallback; aliases A / T)
 static_assert(P_TF + 64 * LDF * 4 <= P_KT, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_KT, "[W^T; U^T] tile");
@@ -464,8 +470,10 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                 sRef[8 * cg + e] = exact ? 1.f : gm;
             }
         }
-        // K~ = K e^(c - G) over the g tile (each thread rewrites only what it
-        // has read); factored: K e^(G - c), Q e^(G - c) in place; exact: G kept
+        // K~ = K e^(c - G), written transposed (K~^T [d][i]) over the g tile, which
+        // every thread has read before the barrier above; factored: K e^(G - c),
+        // Q e^(G - c) in place; exact: G kept
+        float ktv[4][8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = r0 + i;
@@ -473,7 +481,6 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             uint8_t* kp = sm + P_KQ + gblk * 16384 + ro;
             const uint4 kraw = *reinterpret_cast<const uint4*>(kp);
             const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
-            uint32_t kt[4];
             if (!exact) {
                 const uint4 qraw = *reinterpret_cast<const uint4*>(kp + 8192);
                 const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
@@ -487,7 +494,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                     const float b0 = __expf(-x0), b1 = __expf(-x1);
                     kc[e] = pack_bf16(kf.x * f0, kf.y * f1);
                     qc[e] = pack_bf16(qf.x * f0, qf.y * f1);
-                    kt[e] = pack_bf16(kf.x * b0, kf.y * b1);
+                    ktv[i][2 * e] = kf.x * b0;
+                    ktv[i][2 * e + 1] = kf.y * b1;
                 }
                 *reinterpret_cast<uint4*>(kp) = make_uint4(kc[0], kc[1], kc[2], kc[3]);
                 *reinterpret_cast<uint4*>(kp + 8192) = make_uint4(qc[0], qc[1], qc[2], qc[3]);
@@ -495,30 +503,33 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 kf = __bfloat1622float2(k2[e]);
-                    kt[e] = pack_bf16(kf.x * __expf(cv[2 * e] - Gp[i][2 * e]),
-                                      kf.y * __expf(cv[2 * e + 1] - Gp[i][2 * e + 1]));
+                    ktv[i][2 * e] = kf.x * __expf(cv[2 * e] - Gp[i][2 * e]);
+                    ktv[i][2 * e + 1] = kf.y * __expf(cv[2 * e + 1] - Gp[i][2 * e + 1]);
                 }
                 float* grow = Gs + r * LDG + 8 * cg;
                 *reinterpret_cast<float4*>(grow) = make_float4(Gp[i][0], Gp[i][1], Gp[i][2], Gp[i][3]);
                 *reinterpret_cast<float4*>(grow + 4) = make_float4(Gp[i][4], Gp[i][5], Gp[i][6], Gp[i][7]);
             }
-            *reinterpret_cast<uint4*>(sm + PD_KT + gblk * 8192 + ro) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)   // row d of K~^T, columns i = r0 .. r0 + 3
+            *reinterpret_cast<uint2*>(sm + PD_KT + sw128_offset(8 * cg + e, r0)) =
+                make_uint2(pack_bf16(ktv[0][e], ktv[1][e]), pack_bf16(ktv[2][e], ktv[3][e]));
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (tid == 0 && !failed) {   // K~ is final: its image goes out now
-            bulk_store(img + IMG_KT, sm + PD_KT, 16384);
+        if (tid == 0 && !failed) {   // K~^T is final: its image goes out now
+            bulk_store(img + IMG_KP, sm + PD_KT, 16384);
             bulk_commit();
         }
-        if (!exact && tid == 32) {   // S = [K e^(G-c); Q e^(G-c)] K~^T
-            const uint32_t id = idesc_bf16_f32(128, 64, false, false);
+        if (!exact && tid == 32) {   // S = [K e^(G-c); Q e^(G-c)] K~^T (B MN-major: K~^T [d][i])
+            const uint32_t id = idesc_bf16_f32(128, 64, false, true);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const uint32_t a = sb + P_KQ + (k >> 2) * 16384 + (k & 3) * 32;
-                const uint32_t bb = sb + PD_KT + (k >> 2) * 8192 + (k & 3) * 32;
-                mma_bf16(tmem + TM_S, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id, k > 0);
+                const uint32_t bb = sb + PD_KT + k * 2048;
+                mma_bf16(tmem + TM_S, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 8192, 1024), id, k > 0);
             }
             mma_commit(&bars[1]);
         }
@@ -631,28 +642,28 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     }
     __syncthreads();
     forward_substitution(Af, Tf, tid, [&](int t) {
-        if constexpr (!PD) {   // K~ = diag(e^(G_C - G_i)) K into its own tile
+        if constexpr (!PD) {   // K~^T [d][i] = (diag(e^(G_C - G_i)) K)^T into its own tile
             const float* sFt = gbuf + 128;
 #pragma unroll 1
-            for (int idx = t; idx < 1024; idx += NPR - 64) {   // 16-byte chunks, row-swizzle kept
-                const int blk = idx >> 9, r = (idx >> 3) & 63, j = idx & 7;
-                uint4 raw = *reinterpret_cast<const uint4*>(sm + P_KQ + blk * 16384 + r * 128 + j * 16);
-                const float f = sFt[r];
-                __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&raw);
-                uint4 outv;
-                uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
+            for (int idx = t; idx < 512; idx += NPR - 64) {   // (token pair, 8 dims) items
+                const int ip = idx & 31, dc = idx >> 5;
+                const int i0 = 2 * ip, blk = dc >> 3, j = dc & 7;
+                const uint8_t* kb = sm + P_KQ + blk * 16384;
+                uint4 r0 = *reinterpret_cast<const uint4*>(kb + i0 * 128 + ((j ^ (i0 & 7)) * 16));
+                uint4 r1 = *reinterpret_cast<const uint4*>(kb + (i0 + 1) * 128 + ((j ^ ((i0 + 1) & 7)) * 16));
+                const float f0 = sFt[i0], f1 = sFt[i0 + 1];
+                const __nv_bfloat16* e0 = reinterpret_cast<const __nv_bfloat16*>(&r0);
+                const __nv_bfloat16* e1 = reinterpret_cast<const __nv_bfloat16*>(&r1);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 fv = __bfloat1622float2(e2[e]);
-                    o32[e] = pack_bf16(fv.x * f, fv.y * f);
-                }
-                *reinterpret_cast<uint4*>(sm + P_KT + blk * 8192 + r * 128 + j * 16) = outv;
+                for (int e = 0; e < 8; ++e)
+                    *reinterpret_cast<uint32_t*>(sm + P_KT + sw128_offset(8 * dc + e, i0)) =
+                        pack_bf16(__bfloat162float(e0[e]) * f0, __bfloat162float(e1[e]) * f1);
             }
             fence_async_smem();
         }
     });
-    if (!PD && tid == 0 && !failed) {   // K~ is final: its image goes out now
-        bulk_store(img + IMG_KT, sm + P_KT, 16384);
+    if (!PD && tid == 0 && !failed) {   // K~^T is final: its image goes out now
+        bulk_store(img + IMG_KP, sm + P_KT, 16384);
         bulk_commit();
     }
     // T diag(beta) and T diag(beta e^G) as bf16 K-major [r][i]
@@ -713,16 +724,15 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     tc_fence_after();
     if (tid == 0 && !failed) {   // U^T and P are final
         bulk_store(img + IMG_UT, sm + P_WUT + 16384, 16384);
-        bulk_store(img + IMG_P, sm + P_P, 8192);
+        bulk_store(img + IMG_KP + 16384, sm + P_P, 8192);
         bulk_commit();
     }
     if (tid == 32 && !failed) {
         const uint32_t kt = sb + P_KT;
-        const uint32_t ktlbo = 8192;
-        const uint32_t id1 = idesc_bf16_f32(128, 128, true, false);   // K~^T W
+        const uint32_t id1 = idesc_bf16_f32(128, 128, false, false);   // K~^T W (both K-major)
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem + TM_FP, sdesc_sw128(kt + k * 2048, ktlbo, 1024),
+            mma_bf16(tmem + TM_FP, sdesc_sw128(kt + k * 32, 16, 1024),
                      sdesc_sw128(sb + P_WUT + k * 32, 16, 1024), id1, k > 0);
         const uint32_t id2 = idesc_bf16_f32(128, 64, false, false);   // W^T P^T
 #pragma unroll
@@ -749,24 +759,27 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         if (hh == 0) named_bar(1, 128);
         else named_bar(3, 128);
         if ((tid & 127) == 0 && !failed) {
-            bulk_store(img + IMG_PHI + hh * 16384, sm + S_PHI + hh * 16384, 16384);
+            bulk_store(img + IMG_PQ + hh * PQ_BLK, sm + S_PHI + hh * 16384, 16384);
             bulk_commit();
         }
     }
-    {   // Qp^T = (Q e^G)^T - W^T P^T, row d: warps 0-3 columns r 0-31, warps 4-7 r 32-63
+    {   // Qp = Q e^G - P W, stored K-major [r][d] (two [64][64] blocks) from row d of
+        // W^T P^T: warps 0-3 tokens r 0-31, warps 4-7 r 32-63; the 32 lanes of a
+        // warp write 32 consecutive d of one row r (one conflict-free wavefront)
         const int hh = warp >> 2;
         float v[32];
         ld_cols<32>(tmem + TM_PWT + lane_off + 32 * hh, v);
         const int d = row;
         const float qs = PD ? sRef[d] : 1.f;
+        uint8_t* qblk = sm + S_QPT + (d >> 6) * 8192;
+        const uint8_t* qsrc = sm + P_KQ + (d >> 6) * 16384 + 8192;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int r = 32 * hh + i;
-            const float qb = (PD ? qs : gbuf[64 + r]) * ld_bf16(sm + P_KQ + (d >> 6) * 16384 + 8192, r, d & 63);
-            v[i] = qb - v[i];
+            const float qb = (PD ? qs : gbuf[64 + r]) * ld_bf16(qsrc, r, d & 63);
+            *reinterpret_cast<__nv_bfloat16*>(qblk + sw128_offset(r, d & 63)) =
+                __float2bfloat16_rn(qb - v[i]);
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) st_row_chunk(sm + S_QPT, d, 4 * hh + j, v + 8 * j, 1.f);
         if (hh == 1 && !failed) {   // gamma_d
             float gam;
             if constexpr (PD) gam = sGamD[d];
@@ -778,7 +791,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     __syncthreads();
     if (tid == 0) {
         if (!failed) {
-            bulk_store(img + IMG_QP, sm + S_QPT, 16384);
+            bulk_store(img + IMG_PQ + 16384, sm + S_QPT, 8192);
+            bulk_store(img + IMG_PQ + PQ_BLK + 16384, sm + S_QPT + 8192, 8192);
             bulk_commit();
         }
         bulk_wait_read();
@@ -794,56 +808,57 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 
 // ------------------------------------------------------------------ chain
 // The chain runs on the transposed state: h^T [v][d] (fp32 in the state-pass
-// registers, its bf16 copy in TMEM as the A operand of the products), so that
-// neither the state's bf16 copy nor the products' h operand touch shared
-// memory:
-//   X^T_n = U_n^T K~_n (issued ahead) + h_n^T Phi_n^T      (two halves of d')
-//   h_{n+1}^T = h_n^T Diag(gamma_n) + X^T_n                 (state pass)
-//   O^T_n = U_n^T P_n^T + h_n^T Qp_n^T                      (output product)
-// The step image is the one the prep writes: Phi is the K-major B operand of
-// h^T Phi^T, K~ the MN-major B of U^T K~, U^T the K-major A of both U^T
-// products, Qp^T the MN-major B and P the K-major B of the output product.
+// registers, its bf16 copy in TMEM as the A operand of the state product), so
+// that neither the state's bf16 copy nor the product's h operand touch shared
+// memory.  Two products per chunk n, both M = 128 (v), N = 192:
+//   D_n  = U_n^T [K~_n | P_n^T]        (K = 64 tokens; A = U^T from shared memory)
+//   D_n += h_n^T [Phi_n^T | Qp_n^T]    (K = 128; A = h^T from TMEM)
+// Columns 0..127 of D_n are X^T_n = U^T K~ + h^T Phi^T, so the state pass forms
+//   h_{n+1}^T = h_n^T Diag(gamma_n) + X^T_n
+// and columns 128..191 are O^T_n = U^T P^T + h^T Qp^T, the chunk's output.
+// The first product needs no state and runs while the state pass of the
+// previous chunk works; only the second is on the serial path.
 
 // Chain kernel shared memory (bytes from a 1 KB-aligned base).
-constexpr uint32_t CH_PHI = 0;          // 2 slots of Phi (32 KB each); the final state's staging
-constexpr uint32_t CH_KT = 65536;       // 2 slots of K~ (16 KB each)
-constexpr uint32_t CH_UT = 98304;       // 2 slots of U^T (16 KB each)
-constexpr uint32_t CH_QP = 131072;      // 2 slots of Qp^T (16 KB each) } the entering state's
-constexpr uint32_t CH_P = 163840;       // 2 slots of P (8 KB each)     } staging (64 KB)
+constexpr uint32_t CH_PQ = 0;           // 2 slots of [Phi ; Qp] (48 KB each); the final state's staging
+constexpr uint32_t CH_KP = 98304;       // 2 slots of [K~^T ; P] (24 KB each)
+constexpr uint32_t CH_UT = 147456;      // 2 slots of U^T (16 KB each)
 constexpr uint32_t CH_OT = 180224;      // 2 slots of the O tile [r][64 v] x 2 blocks for its TMA store
 constexpr uint32_t CH_GAM = 212992;     // 4 slots of gamma (512 B each)
 constexpr uint32_t CH_BAR = 215040;
 constexpr uint32_t CH_SMEM = CH_BAR + 512 + 1024;
 static_assert(CH_SMEM <= 232448, "chain shared memory");
-static_assert(CH_QP + 65536 <= CH_OT + 16384, "entering-state staging over Qp^T / P / O slot 0");
+static_assert(CH_KP == 2 * 2 * PQ_BLK && CH_UT == CH_KP + 2 * 24576 && CH_OT == CH_UT + 2 * 16384,
+              "chain slots");
 
-constexpr int CH_THREADS = 736;   // 23 warps: loader, 2 MMA issuers, 4 output, 16 state
-constexpr int W_OUT = 3;          // first output warp
-constexpr int W_ST = 7;           // first state-pass warp
+constexpr int CH_THREADS = 704;   // 22 warps: loader, MMA issuer, 4 output, 16 state
+constexpr int W_OUT = 2;          // first output warp
+constexpr int W_ST = 6;           // first state-pass warp
 constexpr int N_ST = 16;          // state-pass warps: lane quarter (v) x column quarter (d)
 // Registers: warps spread over the SM's four sub-partitions of 16 K registers
-// each, so 23 warps (six on some sub-partitions) allow at most 85 a thread.
+// each, so 22 warps (six on two sub-partitions) allow at most 85 a thread,
+// 80 in the allocation granularity of 8.
 
-// TMEM columns of the chain kernel (512 allocated).
-constexpr uint32_t TM_HT = 0;      // h^T bf16, lanes v, 2 slots of 64 columns (d pairs)
-constexpr uint32_t TM_OT = 128;    // O^T, lanes v, 2 slots of 64 columns r
-constexpr uint32_t TM_X = 256;     // X^T, lanes v, 2 slots of 128 columns d'
+// TMEM columns of the chain kernel (512 allocated): slot s of D at 256 s
+// (192 columns: X^T then O^T), slot s of the bf16 h^T at 192 + 256 s (lanes v,
+// d pairs packed two to a 32-bit column).
+constexpr uint32_t TM_D = 0;
+constexpr uint32_t TM_HT = 192;
+constexpr uint32_t TM_SLOT = 256;
 
 enum ChainBar {
-    CB_IMG0, CB_IMG1, CB_GAM0, CB_GAM1, CB_GAM2, CB_GAM3, CB_KU0, CB_KU1, CB_KUFREE0, CB_KUFREE1,
-    CB_UFREE0, CB_UFREE1, CB_QP0, CB_QP1, CB_P0, CB_P1, CB_HREADYA0, CB_HREADYA1, CB_HREADYB0,
-    CB_HREADYB1, CB_XFREE0, CB_XFREE1, CB_SDONEA, CB_SDONEB, CB_SFREE0, CB_SFREE1, CB_SDONEO0,
-    CB_SDONEO1, CB_ODONE0, CB_ODONE1, CB_OFREE0, CB_OFREE1, CB_HBFREE0, CB_HBFREE1, CB_S0,
-    CB_S0FREE, CB_FINAL, CB_OFINAL, CB_COUNT
+    CB_KU0, CB_KU1, CB_PQ0, CB_PQ1, CB_GAM0, CB_GAM1, CB_GAM2, CB_GAM3, CB_KUFREE0, CB_KUFREE1,
+    CB_PQFREE0, CB_PQFREE1, CB_SDONE0, CB_SDONE1, CB_HREADY0, CB_HREADY1, CB_XFREE0, CB_XFREE1,
+    CB_OFREE0, CB_OFREE1, CB_FINAL, CB_COUNT
 };
 static_assert(CB_COUNT * 8 <= 512, "barrier space");
 
 // Tensor maps of the chain kernel: o (bf16, [B][T][H*D], 64 x 64 boxes) and the
-// entering / final state (fp32, [B*H][D][D], boxes of 128 rows x 32 columns =
-// 128 B, swizzled so that the lanes of a warp -- 32 consecutive columns v of
-// one row d -- read or write one row of a box without bank conflicts).
+// final state (fp32, [B*H][D][D], boxes of 128 rows x 32 columns = 128 B,
+// swizzled so that the lanes of a warp -- 32 consecutive columns v of one
+// row d -- write one row of a box without bank conflicts).
 struct ChainMaps {
-    CUtensorMap o, s_in, s_out;
+    CUtensorMap o, s_out;
 };
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, A from tensor memory (row m in lane m, k
@@ -858,22 +873,22 @@ __device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
-
-// Element (d, v) of the entering / final state staged as four TMA boxes of
-// [128 d][32 v] fp32 (128-byte swizzle), box v / 32.
+// Element (d, v) of the final state staged as four TMA boxes of [128 d][32 v]
+// fp32 (128-byte swizzle), box v / 32.
 __device__ __forceinline__ uint32_t st_off(int d, int v) {
     return (uint32_t)(v >> 5) * 16384u + (uint32_t)d * 128u +
            ((uint32_t)(((v & 31) >> 2) ^ (d & 7)) << 4) + ((uint32_t)(v & 3) << 2);
 }
 
-// One CTA per (batch, head): walks the wave's chunks in order.  Per chunk n
-// (slot s = n & 1) the state product in two halves of d' (the state pass of
-// the first half runs while the second half's product is on the tensor pipe),
-// the U^T K~ product of the next chunk issued ahead, and the output product
-// from a second issuing thread, so the output never holds up the serial chain.
-// Every barrier that a role waits on is per slot (or per gamma slot) or
-// completes at most once ahead of that wait, so no parity wait can fall two
-// phases behind.
+// One CTA per (batch, head): walks the wave's chunks in order.  Roles:
+//   warp 0       loader: [K~^T ; P] and U^T, then [Phi ; Qp] and gamma, two
+//                chunks ahead, by bulk copies; L2 prefetch and discard
+//   warp 1       MMA issuer: U^T [K~ | P^T] of chunk n + 1 right after the state
+//                product of chunk n, so it runs while the state pass works
+//   warps 2-5    output: O^T from TMEM -> the bf16 O tile -> TMA store
+//   warps 6-21   state pass (lane quarter x column quarter of d)
+// Every barrier is per slot (or per gamma slot) and completes at most once
+// ahead of its wait, so no parity wait can fall two phases behind.
 // UNIFORM_GAMMA: every column of the state decays by the same gamma (scalar gate
 // or none), so the state pass reads one value per chunk, ahead of the product.
 template <bool UNIFORM_GAMMA>
@@ -896,8 +911,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 
     if (tid == 0) {
         for (int i = 0; i < CB_COUNT; ++i)
-            mbar_init(&bars[i], (i == CB_XFREE0 || i == CB_XFREE1 || i == CB_S0FREE) ? N_ST
-                                : (i >= CB_HREADYA0 && i <= CB_HREADYB1) ? N_ST / 2 : 1);
+            mbar_init(&bars[i], (i == CB_HREADY0 || i == CB_HREADY1 || i == CB_XFREE0 ||
+                                 i == CB_XFREE1) ? N_ST : 1);
         fence_mbar_init();
         prefetch_tmap(&maps.o);
     }
@@ -921,67 +936,60 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
     auto img = [&](int nl) { return wsh + (size_t)nl * IMG_BYTES; };
 
     if (warp == 0) {
-        // =========================== loader: K~ and U^T (2 slots, two chunks
-        // ahead), Phi (2 slots), gamma (4 slots); each image prefetched into L2
-        // two chunks ahead, its lines dropped from L2 once loaded
-        if (lane == 0 && p.s0) {   // the entering state, staged over Qp^T / P / O slot 0
-            mbar_arrive_expect_tx(&bars[CB_S0], 65536);
-            for (int cb = 0; cb < 4; ++cb)
-                tma_load_3d(sm + CH_QP + cb * 16384, &maps.s_in, &bars[CB_S0], 32 * cb, 0, bh);
-        }
+        // =========================== loader: [K~^T ; P] and U^T, [Phi ; Qp] (2 slots
+        // each, two chunks ahead), gamma (4 slots); each image prefetched into L2
+        // two chunks ahead, its lines dropped from L2 once loaded and used
         if (lane == 0) {
             for (int nl = 0; nl < 2 && nl < NC; ++nl) bulk_prefetch_l2(img(nl), IMG_BYTES);
         }
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            if (nl >= 2) {   // U^T K~ and P U of chunk nl - 2 are done with slot s
-                wait(CB_KUFREE0 + s, ((nl - 2) >> 1) & 1);
-                wait(CB_UFREE0 + s, ((nl - 2) >> 1) & 1);
-            }
+            if (nl >= 2) wait(CB_KUFREE0 + s, ((nl - 2) >> 1) & 1);   // U^T [K~|P^T] of nl - 2 done
             if (failed) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&bars[CB_KU0 + s], 32768);
-                bulk_load(sm + CH_KT + s * 16384, img(nl) + IMG_KT, 16384, &bars[CB_KU0 + s]);
+                mbar_arrive_expect_tx(&bars[CB_KU0 + s], 24576 + 16384);
+                bulk_load(sm + CH_KP + s * 24576, img(nl) + IMG_KP, 24576, &bars[CB_KU0 + s]);
                 bulk_load(sm + CH_UT + s * 16384, img(nl) + IMG_UT, 16384, &bars[CB_KU0 + s]);
             }
-            if (nl >= 2) wait(CB_SFREE0 + s, ((nl - 2) >> 1) & 1);
+            if (nl >= 2) wait(CB_PQFREE0 + s, ((nl - 2) >> 1) & 1);   // state product of nl - 2 done
             if (failed) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&bars[CB_IMG0 + s], 32768);
-                bulk_load(sm + CH_PHI + s * 32768, img(nl) + IMG_PHI, 32768, &bars[CB_IMG0 + s]);
+                mbar_arrive_expect_tx(&bars[CB_PQ0 + s], 2 * PQ_BLK);
+                bulk_load(sm + CH_PQ + s * 2 * PQ_BLK, img(nl) + IMG_PQ, 2 * PQ_BLK, &bars[CB_PQ0 + s]);
                 mbar_arrive_expect_tx(&bars[CB_GAM0 + (nl & 3)], 512);
                 bulk_load(sm + CH_GAM + (nl & 3) * 512, img(nl) + IMG_GAM, 512, &bars[CB_GAM0 + (nl & 3)]);
                 if (nl + 2 < NC) bulk_prefetch_l2(img(nl + 2), IMG_BYTES);
             }
-            if (nl >= 2) {   // loaded into shared memory: dead in L2 (gamma of chunk
-                             // nl - 3 is known to be in: the state pass has used it)
-                l2_discard(img(nl - 2) + IMG_KT, 32768, lane);   // K~ and U^T
-                l2_discard(img(nl - 2) + IMG_PHI, 32768, lane);
+            if (nl >= 2) {   // both products of chunk nl - 2 are done: its image is dead in L2
+                             // (gamma of chunk nl - 3 too: the state pass has used it)
+                l2_discard(img(nl - 2), IMG_GAM, lane);
                 if (nl >= 3) l2_discard(img(nl - 3) + IMG_GAM, 512, lane);
             }
         }
     } else if (warp == 1) {
-        // =========================== state-product issuer (descriptors built once;
-        // a k-step adds its byte offset / 16 to the start-address field)
+        // =========================== MMA issuer (descriptors built once; a k-step
+        // adds its byte offset / 16 to the start-address field)
         const bool leader = lane == 0;
-        const uint32_t id_ku = idesc_bf16_f32(128, 128, false, true);   // U^T (K-major) K~ (MN-major)
-        const uint32_t id_ph = idesc_bf16_f32(128, 64, false, false);   // h^T (TMEM) Phi^T half (K-major)
-        const uint64_t d_phi = sdesc_sw128(sb + CH_PHI, 16, 1024);
-        const uint64_t d_kt = sdesc_sw128(sb + CH_KT, 8192, 1024);
+        const uint32_t id = idesc_bf16_f32(128, 192, false, false);
+        const uint64_t d_kp = sdesc_sw128(sb + CH_KP, 16, 1024);
         const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
-        // U^T K~ of chunk nl into X^T slot nl & 1 once K~, U^T are in and the
-        // state pass has read X^T of chunk nl - 2 there
+        const uint64_t d_pq = sdesc_sw128(sb + CH_PQ, 16, 1024);
+        // D_nl = U^T [K~ | P^T] once its operands are in and both readers of D in
+        // this slot (state pass and output, chunk nl - 2) are done with it
         auto issue_ku = [&](int nl) {
             const int s = nl & 1;
             wait(CB_KU0 + s, (nl >> 1) & 1);
-            if (nl >= 2) wait(CB_XFREE0 + s, ((nl - 2) >> 1) & 1);
+            if (nl >= 2) {
+                wait(CB_XFREE0 + s, ((nl - 2) >> 1) & 1);
+                wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
+            }
             tc_fence_after();
             if (leader && !failed) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + TM_X + 128 * s, d_ut + ((s * 16384 + k * 32) >> 4),
-                             d_kt + ((s * 16384 + k * 2048) >> 4), id_ku, k > 0);
+                    mma_bf16(tmem + TM_D + TM_SLOT * s, d_ut + ((s * 16384 + k * 32) >> 4),
+                             d_kp + ((s * 24576 + k * 32) >> 4), id, k > 0);
                 mma_commit(&bars[CB_KUFREE0 + s]);
             }
         };
@@ -989,22 +997,17 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
-            wait(CB_IMG0 + s, (nl >> 1) & 1);
-            wait(CB_HREADYA0 + s, (nl >> 1) & 1);
-            wait(CB_HREADYB0 + s, (nl >> 1) & 1);
+            wait(CB_PQ0 + s, (nl >> 1) & 1);
+            wait(CB_HREADY0 + s, (nl >> 1) & 1);
             tc_fence_after();
             if (leader && !failed) {
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {   // columns d' of half hf: Phi rows 64 hf..
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_bf16_ta(tmem + TM_X + 128 * s + 64 * hf, tmem + TM_HT + 64 * s + 8 * k,
-                                    d_phi + ((s * 32768 + (k >> 2) * 16384 + hf * 8192 + (k & 3) * 32) >> 4),
-                                    id_ph, true);
-                    mma_commit(&bars[hf ? CB_SDONEB : CB_SDONEA]);
-                }
-                mma_commit(&bars[CB_SFREE0 + s]);
-                mma_commit(&bars[CB_SDONEO0 + s]);
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ta(tmem + TM_D + TM_SLOT * s, tmem + TM_HT + TM_SLOT * s + 8 * k,
+                                d_pq + ((s * 2 * PQ_BLK + (k >> 2) * PQ_BLK + (k & 3) * 32) >> 4),
+                                id, true);
+                mma_commit(&bars[CB_SDONE0 + s]);
+                mma_commit(&bars[CB_PQFREE0 + s]);
             }
             if (nl + 1 < NC) issue_ku(nl + 1);
         }
@@ -1012,80 +1015,23 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         int final_failed = 0;
         if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
-    } else if (warp == 2) {
-        // =========================== output-product issuer: O^T = U^T P^T + h^T Qp^T
-        // (lanes v, 64 columns r).  U^T P^T needs no state: it is issued as soon
-        // as U^T and P are in, releasing the U^T slot early; h^T Qp^T once the
-        // state product of the chunk is done, so that it fills the tensor pipe
-        // while the state pass works instead of delaying the chain
-        const bool leader = lane == 0;
-        const uint32_t id_pu = idesc_bf16_f32(128, 64, false, false);   // U^T (K-major) P (K-major)
-        const uint32_t id_qh = idesc_bf16_f32(128, 64, false, true);    // h^T (TMEM) Qp^T (MN-major)
-        const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
-        const uint64_t d_p = sdesc_sw128(sb + CH_P, 16, 1024);
-        const uint64_t d_qp = sdesc_sw128(sb + CH_QP, 8192, 1024);
-#pragma unroll 1
-        for (int nl = 0; nl < NC; ++nl) {
-            const int s = nl & 1;
-            wait(CB_KU0 + s, (nl >> 1) & 1);
-            wait(CB_P0 + s, (nl >> 1) & 1);
-            if (nl >= 2) wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
-            tc_fence_after();
-            if (leader && !failed) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + TM_OT + 64 * s, d_ut + ((s * 16384 + k * 32) >> 4),
-                             d_p + ((s * 8192 + k * 32) >> 4), id_pu, k > 0);
-                mma_commit(&bars[CB_UFREE0 + s]);
-            }
-            wait(CB_SDONEO0 + s, (nl >> 1) & 1);
-            wait(CB_QP0 + s, (nl >> 1) & 1);
-            tc_fence_after();
-            if (leader && !failed) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16_ta(tmem + TM_OT + 64 * s, tmem + TM_HT + 64 * s + 8 * k,
-                                d_qp + ((s * 16384 + k * 2048) >> 4), id_qh, true);
-                mma_commit(&bars[CB_ODONE0 + s]);
-                mma_commit(&bars[CB_HBFREE0 + s]);
-            }
-        }
-        if (leader) mma_commit(&bars[CB_OFINAL]);
-        int final_failed = 0;
-        if (!mbar_wait(&bars[CB_OFINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
-        __syncwarp();
     } else if (warp < W_ST) {
         // =========================== output: O^T row v -> the O tile [r][v]
-        // (bf16, swizzled) in its slot -> TMA store; the Qp^T and P slots are
-        // refilled as soon as the output product is done with them
+        // (bf16, swizzled) in its slot -> TMA store
         const int v = (warp & 3) * 32 + lane;
         const bool leader = warp == W_OUT && lane == 0;
-        auto load_qp_p = [&](int nl) {
-            const int s = nl & 1;
-            mbar_arrive_expect_tx(&bars[CB_QP0 + s], 16384);
-            bulk_load(sm + CH_QP + s * 16384, img(nl) + IMG_QP, 16384, &bars[CB_QP0 + s]);
-            mbar_arrive_expect_tx(&bars[CB_P0 + s], 8192);
-            bulk_load(sm + CH_P + s * 8192, img(nl) + IMG_P, 8192, &bars[CB_P0 + s]);
-        };
-        if (leader) {
-            if (p.s0) {   // the entering state's staging has been read
-                if (!mbar_wait(&bars[CB_S0FREE], 0, &failed)) atomicOr(p.status, kStatusTimeout);
-            }
-            for (int nl = 0; nl < 2 && nl < NC; ++nl) load_qp_p(nl);
-        }
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
             if (leader && nl >= 2) bulk_wait_read_all_but_one();   // the store of chunk nl - 2 read slot s
             named_bar(2, 128);
-            wait(CB_ODONE0 + s, (nl >> 1) & 1);
+            wait(CB_SDONE0 + s, (nl >> 1) & 1);
             tc_fence_after();
-            if (leader && !failed && nl + 2 < NC) load_qp_p(nl + 2);
             uint8_t* ot = sm + CH_OT + s * 16384 + (v >> 6) * 8192;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float ov[32];
-                ld_cols<32>(tmem + TM_OT + 64 * s + 32 * half + lane_off, ov);
+                ld_cols<32>(tmem + TM_D + TM_SLOT * s + 128 + 32 * half + lane_off, ov);
 #pragma unroll
                 for (int r = 0; r < 32; ++r)
                     *reinterpret_cast<__nv_bfloat16*>(ot + sw128_offset(32 * half + r, v & 63)) =
@@ -1094,10 +1040,6 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             fence_async_smem();
             tc_fence_before();
             named_bar(2, 128);
-            if (warp == W_OUT) {   // both images were loaded and read: drop them from L2
-                l2_discard(img(nl) + IMG_QP, 16384, lane);
-                l2_discard(img(nl) + IMG_P, 8192, lane);
-            }
             if (leader) {
                 mbar_arrive(&bars[CB_OFREE0 + s]);
                 if (!failed) {
@@ -1114,19 +1056,19 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         // fp32 registers (row v, columns d = 32c..), its bf16 copy into TMEM
         const int v = (warp & 3) * 32 + lane;
         const int c = (warp - W_ST) >> 2;           // column quarter of d
-        const int hf = c >> 1;                      // half of the state product it waits for
         float hv[32];
         // hv = h_{nl-1}^T Diag(gamma_{nl-1}) + X^T_{nl-1}, once the state product of
-        // chunk nl - 1 is done (half hf); a uniform gamma is read before that wait
+        // chunk nl - 1 is done; a uniform gamma is read before that wait
         auto advance = [&](int nl) {
+            const int sp = (nl - 1) & 1;
             const float* gp = reinterpret_cast<const float*>(sm + CH_GAM + ((nl - 1) & 3) * 512) + 32 * c;
             wait(CB_GAM0 + ((nl - 1) & 3), ((nl - 1) >> 2) & 1);
             float g1 = 1.f;
             if constexpr (UNIFORM_GAMMA) g1 = *gp;
-            wait(hf ? CB_SDONEB : CB_SDONEA, (nl - 1) & 1);
+            wait(CB_SDONE0 + sp, ((nl - 1) >> 1) & 1);
             tc_fence_after();
             float xv[32];
-            ld_cols<32>(tmem + TM_X + 128 * ((nl - 1) & 1) + lane_off + 32 * c, xv);
+            ld_cols<32>(tmem + TM_D + TM_SLOT * sp + lane_off + 32 * c, xv);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 float4 g4 = make_float4(g1, g1, g1, g1);
@@ -1141,13 +1083,12 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
             if (nl == 0) {
-                if (p.s0) {   // column v, rows d = 32c.. of the staged state
-                    wait(CB_S0, 0);
+                if (p.s0) {   // column v, rows d = 32c.. of M = S^T: for each d the 32
+                              // lanes read 128 consecutive bytes (L2 only: the carried
+                              // state was written by the previous launch)
+                    const float* src = p.s0 + (size_t)bh * D * D + (size_t)(32 * c) * D + v;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        hv[e] = *reinterpret_cast<const float*>(sm + CH_QP + st_off(32 * c + e, v));
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars[CB_S0FREE]);
+                    for (int e = 0; e < 32; ++e) hv[e] = __ldcg(src + (size_t)e * D);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) hv[e] = 0.f;
@@ -1158,32 +1099,30 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[CB_XFREE0 + ((nl - 1) & 1)]);
             }
-            if (nl >= 2) wait(CB_HBFREE0 + s, ((nl - 2) >> 1) & 1);   // O of chunk nl - 2 is done with it
             {
                 float pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) pk[e] = __uint_as_float(pack_bf16(hv[2 * e], hv[2 * e + 1]));
-                tmem_st16(tmem + TM_HT + 64 * s + 16 * c + lane_off, pk);
+                tmem_st16(tmem + TM_HT + TM_SLOT * s + 16 * c + lane_off, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[(hf ? CB_HREADYB0 : CB_HREADYA0) + s]);
+            if (lane == 0) mbar_arrive(&bars[CB_HREADY0 + s]);
         }
-        if (NC > 0) {   // final state, staged over the Phi slots (free once both halves
-                        // of the last state product are done), written by four TMA stores
+        if (NC > 0) {   // final state, staged over the [Phi ; Qp] slots (free once the
+                        // last state product is done), written by four TMA stores
             advance(NC);
             if (p.s_out) {
-                if (hf == 0) wait(CB_SDONEB, (NC - 1) & 1);   // the other half still reads Phi
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
-                    *reinterpret_cast<float*>(sm + CH_PHI + st_off(32 * c + e, v)) = hv[e];
+                    *reinterpret_cast<float*>(sm + CH_PQ + st_off(32 * c + e, v)) = hv[e];
                 fence_async_smem();
                 named_bar(1, 32 * N_ST);
                 if (warp == W_ST && lane == 0) {
                     if (!failed) {
                         for (int cb = 0; cb < 4; ++cb)
-                            tma_store_3d(&maps.s_out, sm + CH_PHI + cb * 16384, 32 * cb, 0, bh);
+                            tma_store_3d(&maps.s_out, sm + CH_PQ + cb * 16384, 32 * cb, 0, bh);
                         bulk_commit();
                     }
                     bulk_wait_read();
@@ -1305,12 +1244,10 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
     const int nw = (NC + cw - 1) / cw;
     const size_t buf_bytes = (size_t)nbh * cw * IMG_BYTES;
     float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + 2 * buf_bytes) : nullptr;
-    CUtensorMap m_s0, m_sout, m_carry;
-    memset(&m_s0, 0, sizeof(m_s0));
+    CUtensorMap m_sout, m_carry;
     memset(&m_sout, 0, sizeof(m_sout));
     memset(&m_carry, 0, sizeof(m_carry));
-    if (!state_map(&m_s0, p0.s0) || !state_map(&m_sout, p0.s_out) || !state_map(&m_carry, carry))
-        return cudaErrorInvalidValue;
+    if (!state_map(&m_sout, p0.s_out) || !state_map(&m_carry, carry)) return cudaErrorInvalidValue;
     // Every launch but the first may start before its predecessor ends
     // (programmatic dependent launch); the kernels order themselves with
     // griddepcontrol (see chunk_prep_kernel and chunk_chain_kernel).
@@ -1341,7 +1278,6 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
         cfg.dynamicSmemBytes = CH_SMEM;
         cfg.numAttrs = 1;
         ChainMaps cm = cmap0;
-        cm.s_in = (w == 0) ? m_s0 : m_carry;
         cm.s_out = (w + 1 == nw) ? m_sout : m_carry;
         e = cudaLaunchKernelEx(&cfg, chain, cm, p);
         if (e != cudaSuccess) return e;
