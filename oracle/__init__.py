@@ -20,6 +20,17 @@ Three independent restatements of what the operator computes:
   W = T diag(beta) K_bar, U = T diag(beta) V obtained by forward substitution
   ("OSDN ...", sec. 2.1: the chunk Gram matrix and the WY pipeline).
 
+And the preconditioned variant ("OSDN ...", sec. 2.1-2.3), in two phases:
+
+* :func:`osdn_precondition` -- Phase 1, the O(d_k) scan over the key stream:
+  the diagonal preconditioner d_t, updated by online gradient descent on the
+  closed-form surrogate h_t(d) = ((1 - beta_t <d, k_t^2>)^2 - 1) / (2 |k_t|^2)
+  (sec. 2.2), with the retention gate r_t of adaptive preconditioner forgetting
+  (sec. 2.3), and the write keys kw_t = d_t (.) k_t;
+* :func:`recurrent_wk` -- Phase 2, the recurrence with the write key kw_t in
+  place of k_t in the write (sec. 2.1); :func:`brute_force` and
+  :func:`chunk_form` take the same optional ``kw``.
+
 Readings taken where the pages are garbled or silent (each is pinned by a test
 in tests/test_oracle.py):
   * orientation: S_t k_t = v_t after an exact write, so in M = S^T form
@@ -31,7 +42,15 @@ in tests/test_oracle.py):
     to its own position (Gamma_r), the key of the state update by the decay
     from its position to the chunk end (Gamma_C / Gamma_i);
   * g = log a is the gate input, cumulated in the log domain;
-  * no 1/sqrt(d) scale on q; q and k are used as given.
+  * no 1/sqrt(d) scale on q; q and k are used as given;
+  * OSDN: the preconditioner step descends the surrogate (the page's APF line
+    prints "+ eta grad h"; the text calls the update online gradient descent
+    on h_t, so the step is -eta grad h); d_1 = 1 unless given (the identity
+    preconditioner, so the first token is a plain delta-rule step); no
+    projection of d; k_t^2 is elementwise; the write key of token t uses d_t,
+    the preconditioner before token t's own feedback; a token with k_t = 0
+    leaves d unchanged (its surrogate has no direction); with gates the decay
+    acts before the erase exactly as in the plain rule.
 """
 from __future__ import annotations
 
@@ -70,6 +89,10 @@ def _load():
                                              ctypes.c_long, ctypes.c_long, ctypes.c_long,
                                              ctypes.c_long, ctypes.c_long, ctypes.c_int]
         lib.gdn_oracle_recurrent.restype = ctypes.c_int
+        lib.gdn_oracle_recurrent_wk.argtypes = [dp, dp, dp, dp, dp, dp, ctypes.c_int, dp, dp, dp,
+                                                ctypes.c_long, ctypes.c_long, ctypes.c_long,
+                                                ctypes.c_long, ctypes.c_long, ctypes.c_int]
+        lib.gdn_oracle_recurrent_wk.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -108,6 +131,66 @@ def recurrent(q, k, v, beta, g, gate_kind, S0=None, threads: int | None = None):
     return o, S
 
 
+def recurrent_wk(q, k, kw, v, beta, g, gate_kind, S0=None, threads: int | None = None):
+    """The recurrence with a separate write key (OSDN Phase 2), fp64:
+    per token M <- Diag(a) M; r = beta (v - M^T k); M <- M + kw r^T; o = M^T q.
+    kw: [B, T, H, Dk].  Returns (o, S) as :func:`recurrent`."""
+    q, k, kw, v, beta, g, S0 = map(_f64, (q, k, kw, v, beta, g, S0))
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if gate_kind == GATE_NONE:
+        g = None
+    o = np.empty((B, T, H, Dv), np.float64)
+    S = np.empty((B, H, Dk, Dv), np.float64)
+    rc = _load().gdn_oracle_recurrent_wk(_ptr(q), _ptr(k), _ptr(kw), _ptr(v), _ptr(beta),
+                                         _ptr(g), int(gate_kind), _ptr(S0), _ptr(o), _ptr(S),
+                                         B, T, H, Dk, Dv, int(threads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"gdn_oracle_recurrent_wk failed with code {rc}")
+    return o, S
+
+
+def osdn_surrogate(d, k, beta):
+    """h_t(d) = ((1 - beta <d, k^2>)^2 - 1) / (2 |k|^2), the closed form of
+    (f_t(S_t) - f_t(S_{t-1})) / |grad f_t(S_{t-1})|_F^2 for the
+    right-preconditioned step ("OSDN ...", sec. 2.2)."""
+    d, k = np.asarray(d, np.float64), np.asarray(k, np.float64)
+    s = beta * np.dot(d, k * k)
+    return ((1.0 - s) ** 2 - 1.0) / (2.0 * np.dot(k, k))
+
+
+def osdn_precondition(k, beta, eta, r=None, d0=None):
+    """Phase 1 of OSDN, fp64, token by token for every (batch, head):
+
+        kw_t    = d_t (.) k_t                        (the write key of token t)
+        grad    = -beta_t (1 - beta_t <d_t, k_t^2>) k_t^2 / |k_t|^2
+                                                     (= grad_d h_t(d_t))
+        d_{t+1} = r_t d_t - eta grad
+
+    ("OSDN ...", sec. 2.1 the preconditioned key, sec. 2.2 the surrogate and
+    its online gradient step, sec. 2.3 the retention gate r_t; r = None means
+    r_t = 1, no forgetting).  k: [B, T, H, Dk]; beta, r: [B, T, H]; d0:
+    [B, H, Dk] or None (ones).  Returns (kw [B, T, H, Dk], d_final [B, H, Dk]).
+    """
+    k = np.asarray(k, np.float64)
+    beta = np.asarray(beta, np.float64)
+    B, T, H, Dk = k.shape
+    d = np.ones((B, H, Dk)) if d0 is None else np.array(d0, np.float64, copy=True)
+    kw = np.empty_like(k)
+    for t in range(T):
+        kt = k[:, t]                                   # [B, H, Dk]
+        u = kt * kt
+        n = u.sum(-1)                                  # |k_t|^2
+        s = (d * u).sum(-1)                            # <d_t, k_t^2>
+        bt = beta[:, t]
+        kw[:, t] = d * kt
+        with np.errstate(divide="ignore", invalid="ignore"):
+            step = np.where(n > 0, eta * bt * (1.0 - bt * s) / np.where(n > 0, n, 1.0), 0.0)
+        rt = 1.0 if r is None else np.asarray(r, np.float64)[:, t][..., None]
+        d = rt * d + step[..., None] * u
+    return kw, d
+
+
 def _decay_vector(g, gate_kind, b, t, h, Dk):
     if gate_kind == GATE_NONE:
         return np.ones(Dk)
@@ -116,16 +199,19 @@ def _decay_vector(g, gate_kind, b, t, h, Dk):
     return np.exp(g[b, t, h])
 
 
-def brute_force(q, k, v, beta, g, gate_kind, S0=None):
+def brute_force(q, k, v, beta, g, gate_kind, S0=None, kw=None):
     """Explicit-product expansion of the recurrence, in the S (d_v x d_k) form.
 
-    With E_t = Diag(a_t) (I - beta_t k_t k_t^T) (a d_k x d_k matrix; scalar gate:
-    Diag(a_t) = a_t I), the recurrence S_t = S_{t-1} E_t + beta_t v_t k_t^T gives
-        S_t = S_0 E_1 ... E_t + sum_{i<=t} beta_i v_i k_i^T E_{i+1} ... E_t,
+    With E_t = Diag(a_t) (I - beta_t k_t kw_t^T) (a d_k x d_k matrix; scalar gate:
+    Diag(a_t) = a_t I; kw = k unless a write key is given), the recurrence
+    S_t = S_{t-1} E_t + beta_t v_t kw_t^T gives
+        S_t = S_0 E_1 ... E_t + sum_{i<=t} beta_i v_i kw_i^T E_{i+1} ... E_t,
     evaluated here literally for every t; o_t = S_t q_t.  Meant for T <= 8.
     Returns (o [B,T,H,Dv], M_final = S_T^T [B,H,Dk,Dv]).
     """
-    q, k, v, beta, g, S0 = map(_f64, (q, k, v, beta, g, S0))
+    q, k, v, beta, g, S0, kw = map(_f64, (q, k, v, beta, g, S0, kw))
+    if kw is None:
+        kw = k
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
     o = np.zeros((B, T, H, Dv))
@@ -136,8 +222,9 @@ def brute_force(q, k, v, beta, g, gate_kind, S0=None):
             E = []
             for t in range(T):
                 kt = k[b, t, h][:, None]
+                kwt = kw[b, t, h][:, None]
                 a = _decay_vector(g, gate_kind, b, t, h, Dk)
-                E.append(np.diag(a) @ (I - beta[b, t, h] * (kt @ kt.T)))
+                E.append(np.diag(a) @ (I - beta[b, t, h] * (kt @ kwt.T)))
             for t in range(T):
                 prod = I.copy()
                 for s in range(t + 1):
@@ -147,7 +234,7 @@ def brute_force(q, k, v, beta, g, gate_kind, S0=None):
                     tail = I.copy()
                     for s in range(i + 1, t + 1):
                         tail = tail @ E[s]
-                    S_t = S_t + beta[b, i, h] * (v[b, i, h][:, None] @ k[b, i, h][None, :]) @ tail
+                    S_t = S_t + beta[b, i, h] * (v[b, i, h][:, None] @ kw[b, i, h][None, :]) @ tail
                 o[b, t, h] = S_t @ q[b, t, h]
                 if t == T - 1:
                     M_final[b, h] = S_t.T
@@ -170,7 +257,7 @@ def forward_substitution_inverse(A):
     return Tm
 
 
-def chunk_form(q, k, v, beta, g, gate_kind, S0=None, C: int = 64):
+def chunk_form(q, k, v, beta, g, gate_kind, S0=None, C: int = 64, kw=None):
     """Chunkwise evaluation (fp64) of the same operator, chunk length C.
 
     Per chunk, with h the entering M (= S^T, d_k x d_v), G_r = sum_{i<=r} log a_i
@@ -182,9 +269,14 @@ def chunk_form(q, k, v, beta, g, gate_kind, S0=None, C: int = 64):
       D   = U - W h                            (the chunk's pseudo-values)
       O   = Q_bar h + Tril_incl(Q_bar K_breve^T) D,   Q_bar = Gamma * Q
       h'  = Diag(gamma_C) h + K_tilde^T D,  K_tilde_i = k_i * Gamma_C / Gamma_i
-    The last chunk may be shorter than C.  Returns (o, M_final).
+    The last chunk may be shorter than C.  With a write key kw (OSDN), kw
+    replaces k in K_breve (the Gram matrix and the intra-chunk scores) and in
+    K_tilde (the state update); the read key k stays in K_bar (sec. 2.1 of the
+    OSDN page).  Returns (o, M_final).
     """
-    q, k, v, beta, g, S0 = map(_f64, (q, k, v, beta, g, S0))
+    q, k, v, beta, g, S0, kw = map(_f64, (q, k, v, beta, g, S0, kw))
+    if kw is None:
+        kw = k
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
     o = np.zeros((B, T, H, Dv))
@@ -197,6 +289,7 @@ def chunk_form(q, k, v, beta, g, gate_kind, S0=None, C: int = 64):
                 n = c1 - c0
                 Q = q[b, c0:c1, h_]
                 K = k[b, c0:c1, h_]
+                KW = kw[b, c0:c1, h_]
                 V = v[b, c0:c1, h_]
                 bt = beta[b, c0:c1, h_]
                 if gate_kind == GATE_NONE:
@@ -213,8 +306,8 @@ def chunk_form(q, k, v, beta, g, gate_kind, S0=None, C: int = 64):
                 lower = np.tril(np.ones((n, n), bool))
                 diff = np.where(lower[:, :, None], diff, -np.inf)
                 dec = np.exp(diff)
-                KK = np.einsum("rd,id,rid->ri", K, K, dec)
-                QK = np.einsum("rd,id,rid->ri", Q, K, dec)
+                KK = np.einsum("rd,id,rid->ri", K, KW, dec)
+                QK = np.einsum("rd,id,rid->ri", Q, KW, dec)
                 A = np.tril(bt[:, None] * KK, -1)
                 Tm = forward_substitution_inverse(A)
                 K_bar = Gam * K
@@ -223,7 +316,7 @@ def chunk_form(q, k, v, beta, g, gate_kind, S0=None, C: int = 64):
                 D = U - W @ h
                 Q_bar = Gam * Q
                 o[b, c0:c1, h_] = Q_bar @ h + np.tril(QK) @ D
-                K_tilde = K * np.exp(G[n - 1][None, :] - G)
+                K_tilde = KW * np.exp(G[n - 1][None, :] - G)
                 h = gamma_C[:, None] * h + K_tilde.T @ D
             M_final[b, h_] = h
     return o, M_final

@@ -32,6 +32,14 @@
  *   g    [B][T][H] (gate_kind 1) or [B][T][H][Dk] (gate_kind 2), g = log a;
  *   S0   [B][H][Dk][Dv] or NULL (zero); o [B][T][H][Dv]; S_out [B][H][Dk][Dv].
  * Summation order is fixed (ascending index); build without -ffast-math.
+ *
+ * gdn_oracle_recurrent_wk is the same recurrence with a separate write key
+ * kw_t (the preconditioned key of "OSDN ...", sec. 2.1: right-preconditioning
+ * the gradient step by D_t = diag(d_t) is the update
+ *     S_t = S_{t-1} + beta_t (v_t - S_{t-1} k_t) (d_t (.) k_t)^T,
+ * so the residual is read with k_t and written along kw_t = d_t (.) k_t).  In
+ * M form step 4 becomes M <- M + kw_t r^T; every other step is unchanged.
+ * With kw = k it is gdn_oracle_recurrent exactly (same operations, same order).
  */
 #include <math.h>
 #include <stdlib.h>
@@ -41,12 +49,12 @@
 #define ORACLE_GATE_SCALAR 1
 #define ORACLE_GATE_PER_DIM 2
 
-int gdn_oracle_recurrent(const double* q, const double* k, const double* v,
-                         const double* beta, const double* g, int gate_kind,
-                         const double* S0, double* o, double* S_out,
-                         long B, long T, long H, long Dk, long Dv, int nthreads)
+static int recurrent_impl(const double* q, const double* k, const double* kw,
+                          const double* v, const double* beta, const double* g,
+                          int gate_kind, const double* S0, double* o, double* S_out,
+                          long B, long T, long H, long Dk, long Dv, int nthreads)
 {
-    if (!q || !k || !v || !beta || !o || !S_out) return 1;
+    if (!q || !k || !kw || !v || !beta || !o || !S_out) return 1;
     if (gate_kind != ORACLE_GATE_NONE && !g) return 1;
     if (gate_kind < 0 || gate_kind > 2) return 1;
     if (B < 0 || T < 0 || H < 0 || Dk < 1 || Dv < 1) return 1;
@@ -72,6 +80,7 @@ int gdn_oracle_recurrent(const double* q, const double* k, const double* v,
             const long tok = (b * T + t) * H + h;
             const double* qt = q + tok * Dk;
             const double* kt = k + tok * Dk;
+            const double* kwt = kw + tok * Dk;
             const double* vt = v + tok * Dv;
             const double bt = beta[tok];
 
@@ -93,9 +102,9 @@ int gdn_oracle_recurrent(const double* q, const double* k, const double* v,
             }
             /* 3. r = beta (v - x) */
             for (long j = 0; j < Dv; ++j) r[j] = bt * (vt[j] - x[j]);
-            /* 4. M += k r^T */
+            /* 4. M += kw r^T (the write key; kw = k for the plain rule) */
             for (long i = 0; i < Dk; ++i) {
-                const double ki = kt[i];
+                const double ki = kwt[i];
                 for (long j = 0; j < Dv; ++j) M[i * Dv + j] += ki * r[j];
             }
             /* 5. o = M^T q */
@@ -110,4 +119,22 @@ int gdn_oracle_recurrent(const double* q, const double* k, const double* v,
         free(r);
     }
     return failed ? 2 : 0;
+}
+
+int gdn_oracle_recurrent(const double* q, const double* k, const double* v,
+                         const double* beta, const double* g, int gate_kind,
+                         const double* S0, double* o, double* S_out,
+                         long B, long T, long H, long Dk, long Dv, int nthreads)
+{
+    return recurrent_impl(q, k, k, v, beta, g, gate_kind, S0, o, S_out, B, T, H, Dk, Dv,
+                          nthreads);
+}
+
+int gdn_oracle_recurrent_wk(const double* q, const double* k, const double* kw,
+                            const double* v, const double* beta, const double* g,
+                            int gate_kind, const double* S0, double* o, double* S_out,
+                            long B, long T, long H, long Dk, long Dv, int nthreads)
+{
+    return recurrent_impl(q, k, kw, v, beta, g, gate_kind, S0, o, S_out, B, T, H, Dk, Dv,
+                          nthreads);
 }
