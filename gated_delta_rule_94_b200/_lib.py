@@ -26,7 +26,7 @@ EXPORTED = ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd_wor
             "gdn_decode_step",
             "gdn_read_device_status", "gdn_status_string", "gdn_abi_version",
             "gdn_kernel_launch_count", "gdn_chunk_fwd_kernel_name", "gdn_chunk_fwd_noalloc",
-            "gdn_chunk_fwd_noalloc_scratch_bytes")
+            "gdn_chunk_fwd_noalloc_scratch_bytes", "gdn_osdn_precondition", "gdn_chunk_fwd_wk")
 
 _lib = None
 
@@ -69,6 +69,12 @@ def load() -> ctypes.CDLL:
     lib.gdn_chunk_fwd_noalloc.restype = i
     lib.gdn_chunk_fwd_noalloc_scratch_bytes.argtypes = []
     lib.gdn_chunk_fwd_noalloc_scratch_bytes.restype = sz
+    lib.gdn_osdn_precondition.argtypes = [vp, vp, vp, ctypes.c_float, vp, vp, vp, i, i, i, i, i,
+                                          vp]
+    lib.gdn_osdn_precondition.restype = i
+    lib.gdn_chunk_fwd_wk.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, vp,
+                                     sz, vp]
+    lib.gdn_chunk_fwd_wk.restype = i
     _lib = lib
     return lib
 
@@ -166,6 +172,49 @@ def gdn_chunk_fwd(q, k, v, beta, g, gate_kind, initial_state, o, final_state, *,
         raise GdnError(st, "gdn_chunk_fwd")
 
 
+def gdn_chunk_fwd_wk(q, k, k_write, v, beta, g, gate_kind, initial_state, o, final_state, *,
+                     chunk=64, workspace=None, stream=None) -> None:
+    """gdn_chunk_fwd with a separate write key k_write [B,T,H,Dk] (or None)."""
+    _check_contig(q=q, k=k, k_write=k_write, v=v, beta=beta, g=g, initial_state=initial_state,
+                  o=o, final_state=final_state)
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dtype_code(q.dtype)
+    for name, t in (("k", k), ("k_write", k_write), ("v", v), ("beta", beta), ("g", g), ("o", o)):
+        if t is not None and t.dtype != q.dtype:
+            raise TypeError(f"{name} must have dtype {q.dtype}")
+    for name, t in (("initial_state", initial_state), ("final_state", final_state)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().gdn_chunk_fwd_wk(_ptr(q), _ptr(k), _ptr(k_write), _ptr(v), _ptr(beta), _ptr(g),
+                                 int(gate_kind), _ptr(initial_state), _ptr(o), _ptr(final_state),
+                                 B, T, H, Dk, Dv, chunk, dt, _ptr(workspace), ws_bytes,
+                                 _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd_wk")
+
+
+def gdn_osdn_precondition(k, beta, r, eta, d0, k_write, d_final, *, stream=None) -> None:
+    """Phase 1 of the preconditioned delta rule: write keys k_write = d (.) k.
+    k, k_write [B,T,H,Dk]; beta, r [B,T,H] (r may be None); d0, d_final
+    [B,H,Dk] fp32 or None."""
+    _check_contig(k=k, beta=beta, r=r, d0=d0, k_write=k_write, d_final=d_final)
+    B, T, H, Dk = k.shape
+    dt = _dtype_code(k.dtype)
+    for name, t in (("beta", beta), ("r", r), ("k_write", k_write)):
+        if t is not None and t.dtype != k.dtype:
+            raise TypeError(f"{name} must have dtype {k.dtype}")
+    for name, t in (("d0", d0), ("d_final", d_final)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    st = load().gdn_osdn_precondition(_ptr(k), _ptr(beta), _ptr(r), float(eta), _ptr(d0),
+                                      _ptr(k_write), _ptr(d_final), B, T, H, Dk, dt,
+                                      _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_osdn_precondition")
+
+
 def gdn_decode_step(q, k, v, beta, g, gate_kind, state, o, *, stream=None) -> None:
     """Enqueue one decode step.  q, k [N,H,Dk]; v, o [N,H,Dv]; beta [N,H];
     g [N,H] or [N,H,Dk] or None; state [N,H,Dk,Dv] fp32, updated in place."""
@@ -202,6 +251,27 @@ def chunk_fwd(q, k, v, beta, g=None, initial_state=None, *, output_final_state=T
     gdn_chunk_fwd(q, k, v, beta, g, gate, initial_state, o, S, chunk=chunk, workspace=ws,
                   stream=stream)
     return o, S
+
+
+def osdn_chunk_fwd(q, k, v, beta, g=None, initial_state=None, *, eta, r=None, d0=None,
+                   output_final_state=True, chunk=64, stream=None):
+    """The preconditioned delta rule, both phases: write keys from the
+    preconditioner scan, then the chunk forward with them.  Returns
+    (o, final_state or None, d_final)."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    gate = GDN_GATE_NONE if g is None else (GDN_GATE_SCALAR if g.dim() == 3 else GDN_GATE_PER_DIM)
+    kw = torch.empty_like(k)
+    d_final = torch.empty((B, H, Dk), dtype=torch.float32, device=q.device)
+    gdn_osdn_precondition(k, beta, r, eta, d0, kw, d_final, stream=stream)
+    o = torch.empty((B, T, H, Dv), dtype=q.dtype, device=q.device)
+    S = (torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+         if output_final_state else None)
+    ws_n = gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, chunk, q.dtype, gate)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
+    gdn_chunk_fwd_wk(q, k, kw, v, beta, g, gate, initial_state, o, S, chunk=chunk, workspace=ws,
+                     stream=stream)
+    return o, S, d_final
 
 
 def decode_step(q, k, v, beta, g, state, *, stream=None):

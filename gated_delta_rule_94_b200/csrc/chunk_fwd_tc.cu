@@ -278,6 +278,7 @@ __device__ __forceinline__ void chunk_gates(float* gbuf, int lane) {
 
 struct PrepMaps {
     CUtensorMap q, k, v, g;   // g only for the per-dimension gate
+    CUtensorMap kw;           // the write key (preconditioned delta rule) only
 };
 
 // Prep shared memory (bytes from a 1 KB-aligned base); 111 KB for either
@@ -317,10 +318,17 @@ constexpr uint32_t TM_WT = 64;     // W^T, lanes d, 64 columns r
 constexpr uint32_t TM_UT = 128;    // U^T, lanes v, 64 columns r
 constexpr uint32_t TM_FP = 0;      // K~^T W, lanes d, 128 columns d'   (after S, W^T, U^T are read)
 constexpr uint32_t TM_PWT = 128;   // W^T P^T, lanes d, 64 columns r
+constexpr uint32_t TM_QE = 192;    // Q^T E = (Q e^G)^T, lanes d, 64 columns r
+constexpr uint32_t P_E = 32768;    // E_hi, E_lo bf16 [64 r][64 j] over the dead V tile
 
 // One CTA per (batch, head, chunk) of the wave: every state-independent part
 // of the chunk, written to the workspace as the chunk's step image.
-template <int GATE>
+// WK: a separate write key kw (the preconditioned delta rule of "OSDN ...",
+// sec. 2.1): the read key k stays in the A side of the Gram matrix and in W;
+// kw replaces k as the B side of the Gram matrix and of the intra-chunk scores
+// and in K~ (state update, Phi).  The kw tile occupies the V slot until its
+// last reader is done; V is loaded there afterwards, ahead of the U^T product.
+template <int GATE, bool WK>
 __global__ void __launch_bounds__(NPR, 2)
 chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -365,18 +373,39 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     if (tid == 0) {
         for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
-        // K, Q (and g) first: the Gram product needs only them; V lands behind
-        mbar_arrive_expect_tx(&bars[0], (PD ? 6 : 4) * 8192);
-        mbar_arrive_expect_tx(&bars[4], 2 * 8192);
+        // K, Q (and g, and the write key) first: the Gram product needs only
+        // them; V lands behind
+        mbar_arrive_expect_tx(&bars[0], (PD ? 6 : 4) * 8192 + (WK ? 2 * 8192 : 0));
         for (int blk = 0; blk < 2; ++blk) {
             tma_load_3d(sm + P_KQ + blk * 16384, &maps.k, &bars[0], h * D + 64 * blk, n * C, b);
             tma_load_3d(sm + P_KQ + blk * 16384 + 8192, &maps.q, &bars[0], h * D + 64 * blk, n * C, b);
             if constexpr (PD)
                 tma_load_3d(sm + PD_KT + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b);
+            if constexpr (WK)
+                tma_load_3d(sm + P_V + blk * 8192, &maps.kw, &bars[0], h * D + 64 * blk, n * C, b);
         }
-        for (int blk = 0; blk < 2; ++blk)
-            tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b);
+        if constexpr (!WK) {
+            mbar_arrive_expect_tx(&bars[4], 2 * 8192);
+            for (int blk = 0; blk < 2; ++blk)
+                tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b);
+        }
     }
+    // V into the slot the write key held, once every reader of the key is done
+    // (the caller has passed a CTA barrier after the last read)
+    auto load_v_late = [&]() {
+        if constexpr (WK) {
+            if (tid == 0) {
+                fence_async_smem();
+                mbar_arrive_expect_tx(&bars[4], 2 * 8192);
+                for (int blk = 0; blk < 2; ++blk)
+                    tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b);
+            }
+        }
+    };
+    // the write key's tile: blocks of [64 tokens][64 d] with a stride of 8 KB
+    // (WK, in the V slot) or the K tile's 16 KB (K and Q interleaved)
+    const uint32_t kwo = WK ? P_V : P_KQ;
+    const uint32_t kws = WK ? 8192u : 16384u;
     if (warp == 1) {
         tmem_alloc(&s_tmem, 256);
         tmem_relinquish();
@@ -400,13 +429,14 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     bool exact = false;
     if constexpr (!PD) {
         if (warp == 0) chunk_gates<GATE>(gbuf, lane);
-        if (tid == 32) {   // S = [K; Q] K^T
+        if (tid == 32) {   // S = [K; Q] Kw^T (Kw = K without a separate write key)
             if (mbar_wait(&bars[0], 0, &failed)) {
                 const uint32_t id = idesc_bf16_f32(128, 64, false, false);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t a = sb + P_KQ + (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_bf16(tmem + TM_S, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, k > 0);
+                    const uint32_t bb = sb + kwo + (k >> 2) * kws + (k & 3) * 32;
+                    mma_bf16(tmem + TM_S, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), id, k > 0);
                 }
                 mma_commit(&bars[1]);
             } else {
@@ -481,6 +511,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             uint8_t* kp = sm + P_KQ + gblk * 16384 + ro;
             const uint4 kraw = *reinterpret_cast<const uint4*>(kp);
             const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
+            const uint4 wraw = *reinterpret_cast<const uint4*>(sm + kwo + gblk * kws + ro);
+            const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wraw);
             if (!exact) {
                 const uint4 qraw = *reinterpret_cast<const uint4*>(kp + 8192);
                 const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
@@ -492,19 +524,20 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                     const float x0 = Gp[i][2 * e] - cv[2 * e], x1 = Gp[i][2 * e + 1] - cv[2 * e + 1];
                     const float f0 = __expf(x0), f1 = __expf(x1);
                     const float b0 = __expf(-x0), b1 = __expf(-x1);
+                    const float2 wf = __bfloat1622float2(w2[e]);
                     kc[e] = pack_bf16(kf.x * f0, kf.y * f1);
                     qc[e] = pack_bf16(qf.x * f0, qf.y * f1);
-                    ktv[i][2 * e] = kf.x * b0;
-                    ktv[i][2 * e + 1] = kf.y * b1;
+                    ktv[i][2 * e] = wf.x * b0;
+                    ktv[i][2 * e + 1] = wf.y * b1;
                 }
                 *reinterpret_cast<uint4*>(kp) = make_uint4(kc[0], kc[1], kc[2], kc[3]);
                 *reinterpret_cast<uint4*>(kp + 8192) = make_uint4(qc[0], qc[1], qc[2], qc[3]);
             } else {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 kf = __bfloat1622float2(k2[e]);
-                    ktv[i][2 * e] = kf.x * __expf(cv[2 * e] - Gp[i][2 * e]);
-                    ktv[i][2 * e + 1] = kf.y * __expf(cv[2 * e + 1] - Gp[i][2 * e + 1]);
+                    const float2 wf = __bfloat1622float2(w2[e]);
+                    ktv[i][2 * e] = wf.x * __expf(cv[2 * e] - Gp[i][2 * e]);
+                    ktv[i][2 * e + 1] = wf.y * __expf(cv[2 * e + 1] - Gp[i][2 * e + 1]);
                 }
                 float* grow = Gs + r * LDG + 8 * cg;
                 *reinterpret_cast<float4*>(grow) = make_float4(Gp[i][0], Gp[i][1], Gp[i][2], Gp[i][3]);
@@ -548,38 +581,36 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             const float* sU = gbuf + 256;
             const float* sW = gbuf + 320;
             const bool fact = PD || gbuf[384] != 0.f;
-            if (L < 64) {
-                const int r = L;
-                if (fact) {
-                    const float cr = PD ? sBeta[r] : sBeta[r] * sU[r];
+            // row r of A (lanes 0-63, strictly lower) or of P (lanes 64-127,
+            // inclusive); the per-column factors w_i (or G_i) are read four at a
+            // time (the same address across the warp: one broadcast load)
+            const bool isp = L >= 64;
+            const int r = isp ? L - 64 : L;
+            const int lim = isp ? r + 1 : r;      // columns i < lim are kept
+            const float* colf = (fact ? sW : sG) + 32 * ch;
+            if (fact) {
+                const float cr = isp ? (PD ? 1.f : sU[r]) : (PD ? sBeta[r] : sBeta[r] * sU[r]);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = 32 * ch + e;
-                        sv[e] = (i < r) ? (PD ? cr : cr * sW[i]) * sv[e] : 0.f;
-                    }
-                } else {
-                    const float Gr = sG[r], br = sBeta[r];
+                for (int j = 0; j < 8; ++j) {
+                    const float4 w4 = PD ? make_float4(1.f, 1.f, 1.f, 1.f)
+                                         : *reinterpret_cast<const float4*>(colf + 4 * j);
+                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = 32 * ch + e;
-                        sv[e] = (i < r) ? br * __expf(Gr - sG[i]) * sv[e] : 0.f;
+                    for (int t = 0; t < 4; ++t) {
+                        const int e = 4 * j + t;
+                        sv[e] = (32 * ch + e < lim) ? cr * wv[t] * sv[e] : 0.f;
                     }
                 }
             } else {
-                const int r = L - 64;
-                if (fact) {
-                    const float cr = PD ? 1.f : sU[r];
+                const float Gr = sG[r], br = isp ? 1.f : sBeta[r];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = 32 * ch + e;
-                        sv[e] = (i <= r) ? (PD ? cr : cr * sW[i]) * sv[e] : 0.f;
-                    }
-                } else {
-                    const float Gr = sG[r];
+                for (int j = 0; j < 8; ++j) {
+                    const float4 g4 = *reinterpret_cast<const float4*>(colf + 4 * j);
+                    const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = 32 * ch + e;
-                        sv[e] = (i <= r) ? __expf(Gr - sG[i]) * sv[e] : 0.f;
+                    for (int t = 0; t < 4; ++t) {
+                        const int e = 4 * j + t;
+                        sv[e] = (32 * ch + e < lim) ? br * __expf(Gr - gv[t]) * sv[e] : 0.f;
                     }
                 }
             }
@@ -596,7 +627,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll 4
                     for (int d = 0; d < D; ++d) {
                         const float x = ld_bf16(rowt + (d >> 6) * 16384, r, d & 63);
-                        const float kk = ld_bf16(sm + P_KQ + (d >> 6) * 16384, i, d & 63);
+                        const float kk = ld_bf16(sm + kwo + (d >> 6) * kws, i, d & 63);
                         acc = fmaf(x * kk, expf(Gs[r * LDG + d] - Gs[i * LDG + d]), acc);
                     }
                 }
@@ -641,6 +672,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         }
     }
     __syncthreads();
+    if constexpr (PD) load_v_late();   // the write key's last reader was the scan / exact A, P
     forward_substitution(Af, Tf, tid, [&](int t) {
         if constexpr (!PD) {   // K~^T [d][i] = (diag(e^(G_C - G_i)) K)^T into its own tile
             const float* sFt = gbuf + 128;
@@ -648,7 +680,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             for (int idx = t; idx < 512; idx += NPR - 64) {   // (token pair, 8 dims) items
                 const int ip = idx & 31, dc = idx >> 5;
                 const int i0 = 2 * ip, blk = dc >> 3, j = dc & 7;
-                const uint8_t* kb = sm + P_KQ + blk * 16384;
+                const uint8_t* kb = sm + kwo + blk * kws;
                 uint4 r0 = *reinterpret_cast<const uint4*>(kb + i0 * 128 + ((j ^ (i0 & 7)) * 16));
                 uint4 r1 = *reinterpret_cast<const uint4*>(kb + (i0 + 1) * 128 + ((j ^ ((i0 + 1) & 7)) * 16));
                 const float f0 = sFt[i0], f1 = sFt[i0 + 1];
@@ -662,6 +694,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             fence_async_smem();
         }
     });
+    if constexpr (!PD) load_v_late();  // K~^T, the write key's last reader, is formed
     if (!PD && tid == 0 && !failed) {   // K~^T is final: its image goes out now
         bulk_store(img + IMG_KP, sm + P_KT, 16384);
         bulk_commit();
@@ -676,12 +709,22 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             const float4 t0 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j);
             const float4 t1 = *reinterpret_cast<const float4*>(Tf + r * LDF + 8 * j + 4);
             const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            const float4 b0 = *reinterpret_cast<const float4*>(sBeta + 8 * j);
+            const float4 b1 = *reinterpret_cast<const float4*>(sBeta + 8 * j + 4);
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float gv[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+            if constexpr (!PD) {
+                const float4 g0 = *reinterpret_cast<const float4*>(sGam + 8 * j);
+                const float4 g1 = *reinterpret_cast<const float4*>(sGam + 8 * j + 4);
+                gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w;
+                gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
+            }
             float tu[8], tw[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int i = 8 * j + e;
-                tu[e] = (i <= r) ? tv[e] * sBeta[i] : 0.f;
-                tw[e] = PD ? tu[e] : tu[e] * sGam[i];
+                tu[e] = (i <= r) ? tv[e] * bv[e] : 0.f;
+                tw[e] = tu[e] * gv[e];
             }
             st_row_chunk(sm + P_TU, r, j, tu, 1.f);
             if constexpr (!PD) st_row_chunk(sm + P_TW, r, j, tw, 1.f);
@@ -718,6 +761,24 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) st_row_chunk(sm + P_WUT, (warp < 4 ? 0 : 128) + row, j, v + 8 * j, sc);
     }
+    {   // E = diag(e^(G_r)) split as E_hi + E_lo (bf16 each, so that Q^T E_hi + Q^T E_lo
+        // accumulated in fp32 gives (Q e^G)^T to about 2^-16); identity for the
+        // per-dimension gate (its Q tile already carries the decay) and for no gate.
+        // Each thread zeroes four 16-byte chunks of the two tiles, then row r's
+        // diagonal element is set by the thread owning it.
+        const float* sGam = gbuf + 64;
+        for (int idx = tid; idx < 1024; idx += NPR)
+            *reinterpret_cast<uint4*>(sm + P_E + idx * 16) = make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
+        named_bar(4, NPR);
+        if (tid < 64) {
+            const float x = (GATE == kGateScalar) ? sGam[tid] : 1.f;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+            *reinterpret_cast<__nv_bfloat16*>(sm + P_E + sw128_offset(tid, tid)) = hi;
+            *reinterpret_cast<__nv_bfloat16*>(sm + P_E + 8192 + sw128_offset(tid, tid)) = lo;
+        }
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -739,6 +800,11 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_PWT, sdesc_sw128(sb + P_WUT + k * 32, 16, 1024),
                      sdesc_sw128(sb + P_P + k * 32, 16, 1024), id2, k > 0);
+        const uint32_t id3 = idesc_bf16_f32(128, 64, true, false);    // Q^T (E_hi + E_lo)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            mma_bf16(tmem + TM_QE, sdesc_sw128(sb + P_KQ + 8192 + (k & 3) * 2048, 16384, 1024),
+                     sdesc_sw128(sb + P_E + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), id3, k > 0);
         mma_commit(&bars[3]);
     }
     wait(3, 0);
@@ -767,18 +833,17 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         // W^T P^T: warps 0-3 tokens r 0-31, warps 4-7 r 32-63; the 32 lanes of a
         // warp write 32 consecutive d of one row r (one conflict-free wavefront)
         const int hh = warp >> 2;
-        float v[32];
+        float v[32], qv[32];
         ld_cols<32>(tmem + TM_PWT + lane_off + 32 * hh, v);
+        ld_cols<32>(tmem + TM_QE + lane_off + 32 * hh, qv);
         const int d = row;
         const float qs = PD ? sRef[d] : 1.f;
         uint8_t* qblk = sm + S_QPT + (d >> 6) * 8192;
-        const uint8_t* qsrc = sm + P_KQ + (d >> 6) * 16384 + 8192;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int r = 32 * hh + i;
-            const float qb = (PD ? qs : gbuf[64 + r]) * ld_bf16(qsrc, r, d & 63);
             *reinterpret_cast<__nv_bfloat16*>(qblk + sw128_offset(r, d & 63)) =
-                __float2bfloat16_rn(qb - v[i]);
+                __float2bfloat16_rn(fmaf(qs, qv[i], -v[i]));
         }
         if (hh == 1 && !failed) {   // gamma_d
             float gam;
@@ -1146,7 +1211,9 @@ bool make_maps(const ChunkParams& p, bool perdim, PrepMaps* m) {
               make_tmap_bf16(&m->k, p.k, 3, dims, strides, box) &&
               make_tmap_bf16(&m->v, p.v, 3, dims, strides, box);
     m->g = m->q;
+    m->kw = m->k;
     if (ok && perdim) ok = make_tmap_bf16(&m->g, p.g, 3, dims, strides, box);
+    if (ok && p.kw) ok = make_tmap_bf16(&m->kw, p.kw, 3, dims, strides, box);
     return ok;
 }
 
@@ -1228,9 +1295,14 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
         const uint32_t box[3] = {32, 128, 1};
         return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, 3, dims, strides, box);
     };
-    auto prep = gate == kGateScalar ? chunk_prep_kernel<kGateScalar>
-                : gate == kGatePerDim ? chunk_prep_kernel<kGatePerDim>
-                                      : chunk_prep_kernel<kGateNone>;
+    using PrepFn = void (*)(const PrepMaps, const ChunkParams);
+    const bool wk = p0.kw != nullptr;
+    PrepFn prep = gate == kGateScalar ? (wk ? chunk_prep_kernel<kGateScalar, true>
+                                            : chunk_prep_kernel<kGateScalar, false>)
+                  : gate == kGatePerDim ? (wk ? chunk_prep_kernel<kGatePerDim, true>
+                                              : chunk_prep_kernel<kGatePerDim, false>)
+                                        : (wk ? chunk_prep_kernel<kGateNone, true>
+                                              : chunk_prep_kernel<kGateNone, false>);
     const uint32_t prep_smem = P_SMEM;
     cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
     if (e != cudaSuccess) return e;

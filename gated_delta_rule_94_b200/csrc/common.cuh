@@ -19,6 +19,7 @@ struct ChunkParams {
     const void* v;
     const void* beta;
     const void* g;
+    const void* kw;    // write key [B, T, H, Dk] (preconditioned delta rule), or null (= k)
     const float* s0;   // may be null
     void* o;
     float* s_out;      // may be null
@@ -30,6 +31,18 @@ struct ChunkParams {
     int chunk0;        // first chunk of this wave
     int nchunks;       // chunks in this wave
     int ws_chunk;      // bytes of one chunk's workspace image
+};
+
+// Phase 1 of the preconditioned delta rule (write keys kw = d (.) k).
+struct OsdnParams {
+    const void* k;       // [B, T, H, Dk]
+    const void* beta;    // [B, T, H]
+    const void* r;       // [B, T, H] retention gate, or null (r = 1)
+    void* kw;            // [B, T, H, Dk] write keys (output)
+    const float* d0;     // [B, H, Dk] initial preconditioner, or null (ones)
+    float* d_out;        // [B, H, Dk] final preconditioner (output), or null
+    float eta;           // step size of the preconditioner's gradient descent
+    int B, T, H;
 };
 
 struct DecodeParams {
@@ -82,4 +95,5 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, size_t ws_bytes,
                                 int* launches);
 cudaError_t launch_decode_step(const DecodeParams& p, int Dk, int Dv, int gate, bool bf16,
                                cudaStream_t s);
+cudaError_t launch_osdn_precondition(const OsdnParams& p, int Dk, bool bf16, cudaStream_t s);
 }  // namespace gdn

@@ -106,11 +106,16 @@ size_t gdn_chunk_fwd_workspace_min_bytes(int B, int T, int H, int Dk, int Dv, in
     return 0;
 }
 
-gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* beta,
-                         const void* g, gdn_gate gate_kind, const float* initial_state,
-                         void* o, float* final_state, int B, int T, int H, int Dk, int Dv,
-                         int chunk, gdn_dtype dtype, void* workspace, size_t workspace_bytes,
-                         gdn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The chunk forward, with the write key kw (null: kw = k).
+gdn_status chunk_fwd_impl(const void* q, const void* k, const void* kw, const void* v,
+                          const void* beta, const void* g, gdn_gate gate_kind,
+                          const float* initial_state, void* o, float* final_state, int B, int T,
+                          int H, int Dk, int Dv, int chunk, gdn_dtype dtype, void* workspace,
+                          size_t workspace_bytes, gdn_stream_t stream) {
     if (B < 0 || T < 0 || H < 0) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
     if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return GDN_ERR_INVALID_ARG;
@@ -120,7 +125,10 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
     const bool need_tokens = T > 0;
     if (need_tokens && (!q || !k || !v || !beta || !o)) return GDN_ERR_INVALID_ARG;
     if (need_tokens && (gate_kind == GDN_GATE_NONE) != (g == nullptr)) return GDN_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, beta, g, initial_state, o, final_state, workspace};
+    // a separate write key runs on the tensor-core path only
+    if (kw && !(dtype == GDN_BF16 && gdn::chunk_fwd_tc_supported(Dk, Dv, gate_kind)))
+        return GDN_ERR_UNSUPPORTED;
+    const void* ptrs[] = {q, k, kw, v, beta, g, initial_state, o, final_state, workspace};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
     const size_t es = elem_size(dtype);
@@ -131,6 +139,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
                               : gate_kind == GDN_GATE_SCALAR ? ntok * es : 0;
         if (overlaps(final_state, state_bytes, q, ntok * Dk * es) ||
             overlaps(final_state, state_bytes, k, ntok * Dk * es) ||
+            overlaps(final_state, state_bytes, kw, ntok * Dk * es) ||
             overlaps(final_state, state_bytes, v, ntok * Dv * es) ||
             overlaps(final_state, state_bytes, beta, ntok * es) ||
             overlaps(final_state, state_bytes, g, gbytes) ||
@@ -142,6 +151,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
     }
     if (need_tokens && initial_state && overlaps(o, ntok * Dv * es, initial_state, state_bytes))
         return GDN_ERR_INVALID_ARG;
+    if (need_tokens && kw && overlaps(o, ntok * Dv * es, kw, ntok * Dk * es)) return GDN_ERR_INVALID_ARG;
     const size_t ws_need = gdn_chunk_fwd_workspace_min_bytes(B, T, H, Dk, Dv, chunk, dtype, gate_kind);
     if (ws_need > 0 && (workspace_bytes < ws_need || !workspace)) return GDN_ERR_WORKSPACE;
 
@@ -159,7 +169,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
     }
 
     gdn::ChunkParams p;
-    p.q = q; p.k = k; p.v = v; p.beta = beta; p.g = g;
+    p.q = q; p.k = k; p.v = v; p.beta = beta; p.g = g; p.kw = kw;
     p.s0 = initial_state; p.o = o; p.s_out = final_state;
     p.B = B; p.T = T; p.H = H; p.Dk = Dk; p.Dv = Dv;
     p.status = status_word_ptr();
@@ -177,6 +187,66 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void
         e = gdn::launch_chunk_fwd_simt(p, gate_kind, dtype == GDN_BF16, s);
     g_launches.fetch_add((unsigned long long)launches);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const void* beta,
+                         const void* g, gdn_gate gate_kind, const float* initial_state,
+                         void* o, float* final_state, int B, int T, int H, int Dk, int Dv,
+                         int chunk, gdn_dtype dtype, void* workspace, size_t workspace_bytes,
+                         gdn_stream_t stream) {
+    return chunk_fwd_impl(q, k, nullptr, v, beta, g, gate_kind, initial_state, o, final_state,
+                          B, T, H, Dk, Dv, chunk, dtype, workspace, workspace_bytes, stream);
+}
+
+gdn_status gdn_chunk_fwd_wk(const void* q, const void* k, const void* k_write, const void* v,
+                            const void* beta, const void* g, gdn_gate gate_kind,
+                            const float* initial_state, void* o, float* final_state, int B,
+                            int T, int H, int Dk, int Dv, int chunk, gdn_dtype dtype,
+                            void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    return chunk_fwd_impl(q, k, k_write, v, beta, g, gate_kind, initial_state, o, final_state,
+                          B, T, H, Dk, Dv, chunk, dtype, workspace, workspace_bytes, stream);
+}
+
+gdn_status gdn_osdn_precondition(const void* k, const void* beta, const void* r, float eta,
+                                 const float* d0, void* k_write, float* d_final, int B, int T,
+                                 int H, int Dk, gdn_dtype dtype, gdn_stream_t stream) {
+    if (B < 0 || T < 0 || H < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (!(eta == eta) || eta > 3.0e38f || eta < -3.0e38f) return GDN_ERR_INVALID_ARG;
+    if (!supported_dim(Dk)) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)B * T > INT32_MAX || (int64_t)B * H > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return GDN_OK;
+    if (T > 0 && (!k || !beta || !k_write)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {k, beta, r, d0, k_write, d_final};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t es = elem_size(dtype);
+    const size_t ntok = (size_t)B * T * H;
+    const size_t dbytes = (size_t)B * H * Dk * sizeof(float);
+    if (overlaps(k_write, ntok * Dk * es, k, ntok * Dk * es) ||
+        overlaps(k_write, ntok * Dk * es, beta, ntok * es) ||
+        overlaps(k_write, ntok * Dk * es, r, ntok * es) ||
+        overlaps(k_write, ntok * Dk * es, d0, dbytes) ||
+        overlaps(k_write, ntok * Dk * es, d_final, dbytes) ||
+        overlaps(d_final, dbytes, k, ntok * Dk * es) ||
+        overlaps(d_final, dbytes, beta, ntok * es) ||
+        overlaps(d_final, dbytes, r, ntok * es))
+        return GDN_ERR_INVALID_ARG;
+    if (d0 && d_final && d0 != d_final && overlaps(d0, dbytes, d_final, dbytes))
+        return GDN_ERR_INVALID_ARG;
+    if (T == 0 && !d_final) return GDN_OK;
+    gdn::OsdnParams p;
+    p.k = k; p.beta = beta; p.r = r; p.kw = k_write; p.d0 = d0; p.d_out = d_final;
+    p.eta = eta; p.B = B; p.T = T; p.H = H;
+    cudaError_t e = gdn::launch_osdn_precondition(p, Dk, dtype == GDN_BF16,
+                                                  reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    g_launches.fetch_add(1);
     return GDN_OK;
 }
 

@@ -146,6 +146,57 @@ GDN_API gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
                            float* state, void* o, int N, int H, int Dk, int Dv,
                            gdn_dtype dtype, gdn_stream_t stream);
 
+/*
+ * gdn_osdn_precondition -- phase 1 of the preconditioned delta rule: the
+ * write keys kw_t = d_t (.) k_t of a diagonal preconditioner learned online
+ * ("OSDN: Improving Delta Rule with Provable Online Preconditioning in Linear
+ * Attention", sec. 2.1 the preconditioned key, sec. 2.2 the closed-form
+ * surrogate and its online gradient step, sec. 2.3 the retention gate).  Per
+ * (batch, head), token by token, with s = <d, k_t^2> and n = |k_t|^2:
+ *     kw_t = d (.) k_t
+ *     d   <- r_t d + eta beta_t (1 - beta_t s) k_t^2 / n     (unchanged if n = 0)
+ * i.e. one step of gradient descent on h_t(d) = ((1 - beta_t <d, k_t^2>)^2 - 1)
+ * / (2 |k_t|^2) after scaling d by r_t.  Phase 2 is gdn_chunk_fwd_wk with
+ * these write keys.
+ *
+ *   k        [B, T, H, Dk]  element type `dtype`
+ *   beta     [B, T, H]      element type `dtype`
+ *   r        [B, T, H]      retention gate, element type `dtype`; NULL: r = 1
+ *   eta      step size of the preconditioner (finite)
+ *   d0       [B, H, Dk] fp32 initial preconditioner; NULL: all ones
+ *   k_write  [B, T, H, Dk]  element type `dtype` (output; must not overlap
+ *            any input)
+ *   d_final  [B, H, Dk] fp32 final preconditioner (output) or NULL; may be
+ *            the same pointer as d0
+ *   Dk       64 or 128;  dtype GDN_BF16 or GDN_F32 (fp32 arithmetic either way)
+ * The scan is sequential in t (a 4-lane group per (batch, head)).
+ */
+GDN_API gdn_status gdn_osdn_precondition(const void* k, const void* beta, const void* r,
+                                         float eta, const float* d0, void* k_write,
+                                         float* d_final, int B, int T, int H, int Dk,
+                                         gdn_dtype dtype, gdn_stream_t stream);
+
+/*
+ * gdn_chunk_fwd_wk -- gdn_chunk_fwd with a separate write key (phase 2 of the
+ * preconditioned delta rule, "OSDN ...", sec. 2.1): per token
+ *     M_t = (I - beta_t kw_t k_t^T) Diag(a_t) M_{t-1} + beta_t kw_t v_t^T,
+ *     o_t = M_t^T q_t,
+ * the residual read with k_t and written along kw_t.  Chunkwise, kw replaces
+ * k in the Gram matrix and the intra-chunk scores (and in the state update);
+ * k stays in the WY factor W.  Arguments as gdn_chunk_fwd plus
+ *   k_write  [B, T, H, Dk] element type `dtype`, or NULL (then exactly
+ *            gdn_chunk_fwd); with a write key the call runs on the
+ *            tensor-core path only (GDN_BF16, Dk = Dv = 128), anything else is
+ *            GDN_ERR_UNSUPPORTED.
+ * Workspace as gdn_chunk_fwd (gdn_chunk_fwd_workspace_bytes / _min_bytes).
+ */
+GDN_API gdn_status gdn_chunk_fwd_wk(const void* q, const void* k, const void* k_write,
+                                    const void* v, const void* beta, const void* g,
+                                    gdn_gate gate_kind, const float* initial_state, void* o,
+                                    float* final_state, int B, int T, int H, int Dk, int Dv,
+                                    int chunk, gdn_dtype dtype, void* workspace,
+                                    size_t workspace_bytes, gdn_stream_t stream);
+
 /* Synchronizes `stream`, then reads and clears the library's device status
  * word.  Returns GDN_ERR_TIMEOUT if any kernel since the last call gave up a
  * bounded wait, GDN_ERR_CUDA if the stream reports an error, else GDN_OK.

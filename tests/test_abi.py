@@ -166,3 +166,70 @@ def test_python_binding_rejects_bad_tensors():
         gdn.gdn_chunk_fwd(q, q, q, torch.zeros(1, 64, 1), None, 0, None, q, None)
     with pytest.raises(ValueError):
         gdn.gdn_chunk_fwd(q.transpose(1, 3), q, q, None, None, 0, None, q, None)
+
+
+# ------------------------------------------------ preconditioned delta rule
+def wk_call(**over):
+    args = dict(q=A, k=A, kw=A * 4, v=A, beta=A, g=A, gate=1, s0=None, o=A * 2, s1=None, B=1,
+                T=64, H=1, Dk=128, Dv=128, chunk=64, dtype=0, ws=None, ws_bytes=0, stream=None)
+    args.update(over)
+    return _lib.load().gdn_chunk_fwd_wk(args["q"], args["k"], args["kw"], args["v"],
+                                        args["beta"], args["g"], args["gate"], args["s0"],
+                                        args["o"], args["s1"], args["B"], args["T"], args["H"],
+                                        args["Dk"], args["Dv"], args["chunk"], args["dtype"],
+                                        args["ws"], args["ws_bytes"], args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(dtype=1), _lib.GDN_ERR_UNSUPPORTED),                # a write key needs bf16 ...
+    (dict(Dk=64, Dv=64), _lib.GDN_ERR_UNSUPPORTED),           # ... and d = 128
+    (dict(kw=MIS), _lib.GDN_ERR_INVALID_ARG),
+    (dict(q=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(s1=A * 4), _lib.GDN_ERR_INVALID_ARG),               # final state overlaps the write key
+    (dict(kw=A * 2), _lib.GDN_ERR_INVALID_ARG),               # the write key overlaps o
+    (dict(), _lib.GDN_ERR_WORKSPACE),                         # valid, but no workspace
+])
+def test_chunk_fwd_wk_argument_errors(over, code):
+    assert wk_call(**over) == code
+
+
+def test_chunk_fwd_wk_without_write_key_is_chunk_fwd():
+    """k_write = NULL takes exactly gdn_chunk_fwd's path: the fp32 and d = 64
+    shapes it supports are accepted up to the (missing) device."""
+    assert wk_call(kw=None, B=0) == _lib.GDN_OK
+    assert wk_call(kw=None, dtype=1, Dk=64, Dv=64, B=0) == _lib.GDN_OK
+
+
+def osdn_call(**over):
+    args = dict(k=A, beta=A * 2, r=None, eta=0.5, d0=None, kw=A * 4, d1=None, B=1, T=64, H=1,
+                Dk=128, dtype=0, stream=None)
+    args.update(over)
+    return _lib.load().gdn_osdn_precondition(args["k"], args["beta"], args["r"], args["eta"],
+                                             args["d0"], args["kw"], args["d1"], args["B"],
+                                             args["T"], args["H"], args["Dk"], args["dtype"],
+                                             args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(k=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(kw=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(beta=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(eta=float("nan")), _lib.GDN_ERR_INVALID_ARG),
+    (dict(eta=float("inf")), _lib.GDN_ERR_INVALID_ARG),
+    (dict(Dk=96), _lib.GDN_ERR_UNSUPPORTED),
+    (dict(dtype=5), _lib.GDN_ERR_INVALID_ARG),
+    (dict(B=-1), _lib.GDN_ERR_INVALID_ARG),
+    (dict(kw=MIS), _lib.GDN_ERR_INVALID_ARG),
+    (dict(kw=A), _lib.GDN_ERR_INVALID_ARG),                   # write keys over the keys
+    (dict(d1=A * 4), _lib.GDN_ERR_INVALID_ARG),               # final d over the write keys
+    (dict(d0=A * 1024, d1=A * 1024 + 16), _lib.GDN_ERR_INVALID_ARG),   # partial d overlap
+    (dict(B=65536, T=65536), _lib.GDN_ERR_UNSUPPORTED),
+])
+def test_osdn_precondition_argument_errors(over, code):
+    assert osdn_call(**over) == code
+
+
+def test_osdn_precondition_noop_sizes():
+    assert osdn_call(B=0) == _lib.GDN_OK
+    assert osdn_call(H=0, k=None, kw=None) == _lib.GDN_OK
+    assert osdn_call(T=0, k=None, kw=None, beta=None) == _lib.GDN_OK   # nothing to write
