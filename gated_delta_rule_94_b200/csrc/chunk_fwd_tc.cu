@@ -301,14 +301,14 @@ constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;
 constexpr uint32_t PD_KT = P_KT;             // per-dimension gate: g bf16 (TMA), then K~
 // staging of the step image for its bulk stores (buffers dead by then)
 constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
-constexpr uint32_t S_QPT = P_KT;             // Qp [64 r][128 d] as two [64][64] blocks, over K~^T:
-                                             // dead once the K~^T W product is done and its
-                                             // image store has read it
+constexpr uint32_t S_QPT = P_WUT + 16384;    // Qp [64 r][128 d] as two [64][64] blocks, over the
+                                             // U^T rows of [W^T; U^T]: dead once U^T's image
+                                             // store has read them
 constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (exact fallback; aliases A / T)
 static_assert(P_TF + 64 * LDF * 4 <= P_KT, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_KT, "[W^T; U^T] tile");
 static_assert(P_TW + 8192 <= P_TF && P_KT + 16384 <= P_P, "T_u / T_w over A, K~ tile");
-static_assert(S_PHI + 32768 <= P_WUT + 16384 && S_QPT + 16384 <= P_P, "staging clear of the U^T rows and P");
+static_assert(S_PHI + 32768 <= S_QPT && S_QPT + 16384 <= P_KT, "staging clear of each other and K~^T");
 static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
 static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
 
@@ -352,17 +352,16 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, T = p.T;
-    const int bh = blockIdx.x / p.nchunks, nl = blockIdx.x % p.nchunks;
-    const int b = bh / H, h = bh % H;
-    const int n = p.chunk0 + nl;
-    uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * IMG_BYTES;
+    const int nitems = p.B * p.H * p.nchunks;
     const uint32_t sb = smem_u32(sm);
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int failed = 0;
+    uint32_t ph = 0;   // phase of every barrier: each completes once per item
     auto wait = [&](int i, uint32_t parity) {
         if (!mbar_wait(&bars[i], parity, &failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     };
+    __shared__ int s_item[2];
 
     float* sBeta = gbuf + 192;
     // per-dimension gate
@@ -370,17 +369,32 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     float* sGamD = gbuf + 256;                         // gamma_d = e^(c_d)
     float* sRef = gbuf + 384;                          // e^(c_d); 1 in the exact fallback
 
-    if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
-        fence_mbar_init();
-        // K, Q (and g, and the write key) first: the Gram product needs only
-        // them; V lands behind
+    // item -> (sequence, head, chunk of this wave)
+    auto coords = [&](int item, int& b, int& h, int& n) {
+        const int bh = item / p.nchunks;
+        b = bh / H;
+        h = bh % H;
+        n = p.chunk0 + item % p.nchunks;
+    };
+    // K and Q of an item, with the expect_tx of every byte its bars[0] phase
+    // counts (the g tile and the write key follow in issue_rest)
+    auto issue_kq = [&](int item) {
+        int b, h, n;
+        coords(item, b, h, n);
         mbar_arrive_expect_tx(&bars[0], (PD ? 6 : 4) * 8192 + (WK ? 2 * 8192 : 0));
         for (int blk = 0; blk < 2; ++blk) {
             tma_load_3d(sm + P_KQ + blk * 16384, &maps.k, &bars[0], h * D + 64 * blk, n * C, b);
             tma_load_3d(sm + P_KQ + blk * 16384 + 8192, &maps.q, &bars[0], h * D + 64 * blk, n * C, b);
             if constexpr (PD)
                 tma_load_3d(sm + PD_KT + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b);
+        }
+    };
+    // the rest of an item's tiles, into slots that are free only once the
+    // previous item has finished: the write key, V
+    auto issue_rest = [&](int item) {
+        int b, h, n;
+        coords(item, b, h, n);
+        for (int blk = 0; blk < 2; ++blk) {
             if constexpr (WK)
                 tma_load_3d(sm + P_V + blk * 8192, &maps.kw, &bars[0], h * D + 64 * blk, n * C, b);
         }
@@ -389,7 +403,51 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             for (int blk = 0; blk < 2; ++blk)
                 tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b);
         }
+    };
+    // beta and g of an item, by warps 2-3 into registers
+    float nb = 0.f, ng = 0.f;
+    auto fetch_bg = [&](int item) {
+        int b, h, n;
+        coords(item, b, h, n);
+        const int t = n * C + (tid - 64);
+        nb = ng = 0.f;
+        if (t < T) {
+            const size_t tok = ((size_t)b * T + t) * H + h;
+            nb = __bfloat162float(static_cast<const __nv_bfloat16*>(p.beta)[tok]);
+            if constexpr (GATE == kGateScalar) ng = __bfloat162float(static_cast<const __nv_bfloat16*>(p.g)[tok]);
+        }
+    };
+
+    if (tid == 0) {
+        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        const int first = (int)atomicAdd(p.counter, 1u);
+        s_item[0] = first;
+        if (first < nitems) issue_kq(first);
     }
+    if (warp == 1) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    int item = s_item[0];
+    if ((warp == 2 || warp == 3) && item < nitems) fetch_bg(item);
+    // the write key's tile: blocks of [64 tokens][64 d] with a stride of 8 KB
+    // (WK, in the V slot) or the K tile's 16 KB (K and Q interleaved)
+    const uint32_t kwo = WK ? P_V : P_KQ;
+    const uint32_t kws = WK ? 8192u : 16384u;
+
+#pragma unroll 1
+    for (int it = 0; item < nitems; ++it) {
+    ph = it & 1;
+    int b, h, n;
+    coords(item, b, h, n);
+    const int bh = item / p.nchunks, nl = item % p.nchunks;
+    uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * IMG_BYTES;
+    if (tid == 0) issue_rest(item);
     // V into the slot the write key held, once every reader of the key is done
     // (the caller has passed a CTA barrier after the last read)
     auto load_v_late = [&]() {
@@ -402,35 +460,17 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             }
         }
     };
-    // the write key's tile: blocks of [64 tokens][64 d] with a stride of 8 KB
-    // (WK, in the V slot) or the K tile's 16 KB (K and Q interleaved)
-    const uint32_t kwo = WK ? P_V : P_KQ;
-    const uint32_t kws = WK ? 8192u : 16384u;
-    if (warp == 1) {
-        tmem_alloc(&s_tmem, 256);
-        tmem_relinquish();
+    if (warp == 2 || warp == 3) {   // beta and g (fetched during the previous item)
+        gbuf[tid - 64] = ng;
+        sBeta[tid - 64] = nb;
     }
-    if (warp == 2 || warp == 3) {   // beta and g, off the warps that set up barriers and TMEM
-        const int i = tid - 64, t = n * C + i;
-        float gv = 0.f, bv = 0.f;
-        if (t < T) {
-            const size_t tok = ((size_t)b * T + t) * H + h;
-            bv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.beta)[tok]);
-            if constexpr (GATE == kGateScalar) gv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.g)[tok]);
-        }
-        gbuf[i] = gv;
-        sBeta[i] = bv;
-    }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
 
     bool exact = false;
     if constexpr (!PD) {
         if (warp == 0) chunk_gates<GATE>(gbuf, lane);
         if (tid == 32) {   // S = [K; Q] Kw^T (Kw = K without a separate write key)
-            if (mbar_wait(&bars[0], 0, &failed)) {
+            if (mbar_wait(&bars[0], ph, &failed)) {
                 const uint32_t id = idesc_bf16_f32(128, 64, false, false);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
@@ -445,7 +485,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         }
         __syncthreads();
     } else {
-        wait(0, 0);
+        wait(0, ph);
         // G = in-chunk cumsum of g per key dimension by a segmented scan in
         // registers: lane pair (segment of 4 rows) x column group of 8
         // dimensions, then across the 16 segments; c = G_C per dimension.  The
@@ -565,6 +605,9 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                 mma_bf16(tmem + TM_S, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 8192, 1024), id, k > 0);
             }
             mma_commit(&bars[1]);
+        } else if (exact && tid == 32) {
+            mbar_arrive(&bars[1]);   // no product: complete the phase, so that every
+                                     // barrier completes once per item
         }
     }
 
@@ -574,7 +617,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         const int L = q4 * 32 + lane;
         float sv[32];
         if (!exact) {
-            wait(1, 0);
+            wait(1, ph);
             tc_fence_after();
             ld_cols<32>(tmem + TM_S + lane_off + 32 * ch, sv);
             const float* sG = gbuf;
@@ -744,14 +787,14 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_WT, sdesc_sw128(sb + P_KQ + k * 2048, 16384, 1024),
                      sdesc_sw128(tw + k * 32, 16, 1024), id, k > 0);
-        if (!mbar_wait(&bars[4], 0, &failed)) atomicOr(p.status, kStatusTimeout);
+        if (!mbar_wait(&bars[4], ph, &failed)) atomicOr(p.status, kStatusTimeout);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_UT, sdesc_sw128(sb + P_V + k * 2048, 8192, 1024),
                      sdesc_sw128(sb + P_TU + k * 32, 16, 1024), id, k > 0);
         mma_commit(&bars[2]);
     }
-    wait(2, 0);
+    wait(2, ph);
     tc_fence_after();
     {   // [W^T; U^T] as one K-major bf16 tile of 256 rows (tokens contiguous)
         const int row = (warp & 3) * 32 + lane;
@@ -807,12 +850,24 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                      sdesc_sw128(sb + P_E + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), id3, k > 0);
         mma_commit(&bars[3]);
     }
-    wait(3, 0);
-    // the K~ tile becomes the Qp^T staging: its image store (the older of the two
-    // outstanding groups) must have read it
-    if (tid == 0) bulk_wait_read_all_but_one();
+    wait(3, ph);
+    // The U^T rows become the Qp staging: U^T's image store must have read them
+    // (and K~^T's, whose slot takes the next g tile).  The last readers of K, Q
+    // and K~^T (the W^T, Q^T E and K~^T W products) are done: the next item's
+    // K, Q (and g) can land now.
+    if (tid == 0) {
+        bulk_wait_read();
+        const int nx = (int)atomicAdd(p.counter, 1u);
+        s_item[(it + 1) & 1] = nx;
+        if (nx < nitems) {
+            fence_async_smem();
+            issue_kq(nx);
+        }
+    }
     tc_fence_after();
     __syncthreads();
+    const int next_item = s_item[(it + 1) & 1];
+    if ((warp == 2 || warp == 3) && next_item < nitems) fetch_bg(next_item);
     const int row = (warp & 3) * 32 + lane;
     {   // Phi = -K~^T W, row d: warps 0-3 columns 0-63, warps 4-7 columns 64-127;
         // each half stored as soon as it is staged
@@ -864,6 +919,22 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     }
     if (tid == 128) bulk_wait_read();   // its half of Phi
     tc_fence_before();
+    if (__syncthreads_or(failed)) {
+        // a bounded wait gave up: wait (bounded) for this item's loads and the
+        // next item's K and Q, if they were issued, then take no more items
+        if (tid == 0) {
+            int f2 = 0;
+            const bool cur = mbar_wait(&bars[0], ph, &f2);
+            mbar_wait(&bars[4], ph, &f2);
+            if (cur && next_item < nitems) mbar_wait(&bars[0], ph ^ 1u, &f2);
+        }
+        __syncthreads();
+        break;
+    }
+    tc_fence_after();
+    item = next_item;
+    }   // items
+    tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -875,14 +946,15 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 // The chain runs on the transposed state: h^T [v][d] (fp32 in the state-pass
 // registers, its bf16 copy in TMEM as the A operand of the state product), so
 // that neither the state's bf16 copy nor the product's h operand touch shared
-// memory.  Two products per chunk n, both M = 128 (v), N = 192:
-//   D_n  = U_n^T [K~_n | P_n^T]        (K = 64 tokens; A = U^T from shared memory)
-//   D_n += h_n^T [Phi_n^T | Qp_n^T]    (K = 128; A = h^T from TMEM)
+// memory.  Per chunk n, into one accumulator D_n of 192 columns (M = 128 v):
+//   D_n  = U_n^T [K~_n | P_n^T]        (N = 192, K = 64 tokens; A = U^T from shared memory)
+//   D_n[:, 0..127]   += h_n^T Phi_n^T  (N = 128, K = 128; A = h^T from TMEM)
+//   D_n[:, 128..191] += h_n^T Qp_n^T   (N = 64,  K = 128)
 // Columns 0..127 of D_n are X^T_n = U^T K~ + h^T Phi^T, so the state pass forms
 //   h_{n+1}^T = h_n^T Diag(gamma_n) + X^T_n
 // and columns 128..191 are O^T_n = U^T P^T + h^T Qp^T, the chunk's output.
-// The first product needs no state and runs while the state pass of the
-// previous chunk works; only the second is on the serial path.
+// Only h^T Phi^T is on the serial path: U^T [K~ | P^T] needs no state, and
+// h^T Qp^T is issued behind h^T Phi^T, so both run while the state pass works.
 
 // Chain kernel shared memory (bytes from a 1 KB-aligned base).
 constexpr uint32_t CH_PQ = 0;           // 2 slots of [Phi ; Qp] (48 KB each); the final state's staging
@@ -913,8 +985,8 @@ constexpr uint32_t TM_SLOT = 256;
 
 enum ChainBar {
     CB_KU0, CB_KU1, CB_PQ0, CB_PQ1, CB_GAM0, CB_GAM1, CB_GAM2, CB_GAM3, CB_KUFREE0, CB_KUFREE1,
-    CB_PQFREE0, CB_PQFREE1, CB_SDONE0, CB_SDONE1, CB_HREADY0, CB_HREADY1, CB_XFREE0, CB_XFREE1,
-    CB_OFREE0, CB_OFREE1, CB_FINAL, CB_COUNT
+    CB_PQFREE0, CB_PQFREE1, CB_SDONE0, CB_SDONE1, CB_ODONE0, CB_ODONE1, CB_HREADY0, CB_HREADY1,
+    CB_XFREE0, CB_XFREE1, CB_OFREE0, CB_OFREE1, CB_FINAL, CB_COUNT
 };
 static_assert(CB_COUNT * 8 <= 512, "barrier space");
 
@@ -1037,6 +1109,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         // adds its byte offset / 16 to the start-address field)
         const bool leader = lane == 0;
         const uint32_t id = idesc_bf16_f32(128, 192, false, false);
+        const uint32_t id_phi = idesc_bf16_f32(128, 128, false, false);
+        const uint32_t id_qp = idesc_bf16_f32(128, 64, false, false);
         const uint64_t d_kp = sdesc_sw128(sb + CH_KP, 16, 1024);
         const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
         const uint64_t d_pq = sdesc_sw128(sb + CH_PQ, 16, 1024);
@@ -1067,11 +1141,17 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             tc_fence_after();
             if (leader && !failed) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
+                for (int k = 0; k < 8; ++k)   // X^T += h^T Phi^T: rows 0..127 of [Phi ; Qp]
                     mma_bf16_ta(tmem + TM_D + TM_SLOT * s, tmem + TM_HT + TM_SLOT * s + 8 * k,
                                 d_pq + ((s * 2 * PQ_BLK + (k >> 2) * PQ_BLK + (k & 3) * 32) >> 4),
-                                id, true);
+                                id_phi, true);
                 mma_commit(&bars[CB_SDONE0 + s]);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // O^T += h^T Qp^T: rows 128..191
+                    mma_bf16_ta(tmem + TM_D + TM_SLOT * s + 128, tmem + TM_HT + TM_SLOT * s + 8 * k,
+                                d_pq + ((s * 2 * PQ_BLK + (k >> 2) * PQ_BLK + 16384 + (k & 3) * 32) >> 4),
+                                id_qp, true);
+                mma_commit(&bars[CB_ODONE0 + s]);
                 mma_commit(&bars[CB_PQFREE0 + s]);
             }
             if (nl + 1 < NC) issue_ku(nl + 1);
@@ -1090,7 +1170,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             const int s = nl & 1;
             if (leader && nl >= 2) bulk_wait_read_all_but_one();   // the store of chunk nl - 2 read slot s
             named_bar(2, 128);
-            wait(CB_SDONE0 + s, (nl >> 1) & 1);
+            wait(CB_ODONE0 + s, (nl >> 1) & 1);
             tc_fence_after();
             uint8_t* ot = sm + CH_OT + s * 16384 + (v >> 6) * 8192;
 #pragma unroll
@@ -1179,6 +1259,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                         // last state product is done), written by four TMA stores
             advance(NC);
             if (p.s_out) {
+                // the last chunk's h^T Qp^T (behind h^T Phi^T) may still read its slot
+                wait(CB_ODONE0 + ((NC - 1) & 1), ((NC - 1) >> 1) & 1);
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
                     *reinterpret_cast<float*>(sm + CH_PQ + st_off(32 * c + e, v)) = hv[e];
@@ -1217,6 +1299,10 @@ bool make_maps(const ChunkParams& p, bool perdim, PrepMaps* m) {
     return ok;
 }
 
+// Item counters of the persistent prep, one per wave (at most one wave per
+// chunk), at the end of the workspace.
+size_t counter_bytes(int NC) { return ((size_t)NC * sizeof(unsigned) + 255) & ~(size_t)255; }
+
 // Chunks per (batch, head) of one wave, for a workspace of `budget` bytes.
 // Short sequences (up to 4 chunks) run as one wave.  Otherwise two image
 // buffers alternate (plus the state carried between waves): the longest wave
@@ -1226,6 +1312,8 @@ bool make_maps(const ChunkParams& p, bool perdim, PrepMaps* m) {
 // 90 % (a nearly empty last round costs a whole CTA lifetime).  0 if even one
 // chunk per wave does not fit.
 int wave_chunks(int nbh, int NC, size_t budget) {
+    if (budget < counter_bytes(NC)) return 0;
+    budget -= counter_bytes(NC);
     const size_t per = (size_t)nbh * IMG_BYTES;                  // one chunk of every head
     const size_t carry = (size_t)nbh * D * D * sizeof(float);
     const bool fits_one = (size_t)NC * per <= budget;
@@ -1247,7 +1335,7 @@ size_t workspace_for(int nbh, int NC, int cw) {
     const int nw = (NC + cw - 1) / cw;
     size_t bytes = (size_t)nbh * cw * IMG_BYTES * (nw > 1 ? 2 : 1);   // two alternating buffers
     if (nw > 1) bytes += (size_t)nbh * D * D * sizeof(float);           // state between waves
-    return bytes;
+    return bytes + counter_bytes(NC);
 }
 
 }  // namespace
@@ -1270,7 +1358,7 @@ size_t chunk_fwd_tc_workspace_min_bytes(int B, int T, int H, int gate) {
     if (NC == 0 || B == 0 || H == 0) return 0;
     const size_t per = (size_t)B * H * IMG_BYTES;
     const size_t two = 2 * per + (size_t)B * H * D * D * sizeof(float);
-    return std::min((size_t)NC * per, two);
+    return std::min((size_t)NC * per, two) + counter_bytes(NC);
 }
 
 cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes, cudaStream_t s,
@@ -1316,6 +1404,22 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
     const int nw = (NC + cw - 1) / cw;
     const size_t buf_bytes = (size_t)nbh * cw * IMG_BYTES;
     float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + 2 * buf_bytes) : nullptr;
+    unsigned* counters = reinterpret_cast<unsigned*>(
+        p0.ws + workspace_for(nbh, NC, cw) - counter_bytes(NC));
+    // persistent prep: two CTAs per SM take the wave's items from its counter
+    static int sm_count[64] = {0};
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!sm_count[dev]) {
+        int c = 0;
+        e = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        sm_count[dev] = c;
+    }
+    e = cudaMemsetAsync(counters, 0, (size_t)nw * sizeof(unsigned), s);
+    if (e != cudaSuccess) return e;
     CUtensorMap m_sout, m_carry;
     memset(&m_sout, 0, sizeof(m_sout));
     memset(&m_carry, 0, sizeof(m_carry));
@@ -1335,8 +1439,10 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
         p.nchunks = (w + 1 < nw) ? cw : NC - w * cw;
         p.s0 = (w == 0) ? p0.s0 : carry;
         p.s_out = (w + 1 == nw) ? p0.s_out : carry;
+        p.counter = counters + w;
+        const int items = nbh * p.nchunks;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(nbh * p.nchunks + 1));
+        cfg.gridDim = dim3((unsigned)(std::min(items, 2 * sm_count[dev]) + 1));
         cfg.blockDim = dim3(NPR);
         cfg.dynamicSmemBytes = prep_smem;
         cfg.stream = s;

@@ -31,6 +31,7 @@ struct ChunkParams {
     int chunk0;        // first chunk of this wave
     int nchunks;       // chunks in this wave
     int ws_chunk;      // bytes of one chunk's workspace image
+    unsigned* counter; // this wave's item counter (persistent prep CTAs take items from it)
 };
 
 // Phase 1 of the preconditioned delta rule (write keys kw = d (.) k).
