@@ -353,6 +353,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, T = p.T;
     const int nitems = p.B * p.H * p.nchunks;
+    const uint64_t pol_in = l2_evict_first();    // inputs: read once
+    const uint64_t pol_img = l2_evict_last();    // step images: read back by the chain soon
     const uint32_t sb = smem_u32(sm);
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int failed = 0;
@@ -383,10 +385,10 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         coords(item, b, h, n);
         mbar_arrive_expect_tx(&bars[0], (PD ? 6 : 4) * 8192 + (WK ? 2 * 8192 : 0));
         for (int blk = 0; blk < 2; ++blk) {
-            tma_load_3d(sm + P_KQ + blk * 16384, &maps.k, &bars[0], h * D + 64 * blk, n * C, b);
-            tma_load_3d(sm + P_KQ + blk * 16384 + 8192, &maps.q, &bars[0], h * D + 64 * blk, n * C, b);
+            tma_load_3d_hint(sm + P_KQ + blk * 16384, &maps.k, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
+            tma_load_3d_hint(sm + P_KQ + blk * 16384 + 8192, &maps.q, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
             if constexpr (PD)
-                tma_load_3d(sm + PD_KT + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b);
+                tma_load_3d_hint(sm + PD_KT + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
         }
     };
     // the rest of an item's tiles, into slots that are free only once the
@@ -396,12 +398,12 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         coords(item, b, h, n);
         for (int blk = 0; blk < 2; ++blk) {
             if constexpr (WK)
-                tma_load_3d(sm + P_V + blk * 8192, &maps.kw, &bars[0], h * D + 64 * blk, n * C, b);
+                tma_load_3d_hint(sm + P_V + blk * 8192, &maps.kw, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
         }
         if constexpr (!WK) {
             mbar_arrive_expect_tx(&bars[4], 2 * 8192);
             for (int blk = 0; blk < 2; ++blk)
-                tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b);
+                tma_load_3d_hint(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b, pol_in);
         }
     };
     // beta and g of an item, by warps 2-3 into registers
@@ -456,7 +458,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                 fence_async_smem();
                 mbar_arrive_expect_tx(&bars[4], 2 * 8192);
                 for (int blk = 0; blk < 2; ++blk)
-                    tma_load_3d(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b);
+                    tma_load_3d_hint(sm + P_V + blk * 8192, &maps.v, &bars[4], h * D + 64 * blk, n * C, b, pol_in);
             }
         }
     };
@@ -593,7 +595,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         __syncthreads();
         tc_fence_after();
         if (tid == 0 && !failed) {   // K~^T is final: its image goes out now
-            bulk_store(img + IMG_KP, sm + PD_KT, 16384);
+            bulk_store_hint(img + IMG_KP, sm + PD_KT, 16384, pol_img);
             bulk_commit();
         }
         if (!exact && tid == 32) {   // S = [K e^(G-c); Q e^(G-c)] K~^T (B MN-major: K~^T [d][i])
@@ -739,7 +741,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     });
     if constexpr (!PD) load_v_late();  // K~^T, the write key's last reader, is formed
     if (!PD && tid == 0 && !failed) {   // K~^T is final: its image goes out now
-        bulk_store(img + IMG_KP, sm + P_KT, 16384);
+        bulk_store_hint(img + IMG_KP, sm + P_KT, 16384, pol_img);
         bulk_commit();
     }
     // T diag(beta) and T diag(beta e^G) as bf16 K-major [r][i]
@@ -827,8 +829,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     __syncthreads();
     tc_fence_after();
     if (tid == 0 && !failed) {   // U^T and P are final
-        bulk_store(img + IMG_UT, sm + P_WUT + 16384, 16384);
-        bulk_store(img + IMG_KP + 16384, sm + P_P, 8192);
+        bulk_store_hint(img + IMG_UT, sm + P_WUT + 16384, 16384, pol_img);
+        bulk_store_hint(img + IMG_KP + 16384, sm + P_P, 8192, pol_img);
         bulk_commit();
     }
     if (tid == 32 && !failed) {
@@ -880,7 +882,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         if (hh == 0) named_bar(1, 128);
         else named_bar(3, 128);
         if ((tid & 127) == 0 && !failed) {
-            bulk_store(img + IMG_PQ + hh * PQ_BLK, sm + S_PHI + hh * 16384, 16384);
+            bulk_store_hint(img + IMG_PQ + hh * PQ_BLK, sm + S_PHI + hh * 16384, 16384, pol_img);
             bulk_commit();
         }
     }
@@ -911,8 +913,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     __syncthreads();
     if (tid == 0) {
         if (!failed) {
-            bulk_store(img + IMG_PQ + 16384, sm + S_QPT, 8192);
-            bulk_store(img + IMG_PQ + PQ_BLK + 16384, sm + S_QPT + 8192, 8192);
+            bulk_store_hint(img + IMG_PQ + 16384, sm + S_QPT, 8192, pol_img);
+            bulk_store_hint(img + IMG_PQ + PQ_BLK + 16384, sm + S_QPT + 8192, 8192, pol_img);
             bulk_commit();
         }
         bulk_wait_read();
@@ -1044,6 +1046,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
     const int NC = p.nchunks;
     const uint8_t* wsh = p.ws + (size_t)bh * p.cw * IMG_BYTES;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint64_t pol_once = l2_evict_first();   // images (dead once read) and o
     int failed = 0;
 
     if (tid == 0) {
@@ -1086,16 +1089,16 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             if (failed) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[CB_KU0 + s], 24576 + 16384);
-                bulk_load(sm + CH_KP + s * 24576, img(nl) + IMG_KP, 24576, &bars[CB_KU0 + s]);
-                bulk_load(sm + CH_UT + s * 16384, img(nl) + IMG_UT, 16384, &bars[CB_KU0 + s]);
+                bulk_load_hint(sm + CH_KP + s * 24576, img(nl) + IMG_KP, 24576, &bars[CB_KU0 + s], pol_once);
+                bulk_load_hint(sm + CH_UT + s * 16384, img(nl) + IMG_UT, 16384, &bars[CB_KU0 + s], pol_once);
             }
             if (nl >= 2) wait(CB_PQFREE0 + s, ((nl - 2) >> 1) & 1);   // state product of nl - 2 done
             if (failed) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[CB_PQ0 + s], 2 * PQ_BLK);
-                bulk_load(sm + CH_PQ + s * 2 * PQ_BLK, img(nl) + IMG_PQ, 2 * PQ_BLK, &bars[CB_PQ0 + s]);
+                bulk_load_hint(sm + CH_PQ + s * 2 * PQ_BLK, img(nl) + IMG_PQ, 2 * PQ_BLK, &bars[CB_PQ0 + s], pol_once);
                 mbar_arrive_expect_tx(&bars[CB_GAM0 + (nl & 3)], 512);
-                bulk_load(sm + CH_GAM + (nl & 3) * 512, img(nl) + IMG_GAM, 512, &bars[CB_GAM0 + (nl & 3)]);
+                bulk_load_hint(sm + CH_GAM + (nl & 3) * 512, img(nl) + IMG_GAM, 512, &bars[CB_GAM0 + (nl & 3)], pol_once);
                 if (nl + 2 < NC) bulk_prefetch_l2(img(nl + 2), IMG_BYTES);
             }
             if (nl >= 2) {   // both products of chunk nl - 2 are done: its image is dead in L2
@@ -1189,8 +1192,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 mbar_arrive(&bars[CB_OFREE0 + s]);
                 if (!failed) {
                     const int t0 = (p.chunk0 + nl) * C;
-                    tma_store_3d(&maps.o, sm + CH_OT + s * 16384, h * D, t0, b);
-                    tma_store_3d(&maps.o, sm + CH_OT + s * 16384 + 8192, h * D + 64, t0, b);
+                    tma_store_3d_hint(&maps.o, sm + CH_OT + s * 16384, h * D, t0, b, pol_once);
+                    tma_store_3d_hint(&maps.o, sm + CH_OT + s * 16384 + 8192, h * D + 64, t0, b, pol_once);
                     bulk_commit();
                 }
             }
@@ -1204,25 +1207,32 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         float hv[32];
         // hv = h_{nl-1}^T Diag(gamma_{nl-1}) + X^T_{nl-1}, once the state product of
         // chunk nl - 1 is done; a uniform gamma is read before that wait
+        // (the decay is applied while the product is still running, so that only
+        // the additions follow its completion)
         auto advance = [&](int nl) {
             const int sp = (nl - 1) & 1;
             const float* gp = reinterpret_cast<const float*>(sm + CH_GAM + ((nl - 1) & 3) * 512) + 32 * c;
             wait(CB_GAM0 + ((nl - 1) & 3), ((nl - 1) >> 2) & 1);
-            float g1 = 1.f;
-            if constexpr (UNIFORM_GAMMA) g1 = *gp;
+            if constexpr (UNIFORM_GAMMA) {
+                const float g1 = *gp;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) hv[e] *= g1;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 g4 = *reinterpret_cast<const float4*>(gp + 4 * j);
+                    hv[4 * j] *= g4.x;
+                    hv[4 * j + 1] *= g4.y;
+                    hv[4 * j + 2] *= g4.z;
+                    hv[4 * j + 3] *= g4.w;
+                }
+            }
             wait(CB_SDONE0 + sp, ((nl - 1) >> 1) & 1);
             tc_fence_after();
             float xv[32];
             ld_cols<32>(tmem + TM_D + TM_SLOT * sp + lane_off + 32 * c, xv);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float4 g4 = make_float4(g1, g1, g1, g1);
-                if constexpr (!UNIFORM_GAMMA) g4 = *reinterpret_cast<const float4*>(gp + 4 * j);
-                hv[4 * j] = fmaf(g4.x, hv[4 * j], xv[4 * j]);
-                hv[4 * j + 1] = fmaf(g4.y, hv[4 * j + 1], xv[4 * j + 1]);
-                hv[4 * j + 2] = fmaf(g4.z, hv[4 * j + 2], xv[4 * j + 2]);
-                hv[4 * j + 3] = fmaf(g4.w, hv[4 * j + 3], xv[4 * j + 3]);
-            }
+            for (int e = 0; e < 32; ++e) hv[e] += xv[e];
         };
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
