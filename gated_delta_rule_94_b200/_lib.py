@@ -26,7 +26,8 @@ EXPORTED = ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd_wor
             "gdn_decode_step",
             "gdn_read_device_status", "gdn_status_string", "gdn_abi_version",
             "gdn_kernel_launch_count", "gdn_chunk_fwd_kernel_name", "gdn_chunk_fwd_noalloc",
-            "gdn_chunk_fwd_noalloc_scratch_bytes", "gdn_osdn_precondition", "gdn_chunk_fwd_wk")
+            "gdn_chunk_fwd_noalloc_scratch_bytes", "gdn_osdn_precondition", "gdn_chunk_fwd_wk",
+            "gdn_chunk_fwd_plan")
 
 _lib = None
 
@@ -75,6 +76,9 @@ def load() -> ctypes.CDLL:
     lib.gdn_chunk_fwd_wk.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, vp,
                                      sz, vp]
     lib.gdn_chunk_fwd_wk.restype = i
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.gdn_chunk_fwd_plan.argtypes = [i, i, i, i, i, i, i, i, sz, ip, ip, ip]
+    lib.gdn_chunk_fwd_plan.restype = i
     _lib = lib
     return lib
 
@@ -146,6 +150,21 @@ def gdn_chunk_fwd_workspace_min_bytes(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfl
     if n == ctypes.c_size_t(-1).value:
         raise GdnError(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd_workspace_min_bytes")
     return n
+
+
+def gdn_chunk_fwd_plan(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16, gate_kind=GDN_GATE_SCALAR,
+                       workspace_bytes=None) -> dict:
+    """Waves, chunks per wave and segments per wave the forward uses with
+    `workspace_bytes` (default: the full-speed size)."""
+    if workspace_bytes is None:
+        workspace_bytes = gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, chunk, dtype, gate_kind)
+    w, c, s = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    st = load().gdn_chunk_fwd_plan(B, T, H, Dk, Dv, chunk, _dtype_code(dtype), int(gate_kind),
+                                   workspace_bytes, ctypes.byref(w), ctypes.byref(c),
+                                   ctypes.byref(s))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd_plan")
+    return {"waves": w.value, "chunks_per_wave": c.value, "segments": s.value}
 
 
 def gdn_chunk_fwd(q, k, v, beta, g, gate_kind, initial_state, o, final_state, *, chunk=64,

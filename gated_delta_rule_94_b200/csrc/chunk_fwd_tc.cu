@@ -998,6 +998,7 @@ static_assert(CB_COUNT * 8 <= 512, "barrier space");
 // row d -- write one row of a box without bank conflicts).
 struct ChainMaps {
     CUtensorMap o, s_out;
+    CUtensorMap seg;   // [2][B*H][nseg][D][D] segment offsets then transitions (segment mode 1)
 };
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, A from tensor memory (row m in lane m, k
@@ -1042,9 +1043,30 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const int NC = p.nchunks;
-    const uint8_t* wsh = p.ws + (size_t)bh * p.cw * IMG_BYTES;
+    // Role of this CTA.  Plain mode: one CTA per (batch, head) over the wave,
+    // from the entering state, with outputs.  Segment mode 1: per (batch, head,
+    // segment) the segment's offset (from a zero state, role 1) and, in the
+    // second half of the grid, its transition (from the identity with no
+    // writes, role 2), no outputs.  Segment mode 3: per (batch, head, segment)
+    // the outputs from the segment's entering state (role 0).
+    const int nbh = p.B * p.H;
+    const int S = p.seg_mode ? p.nseg : 1;
+    int role = 0, bh = blockIdx.x, j = 0;
+    if (p.seg_mode == 1) {
+        const int per = nbh * S;
+        role = (int)blockIdx.x < per ? 1 : 2;
+        const int r = (int)blockIdx.x % per;
+        bh = r / S;
+        j = r % S;
+    } else if (p.seg_mode == 3) {
+        bh = blockIdx.x / S;
+        j = blockIdx.x % S;
+    }
+    const int b = bh / H, h = bh % H;
+    const int c0 = p.seg_mode ? j * p.seg_len : 0;
+    const int NC = p.seg_mode ? min(p.seg_len, p.nchunks - c0) : p.nchunks;
+    const bool outputs = role == 0;
+    const uint8_t* wsh = p.ws + ((size_t)bh * p.cw + c0) * IMG_BYTES;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint64_t pol_once = l2_evict_first();   // images (dead once read) and o
     int failed = 0;
@@ -1061,8 +1083,10 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         tmem_relinquish();
     }
     // the next wave's prep may start on the SMs this grid leaves idle; the
-    // images and the carried state of this wave are read only after the wait
-    pdl_launch_dependents();
+    // images and the carried state of this wave are read only after the wait.
+    // (The segment offsets and transitions let the combine start only once
+    // they are done: its CTAs must not hold SMs that theirs still need.)
+    if (p.seg_mode != 1) pdl_launch_dependents();
     pdl_wait();
     tc_fence_before();
     __syncthreads();
@@ -1085,12 +1109,14 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
+            if (role != 2) {   // the transition (role 2) writes nothing: no K~^T, P, U^T
             if (nl >= 2) wait(CB_KUFREE0 + s, ((nl - 2) >> 1) & 1);   // U^T [K~|P^T] of nl - 2 done
             if (failed) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[CB_KU0 + s], 24576 + 16384);
                 bulk_load_hint(sm + CH_KP + s * 24576, img(nl) + IMG_KP, 24576, &bars[CB_KU0 + s], pol_once);
                 bulk_load_hint(sm + CH_UT + s * 16384, img(nl) + IMG_UT, 16384, &bars[CB_KU0 + s], pol_once);
+            }
             }
             if (nl >= 2) wait(CB_PQFREE0 + s, ((nl - 2) >> 1) & 1);   // state product of nl - 2 done
             if (failed) break;
@@ -1101,8 +1127,9 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 bulk_load_hint(sm + CH_GAM + (nl & 3) * 512, img(nl) + IMG_GAM, 512, &bars[CB_GAM0 + (nl & 3)], pol_once);
                 if (nl + 2 < NC) bulk_prefetch_l2(img(nl + 2), IMG_BYTES);
             }
-            if (nl >= 2) {   // both products of chunk nl - 2 are done: its image is dead in L2
-                             // (gamma of chunk nl - 3 too: the state pass has used it)
+            if (nl >= 2 && outputs) {   // both products of chunk nl - 2 are done: its image is
+                             // dead in L2 (gamma of chunk nl - 3 too: the state pass has used
+                             // it); segment offsets and transitions leave them for the outputs
                 l2_discard(img(nl - 2), IMG_GAM, lane);
                 if (nl >= 3) l2_discard(img(nl - 3) + IMG_GAM, 512, lane);
             }
@@ -1124,7 +1151,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             wait(CB_KU0 + s, (nl >> 1) & 1);
             if (nl >= 2) {
                 wait(CB_XFREE0 + s, ((nl - 2) >> 1) & 1);
-                wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
+                if (outputs) wait(CB_OFREE0 + s, ((nl - 2) >> 1) & 1);
             }
             tc_fence_after();
             if (leader && !failed) {
@@ -1135,7 +1162,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 mma_commit(&bars[CB_KUFREE0 + s]);
             }
         };
-        if (NC > 0) issue_ku(0);
+        if (NC > 0 && role != 2) issue_ku(0);
 #pragma unroll 1
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
@@ -1147,17 +1174,19 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 for (int k = 0; k < 8; ++k)   // X^T += h^T Phi^T: rows 0..127 of [Phi ; Qp]
                     mma_bf16_ta(tmem + TM_D + TM_SLOT * s, tmem + TM_HT + TM_SLOT * s + 8 * k,
                                 d_pq + ((s * 2 * PQ_BLK + (k >> 2) * PQ_BLK + (k & 3) * 32) >> 4),
-                                id_phi, true);
+                                id_phi, role != 2 || k > 0);   // the transition has no U^T K~
                 mma_commit(&bars[CB_SDONE0 + s]);
+                if (outputs) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k)   // O^T += h^T Qp^T: rows 128..191
-                    mma_bf16_ta(tmem + TM_D + TM_SLOT * s + 128, tmem + TM_HT + TM_SLOT * s + 8 * k,
-                                d_pq + ((s * 2 * PQ_BLK + (k >> 2) * PQ_BLK + 16384 + (k & 3) * 32) >> 4),
-                                id_qp, true);
-                mma_commit(&bars[CB_ODONE0 + s]);
+                    for (int k = 0; k < 8; ++k)   // O^T += h^T Qp^T: rows 128..191
+                        mma_bf16_ta(tmem + TM_D + TM_SLOT * s + 128, tmem + TM_HT + TM_SLOT * s + 8 * k,
+                                    d_pq + ((s * 2 * PQ_BLK + (k >> 2) * PQ_BLK + 16384 + (k & 3) * 32) >> 4),
+                                    id_qp, true);
+                    mma_commit(&bars[CB_ODONE0 + s]);
+                }
                 mma_commit(&bars[CB_PQFREE0 + s]);
             }
-            if (nl + 1 < NC) issue_ku(nl + 1);
+            if (nl + 1 < NC && role != 2) issue_ku(nl + 1);
         }
         if (leader) mma_commit(&bars[CB_FINAL]);
         int final_failed = 0;
@@ -1169,7 +1198,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         const int v = (warp & 3) * 32 + lane;
         const bool leader = warp == W_OUT && lane == 0;
 #pragma unroll 1
-        for (int nl = 0; nl < NC; ++nl) {
+        for (int nl = 0; nl < (outputs ? NC : 0); ++nl) {
             const int s = nl & 1;
             if (leader && nl >= 2) bulk_wait_read_all_but_one();   // the store of chunk nl - 2 read slot s
             named_bar(2, 128);
@@ -1191,7 +1220,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             if (leader) {
                 mbar_arrive(&bars[CB_OFREE0 + s]);
                 if (!failed) {
-                    const int t0 = (p.chunk0 + nl) * C;
+                    const int t0 = (p.chunk0 + c0 + nl) * C;
                     tma_store_3d_hint(&maps.o, sm + CH_OT + s * 16384, h * D, t0, b, pol_once);
                     tma_store_3d_hint(&maps.o, sm + CH_OT + s * 16384 + 8192, h * D + 64, t0, b, pol_once);
                     bulk_commit();
@@ -1238,15 +1267,21 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         for (int nl = 0; nl < NC; ++nl) {
             const int s = nl & 1;
             if (nl == 0) {
-                if (p.s0) {   // column v, rows d = 32c.. of M = S^T: for each d the 32
-                              // lanes read 128 consecutive bytes (L2 only: the carried
-                              // state was written by the previous launch)
-                    const float* src = p.s0 + (size_t)bh * D * D + (size_t)(32 * c) * D + v;
+                // the entering state: the wave's (plain mode, first segment), the
+                // segment's from the combine (later segments), zero (offsets) or
+                // the identity (transitions)
+                const float* s0 = role != 0 ? nullptr
+                                  : j == 0  ? (p.s0 ? p.s0 + (size_t)bh * D * D : nullptr)
+                                            : p.seg_h + ((size_t)bh * S + j) * D * D;
+                if (s0) {   // column v, rows d = 32c.. of M = S^T: for each d the 32
+                            // lanes read 128 consecutive bytes (L2 only: the carried
+                            // state was written by an earlier launch)
+                    const float* src = s0 + (size_t)(32 * c) * D + v;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) hv[e] = __ldcg(src + (size_t)e * D);
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) hv[e] = 0.f;
+                    for (int e = 0; e < 32; ++e) hv[e] = (role == 2 && 32 * c + e == v) ? 1.f : 0.f;
                 }
             } else {
                 advance(nl);
@@ -1268,9 +1303,13 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         if (NC > 0) {   // final state, staged over the [Phi ; Qp] slots (free once the
                         // last state product is done), written by four TMA stores
             advance(NC);
-            if (p.s_out) {
+            // where the final state goes: the wave's (plain mode, last segment), the
+            // segment's offset or transition (segment mode 1), or nowhere
+            const CUtensorMap* smap = role != 0 ? &maps.seg : (j == S - 1 ? &maps.s_out : nullptr);
+            const int sidx = role == 0 ? bh : (role - 1) * nbh * S + bh * S + j;
+            if (role != 0 || (j == S - 1 && p.s_out)) {
                 // the last chunk's h^T Qp^T (behind h^T Phi^T) may still read its slot
-                wait(CB_ODONE0 + ((NC - 1) & 1), ((NC - 1) >> 1) & 1);
+                if (outputs) wait(CB_ODONE0 + ((NC - 1) & 1), ((NC - 1) >> 1) & 1);
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
                     *reinterpret_cast<float*>(sm + CH_PQ + st_off(32 * c + e, v)) = hv[e];
@@ -1279,7 +1318,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 if (warp == W_ST && lane == 0) {
                     if (!failed) {
                         for (int cb = 0; cb < 4; ++cb)
-                            tma_store_3d(&maps.s_out, sm + CH_PQ + cb * 16384, 32 * cb, 0, bh);
+                            tma_store_3d(smap, sm + CH_PQ + cb * 16384, 32 * cb, 0, sidx);
                         bulk_commit();
                     }
                     bulk_wait_read();
@@ -1293,6 +1332,80 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+
+// ------------------------------------------------------------- segments
+// Segment-parallel state pass.  Each chunk maps the entering state affinely,
+// h' = (Diag(gamma) + Phi) h + K~^T U, so a run of chunks (a segment j) does
+// too: h_out = A_j h_in + b_j.  The chain kernel in segment mode 1 forms b_j
+// (from a zero state) and A_j (from the identity, with no writes) for every
+// segment at once; this kernel composes them in order, h_{j+1} = A_j h_j + b_j
+// in fp32 from the wave's entering state h_0; the chain kernel in segment
+// mode 3 then runs every segment from its h_j with outputs.  One CTA per
+// (batch, head), 1024 threads: thread (row d, 16 columns v); h and A_j in
+// shared memory (A_j rows padded by one word).
+constexpr int SEGC_THREADS = 1024;
+constexpr uint32_t SEGC_SMEM = (D * D + D * (D + 1)) * sizeof(float);
+
+__global__ void __launch_bounds__(SEGC_THREADS)
+segment_combine_kernel(const ChunkParams p, const float* __restrict__ seg_b,
+                       const float* __restrict__ seg_a) {
+    extern __shared__ float smf[];
+    float* hs = smf;             // h_j [D][D]
+    float* As = smf + D * D;     // A_j [D][D + 1]
+    pdl_wait();                  // offsets and transitions are complete and visible
+                                 // (no early launch of the output pass: its CTAs wait
+                                 // for this grid and must not hold SMs it needs)
+    const int bh = blockIdx.x, S = p.nseg, t = threadIdx.x;
+    const int d = t >> 3, cg = t & 7;
+    for (int idx = t; idx < D * D; idx += SEGC_THREADS)
+        hs[idx] = p.s0 ? __ldcg(p.s0 + (size_t)bh * D * D + idx) : 0.f;
+#pragma unroll 1
+    for (int jj = 0; jj + 1 < S; ++jj) {
+        const size_t off = ((size_t)bh * S + jj) * D * D;
+        for (int idx = t; idx < D * D; idx += SEGC_THREADS)
+            As[(idx >> 7) * (D + 1) + (idx & 127)] = __ldcg(seg_a + off + idx);
+        float acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = __ldcg(seg_b + off + d * D + 16 * cg + e);
+        __syncthreads();
+#pragma unroll 4
+        for (int dp = 0; dp < D; ++dp) {
+            const float a = As[d * (D + 1) + dp];
+            const float4* hr = reinterpret_cast<const float4*>(hs + dp * D + 16 * cg);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 x = hr[q];
+                acc[4 * q] = fmaf(a, x.x, acc[4 * q]);
+                acc[4 * q + 1] = fmaf(a, x.y, acc[4 * q + 1]);
+                acc[4 * q + 2] = fmaf(a, x.z, acc[4 * q + 2]);
+                acc[4 * q + 3] = fmaf(a, x.w, acc[4 * q + 3]);
+            }
+        }
+        __syncthreads();         // every thread is done with h_j and A_j
+        float* dst = p.seg_h + ((size_t)bh * S + jj + 1) * D * D + d * D + 16 * cg;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            hs[d * D + 16 * cg + e] = acc[e];
+            dst[e] = acc[e];
+        }
+        __syncthreads();
+    }
+}
+
+// Segments per (batch, head) for a wave of nchunks chunks: only when the
+// heads leave most SMs idle (pass 1 runs two CTAs per segment, one per SM),
+// with at least eight chunks a segment; 1 means the plain chain.
+constexpr int kSegSMs = 148;
+int segments_for(int nbh, int nchunks) {
+    if (nbh > 16) return 1;
+    const int S = std::min(kSegSMs / (2 * nbh), nchunks / 8);
+    return std::max(S, 1);
+}
+size_t seg_bytes(int nbh, int NC) {
+    const int S = segments_for(nbh, NC);
+    return S > 1 ? (size_t)3 * nbh * S * D * D * sizeof(float) : 0;
 }
 
 bool make_maps(const ChunkParams& p, bool perdim, PrepMaps* m) {
@@ -1348,6 +1461,14 @@ size_t workspace_for(int nbh, int NC, int cw) {
     return bytes + counter_bytes(NC);
 }
 
+// How a forward of NC chunks over nbh heads runs with ws_bytes of workspace:
+// chunks per wave, waves, and whether the segment buffers are reserved.
+struct Plan {
+    int cw, nw, S_size;
+    bool use_seg;
+};
+Plan plan_for(int B, int T, int H, int gate, size_t ws_bytes);
+
 }  // namespace
 
 bool chunk_fwd_tc_supported(int Dk, int Dv, int gate) {
@@ -1359,7 +1480,40 @@ size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H, int gate) {
     const int NC = (T + C - 1) / C;
     if (NC == 0 || B == 0 || H == 0) return 0;
     const int nbh = B * H;
-    return workspace_for(nbh, NC, wave_chunks(nbh, NC, ~static_cast<size_t>(0)));
+    return workspace_for(nbh, NC, wave_chunks(nbh, NC, ~static_cast<size_t>(0))) + seg_bytes(nbh, NC);
+}
+
+namespace {
+Plan plan_for(int B, int T, int H, int gate, size_t ws_bytes) {
+    Plan pl{0, 0, 1, false};
+    const int NC = (T + C - 1) / C;
+    const int nbh = B * H;
+    // segment buffers first, when the workspace holds them beside the least the
+    // forward needs (the full-speed size does); then waves as long as the rest allows
+    const size_t sbytes = seg_bytes(nbh, NC);
+    pl.use_seg = sbytes > 0 && ws_bytes >= chunk_fwd_tc_workspace_min_bytes(B, T, H, gate) + sbytes;
+    pl.cw = wave_chunks(nbh, NC, pl.use_seg ? ws_bytes - sbytes : ws_bytes);
+    pl.nw = pl.cw > 0 ? (NC + pl.cw - 1) / pl.cw : 0;
+    pl.S_size = pl.use_seg ? segments_for(nbh, NC) : 1;
+    return pl;
+}
+// Segments of a wave of nchunks chunks (the launcher's rule).
+int wave_segments(const Plan& pl, int nbh, int nchunks) {
+    int Sw = pl.use_seg ? std::min(segments_for(nbh, nchunks), pl.S_size) : 1;
+    if (Sw > 1) {
+        const int L = (nchunks + Sw - 1) / Sw;
+        Sw = (nchunks + L - 1) / L;
+    }
+    return Sw;
+}
+}  // namespace
+
+void chunk_fwd_tc_plan(int B, int T, int H, int gate, size_t ws_bytes, int* waves,
+                       int* chunks_per_wave, int* segments) {
+    const Plan pl = plan_for(B, T, H, gate, ws_bytes);
+    *waves = pl.nw;
+    *chunks_per_wave = pl.cw;
+    *segments = pl.cw > 0 ? wave_segments(pl, B * H, pl.cw) : 0;
 }
 
 size_t chunk_fwd_tc_workspace_min_bytes(int B, int T, int H, int gate) {
@@ -1407,11 +1561,16 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
     auto chain = gate == kGatePerDim ? chunk_chain_kernel<false> : chunk_chain_kernel<true>;
     e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CH_SMEM);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SEGC_SMEM);
+    if (e != cudaSuccess) return e;
     const int NC = (p0.T + C - 1) / C;
     const int nbh = p0.B * p0.H;
-    const int cw = wave_chunks(nbh, NC, ws_bytes);
+    const Plan pl = plan_for(p0.B, p0.T, p0.H, gate, ws_bytes);
+    const bool use_seg = pl.use_seg;
+    const int cw = pl.cw;
     if (cw < 1) return cudaErrorInvalidValue;
-    const int nw = (NC + cw - 1) / cw;
+    const int nw = pl.nw;
     const size_t buf_bytes = (size_t)nbh * cw * IMG_BYTES;
     float* carry = nw > 1 ? reinterpret_cast<float*>(p0.ws + 2 * buf_bytes) : nullptr;
     unsigned* counters = reinterpret_cast<unsigned*>(
@@ -1434,6 +1593,11 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
     memset(&m_sout, 0, sizeof(m_sout));
     memset(&m_carry, 0, sizeof(m_carry));
     if (!state_map(&m_sout, p0.s_out) || !state_map(&m_carry, carry)) return cudaErrorInvalidValue;
+    // segment buffers after the counters: entering states [B*H][S][D][D], then
+    // offsets and transitions [2][B*H][S][D][D]
+    const int S_size = pl.S_size;
+    float* seg_h = use_seg ? reinterpret_cast<float*>(p0.ws + workspace_for(nbh, NC, cw)) : nullptr;
+    float* seg2 = use_seg ? seg_h + (size_t)nbh * S_size * D * D : nullptr;
     // Every launch but the first may start before its predecessor ends
     // (programmatic dependent launch); the kernels order themselves with
     // griddepcontrol (see chunk_prep_kernel and chunk_chain_kernel).
@@ -1461,12 +1625,45 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
         e = cudaLaunchKernelEx(&cfg, prep, maps, p);
         if (e != cudaSuccess) return e;
         ++*launches;
-        cfg.gridDim = dim3((unsigned)nbh);
         cfg.blockDim = dim3(CH_THREADS);
         cfg.dynamicSmemBytes = CH_SMEM;
         cfg.numAttrs = 1;
         ChainMaps cm = cmap0;
         cm.s_out = (w + 1 == nw) ? m_sout : m_carry;
+        const int Sw = wave_segments(pl, nbh, p.nchunks);
+        if (Sw > 1) {   // segment-parallel state pass: offsets and transitions,
+                        // their composition, then every segment with outputs
+            const int L = (p.nchunks + Sw - 1) / Sw;
+            p.nseg = Sw;
+            p.seg_len = L;
+            p.seg_h = seg_h;
+            {
+                const uint64_t dims[3] = {(uint64_t)D, (uint64_t)D, (uint64_t)2 * nbh * Sw};
+                const uint64_t strides[2] = {(uint64_t)D * 4, (uint64_t)D * D * 4};
+                const uint32_t box[3] = {32, 128, 1};
+                if (!make_tmap(&cm.seg, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, seg2, 3, dims, strides, box))
+                    return cudaErrorInvalidValue;
+            }
+            p.seg_mode = 1;
+            cfg.gridDim = dim3((unsigned)(2 * nbh * Sw));
+            e = cudaLaunchKernelEx(&cfg, chain, cm, p);
+            if (e != cudaSuccess) return e;
+            ++*launches;
+            cudaLaunchConfig_t cc = cfg;
+            cc.gridDim = dim3((unsigned)nbh);
+            cc.blockDim = dim3(SEGC_THREADS);
+            cc.dynamicSmemBytes = SEGC_SMEM;
+            const float* sb_ = seg2;
+            const float* sa_ = seg2 + (size_t)nbh * Sw * D * D;
+            e = cudaLaunchKernelEx(&cc, segment_combine_kernel, p, sb_, sa_);
+            if (e != cudaSuccess) return e;
+            ++*launches;
+            p.seg_mode = 3;
+            cfg.gridDim = dim3((unsigned)(nbh * Sw));
+        } else {
+            p.seg_mode = 0;
+            cfg.gridDim = dim3((unsigned)nbh);
+        }
         e = cudaLaunchKernelEx(&cfg, chain, cm, p);
         if (e != cudaSuccess) return e;
         ++*launches;

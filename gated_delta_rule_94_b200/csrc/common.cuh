@@ -32,6 +32,10 @@ struct ChunkParams {
     int nchunks;       // chunks in this wave
     int ws_chunk;      // bytes of one chunk's workspace image
     unsigned* counter; // this wave's item counter (persistent prep CTAs take items from it)
+    // segment-parallel state pass (seg_mode 0: one chain CTA per (batch, head))
+    int seg_mode;      // 1: offsets and transitions of every segment; 3: outputs of every segment
+    int nseg, seg_len; // segments per (batch, head) in this wave, chunks per segment
+    float* seg_h;      // [B*H][nseg][Dk][Dv] entering state of each segment (j >= 1)
 };
 
 // Phase 1 of the preconditioned delta rule (write keys kw = d (.) k).
@@ -89,6 +93,9 @@ bool chunk_fwd_tc_supported(int Dk, int Dv, int gate);
 // Workspace for the longest waves the forward uses / the least it runs with.
 size_t chunk_fwd_tc_workspace_bytes(int B, int T, int H, int gate);
 size_t chunk_fwd_tc_workspace_min_bytes(int B, int T, int H, int gate);
+// Waves, chunks per wave and segments per wave of a forward with ws_bytes.
+void chunk_fwd_tc_plan(int B, int T, int H, int gate, size_t ws_bytes, int* waves,
+                       int* chunks_per_wave, int* segments);
 // Enqueues the tensor-core forward with a workspace of ws_bytes (at least the
 // minimum; waves as long as it allows); *launches receives the number of
 // kernels.

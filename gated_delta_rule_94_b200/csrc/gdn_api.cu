@@ -106,6 +106,29 @@ size_t gdn_chunk_fwd_workspace_min_bytes(int B, int T, int H, int Dk, int Dv, in
     return 0;
 }
 
+gdn_status gdn_chunk_fwd_plan(int B, int T, int H, int Dk, int Dv, int chunk, gdn_dtype dtype,
+                              gdn_gate gate_kind, size_t workspace_bytes, int* waves,
+                              int* chunks_per_wave, int* segments) {
+    if (!waves || !chunks_per_wave || !segments) return GDN_ERR_INVALID_ARG;
+    const size_t least =
+        gdn_chunk_fwd_workspace_min_bytes(B, T, H, Dk, Dv, chunk, dtype, gate_kind);
+    if (least == (size_t)-1) {
+        if (B < 0 || T < 0 || H < 0 || (dtype != GDN_BF16 && dtype != GDN_F32) ||
+            gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM)
+            return GDN_ERR_INVALID_ARG;
+        return GDN_ERR_UNSUPPORTED;
+    }
+    if (workspace_bytes < least) return GDN_ERR_WORKSPACE;
+    const int NC = (T + 63) / 64;
+    *waves = B * H > 0 && NC > 0 ? 1 : 0;
+    *chunks_per_wave = NC;
+    *segments = *waves;
+    if (least > 0)   // the tensor-core path
+        gdn::chunk_fwd_tc_plan(B, T, H, gate_kind, workspace_bytes, waves, chunks_per_wave,
+                               segments);
+    return GDN_OK;
+}
+
 }  // extern "C"
 
 namespace {
@@ -168,7 +191,7 @@ gdn_status chunk_fwd_impl(const void* q, const void* k, const void* kw, const vo
         return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
     }
 
-    gdn::ChunkParams p;
+    gdn::ChunkParams p{};
     p.q = q; p.k = k; p.v = v; p.beta = beta; p.g = g; p.kw = kw;
     p.s0 = initial_state; p.o = o; p.s_out = final_state;
     p.B = B; p.T = T; p.H = H; p.Dk = Dk; p.Dv = Dv;

@@ -119,10 +119,36 @@ GDN_API size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int Dk, int Dv
  * none; never more than gdn_chunk_fwd_workspace_bytes).  Any size in between
  * works: the forward runs the sequence in waves of chunks whose step images
  * fit the workspace, so less workspace means shorter waves and less overlap,
- * with results identical to the bit.  Returns (size_t)-1 for an unsupported
- * or invalid shape. */
+ * with results identical to the bit -- except that with few (batch, head)
+ * pairs and long waves the full-speed size also holds the buffers of the
+ * segment-parallel state pass, which rounds differently (within the
+ * tolerance); gdn_chunk_fwd_plan tells which.  Returns (size_t)-1 for an
+ * unsupported or invalid shape. */
 GDN_API size_t gdn_chunk_fwd_workspace_min_bytes(int B, int T, int H, int Dk, int Dv, int chunk,
                                                  gdn_dtype dtype, gdn_gate gate_kind);
+
+/*
+ * gdn_chunk_fwd_plan -- how gdn_chunk_fwd runs these arguments with
+ * `workspace_bytes` of workspace (no device access, nothing enqueued):
+ *   *waves            number of waves (launch groups) the sequence runs in
+ *   *chunks_per_wave  chunks of every (batch, head) in a full wave
+ *   *segments         segments per (batch, head) of a full wave: 1 is the
+ *                     serial state pass; S > 1 is the segment-parallel pass
+ *                     (each chunk maps the entering state affinely, so a run of
+ *                     chunks does too: the offsets and transitions of all S
+ *                     segments are formed in parallel, composed in order, and
+ *                     every segment then runs from its own entering state;
+ *                     "Moonshot AI's New Attention Architecture", sec. 3, the
+ *                     chunkwise state recurrence).  Chosen when the (batch,
+ *                     head) pairs leave most SMs idle and the workspace holds
+ *                     its buffers (gdn_chunk_fwd_workspace_bytes does).
+ * Returns GDN_ERR_WORKSPACE below gdn_chunk_fwd_workspace_min_bytes and the
+ * argument errors of gdn_chunk_fwd_workspace_bytes.
+ */
+GDN_API gdn_status gdn_chunk_fwd_plan(int B, int T, int H, int Dk, int Dv, int chunk,
+                                      gdn_dtype dtype, gdn_gate gate_kind,
+                                      size_t workspace_bytes, int* waves, int* chunks_per_wave,
+                                      int* segments);
 
 /*
  * gdn_decode_step -- one recurrent step for N independent sequences: the
