@@ -322,6 +322,161 @@ def chunk_form(q, k, v, beta, g, gate_kind, S0=None, C: int = 64, kw=None):
     return o, M_final
 
 
+def backward(q, k, v, beta, g, gate_kind, S0, do, dS=None):
+    """Gradients of the operator by reverse-mode automatic differentiation of
+    the plain token loop (torch autograd, fp64, CPU): the scalar
+        L = sum(o * do) + sum(S_T * dS)
+    differentiated with respect to q, k, v, beta, g and S0.  The loop is the
+    recurrence of :func:`recurrent` (decay, recall, residual, write, output),
+    written with torch ops so that autograd can run through it; the pages print
+    no backward formula, so the definition of the gradient is the derivative of
+    the forward itself.  Returns a dict dq, dk, dv, dbeta, dg (None without a
+    gate), dS0 (of the same shapes as the inputs; dS0 also when S0 is None).
+    """
+    import torch
+    t = {n: None if a is None else torch.tensor(np.asarray(a, np.float64), requires_grad=True)
+         for n, a in (("q", q), ("k", k), ("v", v), ("beta", beta), ("g", g))}
+    B, T, H, Dk = t["q"].shape
+    Dv = t["v"].shape[-1]
+    S0t = torch.zeros(B, H, Dk, Dv, dtype=torch.float64) if S0 is None else \
+        torch.tensor(np.asarray(S0, np.float64))
+    S0t.requires_grad_(True)
+    M = S0t
+    outs = []
+    for step in range(T):
+        if gate_kind == GATE_SCALAR:
+            M = torch.exp(t["g"][:, step])[:, :, None, None] * M
+        elif gate_kind == GATE_PER_DIM:
+            M = torch.exp(t["g"][:, step])[:, :, :, None] * M
+        kt, vt, qt = t["k"][:, step], t["v"][:, step], t["q"][:, step]
+        x = torch.einsum("bhij,bhi->bhj", M, kt)
+        r = t["beta"][:, step][..., None] * (vt - x)
+        M = M + kt[..., :, None] * r[..., None, :]
+        outs.append(torch.einsum("bhij,bhi->bhj", M, qt))
+    o = torch.stack(outs, 1) if T else torch.zeros(B, 0, H, Dv, dtype=torch.float64)
+    loss = (o * torch.tensor(np.asarray(do, np.float64))).sum()
+    if dS is not None:
+        loss = loss + (M * torch.tensor(np.asarray(dS, np.float64))).sum()
+    wrt = [t["q"], t["k"], t["v"], t["beta"], S0t] + ([t["g"]] if gate_kind != GATE_NONE else [])
+    grads = torch.autograd.grad(loss, wrt, allow_unused=True)
+    z = lambda gr, ref: (np.zeros(ref.shape) if gr is None else gr.detach().numpy())
+    out = {"dq": z(grads[0], t["q"]), "dk": z(grads[1], t["k"]), "dv": z(grads[2], t["v"]),
+           "dbeta": z(grads[3], t["beta"]), "dS0": z(grads[4], S0t),
+           "dg": z(grads[5], t["g"]) if gate_kind != GATE_NONE else None}
+    return out
+
+
+def chunk_backward(q, k, v, beta, g, gate_kind, S0, do, dS=None, C: int = 64):
+    """The same gradients as :func:`backward`, chunk by chunk (fp64 NumPy), by
+    differentiating the chunk form of :func:`chunk_form` by hand.  Per chunk,
+    with h the entering state, h' = Diag(gamma) h + K_tilde^T D the leaving one,
+    O = Q_bar h + P D, D = U - W h, and the upstream dO, dh':
+
+      dD  = P^T dO + K_tilde dh'
+      dh  = Q_bar^T dO - W^T dD + Diag(gamma) dh'       (the adjoint state: the
+            transpose of the chunk's affine map, run from the last chunk back)
+      dU = dD,  dW = -dD h^T,  dT = dU (beta V)^T + dW (beta K_bar)^T,
+      dA = StrictTril(-T^T dT T^T)                       (T = (I + A)^-1)
+      then through P = Tril(Q_bar K_breve^T), A = StrictTril(beta K_bar
+      K_breve^T), K_bar = Gamma K, Q_bar = Gamma Q, K_tilde = K Gamma_C / Gamma
+      to dq, dk, dv, dbeta and the in-chunk log-decays G, and dg as the
+      reverse cumulative sum of dG within the chunk (a scalar gate sums dG over
+      the key dimensions).
+    Returns the dict of :func:`backward`.
+    """
+    q, k, v, beta, g, S0, do, dS = map(_f64, (q, k, v, beta, g, S0, do, dS))
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    out = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v),
+           "dbeta": np.zeros_like(beta), "dS0": np.zeros((B, H, Dk, Dv)),
+           "dg": None if gate_kind == GATE_NONE else np.zeros_like(g)}
+    for b in range(B):
+        for h_ in range(H):
+            # forward over the chunks, keeping each entering state
+            chunks = [(c0, min(T, c0 + C)) for c0 in range(0, T, C)]
+            hs = []
+            h = np.zeros((Dk, Dv)) if S0 is None else S0[b, h_].copy()
+            saved = []
+            for c0, c1 in chunks:
+                n = c1 - c0
+                Q, K, V = q[b, c0:c1, h_], k[b, c0:c1, h_], v[b, c0:c1, h_]
+                bt = beta[b, c0:c1, h_]
+                if gate_kind == GATE_NONE:
+                    logs = np.zeros((n, Dk))
+                elif gate_kind == GATE_SCALAR:
+                    logs = np.repeat(g[b, c0:c1, h_][:, None], Dk, axis=1)
+                else:
+                    logs = g[b, c0:c1, h_]
+                G = np.cumsum(logs, axis=0)
+                Gam = np.exp(G)
+                diff = G[:, None, :] - G[None, :, :]
+                lower = np.tril(np.ones((n, n), bool))
+                E = np.exp(np.where(lower[:, :, None], diff, -np.inf))      # [r, i, d]
+                KK = np.einsum("rd,id,rid->ri", K, K, E)
+                QK = np.einsum("rd,id,rid->ri", Q, K, E)
+                A = np.tril(bt[:, None] * KK, -1)
+                Tm = forward_substitution_inverse(A)
+                Kbar, Qbar = Gam * K, Gam * Q
+                W, U = Tm @ (bt[:, None] * Kbar), Tm @ (bt[:, None] * V)
+                D = U - W @ h
+                P = np.tril(QK)
+                Kt = K * np.exp(G[n - 1][None, :] - G)
+                gam = Gam[n - 1]
+                hs.append(h)
+                saved.append((c0, c1, n, Q, K, V, bt, G, E, KK, Tm, Kbar, Qbar, W, D, P, Kt, gam))
+                h = gam[:, None] * h + Kt.T @ D
+            # backward over the chunks
+            dhn = np.zeros((Dk, Dv)) if dS is None else dS[b, h_].copy()
+            for (c0, c1, n, Q, K, V, bt, G, E, KK, Tm, Kbar, Qbar, W, D, P, Kt, gam), h in \
+                    zip(reversed(saved), reversed(hs)):
+                dO = do[b, c0:c1, h_]
+                dD = P.T @ dO + Kt @ dhn
+                dh = Qbar.T @ dO - W.T @ dD + gam[:, None] * dhn
+                dq = np.zeros((n, Dk)); dk = np.zeros((n, Dk)); dG = np.zeros((n, Dk))
+                dQbar = dO @ h.T
+                dq += np.exp(G) * dQbar
+                dG += dQbar * Qbar
+                dP = np.tril(dO @ D.T)
+                dq += np.einsum("ri,id,rid->rd", dP, K, E)
+                dk += np.einsum("ri,rd,rid->id", dP, Q, E)
+                tP = np.einsum("ri,rd,id,rid->rid", dP, Q, K, E)
+                dG += tP.sum(1)
+                dG -= tP.sum(0)
+                dKt = D @ dhn.T
+                dk += dKt * np.exp(G[n - 1][None, :] - G)
+                tK = dKt * Kt
+                dG -= tK
+                dG[n - 1] += tK.sum(0)
+                dG[n - 1] += gam * np.sum(h * dhn, axis=1)
+                dU, dW = dD, -dD @ h.T
+                dT = dU @ (bt[:, None] * V).T + dW @ (bt[:, None] * Kbar).T
+                TdU, TdW = Tm.T @ dU, Tm.T @ dW
+                out["dv"][b, c0:c1, h_] = bt[:, None] * TdU
+                dbeta = np.sum(TdU * V, axis=1) + np.sum(TdW * Kbar, axis=1)
+                dKbar = bt[:, None] * TdW
+                dk += np.exp(G) * dKbar
+                dG += dKbar * Kbar
+                dA = np.tril(-Tm.T @ dT @ Tm.T, -1)
+                dbeta += np.sum(dA * KK, axis=1)
+                dKK = bt[:, None] * dA
+                dk += np.einsum("ri,id,rid->rd", dKK, K, E)
+                dk += np.einsum("ri,rd,rid->id", dKK, K, E)
+                tA = np.einsum("ri,rd,id,rid->rid", dKK, K, K, E)
+                dG += tA.sum(1)
+                dG -= tA.sum(0)
+                out["dq"][b, c0:c1, h_] = dq
+                out["dk"][b, c0:c1, h_] = dk
+                out["dbeta"][b, c0:c1, h_] = dbeta
+                dgc = np.cumsum(dG[::-1], axis=0)[::-1]      # dg_t = sum_{r >= t} dG_r
+                if gate_kind == GATE_SCALAR:
+                    out["dg"][b, c0:c1, h_] = dgc.sum(1)
+                elif gate_kind == GATE_PER_DIM:
+                    out["dg"][b, c0:c1, h_] = dgc
+                dhn = dh
+            out["dS0"][b, h_] = dhn
+    return out
+
+
 def rel_err(x, ref) -> float:
     """max|x - ref| / max|ref| over the whole tensor (0 when both are zero)."""
     x = np.asarray(x, np.float64)
