@@ -27,7 +27,7 @@ EXPORTED = ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd_wor
             "gdn_read_device_status", "gdn_status_string", "gdn_abi_version",
             "gdn_kernel_launch_count", "gdn_chunk_fwd_kernel_name", "gdn_chunk_fwd_noalloc",
             "gdn_chunk_fwd_noalloc_scratch_bytes", "gdn_osdn_precondition", "gdn_chunk_fwd_wk",
-            "gdn_chunk_fwd_plan")
+            "gdn_chunk_fwd_plan", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes")
 
 _lib = None
 
@@ -79,6 +79,11 @@ def load() -> ctypes.CDLL:
     ip = ctypes.POINTER(ctypes.c_int)
     lib.gdn_chunk_fwd_plan.argtypes = [i, i, i, i, i, i, i, i, sz, ip, ip, ip]
     lib.gdn_chunk_fwd_plan.restype = i
+    lib.gdn_chunk_bwd.argtypes = [vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i,
+                                  i, i, i, i, i, vp, sz, vp]
+    lib.gdn_chunk_bwd.restype = i
+    lib.gdn_chunk_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    lib.gdn_chunk_bwd_workspace_bytes.restype = sz
     _lib = lib
     return lib
 
@@ -232,6 +237,60 @@ def gdn_osdn_precondition(k, beta, r, eta, d0, k_write, d_final, *, stream=None)
                                       _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_osdn_precondition")
+
+
+def gdn_chunk_bwd_workspace_bytes(B, T, H, Dk, Dv, chunk=64, dtype=torch.bfloat16,
+                                  gate_kind=GDN_GATE_SCALAR) -> int:
+    n = load().gdn_chunk_bwd_workspace_bytes(B, T, H, Dk, Dv, chunk, _dtype_code(dtype),
+                                             int(gate_kind))
+    if n == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_UNSUPPORTED, "gdn_chunk_bwd_workspace_bytes")
+    return n
+
+
+def gdn_chunk_bwd(q, k, v, beta, g, gate_kind, initial_state, d_o, d_final_state, dq, dk, dv,
+                  dbeta, dg, d_initial_state, *, chunk=64, workspace=None, stream=None) -> None:
+    """Enqueue the backward of the chunk forward: fp32 gradients dq, dk [B,T,H,Dk],
+    dv [B,T,H,Dv], dbeta, dg [B,T,H] (dg None without a gate), d_initial_state
+    [B,H,Dk,Dv] or None, from d_o [B,T,H,Dv] (dtype of q) and d_final_state."""
+    _check_contig(q=q, k=k, v=v, beta=beta, g=g, initial_state=initial_state, d_o=d_o,
+                  d_final_state=d_final_state, dq=dq, dk=dk, dv=dv, dbeta=dbeta, dg=dg,
+                  d_initial_state=d_initial_state)
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv), ("dbeta", dbeta), ("dg", dg),
+                    ("d_initial_state", d_initial_state), ("d_final_state", d_final_state),
+                    ("initial_state", initial_state)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().gdn_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), int(gate_kind),
+                              _ptr(initial_state), _ptr(d_o), _ptr(d_final_state), _ptr(dq),
+                              _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dg), _ptr(d_initial_state),
+                              B, T, H, Dk, Dv, chunk, _dtype_code(q.dtype), _ptr(workspace),
+                              ws_bytes, _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_bwd")
+
+
+def chunk_bwd(q, k, v, beta, g, initial_state, d_o, d_final_state=None, *, chunk=64,
+              stream=None):
+    """Allocate the gradients and the workspace with torch and run gdn_chunk_bwd.
+    Returns dict dq, dk, dv, dbeta, dg (None without a gate), d_initial_state."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    gate = GDN_GATE_NONE if g is None else GDN_GATE_SCALAR
+    dev = q.device
+    out = {"dq": torch.empty(B, T, H, Dk, device=dev), "dk": torch.empty(B, T, H, Dk, device=dev),
+           "dv": torch.empty(B, T, H, Dv, device=dev), "dbeta": torch.empty(B, T, H, device=dev),
+           "dg": None if g is None else torch.empty(B, T, H, device=dev),
+           "d_initial_state": torch.empty(B, H, Dk, Dv, device=dev)}
+    n = gdn_chunk_bwd_workspace_bytes(B, T, H, Dk, Dv, chunk, q.dtype, gate)
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    gdn_chunk_bwd(q, k, v, beta, g, gate, initial_state, d_o, d_final_state, out["dq"], out["dk"],
+                  out["dv"], out["dbeta"], out["dg"], out["d_initial_state"], chunk=chunk,
+                  workspace=ws, stream=stream)
+    return out
 
 
 def gdn_decode_step(q, k, v, beta, g, gate_kind, state, o, *, stream=None) -> None:

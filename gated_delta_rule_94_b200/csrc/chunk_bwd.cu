@@ -1,0 +1,616 @@
+// chunk_bwd.cu -- the backward of the chunkwise gated delta rule (scalar gate or
+// none; bf16 inputs, d_k = d_v = 128; fp32 gradients).
+//
+// The pages print no backward formula: the gradient is the derivative of the
+// chunkwise forward ("Moonshot AI's New Attention Architecture: Key
+// Innovations Explained", sec. 3; the WY factors of "OSDN: Improving Delta
+// Rule ...", sec. 2.1), taken by hand.  Per chunk, with h the entering state,
+//   A = StrictTril(diag(beta) Kbar Kbrev^T), T = (I + A)^-1,
+//   W = T diag(beta) Kbar, U = T diag(beta) V, D = U - W h,
+//   O = Qbar h + P D, P = Tril(Qbar Kbrev^T), h' = gamma h + Ktil^T D,
+// (Kbar = Gamma K, Kbrev = K / Gamma, Qbar = Gamma Q, Ktil = (gamma / Gamma) K)
+// and upstream dO, dh':
+//   dD = P^T dO + Ktil dh'
+//   dh = Qbar^T dO - W^T dD + gamma dh' = (gamma I + Phi^T) dh' + Qp^T dO,
+// Phi = -Ktil^T W and Qp = Qbar - P W being the forward's own step-image
+// operands: the adjoint state runs the transpose of the forward's affine chunk
+// map from the last chunk back.  Then, inside the chunk, dU = dD, dW = -dD h^T,
+// dT = dU (beta V)^T + dW (beta Kbar)^T, dA = StrictTril(-T^T dT T^T), and the
+// products through P, A, Kbar, Kbrev, Qbar, Ktil give dq, dk, dv, dbeta and
+// the log-decays' dG, whose reverse cumulative sum in the chunk is dg.
+//
+// Three launches after the forward (run in one wave, keeping every step image
+// and every chunk's entering state):
+//   adjoint_chain_kernel  one CTA per (batch, head), chunks from the last back:
+//                         stores the adjoint of each chunk's leaving state,
+//                         then dS0; fp32 on CUDA cores (the transition in bf16
+//                         as the forward's image holds it)
+//   chunk_bwd_kernel      one CTA per (batch, head, chunk): recomputes the
+//                         chunk's A, T, W, U, D and forms every gradient of the
+//                         chunk; fp32 on CUDA cores, dq and dk accumulated in
+//                         registers across the products that feed them
+#include <string.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace {
+
+using sm100::sw128_offset;
+
+constexpr int D = 128;
+constexpr int C = 64;
+
+__device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+// C[m][n] (+)= sum_k a(m, k) b(k, n) for an output tile of (RM * TR) x (RN * TC)
+// on TR x TC threads: thread (tr, tc) owns rows i * TR + tr and columns
+// j * TC + tc (strided, so that a warp's 16 column threads read 16 consecutive
+// words of a row of b).  acc is the thread's accumulator (kept by the caller
+// across calls when the same output is summed over several products).
+template <int RM, int RN, int TR, int TC, typename FA, typename FB>
+__device__ __forceinline__ void gemm_acc(float (&acc)[RM][RN], int K, int tid, FA a, FB b) {
+    const int tr = tid / TC, tc = tid % TC;
+#pragma unroll 2
+    for (int kk = 0; kk < K; ++kk) {
+        float av[RM], bv[RN];
+#pragma unroll
+        for (int i = 0; i < RM; ++i) av[i] = a(i * TR + tr, kk);
+#pragma unroll
+        for (int j = 0; j < RN; ++j) bv[j] = b(kk, j * TC + tc);
+#pragma unroll
+        for (int i = 0; i < RM; ++i)
+#pragma unroll
+            for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+}
+
+template <int RM, int RN>
+__device__ __forceinline__ void zero(float (&acc)[RM][RN]) {
+#pragma unroll
+    for (int i = 0; i < RM; ++i)
+#pragma unroll
+        for (int j = 0; j < RN; ++j) acc[i][j] = 0.f;
+}
+
+// ------------------------------------------------------------ adjoint chain
+constexpr int AC_THREADS = 512;
+constexpr int LDH = D + 4;   // fp32 row stride of dh in shared memory
+constexpr uint32_t AC_DH = 0;                               // dh [D][LDH] fp32
+constexpr uint32_t AC_PQ = AC_DH + D * LDH * 4;             // [Phi ; Qp] image, 2 x 24 KB
+constexpr uint32_t AC_DO = AC_PQ + 2 * kImgPQBlock;         // dO [64][128] bf16
+constexpr uint32_t AC_GAM = AC_DO + C * D * 2;              // gamma [128] fp32
+constexpr uint32_t AC_SMEM = AC_GAM + D * 4 + 1024;
+
+// One CTA per (batch, head).  dh starts at dS_final (or 0); for each chunk c
+// from the last: dh_all[c] = dh (the adjoint of the chunk's leaving state),
+// then dh = gamma dh + Phi^T dh + Qp^T dO_c.  The last dh is dS0.
+__global__ void __launch_bounds__(AC_THREADS)
+adjoint_chain_kernel(const BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    float* dh = reinterpret_cast<float*>(sm + AC_DH);
+    const uint8_t* pq = sm + AC_PQ;
+    const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(sm + AC_DO);
+    float* gam = reinterpret_cast<float*>(sm + AC_GAM);
+    const int tid = threadIdx.x, bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+    const int NC = (p.T + C - 1) / C;
+    for (int idx = tid; idx < D * D; idx += AC_THREADS)
+        dh[(idx >> 7) * LDH + (idx & 127)] = p.dS ? p.dS[(size_t)bh * D * D + idx] : 0.f;
+#pragma unroll 1
+    for (int c = NC - 1; c >= 0; --c) {
+        const uint8_t* img = p.images + ((size_t)bh * NC + c) * kImgBytes;
+        __syncthreads();   // dh of this chunk is complete
+        float* dst = p.dh_all + ((size_t)bh * NC + c) * D * D;
+        for (int idx = tid; idx < D * D; idx += AC_THREADS) dst[idx] = dh[(idx >> 7) * LDH + (idx & 127)];
+        for (int idx = tid; idx < 2 * (int)kImgPQBlock / 16; idx += AC_THREADS)
+            reinterpret_cast<uint4*>(sm + AC_PQ)[idx] = __ldcg(reinterpret_cast<const uint4*>(img + kImgPQ) + idx);
+        if (tid < D) gam[tid] = __ldcg(reinterpret_cast<const float*>(img + kImgGam) + tid);
+        for (int idx = tid; idx < C * D / 8; idx += AC_THREADS) {   // dO tile, 8 values a load
+            const int r = idx >> 4, j = idx & 15, t = c * C + r;
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (t < p.T) w = *reinterpret_cast<const uint4*>(
+                static_cast<const __nv_bfloat16*>(p.dO) + (((size_t)b * p.T + t) * p.H + h) * D + 8 * j);
+            reinterpret_cast<uint4*>(sm + AC_DO)[idx] = w;
+        }
+        __syncthreads();
+        // new dh[d'][v] = gamma_d' dh[d'][v] + sum_d Phi[d][d'] dh[d][v] + sum_r Qp[r][d'] dO[r][v]
+        float acc[4][8];
+        zero(acc);
+        gemm_acc<4, 8, 32, 16>(acc, D, tid,
+            [&](int dp, int d) {   // Phi^T: row d of Phi in the image, column d'
+                return bf(reinterpret_cast<const __nv_bfloat16*>(pq + (dp >> 6) * kImgPQBlock +
+                                                                 sw128_offset(d, dp & 63)));
+            },
+            [&](int d, int v) { return dh[d * LDH + v]; });
+        gemm_acc<4, 8, 32, 16>(acc, C, tid,
+            [&](int dp, int r) {   // Qp^T: row 128 + r of [Phi ; Qp], column d'
+                return bf(reinterpret_cast<const __nv_bfloat16*>(pq + (dp >> 6) * kImgPQBlock +
+                                                                 sw128_offset(128 + r, dp & 63)));
+            },
+            [&](int r, int v) { return __bfloat162float(dO[r * D + v]); });
+        const int tr = tid / 16, tc = tid % 16;
+        float keep[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int dp = i * 32 + tr, v = j * 16 + tc;
+                keep[i][j] = fmaf(gam[dp], dh[dp * LDH + v], acc[i][j]);
+            }
+        __syncthreads();   // every thread has read dh
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dh[(i * 32 + tr) * LDH + j * 16 + tc] = keep[i][j];
+    }
+    __syncthreads();
+    if (p.dS0)
+        for (int idx = tid; idx < D * D; idx += AC_THREADS)
+            p.dS0[(size_t)bh * D * D + idx] = dh[(idx >> 7) * LDH + (idx & 127)];
+}
+
+// --------------------------------------------------------- chunk backward
+constexpr int CB_THREADS = 256;
+constexpr int LDM = D + 4;   // fp32 row stride of [64][128] matrices
+constexpr int LDS = C + 1;   // fp32 row stride of [64][64] matrices
+constexpr uint32_t BW_Q = 0, BW_K = 16384, BW_V = 32768, BW_DO = 49152;   // bf16 [64][128]
+constexpr uint32_t BW_STAGE = 65536;                                      // [64][LDM] fp32
+constexpr uint32_t BW_P = BW_STAGE + C * LDM * 4;                         // [64][LDS]
+constexpr uint32_t BW_T = BW_P + C * LDS * 4;
+constexpr uint32_t BW_A = BW_T + C * LDS * 4;
+constexpr uint32_t BW_MD = BW_A + C * LDS * 4;                            // [64][LDM]
+constexpr uint32_t BW_MW = BW_MD + C * LDM * 4;
+constexpr uint32_t BW_VEC = BW_MW + C * LDM * 4;                          // vectors
+constexpr uint32_t BW_SMEM = BW_VEC + 8 * C * 4 + 1024;
+static_assert(BW_SMEM <= 232448, "chunk backward shared memory");
+
+template <bool GATED>
+__global__ void __launch_bounds__(CB_THREADS, 1)
+chunk_bwd_kernel(const BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const __nv_bfloat16* sQ = reinterpret_cast<const __nv_bfloat16*>(sm + BW_Q);
+    const __nv_bfloat16* sK = reinterpret_cast<const __nv_bfloat16*>(sm + BW_K);
+    const __nv_bfloat16* sV = reinterpret_cast<const __nv_bfloat16*>(sm + BW_V);
+    const __nv_bfloat16* sdO = reinterpret_cast<const __nv_bfloat16*>(sm + BW_DO);
+    float* stage = reinterpret_cast<float*>(sm + BW_STAGE);
+    float* sP = reinterpret_cast<float*>(sm + BW_P);
+    float* sT = reinterpret_cast<float*>(sm + BW_T);
+    float* sA = reinterpret_cast<float*>(sm + BW_A);
+    float* MD = reinterpret_cast<float*>(sm + BW_MD);
+    float* MW = reinterpret_cast<float*>(sm + BW_MW);
+    float* sG = reinterpret_cast<float*>(sm + BW_VEC);   // G (in-chunk log-decay cumsum)
+    float* sGam = sG + C;                                // Gamma = e^G
+    float* sBeta = sG + 2 * C;
+    float* sdG = sG + 3 * C;
+    float* sdB = sG + 4 * C;                             // dbeta
+    float* sRed = sG + 5 * C;                            // a reduction slot
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int NC = (p.T + C - 1) / C;
+    const int item = blockIdx.x, bh = item / NC, c = item % NC;
+    const int b = bh / p.H, h = bh % p.H;
+    auto tok = [&](int r) { return ((size_t)b * p.T + (size_t)c * C + r) * p.H + h; };
+    const int n = min(C, p.T - c * C);
+
+    // ---- inputs of the chunk (rows past the sequence end are zero)
+    for (int idx = tid; idx < 4 * C * D / 8; idx += CB_THREADS) {
+        const int m = idx / (C * D / 8), rem = idx % (C * D / 8), r = rem >> 4, j = rem & 15;
+        const __nv_bfloat16* src = m == 0 ? static_cast<const __nv_bfloat16*>(p.q)
+                                   : m == 1 ? static_cast<const __nv_bfloat16*>(p.k)
+                                   : m == 2 ? static_cast<const __nv_bfloat16*>(p.v)
+                                            : static_cast<const __nv_bfloat16*>(p.dO);
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (r < n) w = *reinterpret_cast<const uint4*>(src + tok(r) * D + 8 * j);
+        reinterpret_cast<uint4*>(sm + m * 16384)[rem] = w;
+    }
+    if (tid < C) {
+        float bt = 0.f, gv = 0.f;
+        if (tid < n) {
+            bt = __bfloat162float(static_cast<const __nv_bfloat16*>(p.beta)[tok(tid)]);
+            if (GATED) gv = __bfloat162float(static_cast<const __nv_bfloat16*>(p.g)[tok(tid)]);
+        }
+        sBeta[tid] = bt;
+        sG[tid] = gv;
+        sdG[tid] = 0.f;
+        sdB[tid] = 0.f;
+    }
+    __syncthreads();
+    if (warp == 0) {   // in-chunk cumulative sum of g (two tokens a lane)
+        const float a0 = sG[2 * lane], a1 = sG[2 * lane + 1];
+        float incl = a0 + a1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+        if (lane == 0) excl = 0.f;
+        sG[2 * lane] = excl + a0;
+        sG[2 * lane + 1] = incl;
+        sGam[2 * lane] = __expf(excl + a0);
+        sGam[2 * lane + 1] = __expf(incl);
+    }
+    __syncthreads();
+    const float Glast = sG[C - 1], gamma = sGam[C - 1];
+    auto E = [&](int r, int i) { return i <= r ? __expf(sG[r] - sG[i]) : 0.f; };
+    auto kf = [&](int r, int d) { return __bfloat162float(sK[r * D + d]); };
+    auto qf = [&](int r, int d) { return __bfloat162float(sQ[r * D + d]); };
+    auto vf = [&](int r, int d) { return __bfloat162float(sV[r * D + d]); };
+    auto of = [&](int r, int d) { return __bfloat162float(sdO[r * D + d]); };
+    const int tr = tid / 16, tc = tid % 16;   // gemm thread layout (16 x 16)
+
+    // ---- P = Tril(E (.) Q K^T), A = StrictTril(beta_r E (.) K K^T)
+    {
+        float aq[4][4], ak[4][4];
+        zero(aq);
+        zero(ak);
+        gemm_acc<4, 4, 16, 16>(aq, D, tid, qf, [&](int d, int i) { return kf(i, d); });
+        gemm_acc<4, 4, 16, 16>(ak, D, tid, kf, [&](int d, int i) { return kf(i, d); });
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = a * 16 + tr, i = j * 16 + tc;
+                const float e = E(r, i);
+                sP[r * LDS + i] = e * aq[a][j];
+                sA[r * LDS + i] = i < r ? sBeta[r] * e * ak[a][j] : 0.f;
+            }
+    }
+    __syncthreads();
+    // ---- T = (I + A)^-1 by forward substitution, one column a thread
+    if (tid < C) {
+        const int col = tid;
+        for (int r = 0; r < C; ++r) {
+            float x = (r == col) ? 1.f : 0.f;
+            if (r > col) {
+                for (int i = col; i < r; ++i) x = fmaf(-sA[r * LDS + i], sT[i * LDS + col], x);
+            }
+            sT[r * LDS + col] = r >= col ? x : 0.f;
+        }
+    }
+    __syncthreads();
+    // ---- W = T diag(beta Gamma) K, U = T diag(beta) V
+    {
+        float aw[4][8], au[4][8];
+        zero(aw);
+        zero(au);
+        gemm_acc<4, 8, 16, 16>(aw, C, tid, [&](int r, int i) { return sT[r * LDS + i] * sBeta[i] * sGam[i]; }, kf);
+        gemm_acc<4, 8, 16, 16>(au, C, tid, [&](int r, int i) { return sT[r * LDS + i] * sBeta[i]; }, vf);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = a * 16 + tr, v = j * 16 + tc;
+                MW[r * LDM + v] = aw[a][j];
+                MD[r * LDM + v] = au[a][j];
+            }
+    }
+    // ---- D = U - W h (h staged by halves of 64 rows)
+    const float* hsrc = p.h_all + ((size_t)bh * NC + c) * D * D;
+    const float* dhsrc = p.dh_all + ((size_t)bh * NC + c) * D * D;
+    auto stage_half = [&](const float* src, int half) {
+        __syncthreads();
+        for (int idx = tid; idx < C * D; idx += CB_THREADS)
+            stage[(idx >> 7) * LDM + (idx & 127)] = __ldcg(src + (size_t)half * C * D + idx);
+        __syncthreads();
+    };
+    {
+        float ad[4][8];
+        zero(ad);
+        for (int half = 0; half < 2; ++half) {
+            stage_half(hsrc, half);
+            gemm_acc<4, 8, 16, 16>(ad, C, tid, [&](int r, int d) { return MW[r * LDM + 64 * half + d]; },
+                                   [&](int d, int v) { return stage[d * LDM + v]; });
+        }
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = a * 16 + tr, v = j * 16 + tc;
+                MD[r * LDM + v] -= ad[a][j];
+            }
+    }
+    __syncthreads();
+    // dq and dk of this thread's 4 x 8 elements, summed over every product below
+    float dq[4][8], dk[4][8];
+    zero(dq);
+    zero(dk);
+    // ---- dD = P^T dO + Ktil dh' (into MW, W being dead), dKtil = D dh'^T,
+    //      <h, dh'>; dh' staged by halves of 64 rows (d)
+    {
+        float add[4][8];
+        zero(add);
+        gemm_acc<4, 8, 16, 16>(add, C, tid, [&](int i, int r) { return sP[r * LDS + i]; }, of);
+        float hdh = 0.f;
+        for (int half = 0; half < 2; ++half) {
+            stage_half(dhsrc, half);
+            // Ktil[i][d] = k_id e^(Glast - G_i), d in this half
+            gemm_acc<4, 8, 16, 16>(add, C, tid,
+                [&](int i, int d) { return kf(i, 64 * half + d) * __expf(Glast - sG[i]); },
+                [&](int d, int v) { return stage[d * LDM + v]; });
+            // dKtil[i][d] = sum_v D[i][v] dh'[d][v], for d = 64 half + 16 j' + tc (4 x 4 tile)
+            float akt[4][4];
+            zero(akt);
+            gemm_acc<4, 4, 16, 16>(akt, D, tid, [&](int i, int v) { return MD[i * LDM + v]; },
+                                   [&](int v, int d) { return stage[d * LDM + v]; });
+            for (int idx = tid; idx < C * D; idx += CB_THREADS)
+                hdh = fmaf(__ldcg(hsrc + (size_t)half * C * D + idx), stage[(idx >> 7) * LDM + (idx & 127)], hdh);
+            // dk_i += dKtil e^(Glast - G_i); dG_i -= <dKtil_i, Ktil_i>; dG_last += sum
+            // (the 4 x 4 tile covers columns 64 half + j * 16 + tc of the 4 x 8 layout:
+            //  column slot j' = 4 half + j)
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int i = a * 16 + tr;
+                const float f = __expf(Glast - sG[i]);
+                float part = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int d = 64 * half + j * 16 + tc;
+                    dk[a][4 * half + j] = fmaf(akt[a][j], f, dk[a][4 * half + j]);
+                    part = fmaf(akt[a][j], kf(i, d) * f, part);
+                }
+                atomicAdd(&sdG[i], -part);
+                atomicAdd(&sdG[C - 1], part);
+            }
+        }
+        // <h, dh'> over the block, into dG_last (gamma <h, dh'>)
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) hdh += __shfl_xor_sync(0xffffffffu, hdh, off);
+        if (lane == 0) atomicAdd(&sdG[C - 1], gamma * hdh);
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) MW[(a * 16 + tr) * LDM + j * 16 + tc] = add[a][j];   // dD
+    }
+    __syncthreads();
+    // ---- dP = Tril(dO D^T); tP = dP (.) P -> dG; dPE = dP (.) E into sP
+    {
+        float adp[4][4];
+        zero(adp);
+        gemm_acc<4, 4, 16, 16>(adp, D, tid, of, [&](int v, int i) { return MD[i * LDM + v]; });
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = a * 16 + tr, i = j * 16 + tc;
+                if (i <= r) {
+                    const float t = adp[a][j] * sP[r * LDS + i];
+                    atomicAdd(&sdG[r], t);
+                    atomicAdd(&sdG[i], -t);
+                }
+            }
+        __syncthreads();   // every thread has read P
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = a * 16 + tr, i = j * 16 + tc;
+                sP[r * LDS + i] = i <= r ? adp[a][j] * E(r, i) : 0.f;
+            }
+    }
+    __syncthreads();
+    // dq_r += sum_i dPE_ri k_i;  dk_i += sum_r dPE_ri q_r
+    gemm_acc<4, 8, 16, 16>(dq, C, tid, [&](int r, int i) { return sP[r * LDS + i]; }, kf);
+    gemm_acc<4, 8, 16, 16>(dk, C, tid, [&](int i, int r) { return sP[r * LDS + i]; }, qf);
+    // ---- dQbar = dO h^T -> dq += Gamma dQbar, dG_r += Gamma_r <dQbar_r, q_r>;
+    //      dW = -dD h^T (into MD, D being dead from here)
+    {
+        float aqb[4][8], awb[4][8];
+        zero(aqb);
+        zero(awb);
+        for (int half = 0; half < 2; ++half) {   // h by halves of 64 rows: columns d of the outputs
+            stage_half(hsrc, half);
+            float t1[4][4], t2[4][4];
+            zero(t1);
+            zero(t2);
+            gemm_acc<4, 4, 16, 16>(t1, D, tid, of, [&](int v, int d) { return stage[d * LDM + v]; });
+            gemm_acc<4, 4, 16, 16>(t2, D, tid, [&](int r, int v) { return MW[r * LDM + v]; },
+                                   [&](int v, int d) { return stage[d * LDM + v]; });
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    aqb[a][4 * half + j] = t1[a][j];
+                    awb[a][4 * half + j] = -t2[a][j];
+                }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int r = a * 16 + tr;
+            float part = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int d = (j & 3) * 16 + tc + 64 * (j >> 2);
+                dq[a][j] = fmaf(sGam[r], aqb[a][j], dq[a][j]);
+                part = fmaf(aqb[a][j], qf(r, d), part);
+                MD[r * LDM + d] = awb[a][j];   // dW
+            }
+            atomicAdd(&sdG[r], sGam[r] * part);
+        }
+    }
+    __syncthreads();
+    // ---- dv = beta T^T dU (dU = dD);  dbeta += <T^T dU, V> + <T^T dW, Kbar>;
+    //      dKbar = beta T^T dW -> dk += Gamma dKbar, dG += <dKbar, Kbar>
+    {
+        float tu[4][8], tw[4][8];
+        zero(tu);
+        zero(tw);
+        gemm_acc<4, 8, 16, 16>(tu, C, tid, [&](int r, int i) { return sT[i * LDS + r]; },
+                               [&](int i, int v) { return MW[i * LDM + v]; });
+        gemm_acc<4, 8, 16, 16>(tw, C, tid, [&](int r, int i) { return sT[i * LDS + r]; },
+                               [&](int i, int v) { return MD[i * LDM + v]; });
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int r = a * 16 + tr;
+            float db = 0.f, dg = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int v = j * 16 + tc;
+                if (r < n) p.dv[tok(r) * D + v] = sBeta[r] * tu[a][j];
+                const float kbar = sGam[r] * kf(r, v);
+                db = fmaf(tu[a][j], vf(r, v), db);
+                db = fmaf(tw[a][j], kbar, db);
+                const float dkb = sBeta[r] * tw[a][j];
+                dk[a][j] = fmaf(sGam[r], dkb, dk[a][j]);
+                dg = fmaf(dkb, kbar, dg);
+            }
+            atomicAdd(&sdB[r], db);
+            atomicAdd(&sdG[r], dg);
+        }
+    }
+    // ---- dT = dD (beta V)^T + dW (beta Kbar)^T  (into sA);  tmp = T^T dT  (into stage)
+    {
+        float adt[4][4];
+        zero(adt);
+        gemm_acc<4, 4, 16, 16>(adt, D, tid, [&](int r, int v) { return MW[r * LDM + v]; },
+                               [&](int v, int i) { return sBeta[i] * vf(i, v); });
+        gemm_acc<4, 4, 16, 16>(adt, D, tid, [&](int r, int d) { return MD[r * LDM + d]; },
+                               [&](int d, int i) { return sBeta[i] * sGam[i] * kf(i, d); });
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sA[(a * 16 + tr) * LDS + j * 16 + tc] = adt[a][j];
+    }
+    __syncthreads();
+    {
+        float at[4][4];
+        zero(at);
+        gemm_acc<4, 4, 16, 16>(at, C, tid, [&](int r, int i) { return sT[i * LDS + r]; },
+                               [&](int i, int j) { return sA[i * LDS + j]; });
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) stage[(a * 16 + tr) * LDS + j * 16 + tc] = at[a][j];
+    }
+    __syncthreads();
+    // ---- dA = StrictTril(-tmp T^T); dKK = beta_r dA; dbeta += sum_i dA KKE;
+    //      dKKE = dKK (.) E into sA; KKE recomputed (E (.) K K^T)
+    {
+        float ada[4][4], akk[4][4];
+        zero(ada);
+        zero(akk);
+        gemm_acc<4, 4, 16, 16>(ada, C, tid, [&](int r, int i) { return stage[r * LDS + i]; },
+                               [&](int i, int j) { return sT[j * LDS + i]; });
+        gemm_acc<4, 4, 16, 16>(akk, D, tid, kf, [&](int d, int i) { return kf(i, d); });
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int r = a * 16 + tr;
+            float db = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = j * 16 + tc;
+                float val = 0.f;
+                if (i < r) {
+                    const float dA = -ada[a][j];
+                    const float e = E(r, i);
+                    db = fmaf(dA, e * akk[a][j], db);
+                    const float dkke = sBeta[r] * dA * e;
+                    const float t = dkke * akk[a][j];
+                    atomicAdd(&sdG[r], t);
+                    atomicAdd(&sdG[i], -t);
+                    val = dkke;
+                }
+                sA[r * LDS + i] = val;
+            }
+            atomicAdd(&sdB[r], db);
+        }
+    }
+    __syncthreads();
+    // dk_r += sum_i dKKE_ri k_i;  dk_i += sum_r dKKE_ri k_r
+    gemm_acc<4, 8, 16, 16>(dk, C, tid, [&](int r, int i) { return sA[r * LDS + i]; }, kf);
+    gemm_acc<4, 8, 16, 16>(dk, C, tid, [&](int i, int r) { return sA[r * LDS + i]; }, kf);
+    __syncthreads();
+    // ---- outputs: dq, dk (this thread's elements), dbeta, dg (reverse cumsum of dG)
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int r = a * 16 + tr;
+        if (r < n) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                p.dq[tok(r) * D + j * 16 + tc] = dq[a][j];
+                p.dk[tok(r) * D + j * 16 + tc] = dk[a][j];
+            }
+        }
+    }
+    if (warp == 0) {   // dg_t = sum_{r >= t} dG_r: a reverse scan, two tokens a lane
+        const int r0 = C - 2 - 2 * lane;     // lane 0 takes the last two tokens
+        const float a1 = sdG[r0 + 1], a0 = sdG[r0];
+        float incl = a0 + a1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+        if (lane == 0) excl = 0.f;
+        const float g1 = excl + a1, g0 = incl;
+        if (GATED && p.dg) {
+            if (r0 + 1 < n) p.dg[tok(r0 + 1)] = g1;
+            if (r0 < n) p.dg[tok(r0)] = g0;
+        }
+        if (r0 + 1 < n) p.dbeta[tok(r0 + 1)] = sdB[r0 + 1];
+        if (r0 < n) p.dbeta[tok(r0)] = sdB[r0];
+    }
+    (void)sRed;
+}
+
+}  // namespace
+
+size_t chunk_bwd_workspace_bytes(int B, int T, int H) {
+    const int NC = (T + C - 1) / C;
+    if (NC == 0 || B == 0 || H == 0) return 0;
+    const size_t nbh = (size_t)B * H;
+    const size_t fwd = chunk_fwd_tc_capture_bytes(B, T, H);
+    const size_t o = ((size_t)B * T * H * D * 2 + 255) & ~(size_t)255;
+    return fwd + o + 2 * nbh * NC * D * D * sizeof(float);
+}
+
+cudaError_t launch_chunk_bwd(const ChunkParams& pf, const BwdParams& pb0, int gate,
+                             uint8_t* ws, size_t ws_bytes, cudaStream_t s, int* launches) {
+    *launches = 0;
+    const int NC = (pf.T + C - 1) / C;
+    const size_t nbh = (size_t)pf.B * pf.H;
+    const size_t fwd = chunk_fwd_tc_capture_bytes(pf.B, pf.T, pf.H);
+    const size_t o_bytes = ((size_t)pf.B * pf.T * pf.H * D * 2 + 255) & ~(size_t)255;
+    if (ws_bytes < chunk_bwd_workspace_bytes(pf.B, pf.T, pf.H)) return cudaErrorInvalidValue;
+    BwdParams pb = pb0;
+    pb.images = ws;
+    pb.h_all = reinterpret_cast<float*>(ws + fwd + o_bytes);
+    pb.dh_all = pb.h_all + nbh * NC * D * D;
+    // 1. the forward in one wave, keeping the images and every entering state
+    ChunkParams p = pf;
+    p.ws = ws;
+    p.o = ws + fwd;
+    p.s_out = nullptr;
+    int nf = 0;
+    cudaError_t e = launch_chunk_fwd_tc_capture(p, gate, fwd, pb.h_all, s, &nf);
+    *launches += nf;
+    if (e != cudaSuccess) return e;
+    // 2. the adjoint state, chunks from the last back
+    e = cudaFuncSetAttribute(adjoint_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)AC_SMEM);
+    if (e != cudaSuccess) return e;
+    e = launch_on(adjoint_chain_kernel, dim3((unsigned)nbh), dim3(AC_THREADS), AC_SMEM, s, pb);
+    if (e != cudaSuccess) return e;
+    ++*launches;
+    // 3. every chunk's gradients
+    auto kern = gate == kGateScalar ? chunk_bwd_kernel<true> : chunk_bwd_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BW_SMEM);
+    if (e != cudaSuccess) return e;
+    e = launch_on(kern, dim3((unsigned)(nbh * NC)), dim3(CB_THREADS), BW_SMEM, s, pb);
+    if (e != cudaSuccess) return e;
+    ++*launches;
+    return cudaSuccess;
+}
+
+}  // namespace gdn

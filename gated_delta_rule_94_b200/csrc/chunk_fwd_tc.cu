@@ -72,6 +72,8 @@ constexpr uint32_t IMG_UT = 73728;     // U^T  [128 v][64 i]     (K-major A)
 constexpr uint32_t IMG_GAM = 90112;    // gamma fp32 [128]
 constexpr uint32_t IMG_BYTES = 90624;
 constexpr uint32_t PQ_BLK = 24576;     // one K-block of [Phi ; Qp]
+static_assert(IMG_BYTES == kImgBytes && IMG_PQ == kImgPQ && PQ_BLK == kImgPQBlock &&
+              IMG_GAM == kImgGam, "image layout the backward reads");
 constexpr size_t WAVE_BYTES = size_t(160) << 20;  // cap of one wave's image buffer
 constexpr int PREP_SLOTS = 2 * 148;                // prep CTAs resident at once on a B200
 
@@ -1127,9 +1129,10 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 bulk_load_hint(sm + CH_GAM + (nl & 3) * 512, img(nl) + IMG_GAM, 512, &bars[CB_GAM0 + (nl & 3)], pol_once);
                 if (nl + 2 < NC) bulk_prefetch_l2(img(nl + 2), IMG_BYTES);
             }
-            if (nl >= 2 && outputs) {   // both products of chunk nl - 2 are done: its image is
-                             // dead in L2 (gamma of chunk nl - 3 too: the state pass has used
-                             // it); segment offsets and transitions leave them for the outputs
+            if (nl >= 2 && outputs && !p.h_all) {   // both products of chunk nl - 2 are done:
+                             // its image is dead in L2 (gamma of chunk nl - 3 too: the state
+                             // pass has used it); segment offsets and transitions leave them for
+                             // the outputs, and the backward's forward keeps them all
                 l2_discard(img(nl - 2), IMG_GAM, lane);
                 if (nl >= 3) l2_discard(img(nl - 3) + IMG_GAM, 512, lane);
             }
@@ -1288,6 +1291,12 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[CB_XFREE0 + ((nl - 1) & 1)]);
+            }
+            if (p.h_all) {   // keep the chunk's entering state (fp32) for the backward
+                float* dst = p.h_all + ((size_t)bh * p.nc_total + p.chunk0 + c0 + nl) * D * D +
+                             (size_t)(32 * c) * D + v;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) dst[(size_t)e * D] = hv[e];
             }
             {
                 float pk[16];
@@ -1471,6 +1480,21 @@ Plan plan_for(int B, int T, int H, int gate, size_t ws_bytes);
 
 }  // namespace
 
+size_t chunk_fwd_tc_capture_bytes(int B, int T, int H) {
+    const int NC = (T + C - 1) / C;
+    if (NC == 0 || B == 0 || H == 0) return 0;
+    return (size_t)B * H * NC * IMG_BYTES + counter_bytes(NC);
+}
+
+cudaError_t launch_chunk_fwd_tc_capture(const ChunkParams& p0, int gate, size_t ws_bytes,
+                                        float* h_all, cudaStream_t s, int* launches) {
+    ChunkParams p = p0;
+    p.h_all = h_all;
+    p.nc_total = (p0.T + C - 1) / C;
+    if (ws_bytes < chunk_fwd_tc_capture_bytes(p0.B, p0.T, p0.H)) return cudaErrorInvalidValue;
+    return launch_chunk_fwd_tc(p, gate, ws_bytes, s, launches);
+}
+
 bool chunk_fwd_tc_supported(int Dk, int Dv, int gate) {
     return Dk == D && Dv == D && (gate == kGateNone || gate == kGateScalar || gate == kGatePerDim);
 }
@@ -1566,7 +1590,13 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
     if (e != cudaSuccess) return e;
     const int NC = (p0.T + C - 1) / C;
     const int nbh = p0.B * p0.H;
-    const Plan pl = plan_for(p0.B, p0.T, p0.H, gate, ws_bytes);
+    Plan pl = plan_for(p0.B, p0.T, p0.H, gate, ws_bytes);
+    if (p0.h_all) {   // the backward's forward: one wave, every image kept, no segments
+        pl.cw = NC;
+        pl.nw = 1;
+        pl.use_seg = false;
+        pl.S_size = 1;
+    }
     const bool use_seg = pl.use_seg;
     const int cw = pl.cw;
     if (cw < 1) return cudaErrorInvalidValue;

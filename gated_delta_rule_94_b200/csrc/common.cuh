@@ -36,6 +36,9 @@ struct ChunkParams {
     int seg_mode;      // 1: offsets and transitions of every segment; 3: outputs of every segment
     int nseg, seg_len; // segments per (batch, head) in this wave, chunks per segment
     float* seg_h;      // [B*H][nseg][Dk][Dv] entering state of each segment (j >= 1)
+    // backward support: the entering state of every chunk, fp32 [B*H][nchunks][Dk][Dv]
+    float* h_all;      // null: not kept
+    int nc_total;      // chunks per (batch, head) of the whole sequence
 };
 
 // Phase 1 of the preconditioned delta rule (write keys kw = d (.) k).
@@ -47,6 +50,27 @@ struct OsdnParams {
     const float* d0;     // [B, H, Dk] initial preconditioner, or null (ones)
     float* d_out;        // [B, H, Dk] final preconditioner (output), or null
     float eta;           // step size of the preconditioner's gradient descent
+    int B, T, H;
+};
+
+// Backward of the chunk forward (scalar gate or none, bf16 inputs, d = 128).
+struct BwdParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* beta;
+    const void* g;       // [B, T, H] (scalar gate) or null
+    const void* dO;      // [B, T, H, Dv] upstream gradient of o, bf16
+    const float* dS;     // [B, H, Dk, Dv] upstream gradient of the final state, or null
+    float* dq;           // [B, T, H, Dk] fp32
+    float* dk;           // [B, T, H, Dk] fp32
+    float* dv;           // [B, T, H, Dv] fp32
+    float* dbeta;        // [B, T, H] fp32
+    float* dg;           // [B, T, H] fp32 (scalar gate) or null
+    float* dS0;          // [B, H, Dk, Dv] fp32 or null
+    const uint8_t* images;   // the forward's step images, [B*H][NC]
+    float* h_all;        // entering state of every chunk
+    float* dh_all;       // adjoint of every chunk's leaving state
     int B, T, H;
 };
 
@@ -104,4 +128,15 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, size_t ws_bytes,
 cudaError_t launch_decode_step(const DecodeParams& p, int Dk, int Dv, int gate, bool bf16,
                                cudaStream_t s);
 cudaError_t launch_osdn_precondition(const OsdnParams& p, int Dk, bool bf16, cudaStream_t s);
+// The forward in one wave, keeping every chunk's step image in ws (at offset 0,
+// [B*H][NC] images) and every chunk's entering state in h_all.  ws_bytes >=
+// chunk_fwd_tc_capture_bytes.
+size_t chunk_fwd_tc_capture_bytes(int B, int T, int H);
+cudaError_t launch_chunk_fwd_tc_capture(const ChunkParams& p, int gate, size_t ws_bytes,
+                                        float* h_all, cudaStream_t s, int* launches);
+size_t chunk_bwd_workspace_bytes(int B, int T, int H);
+cudaError_t launch_chunk_bwd(const ChunkParams& pf, const BwdParams& pb, int gate, uint8_t* ws,
+                             size_t ws_bytes, cudaStream_t s, int* launches);
+// Image layout facts the backward reads (bytes): the [Phi ; Qp] operand and gamma.
+constexpr uint32_t kImgBytes = 90624, kImgPQ = 0, kImgPQBlock = 24576, kImgGam = 90112;
 }  // namespace gdn

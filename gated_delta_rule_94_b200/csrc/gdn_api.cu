@@ -235,6 +235,79 @@ gdn_status gdn_chunk_fwd_wk(const void* q, const void* k, const void* k_write, c
                           B, T, H, Dk, Dv, chunk, dtype, workspace, workspace_bytes, stream);
 }
 
+size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk,
+                                     gdn_dtype dtype, gdn_gate gate_kind) {
+    if (B < 0 || T < 0 || H < 0) return (size_t)-1;
+    if (Dk != 128 || Dv != 128 || chunk != 64 || dtype != GDN_BF16) return (size_t)-1;
+    if (gate_kind != GDN_GATE_NONE && gate_kind != GDN_GATE_SCALAR) return (size_t)-1;
+    return gdn::chunk_bwd_workspace_bytes(B, T, H);
+}
+
+gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const void* beta,
+                         const void* g, gdn_gate gate_kind, const float* initial_state,
+                         const void* d_o, const float* d_final_state, float* dq, float* dk,
+                         float* dv, float* dbeta, float* dg, float* d_initial_state, int B,
+                         int T, int H, int Dk, int Dv, int chunk, gdn_dtype dtype,
+                         void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    if (B < 0 || T < 0 || H < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (gate_kind < GDN_GATE_NONE || gate_kind > GDN_GATE_PER_DIM) return GDN_ERR_INVALID_ARG;
+    if (Dk != 128 || Dv != 128 || chunk != 64 || dtype != GDN_BF16 ||
+        gate_kind == GDN_GATE_PER_DIM)
+        return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)B * T > INT32_MAX || (int64_t)B * H > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return GDN_OK;
+    const bool tokens = T > 0;
+    if (tokens && (!q || !k || !v || !beta || !d_o || !dq || !dk || !dv || !dbeta))
+        return GDN_ERR_INVALID_ARG;
+    if (tokens && (gate_kind == GDN_GATE_NONE) != (g == nullptr)) return GDN_ERR_INVALID_ARG;
+    if (tokens && gate_kind == GDN_GATE_SCALAR && !dg) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, beta, g, initial_state, d_o, d_final_state, dq, dk, dv,
+                          dbeta, dg, d_initial_state, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t ntok = (size_t)B * T * H;
+    const size_t sb = (size_t)B * H * Dk * Dv * sizeof(float);
+    // every output must be clear of every input and of the other outputs
+    const void* outs[] = {dq, dk, dv, dbeta, dg, d_initial_state};
+    const size_t outn[] = {ntok * Dk * 4, ntok * Dk * 4, ntok * Dv * 4, ntok * 4,
+                           g ? ntok * 4 : 0, sb};
+    const void* ins[] = {q, k, v, beta, g, initial_state, d_o, d_final_state};
+    const size_t inn[] = {ntok * Dk * 2, ntok * Dk * 2, ntok * Dv * 2, ntok * 2, ntok * 2, sb,
+                          ntok * Dv * 2, sb};
+    for (int i = 0; i < 6; ++i) {
+        for (int j = 0; j < 8; ++j)
+            if (overlaps(outs[i], outn[i], ins[j], inn[j])) return GDN_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 6; ++j)
+            if (overlaps(outs[i], outn[i], outs[j], outn[j])) return GDN_ERR_INVALID_ARG;
+    }
+    const size_t need = gdn::chunk_bwd_workspace_bytes(B, T, H);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) {   // no tokens: the final state is the initial state
+        if (!d_initial_state) return GDN_OK;
+        const cudaError_t e = d_final_state
+            ? cudaMemcpyAsync(d_initial_state, d_final_state, sb, cudaMemcpyDeviceToDevice, s)
+            : cudaMemsetAsync(d_initial_state, 0, sb, s);
+        return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    }
+    gdn::ChunkParams pf{};
+    pf.q = q; pf.k = k; pf.v = v; pf.beta = beta; pf.g = g;
+    pf.s0 = initial_state; pf.B = B; pf.T = T; pf.H = H; pf.Dk = Dk; pf.Dv = Dv;
+    pf.status = status_word_ptr();
+    if (!pf.status) return GDN_ERR_CUDA;
+    gdn::BwdParams pb{};
+    pb.q = q; pb.k = k; pb.v = v; pb.beta = beta; pb.g = g; pb.dO = d_o; pb.dS = d_final_state;
+    pb.dq = dq; pb.dk = dk; pb.dv = dv; pb.dbeta = dbeta; pb.dg = dg; pb.dS0 = d_initial_state;
+    pb.B = B; pb.T = T; pb.H = H;
+    int launches = 0;
+    const cudaError_t e = gdn::launch_chunk_bwd(pf, pb, gate_kind,
+                                                static_cast<uint8_t*>(workspace), workspace_bytes,
+                                                s, &launches);
+    g_launches.fetch_add((unsigned long long)launches);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status gdn_osdn_precondition(const void* k, const void* beta, const void* r, float eta,
                                  const float* d0, void* k_write, float* d_final, int B, int T,
                                  int H, int Dk, gdn_dtype dtype, gdn_stream_t stream) {

@@ -223,6 +223,43 @@ GDN_API gdn_status gdn_chunk_fwd_wk(const void* q, const void* k, const void* k_
                                     int chunk, gdn_dtype dtype, void* workspace,
                                     size_t workspace_bytes, gdn_stream_t stream);
 
+/*
+ * gdn_chunk_bwd -- gradients of gdn_chunk_fwd.  The pages print no backward;
+ * the gradient is the derivative of the chunkwise forward ("Moonshot AI's New
+ * Attention Architecture", sec. 3; the WY factors of "OSDN ...", sec. 2.1)
+ * taken by hand.  The adjoint state dh = (gamma I + Phi^T) dh' + Qp^T dO runs
+ * the transpose of the forward's affine chunk map from the last chunk back;
+ * inside each chunk the products through T = (I + A)^-1, W, U, P and the
+ * decays give the input gradients.  The call runs the forward again (one wave,
+ * keeping its step images and every chunk's entering state), the adjoint
+ * chain, then every chunk's gradients.
+ *
+ *   q, k, v, beta, g, gate_kind, initial_state   the forward's inputs (as
+ *                 gdn_chunk_fwd; GDN_BF16, Dk = Dv = 128, gate none or scalar)
+ *   d_o           [B, T, H, Dv] bf16, dL/do
+ *   d_final_state [B, H, Dk, Dv] fp32, dL/dS_final, or NULL (zero)
+ *   dq, dk        [B, T, H, Dk] fp32 (outputs)
+ *   dv            [B, T, H, Dv] fp32 (output)
+ *   dbeta         [B, T, H] fp32 (output)
+ *   dg            [B, T, H] fp32 (output; NULL iff gate_kind == GDN_GATE_NONE)
+ *   d_initial_state [B, H, Dk, Dv] fp32 (output) or NULL
+ *   workspace     at least gdn_chunk_bwd_workspace_bytes bytes
+ * Outputs must not overlap the inputs or one another.  Anything else than
+ * bf16, d = 128 and a scalar gate or none is GDN_ERR_UNSUPPORTED.
+ */
+GDN_API gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const void* beta,
+                                 const void* g, gdn_gate gate_kind, const float* initial_state,
+                                 const void* d_o, const float* d_final_state, float* dq,
+                                 float* dk, float* dv, float* dbeta, float* dg,
+                                 float* d_initial_state, int B, int T, int H, int Dk, int Dv,
+                                 int chunk, gdn_dtype dtype, void* workspace,
+                                 size_t workspace_bytes, gdn_stream_t stream);
+
+/* Workspace of gdn_chunk_bwd (the forward's images, its output, the entering
+ * state and the adjoint of every chunk); (size_t)-1 for an unsupported shape. */
+GDN_API size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk,
+                                             gdn_dtype dtype, gdn_gate gate_kind);
+
 /* Synchronizes `stream`, then reads and clears the library's device status
  * word.  Returns GDN_ERR_TIMEOUT if any kernel since the last call gave up a
  * bounded wait, GDN_ERR_CUDA if the stream reports an error, else GDN_OK.

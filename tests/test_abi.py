@@ -233,3 +233,43 @@ def test_osdn_precondition_noop_sizes():
     assert osdn_call(B=0) == _lib.GDN_OK
     assert osdn_call(H=0, k=None, kw=None) == _lib.GDN_OK
     assert osdn_call(T=0, k=None, kw=None, beta=None) == _lib.GDN_OK   # nothing to write
+
+
+# -------------------------------------------------------------------- backward
+def bwd_call(**over):
+    args = dict(q=A, k=A, v=A, beta=A, g=A, gate=1, s0=None, do_=A, ds=None, dq=A * 64,
+                dk=A * 128, dv=A * 192, dbeta=A * 256, dg=A * 320, ds0=None, B=1, T=64, H=1,
+                Dk=128, Dv=128, chunk=64, dtype=0, ws=None, ws_bytes=0, stream=None)
+    args.update(over)
+    a = args
+    return _lib.load().gdn_chunk_bwd(a["q"], a["k"], a["v"], a["beta"], a["g"], a["gate"], a["s0"],
+                                     a["do_"], a["ds"], a["dq"], a["dk"], a["dv"], a["dbeta"],
+                                     a["dg"], a["ds0"], a["B"], a["T"], a["H"], a["Dk"], a["Dv"],
+                                     a["chunk"], a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(gate=2), _lib.GDN_ERR_UNSUPPORTED),                 # per-dimension gate: not built
+    (dict(dtype=1), _lib.GDN_ERR_UNSUPPORTED),
+    (dict(Dk=64, Dv=64), _lib.GDN_ERR_UNSUPPORTED),
+    (dict(dq=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(dg=None), _lib.GDN_ERR_INVALID_ARG),                # scalar gate needs dg
+    (dict(g=None), _lib.GDN_ERR_INVALID_ARG),
+    (dict(dq=MIS), _lib.GDN_ERR_INVALID_ARG),
+    (dict(dq=A), _lib.GDN_ERR_INVALID_ARG),                   # output over an input
+    (dict(dk=A * 64), _lib.GDN_ERR_INVALID_ARG),              # two outputs overlap
+    (dict(), _lib.GDN_ERR_WORKSPACE),
+    (dict(gate=3), _lib.GDN_ERR_INVALID_ARG),
+])
+def test_chunk_bwd_argument_errors(over, code):
+    assert bwd_call(**over) == code
+
+
+def test_chunk_bwd_workspace_bytes():
+    lib = _lib.load()
+    bad = ctypes.c_size_t(-1).value
+    n = lib.gdn_chunk_bwd_workspace_bytes(4, 2048, 16, 128, 128, 64, 0, 1)
+    assert n != bad and n > 2 * 64 * 32 * 128 * 128 * 4
+    assert lib.gdn_chunk_bwd_workspace_bytes(4, 2048, 16, 128, 128, 64, 0, 2) == bad
+    assert lib.gdn_chunk_bwd_workspace_bytes(4, 2048, 16, 64, 64, 64, 0, 1) == bad
+    assert lib.gdn_chunk_bwd_workspace_bytes(4, 0, 16, 128, 128, 64, 0, 1) == 0
