@@ -66,6 +66,20 @@ __device__ __forceinline__ void gemm_acc(float (&acc)[RM][RN], int K, int tid, F
     }
 }
 
+// Reductions before a shared-memory atomic, for the 16 x 16 thread layout
+// (thread = 16 row threads x 16 column threads; lanes 0-15 of a warp share a
+// row thread, lanes 16-31 the next): the sum over the 16 lanes of a row, added
+// by one lane; the sum over the two row threads of a warp, added by one lane.
+__device__ __forceinline__ void row_add(float* dst, float val, int lane) {
+#pragma unroll
+    for (int off = 1; off < 16; off <<= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
+    if ((lane & 15) == 0) atomicAdd(dst, val);
+}
+__device__ __forceinline__ void col_add(float* dst, float val, int lane) {
+    val += __shfl_xor_sync(0xffffffffu, val, 16);
+    if (lane < 16) atomicAdd(dst, val);
+}
+
 template <int RM, int RN>
 __device__ __forceinline__ void zero(float (&acc)[RM][RN]) {
 #pragma unroll
@@ -156,8 +170,12 @@ adjoint_chain_kernel(const BwdParams p) {
 constexpr int CB_THREADS = 256;
 constexpr int LDM = D + 4;   // fp32 row stride of [64][128] matrices
 constexpr int LDS = C + 1;   // fp32 row stride of [64][64] matrices
-constexpr uint32_t BW_Q = 0, BW_K = 16384, BW_V = 32768, BW_DO = 49152;   // bf16 [64][128]
-constexpr uint32_t BW_STAGE = 65536;                                      // [64][LDM] fp32
+// bf16 [64][LDB] tiles: rows padded to 136 elements (272 B), so that reading a
+// column (16 rows, one element each) touches 8 banks instead of one
+constexpr int LDB = D + 8;
+constexpr uint32_t BW_TILE = C * LDB * 2;
+constexpr uint32_t BW_Q = 0, BW_K = BW_TILE, BW_V = 2 * BW_TILE, BW_DO = 3 * BW_TILE;
+constexpr uint32_t BW_STAGE = 4 * BW_TILE;                                // [64][LDM] fp32
 constexpr uint32_t BW_P = BW_STAGE + C * LDM * 4;                         // [64][LDS]
 constexpr uint32_t BW_T = BW_P + C * LDS * 4;
 constexpr uint32_t BW_A = BW_T + C * LDS * 4;
@@ -206,7 +224,7 @@ chunk_bwd_kernel(const BwdParams p) {
                                             : static_cast<const __nv_bfloat16*>(p.dO);
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
         if (r < n) w = *reinterpret_cast<const uint4*>(src + tok(r) * D + 8 * j);
-        reinterpret_cast<uint4*>(sm + m * 16384)[rem] = w;
+        *reinterpret_cast<uint4*>(sm + m * BW_TILE + r * LDB * 2 + 16 * j) = w;
     }
     if (tid < C) {
         float bt = 0.f, gv = 0.f;
@@ -238,10 +256,10 @@ chunk_bwd_kernel(const BwdParams p) {
     __syncthreads();
     const float Glast = sG[C - 1], gamma = sGam[C - 1];
     auto E = [&](int r, int i) { return i <= r ? __expf(sG[r] - sG[i]) : 0.f; };
-    auto kf = [&](int r, int d) { return __bfloat162float(sK[r * D + d]); };
-    auto qf = [&](int r, int d) { return __bfloat162float(sQ[r * D + d]); };
-    auto vf = [&](int r, int d) { return __bfloat162float(sV[r * D + d]); };
-    auto of = [&](int r, int d) { return __bfloat162float(sdO[r * D + d]); };
+    auto kf = [&](int r, int d) { return __bfloat162float(sK[r * LDB + d]); };
+    auto qf = [&](int r, int d) { return __bfloat162float(sQ[r * LDB + d]); };
+    auto vf = [&](int r, int d) { return __bfloat162float(sV[r * LDB + d]); };
+    auto of = [&](int r, int d) { return __bfloat162float(sdO[r * LDB + d]); };
     const int tr = tid / 16, tc = tid % 16;   // gemm thread layout (16 x 16)
 
     // ---- P = Tril(E (.) Q K^T), A = StrictTril(beta_r E (.) K K^T)
@@ -327,7 +345,7 @@ chunk_bwd_kernel(const BwdParams p) {
         float add[4][8];
         zero(add);
         gemm_acc<4, 8, 16, 16>(add, C, tid, [&](int i, int r) { return sP[r * LDS + i]; }, of);
-        float hdh = 0.f;
+        float hdh = 0.f, lastsum = 0.f;   // <h, dh'>; the K~ terms of dG_last
         for (int half = 0; half < 2; ++half) {
             stage_half(dhsrc, half);
             // Ktil[i][d] = k_id e^(Glast - G_i), d in this half
@@ -355,14 +373,15 @@ chunk_bwd_kernel(const BwdParams p) {
                     dk[a][4 * half + j] = fmaf(akt[a][j], f, dk[a][4 * half + j]);
                     part = fmaf(akt[a][j], kf(i, d) * f, part);
                 }
-                atomicAdd(&sdG[i], -part);
-                atomicAdd(&sdG[C - 1], part);
+                row_add(&sdG[i], -part, lane);
+                lastsum += part;
             }
         }
         // <h, dh'> over the block, into dG_last (gamma <h, dh'>)
+        float last = gamma * hdh + lastsum;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) hdh += __shfl_xor_sync(0xffffffffu, hdh, off);
-        if (lane == 0) atomicAdd(&sdG[C - 1], gamma * hdh);
+        for (int off = 16; off > 0; off >>= 1) last += __shfl_xor_sync(0xffffffffu, last, off);
+        if (lane == 0) atomicAdd(&sdG[C - 1], last);
         __syncthreads();
 #pragma unroll
         for (int a = 0; a < 4; ++a)
@@ -375,17 +394,22 @@ chunk_bwd_kernel(const BwdParams p) {
         float adp[4][4];
         zero(adp);
         gemm_acc<4, 4, 16, 16>(adp, D, tid, of, [&](int v, int i) { return MD[i * LDM + v]; });
+        float colp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < 4; ++a) {
+            const int r = a * 16 + tr;
+            float rowp = 0.f;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int r = a * 16 + tr, i = j * 16 + tc;
-                if (i <= r) {
-                    const float t = adp[a][j] * sP[r * LDS + i];
-                    atomicAdd(&sdG[r], t);
-                    atomicAdd(&sdG[i], -t);
-                }
+                const int i = j * 16 + tc;
+                const float t = i <= r ? adp[a][j] * sP[r * LDS + i] : 0.f;
+                rowp += t;
+                colp[j] += t;
             }
+            row_add(&sdG[r], rowp, lane);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) col_add(&sdG[j * 16 + tc], -colp[j], lane);
         __syncthreads();   // every thread has read P
 #pragma unroll
         for (int a = 0; a < 4; ++a)
@@ -433,7 +457,7 @@ chunk_bwd_kernel(const BwdParams p) {
                 part = fmaf(aqb[a][j], qf(r, d), part);
                 MD[r * LDM + d] = awb[a][j];   // dW
             }
-            atomicAdd(&sdG[r], sGam[r] * part);
+            row_add(&sdG[r], sGam[r] * part, lane);
         }
     }
     __syncthreads();
@@ -462,8 +486,8 @@ chunk_bwd_kernel(const BwdParams p) {
                 dk[a][j] = fmaf(sGam[r], dkb, dk[a][j]);
                 dg = fmaf(dkb, kbar, dg);
             }
-            atomicAdd(&sdB[r], db);
-            atomicAdd(&sdG[r], dg);
+            row_add(&sdB[r], db, lane);
+            row_add(&sdG[r], dg, lane);
         }
     }
     // ---- dT = dD (beta V)^T + dW (beta Kbar)^T  (into sA);  tmp = T^T dT  (into stage)
@@ -502,10 +526,11 @@ chunk_bwd_kernel(const BwdParams p) {
                                [&](int i, int j) { return sT[j * LDS + i]; });
         gemm_acc<4, 4, 16, 16>(akk, D, tid, kf, [&](int d, int i) { return kf(i, d); });
         __syncthreads();
+        float cola[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
             const int r = a * 16 + tr;
-            float db = 0.f;
+            float db = 0.f, rowa = 0.f;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int i = j * 16 + tc;
@@ -516,14 +541,17 @@ chunk_bwd_kernel(const BwdParams p) {
                     db = fmaf(dA, e * akk[a][j], db);
                     const float dkke = sBeta[r] * dA * e;
                     const float t = dkke * akk[a][j];
-                    atomicAdd(&sdG[r], t);
-                    atomicAdd(&sdG[i], -t);
+                    rowa += t;
+                    cola[j] += t;
                     val = dkke;
                 }
                 sA[r * LDS + i] = val;
             }
-            atomicAdd(&sdB[r], db);
+            row_add(&sdB[r], db, lane);
+            row_add(&sdG[r], rowa, lane);
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) col_add(&sdG[j * 16 + tc], -cola[j], lane);
     }
     __syncthreads();
     // dk_r += sum_i dKKE_ri k_i;  dk_i += sum_r dKKE_ri k_r
