@@ -303,14 +303,14 @@ constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;
 constexpr uint32_t PD_KT = P_KT;             // per-dimension gate: g bf16 (TMA), then K~
 // staging of the step image for its bulk stores (buffers dead by then)
 constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
-constexpr uint32_t S_QPT = P_WUT + 16384;    // Qp [64 r][128 d] as two [64][64] blocks, over the
-                                             // U^T rows of [W^T; U^T]: dead once U^T's image
-                                             // store has read them
+constexpr uint32_t S_QPT = P_KT;             // Qp [64 r][128 d] as two [64][64] blocks, over
+                                             // K~^T: dead once the K~^T W product is done and
+                                             // K~^T's image store (the oldest) has read it
 constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (exact fallback; aliases A / T)
 static_assert(P_TF + 64 * LDF * 4 <= P_KT, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_KT, "[W^T; U^T] tile");
 static_assert(P_TW + 8192 <= P_TF && P_KT + 16384 <= P_P, "T_u / T_w over A, K~ tile");
-static_assert(S_PHI + 32768 <= S_QPT && S_QPT + 16384 <= P_KT, "staging clear of each other and K~^T");
+static_assert(S_PHI + 32768 <= P_WUT + 16384 && S_QPT + 16384 <= P_P, "staging clear of the U^T rows and P");
 static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
 static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
 
@@ -389,16 +389,17 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         for (int blk = 0; blk < 2; ++blk) {
             tma_load_3d_hint(sm + P_KQ + blk * 16384, &maps.k, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
             tma_load_3d_hint(sm + P_KQ + blk * 16384 + 8192, &maps.q, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
-            if constexpr (PD)
-                tma_load_3d_hint(sm + PD_KT + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
         }
     };
     // the rest of an item's tiles, into slots that are free only once the
-    // previous item has finished: the write key, V
+    // previous item has finished: g (per-dimension gate; its slot held the
+    // previous item's Qp staging), the write key, V
     auto issue_rest = [&](int item) {
         int b, h, n;
         coords(item, b, h, n);
         for (int blk = 0; blk < 2; ++blk) {
+            if constexpr (PD)
+                tma_load_3d_hint(sm + PD_KT + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
             if constexpr (WK)
                 tma_load_3d_hint(sm + P_V + blk * 8192, &maps.kw, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
         }
@@ -464,11 +465,15 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             }
         }
     };
+    if (tid == 0) bulk_wait_read();   // the previous item's Qp staging (its g slot, K~^T) is read
     if (warp == 2 || warp == 3) {   // beta and g (fetched during the previous item)
         gbuf[tid - 64] = ng;
         sBeta[tid - 64] = nb;
     }
     __syncthreads();
+    // the next item, taken now so that the global atomic is off the path; its
+    // K and Q are issued once this item's last readers of both are done
+    if (tid == 64) s_item[(it + 1) & 1] = (int)atomicAdd(p.counter, 1u);
 
     bool exact = false;
     if constexpr (!PD) {
@@ -487,6 +492,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                 atomicOr(p.status, kStatusTimeout);
             }
         }
+        // the previous item's second Phi half (over the A scratch) is read
+        if (tid == 128) bulk_wait_read();
         __syncthreads();
     } else {
         wait(0, ph);
@@ -535,6 +542,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                 wide |= g0 - cv[e] >= 80.f;
             }
         }
+        // the previous item's second Phi half (over the A / G scratch) is read
+        if (tid == 128) bulk_wait_read();
         exact = __syncthreads_or(wide) != 0;
         if (seg == 15) {
 #pragma unroll
@@ -855,14 +864,12 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         mma_commit(&bars[3]);
     }
     wait(3, ph);
-    // The U^T rows become the Qp staging: U^T's image store must have read them
-    // (and K~^T's, whose slot takes the next g tile).  The last readers of K, Q
-    // and K~^T (the W^T, Q^T E and K~^T W products) are done: the next item's
-    // K, Q (and g) can land now.
+    // The K~^T tile becomes the Qp staging: its image store (the oldest of this
+    // item's groups) must have read it.  The last readers of K and Q (the W^T
+    // and Q^T E products) are done: the next item's K and Q can land now.
     if (tid == 0) {
-        bulk_wait_read();
-        const int nx = (int)atomicAdd(p.counter, 1u);
-        s_item[(it + 1) & 1] = nx;
+        bulk_wait_read_all_but_one();
+        const int nx = s_item[(it + 1) & 1];
         if (nx < nitems) {
             fence_async_smem();
             issue_kq(nx);
@@ -919,9 +926,10 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             bulk_store_hint(img + IMG_PQ + PQ_BLK + 16384, sm + S_QPT + 8192, 8192, pol_img);
             bulk_commit();
         }
-        bulk_wait_read();
+        // Phi's first half (over the V slot, which the next item loads first) is
+        // read; Qp's staging is waited for at the next item's top
+        bulk_wait_read_all_but_one();
     }
-    if (tid == 128) bulk_wait_read();   // its half of Phi
     tc_fence_before();
     if (__syncthreads_or(failed)) {
         // a bounded wait gave up: wait (bounded) for this item's loads and the
@@ -938,6 +946,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     tc_fence_after();
     item = next_item;
     }   // items
+    if (tid == 0 || tid == 128) bulk_wait_all();   // the last item's stores are complete
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
