@@ -119,6 +119,9 @@ __device__ __forceinline__ void l2_discard(const void* p, uint32_t bytes, int la
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 template <int N>
 __device__ __forceinline__ void ld_cols(uint32_t addr, float (&v)[N]) {
@@ -311,6 +314,7 @@ static_assert(P_TF + 64 * LDF * 4 <= P_KT, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_KT, "[W^T; U^T] tile");
 static_assert(P_TW + 8192 <= P_TF && P_KT + 16384 <= P_P, "T_u / T_w over A, K~ tile");
 static_assert(S_PHI + 32768 <= P_WUT + 16384 && S_QPT + 16384 <= P_P, "staging clear of the U^T rows and P");
+static_assert(P_P == P_KT + 16384, "P right after K~^T: rows 64..127 of the A operand of P W");
 static_assert(64 * LDG * 4 <= 2 * 64 * LDF * 4, "G fits in the A / T scratch");
 static_assert(2 * (P_SMEM + 1024) <= 233472, "two prep CTAs per SM");
 
@@ -319,9 +323,7 @@ constexpr uint32_t TM_S = 0;       // [K;Q] K^T, 64 columns
 constexpr uint32_t TM_WT = 64;     // W^T, lanes d, 64 columns r
 constexpr uint32_t TM_UT = 128;    // U^T, lanes v, 64 columns r
 constexpr uint32_t TM_FP = 0;      // K~^T W, lanes d, 128 columns d'   (after S, W^T, U^T are read)
-constexpr uint32_t TM_PWT = 128;   // W^T P^T, lanes d, 64 columns r
-constexpr uint32_t TM_QE = 192;    // Q^T E = (Q e^G)^T, lanes d, 64 columns r
-constexpr uint32_t P_E = 32768;    // E_hi, E_lo bf16 [64 r][64 j] over the dead V tile
+constexpr uint32_t TM_PW = 128;    // P W, lanes 64 + r, 128 columns d (lanes 0..63 unused)
 
 // One CTA per (batch, head, chunk) of the wave: every state-independent part
 // of the chunk, written to the workspace as the chunk's step image.
@@ -817,24 +819,6 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) st_row_chunk(sm + P_WUT, (warp < 4 ? 0 : 128) + row, j, v + 8 * j, sc);
     }
-    {   // E = diag(e^(G_r)) split as E_hi + E_lo (bf16 each, so that Q^T E_hi + Q^T E_lo
-        // accumulated in fp32 gives (Q e^G)^T to about 2^-16); identity for the
-        // per-dimension gate (its Q tile already carries the decay) and for no gate.
-        // Each thread zeroes four 16-byte chunks of the two tiles, then row r's
-        // diagonal element is set by the thread owning it.
-        const float* sGam = gbuf + 64;
-        for (int idx = tid; idx < 1024; idx += NPR)
-            *reinterpret_cast<uint4*>(sm + P_E + idx * 16) = make_uint4(0u, 0u, 0u, 0u);
-        __syncwarp();
-        named_bar(4, NPR);
-        if (tid < 64) {
-            const float x = (GATE == kGateScalar) ? sGam[tid] : 1.f;
-            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-            *reinterpret_cast<__nv_bfloat16*>(sm + P_E + sw128_offset(tid, tid)) = hi;
-            *reinterpret_cast<__nv_bfloat16*>(sm + P_E + 8192 + sw128_offset(tid, tid)) = lo;
-        }
-    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -851,35 +835,40 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         for (int k = 0; k < 4; ++k)
             mma_bf16(tmem + TM_FP, sdesc_sw128(kt + k * 32, 16, 1024),
                      sdesc_sw128(sb + P_WUT + k * 32, 16, 1024), id1, k > 0);
-        const uint32_t id2 = idesc_bf16_f32(128, 64, false, false);   // W^T P^T
+        // P W (B = W^T as for K~^T W): the A operand starts at row 64 of K~^T, so
+        // that its rows 64..127 are P (the tile after K~^T); lanes 0..63 of the
+        // result are not used
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem + TM_PWT, sdesc_sw128(sb + P_WUT + k * 32, 16, 1024),
-                     sdesc_sw128(sb + P_P + k * 32, 16, 1024), id2, k > 0);
-        const uint32_t id3 = idesc_bf16_f32(128, 64, true, false);    // Q^T (E_hi + E_lo)
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-            mma_bf16(tmem + TM_QE, sdesc_sw128(sb + P_KQ + 8192 + (k & 3) * 2048, 16384, 1024),
-                     sdesc_sw128(sb + P_E + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), id3, k > 0);
+            mma_bf16(tmem + TM_PW, sdesc_sw128(kt + 8192 + k * 32, 16, 1024),
+                     sdesc_sw128(sb + P_WUT + k * 32, 16, 1024), id1, k > 0);
         mma_commit(&bars[3]);
     }
     wait(3, ph);
-    // The K~^T tile becomes the Qp staging: its image store (the oldest of this
-    // item's groups) must have read it.  The last readers of K and Q (the W^T
-    // and Q^T E products) are done: the next item's K and Q can land now.
+    // Row r of Q (its half hh of the columns) into the registers of the thread
+    // that forms row r of Qp (lanes 64 + r), so that the next item's K and Q
+    // can land once every thread has passed the barrier below.  The K~^T tile
+    // becomes the Qp staging: its image store (the oldest of this item's
+    // groups) must have read it.
+    const int row = (warp & 3) * 32 + lane;
+    uint4 qrow[8];
+    if (row >= 64) {
+        const uint8_t* qb = sm + P_KQ + 8192 + (warp >> 2) * 16384;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) qrow[j] = *reinterpret_cast<const uint4*>(qb + sw128_offset(row - 64, 8 * j));
+    }
+    if (tid == 0) bulk_wait_read_all_but_one();
+    tc_fence_after();
+    __syncthreads();
     if (tid == 0) {
-        bulk_wait_read_all_but_one();
         const int nx = s_item[(it + 1) & 1];
         if (nx < nitems) {
             fence_async_smem();
             issue_kq(nx);
         }
     }
-    tc_fence_after();
-    __syncthreads();
     const int next_item = s_item[(it + 1) & 1];
     if ((warp == 2 || warp == 3) && next_item < nitems) fetch_bg(next_item);
-    const int row = (warp & 3) * 32 + lane;
     {   // Phi = -K~^T W, row d: warps 0-3 columns 0-63, warps 4-7 columns 64-127;
         // each half stored as soon as it is staged
         const int hh = warp >> 2;
@@ -895,27 +884,29 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             bulk_commit();
         }
     }
-    {   // Qp = Q e^G - P W, stored K-major [r][d] (two [64][64] blocks) from row d of
-        // W^T P^T: warps 0-3 tokens r 0-31, warps 4-7 r 32-63; the 32 lanes of a
-        // warp write 32 consecutive d of one row r (one conflict-free wavefront)
-        const int hh = warp >> 2;
-        float v[32], qv[32];
-        ld_cols<32>(tmem + TM_PWT + lane_off + 32 * hh, v);
-        ld_cols<32>(tmem + TM_QE + lane_off + 32 * hh, qv);
-        const int d = row;
-        const float qs = PD ? sRef[d] : 1.f;
-        uint8_t* qblk = sm + S_QPT + (d >> 6) * 8192;
+    if (warp >= 4 && !failed) {   // gamma_d, d = row
+        float gam;
+        if constexpr (PD) gam = sGamD[row];
+        else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
+        reinterpret_cast<float*>(img + IMG_GAM)[row] = gam;
+    }
+    if (row >= 64) {   // Qp = Q e^G - P W, row r, columns 64 hh ..: K-major [r][d] (two
+                       // [64][64] blocks), 16-byte chunks
+        const int hh = warp >> 2, r = row - 64;
+        float v[64];
+        ld_cols<64>(tmem + TM_PW + lane_off + 64 * hh, v);
+        const float er = gbuf[64 + r];   // e^(G_r); 1 without a gate
+        uint8_t* qblk = sm + S_QPT + hh * 8192;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = 32 * hh + i;
-            *reinterpret_cast<__nv_bfloat16*>(qblk + sw128_offset(r, d & 63)) =
-                __float2bfloat16_rn(fmaf(qs, qv[i], -v[i]));
-        }
-        if (hh == 1 && !failed) {   // gamma_d
-            float gam;
-            if constexpr (PD) gam = sGamD[d];
-            else gam = gbuf[64 + 63];   // e^(G_C); 1 without a gate
-            reinterpret_cast<float*>(img + IMG_GAM)[d] = gam;
+        for (int j = 0; j < 8; ++j) {
+            const __nv_bfloat16* q8 = reinterpret_cast<const __nv_bfloat16*>(&qrow[j]);
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float qs = PD ? sRef[64 * hh + 8 * j + e] : er;
+                x[e] = fmaf(qs, __bfloat162float(q8[e]), -v[8 * j + e]);
+            }
+            st_row_chunk(qblk, r, j, x, 1.f);
         }
     }
     fence_async_smem();
@@ -961,13 +952,17 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 // that neither the state's bf16 copy nor the product's h operand touch shared
 // memory.  Per chunk n, into one accumulator D_n of 192 columns (M = 128 v):
 //   D_n  = U_n^T [K~_n | P_n^T]        (N = 192, K = 64 tokens; A = U^T from shared memory)
-//   D_n[:, 0..127]   += h_n^T Phi_n^T  (N = 128, K = 128; A = h^T from TMEM)
-//   D_n[:, 128..191] += h_n^T Qp_n^T   (N = 64,  K = 128)
+//   D_n += h_n^T [Phi_n^T | Qp_n^T]    (N = 192, K = 128; A = h^T from TMEM)
 // Columns 0..127 of D_n are X^T_n = U^T K~ + h^T Phi^T, so the state pass forms
 //   h_{n+1}^T = h_n^T Diag(gamma_n) + X^T_n
 // and columns 128..191 are O^T_n = U^T P^T + h^T Qp^T, the chunk's output.
-// Only h^T Phi^T is on the serial path: U^T [K~ | P^T] needs no state, and
-// h^T Qp^T is issued behind h^T Phi^T, so both run while the state pass works.
+// Only the second product is on the serial path; U^T [K~ | P^T] needs no
+// state and is issued a chunk ahead by its own warp, so that it runs while the
+// state pass works.  The tensor pipe takes ~80-140 cycles per instruction
+// whatever N up to 256 and a satisfied mbarrier wait costs ~100-200 cycles, so
+// the serial loop has one product of 8 instructions, one wait on the state
+// product's completion, and one named barrier from the state pass to the
+// issuing thread.
 
 // Chain kernel shared memory (bytes from a 1 KB-aligned base).
 constexpr uint32_t CH_PQ = 0;           // 2 slots of [Phi ; Qp] (48 KB each); the final state's staging
@@ -981,12 +976,15 @@ static_assert(CH_SMEM <= 232448, "chain shared memory");
 static_assert(CH_KP == 2 * 2 * PQ_BLK && CH_UT == CH_KP + 2 * 24576 && CH_OT == CH_UT + 2 * 16384,
               "chain slots");
 
-constexpr int CH_THREADS = 704;   // 22 warps: loader, MMA issuer, 4 output, 16 state
-constexpr int W_OUT = 2;          // first output warp
-constexpr int W_ST = 6;           // first state-pass warp
+constexpr int CH_THREADS = 736;   // 23 warps: loader, 2 MMA issuers, 4 output, 16 state
+constexpr int W_UK = 2;           // issuer of U^T [K~ | P^T]
+constexpr int W_OUT = 3;          // first output warp
+constexpr int W_ST = 7;           // first state-pass warp
 constexpr int N_ST = 16;          // state-pass warps: lane quarter (v) x column quarter (d)
+constexpr int BAR_H = 3;          // named barrier: h^T of the chunk is in TMEM (state pass ->
+                                  //   state-product issuer)
 // Registers: warps spread over the SM's four sub-partitions of 16 K registers
-// each, so 22 warps (six on two sub-partitions) allow at most 85 a thread,
+// each, so 23 warps (six on three sub-partitions) allow at most 85 a thread,
 // 80 in the allocation granularity of 8.
 
 // TMEM columns of the chain kernel (512 allocated): slot s of D at 256 s
@@ -998,7 +996,7 @@ constexpr uint32_t TM_SLOT = 256;
 
 enum ChainBar {
     CB_KU0, CB_KU1, CB_PQ0, CB_PQ1, CB_GAM0, CB_GAM1, CB_GAM2, CB_GAM3, CB_KUFREE0, CB_KUFREE1,
-    CB_PQFREE0, CB_PQFREE1, CB_SDONE0, CB_SDONE1, CB_ODONE0, CB_ODONE1, CB_HREADY0, CB_HREADY1,
+    CB_PQFREE0, CB_PQFREE1, CB_SDONE0, CB_SDONE1, CB_ODONE0, CB_ODONE1,
     CB_XFREE0, CB_XFREE1, CB_OFREE0, CB_OFREE1, CB_FINAL, CB_COUNT
 };
 static_assert(CB_COUNT * 8 <= 512, "barrier space");
@@ -1034,12 +1032,16 @@ __device__ __forceinline__ uint32_t st_off(int d, int v) {
 // One CTA per (batch, head): walks the wave's chunks in order.  Roles:
 //   warp 0       loader: [K~^T ; P] and U^T, then [Phi ; Qp] and gamma, two
 //                chunks ahead, by bulk copies; L2 prefetch and discard
-//   warp 1       MMA issuer: U^T [K~ | P^T] of chunk n + 1 right after the state
-//                product of chunk n, so it runs while the state pass works
-//   warps 2-5    output: O^T from TMEM -> the bf16 O tile -> TMA store
-//   warps 6-21   state pass (lane quarter x column quarter of d)
-// Every barrier is per slot (or per gamma slot) and completes at most once
-// ahead of its wait, so no parity wait can fall two phases behind.
+//   warp 1       state-product issuer: h^T [Phi^T | Qp^T] of chunk n as soon as
+//                the state pass has written h^T (named barrier BAR_H)
+//   warp 2       U^T [K~ | P^T] of chunk n + 1 as soon as its slot of D is free,
+//                so it runs while the state pass of chunk n works
+//   warps 3-6    output: O^T from TMEM -> the bf16 O tile -> TMA store
+//   warps 7-22   state pass (lane quarter x column quarter of d)
+// Every mbarrier is per slot (or per gamma slot) and completes at most once
+// ahead of its wait, so no parity wait can fall two phases behind; the state
+// pass and the state-product issuer alternate on BAR_H (the pass of chunk
+// n + 1 needs the product of chunk n).
 // UNIFORM_GAMMA: every column of the state decays by the same gamma (scalar gate
 // or none), so the state pass reads one value per chunk, ahead of the product.
 template <bool UNIFORM_GAMMA>
@@ -1084,8 +1086,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 
     if (tid == 0) {
         for (int i = 0; i < CB_COUNT; ++i)
-            mbar_init(&bars[i], (i == CB_HREADY0 || i == CB_HREADY1 || i == CB_XFREE0 ||
-                                 i == CB_XFREE1) ? N_ST : 1);
+            mbar_init(&bars[i], (i == CB_XFREE0 || i == CB_XFREE1) ? N_ST : 1);
         fence_mbar_init();
         prefetch_tmap(&maps.o);
     }
@@ -1147,18 +1148,44 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             }
         }
     } else if (warp == 1) {
-        // =========================== MMA issuer (descriptors built once; a k-step
-        // adds its byte offset / 16 to the start-address field)
+        // =========================== state-product issuer: D_nl += h^T [Phi^T | Qp^T]
+        // (N = 128 without outputs) once the state pass has written h^T; the
+        // waits that are normally satisfied by then come before the barrier
+        const bool leader = lane == 0;
+        const uint32_t id = idesc_bf16_f32(128, outputs ? 192 : 128, false, false);
+        const uint64_t d_pq = sdesc_sw128(sb + CH_PQ, 16, 1024);
+#pragma unroll 1
+        for (int nl = 0; nl < NC; ++nl) {
+            const int s = nl & 1;
+            wait(CB_PQ0 + s, (nl >> 1) & 1);
+            if (role != 2) wait(CB_KUFREE0 + s, (nl >> 1) & 1);   // U^T [K~ | P^T] of nl is in D
+            named_bar(BAR_H, 32 + 32 * N_ST);                        // h^T of nl is in TMEM
+            tc_fence_after();
+            if (leader && !failed) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ta(tmem + TM_D + TM_SLOT * s, tmem + TM_HT + TM_SLOT * s + 8 * k,
+                                d_pq + ((s * 2 * PQ_BLK + (k >> 2) * PQ_BLK + (k & 3) * 32) >> 4),
+                                id, role != 2 || k > 0);   // the transition has no U^T K~
+                mma_commit(&bars[CB_SDONE0 + s]);
+                if (outputs) mma_commit(&bars[CB_ODONE0 + s]);
+                mma_commit(&bars[CB_PQFREE0 + s]);
+            }
+        }
+        if (leader) mma_commit(&bars[CB_FINAL]);
+        int final_failed = 0;
+        if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+    } else if (warp == W_UK) {
+        // =========================== D_nl = U^T [K~ | P^T] once its operands are in
+        // and both readers of D in this slot (state pass and output, chunk
+        // nl - 2) are done with it; runs a chunk ahead of the state product
         const bool leader = lane == 0;
         const uint32_t id = idesc_bf16_f32(128, 192, false, false);
-        const uint32_t id_phi = idesc_bf16_f32(128, 128, false, false);
-        const uint32_t id_qp = idesc_bf16_f32(128, 64, false, false);
         const uint64_t d_kp = sdesc_sw128(sb + CH_KP, 16, 1024);
         const uint64_t d_ut = sdesc_sw128(sb + CH_UT, 16, 1024);
-        const uint64_t d_pq = sdesc_sw128(sb + CH_PQ, 16, 1024);
-        // D_nl = U^T [K~ | P^T] once its operands are in and both readers of D in
-        // this slot (state pass and output, chunk nl - 2) are done with it
-        auto issue_ku = [&](int nl) {
+#pragma unroll 1
+        for (int nl = 0; nl < (role != 2 ? NC : 0); ++nl) {
             const int s = nl & 1;
             wait(CB_KU0 + s, (nl >> 1) & 1);
             if (nl >= 2) {
@@ -1173,38 +1200,9 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
                              d_kp + ((s * 24576 + k * 32) >> 4), id, k > 0);
                 mma_commit(&bars[CB_KUFREE0 + s]);
             }
-        };
-        if (NC > 0 && role != 2) issue_ku(0);
-#pragma unroll 1
-        for (int nl = 0; nl < NC; ++nl) {
-            const int s = nl & 1;
-            wait(CB_PQ0 + s, (nl >> 1) & 1);
-            wait(CB_HREADY0 + s, (nl >> 1) & 1);
-            tc_fence_after();
-            if (leader && !failed) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k)   // X^T += h^T Phi^T: rows 0..127 of [Phi ; Qp]
-                    mma_bf16_ta(tmem + TM_D + TM_SLOT * s, tmem + TM_HT + TM_SLOT * s + 8 * k,
-                                d_pq + ((s * 2 * PQ_BLK + (k >> 2) * PQ_BLK + (k & 3) * 32) >> 4),
-                                id_phi, role != 2 || k > 0);   // the transition has no U^T K~
-                mma_commit(&bars[CB_SDONE0 + s]);
-                if (outputs) {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)   // O^T += h^T Qp^T: rows 128..191
-                        mma_bf16_ta(tmem + TM_D + TM_SLOT * s + 128, tmem + TM_HT + TM_SLOT * s + 8 * k,
-                                    d_pq + ((s * 2 * PQ_BLK + (k >> 2) * PQ_BLK + 16384 + (k & 3) * 32) >> 4),
-                                    id_qp, true);
-                    mma_commit(&bars[CB_ODONE0 + s]);
-                }
-                mma_commit(&bars[CB_PQFREE0 + s]);
-            }
-            if (nl + 1 < NC && role != 2) issue_ku(nl + 1);
+            __syncwarp();
         }
-        if (leader) mma_commit(&bars[CB_FINAL]);
-        int final_failed = 0;
-        if (!mbar_wait(&bars[CB_FINAL], 0, &final_failed)) atomicOr(p.status, kStatusTimeout);
-        __syncwarp();
-    } else if (warp < W_ST) {
+    } else if (warp < W_ST) {   // warps W_OUT ..
         // =========================== output: O^T row v -> the O tile [r][v]
         // (bf16, swizzled) in its slot -> TMA store
         const int v = (warp & 3) * 32 + lane;
@@ -1316,7 +1314,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CB_HREADY0 + s]);
+            named_bar_arrive(BAR_H, 32 + 32 * N_ST);
         }
         if (NC > 0) {   // final state, staged over the [Phi ; Qp] slots (free once the
                         // last state product is done), written by four TMA stores
