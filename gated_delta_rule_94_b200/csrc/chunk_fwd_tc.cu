@@ -308,7 +308,7 @@ constexpr uint32_t PD_KT = P_KT;             // per-dimension gate: g bf16 (TMA)
 constexpr uint32_t S_PHI = 32768;            // over V and the W^T rows
 constexpr uint32_t S_QPT = P_KT;             // Qp [64 r][128 d] as two [64][64] blocks, over
                                              // K~^T: dead once the K~^T W product is done and
-                                             // K~^T's image store (the oldest) has read it
+                                             // K~^T's image store has read it
 constexpr int LDG = 132;                     // fp32 row stride of G [64][128] (exact fallback; aliases A / T)
 static_assert(P_TF + 64 * LDF * 4 <= P_KT, "A / T scratch");
 static_assert(P_WUT + 32768 <= P_KT, "[W^T; U^T] tile");
@@ -344,6 +344,10 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P_BAR);   // kq, s, wu, f, v
     __shared__ uint32_t s_tmem;
     constexpr bool PD = GATE == kGatePerDim;
+    // the g tile and the write key feed the first step of an item: their loads
+    // (and V's) are issued at the end of the previous item; otherwise V alone,
+    // needed only by the U^T product, is issued after the item's first barrier
+    constexpr bool EARLY = PD || WK;
 
     // The grid's last block only waits for the kernel before it (the previous
     // wave's chain): this grid then completes after that chain, so the chain of
@@ -362,12 +366,12 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     const uint32_t sb = smem_u32(sm);
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int failed = 0;
+    bool rest_issued = false;   // thread 0: the next item's g / write key / V loads are out
     uint32_t ph = 0;   // phase of every barrier: each completes once per item
     auto wait = [&](int i, uint32_t parity) {
         if (!mbar_wait(&bars[i], parity, &failed)) atomicOr(p.status, kStatusTimeout);
         __syncwarp();
     };
-    __shared__ int s_item[2];
 
     float* sBeta = gbuf + 192;
     // per-dimension gate
@@ -375,18 +379,24 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     float* sGamD = gbuf + 256;                         // gamma_d = e^(c_d)
     float* sRef = gbuf + 384;                          // e^(c_d); 1 in the exact fallback
 
-    // item -> (sequence, head, chunk of this wave)
-    auto coords = [&](int item, int& b, int& h, int& n) {
-        const int bh = item / p.nchunks;
-        b = bh / H;
-        h = bh % H;
-        n = p.chunk0 + item % p.nchunks;
+    // Items are claimed one ahead, by one thread, which also stores the item's
+    // (sequence, head, chunk, sequence * H + head) for every thread to read, so
+    // that no thread on the item's path divides.
+    __shared__ int s_item[2];
+    __shared__ int4 s_crd[2];
+    auto claim = [&](int slot) {
+        const int item = (int)atomicAdd(p.counter, 1u);
+        s_item[slot] = item;
+        if (item < nitems) {
+            const int bh = item / p.nchunks;
+            s_crd[slot] = make_int4(bh / H, bh % H, p.chunk0 + item % p.nchunks, bh);
+        }
     };
-    // K and Q of an item, with the expect_tx of every byte its bars[0] phase
-    // counts (the g tile and the write key follow in issue_rest)
-    auto issue_kq = [&](int item) {
-        int b, h, n;
-        coords(item, b, h, n);
+    // K and Q of the item in slot `slot`, with the expect_tx of every byte its
+    // bars[0] phase counts (the g tile and the write key follow in issue_rest)
+    auto issue_kq = [&](int slot) {
+        const int4 c = s_crd[slot];
+        const int b = c.x, h = c.y, n = c.z;
         mbar_arrive_expect_tx(&bars[0], (PD ? 6 : 4) * 8192 + (WK ? 2 * 8192 : 0));
         for (int blk = 0; blk < 2; ++blk) {
             tma_load_3d_hint(sm + P_KQ + blk * 16384, &maps.k, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
@@ -396,9 +406,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     // the rest of an item's tiles, into slots that are free only once the
     // previous item has finished: g (per-dimension gate; its slot held the
     // previous item's Qp staging), the write key, V
-    auto issue_rest = [&](int item) {
-        int b, h, n;
-        coords(item, b, h, n);
+    auto issue_rest = [&](int b, int h, int n) {
         for (int blk = 0; blk < 2; ++blk) {
             if constexpr (PD)
                 tma_load_3d_hint(sm + PD_KT + blk * 8192, &maps.g, &bars[0], h * D + 64 * blk, n * C, b, pol_in);
@@ -413,9 +421,9 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     };
     // beta and g of an item, by warps 2-3 into registers
     float nb = 0.f, ng = 0.f;
-    auto fetch_bg = [&](int item) {
-        int b, h, n;
-        coords(item, b, h, n);
+    auto fetch_bg = [&](int slot) {
+        const int4 c = s_crd[slot];
+        const int b = c.x, h = c.y, n = c.z;
         const int t = n * C + (tid - 64);
         nb = ng = 0.f;
         if (t < T) {
@@ -428,9 +436,11 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     if (tid == 0) {
         for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
-        const int first = (int)atomicAdd(p.counter, 1u);
-        s_item[0] = first;
-        if (first < nitems) issue_kq(first);
+        claim(0);
+        if (s_item[0] < nitems) {
+            issue_kq(0);
+            if (EARLY) issue_rest(s_crd[0].x, s_crd[0].y, s_crd[0].z);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&s_tmem, 256);
@@ -441,7 +451,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     tc_fence_after();
     const uint32_t tmem = s_tmem;
     int item = s_item[0];
-    if ((warp == 2 || warp == 3) && item < nitems) fetch_bg(item);
+    if ((warp == 2 || warp == 3) && item < nitems) fetch_bg(0);
     // the write key's tile: blocks of [64 tokens][64 d] with a stride of 8 KB
     // (WK, in the V slot) or the K tile's 16 KB (K and Q interleaved)
     const uint32_t kwo = WK ? P_V : P_KQ;
@@ -450,11 +460,9 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll 1
     for (int it = 0; item < nitems; ++it) {
     ph = it & 1;
-    int b, h, n;
-    coords(item, b, h, n);
-    const int bh = item / p.nchunks, nl = item % p.nchunks;
+    const int4 crd = s_crd[it & 1];
+    const int b = crd.x, h = crd.y, n = crd.z, bh = crd.w, nl = n - p.chunk0;
     uint8_t* img = p.ws + ((size_t)bh * p.cw + nl) * IMG_BYTES;
-    if (tid == 0) issue_rest(item);
     // V into the slot the write key held, once every reader of the key is done
     // (the caller has passed a CTA barrier after the last read)
     auto load_v_late = [&]() {
@@ -467,15 +475,18 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             }
         }
     };
-    if (tid == 0) bulk_wait_read();   // the previous item's Qp staging (its g slot, K~^T) is read
     if (warp == 2 || warp == 3) {   // beta and g (fetched during the previous item)
         gbuf[tid - 64] = ng;
         sBeta[tid - 64] = nb;
     }
     __syncthreads();
+    // the rest of the item's tiles, by a thread that is idle until the S
+    // product is done (their slots were read by the previous item's stores
+    // before the barrier at its end)
+    if (!EARLY && tid == 160) issue_rest(b, h, n);
     // the next item, taken now so that the global atomic is off the path; its
     // K and Q are issued once this item's last readers of both are done
-    if (tid == 64) s_item[(it + 1) & 1] = (int)atomicAdd(p.counter, 1u);
+    if (tid == 64) claim((it + 1) & 1);
 
     bool exact = false;
     if constexpr (!PD) {
@@ -607,7 +618,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (tid == 0 && !failed) {   // K~^T is final: its image goes out now
+        if (tid == 64 && !failed) {   // K~^T is final: its image goes out now
             bulk_store_hint(img + IMG_KP, sm + PD_KT, 16384, pol_img);
             bulk_commit();
         }
@@ -750,13 +761,14 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
                         pack_bf16(__bfloat162float(e0[e]) * f0, __bfloat162float(e1[e]) * f1);
             }
             fence_async_smem();
+            named_bar(5, NPR - 64);
+            if (t == 0 && !failed) {   // K~^T is final: its image goes out now (thread 64)
+                bulk_store_hint(img + IMG_KP, sm + P_KT, 16384, pol_img);
+                bulk_commit();
+            }
         }
     });
     if constexpr (!PD) load_v_late();  // K~^T, the write key's last reader, is formed
-    if (!PD && tid == 0 && !failed) {   // K~^T is final: its image goes out now
-        bulk_store_hint(img + IMG_KP, sm + P_KT, 16384, pol_img);
-        bulk_commit();
-    }
     // T diag(beta) and T diag(beta e^G) as bf16 K-major [r][i]
     {
         const float* sGam = gbuf + 64;
@@ -848,8 +860,8 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     // Row r of Q (its half hh of the columns) into the registers of the thread
     // that forms row r of Qp (lanes 64 + r), so that the next item's K and Q
     // can land once every thread has passed the barrier below.  The K~^T tile
-    // becomes the Qp staging: its image store (the oldest of this item's
-    // groups) must have read it.
+    // becomes the Qp staging: its image store (issued by thread 64) must have
+    // read it.
     const int row = (warp & 3) * 32 + lane;
     uint4 qrow[8];
     if (row >= 64) {
@@ -857,18 +869,11 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) qrow[j] = *reinterpret_cast<const uint4*>(qb + sw128_offset(row - 64, 8 * j));
     }
-    if (tid == 0) bulk_wait_read_all_but_one();
+    if (tid == 64) bulk_wait_read();   // K~^T's image store (thread 64's only group)
     tc_fence_after();
     __syncthreads();
-    if (tid == 0) {
-        const int nx = s_item[(it + 1) & 1];
-        if (nx < nitems) {
-            fence_async_smem();
-            issue_kq(nx);
-        }
-    }
     const int next_item = s_item[(it + 1) & 1];
-    if ((warp == 2 || warp == 3) && next_item < nitems) fetch_bg(next_item);
+    if ((warp == 2 || warp == 3) && next_item < nitems) fetch_bg((it + 1) & 1);
     {   // Phi = -K~^T W, row d: warps 0-3 columns 0-63, warps 4-7 columns 64-127;
         // each half stored as soon as it is staged
         const int hh = warp >> 2;
@@ -882,6 +887,13 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
         if ((tid & 127) == 0 && !failed) {
             bulk_store_hint(img + IMG_PQ + hh * PQ_BLK, sm + S_PHI + hh * 16384, 16384, pol_img);
             bulk_commit();
+        }
+        // the next item's K and Q: every reader of this item's is done (the Q
+        // rows of Qp were read before the barrier above); issued by a thread
+        // whose warps have no Qp rows, after its share of Phi
+        if (tid == 0 && next_item < nitems) {
+            fence_async_smem();
+            issue_kq((it + 1) & 1);
         }
     }
     if (warp >= 4 && !failed) {   // gamma_d, d = row
@@ -917,9 +929,16 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             bulk_store_hint(img + IMG_PQ + PQ_BLK + 16384, sm + S_QPT + 8192, 8192, pol_img);
             bulk_commit();
         }
-        // Phi's first half (over the V slot, which the next item loads first) is
-        // read; Qp's staging is waited for at the next item's top
-        bulk_wait_read_all_but_one();
+        // every staging of this item is read (Phi's first half is over the V
+        // slot, Qp's over the g slot and K~^T: the next item loads V and g first)
+        bulk_wait_read();
+        rest_issued = false;
+        if (EARLY && next_item < nitems && !failed) {
+            const int4 c = s_crd[(it + 1) & 1];
+            fence_async_smem();
+            issue_rest(c.x, c.y, c.z);
+            rest_issued = true;
+        }
     }
     tc_fence_before();
     if (__syncthreads_or(failed)) {
@@ -930,6 +949,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
             const bool cur = mbar_wait(&bars[0], ph, &f2);
             mbar_wait(&bars[4], ph, &f2);
             if (cur && next_item < nitems) mbar_wait(&bars[0], ph ^ 1u, &f2);
+            if (rest_issued && !WK) mbar_wait(&bars[4], ph ^ 1u, &f2);
         }
         __syncthreads();
         break;
@@ -937,7 +957,7 @@ chunk_prep_kernel(const __grid_constant__ PrepMaps maps, const ChunkParams p) {
     tc_fence_after();
     item = next_item;
     }   // items
-    if (tid == 0 || tid == 128) bulk_wait_all();   // the last item's stores are complete
+    if (tid == 0 || tid == 64 || tid == 128) bulk_wait_all();   // the last item's stores are complete
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
