@@ -546,6 +546,205 @@ def time_decode(ctx: Ctx):
     return rec, launches
 
 
+# ------------------------------------------------- the rows beyond the forward
+def time_events(ctx: Ctx, fn, flush=True):
+    """Mean and min CUDA-event time (ms) of fn over --steps calls after
+    --warmup, L2 flushed before each call (outside the events)."""
+    for _ in range(ctx.args.warmup):
+        if flush:
+            ctx.flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(ctx.args.steps):
+        if flush:
+            ctx.flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(ctx.stream)
+        fn()
+        e1.record(ctx.stream)
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    return sum(ms) / len(ms), min(ms)
+
+
+def hbm_roofline(ctx: Ctx, nbytes, ms, kernel):
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": gbs, "peak": ctx.peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / ctx.peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes": nbytes,
+            "kernel": kernel, "peak_source": ctx.peak_src + ", hbm_gbs (copy bandwidth)"}
+
+
+def retention_gate(B, T, H, seed, device):
+    """Retention gate of the preconditioner scan: sigmoid(N(0,1) + 2), bf16."""
+    gen = torch.Generator().manual_seed(seed)
+    return torch.sigmoid(torch.randn(B, T, H, generator=gen) + 2.0).to(torch.bfloat16).to(device)
+
+
+def time_osdn(ctx: Ctx):
+    """The preconditioned delta rule on the GDN workload's shape (B4 H16 T2048,
+    scalar gate, bf16): phase 1 (write keys by the preconditioner scan, eta 0.5,
+    retention gate) and phase 2 (the chunk forward with the write keys)."""
+    gdn, args = ctx.gdn, ctx.args
+    w = gi.WORKLOADS[1]
+    B, T, H, Dk, Dv = w.B, w.T, w.H, w.Dk, w.Dv
+    d = gi.workload_inputs(w, device=ctx.dev)
+    r = retention_gate(B, T, H, 7, ctx.dev)
+    kw = torch.empty_like(d["k"])
+    d1 = torch.empty(B, H, Dk, device=ctx.dev)
+    o = torch.empty(B, T, H, Dv, dtype=torch.bfloat16, device=ctx.dev)
+    S = torch.empty(B, H, Dk, Dv, device=ctx.dev)
+    nws = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, 64, torch.bfloat16, w.gate_kind)
+    ws = torch.empty(nws, dtype=torch.uint8, device=ctx.dev)
+
+    def phase1():
+        gdn.gdn_osdn_precondition(d["k"], d["beta"], r, 0.5, None, kw, d1, stream=ctx.stream)
+
+    def both():
+        phase1()
+        gdn.gdn_chunk_fwd_wk(d["q"], d["k"], kw, d["v"], d["beta"], d["g"], w.gate_kind, d["S0"],
+                             o, S, workspace=ws, stream=ctx.stream)
+    n0 = gdn.gdn_kernel_launch_count()
+    both()
+    torch.cuda.synchronize()
+    launches = gdn.gdn_kernel_launch_count() - n0
+    ms1, _ = time_events(ctx, phase1)
+    ms, ms_min = time_events(ctx, both)
+    N = B * T * H
+    b1 = N * (2 * Dk * 2 + 2 + 2) + B * H * Dk * 4          # k, beta, r in; k_write, d out
+    b2 = chunk_bytes(w) + N * Dk * 2                          # the forward, plus k_write
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        cores = len(os.sched_getaffinity(0))
+        Hs, Ts = min(H, cores), 1024
+        x = gi.workload_inputs(w, B=1, T=Ts, H=Hs)
+        f = gi.to_f64_numpy(x)
+        rr = retention_gate(1, Ts, Hs, 7, "cpu").double().numpy()
+        reps, total = 0, 0.0
+        while total < args.cpu_seconds or reps == 0:
+            t0 = time.perf_counter()
+            kw_ref, _ = oracle.osdn_precondition(f["k"], f["beta"], 0.5, r=rr)
+            oracle.recurrent_wk(f["q"], f["k"], kw_ref, f["v"], f["beta"], f["g"], f["gate_kind"],
+                                f["S0"], threads=cores)
+            total += time.perf_counter() - t0
+            reps += 1
+        cpu = {"value": Hs * Ts * reps / total / H, "unit": "tokens/s", "cores": cores,
+               "kind": "oracle", "sample": f"{Hs} heads x {Ts} tokens of one sequence, both "
+                                          f"phases, {reps} runs, {total:.1f} s; tokens/s = "
+                                          f"token-heads/s / {H} heads"}
+    del d, r, kw, d1, o, S, ws
+    torch.cuda.empty_cache()
+    return {
+        "workload": f"preconditioned delta rule (eta 0.5, retention gate), {w.name}",
+        "ms_per_step": ms, "ms_min": ms_min, "tokens_per_s": B * T / (ms * 1e-3),
+        "phase1_ms": ms1,
+        "phase1_roofline": hbm_roofline(ctx, b1, ms1, "osdn_precondition_kernel"),
+        "roofline": hbm_roofline(ctx, b1 + b2, ms, "osdn_precondition_kernel + chunk_prep_kernel,"
+                                                   "chunk_chain_kernel (both phases)"),
+        "gpu_launches_per_step": launches, "cpu_baseline": cpu,
+    }
+
+
+def time_segments(ctx: Ctx):
+    """A few-head long sequence (B1 H4 T65536, scalar gate, bf16), where the
+    segment-parallel state pass engages with the full-speed workspace; timed
+    beside the largest workspace whose plan runs the plain chain."""
+    gdn, args = ctx.gdn, ctx.args
+    w = gi.Workload("few-head long-sequence scalar-gated chunk fwd bf16 B1 H4 T65536 d128",
+                    "chunk", B=1, T=65536, H=4, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                    gate="scalar", gate_scale=0.1, s0_std=None)
+    B, T, H, Dk, Dv = w.B, w.T, w.H, w.Dk, w.Dv
+    d = gi.workload_inputs(w, device=ctx.dev)
+    o = torch.empty(B, T, H, Dv, dtype=torch.bfloat16, device=ctx.dev)
+    S = torch.empty(B, H, Dk, Dv, device=ctx.dev)
+    full = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, 64, torch.bfloat16, w.gate_kind)
+    plain = None
+    for frac in [x / 20 for x in range(19, 0, -1)]:
+        n = int(full * frac) // 256 * 256
+        if gdn.gdn_chunk_fwd_plan(B, T, H, Dk, Dv, 64, torch.bfloat16, w.gate_kind, n)["segments"] == 1:
+            plain = n
+            break
+    rec = {"workload": w.name}
+    for name, nws in (("segmented", full), ("plain_chain", plain)):
+        if nws is None:
+            continue
+        ws = torch.empty(nws, dtype=torch.uint8, device=ctx.dev)
+        plan = gdn.gdn_chunk_fwd_plan(B, T, H, Dk, Dv, 64, torch.bfloat16, w.gate_kind, nws)
+
+        def step():
+            gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], w.gate_kind, d["S0"], o,
+                              S, workspace=ws, stream=ctx.stream)
+        ms, ms_min = time_events(ctx, step)
+        rec[name] = {"ms_per_step": ms, "ms_min": ms_min, "tokens_per_s": B * T / (ms * 1e-3),
+                     "workspace_bytes": nws, "plan": plan,
+                     "roofline": hbm_roofline(ctx, chunk_bytes(w), ms,
+                                              "chunk_prep_kernel,chunk_chain_kernel,"
+                                              "segment_combine_kernel (one forward)")}
+        del ws
+    del d, o, S
+    torch.cuda.empty_cache()
+    return rec
+
+
+def time_backward(ctx: Ctx):
+    """The backward of the chunk forward on the GDN workload's shape (B4 H16
+    T2048, scalar gate, bf16 tokens): fp32 dq, dk, dv, dbeta, dg and the
+    initial state's gradient from dO (bf16) and the final state's gradient."""
+    gdn, args = ctx.gdn, ctx.args
+    w = gi.WORKLOADS[1]
+    B, T, H, Dk, Dv = w.B, w.T, w.H, w.Dk, w.Dv
+    d = gi.workload_inputs(w, device=ctx.dev)
+    gen = torch.Generator().manual_seed(11)
+    do = torch.randn(B, T, H, Dv, generator=gen).to(torch.bfloat16).to(ctx.dev)
+    dS = (0.02 * torch.randn(B, H, Dk, Dv, generator=gen)).to(ctx.dev)
+    g = {n: torch.empty(B, T, H, *s, device=ctx.dev) for n, s in
+         (("dq", (Dk,)), ("dk", (Dk,)), ("dv", (Dv,)), ("dbeta", ()), ("dg", ()))}
+    dS0 = torch.empty(B, H, Dk, Dv, device=ctx.dev)
+    nws = gdn.gdn_chunk_bwd_workspace_bytes(B, T, H, Dk, Dv, 64, torch.bfloat16, w.gate_kind)
+    ws = torch.empty(nws, dtype=torch.uint8, device=ctx.dev)
+
+    def step():
+        gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], w.gate_kind, d["S0"], do, dS,
+                          g["dq"], g["dk"], g["dv"], g["dbeta"], g["dg"], dS0, workspace=ws,
+                          stream=ctx.stream)
+    n0 = gdn.gdn_kernel_launch_count()
+    step()
+    torch.cuda.synchronize()
+    launches = gdn.gdn_kernel_launch_count() - n0
+    ms, ms_min = time_events(ctx, step)
+    N = B * T * H
+    nbytes = N * (2 * (2 * Dk + 2 * Dv + 2)) + N * 4 * (2 * Dk + Dv + 2) + 2 * B * H * Dk * Dv * 4
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        Hs, Ts = 2, 128
+        x = gi.workload_inputs(w, B=1, T=Ts, H=Hs)
+        f = gi.to_f64_numpy(x)
+        dof = do[:1, :Ts, :Hs].double().cpu().numpy()
+        reps, total = 0, 0.0
+        while total < args.cpu_seconds or reps == 0:
+            t0 = time.perf_counter()
+            oracle.backward(f["q"], f["k"], f["v"], f["beta"], f["g"], f["gate_kind"], f["S0"], dof)
+            total += time.perf_counter() - t0
+            reps += 1
+        cpu = {"value": Hs * Ts * reps / total / H, "unit": "tokens/s",
+               "cores": torch.get_num_threads(), "kind": "oracle",
+               "sample": f"{Hs} heads x {Ts} tokens of one sequence (reverse-mode autograd of the "
+                         f"fp64 token loop), {reps} runs, {total:.1f} s; tokens/s = "
+                         f"token-heads/s / {H} heads"}
+    del d, do, dS, g, dS0, ws
+    torch.cuda.empty_cache()
+    return {
+        "workload": f"backward, {w.name}", "ms_per_step": ms, "ms_min": ms_min,
+        "tokens_per_s": B * T / (ms * 1e-3),
+        "roofline": hbm_roofline(ctx, nbytes, ms, "chunk_prep_kernel,chunk_chain_kernel (forward "
+                                                  "rerun), adjoint_chain_kernel, chunk_bwd_kernel"),
+        "gpu_launches_per_step": launches, "cpu_baseline": cpu,
+    }
+
+
 def run_only(args, world, rank, local):
     """One forward workload alone (for profiling): its record, no CPU baseline."""
     args.no_cpu_baseline = True
@@ -570,6 +769,12 @@ def run_ours(args, world, rank, local):
     dec = None
     if not args.no_decode:
         dec, _ = time_decode(ctx)
+    extras = {}
+    if rank == 0 and world == 1 and not args.no_extras:
+        t0 = time.perf_counter()
+        extras = {"osdn": time_osdn(ctx), "segments": time_segments(ctx),
+                  "backward": time_backward(ctx)}
+        ctx.sampler.mark(t0, time.perf_counter())
     clocks = ctx.sampler.stop()
     if rank != 0:
         return
@@ -593,6 +798,7 @@ def run_ours(args, world, rank, local):
         "cpu_baseline": head["cpu_baseline"],
         "workloads": subs,
         "decode": dec,
+        "extras": extras,
         "gpu": torch.cuda.get_device_name(ctx.dev),
     }
     _ = w
@@ -612,6 +818,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the preconditioned-rule, segment and backward records")
     ap.add_argument("--only", type=int, default=None, choices=(0, 1, 2, 3),
                     help="time one forward workload alone and print its record (profiling)")
     args = ap.parse_args()

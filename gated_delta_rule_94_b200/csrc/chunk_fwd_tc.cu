@@ -1378,55 +1378,86 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const ChunkParams p) 
 // (from a zero state) and A_j (from the identity, with no writes) for every
 // segment at once; this kernel composes them in order, h_{j+1} = A_j h_j + b_j
 // in fp32 from the wave's entering state h_0; the chain kernel in segment
-// mode 3 then runs every segment from its h_j with outputs.  One CTA per
-// (batch, head), 1024 threads: thread (row d, 16 columns v); h and A_j in
-// shared memory (A_j rows padded by one word).
-constexpr int SEGC_THREADS = 1024;
-constexpr uint32_t SEGC_SMEM = (D * D + D * (D + 1)) * sizeof(float);
+// mode 3 then runs every segment from its h_j with outputs.  The columns v of
+// the state evolve independently, so one CTA takes 16 of them for one
+// (batch, head): thread (row d, 8 columns), h_j's 16 columns in shared
+// memory, A_j there too (rows padded to 132 words: 16-byte aligned, two-way
+// bank conflicts at most), the next A_j copied in (cp.async) while the
+// current one is applied.
+constexpr int SEGC_THREADS = 256;
+constexpr int SEGC_COLS = 16;                  // state columns per CTA
+constexpr int SEGC_LDA = 132;                  // row stride of A_j in shared memory (words)
+constexpr uint32_t SEGC_SMEM = (2 * D * SEGC_LDA + D * SEGC_COLS) * sizeof(float);
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __global__ void __launch_bounds__(SEGC_THREADS)
 segment_combine_kernel(const ChunkParams p, const float* __restrict__ seg_b,
                        const float* __restrict__ seg_a) {
-    extern __shared__ float smf[];
-    float* hs = smf;             // h_j [D][D]
-    float* As = smf + D * D;     // A_j [D][D + 1]
+    extern __shared__ __align__(16) float smf[];
+    float* As = smf;                          // A_j [2][D][SEGC_LDA]
+    float* hs = smf + 2 * D * SEGC_LDA;       // h_j [D][SEGC_COLS]
     pdl_wait();                  // offsets and transitions are complete and visible
                                  // (no early launch of the output pass: its CTAs wait
                                  // for this grid and must not hold SMs it needs)
-    const int bh = blockIdx.x, S = p.nseg, t = threadIdx.x;
-    const int d = t >> 3, cg = t & 7;
-    for (int idx = t; idx < D * D; idx += SEGC_THREADS)
-        hs[idx] = p.s0 ? __ldcg(p.s0 + (size_t)bh * D * D + idx) : 0.f;
+    constexpr int NG = D / SEGC_COLS;
+    const int bh = blockIdx.x / NG, v0 = SEGC_COLS * (blockIdx.x % NG);
+    const int S = p.nseg, t = threadIdx.x;
+    const int d = t >> 1, c0 = 8 * (t & 1);
+    // A_j -> buffer j & 1: 16 copies of 16 bytes a thread (rows of 32 chunks)
+    auto fetch_a = [&](int j) {
+        const float* src = seg_a + ((size_t)bh * S + j) * D * D;
+        float* dst = As + (j & 1) * D * SEGC_LDA;
+#pragma unroll
+        for (int i = 0; i < D * D / 4 / SEGC_THREADS; ++i) {
+            const int idx = t + SEGC_THREADS * i, row = idx >> 5, ch = idx & 31;
+            cp_async16(dst + row * SEGC_LDA + 4 * ch, src + row * D + 4 * ch);
+        }
+        cp_async_commit();
+    };
+    if (S > 1) fetch_a(0);
+    for (int idx = t; idx < D * SEGC_COLS; idx += SEGC_THREADS) {
+        const int r = idx / SEGC_COLS, cc = idx % SEGC_COLS;
+        hs[idx] = p.s0 ? __ldcg(p.s0 + (size_t)bh * D * D + r * D + v0 + cc) : 0.f;
+    }
 #pragma unroll 1
     for (int jj = 0; jj + 1 < S; ++jj) {
-        const size_t off = ((size_t)bh * S + jj) * D * D;
-        for (int idx = t; idx < D * D; idx += SEGC_THREADS)
-            As[(idx >> 7) * (D + 1) + (idx & 127)] = __ldcg(seg_a + off + idx);
-        float acc[16];
+        const bool more = jj + 2 < S;
+        if (more) fetch_a(jj + 1);
+        float acc[8];
+        const float* bsrc = seg_b + ((size_t)bh * S + jj) * D * D + d * D + v0 + c0;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc[e] = __ldcg(seg_b + off + d * D + 16 * cg + e);
-        __syncthreads();
-#pragma unroll 4
+        for (int e = 0; e < 8; ++e) acc[e] = __ldcg(bsrc + e);
+        if (more) cp_async_wait<1>();
+        else cp_async_wait<0>();
+        __syncthreads();         // A_j and h_j are in shared memory
+        const float* arow = As + (jj & 1) * D * SEGC_LDA + d * SEGC_LDA;
+#pragma unroll 8
         for (int dp = 0; dp < D; ++dp) {
-            const float a = As[d * (D + 1) + dp];
-            const float4* hr = reinterpret_cast<const float4*>(hs + dp * D + 16 * cg);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 x = hr[q];
-                acc[4 * q] = fmaf(a, x.x, acc[4 * q]);
-                acc[4 * q + 1] = fmaf(a, x.y, acc[4 * q + 1]);
-                acc[4 * q + 2] = fmaf(a, x.z, acc[4 * q + 2]);
-                acc[4 * q + 3] = fmaf(a, x.w, acc[4 * q + 3]);
-            }
+            const float a = arow[dp];
+            const float4 x0 = *reinterpret_cast<const float4*>(hs + dp * SEGC_COLS + c0);
+            const float4 x1 = *reinterpret_cast<const float4*>(hs + dp * SEGC_COLS + c0 + 4);
+            acc[0] = fmaf(a, x0.x, acc[0]);
+            acc[1] = fmaf(a, x0.y, acc[1]);
+            acc[2] = fmaf(a, x0.z, acc[2]);
+            acc[3] = fmaf(a, x0.w, acc[3]);
+            acc[4] = fmaf(a, x1.x, acc[4]);
+            acc[5] = fmaf(a, x1.y, acc[5]);
+            acc[6] = fmaf(a, x1.z, acc[6]);
+            acc[7] = fmaf(a, x1.w, acc[7]);
         }
-        __syncthreads();         // every thread is done with h_j and A_j
-        float* dst = p.seg_h + ((size_t)bh * S + jj + 1) * D * D + d * D + 16 * cg;
+        __syncthreads();         // every thread is done with h_j and A_j's buffer
+        float* dst = p.seg_h + ((size_t)bh * S + jj + 1) * D * D + d * D + v0 + c0;
+        *reinterpret_cast<float4*>(hs + d * SEGC_COLS + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(hs + d * SEGC_COLS + c0 + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            hs[d * D + 16 * cg + e] = acc[e];
-            dst[e] = acc[e];
-        }
-        __syncthreads();
+        for (int e = 0; e < 8; ++e) dst[e] = acc[e];
     }
 }
 
@@ -1707,7 +1738,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p0, int gate, size_t ws_bytes
             if (e != cudaSuccess) return e;
             ++*launches;
             cudaLaunchConfig_t cc = cfg;
-            cc.gridDim = dim3((unsigned)nbh);
+            cc.gridDim = dim3((unsigned)(nbh * (D / SEGC_COLS)));
             cc.blockDim = dim3(SEGC_THREADS);
             cc.dynamicSmemBytes = SEGC_SMEM;
             const float* sb_ = seg2;
