@@ -23,8 +23,8 @@
 // and every chunk's entering state):
 //   adjoint_chain_kernel  one CTA per (batch, head), chunks from the last back:
 //                         stores the adjoint of each chunk's leaving state,
-//                         then dS0; fp32 on CUDA cores (the transition in bf16
-//                         as the forward's image holds it)
+//                         then dS0; the products on the tensor cores, straight
+//                         from the forward's step images, the adjoint in fp32
 //   chunk_bwd_kernel      one CTA per (batch, head, chunk): recomputes the
 //                         chunk's A, T, W, U, D and forms every gradient of the
 //                         chunk; fp32 on CUDA cores, dq and dk accumulated in
@@ -33,6 +33,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tmap.cuh"
 
 namespace gdn {
 namespace {
@@ -42,7 +43,6 @@ using sm100::sw128_offset;
 constexpr int D = 128;
 constexpr int C = 64;
 
-__device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
 // C[m][n] (+)= sum_k a(m, k) b(k, n) for an output tile of (RM * TR) x (RN * TC)
 // on TR x TC threads: thread (tr, tc) owns rows i * TR + tr and columns
@@ -89,81 +89,182 @@ __device__ __forceinline__ void zero(float (&acc)[RM][RN]) {
 }
 
 // ------------------------------------------------------------ adjoint chain
-constexpr int AC_THREADS = 512;
-constexpr int LDH = D + 4;   // fp32 row stride of dh in shared memory
-constexpr uint32_t AC_DH = 0;                               // dh [D][LDH] fp32
-constexpr uint32_t AC_PQ = AC_DH + D * LDH * 4;             // [Phi ; Qp] image, 2 x 24 KB
-constexpr uint32_t AC_DO = AC_PQ + 2 * kImgPQBlock;         // dO [64][128] bf16
-constexpr uint32_t AC_GAM = AC_DO + C * D * 2;              // gamma [128] fp32
-constexpr uint32_t AC_SMEM = AC_GAM + D * 4 + 1024;
+// The transpose of the forward's chain, on the tensor cores.  The adjoint dh
+// of a chunk's leaving state maps to the adjoint of its entering state by
+//     dh <- gamma (.) dh + Phi^T dh + Qp^T dO_c,
+// which, on the transposed adjoint dh^T [v][d] (as the forward chain carries
+// h^T), is one accumulator per chunk:
+//     D = dh^T Phi   (M = 128 v, N = 128 d', K = 128 d; A = bf16 dh^T in TMEM,
+//                     B = Phi straight from the forward's step image: its rows d,
+//                     columns d' contiguous, are the MN-major form of B)
+//       + dO^T Qp    (K = 64 r; A = the dO tile [r][v] loaded by TMA, MN-major;
+//                     B = rows 128.. of the same image tile, MN-major)
+//     dh^T <- gamma (.) dh^T + D          (fp32, in the state-pass registers).
+// One CTA per (batch, head), chunks from the last back.  Roles:
+//   warp 0      loader: [Phi ; Qp] and dO of the next two chunks (two slots),
+//               gamma (a ring of four)
+//   warp 1      MMA issuer: the 12 instructions of a chunk once the state pass
+//               has written dh^T (named barrier AJ_BAR_H)
+//   warps 2-17  state pass (lane quarter v x column quarter d): stores each
+//               chunk's leaving-state adjoint, then folds in the product
+// Every mbarrier wait is bounded; named barriers join warps that run the same
+// number of iterations whatever happens.
+struct AdjMaps {
+    CUtensorMap dO;   // dO [B][T][H*D] bf16, 64 x 64 boxes, 128-byte swizzle
+};
+constexpr int AJ_THREADS = 32 * 18;
+constexpr int AJ_ST = 2;                       // first state-pass warp
+constexpr int AJ_NST = 16;
+constexpr int AJ_BAR_H = 1;
+constexpr uint32_t AJ_PQ = 0;                  // 2 slots of [Phi ; Qp] (2 K-blocks each)
+constexpr uint32_t AJ_DO = 2 * 2 * kImgPQBlock;   // 2 slots of dO [64 r][128 v] (two blocks)
+constexpr uint32_t AJ_GAM = AJ_DO + 2 * 16384;    // 4 slots of gamma [128]
+constexpr uint32_t AJ_BAR = AJ_GAM + 4 * 512;
+constexpr uint32_t AJ_SMEM = AJ_BAR + 256 + 1024;
+enum AjBar { AJ_FULL0, AJ_FULL1, AJ_GAM0, AJ_GAM1, AJ_GAM2, AJ_GAM3, AJ_DONE0, AJ_DONE1,
+             AJ_FREE0, AJ_FREE1, AJ_FINAL, AJ_NBARS };
+// TMEM (512 columns): D of slot s at 128 s, bf16 dh^T of slot s at 256 + 64 s
+constexpr uint32_t AJ_TM_D = 0;
+constexpr uint32_t AJ_TM_H = 256;
 
-// One CTA per (batch, head).  dh starts at dS_final (or 0); for each chunk c
-// from the last: dh_all[c] = dh (the adjoint of the chunk's leaving state),
-// then dh = gamma dh + Phi^T dh + Qp^T dO_c.  The last dh is dS0.
-__global__ void __launch_bounds__(AC_THREADS)
-adjoint_chain_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(AJ_THREADS, 1)
+adjoint_chain_kernel(const __grid_constant__ AdjMaps maps, const BwdParams p) {
+    using namespace sm100;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-    float* dh = reinterpret_cast<float*>(sm + AC_DH);
-    const uint8_t* pq = sm + AC_PQ;
-    const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(sm + AC_DO);
-    float* gam = reinterpret_cast<float*>(sm + AC_GAM);
-    const int tid = threadIdx.x, bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + AJ_BAR);
+    __shared__ uint32_t s_tmem;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
     const int NC = (p.T + C - 1) / C;
-    for (int idx = tid; idx < D * D; idx += AC_THREADS)
-        dh[(idx >> 7) * LDH + (idx & 127)] = p.dS ? p.dS[(size_t)bh * D * D + idx] : 0.f;
-#pragma unroll 1
-    for (int c = NC - 1; c >= 0; --c) {
-        const uint8_t* img = p.images + ((size_t)bh * NC + c) * kImgBytes;
-        __syncthreads();   // dh of this chunk is complete
-        float* dst = p.dh_all + ((size_t)bh * NC + c) * D * D;
-        for (int idx = tid; idx < D * D; idx += AC_THREADS) dst[idx] = dh[(idx >> 7) * LDH + (idx & 127)];
-        for (int idx = tid; idx < 2 * (int)kImgPQBlock / 16; idx += AC_THREADS)
-            reinterpret_cast<uint4*>(sm + AC_PQ)[idx] = __ldcg(reinterpret_cast<const uint4*>(img + kImgPQ) + idx);
-        if (tid < D) gam[tid] = __ldcg(reinterpret_cast<const float*>(img + kImgGam) + tid);
-        for (int idx = tid; idx < C * D / 8; idx += AC_THREADS) {   // dO tile, 8 values a load
-            const int r = idx >> 4, j = idx & 15, t = c * C + r;
-            uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            if (t < p.T) w = *reinterpret_cast<const uint4*>(
-                static_cast<const __nv_bfloat16*>(p.dO) + (((size_t)b * p.T + t) * p.H + h) * D + 8 * j);
-            reinterpret_cast<uint4*>(sm + AC_DO)[idx] = w;
-        }
-        __syncthreads();
-        // new dh[d'][v] = gamma_d' dh[d'][v] + sum_d Phi[d][d'] dh[d][v] + sum_r Qp[r][d'] dO[r][v]
-        float acc[4][8];
-        zero(acc);
-        gemm_acc<4, 8, 32, 16>(acc, D, tid,
-            [&](int dp, int d) {   // Phi^T: row d of Phi in the image, column d'
-                return bf(reinterpret_cast<const __nv_bfloat16*>(pq + (dp >> 6) * kImgPQBlock +
-                                                                 sw128_offset(d, dp & 63)));
-            },
-            [&](int d, int v) { return dh[d * LDH + v]; });
-        gemm_acc<4, 8, 32, 16>(acc, C, tid,
-            [&](int dp, int r) {   // Qp^T: row 128 + r of [Phi ; Qp], column d'
-                return bf(reinterpret_cast<const __nv_bfloat16*>(pq + (dp >> 6) * kImgPQBlock +
-                                                                 sw128_offset(128 + r, dp & 63)));
-            },
-            [&](int r, int v) { return __bfloat162float(dO[r * D + v]); });
-        const int tr = tid / 16, tc = tid % 16;
-        float keep[4][8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int dp = i * 32 + tr, v = j * 16 + tc;
-                keep[i][j] = fmaf(gam[dp], dh[dp * LDH + v], acc[i][j]);
-            }
-        __syncthreads();   // every thread has read dh
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) dh[(i * 32 + tr) * LDH + j * 16 + tc] = keep[i][j];
+    int failed = 0;
+    if (tid == 0) {
+        for (int i = 0; i < AJ_NBARS; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        prefetch_tmap(&maps.dO);
     }
+    if (warp == 1) {
+        tmem_alloc(&s_tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    if (p.dS0)
-        for (int idx = tid; idx < D * D; idx += AC_THREADS)
-            p.dS0[(size_t)bh * D * D + idx] = dh[(idx >> 7) * LDH + (idx & 127)];
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    auto wait = [&](int bar, uint32_t parity) {
+        if (!mbar_wait(&bars[bar], parity, &failed)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+    };
+    auto img = [&](int c) { return p.images + ((size_t)bh * NC + c) * kImgBytes; };
+
+    if (warp == 0) {
+        // =========================== loader (step j = chunk NC - 1 - j)
+#pragma unroll 1
+        for (int j = 0; j < NC; ++j) {
+            const int c = NC - 1 - j, s = j & 1;
+            if (j >= 2) wait(AJ_FREE0 + s, ((j - 2) >> 1) & 1);   // the MMA of step j - 2 is done
+            if (failed) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars[AJ_FULL0 + s], 2 * kImgPQBlock + 16384);
+                bulk_load(sm + AJ_PQ + s * 2 * kImgPQBlock, img(c) + kImgPQ, 2 * kImgPQBlock,
+                          &bars[AJ_FULL0 + s]);
+                for (int blk = 0; blk < 2; ++blk)
+                    tma_load_3d(sm + AJ_DO + s * 16384 + blk * 8192, &maps.dO, &bars[AJ_FULL0 + s],
+                                h * D + 64 * blk, c * C, b);
+                mbar_arrive_expect_tx(&bars[AJ_GAM0 + (j & 3)], 512);
+                bulk_load(sm + AJ_GAM + (j & 3) * 512, img(c) + kImgGam, 512, &bars[AJ_GAM0 + (j & 3)]);
+            }
+        }
+    } else if (warp == 1) {
+        // =========================== MMA issuer
+        const bool leader = lane == 0;
+        const uint32_t id_h = idesc_bf16_f32(128, 128, false, true);   // A in TMEM, B MN-major
+        const uint32_t id_o = idesc_bf16_f32(128, 128, true, true);    // A, B MN-major
+#pragma unroll 1
+        for (int j = 0; j < NC; ++j) {
+            const int s = j & 1;
+            wait(AJ_FULL0 + s, (j >> 1) & 1);
+            named_bar(AJ_BAR_H, 32 + 32 * AJ_NST);   // dh^T of step j is in TMEM
+            tc_fence_after();
+            if (leader && !failed) {
+                const uint32_t pq = sb + AJ_PQ + s * 2 * kImgPQBlock;
+                const uint32_t dO = sb + AJ_DO + s * 16384;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // dh^T Phi: K = d, rows d of Phi at 128 B
+                    mma_bf16_ta(tmem + AJ_TM_D + 128 * s, tmem + AJ_TM_H + 64 * s + 8 * k,
+                                sdesc_sw128(pq + k * 2048, kImgPQBlock, 1024), id_h, k > 0);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)   // dO^T Qp: K = r, Qp rows 128 + r
+                    mma_bf16(tmem + AJ_TM_D + 128 * s, sdesc_sw128(dO + k * 2048, 8192, 1024),
+                             sdesc_sw128(pq + 16384 + k * 2048, kImgPQBlock, 1024), id_o, true);
+                mma_commit(&bars[AJ_DONE0 + s]);
+                mma_commit(&bars[AJ_FREE0 + s]);
+            }
+            __syncwarp();
+        }
+        if (leader) mma_commit(&bars[AJ_FINAL]);
+        int f2 = 0;
+        if (!mbar_wait(&bars[AJ_FINAL], 0, &f2)) atomicOr(p.status, kStatusTimeout);
+        __syncwarp();
+    } else {
+        // =========================== state pass: dh^T row v, columns d = 32 cq ..
+        const int v = (warp & 3) * 32 + lane;
+        const int cq = (warp - AJ_ST) >> 2;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        float dh[32];
+        {
+            const float* src = p.dS ? p.dS + (size_t)bh * D * D + (size_t)(32 * cq) * D + v : nullptr;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) dh[e] = src ? __ldcg(src + (size_t)e * D) : 0.f;
+        }
+        // dh <- gamma_j (.) dh + D_j, once the product of step j is done
+        auto fold = [&](int j) {
+            wait(AJ_GAM0 + (j & 3), (j >> 2) & 1);
+            const float* gp = reinterpret_cast<const float*>(sm + AJ_GAM + (j & 3) * 512) + 32 * cq;
+            wait(AJ_DONE0 + (j & 1), (j >> 1) & 1);
+            tc_fence_after();
+            float x[32];
+            tmem_ld32(tmem + AJ_TM_D + 128 * (j & 1) + lane_off + 32 * cq, x);
+            tmem_wait_ld();
+            reg_fence(x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) dh[e] = fmaf(gp[e], dh[e], x[e]);
+        };
+#pragma unroll 1
+        for (int j = 0; j < NC; ++j) {
+            const int c = NC - 1 - j;
+            if (j > 0) fold(j - 1);
+            // the adjoint of chunk c's leaving state
+            float* dst = p.dh_all + ((size_t)bh * NC + c) * D * D + (size_t)(32 * cq) * D + v;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) dst[(size_t)e * D] = dh[e];
+            float pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                __nv_bfloat162 t2 = __floats2bfloat162_rn(dh[2 * e], dh[2 * e + 1]);
+                pk[e] = __uint_as_float(*reinterpret_cast<uint32_t*>(&t2));
+            }
+            tmem_st16(tmem + AJ_TM_H + 64 * (j & 1) + 16 * cq + lane_off, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            named_bar_arrive(AJ_BAR_H, 32 + 32 * AJ_NST);
+        }
+        if (NC > 0) fold(NC - 1);
+        if (p.dS0) {
+            float* dst = p.dS0 + (size_t)bh * D * D + (size_t)(32 * cq) * D + v;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) dst[(size_t)e * D] = dh[e];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
 }
 
 // --------------------------------------------------------- chunk backward
@@ -625,10 +726,18 @@ cudaError_t launch_chunk_bwd(const ChunkParams& pf, const BwdParams& pb0, int ga
     *launches += nf;
     if (e != cudaSuccess) return e;
     // 2. the adjoint state, chunks from the last back
+    AdjMaps am;
+    memset(&am, 0, sizeof(am));
+    {
+        const uint64_t dims[3] = {(uint64_t)pf.H * D, (uint64_t)pf.T, (uint64_t)pf.B};
+        const uint64_t strides[2] = {(uint64_t)pf.H * D * 2, (uint64_t)pf.T * pf.H * D * 2};
+        const uint32_t box[3] = {64, 64, 1};
+        if (!make_tmap_bf16(&am.dO, pb.dO, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
     e = cudaFuncSetAttribute(adjoint_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)AC_SMEM);
+                             (int)AJ_SMEM);
     if (e != cudaSuccess) return e;
-    e = launch_on(adjoint_chain_kernel, dim3((unsigned)nbh), dim3(AC_THREADS), AC_SMEM, s, pb);
+    e = launch_on(adjoint_chain_kernel, dim3((unsigned)nbh), dim3(AJ_THREADS), AJ_SMEM, s, am, pb);
     if (e != cudaSuccess) return e;
     ++*launches;
     // 3. every chunk's gradients

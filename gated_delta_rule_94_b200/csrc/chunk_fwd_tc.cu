@@ -116,12 +116,6 @@ __device__ __forceinline__ void l2_discard(const void* p, uint32_t bytes, int la
         asm volatile("discard.global.L2 [%0], 128;" ::"l"(c + off) : "memory");
 }
 
-__device__ __forceinline__ void named_bar(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-__device__ __forceinline__ void named_bar_arrive(int id, int count) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 template <int N>
 __device__ __forceinline__ void ld_cols(uint32_t addr, float (&v)[N]) {
@@ -1030,17 +1024,6 @@ struct ChainMaps {
     CUtensorMap seg;   // [2][B*H][nseg][D][D] segment offsets then transitions (segment mode 1)
 };
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, A from tensor memory (row m in lane m, k
-// pairs packed two bf16 to a 32-bit column, 8 columns a k-step of 16).
-__device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, bool accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
-        : "memory");
-}
 
 // Element (d, v) of the final state staged as four TMA boxes of [128 d][32 v]
 // fp32 (128-byte swizzle), box v / 32.

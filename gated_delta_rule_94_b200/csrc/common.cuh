@@ -71,6 +71,7 @@ struct BwdParams {
     const uint8_t* images;   // the forward's step images, [B*H][NC]
     float* h_all;        // entering state of every chunk
     float* dh_all;       // adjoint of every chunk's leaving state
+    unsigned* status;    // device status word (a bounded wait that gave up)
     int B, T, H;
 };
 

@@ -300,6 +300,7 @@ gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const void
     pb.q = q; pb.k = k; pb.v = v; pb.beta = beta; pb.g = g; pb.dO = d_o; pb.dS = d_final_state;
     pb.dq = dq; pb.dk = dk; pb.dv = dv; pb.dbeta = dbeta; pb.dg = dg; pb.dS0 = d_initial_state;
     pb.B = B; pb.T = T; pb.H = H;
+    pb.status = pf.status;
     int launches = 0;
     const cudaError_t e = gdn::launch_chunk_bwd(pf, pb, gate_kind,
                                                 static_cast<uint8_t*>(workspace), workspace_bytes,
