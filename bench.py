@@ -598,8 +598,12 @@ def time_osdn(ctx: Ctx):
     nws = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, Dk, Dv, 64, torch.bfloat16, w.gate_kind)
     ws = torch.empty(nws, dtype=torch.uint8, device=ctx.dev)
 
+    ws1 = torch.empty(gdn.gdn_osdn_precondition_workspace_bytes(B, T, H, Dk), dtype=torch.uint8,
+                      device=ctx.dev)
+
     def phase1():
-        gdn.gdn_osdn_precondition(d["k"], d["beta"], r, 0.5, None, kw, d1, stream=ctx.stream)
+        gdn.gdn_osdn_precondition(d["k"], d["beta"], r, 0.5, None, kw, d1, workspace=ws1,
+                                  stream=ctx.stream)
 
     def both():
         phase1()
@@ -634,14 +638,15 @@ def time_osdn(ctx: Ctx):
                "kind": "oracle", "sample": f"{Hs} heads x {Ts} tokens of one sequence, both "
                                           f"phases, {reps} runs, {total:.1f} s; tokens/s = "
                                           f"token-heads/s / {H} heads"}
-    del d, r, kw, d1, o, S, ws
+    del d, r, kw, d1, o, S, ws, ws1
     torch.cuda.empty_cache()
     return {
         "workload": f"preconditioned delta rule (eta 0.5, retention gate), {w.name}",
         "ms_per_step": ms, "ms_min": ms_min, "tokens_per_s": B * T / (ms * 1e-3),
         "phase1_ms": ms1,
-        "phase1_roofline": hbm_roofline(ctx, b1, ms1, "osdn_precondition_kernel"),
-        "roofline": hbm_roofline(ctx, b1 + b2, ms, "osdn_precondition_kernel + chunk_prep_kernel,"
+        "phase1_roofline": hbm_roofline(ctx, b1, ms1, "osdn_block_kernel, osdn_chain_kernel, "
+                                                      "osdn_write_kernel"),
+        "roofline": hbm_roofline(ctx, b1 + b2, ms, "osdn_block_kernel, osdn_chain_kernel, osdn_write_kernel + chunk_prep_kernel,"
                                                    "chunk_chain_kernel (both phases)"),
         "gpu_launches_per_step": launches, "cpu_baseline": cpu,
     }

@@ -27,7 +27,8 @@ EXPORTED = ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_chunk_fwd_wor
             "gdn_read_device_status", "gdn_status_string", "gdn_abi_version",
             "gdn_kernel_launch_count", "gdn_chunk_fwd_kernel_name", "gdn_chunk_fwd_noalloc",
             "gdn_chunk_fwd_noalloc_scratch_bytes", "gdn_osdn_precondition", "gdn_chunk_fwd_wk",
-            "gdn_chunk_fwd_plan", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes")
+            "gdn_chunk_fwd_plan", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes",
+            "gdn_osdn_precondition_workspace_bytes")
 
 _lib = None
 
@@ -71,8 +72,10 @@ def load() -> ctypes.CDLL:
     lib.gdn_chunk_fwd_noalloc_scratch_bytes.argtypes = []
     lib.gdn_chunk_fwd_noalloc_scratch_bytes.restype = sz
     lib.gdn_osdn_precondition.argtypes = [vp, vp, vp, ctypes.c_float, vp, vp, vp, i, i, i, i, i,
-                                          vp]
+                                          vp, sz, vp]
     lib.gdn_osdn_precondition.restype = i
+    lib.gdn_osdn_precondition_workspace_bytes.argtypes = [i, i, i, i]
+    lib.gdn_osdn_precondition_workspace_bytes.restype = sz
     lib.gdn_chunk_fwd_wk.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, vp,
                                      sz, vp]
     lib.gdn_chunk_fwd_wk.restype = i
@@ -219,10 +222,19 @@ def gdn_chunk_fwd_wk(q, k, k_write, v, beta, g, gate_kind, initial_state, o, fin
         raise GdnError(st, "gdn_chunk_fwd_wk")
 
 
-def gdn_osdn_precondition(k, beta, r, eta, d0, k_write, d_final, *, stream=None) -> None:
+def gdn_osdn_precondition_workspace_bytes(B, T, H, Dk) -> int:
+    n = load().gdn_osdn_precondition_workspace_bytes(B, T, H, Dk)
+    if n == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_INVALID_ARG, "gdn_osdn_precondition_workspace_bytes")
+    return n
+
+
+def gdn_osdn_precondition(k, beta, r, eta, d0, k_write, d_final, *, workspace=None,
+                          stream=None) -> None:
     """Phase 1 of the preconditioned delta rule: write keys k_write = d (.) k.
     k, k_write [B,T,H,Dk]; beta, r [B,T,H] (r may be None); d0, d_final
-    [B,H,Dk] fp32 or None."""
+    [B,H,Dk] fp32 or None; workspace a uint8 device tensor (allocated here
+    with torch when None)."""
     _check_contig(k=k, beta=beta, r=r, d0=d0, k_write=k_write, d_final=d_final)
     B, T, H, Dk = k.shape
     dt = _dtype_code(k.dtype)
@@ -232,9 +244,13 @@ def gdn_osdn_precondition(k, beta, r, eta, d0, k_write, d_final, *, stream=None)
     for name, t in (("d0", d0), ("d_final", d_final)):
         if t is not None and t.dtype != torch.float32:
             raise TypeError(f"{name} must be float32")
+    if workspace is None:
+        n = gdn_osdn_precondition_workspace_bytes(B, T, H, Dk)
+        workspace = torch.empty(n, dtype=torch.uint8, device=k.device) if n else None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = load().gdn_osdn_precondition(_ptr(k), _ptr(beta), _ptr(r), float(eta), _ptr(d0),
                                       _ptr(k_write), _ptr(d_final), B, T, H, Dk, dt,
-                                      _stream(stream))
+                                      _ptr(workspace), ws_bytes, _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_osdn_precondition")
 

@@ -128,7 +128,11 @@ cudaError_t launch_chunk_fwd_tc(const ChunkParams& p, int gate, size_t ws_bytes,
                                 int* launches);
 cudaError_t launch_decode_step(const DecodeParams& p, int Dk, int Dv, int gate, bool bf16,
                                cudaStream_t s);
-cudaError_t launch_osdn_precondition(const OsdnParams& p, int Dk, bool bf16, cudaStream_t s);
+// Phase 1 of the preconditioned delta rule in blocks of 64 tokens (three
+// launches); ws holds osdn_precondition_workspace_bytes(B, T, H, Dk).
+size_t osdn_precondition_workspace_bytes(int B, int T, int H, int Dk);
+cudaError_t launch_osdn_precondition(const OsdnParams& p, int Dk, bool bf16, uint8_t* ws,
+                                     cudaStream_t s, int* launches);
 // The forward in one wave, keeping every chunk's step image in ws (at offset 0,
 // [B*H][NC] images) and every chunk's entering state in h_all.  ws_bytes >=
 // chunk_fwd_tc_capture_bytes.

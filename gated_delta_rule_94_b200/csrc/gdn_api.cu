@@ -309,9 +309,15 @@ gdn_status gdn_chunk_bwd(const void* q, const void* k, const void* v, const void
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+size_t gdn_osdn_precondition_workspace_bytes(int B, int T, int H, int Dk) {
+    if (B < 0 || T < 0 || H < 0 || !supported_dim(Dk)) return (size_t)-1;
+    return gdn::osdn_precondition_workspace_bytes(B, T, H, Dk);
+}
+
 gdn_status gdn_osdn_precondition(const void* k, const void* beta, const void* r, float eta,
                                  const float* d0, void* k_write, float* d_final, int B, int T,
-                                 int H, int Dk, gdn_dtype dtype, gdn_stream_t stream) {
+                                 int H, int Dk, gdn_dtype dtype, void* workspace,
+                                 size_t workspace_bytes, gdn_stream_t stream) {
     if (B < 0 || T < 0 || H < 0) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
     if (!(eta == eta) || eta > 3.0e38f || eta < -3.0e38f) return GDN_ERR_INVALID_ARG;
@@ -319,12 +325,18 @@ gdn_status gdn_osdn_precondition(const void* k, const void* beta, const void* r,
     if ((int64_t)B * T > INT32_MAX || (int64_t)B * H > INT32_MAX) return GDN_ERR_UNSUPPORTED;
     if (B == 0 || H == 0) return GDN_OK;
     if (T > 0 && (!k || !beta || !k_write)) return GDN_ERR_INVALID_ARG;
-    const void* ptrs[] = {k, beta, r, d0, k_write, d_final};
+    const void* ptrs[] = {k, beta, r, d0, k_write, d_final, workspace};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
     const size_t es = elem_size(dtype);
     const size_t ntok = (size_t)B * T * H;
     const size_t dbytes = (size_t)B * H * Dk * sizeof(float);
+    const size_t need = gdn::osdn_precondition_workspace_bytes(B, T, H, Dk);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
+    const void* others[] = {k, beta, r, d0, k_write, d_final};
+    const size_t othern[] = {ntok * Dk * es, ntok * es, ntok * es, dbytes, ntok * Dk * es, dbytes};
+    for (int i = 0; i < 6; ++i)
+        if (overlaps(workspace, need, others[i], othern[i])) return GDN_ERR_INVALID_ARG;
     if (overlaps(k_write, ntok * Dk * es, k, ntok * Dk * es) ||
         overlaps(k_write, ntok * Dk * es, beta, ntok * es) ||
         overlaps(k_write, ntok * Dk * es, r, ntok * es) ||
@@ -340,10 +352,12 @@ gdn_status gdn_osdn_precondition(const void* k, const void* beta, const void* r,
     gdn::OsdnParams p;
     p.k = k; p.beta = beta; p.r = r; p.kw = k_write; p.d0 = d0; p.d_out = d_final;
     p.eta = eta; p.B = B; p.T = T; p.H = H;
+    int launches = 0;
     cudaError_t e = gdn::launch_osdn_precondition(p, Dk, dtype == GDN_BF16,
-                                                  reinterpret_cast<cudaStream_t>(stream));
+                                                  static_cast<uint8_t*>(workspace),
+                                                  reinterpret_cast<cudaStream_t>(stream), &launches);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
-    g_launches.fetch_add(1);
+    g_launches.fetch_add((unsigned long long)launches);
     return GDN_OK;
 }
 

@@ -195,12 +195,24 @@ GDN_API gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
  *   d_final  [B, H, Dk] fp32 final preconditioner (output) or NULL; may be
  *            the same pointer as d0
  *   Dk       64 or 128;  dtype GDN_BF16 or GDN_F32 (fp32 arithmetic either way)
- * The scan is sequential in t (a 4-lane group per (batch, head)).
+ *   workspace, workspace_bytes: caller-owned device scratch of at least
+ *            gdn_osdn_precondition_workspace_bytes(B, T, H, Dk) bytes (16-byte
+ *            aligned, clear of every other argument); NULL / 0 when that is 0;
+ *            less returns GDN_ERR_WORKSPACE before any launch.
+ * The scan runs in blocks of 64 tokens: the step e_t = eta beta_t (1 - beta_t
+ * s_t) / n_t is affine in s_t = <d_t, k_t^2>, so a block entering with d
+ * solves a unit lower-triangular system through the Gram matrix of the k_t^2
+ * (formed for every block at once); only a short pass per (batch, head) runs
+ * the blocks in order (three launches).  Results equal the token-by-token scan
+ * up to fp32 rounding.
  */
 GDN_API gdn_status gdn_osdn_precondition(const void* k, const void* beta, const void* r,
                                          float eta, const float* d0, void* k_write,
                                          float* d_final, int B, int T, int H, int Dk,
-                                         gdn_dtype dtype, gdn_stream_t stream);
+                                         gdn_dtype dtype, void* workspace,
+                                         size_t workspace_bytes, gdn_stream_t stream);
+/* Workspace of gdn_osdn_precondition (bytes; (size_t)-1 for invalid sizes). */
+GDN_API size_t gdn_osdn_precondition_workspace_bytes(int B, int T, int H, int Dk);
 
 /*
  * gdn_chunk_fwd_wk -- gdn_chunk_fwd with a separate write key (phase 2 of the

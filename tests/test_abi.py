@@ -202,12 +202,12 @@ def test_chunk_fwd_wk_without_write_key_is_chunk_fwd():
 
 def osdn_call(**over):
     args = dict(k=A, beta=A * 2, r=None, eta=0.5, d0=None, kw=A * 4, d1=None, B=1, T=64, H=1,
-                Dk=128, dtype=0, stream=None)
+                Dk=128, dtype=0, ws=A * 8, ws_bytes=1 << 20, stream=None)
     args.update(over)
     return _lib.load().gdn_osdn_precondition(args["k"], args["beta"], args["r"], args["eta"],
                                              args["d0"], args["kw"], args["d1"], args["B"],
                                              args["T"], args["H"], args["Dk"], args["dtype"],
-                                             args["stream"])
+                                             args["ws"], args["ws_bytes"], args["stream"])
 
 
 @pytest.mark.parametrize("over,code", [
@@ -224,6 +224,10 @@ def osdn_call(**over):
     (dict(d1=A * 4), _lib.GDN_ERR_INVALID_ARG),               # final d over the write keys
     (dict(d0=A * 1024, d1=A * 1024 + 16), _lib.GDN_ERR_INVALID_ARG),   # partial d overlap
     (dict(B=65536, T=65536), _lib.GDN_ERR_UNSUPPORTED),
+    (dict(ws=None), _lib.GDN_ERR_WORKSPACE),
+    (dict(ws_bytes=1024), _lib.GDN_ERR_WORKSPACE),            # below one block's 18 KB
+    (dict(ws=A), _lib.GDN_ERR_INVALID_ARG),                   # workspace over the keys
+    (dict(ws=A * 8 + 8), _lib.GDN_ERR_INVALID_ARG),           # misaligned workspace
 ])
 def test_osdn_precondition_argument_errors(over, code):
     assert osdn_call(**over) == code
