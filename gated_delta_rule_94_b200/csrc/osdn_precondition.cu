@@ -102,7 +102,7 @@ osdn_block_kernel(const OsdnParams p, uint8_t* ws) {
     float* us = smf;                          // u [L][DK + 1]
     float* Lm = us + L * (DK + 1);            // Lm [L][LDL]
     float* Rm = Lm + L * LDL;                 // R_{j->t} [L][LDL]
-    float* sv = Rm + L * LDL;                 // a, c, r [L] each
+    float* sv = Rm + L * LDL;                 // a, c, r [L] each, then a [32][33] scratch
     float* sa = sv, *sc = sv + L, *sr = sv + 2 * L;
     const int NB = (p.T + L - 1) / L;
     const long long q = blockIdx.x;
@@ -164,8 +164,8 @@ osdn_block_kernel(const OsdnParams p, uint8_t* ws) {
 #pragma unroll
             for (int a = 0; a < 4; ++a)
 #pragma unroll
-                for (int bb = 0; bb < 4; ++bb) g[a][bb] = fmaf(ut[a], uj[bb], g[a][bb]);
-        }
+                for (int bb = 0; bb <= a; ++bb) g[a][bb] = fmaf(ut[a], uj[bb], g[a][bb]);
+        }   // (tiles above the diagonal, bb > a, are never used)
         __syncthreads();   // R_{j->t} is complete
         // Lm_tj = c_t R_{j->t} <u_j, u_t> for j < t
 #pragma unroll
@@ -177,24 +177,75 @@ osdn_block_kernel(const OsdnParams p, uint8_t* ws) {
             }
     }
     __syncthreads();
-    // T = (I + Lm)^-1, one column a thread (left-looking substitution)
+    // T = (I + Lm)^-1 in blocks (R_{j->t} is dead: Ts takes its place):
+    // (1) the four 16 x 16 diagonal inverses by substitution, one column a
+    // thread; (2) 16 -> 32: T_10 = -D_1 (Lm_10 D_0) for the two 32 x 32
+    // diagonal blocks; (3) 32 -> 64 the same with 32 x 32 blocks.  Every sum
+    // runs over the lower-triangular parts only.
+    float* Ts = Rm;
     if (tid < L) {
-        const int col = tid;
-        float x[L];
+        const int o = 16 * (tid >> 4), c = tid & 15;
+        float pr[16], x[16];
 #pragma unroll
-        for (int r = 0; r < L; ++r) x[r] = 0.f;
-        x[col] = 1.f;
+        for (int r = 0; r < 16; ++r) pr[r] = 0.f;
 #pragma unroll
-        for (int r = 1; r < L; ++r) {
-            if (r > col) {
-                float acc = 0.f;
+        for (int i = 0; i < 16; ++i) {
+            x[i] = (i == c) ? 1.f : (i < c ? 0.f : -pr[i]);
 #pragma unroll
-                for (int i = 0; i < r; ++i) acc = fmaf(Lm[r * LDL + i], x[i], acc);
-                x[r] = -acc;
-            }
+            for (int r = i + 1; r < 16; ++r) pr[r] = fmaf(Lm[(o + r) * LDL + o + i], x[i], pr[r]);
         }
 #pragma unroll
-        for (int r = 0; r < L; ++r) w.T[r * L + col] = x[r];
+        for (int r = 0; r < 16; ++r) Ts[(o + r) * LDL + o + c] = x[r];
+    }
+    __syncthreads();
+    float* Xs = sv + 3 * L;   // scratch [32][33]
+    {   // (2): pair pp of diagonal blocks (2 pp + 1, 2 pp); thread: row r, columns c0, c0 + 1
+        const int pp = tid >> 7, idx = tid & 127, r = idx >> 3, c0 = 2 * (idx & 7);
+        const int ri = 32 * pp + 16, cj = 32 * pp;
+        float x0 = 0.f, x1 = 0.f;
+        for (int i = c0; i < 16; ++i) {
+            const float lm = Lm[(ri + r) * LDL + cj + i];
+            x0 = fmaf(lm, Ts[(cj + i) * LDL + cj + c0], x0);
+            if (i > c0) x1 = fmaf(lm, Ts[(cj + i) * LDL + cj + c0 + 1], x1);
+        }
+        Xs[(16 * pp + r) * 33 + c0] = x0;
+        Xs[(16 * pp + r) * 33 + c0 + 1] = x1;
+        __syncthreads();
+        float t0 = 0.f, t1 = 0.f;
+        for (int i = 0; i <= r; ++i) {
+            const float d1 = Ts[(ri + r) * LDL + ri + i];
+            t0 = fmaf(d1, Xs[(16 * pp + i) * 33 + c0], t0);
+            t1 = fmaf(d1, Xs[(16 * pp + i) * 33 + c0 + 1], t1);
+        }
+        Ts[(ri + r) * LDL + cj + c0] = -t0;
+        Ts[(ri + r) * LDL + cj + c0 + 1] = -t1;
+    }
+    __syncthreads();
+    {   // (3): thread: row r of the 32 x 32 block, columns c0 .. c0 + 3
+        const int r = tid >> 3, c0 = 4 * (tid & 7);
+        float xv[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int i = c0; i < 32; ++i) {
+            const float lm = Lm[(32 + r) * LDL + i];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (i >= c0 + q) xv[q] = fmaf(lm, Ts[i * LDL + c0 + q], xv[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) Xs[r * 33 + c0 + q] = xv[q];
+        __syncthreads();
+        float tv[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int i = 0; i <= r; ++i) {
+            const float t11 = Ts[(32 + r) * LDL + 32 + i];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tv[q] = fmaf(t11, Xs[i * 33 + c0 + q], tv[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) Ts[(32 + r) * LDL + c0 + q] = -tv[q];
+    }
+    __syncthreads();
+    for (int idx = tid; idx < L * L; idx += OB_THREADS) {   // lower triangle, zeros above
+        const int r = idx >> 6, cc = idx & 63;
+        w.T[idx] = cc <= r ? Ts[r * LDL + cc] : 0.f;
     }
     // vectors: R_t = prod_{i<t} r_i, cR_t = c_t R_t, rho_j = prod_{j<i<L} r_i, R_L
     if (tid == 64) {
@@ -371,17 +422,23 @@ osdn_write_kernel(const OsdnParams p, uint8_t* ws) {
     for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int cc = 0; cc < NCOL; ++cc) acc[a][cc] = sR[16 * a + tr] * sd[16 * cc + tc];
+    // M is strictly lower triangular: the 16 columns j of segment js reach
+    // only the row tiles a >= js
+#pragma unroll
+    for (int js = 0; js < 4; ++js) {
 #pragma unroll 4
-    for (int j = 0; j < L; ++j) {
-        float m[4], uj[NCOL];
+        for (int jj = 0; jj < 16; ++jj) {
+            const int j = 16 * js + jj;
+            float m[4], uj[NCOL];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) m[a] = Ms[(16 * a + tr) * LDL + j];
+            for (int a = js; a < 4; ++a) m[a] = Ms[(16 * a + tr) * LDL + j];
 #pragma unroll
-        for (int cc = 0; cc < NCOL; ++cc) uj[cc] = us[j * (DK + 1) + 16 * cc + tc];
+            for (int cc = 0; cc < NCOL; ++cc) uj[cc] = us[j * (DK + 1) + 16 * cc + tc];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+            for (int a = js; a < 4; ++a)
 #pragma unroll
-            for (int cc = 0; cc < NCOL; ++cc) acc[a][cc] = fmaf(m[a], uj[cc], acc[a][cc]);
+                for (int cc = 0; cc < NCOL; ++cc) acc[a][cc] = fmaf(m[a], uj[cc], acc[a][cc]);
+        }
     }
     const Tin* kp = static_cast<const Tin*>(p.k);
     Tin* kwp = static_cast<Tin*>(p.kw);
@@ -400,7 +457,7 @@ template <typename Tin, int DK>
 cudaError_t launch_dk(const OsdnParams& p, uint8_t* ws, cudaStream_t s) {
     const long long nbh = (long long)p.B * p.H;
     const int NB = (p.T + L - 1) / L;
-    const size_t sm_block = ((size_t)L * (DK + 1) + 2 * (size_t)L * LDL + 3 * L) * 4;
+    const size_t sm_block = ((size_t)L * (DK + 1) + 2 * (size_t)L * LDL + 3 * L + 32 * 33) * 4;
     const size_t sm_chain = chain_smem<Tin, DK>();
     const size_t sm_write = ((size_t)L * (DK + 1) + (size_t)L * LDL + 3 * L + DK) * 4;
     cudaError_t e;
