@@ -91,19 +91,40 @@ __global__ void __launch_bounds__(NT) chunk_fwd_simt_kernel(ChunkParams p) {
     for (int t0 = 0; t0 < T; t0 += C) {
         const int n = min(C, T - t0);
         __syncthreads();
-        // ---- load the chunk (rows >= n are zero, beta = 0, g = 0)
-        for (int idx = tid; idx < C * DK; idx += NT) {
-            const int r = idx / DK, d = idx % DK;
-            const size_t tok = ((size_t)b * T + t0 + r) * H + h;
-            const bool ok = r < n;
-            Ks[r * LD + d] = ok ? to_f32(k[tok * DK + d]) : 0.f;
-            Qs[r * LD + d] = ok ? to_f32(q[tok * DK + d]) : 0.f;
-            if constexpr (GATE == kGatePerDim) Gs[r * LD + d] = ok ? to_f32(g[tok * DK + d]) : 0.f;
-        }
-        for (int idx = tid; idx < C * BV; idx += NT) {
-            const int r = idx / BV, c = idx % BV;
-            const size_t tok = ((size_t)b * T + t0 + r) * H + h;
-            Vs[r * (BV + 1) + c] = r < n ? to_f32(v[tok * Dv + v0 + c]) : 0.f;
+        // ---- load the chunk (rows >= n are zero, beta = 0, g = 0); every load
+        // of a thread is issued before the first is stored, so the chunk costs
+        // one memory latency rather than one per element
+        {
+            constexpr int PK = C * DK / NT, PV = C * BV / NT;
+            static_assert(C * DK % NT == 0 && C * BV % NT == 0, "whole rounds");
+            float kv[PK], qv[PK], gv[GATE == kGatePerDim ? PK : 1], vv[PV];
+#pragma unroll
+            for (int m = 0; m < PK; ++m) {
+                const int idx = tid + m * NT, r = idx / DK, d = idx % DK;
+                const size_t tok = ((size_t)b * T + t0 + r) * H + h;
+                const bool ok = r < n;
+                kv[m] = ok ? to_f32(k[tok * DK + d]) : 0.f;
+                qv[m] = ok ? to_f32(q[tok * DK + d]) : 0.f;
+                if constexpr (GATE == kGatePerDim) gv[m] = ok ? to_f32(g[tok * DK + d]) : 0.f;
+            }
+#pragma unroll
+            for (int m = 0; m < PV; ++m) {
+                const int idx = tid + m * NT, r = idx / BV, c = idx % BV;
+                const size_t tok = ((size_t)b * T + t0 + r) * H + h;
+                vv[m] = r < n ? to_f32(v[tok * Dv + v0 + c]) : 0.f;
+            }
+#pragma unroll
+            for (int m = 0; m < PK; ++m) {
+                const int idx = tid + m * NT, r = idx / DK, d = idx % DK;
+                Ks[r * LD + d] = kv[m];
+                Qs[r * LD + d] = qv[m];
+                if constexpr (GATE == kGatePerDim) Gs[r * LD + d] = gv[m];
+            }
+#pragma unroll
+            for (int m = 0; m < PV; ++m) {
+                const int idx = tid + m * NT, r = idx / BV, c = idx % BV;
+                Vs[r * (BV + 1) + c] = vv[m];
+            }
         }
         if (tid < C) {
             const size_t tok = ((size_t)b * T + t0 + tid) * H + h;
