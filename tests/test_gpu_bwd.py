@@ -66,3 +66,29 @@ def test_bwd_deterministic():
         # the bit (the first token's dg is a sum over the whole chunk that nearly
         # cancels)
         check(key, a[key], b[key].double().cpu().numpy(), 1e-5)
+
+
+def test_bwd_gdn_workload_sampled_heads():
+    """The bench's backward record, B4 H16 T2048 (scalar gate): every head runs
+    on the GPU; two whole (sequence, head) pairs -- heads are independent --
+    against the oracle's chunkwise backward (pinned to autograd of the token
+    loop in test_backward_oracle)."""
+    w = gi.WORKLOADS[1]
+    x = gi.workload_inputs(w)
+    gen = torch.Generator().manual_seed(11)
+    dO = torch.randn(w.B, w.T, w.H, 128, generator=gen).to(torch.bfloat16)
+    dS = 0.02 * torch.randn(w.B, w.H, 128, 128, generator=gen)
+    d = to_dev(x)
+    gr = gdn.chunk_bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], dO.cuda(), dS.cuda())
+    torch.cuda.synchronize()
+    f = gi.to_f64_numpy(x)
+    tol = TOL[torch.bfloat16]
+    for b, h in ((0, 0), (3, 15)):
+        sl = lambda a: None if a is None else np.ascontiguousarray(a[b:b + 1, :, h:h + 1])
+        ref = oracle.chunk_backward(sl(f["q"]), sl(f["k"]), sl(f["v"]), sl(f["beta"]), sl(f["g"]),
+                                    x["gate_kind"], None, dO[b:b + 1, :, h:h + 1].double().numpy(),
+                                    dS[b:b + 1, h:h + 1].double().numpy())
+        for name, key in (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dbeta", "dbeta"),
+                          ("dg", "dg")):
+            check(f"{name}[{b},{h}]", gr[name][b:b + 1, :, h:h + 1], ref[key], tol)
+        check(f"dS0[{b},{h}]", gr["d_initial_state"][b:b + 1, h:h + 1], ref["dS0"], tol)

@@ -73,3 +73,17 @@ def test_segments_with_write_key():
                                        x["gate_kind"], f["S0"])
     check("o", o, o_ref, TOL[torch.bfloat16])
     check("S", S, S_ref, TOL[torch.bfloat16])
+
+
+def test_segments_few_head_long_sequence_workload():
+    """The bench's segment record, B1 H4 T65536 (scalar gate, the long-sequence
+    recipe) with the full-speed workspace: three waves of 18 segments; every
+    head against the oracle."""
+    x = gi.make_inputs(1, 65536, 4, 128, 128, dtype=torch.bfloat16, gate="scalar", seed=0)
+    plan = gdn.gdn_chunk_fwd_plan(1, 65536, 4, 128, 128, 64, torch.bfloat16, x["gate_kind"])
+    assert plan["segments"] > 1 and plan["waves"] > 1
+    o, S = run(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check("o", o, o_ref, TOL[torch.bfloat16])
+    check("S", S, S_ref, TOL[torch.bfloat16])
+    assert gdn.gdn_read_device_status() == 0
