@@ -44,48 +44,74 @@ constexpr int D = 128;
 constexpr int C = 64;
 
 
-// C[m][n] (+)= sum_k a(m, k) b(k, n) for an output tile of (RM * TR) x (RN * TC)
-// on TR x TC threads: thread (tr, tc) owns rows i * TR + tr and columns
-// j * TC + tc (strided, so that a warp's 16 column threads read 16 consecutive
-// words of a row of b).  acc is the thread's accumulator (kept by the caller
-// across calls when the same output is summed over several products).
-template <int RM, int RN, int TR, int TC, typename FA, typename FB>
-__device__ __forceinline__ void gemm_acc(float (&acc)[RM][RN], int K, int tid, FA a, FB b) {
-    const int tr = tid / TC, tc = tid % TC;
+// Warp MMAs on tf32 operands with fp32 accumulation (m16n8k8).  A 64 x N
+// output is split over the 8 warps: row strip 16 (w % 4), column half
+// (N / 2) (w / 4); lane (g = lane / 4, t = lane % 4) holds, for n-tile j,
+// rows r0 + g and r0 + g + 8 and columns c0 + 8 j + 2 t and + 1 (element e of
+// acc[j]: row r0 + g + 8 (e / 2), column c0 + 8 j + 2 t + e % 2).  Operands
+// are read through accessors a(row, k), b(k, col) from shared memory.
+__device__ __forceinline__ uint32_t tf32_of(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_16x8x8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                           uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+struct Frag {
+    int r0, c0, g, t;
+    __device__ int row(int e) const { return r0 + g + 8 * (e >> 1); }
+    __device__ int col(int j, int e) const { return c0 + 8 * j + 2 * t + (e & 1); }
+};
+__device__ __forceinline__ Frag frag_of(int warp, int lane, int N) {
+    return Frag{16 * (warp & 3), (N / 2) * (warp >> 2), lane >> 2, lane & 3};
+}
+// acc (+)= A B over K (a multiple of 8)
+template <int NT, typename FA, typename FB>
+__device__ __forceinline__ void mma_acc(float (&acc)[NT][4], int K, const Frag& f, FA a, FB b) {
 #pragma unroll 2
-    for (int kk = 0; kk < K; ++kk) {
-        float av[RM], bv[RN];
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = tf32_of(a(f.r0 + f.g, k0 + f.t));
+        const uint32_t a1 = tf32_of(a(f.r0 + f.g + 8, k0 + f.t));
+        const uint32_t a2 = tf32_of(a(f.r0 + f.g, k0 + f.t + 4));
+        const uint32_t a3 = tf32_of(a(f.r0 + f.g + 8, k0 + f.t + 4));
 #pragma unroll
-        for (int i = 0; i < RM; ++i) av[i] = a(i * TR + tr, kk);
-#pragma unroll
-        for (int j = 0; j < RN; ++j) bv[j] = b(kk, j * TC + tc);
-#pragma unroll
-        for (int i = 0; i < RM; ++i)
-#pragma unroll
-            for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < NT; ++j) {
+            const int col = f.c0 + 8 * j + f.g;
+            mma_16x8x8(acc[j], a0, a1, a2, a3, tf32_of(b(k0 + f.t, col)), tf32_of(b(k0 + f.t + 4, col)));
+        }
     }
 }
-
-// Reductions before a shared-memory atomic, for the 16 x 16 thread layout
-// (thread = 16 row threads x 16 column threads; lanes 0-15 of a warp share a
-// row thread, lanes 16-31 the next): the sum over the 16 lanes of a row, added
-// by one lane; the sum over the two row threads of a warp, added by one lane.
-__device__ __forceinline__ void row_add(float* dst, float val, int lane) {
+template <int NT>
+__device__ __forceinline__ void zero(float (&acc)[NT][4]) {
 #pragma unroll
-    for (int off = 1; off < 16; off <<= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
-    if ((lane & 15) == 0) atomicAdd(dst, val);
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 }
-__device__ __forceinline__ void col_add(float* dst, float val, int lane) {
-    val += __shfl_xor_sync(0xffffffffu, val, 16);
-    if (lane < 16) atomicAdd(dst, val);
+// Sums before a shared-memory atomic: over the four lanes (t) that share a
+// row of the fragment (s_lo for row r0 + g, s_hi for row r0 + g + 8), and over
+// the eight lanes (g) that share a column.
+__device__ __forceinline__ void frag_row_add(float* dst, const Frag& f, float s_lo, float s_hi) {
+    s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 1);
+    s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 2);
+    s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 1);
+    s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 2);
+    if (f.t == 0) {
+        atomicAdd(dst + f.r0 + f.g, s_lo);
+        atomicAdd(dst + f.r0 + f.g + 8, s_hi);
+    }
 }
-
-template <int RM, int RN>
-__device__ __forceinline__ void zero(float (&acc)[RM][RN]) {
-#pragma unroll
-    for (int i = 0; i < RM; ++i)
-#pragma unroll
-        for (int j = 0; j < RN; ++j) acc[i][j] = 0.f;
+__device__ __forceinline__ void frag_col_add(float* dst, const Frag& f, int col, float s) {
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    s += __shfl_xor_sync(0xffffffffu, s, 8);
+    s += __shfl_xor_sync(0xffffffffu, s, 16);
+    if (f.g == 0) atomicAdd(dst + col, s);
 }
 
 // ------------------------------------------------------------ adjoint chain
@@ -361,23 +387,23 @@ chunk_bwd_kernel(const BwdParams p) {
     auto qf = [&](int r, int d) { return __bfloat162float(sQ[r * LDB + d]); };
     auto vf = [&](int r, int d) { return __bfloat162float(sV[r * LDB + d]); };
     auto of = [&](int r, int d) { return __bfloat162float(sdO[r * LDB + d]); };
-    const int tr = tid / 16, tc = tid % 16;   // gemm thread layout (16 x 16)
+    const Frag F64 = frag_of(warp, lane, C), F128 = frag_of(warp, lane, D);
 
     // ---- P = Tril(E (.) Q K^T), A = StrictTril(beta_r E (.) K K^T)
     {
         float aq[4][4], ak[4][4];
         zero(aq);
         zero(ak);
-        gemm_acc<4, 4, 16, 16>(aq, D, tid, qf, [&](int d, int i) { return kf(i, d); });
-        gemm_acc<4, 4, 16, 16>(ak, D, tid, kf, [&](int d, int i) { return kf(i, d); });
+        mma_acc<4>(aq, D, F64, qf, [&](int d, int i) { return kf(i, d); });
+        mma_acc<4>(ak, D, F64, kf, [&](int d, int i) { return kf(i, d); });
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = a * 16 + tr, i = j * 16 + tc;
-                const float e = E(r, i);
-                sP[r * LDS + i] = e * aq[a][j];
-                sA[r * LDS + i] = i < r ? sBeta[r] * e * ak[a][j] : 0.f;
+            for (int e = 0; e < 4; ++e) {
+                const int r = F64.row(e), i = F64.col(j, e);
+                const float ev = E(r, i);
+                sP[r * LDS + i] = ev * aq[j][e];
+                sA[r * LDS + i] = i < r ? sBeta[r] * ev * ak[j][e] : 0.f;
             }
     }
     __syncthreads();
@@ -395,18 +421,18 @@ chunk_bwd_kernel(const BwdParams p) {
     __syncthreads();
     // ---- W = T diag(beta Gamma) K, U = T diag(beta) V
     {
-        float aw[4][8], au[4][8];
+        float aw[8][4], au[8][4];
         zero(aw);
         zero(au);
-        gemm_acc<4, 8, 16, 16>(aw, C, tid, [&](int r, int i) { return sT[r * LDS + i] * sBeta[i] * sGam[i]; }, kf);
-        gemm_acc<4, 8, 16, 16>(au, C, tid, [&](int r, int i) { return sT[r * LDS + i] * sBeta[i]; }, vf);
+        mma_acc<8>(aw, C, F128, [&](int r, int i) { return sT[r * LDS + i] * sBeta[i] * sGam[i]; }, kf);
+        mma_acc<8>(au, C, F128, [&](int r, int i) { return sT[r * LDS + i] * sBeta[i]; }, vf);
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = a * 16 + tr, v = j * 16 + tc;
-                MW[r * LDM + v] = aw[a][j];
-                MD[r * LDM + v] = au[a][j];
+            for (int e = 0; e < 4; ++e) {
+                const int r = F128.row(e), v = F128.col(j, e);
+                MW[r * LDM + v] = aw[j][e];
+                MD[r * LDM + v] = au[j][e];
             }
     }
     // ---- D = U - W h (h staged by halves of 64 rows)
@@ -419,64 +445,65 @@ chunk_bwd_kernel(const BwdParams p) {
         __syncthreads();
     };
     {
-        float ad[4][8];
+        float ad[8][4];
         zero(ad);
         for (int half = 0; half < 2; ++half) {
             stage_half(hsrc, half);
-            gemm_acc<4, 8, 16, 16>(ad, C, tid, [&](int r, int d) { return MW[r * LDM + 64 * half + d]; },
-                                   [&](int d, int v) { return stage[d * LDM + v]; });
+            mma_acc<8>(ad, C, F128, [&](int r, int d) { return MW[r * LDM + 64 * half + d]; },
+                       [&](int d, int v) { return stage[d * LDM + v]; });
         }
         __syncthreads();
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = a * 16 + tr, v = j * 16 + tc;
-                MD[r * LDM + v] -= ad[a][j];
+            for (int e = 0; e < 4; ++e) {
+                const int r = F128.row(e), v = F128.col(j, e);
+                MD[r * LDM + v] -= ad[j][e];
             }
     }
     __syncthreads();
-    // dq and dk of this thread's 4 x 8 elements, summed over every product below
-    float dq[4][8], dk[4][8];
+    // dq and dk of this thread's fragment elements (rows r, columns d of the
+    // 64 x 128 layout), summed over every product below
+    float dq[8][4], dk[8][4];
     zero(dq);
     zero(dk);
     // ---- dD = P^T dO + Ktil dh' (into MW, W being dead), dKtil = D dh'^T,
     //      <h, dh'>; dh' staged by halves of 64 rows (d)
     {
-        float add[4][8];
+        float add[8][4];
         zero(add);
-        gemm_acc<4, 8, 16, 16>(add, C, tid, [&](int i, int r) { return sP[r * LDS + i]; }, of);
+        mma_acc<8>(add, C, F128, [&](int i, int r) { return sP[r * LDS + i]; }, of);
         float hdh = 0.f, lastsum = 0.f;   // <h, dh'>; the K~ terms of dG_last
         for (int half = 0; half < 2; ++half) {
             stage_half(dhsrc, half);
             // Ktil[i][d] = k_id e^(Glast - G_i), d in this half
-            gemm_acc<4, 8, 16, 16>(add, C, tid,
-                [&](int i, int d) { return kf(i, 64 * half + d) * __expf(Glast - sG[i]); },
-                [&](int d, int v) { return stage[d * LDM + v]; });
-            // dKtil[i][d] = sum_v D[i][v] dh'[d][v], for d = 64 half + 16 j' + tc (4 x 4 tile)
-            float akt[4][4];
-            zero(akt);
-            gemm_acc<4, 4, 16, 16>(akt, D, tid, [&](int i, int v) { return MD[i * LDM + v]; },
-                                   [&](int v, int d) { return stage[d * LDM + v]; });
+            mma_acc<8>(add, C, F128,
+                       [&](int i, int d) { return kf(i, 64 * half + d) * __expf(Glast - sG[i]); },
+                       [&](int d, int v) { return stage[d * LDM + v]; });
+            // dKtil[i][d] = sum_v D[i][v] dh'[d][v] for the columns d of this
+            // half: the warps that own them in the 64 x 128 layout
+            if ((warp >> 2) == half) {
+                float akt[8][4];
+                zero(akt);
+                mma_acc<8>(akt, D, F128, [&](int i, int v) { return MD[i * LDM + v]; },
+                           [&](int v, int d) { return stage[(d - 64 * half) * LDM + v]; });
+                float lo = 0.f, hi = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = F128.row(e), d = F128.col(j, e);
+                        const float f = __expf(Glast - sG[i]);
+                        dk[j][e] = fmaf(akt[j][e], f, dk[j][e]);
+                        const float part = akt[j][e] * kf(i, d) * f;
+                        if (e < 2) lo += part;
+                        else hi += part;
+                    }
+                frag_row_add(sdG, F128, -lo, -hi);
+                lastsum += lo + hi;
+            }
             for (int idx = tid; idx < C * D; idx += CB_THREADS)
                 hdh = fmaf(__ldcg(hsrc + (size_t)half * C * D + idx), stage[(idx >> 7) * LDM + (idx & 127)], hdh);
-            // dk_i += dKtil e^(Glast - G_i); dG_i -= <dKtil_i, Ktil_i>; dG_last += sum
-            // (the 4 x 4 tile covers columns 64 half + j * 16 + tc of the 4 x 8 layout:
-            //  column slot j' = 4 half + j)
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                const int i = a * 16 + tr;
-                const float f = __expf(Glast - sG[i]);
-                float part = 0.f;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int d = 64 * half + j * 16 + tc;
-                    dk[a][4 * half + j] = fmaf(akt[a][j], f, dk[a][4 * half + j]);
-                    part = fmaf(akt[a][j], kf(i, d) * f, part);
-                }
-                row_add(&sdG[i], -part, lane);
-                lastsum += part;
-            }
         }
         // <h, dh'> over the block, into dG_last (gamma <h, dh'>)
         float last = gamma * hdh + lastsum;
@@ -485,136 +512,138 @@ chunk_bwd_kernel(const BwdParams p) {
         if (lane == 0) atomicAdd(&sdG[C - 1], last);
         __syncthreads();
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) MW[(a * 16 + tr) * LDM + j * 16 + tc] = add[a][j];   // dD
+            for (int e = 0; e < 4; ++e) MW[F128.row(e) * LDM + F128.col(j, e)] = add[j][e];   // dD
     }
     __syncthreads();
     // ---- dP = Tril(dO D^T); tP = dP (.) P -> dG; dPE = dP (.) E into sP
     {
         float adp[4][4];
         zero(adp);
-        gemm_acc<4, 4, 16, 16>(adp, D, tid, of, [&](int v, int i) { return MD[i * LDM + v]; });
-        float colp[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_acc<4>(adp, D, F64, of, [&](int v, int i) { return MD[i * LDM + v]; });
+        float lo = 0.f, hi = 0.f, colp[4][2];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const int r = a * 16 + tr;
-            float rowp = 0.f;
+        for (int j = 0; j < 4; ++j) colp[j][0] = colp[j][1] = 0.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int i = j * 16 + tc;
-                const float t = i <= r ? adp[a][j] * sP[r * LDS + i] : 0.f;
-                rowp += t;
-                colp[j] += t;
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = F64.row(e), i = F64.col(j, e);
+                const float t = i <= r ? adp[j][e] * sP[r * LDS + i] : 0.f;
+                if (e < 2) lo += t;
+                else hi += t;
+                colp[j][e & 1] += t;
             }
-            row_add(&sdG[r], rowp, lane);
-        }
+        frag_row_add(sdG, F64, lo, hi);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) col_add(&sdG[j * 16 + tc], -colp[j], lane);
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int q = 0; q < 2; ++q) frag_col_add(sdG, F64, F64.c0 + 8 * j + 2 * F64.t + q, -colp[j][q]);
         __syncthreads();   // every thread has read P
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = a * 16 + tr, i = j * 16 + tc;
-                sP[r * LDS + i] = i <= r ? adp[a][j] * E(r, i) : 0.f;
+            for (int e = 0; e < 4; ++e) {
+                const int r = F64.row(e), i = F64.col(j, e);
+                sP[r * LDS + i] = i <= r ? adp[j][e] * E(r, i) : 0.f;
             }
     }
     __syncthreads();
     // dq_r += sum_i dPE_ri k_i;  dk_i += sum_r dPE_ri q_r
-    gemm_acc<4, 8, 16, 16>(dq, C, tid, [&](int r, int i) { return sP[r * LDS + i]; }, kf);
-    gemm_acc<4, 8, 16, 16>(dk, C, tid, [&](int i, int r) { return sP[r * LDS + i]; }, qf);
+    mma_acc<8>(dq, C, F128, [&](int r, int i) { return sP[r * LDS + i]; }, kf);
+    mma_acc<8>(dk, C, F128, [&](int i, int r) { return sP[r * LDS + i]; }, qf);
     // ---- dQbar = dO h^T -> dq += Gamma dQbar, dG_r += Gamma_r <dQbar_r, q_r>;
-    //      dW = -dD h^T (into MD, D being dead from here)
-    {
-        float aqb[4][8], awb[4][8];
-        zero(aqb);
-        zero(awb);
-        for (int half = 0; half < 2; ++half) {   // h by halves of 64 rows: columns d of the outputs
-            stage_half(hsrc, half);
-            float t1[4][4], t2[4][4];
+    //      dW = -dD h^T (into MD, D being dead from here); h by halves of 64
+    //      rows d, each half's columns by the warps that own them
+    for (int half = 0; half < 2; ++half) {
+        stage_half(hsrc, half);
+        if ((warp >> 2) == half) {
+            float t1[8][4], t2[8][4];
             zero(t1);
             zero(t2);
-            gemm_acc<4, 4, 16, 16>(t1, D, tid, of, [&](int v, int d) { return stage[d * LDM + v]; });
-            gemm_acc<4, 4, 16, 16>(t2, D, tid, [&](int r, int v) { return MW[r * LDM + v]; },
-                                   [&](int v, int d) { return stage[d * LDM + v]; });
+            mma_acc<8>(t1, D, F128, of, [&](int v, int d) { return stage[(d - 64 * half) * LDM + v]; });
+            mma_acc<8>(t2, D, F128, [&](int r, int v) { return MW[r * LDM + v]; },
+                       [&](int v, int d) { return stage[(d - 64 * half) * LDM + v]; });
+            float lo = 0.f, hi = 0.f;
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int j = 0; j < 8; ++j)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    aqb[a][4 * half + j] = t1[a][j];
-                    awb[a][4 * half + j] = -t2[a][j];
+                for (int e = 0; e < 4; ++e) {
+                    const int r = F128.row(e), d = F128.col(j, e);
+                    dq[j][e] = fmaf(sGam[r], t1[j][e], dq[j][e]);
+                    const float part = sGam[r] * t1[j][e] * qf(r, d);
+                    if (e < 2) lo += part;
+                    else hi += part;
+                    t2[j][e] = -t2[j][e];
                 }
-        }
-        __syncthreads();
+            frag_row_add(sdG, F128, lo, hi);
+            // every warp of this half has read MD's D values (the dP product
+            // above, behind a barrier): dW may overwrite them
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const int r = a * 16 + tr;
-            float part = 0.f;
+            for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int d = (j & 3) * 16 + tc + 64 * (j >> 2);
-                dq[a][j] = fmaf(sGam[r], aqb[a][j], dq[a][j]);
-                part = fmaf(aqb[a][j], qf(r, d), part);
-                MD[r * LDM + d] = awb[a][j];   // dW
-            }
-            row_add(&sdG[r], sGam[r] * part, lane);
+                for (int e = 0; e < 4; ++e) MD[F128.row(e) * LDM + F128.col(j, e)] = t2[j][e];
         }
     }
     __syncthreads();
     // ---- dv = beta T^T dU (dU = dD);  dbeta += <T^T dU, V> + <T^T dW, Kbar>;
     //      dKbar = beta T^T dW -> dk += Gamma dKbar, dG += <dKbar, Kbar>
     {
-        float tu[4][8], tw[4][8];
+        float tu[8][4], tw[8][4];
         zero(tu);
         zero(tw);
-        gemm_acc<4, 8, 16, 16>(tu, C, tid, [&](int r, int i) { return sT[i * LDS + r]; },
-                               [&](int i, int v) { return MW[i * LDM + v]; });
-        gemm_acc<4, 8, 16, 16>(tw, C, tid, [&](int r, int i) { return sT[i * LDS + r]; },
-                               [&](int i, int v) { return MD[i * LDM + v]; });
+        mma_acc<8>(tu, C, F128, [&](int r, int i) { return sT[i * LDS + r]; },
+                   [&](int i, int v) { return MW[i * LDM + v]; });
+        mma_acc<8>(tw, C, F128, [&](int r, int i) { return sT[i * LDS + r]; },
+                   [&](int i, int v) { return MD[i * LDM + v]; });
+        float db_lo = 0.f, db_hi = 0.f, dg_lo = 0.f, dg_hi = 0.f;
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const int r = a * 16 + tr;
-            float db = 0.f, dg = 0.f;
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int v = j * 16 + tc;
-                if (r < n) p.dv[tok(r) * D + v] = sBeta[r] * tu[a][j];
+            for (int e = 0; e < 4; ++e) {
+                const int r = F128.row(e), v = F128.col(j, e);
+                if (r < n) p.dv[tok(r) * D + v] = sBeta[r] * tu[j][e];
                 const float kbar = sGam[r] * kf(r, v);
-                db = fmaf(tu[a][j], vf(r, v), db);
-                db = fmaf(tw[a][j], kbar, db);
-                const float dkb = sBeta[r] * tw[a][j];
-                dk[a][j] = fmaf(sGam[r], dkb, dk[a][j]);
-                dg = fmaf(dkb, kbar, dg);
+                const float db = fmaf(tu[j][e], vf(r, v), tw[j][e] * kbar);
+                const float dkb = sBeta[r] * tw[j][e];
+                dk[j][e] = fmaf(sGam[r], dkb, dk[j][e]);
+                const float dg = dkb * kbar;
+                if (e < 2) {
+                    db_lo += db;
+                    dg_lo += dg;
+                } else {
+                    db_hi += db;
+                    dg_hi += dg;
+                }
             }
-            row_add(&sdB[r], db, lane);
-            row_add(&sdG[r], dg, lane);
-        }
+        frag_row_add(sdB, F128, db_lo, db_hi);
+        frag_row_add(sdG, F128, dg_lo, dg_hi);
     }
     // ---- dT = dD (beta V)^T + dW (beta Kbar)^T  (into sA);  tmp = T^T dT  (into stage)
     {
         float adt[4][4];
         zero(adt);
-        gemm_acc<4, 4, 16, 16>(adt, D, tid, [&](int r, int v) { return MW[r * LDM + v]; },
-                               [&](int v, int i) { return sBeta[i] * vf(i, v); });
-        gemm_acc<4, 4, 16, 16>(adt, D, tid, [&](int r, int d) { return MD[r * LDM + d]; },
-                               [&](int d, int i) { return sBeta[i] * sGam[i] * kf(i, d); });
+        mma_acc<4>(adt, D, F64, [&](int r, int v) { return MW[r * LDM + v]; },
+                   [&](int v, int i) { return sBeta[i] * vf(i, v); });
+        mma_acc<4>(adt, D, F64, [&](int r, int d) { return MD[r * LDM + d]; },
+                   [&](int d, int i) { return sBeta[i] * sGam[i] * kf(i, d); });
         __syncthreads();
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) sA[(a * 16 + tr) * LDS + j * 16 + tc] = adt[a][j];
+            for (int e = 0; e < 4; ++e) sA[F64.row(e) * LDS + F64.col(j, e)] = adt[j][e];
     }
     __syncthreads();
     {
         float at[4][4];
         zero(at);
-        gemm_acc<4, 4, 16, 16>(at, C, tid, [&](int r, int i) { return sT[i * LDS + r]; },
-                               [&](int i, int j) { return sA[i * LDS + j]; });
+        mma_acc<4>(at, C, F64, [&](int r, int i) { return sT[i * LDS + r]; },
+                   [&](int i, int j) { return sA[i * LDS + j]; });
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) stage[(a * 16 + tr) * LDS + j * 16 + tc] = at[a][j];
+            for (int e = 0; e < 4; ++e) stage[F64.row(e) * LDS + F64.col(j, e)] = at[j][e];
     }
     __syncthreads();
     // ---- dA = StrictTril(-tmp T^T); dKK = beta_r dA; dbeta += sum_i dA KKE;
@@ -623,54 +652,61 @@ chunk_bwd_kernel(const BwdParams p) {
         float ada[4][4], akk[4][4];
         zero(ada);
         zero(akk);
-        gemm_acc<4, 4, 16, 16>(ada, C, tid, [&](int r, int i) { return stage[r * LDS + i]; },
-                               [&](int i, int j) { return sT[j * LDS + i]; });
-        gemm_acc<4, 4, 16, 16>(akk, D, tid, kf, [&](int d, int i) { return kf(i, d); });
+        mma_acc<4>(ada, C, F64, [&](int r, int i) { return stage[r * LDS + i]; },
+                   [&](int i, int j) { return sT[j * LDS + i]; });
+        mma_acc<4>(akk, D, F64, kf, [&](int d, int i) { return kf(i, d); });
         __syncthreads();
-        float cola[4] = {0.f, 0.f, 0.f, 0.f};
+        float db_lo = 0.f, db_hi = 0.f, ra_lo = 0.f, ra_hi = 0.f, cola[4][2];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const int r = a * 16 + tr;
-            float db = 0.f, rowa = 0.f;
+        for (int j = 0; j < 4; ++j) cola[j][0] = cola[j][1] = 0.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int i = j * 16 + tc;
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = F64.row(e), i = F64.col(j, e);
                 float val = 0.f;
                 if (i < r) {
-                    const float dA = -ada[a][j];
-                    const float e = E(r, i);
-                    db = fmaf(dA, e * akk[a][j], db);
-                    const float dkke = sBeta[r] * dA * e;
-                    const float t = dkke * akk[a][j];
-                    rowa += t;
-                    cola[j] += t;
+                    const float dA = -ada[j][e];
+                    const float ev = E(r, i);
+                    const float db = dA * ev * akk[j][e];
+                    const float dkke = sBeta[r] * dA * ev;
+                    const float t = dkke * akk[j][e];
+                    if (e < 2) {
+                        db_lo += db;
+                        ra_lo += t;
+                    } else {
+                        db_hi += db;
+                        ra_hi += t;
+                    }
+                    cola[j][e & 1] += t;
                     val = dkke;
                 }
                 sA[r * LDS + i] = val;
             }
-            row_add(&sdB[r], db, lane);
-            row_add(&sdG[r], rowa, lane);
-        }
+        frag_row_add(sdB, F64, db_lo, db_hi);
+        frag_row_add(sdG, F64, ra_lo, ra_hi);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) col_add(&sdG[j * 16 + tc], -cola[j], lane);
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int q = 0; q < 2; ++q) frag_col_add(sdG, F64, F64.c0 + 8 * j + 2 * F64.t + q, -cola[j][q]);
     }
     __syncthreads();
     // dk_r += sum_i dKKE_ri k_i;  dk_i += sum_r dKKE_ri k_r
-    gemm_acc<4, 8, 16, 16>(dk, C, tid, [&](int r, int i) { return sA[r * LDS + i]; }, kf);
-    gemm_acc<4, 8, 16, 16>(dk, C, tid, [&](int i, int r) { return sA[r * LDS + i]; }, kf);
+    mma_acc<8>(dk, C, F128, [&](int r, int i) { return sA[r * LDS + i]; }, kf);
+    mma_acc<8>(dk, C, F128, [&](int i, int r) { return sA[r * LDS + i]; }, kf);
     __syncthreads();
-    // ---- outputs: dq, dk (this thread's elements), dbeta, dg (reverse cumsum of dG)
+    // ---- outputs: dq, dk (this thread's elements, two adjacent columns a
+    // store), dbeta, dg (reverse cumsum of dG)
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const int r = a * 16 + tr;
-        if (r < n) {
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                p.dq[tok(r) * D + j * 16 + tc] = dq[a][j];
-                p.dk[tok(r) * D + j * 16 + tc] = dk[a][j];
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int r = F128.row(2 * h2), d = F128.col(j, 0);
+            if (r < n) {
+                *reinterpret_cast<float2*>(p.dq + tok(r) * D + d) = make_float2(dq[j][2 * h2], dq[j][2 * h2 + 1]);
+                *reinterpret_cast<float2*>(p.dk + tok(r) * D + d) = make_float2(dk[j][2 * h2], dk[j][2 * h2 + 1]);
             }
         }
-    }
     if (warp == 0) {   // dg_t = sum_{r >= t} dG_r: a reverse scan, two tokens a lane
         const int r0 = C - 2 - 2 * lane;     // lane 0 takes the last two tokens
         const float a1 = sdG[r0 + 1], a0 = sdG[r0];
