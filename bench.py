@@ -751,18 +751,23 @@ def time_backward(ctx: Ctx):
 
 
 def run_only(args, world, rank, local):
-    """One forward workload alone (for profiling): its record, no CPU baseline."""
+    """One forward workload, or one extra record, alone (for profiling): its
+    record, no CPU baseline."""
     args.no_cpu_baseline = True
     ctx = Ctx(args, world, rank, local)
     ctx.sampler.start()
-    rec, _ = time_forward(ctx, args.only)
+    if args.only_extra:
+        rec = {"osdn": time_osdn, "segments": time_segments,
+               "backward": time_backward}[args.only_extra](ctx)
+    else:
+        rec, _ = time_forward(ctx, args.only)
     ctx.sampler.stop()
     if rank == 0:
         print(json.dumps(rec), flush=True)
 
 
 def run_ours(args, world, rank, local):
-    if args.only is not None:
+    if args.only is not None or args.only_extra:
         return run_only(args, world, rank, local)
     ctx = Ctx(args, world, rank, local)
     ctx.sampler.start()
@@ -827,6 +832,8 @@ def main():
                     help="skip the preconditioned-rule, segment and backward records")
     ap.add_argument("--only", type=int, default=None, choices=(0, 1, 2, 3),
                     help="time one forward workload alone and print its record (profiling)")
+    ap.add_argument("--only-extra", default=None, choices=("osdn", "segments", "backward"),
+                    help="time one extra record alone and print it (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
