@@ -294,6 +294,18 @@ adjoint_chain_kernel(const __grid_constant__ AdjMaps maps, const BwdParams p) {
 }
 
 // --------------------------------------------------------- chunk backward
+// 16-byte copies global -> shared that bypass the registers (L2 only), so a
+// thread issues all of its copies of a tile before waiting once; a source size
+// of 0 fills the 16 bytes with zeros (rows past the end of the sequence).
+__device__ __forceinline__ void cpa16(void* dst, const void* src, uint32_t src_bytes = 16u) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sm100::smem_u32(dst)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cpa_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 constexpr int CB_THREADS = 256;
 constexpr int LDM = D + 4;   // fp32 row stride of [64][128] matrices
 constexpr int LDS = C + 1;   // fp32 row stride of [64][64] matrices
@@ -342,17 +354,18 @@ chunk_bwd_kernel(const BwdParams p) {
     auto tok = [&](int r) { return ((size_t)b * p.T + (size_t)c * C + r) * p.H + h; };
     const int n = min(C, p.T - c * C);
 
-    // ---- inputs of the chunk (rows past the sequence end are zero)
+    // ---- inputs of the chunk (rows past the sequence end are zero-filled; their
+    // copies read nothing and name row 0, which exists)
     for (int idx = tid; idx < 4 * C * D / 8; idx += CB_THREADS) {
         const int m = idx / (C * D / 8), rem = idx % (C * D / 8), r = rem >> 4, j = rem & 15;
         const __nv_bfloat16* src = m == 0 ? static_cast<const __nv_bfloat16*>(p.q)
                                    : m == 1 ? static_cast<const __nv_bfloat16*>(p.k)
                                    : m == 2 ? static_cast<const __nv_bfloat16*>(p.v)
                                             : static_cast<const __nv_bfloat16*>(p.dO);
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (r < n) w = *reinterpret_cast<const uint4*>(src + tok(r) * D + 8 * j);
-        *reinterpret_cast<uint4*>(sm + m * BW_TILE + r * LDB * 2 + 16 * j) = w;
+        cpa16(sm + m * BW_TILE + r * LDB * 2 + 16 * j, src + tok(r < n ? r : 0) * D + 8 * j,
+              r < n ? 16u : 0u);
     }
+    cpa_wait_all();
     if (tid < C) {
         float bt = 0.f, gv = 0.f;
         if (tid < n) {
@@ -440,8 +453,10 @@ chunk_bwd_kernel(const BwdParams p) {
     const float* dhsrc = p.dh_all + ((size_t)bh * NC + c) * D * D;
     auto stage_half = [&](const float* src, int half) {
         __syncthreads();
-        for (int idx = tid; idx < C * D; idx += CB_THREADS)
-            stage[(idx >> 7) * LDM + (idx & 127)] = __ldcg(src + (size_t)half * C * D + idx);
+#pragma unroll
+        for (int idx = 4 * tid; idx < C * D; idx += 4 * CB_THREADS)
+            cpa16(stage + (idx >> 7) * LDM + (idx & 127), src + (size_t)half * C * D + idx);
+        cpa_wait_all();
         __syncthreads();
     };
     {
@@ -502,8 +517,15 @@ chunk_bwd_kernel(const BwdParams p) {
                 frag_row_add(sdG, F128, -lo, -hi);
                 lastsum += lo + hi;
             }
-            for (int idx = tid; idx < C * D; idx += CB_THREADS)
-                hdh = fmaf(__ldcg(hsrc + (size_t)half * C * D + idx), stage[(idx >> 7) * LDM + (idx & 127)], hdh);
+#pragma unroll 4
+            for (int idx = 4 * tid; idx < C * D; idx += 4 * CB_THREADS) {
+                const float4 hv = __ldcg(reinterpret_cast<const float4*>(hsrc + (size_t)half * C * D + idx));
+                const float* sp = stage + (idx >> 7) * LDM + (idx & 127);
+                hdh = fmaf(hv.x, sp[0], hdh);
+                hdh = fmaf(hv.y, sp[1], hdh);
+                hdh = fmaf(hv.z, sp[2], hdh);
+                hdh = fmaf(hv.w, sp[3], hdh);
+            }
         }
         // <h, dh'> over the block, into dG_last (gamma <h, dh'>)
         float last = gamma * hdh + lastsum;
