@@ -196,6 +196,51 @@ def test_split_sequence_carry(gate):
 
 
 @pytest.mark.parametrize("gate", GATES)
+def test_a_run_of_tokens_maps_the_state_affinely(gate):
+    """A run of tokens maps the entering state affinely, column by column:
+    S_out[:, j] = A S_in[:, j] + b[:, j] with one Dk x Dk matrix A for every
+    value column (each step is (Diag(a) - beta k k^T Diag(a)) applied to the
+    state plus beta k v^T; "Moonshot AI's New Attention Architecture", sec. 3).
+    Two runs compose as
+    A2 (A1 S + b1) + b2, which is how the segment-parallel pass combines
+    segment offsets b and transitions A."""
+    B, T, H, Dk, Dv = 1, 24, 2, 6, 5
+    q, k, v, beta, g, S0 = rand_case(B, T, H, Dk, Dv, gate, seed=31)
+    gsl = (lambda a, b: None) if g is None else (lambda a, b: g[:, a:b])
+
+    def run(a, b, S):
+        return oracle.recurrent(q[:, a:b], k[:, a:b], v[:, a:b], beta[:, a:b], gsl(a, b), gate, S)[1]
+
+    def transition(a, b):
+        """A (per head, [H][Dk][Dk]) and b ([H][Dk][Dv]) of tokens a..b-1."""
+        zero = np.zeros((B, H, Dk, Dv))
+        off = run(a, b, zero)
+        A = np.empty((H, Dk, Dk))
+        for i in range(Dk):
+            E = np.zeros((B, H, Dk, Dv))
+            E[:, :, i, :] = 1.0                  # e_i in every value column
+            cols = run(a, b, E) - off            # A e_i, the same in every column
+            np.testing.assert_allclose(cols, cols[..., :1].repeat(Dv, axis=-1), rtol=0, atol=1e-12)
+            A[:, :, i] = cols[0, :, :, 0]
+        return A, off[0]
+
+    A1, b1 = transition(0, 11)
+    A2, b2 = transition(11, T)
+    S_in = S0
+    # the affine form reproduces each run and the whole sequence
+    np.testing.assert_allclose(run(0, 11, S_in)[0], A1 @ S_in[0] + b1, rtol=0, atol=1e-11)
+    whole = run(0, T, S_in)[0]
+    np.testing.assert_allclose(whole, A2 @ (A1 @ S_in[0] + b1) + b2, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(whole, (A2 @ A1) @ S_in[0] + (A2 @ b1 + b2), rtol=0, atol=1e-11)
+    # affine combinations of entering states are preserved
+    S_alt = np.random.default_rng(5).standard_normal(S_in.shape)
+    lam = 0.3
+    mix = run(0, T, lam * S_in + (1 - lam) * S_alt)
+    np.testing.assert_allclose(mix, lam * run(0, T, S_in) + (1 - lam) * run(0, T, S_alt),
+                               rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("gate", GATES)
 def test_causality(gate):
     """Perturbing tokens after t leaves o_{<=t} unchanged."""
     q, k, v, beta, g, S0 = rand_case(1, 24, 2, 8, 8, gate, seed=13)
