@@ -19,7 +19,7 @@
 // products through P, A, Kbar, Kbrev, Qbar, Ktil give dq, dk, dv, dbeta and
 // the log-decays' dG, whose reverse cumulative sum in the chunk is dg.
 //
-// Three launches after the forward (run in one wave, keeping every step image
+// Two launches after the forward (run in one wave, keeping every step image
 // and every chunk's entering state):
 //   adjoint_chain_kernel  one CTA per (batch, head), chunks from the last back:
 //                         stores the adjoint of each chunk's leaving state,
@@ -27,8 +27,10 @@
 //                         from the forward's step images, the adjoint in fp32
 //   chunk_bwd_kernel      one CTA per (batch, head, chunk): recomputes the
 //                         chunk's A, T, W, U, D and forms every gradient of the
-//                         chunk; fp32 on CUDA cores, dq and dk accumulated in
-//                         registers across the products that feed them
+//                         chunk; every product as tf32 warp MMAs (m16n8k8, fp32
+//                         accumulation), tiles staged by cp.async, dq and dk
+//                         accumulated in registers across the products that
+//                         feed them
 #include <string.h>
 
 #include "common.cuh"
